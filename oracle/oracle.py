@@ -1,0 +1,218 @@
+"""ctypes front end of the fp64 CPU oracle (twell_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: imported by the tests, by the smoke check and by the
+benchmark's CPU-baseline leg, never by the product path. All arrays are numpy;
+bfloat16 tensors are passed as uint16 bit patterns.
+
+Parity status of each function (what pins it is in tests/test_oracle_pins.py):
+  bf16_round        pinned: torch's float32->bfloat16 RNE cast, hand-made ties
+  gate              pinned: brute-force loops, torch float64 matmul
+  pack / unpack     pinned: round trip, invariants, hand-built identity-gate case
+  ffn_fwd           pinned: brute-force loops, torch float64, closed forms
+  ffn_fwd_hybrid    pinned: equals ffn_fwd (round_g=1) on the same active set
+  ffn_bwd           pinned: torch float64 autograd, closed form of the L1 term
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "twell_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "libtwell_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_u16p = np.ctypeslib.ndpointer(np.uint16, flags="C_CONTIGUOUS")
+_u8p = np.ctypeslib.ndpointer(np.uint8, flags="C_CONTIGUOUS")
+_i32p = np.ctypeslib.ndpointer(np.int32, flags="C_CONTIGUOUS")
+_f64p = np.ctypeslib.ndpointer(np.float64, flags="C_CONTIGUOUS")
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int32
+_vp = ctypes.c_void_p
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O3, no fused or re-associated arithmetic)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O3", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
+               "-std=c11", _SRC, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            L = ctypes.CDLL(build())
+            L.oracle_bf16_round.restype = ctypes.c_uint16
+            L.oracle_bf16_round.argtypes = [ctypes.c_double]
+            L.oracle_bf16_round_array.argtypes = [_f64p, _u16p, _i64]
+            L.oracle_bf16_to_double_array.argtypes = [_u16p, _f64p, _i64]
+            L.oracle_set_threads.argtypes = [ctypes.c_int]
+            L.oracle_get_threads.restype = ctypes.c_int
+            L.oracle_gate.restype = ctypes.c_int
+            L.oracle_gate.argtypes = [_u16p, _u16p, _u16p, _i64, _i64, _i64, _vp, _i64, _f64p]
+            L.oracle_pack.restype = ctypes.c_int
+            L.oracle_pack.argtypes = [_f64p, _i64, _i64, _i32, _i32, _i64, _u16p, _u16p, _u8p, _u8p,
+                                      _i32p, ctypes.POINTER(ctypes.c_int64), _u16p]
+            L.oracle_unpack.argtypes = [_u16p, _u16p, _u8p, _u8p, _i32p, _i64, _u16p, _i64, _i64, _i32,
+                                        _i32, _u16p]
+            L.oracle_ffn_fwd.restype = ctypes.c_int
+            L.oracle_ffn_fwd.argtypes = [_u16p, _u16p, _u16p, _u16p, _u16p, _i64, _i64, _i64, _vp, _i64,
+                                         _vp, _i32, _f64p]
+            L.oracle_ffn_fwd_hybrid.restype = ctypes.c_int
+            L.oracle_ffn_fwd_hybrid.argtypes = [_u16p, _u16p, _u16p, _u16p, _u16p, _u8p, _u8p, _i32p, _i64,
+                                                _u16p, _i64, _i64, _i64, _i32, _i32, _f64p]
+            L.oracle_ffn_bwd.restype = ctypes.c_int
+            L.oracle_ffn_bwd.argtypes = [_u16p, _u16p, _u16p, _u16p, _u16p, _u16p, ctypes.c_double, _i64,
+                                         _i64, _i64, _vp, _i32, _f64p, _f64p, _f64p, _f64p, _vp]
+            _lib = L
+    return _lib
+
+
+def _c(a, dt):
+    return np.ascontiguousarray(a, dtype=dt)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def set_threads(n: int) -> None:
+    lib().oracle_set_threads(int(n))
+
+
+def get_threads() -> int:
+    return int(lib().oracle_get_threads())
+
+
+def bf16_round(x) -> np.ndarray:
+    """float64 values -> bfloat16 bits (RNE)."""
+    a = _c(x, np.float64)
+    out = np.empty(a.shape, np.uint16)
+    lib().oracle_bf16_round_array(a.reshape(-1), out.reshape(-1), a.size)
+    return out
+
+
+def bf16_to_f64(b) -> np.ndarray:
+    a = _c(b, np.uint16)
+    out = np.empty(a.shape, np.float64)
+    lib().oracle_bf16_to_double_array(a.reshape(-1), out.reshape(-1), a.size)
+    return out
+
+
+def gate(X, W_g, b_g, rows=None) -> np.ndarray:
+    """z = X W_g^T + b_g in float64, for all rows or for the listed rows."""
+    X, W_g, b_g = _c(X, np.uint16), _c(W_g, np.uint16), _c(b_g, np.uint16)
+    M, d = X.shape
+    f = W_g.shape[0]
+    r = None if rows is None else _c(rows, np.int32)
+    n = M if r is None else r.size
+    Z = np.empty((n, f), np.float64)
+    if lib().oracle_gate(X, W_g, b_g, M, d, f, _ptr(r), n, Z):
+        raise MemoryError("oracle_gate")
+    return Z
+
+
+def pack(Z, T_n: int, K: int, cap=None) -> dict:
+    """TwELL + hybrid routing of a dense float64 Z [M, f]."""
+    Z = _c(Z, np.float64)
+    M, f = Z.shape
+    if f % T_n or not (1 <= T_n <= 256) or K < 1:
+        raise ValueError("need d_ff % T_n == 0, 1 <= T_n <= 256 and K >= 1")
+    T = f // T_n
+    cap = M if cap is None else int(cap)
+    out = dict(
+        count=np.empty((M, T), np.uint16), val=np.empty((M, T, K), np.uint16),
+        col=np.empty((M, T, K), np.uint8), row_ovf=np.empty(M, np.uint8),
+        ovf_rows=np.zeros(max(cap, 1), np.int32), g_ovf=np.zeros((max(cap, 1), f), np.uint16),
+    )
+    n = ctypes.c_int64(0)
+    rc = lib().oracle_pack(Z, M, f, T_n, K, cap, out["count"], out["val"], out["col"], out["row_ovf"],
+                           out["ovf_rows"], ctypes.byref(n), out["g_ovf"])
+    if rc == 1:
+        raise ValueError("oracle_pack rejected the shape")
+    out["n_ovf_total"] = int(n.value)
+    out["n_ovf"] = min(int(n.value), cap)
+    out["status"] = int(rc)
+    out["ovf_rows"] = out["ovf_rows"][:cap]
+    out["g_ovf"] = out["g_ovf"][:cap]
+    return out
+
+
+def unpack(p: dict, f: int, T_n: int, K: int) -> np.ndarray:
+    """Dense bf16 bits of ReLU(z) [M, f] rebuilt from a packed dict."""
+    M = p["count"].shape[0]
+    G = np.empty((M, f), np.uint16)
+    ovf_rows = _c(p["ovf_rows"][: p["n_ovf"]], np.int32)
+    g_ovf = _c(p["g_ovf"][: p["n_ovf"]], np.uint16)
+    if ovf_rows.size == 0:
+        ovf_rows = np.zeros(1, np.int32)
+        g_ovf = np.zeros((1, f), np.uint16)
+    lib().oracle_unpack(_c(p["count"], np.uint16), _c(p["val"], np.uint16), _c(p["col"], np.uint8),
+                        _c(p["row_ovf"], np.uint8), ovf_rows, p["n_ovf"], g_ovf, M, f, T_n, K, G)
+    return G
+
+
+def ffn_fwd(X, W_g, b_g, W_u, W_d, rows=None, mask=None, round_g: bool = False) -> np.ndarray:
+    """Y = (ReLU(X W_g^T + b_g) * (X W_u^T)) W_d^T in float64 (rows subset optional)."""
+    X, W_g, b_g, W_u, W_d = (_c(a, np.uint16) for a in (X, W_g, b_g, W_u, W_d))
+    M, d = X.shape
+    f = W_g.shape[0]
+    r = None if rows is None else _c(rows, np.int32)
+    n = M if r is None else r.size
+    m = None if mask is None else _c(mask, np.uint8)
+    if m is not None and m.shape != (n, f):
+        raise ValueError("mask must be [nrows, d_ff]")
+    Y = np.empty((n, d), np.float64)
+    if lib().oracle_ffn_fwd(X, W_g, b_g, W_u, W_d, M, d, f, _ptr(r), n, _ptr(m), int(round_g), Y):
+        raise MemoryError("oracle_ffn_fwd")
+    return Y
+
+
+def ffn_fwd_hybrid(X, W_u, W_d, p: dict, T_n: int, K: int) -> np.ndarray:
+    """Y computed from a packed hybrid representation (ELL rows + dense rows)."""
+    X, W_u, W_d = (_c(a, np.uint16) for a in (X, W_u, W_d))
+    M, d = X.shape
+    f = W_u.shape[0]
+    n_ovf = p["n_ovf"]
+    ovf_rows = _c(p["ovf_rows"][:n_ovf], np.int32)
+    g_ovf = _c(p["g_ovf"][:n_ovf], np.uint16)
+    if n_ovf == 0:
+        ovf_rows = np.zeros(1, np.int32)
+        g_ovf = np.zeros((1, f), np.uint16)
+    Y = np.empty((M, d), np.float64)
+    rc = lib().oracle_ffn_fwd_hybrid(X, W_u, W_d, _c(p["count"], np.uint16), _c(p["val"], np.uint16),
+                                     _c(p["col"], np.uint8), _c(p["row_ovf"], np.uint8), ovf_rows, n_ovf,
+                                     g_ovf, M, d, f, T_n, K, Y)
+    if rc:
+        raise MemoryError("oracle_ffn_fwd_hybrid")
+    return Y
+
+
+def ffn_bwd(X, W_g, b_g, W_u, W_d, dY, lam: float = 0.0, mask=None, round_g: bool = False) -> dict:
+    """Gradients of sum(Y * dY) + lam * sum(ReLU(z)): dX, dW_g, dW_u, dW_d, db_g (float64)."""
+    X, W_g, b_g, W_u, W_d, dY = (_c(a, np.uint16) for a in (X, W_g, b_g, W_u, W_d, dY))
+    M, d = X.shape
+    f = W_g.shape[0]
+    m = None if mask is None else _c(mask, np.uint8)
+    if m is not None and m.shape != (M, f):
+        raise ValueError("mask must be [M, d_ff]")
+    out = dict(dX=np.empty((M, d)), dW_g=np.empty((f, d)), dW_u=np.empty((f, d)), dW_d=np.empty((d, f)),
+               db_g=np.empty(f))
+    rc = lib().oracle_ffn_bwd(X, W_g, b_g, W_u, W_d, dY, float(lam), M, d, f, _ptr(m), int(round_g),
+                              out["dX"], out["dW_g"], out["dW_u"], out["dW_d"], _ptr(out["db_g"]))
+    if rc:
+        raise MemoryError("oracle_ffn_bwd")
+    return out

@@ -1,0 +1,338 @@
+"""Pins of the fp64 CPU oracle against things other than itself.
+
+Each check ties one oracle function to the mathematics or to an independent
+library routine: brute-force loops on tiny inputs, torch float64 matmuls and
+autograd, a hand-built packing known by construction, closed forms of special
+cases, and format invariants. A dropped term, a wrong sign, a transposed operand
+or a wrong slot order in the oracle fails at least one of them.
+"""
+
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from synthetic import bf16_bits_from_f64, bf16_bits_to_f32
+
+
+def _rand_bf16(rng, shape, scale=1.0):
+    return bf16_bits_from_f64(rng.standard_normal(shape) * scale)
+
+
+def _f64(bits):
+    return bf16_bits_to_f32(bits).astype(np.float64)
+
+
+def _problem(seed, M, d, f, bias):
+    rng = np.random.default_rng(seed)
+    X = _rand_bf16(rng, (M, d))
+    Wg = _rand_bf16(rng, (f, d), 1 / math.sqrt(d))
+    Wu = _rand_bf16(rng, (f, d), 1 / math.sqrt(d))
+    Wd = _rand_bf16(rng, (d, f), 1 / math.sqrt(f))
+    bg = bf16_bits_from_f64(np.full(f, bias))
+    dY = _rand_bf16(rng, (M, d))
+    return X, Wg, bg, Wu, Wd, dY
+
+
+def _torch_ffn(X, Wg, bg, Wu, Wd, lam=0.0, dY=None):
+    t = lambda a: torch.tensor(_f64(a), dtype=torch.float64, requires_grad=True)  # noqa: E731
+    x, wg, b, wu, wd = t(X), t(Wg), t(bg), t(Wu), t(Wd)
+    z = x @ wg.T + b
+    g = torch.relu(z)
+    y = (g * (x @ wu.T)) @ wd.T
+    out = dict(Y=y.detach().numpy(), Z=z.detach().numpy())
+    if dY is not None:
+        loss = (y * torch.tensor(_f64(dY), dtype=torch.float64)).sum() + lam * g.sum()
+        loss.backward()
+        out.update(dX=x.grad.numpy(), dW_g=wg.grad.numpy(), dW_u=wu.grad.numpy(), dW_d=wd.grad.numpy(),
+                   db_g=b.grad.numpy())
+    return out
+
+
+def _rel(a, b):
+    return np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300)
+
+
+# ------------------------------------------------------------------ bfloat16
+
+
+def test_bf16_round_matches_torch_cast(orc):
+    rng = np.random.default_rng(1)
+    vals = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32),
+        (rng.standard_normal(2000) * 1e-39).astype(np.float32),   # binary32 subnormals
+        (rng.standard_normal(2000) * 1e37).astype(np.float32),
+        # exact halfway cases: low 16 bits 0x8000, both parities of the kept bit
+        (rng.integers(0x0080, 0x7F00, 4000, dtype=np.uint32) << 16 | 0x8000).view(np.float32),
+    ])
+    vals = np.concatenate([vals, -vals])
+    ours = orc.bf16_round(vals.astype(np.float64))
+    ref = torch.from_numpy(vals).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_bf16_round_double_inputs_by_hand(orc):
+    # 1 + 2^-8 lies halfway between 1 and 1 + 2^-7: ties go to the even significand (1.0).
+    assert orc.bf16_round([1.0 + 2.0**-8])[0] == 0x3F80
+    # (1 + 2^-7) + 2^-8 is halfway between 1 + 2^-7 (odd) and 1 + 2^-6 (even): rounds up.
+    assert orc.bf16_round([1.0 + 2.0**-7 + 2.0**-8])[0] == 0x3F82
+    # a hair above the first tie (not representable in binary32) rounds up.
+    assert orc.bf16_round([1.0 + 2.0**-8 + 2.0**-40])[0] == 0x3F81
+    assert orc.bf16_round([-(1.0 + 2.0**-8 + 2.0**-40)])[0] == 0xBF81
+    assert orc.bf16_round([0.0])[0] == 0x0000 and orc.bf16_round([-0.0])[0] == 0x8000
+    # largest finite bf16 and overflow to infinity
+    assert orc.bf16_round([(2 - 2.0**-7) * 2.0**127])[0] == 0x7F7F
+    assert orc.bf16_round([2.0**128])[0] == 0x7F80
+    # smallest subnormal 2^-133, and half of it (a tie with 0, goes to 0)
+    assert orc.bf16_round([2.0**-133])[0] == 0x0001
+    assert orc.bf16_round([2.0**-134])[0] == 0x0000
+    assert orc.bf16_round([1.5 * 2.0**-134 * 2])[0] == 0x0002  # 3 * 2^-134 = 1.5 ulp -> 2 ulp (even)
+    b = np.arange(0, 0x7F80, 7, dtype=np.uint16)
+    assert np.array_equal(orc.bf16_round(orc.bf16_to_f64(b)), b)
+
+
+# ----------------------------------------------------------------------- gate
+
+
+def test_gate_brute_force(orc):
+    X, Wg, bg, *_ = _problem(2, 3, 8, 16, -0.25)
+    Z = orc.gate(X, Wg, bg)
+    x, w, b = _f64(X), _f64(Wg), _f64(bg)
+    for i, j in itertools.product(range(3), range(16)):
+        s = 0.0
+        for k in range(8):
+            s += x[i, k] * w[j, k]
+        assert Z[i, j] == pytest.approx(s + b[j], rel=1e-14, abs=1e-14)
+
+
+def test_gate_torch_and_rows(orc):
+    X, Wg, bg, *_ = _problem(3, 40, 96, 384, 0.1)
+    Z = orc.gate(X, Wg, bg)
+    ref = _f64(X) @ _f64(Wg).T + _f64(bg)
+    assert np.abs(Z - ref).max() < 1e-12
+    rows = np.array([39, 0, 17], np.int32)
+    assert np.array_equal(orc.gate(X, Wg, bg, rows=rows), Z[rows])
+
+
+# ----------------------------------------------------------------------- pack
+
+
+def test_pack_hand_built_identity_gate(orc):
+    """W_g = I, b = 0 gives z = X exactly, so the packing is known by construction."""
+    d = f = 256
+    T_n, K = 128, 8
+    Xv = np.zeros((4, d))
+    Xv[0, [3, 7, 130]] = [1.5, 2.0, 0.75]
+    Xv[0, [5, 200]] = [-1.0, -3.0]
+    ten = [0, 1, 2, 10, 20, 30, 40, 50, 60, 127]               # 10 > K actives in tile 0 of row 1
+    Xv[1, ten] = np.arange(1, 11, dtype=np.float64)
+    Xv[1, 128 + 5] = 4.0
+    Xv[2, :] = -1.0
+    Xv[2, 9] = 0.0                                              # z == 0 is inactive
+    Xv[3, 255] = 0.5
+    X = bf16_bits_from_f64(Xv)
+    Wg = bf16_bits_from_f64(np.eye(f, d))
+    bg = np.zeros(f, np.uint16)
+    Z = orc.gate(X, Wg, bg)
+    assert np.array_equal(Z, _f64(X))
+    p = orc.pack(Z, T_n, K)
+    one = lambda v: int(bf16_bits_from_f64(np.array([v]))[0])  # noqa: E731
+
+    assert p["count"].tolist() == [[2, 1], [10, 1], [0, 0], [0, 1]]
+    assert p["col"][0, 0].tolist() == [3, 7, 0, 0, 0, 0, 0, 0]
+    assert p["val"][0, 0].tolist() == [one(1.5), one(2.0), 0, 0, 0, 0, 0, 0]
+    assert p["col"][0, 1].tolist() == [2, 0, 0, 0, 0, 0, 0, 0]
+    assert p["val"][0, 1].tolist()[0] == one(0.75)
+    assert p["col"][1, 0].tolist() == ten[:8]                   # first K in ascending column order
+    assert p["val"][1, 0].tolist() == [one(v) for v in range(1, 9)]
+    assert p["col"][1, 1].tolist()[0] == 5
+    assert not p["val"][2].any() and not p["col"][2].any()
+    assert p["col"][3, 1].tolist()[0] == 127
+    assert p["row_ovf"].tolist() == [0, 1, 0, 0]
+    assert p["n_ovf"] == 1 and p["ovf_rows"][:1].tolist() == [1]
+    expect_row1 = np.zeros(f)
+    expect_row1[ten] = np.arange(1, 11)
+    expect_row1[133] = 4.0
+    assert np.array_equal(p["g_ovf"][0], bf16_bits_from_f64(expect_row1))
+
+
+@pytest.mark.parametrize("T_n,K", [(128, 8), (128, 16), (64, 4), (256, 8), (256, 256), (128, 128)])
+def test_pack_roundtrip_and_invariants(orc, T_n, K):
+    rng = np.random.default_rng(T_n + K)
+    M, f = 37, 1024
+    # heavy-tailed activity: a few rows dense enough to overflow
+    Z = rng.standard_normal((M, f)) * np.exp(0.9 * rng.standard_normal((M, 1))) - 2.0
+    Z[5, :] = 0.0
+    p = orc.pack(Z, T_n, K)
+    T = f // T_n
+    # round trip to the dense bf16 ReLU
+    G = orc.unpack(p, f, T_n, K)
+    assert np.array_equal(G, orc.bf16_round(np.maximum(Z, 0.0) + 0.0))
+    # counts by a different route
+    cnt = (Z.reshape(M, T, T_n) > 0).sum(-1)
+    assert np.array_equal(p["count"], cnt)
+    assert p["count"].sum() == (Z > 0).sum()
+    assert (p["count"] <= T_n).all()
+    # slots: columns strictly ascending and < T_n, padding is (0, 0)
+    for i in range(M):
+        for t in range(T):
+            n = min(int(p["count"][i, t]), K)
+            c = p["col"][i, t, :n].astype(int)
+            assert (np.diff(c) > 0).all() and (c < T_n).all()
+            assert not p["col"][i, t, n:].any() and not p["val"][i, t, n:].any()
+            assert (Z[i, t * T_n + c] > 0).all()
+    # row routing and its order
+    assert np.array_equal(p["row_ovf"].astype(bool), (cnt > K).any(1))
+    rows = np.nonzero(cnt.max(1) > K)[0]
+    assert p["n_ovf"] == rows.size and np.array_equal(p["ovf_rows"][: rows.size], rows)
+    if K >= T_n:
+        assert p["n_ovf"] == 0
+
+
+def test_pack_single_tile_is_row_ellpack(orc):
+    rng = np.random.default_rng(9)
+    Z = rng.standard_normal((5, 64)) - 1.0
+    p = orc.pack(Z, 64, 64)
+    for i in range(5):
+        nz = np.nonzero(Z[i] > 0)[0]
+        assert p["count"][i, 0] == nz.size
+        assert np.array_equal(p["col"][i, 0, : nz.size], nz)
+        assert np.array_equal(p["val"][i, 0, : nz.size], orc.bf16_round(Z[i, nz]))
+
+
+def test_pack_rejects_unpackable_shapes(orc):
+    Z = np.ones((2, 1024))
+    for T_n, K in [(512, 8), (1024, 64), (96, 8), (128, 0)]:
+        with pytest.raises(ValueError):
+            orc.pack(Z, T_n, K)
+
+
+def test_pack_capacity(orc):
+    Z = np.ones((6, 256))
+    Z[2] = -1
+    p = orc.pack(Z, 128, 8, cap=3)
+    assert p["status"] == 3 and p["n_ovf_total"] == 5 and p["n_ovf"] == 3
+    assert p["ovf_rows"].tolist() == [0, 1, 3]
+
+
+# -------------------------------------------------------------------- forward
+
+
+def test_fwd_brute_force(orc):
+    X, Wg, bg, Wu, Wd, _ = _problem(4, 3, 8, 16, 0.05)
+    Y = orc.ffn_fwd(X, Wg, bg, Wu, Wd)
+    x, wg, b, wu, wd = map(_f64, (X, Wg, bg, Wu, Wd))
+    for i in range(3):
+        for c in range(8):
+            acc = 0.0
+            for j in range(16):
+                z = sum(x[i, k] * wg[j, k] for k in range(8)) + b[j]
+                if z > 0:
+                    u = sum(x[i, k] * wu[j, k] for k in range(8))
+                    acc += z * u * wd[c, j]
+            assert Y[i, c] == pytest.approx(acc, rel=1e-12, abs=1e-14)
+
+
+@pytest.mark.parametrize("bias", [-2.0, 0.0, 1.0])
+def test_fwd_torch(orc, bias):
+    X, Wg, bg, Wu, Wd, _ = _problem(5, 33, 64, 256, bias)
+    Y = orc.ffn_fwd(X, Wg, bg, Wu, Wd)
+    ref = _torch_ffn(X, Wg, bg, Wu, Wd)["Y"]
+    assert _rel(Y, ref) < 1e-12
+    rows = np.array([32, 1, 7], np.int32)
+    assert np.array_equal(orc.ffn_fwd(X, Wg, bg, Wu, Wd, rows=rows), Y[rows])
+
+
+def test_fwd_special_cases(orc):
+    X, Wg, _, Wu, Wd, _ = _problem(6, 9, 32, 128, 0.0)
+    f = 128
+    # nothing active: Y == 0 exactly
+    neg = bf16_bits_from_f64(np.full(f, -1e4))
+    assert not orc.ffn_fwd(X, Wg, neg, Wu, Wd).any()
+    # everything active: ReLU is the identity, a plain bilinear product (torch)
+    pos = bf16_bits_from_f64(np.full(f, 1e4))
+    x, wg, wu, wd, b = map(_f64, (X, Wg, Wu, Wd, pos))
+    full = ((x @ wg.T + b) * (x @ wu.T)) @ wd.T
+    assert _rel(orc.ffn_fwd(X, Wg, pos, Wu, Wd), full) < 1e-12
+    # exactly one active unit j: y = (x.w_g[j] + b_j)(x.w_u[j]) W_d[:, j]
+    j = 37
+    bv = np.full(f, -1e4)
+    bv[j] = 64.0
+    one = bf16_bits_from_f64(bv)
+    Y = orc.ffn_fwd(X, Wg, one, Wu, Wd)
+    closed = np.outer((x @ wg[j] + 64.0) * (x @ wu[j]), wd[:, j])
+    assert _rel(Y, closed) < 1e-13
+
+
+def test_fwd_mask_override(orc):
+    X, Wg, bg, Wu, Wd, _ = _problem(7, 12, 32, 256, -0.5)
+    Z = orc.gate(X, Wg, bg)
+    mask = (Z > 0).astype(np.uint8)
+    Y = orc.ffn_fwd(X, Wg, bg, Wu, Wd)
+    assert np.array_equal(orc.ffn_fwd(X, Wg, bg, Wu, Wd, mask=mask), Y)
+    # flip one unit on: the definition evaluated with that active set (torch, masked)
+    i, j = 3, int(np.argmin(Z[3]))
+    mask[i, j] = 1
+    x, wg, b, wu, wd = map(_f64, (X, Wg, bg, Wu, Wd))
+    z = x @ wg.T + b
+    ref = ((z * mask) * (x @ wu.T)) @ wd.T
+    assert _rel(orc.ffn_fwd(X, Wg, bg, Wu, Wd, mask=mask), ref) < 1e-12
+
+
+@pytest.mark.parametrize("K", [2, 8, 128])
+def test_hybrid_equals_dense(orc, K):
+    """Sparse (ELL rows + dense backup rows) equals the dense definition on bf16(g)."""
+    rng = np.random.default_rng(K)
+    M, d, f = 24, 64, 512
+    X, Wg, bg, Wu, Wd, _ = _problem(K, M, d, f, -1.0)
+    X = bf16_bits_from_f64(_f64(X) * np.exp(0.8 * rng.standard_normal((M, 1))))
+    Z = orc.gate(X, Wg, bg)
+    p = orc.pack(Z, 128, K)
+    if K == 2:
+        assert 0 < p["n_ovf"] < M
+    Yh = orc.ffn_fwd_hybrid(X, Wu, Wd, p, 128, K)
+    Yd = orc.ffn_fwd(X, Wg, bg, Wu, Wd, round_g=True)
+    assert _rel(Yh, Yd) < 1e-12
+    # and rounding g changes the result by about one bf16 half-ulp, not more
+    assert _rel(Yd, orc.ffn_fwd(X, Wg, bg, Wu, Wd)) < 4e-3
+
+
+# ------------------------------------------------------------------- backward
+
+
+@pytest.mark.parametrize("lam", [0.0, 0.3])
+@pytest.mark.parametrize("bias", [-0.7, 0.4])
+def test_bwd_torch_autograd(orc, lam, bias):
+    X, Wg, bg, Wu, Wd, dY = _problem(11, 10, 32, 128, bias)
+    g = orc.ffn_bwd(X, Wg, bg, Wu, Wd, dY, lam)
+    ref = _torch_ffn(X, Wg, bg, Wu, Wd, lam, dY)
+    for k in ("dX", "dW_g", "dW_u", "dW_d", "db_g"):
+        assert _rel(g[k], ref[k]) < 1e-11, k
+
+
+def test_bwd_l1_closed_form(orc):
+    """With dY = 0 only the L1 term remains: dZ = lambda on active units."""
+    X, Wg, bg, Wu, Wd, _ = _problem(12, 14, 32, 256, -0.3)
+    dY = np.zeros((14, 32), np.uint16)
+    lam = 0.125
+    g = orc.ffn_bwd(X, Wg, bg, Wu, Wd, dY, lam)
+    act = (orc.gate(X, Wg, bg) > 0).astype(np.float64)
+    x, wg = _f64(X), _f64(Wg)
+    assert np.allclose(g["db_g"], lam * act.sum(0), rtol=0, atol=1e-12)
+    assert _rel(g["dW_g"], lam * act.T @ x) < 1e-13
+    assert _rel(g["dX"], lam * act @ wg) < 1e-13
+    assert not g["dW_u"].any() and not g["dW_d"].any()
+
+
+def test_bwd_special_and_mask(orc):
+    X, Wg, bg, Wu, Wd, dY = _problem(13, 8, 32, 128, -0.4)
+    neg = bf16_bits_from_f64(np.full(128, -1e4))
+    g0 = orc.ffn_bwd(X, Wg, neg, Wu, Wd, dY, 0.5)
+    assert all(not g0[k].any() for k in g0)
+    mask = (orc.gate(X, Wg, bg) > 0).astype(np.uint8)
+    a = orc.ffn_bwd(X, Wg, bg, Wu, Wd, dY, 0.01)
+    b = orc.ffn_bwd(X, Wg, bg, Wu, Wd, dY, 0.01, mask=mask)
+    for k in a:
+        assert np.array_equal(a[k], b[k]), k
