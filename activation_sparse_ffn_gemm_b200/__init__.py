@@ -1,0 +1,219 @@
+"""Python binding of libtwell, the sm_100a TwELL activation-sparse gated FFN.
+
+Argument marshalling only: every step runs in the CUDA library declared in
+include/twell.h. PyTorch supplies device memory and the current CUDA stream.
+There is no fallback: if libtwell.so is missing or a call fails, an exception
+is raised.
+
+    Y, st = ffn_fwd(X, W_g, b_g, W_u, W_d, T_n=128, K=8)
+    grads = ffn_bwd(X, W_g, W_u, W_d, st, dY, lam=1e-3)
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtwell.so")
+
+OP_PACK, OP_FWD, OP_BWD = 0, 1, 2
+STATUS_OVERFLOW_CAP = 1 << 3
+STATUS_TIMEOUT = 1 << 5
+_STATUS_NAMES = {0: "TWELL_OK", 1: "TWELL_EINVAL", 2: "TWELL_EUNSUPPORTED", 3: "TWELL_EOVERFLOW_CAP",
+                 4: "TWELL_ECUDA", 5: "TWELL_ETIMEOUT", 6: "TWELL_EWORKSPACE"}
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+
+
+class TwellError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {_STATUS_NAMES.get(code, code)} ({lib().twell_status_string(code).decode()})")
+
+
+class TwellHybrid(ctypes.Structure):
+    """Mirror of struct twell_hybrid."""
+
+    _fields_ = [("M", ctypes.c_int32), ("d_ff", ctypes.c_int32), ("T_n", ctypes.c_int32), ("K", ctypes.c_int32),
+                ("ovf_cap", ctypes.c_int32), ("count", _vp), ("val", _vp), ("col", _vp), ("row_ovf", _vp),
+                ("ovf_rows", _vp), ("n_ovf", _vp), ("g_ovf", _vp), ("u_ell", _vp), ("u_ovf", _vp),
+                ("status", _vp)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib():
+    """Loads libtwell.so (built in-tree by activation_sparse_ffn_gemm_b200.build)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "`python -m activation_sparse_ffn_gemm_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            L.twell_status_string.restype = ctypes.c_char_p
+            L.twell_status_string.argtypes = [ctypes.c_int]
+            L.twell_query_support.restype = ctypes.c_int
+            L.twell_query_support.argtypes = [_i64] * 6
+            L.twell_workspace_bytes.restype = ctypes.c_size_t
+            L.twell_workspace_bytes.argtypes = [ctypes.c_int] + [_i64] * 6
+            L.twell_transpose_wd.restype = ctypes.c_int
+            L.twell_transpose_wd.argtypes = [_vp, _i64, _i64, _vp, _vp]
+            L.twell_pack.restype = ctypes.c_int
+            L.twell_pack.argtypes = [_vp, _vp, _vp, _i64, ctypes.POINTER(TwellHybrid), _vp, _vp, ctypes.c_size_t, _vp]
+            L.twell_ffn_fwd.restype = ctypes.c_int
+            L.twell_ffn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, ctypes.POINTER(TwellHybrid), _vp,
+                                        _vp, ctypes.c_size_t, _vp]
+            L.twell_ffn_bwd.restype = ctypes.c_int
+            L.twell_ffn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, ctypes.POINTER(TwellHybrid), _vp,
+                                        ctypes.c_float, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+            L.twell_status_read.restype = ctypes.c_int
+            L.twell_status_read.argtypes = [ctypes.POINTER(TwellHybrid), ctypes.POINTER(ctypes.c_uint32),
+                                            ctypes.c_int, _vp]
+            _lib = L
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(code: int, what: str) -> None:
+    if code != 0:
+        raise TwellError(code, what)
+
+
+def _bf16(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous CUDA bfloat16 tensor")
+    return t
+
+
+def query_support(M, d_model, d_ff, T_n, K, ovf_cap) -> int:
+    return int(lib().twell_query_support(M, d_model, d_ff, T_n, K, ovf_cap))
+
+
+def workspace_bytes(op: int, M: int, d_model: int, d_ff: int, T_n: int, K: int, ovf_cap: int) -> int:
+    return int(lib().twell_workspace_bytes(op, M, d_model, d_ff, T_n, K, ovf_cap))
+
+
+def workspace(op: int, M: int, d_model: int, d_ff: int, T_n: int, K: int, ovf_cap: int, device=None) -> torch.Tensor:
+    n = workspace_bytes(op, M, d_model, d_ff, T_n, K, ovf_cap)
+    if n == 0 and query_support(M, d_model, d_ff, T_n, K, ovf_cap) != 0:
+        _check(query_support(M, d_model, d_ff, T_n, K, ovf_cap), "workspace")
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+class HybridState:
+    """Device buffers of one hybrid TwELL representation (see struct twell_hybrid)."""
+
+    def __init__(self, M: int, d_ff: int, T_n: int = 128, K: int = 8, ovf_cap: Optional[int] = None,
+                 device=None, with_u: bool = True):
+        dev = torch.device(device or "cuda")
+        T = d_ff // T_n
+        cap = M if ovf_cap is None else int(ovf_cap)
+        cap1 = max(cap, 1)
+        self.M, self.d_ff, self.T_n, self.K, self.ovf_cap = M, d_ff, T_n, K, cap
+        self.count = torch.empty((M, T), dtype=torch.int16, device=dev)
+        self.val = torch.empty((M, T, K), dtype=torch.bfloat16, device=dev)
+        self.col = torch.empty((M, T, K), dtype=torch.uint8, device=dev)
+        self.row_ovf = torch.empty(max(M, 1), dtype=torch.uint8, device=dev)
+        self.ovf_rows = torch.empty(cap1, dtype=torch.int32, device=dev)
+        self.n_ovf = torch.zeros(2, dtype=torch.int32, device=dev)
+        self.g_ovf = torch.empty((cap1, d_ff), dtype=torch.bfloat16, device=dev)
+        self.u_ell = torch.empty((M, T, K), dtype=torch.float32, device=dev) if with_u else None
+        self.u_ovf = torch.empty((cap1, d_ff), dtype=torch.float32, device=dev) if with_u else None
+        self.status = torch.zeros(4, dtype=torch.int32, device=dev)
+        self.c = TwellHybrid(M, d_ff, T_n, K, cap, *(
+            (t.data_ptr() if t is not None else None) for t in
+            (self.count, self.val, self.col, self.row_ovf, self.ovf_rows, self.n_ovf, self.g_ovf, self.u_ell,
+             self.u_ovf, self.status)))
+
+    def read_status(self, clear: bool = False, stream=None) -> int:
+        out = ctypes.c_uint32(0)
+        _check(lib().twell_status_read(ctypes.byref(self.c), ctypes.byref(out), int(clear), _stream(stream)),
+               "twell_status_read")
+        return int(out.value)
+
+    def n_overflow(self) -> tuple[int, int]:
+        v = self.n_ovf.cpu().tolist()
+        return int(v[0]), int(v[1])
+
+
+def transpose_wd(W_d: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    _bf16(W_d, "W_d")
+    d, f = W_d.shape
+    out = torch.empty((f, d), dtype=torch.bfloat16, device=W_d.device) if out is None else out
+    _check(lib().twell_transpose_wd(_ptr(W_d), d, f, _ptr(out), _stream(stream)), "twell_transpose_wd")
+    return out
+
+
+def pack(X, W_g, b_g, T_n: int = 128, K: int = 8, ovf_cap: Optional[int] = None, z_debug: bool = False,
+         state: Optional[HybridState] = None, ws: Optional[torch.Tensor] = None, stream=None):
+    """Gate GEMM + TwELL pack + row routing. Returns (state, z or None)."""
+    for t, n in ((X, "X"), (W_g, "W_g"), (b_g, "b_g")):
+        _bf16(t, n)
+    M, d = X.shape
+    f = W_g.shape[0]
+    st = state or HybridState(M, f, T_n, K, ovf_cap, X.device, with_u=False)
+    z = torch.empty((M, f), dtype=torch.float32, device=X.device) if z_debug else None
+    if ws is None:
+        ws = workspace(OP_PACK, M, d, f, T_n, K, st.ovf_cap, X.device)
+    _check(lib().twell_pack(_ptr(X), _ptr(W_g), _ptr(b_g), d, ctypes.byref(st.c), _ptr(z), _ptr(ws), ws.numel(),
+                            _stream(stream)), "twell_pack")
+    return st, z
+
+
+def ffn_fwd(X, W_g, b_g, W_u, W_d, T_n: int = 128, K: int = 8, ovf_cap: Optional[int] = None, W_dt=None,
+            save_for_backward: bool = True, z_debug: bool = False, state: Optional[HybridState] = None,
+            ws: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None, stream=None):
+    """Sparse gated FFN forward. Returns (Y, state) or (Y, state, z) with z_debug."""
+    for t, n in ((X, "X"), (W_g, "W_g"), (b_g, "b_g"), (W_u, "W_u"), (W_d, "W_d")):
+        _bf16(t, n)
+    M, d = X.shape
+    f = W_g.shape[0]
+    st = state or HybridState(M, f, T_n, K, ovf_cap, X.device, with_u=save_for_backward)
+    Y = torch.empty((M, d), dtype=torch.bfloat16, device=X.device) if Y is None else Y
+    z = torch.empty((M, f), dtype=torch.float32, device=X.device) if z_debug else None
+    if ws is None:
+        ws = workspace(OP_FWD, M, d, f, T_n, K, st.ovf_cap, X.device)
+    _check(lib().twell_ffn_fwd(_ptr(X), _ptr(W_g), _ptr(b_g), _ptr(W_u), _ptr(W_d), _ptr(W_dt), d, _ptr(Y),
+                               ctypes.byref(st.c), _ptr(z), _ptr(ws), ws.numel(), _stream(stream)), "twell_ffn_fwd")
+    return (Y, st, z) if z_debug else (Y, st)
+
+
+def ffn_bwd(X, W_g, W_u, W_d, state: HybridState, dY, lam: float = 0.0, W_dt=None, with_db: bool = True,
+            ws: Optional[torch.Tensor] = None, out: Optional[dict] = None, stream=None) -> dict:
+    """Backward over the hybrid format. Returns dict dX, dW_g, dW_u, dW_d[, db_g] (fp32)."""
+    for t, n in ((X, "X"), (W_g, "W_g"), (W_u, "W_u"), (W_d, "W_d"), (dY, "dY")):
+        _bf16(t, n)
+    M, d = X.shape
+    f = W_g.shape[0]
+    dev = X.device
+    if out is None:
+        out = dict(dX=torch.empty((M, d), dtype=torch.float32, device=dev),
+                   dW_g=torch.empty((f, d), dtype=torch.float32, device=dev),
+                   dW_u=torch.empty((f, d), dtype=torch.float32, device=dev),
+                   dW_d=torch.empty((d, f), dtype=torch.float32, device=dev))
+        if with_db:
+            out["db_g"] = torch.empty(f, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(OP_BWD, M, d, f, state.T_n, state.K, state.ovf_cap, dev)
+    _check(lib().twell_ffn_bwd(_ptr(X), _ptr(W_g), _ptr(W_u), _ptr(W_d), _ptr(W_dt), d, ctypes.byref(state.c),
+                               _ptr(dY), float(lam), _ptr(out["dX"]), _ptr(out["dW_g"]), _ptr(out["dW_u"]),
+                               _ptr(out["dW_d"]), _ptr(out.get("db_g")), _ptr(ws), ws.numel(), _stream(stream)),
+           "twell_ffn_bwd")
+    return out

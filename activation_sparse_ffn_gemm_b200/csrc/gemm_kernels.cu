@@ -1,0 +1,377 @@
+// gemm_kernels.cu — the tcgen05 GEMMs of the path and their epilogues.
+//
+//   gate + pack   z = X W_g^T + b_g; ReLU and the TwELL pack happen in the
+//                 epilogue, straight out of tensor memory, so the dense z never
+//                 reaches global memory ("Sakana AI и NVIDIA представили TwELL
+//                 — формат и CUDA-ядра ...", paragraph 2: the format is formed in
+//                 the epilogue of the gate-projection kernel, with no separate
+//                 conversion pass). One 256-wide N tile covers two TwELL tiles
+//                 of T_n = 128; each epilogue thread owns one token row, so the
+//                 per-(row, tile) compaction into K slots is thread-local.
+//   dense backup  overflow rows (same page, paragraph 2: rows that overflow
+//                 go to a dense backup) run as dense GEMMs:
+//                 forward  H = bf16(g * (X_ovf W_u^T)),  Y[rows] = bf16(H W_d^T)
+//                 backward [dU | dZ] from dH = dY_ovf W_d,  dX[rows] = dU W_u + dZ W_g
+#include "umma_gemm.cuh"
+
+namespace twell {
+
+namespace {
+
+constexpr int kStages = 4;
+
+__device__ __forceinline__ void load_bias32(const uint16_t* b, float (&out)[32]) {
+  const uint4* p = reinterpret_cast<const uint4*>(b);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float f[8];
+    unpack8(__ldg(p + q), f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[q * 8 + e] = f[e];
+  }
+}
+
+// Keeps the first n of the eight bf16 in v (slot s0 + e kept when s0 + e < n).
+__device__ __forceinline__ uint4 mask_slots(uint4 v, int s0, int n) {
+  uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int lo = s0 + 2 * q, hi = lo + 1;
+    w[q] = (lo < n ? (w[q] & 0x0000FFFFu) : 0u) | (hi < n ? (w[q] & 0xFFFF0000u) : 0u);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// ------------------------------------------------------------- gate + pack
+struct EpiTwell {
+  struct Args {
+    const uint16_t* bias;  // [f] bf16
+    uint16_t* count;       // [M][T]
+    uint16_t* val;         // [M][T][K]
+    uint8_t* col;          // [M][T][K]
+    uint16_t* spill;       // [M][f] dense bf16 ReLU(z), only at tiles with count > K
+    float* z_debug;        // nullable [M][f]
+    int T, K, f;
+  };
+  // per-thread slot staging: K bf16 values + K column bytes (K <= 64)
+  static constexpr int SMEM_BYTES = 128 * kMaxK * 3;
+
+  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int /*N*/, int r, uint32_t taddr,
+                             uint8_t* smem) {
+    const int row = m0 + r;
+    const bool valid = row < M_eff;
+    const int K = a.K;
+    uint16_t* sval = reinterpret_cast<uint16_t*>(smem) + r * kMaxK;
+    uint8_t* scol = smem + 128 * kMaxK * 2 + r * kMaxK;
+#pragma unroll 1
+    for (int tt = 0; tt < 2; ++tt) {
+      const int t = n0 / kTn + tt;
+      if (t >= a.T) break;
+      int cnt = 0;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t v[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(taddr + tt * kTn + ch * 32, v);
+        tmem_wait_ld();
+        float bias[32];
+        load_bias32(a.bias + t * kTn + ch * 32, bias);
+        float z[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) z[c] = __uint_as_float(v[c]) + bias[c];
+        if (a.z_debug != nullptr && valid) {
+          float4* dst = reinterpret_cast<float4*>(a.z_debug + static_cast<size_t>(row) * a.f + t * kTn + ch * 32);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) dst[q] = make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
+        }
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          if (z[c] > 0.f) {
+            if (cnt < K) {
+              sval[cnt] = f32_to_bf16_bits(z[c]);
+              scol[cnt] = static_cast<uint8_t>(ch * 32 + c);
+            }
+            ++cnt;
+          }
+        }
+      }
+      if (valid) {
+        const size_t rt = static_cast<size_t>(row) * a.T + t;
+        a.count[rt] = static_cast<uint16_t>(cnt);
+        const int nk = cnt < K ? cnt : K;
+        uint4* vdst = reinterpret_cast<uint4*>(a.val + rt * K);
+        const uint4* vsrc = reinterpret_cast<const uint4*>(sval);
+        for (int s0 = 0; s0 < K; s0 += 8) vdst[s0 / 8] = mask_slots(vsrc[s0 / 8], s0, nk);
+        if (K == 8) {
+          uint2 c8 = *reinterpret_cast<const uint2*>(scol);
+          uint32_t w[2] = {c8.x, c8.y};
+#pragma unroll
+          for (int b = 0; b < 8; ++b)
+            if (b >= nk) w[b / 4] &= ~(0xFFu << (8 * (b % 4)));
+          *reinterpret_cast<uint2*>(a.col + rt * K) = make_uint2(w[0], w[1]);
+        } else {
+          for (int s0 = 0; s0 < K; s0 += 16) {
+            uint4 c16 = *reinterpret_cast<const uint4*>(scol + s0);
+            uint32_t w[4] = {c16.x, c16.y, c16.z, c16.w};
+#pragma unroll
+            for (int b = 0; b < 16; ++b)
+              if (s0 + b >= nk) w[b / 4] &= ~(0xFFu << (8 * (b % 4)));
+            *reinterpret_cast<uint4*>(a.col + rt * K + s0) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      // An overflowing tile keeps its dense slice so that the row can be
+      // rebuilt densely once the whole row is known to overflow.
+      const bool sp = valid && cnt > K;
+      if (__any_sync(0xFFFFFFFFu, sp)) {
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(taddr + tt * kTn + ch * 32, v);
+          tmem_wait_ld();
+          if (sp) {
+            float bias[32];
+            load_bias32(a.bias + t * kTn + ch * 32, bias);
+            uint4* dst = reinterpret_cast<uint4*>(a.spill + static_cast<size_t>(row) * a.f + t * kTn + ch * 32);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float z[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float zz = __uint_as_float(v[q * 8 + e]) + bias[q * 8 + e];
+                z[e] = zz > 0.f ? zz : 0.f;
+              }
+              dst[q] = make_uint4(pack_bf16x2(z[0], z[1]), pack_bf16x2(z[2], z[3]), pack_bf16x2(z[4], z[5]),
+                                  pack_bf16x2(z[6], z[7]));
+            }
+          }
+        }
+      }
+    }
+  }
+};
+
+// ---------------------------------------- dense backup forward, first GEMM
+struct EpiGateMul {
+  struct Args {
+    const uint16_t* g;  // [cap][f] bf16 ReLU(z)
+    uint16_t* H;        // [cap][f] bf16 g * u
+    float* u_save;      // nullable [cap][f]
+    int f;
+  };
+  static constexpr int SMEM_BYTES = 0;
+  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
+    const int row = m0 + r;
+    const bool valid = row < M_eff;
+#pragma unroll 1
+    for (int ch = 0; ch < 8; ++ch) {
+      const int n = n0 + ch * 32;
+      if (n >= N) break;
+      uint32_t v[32];
+      __syncwarp();
+      tmem_ld_32x32b_x32(taddr + ch * 32, v);
+      tmem_wait_ld();
+      if (!valid) continue;
+      const size_t off = static_cast<size_t>(row) * a.f + n;
+      const uint4* gp = reinterpret_cast<const uint4*>(a.g + off);
+      uint4* hp = reinterpret_cast<uint4*>(a.H + off);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float g8[8];
+        unpack8(gp[q], g8);
+        float h[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) h[e] = g8[e] * __uint_as_float(v[q * 8 + e]);
+        hp[q] = make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]), pack_bf16x2(h[4], h[5]),
+                           pack_bf16x2(h[6], h[7]));
+      }
+      if (a.u_save) {
+        float4* up = reinterpret_cast<float4*>(a.u_save + off);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          up[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
+                              __uint_as_float(v[4 * q + 3]));
+      }
+    }
+  }
+};
+
+// ----------------------------- row-scatter epilogues (bf16 out / fp32 out)
+struct EpiScatterBf16 {
+  struct Args {
+    const int* rows;  // destination row of each GEMM row
+    uint16_t* out;
+    int ld;
+  };
+  static constexpr int SMEM_BYTES = 0;
+  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
+    const int row = m0 + r;
+    const bool valid = row < M_eff;
+    const int dst = valid ? a.rows[row] : 0;
+#pragma unroll 1
+    for (int ch = 0; ch < 8; ++ch) {
+      const int n = n0 + ch * 32;
+      if (n >= N) break;
+      uint32_t v[32];
+      __syncwarp();
+      tmem_ld_32x32b_x32(taddr + ch * 32, v);
+      tmem_wait_ld();
+      if (!valid) continue;
+      uint4* p = reinterpret_cast<uint4*>(a.out + static_cast<size_t>(dst) * a.ld + n);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        p[q] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                          pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                          pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                          pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+    }
+  }
+};
+
+struct EpiScatterF32 {
+  struct Args {
+    const int* rows;
+    float* out;
+    int ld;
+  };
+  static constexpr int SMEM_BYTES = 0;
+  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
+    const int row = m0 + r;
+    const bool valid = row < M_eff;
+    const int dst = valid ? a.rows[row] : 0;
+#pragma unroll 1
+    for (int ch = 0; ch < 8; ++ch) {
+      const int n = n0 + ch * 32;
+      if (n >= N) break;
+      uint32_t v[32];
+      __syncwarp();
+      tmem_ld_32x32b_x32(taddr + ch * 32, v);
+      tmem_wait_ld();
+      if (!valid) continue;
+      float4* p = reinterpret_cast<float4*>(a.out + static_cast<size_t>(dst) * a.ld + n);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        p[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
+                           __uint_as_float(v[4 * q + 3]));
+    }
+  }
+};
+
+// -------------------------------------- dense backup backward, dH epilogue
+struct EpiBwdDH {
+  struct Args {
+    const uint16_t* g;  // [cap][f]
+    const float* u;     // [cap][f]
+    uint16_t* duz;      // [cap][2f] bf16: dU in [0, f), dZ in [f, 2f) (tensor-core operand of dX)
+    float* du;          // [cap][f] fp32 dU (weight gradients)
+    float* dz;          // [cap][f] fp32 dZ (weight gradients)
+    float lambda;
+    int f;
+  };
+  static constexpr int SMEM_BYTES = 0;
+  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
+    const int row = m0 + r;
+    const bool valid = row < M_eff;
+#pragma unroll 1
+    for (int ch = 0; ch < 8; ++ch) {
+      const int n = n0 + ch * 32;
+      if (n >= N) break;
+      uint32_t v[32];
+      __syncwarp();
+      tmem_ld_32x32b_x32(taddr + ch * 32, v);
+      tmem_wait_ld();
+      if (!valid) continue;
+      const size_t off = static_cast<size_t>(row) * a.f + n;
+      const uint4* gp = reinterpret_cast<const uint4*>(a.g + off);
+      const float4* up = reinterpret_cast<const float4*>(a.u + off);
+      uint4* dup = reinterpret_cast<uint4*>(a.duz + static_cast<size_t>(row) * 2 * a.f + n);
+      uint4* dzp = reinterpret_cast<uint4*>(a.duz + static_cast<size_t>(row) * 2 * a.f + a.f + n);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float g8[8];
+        unpack8(gp[q], g8);
+        const float4 u0 = up[2 * q], u1 = up[2 * q + 1];
+        const float u8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+        float du[8], dz[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float dh = __uint_as_float(v[q * 8 + e]);
+          du[e] = dh * g8[e];
+          dz[e] = g8[e] > 0.f ? fmaf(dh, u8[e], a.lambda) : 0.f;
+        }
+        dup[q] = make_uint4(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]), pack_bf16x2(du[4], du[5]),
+                            pack_bf16x2(du[6], du[7]));
+        float4* du32 = reinterpret_cast<float4*>(a.du + off) + 2 * q;
+        float4* dz32 = reinterpret_cast<float4*>(a.dz + off) + 2 * q;
+        du32[0] = make_float4(du[0], du[1], du[2], du[3]);
+        du32[1] = make_float4(du[4], du[5], du[6], du[7]);
+        dz32[0] = make_float4(dz[0], dz[1], dz[2], dz[3]);
+        dz32[1] = make_float4(dz[4], dz[5], dz[6], dz[7]);
+        dzp[q] = make_uint4(pack_bf16x2(dz[0], dz[1]), pack_bf16x2(dz[2], dz[3]), pack_bf16x2(dz[4], dz[5]),
+                            pack_bf16x2(dz[6], dz[7]));
+      }
+    }
+  }
+};
+
+}  // namespace
+
+// -------------------------------------------------------------- launchers
+
+cudaError_t launch_gate_pack(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_g, int M, int d, int f,
+                             int K, const PackOut& out, uint32_t* status, cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  CUtensorMap ta, tb;
+  if (!make_tmap_bf16(&ta, X, d, M, static_cast<uint64_t>(d) * 2, kBK, kBM) ||
+      !make_tmap_bf16(&tb, W_g, d, f, static_cast<uint64_t>(d) * 2, kBK, 256))
+    return cudaErrorInvalidValue;
+  GemmShape shp{M, nullptr, f, d, 0, status};
+  EpiTwell::Args ea{b_g, out.count, out.val, out.col, out.spill, out.z_debug, f / kTn, K, f};
+  return launch_umma_gemm<EpiTwell, 256, false, kStages>(ta, tb, ta, tb, shp, ea, s);
+}
+
+cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uint16_t* W_d,
+                           const uint16_t* g_ovf, const int* ovf_rows, const int* n_ovf, int cap, int d, int f,
+                           uint16_t* h_ovf, float* u_ovf, uint16_t* Y, uint32_t* status, cudaStream_t s) {
+  if (cap <= 0) return cudaSuccess;
+  CUtensorMap ta, tb, ta2, tb2;
+  if (!make_tmap_bf16(&ta, x_ovf, d, cap, static_cast<uint64_t>(d) * 2, kBK, kBM) ||
+      !make_tmap_bf16(&tb, W_u, d, f, static_cast<uint64_t>(d) * 2, kBK, 256) ||
+      !make_tmap_bf16(&ta2, h_ovf, f, cap, static_cast<uint64_t>(f) * 2, kBK, kBM) ||
+      !make_tmap_bf16(&tb2, W_d, f, d, static_cast<uint64_t>(f) * 2, kBK, 256))
+    return cudaErrorInvalidValue;
+  GemmShape s1{cap, n_ovf, f, d, 0, status};
+  EpiGateMul::Args e1{g_ovf, h_ovf, u_ovf, f};
+  cudaError_t e = launch_umma_gemm<EpiGateMul, 256, false, kStages>(ta, tb, ta, tb, s1, e1, s);
+  if (e != cudaSuccess) return e;
+  GemmShape s2{cap, n_ovf, d, f, 0, status};
+  EpiScatterBf16::Args e2{ovf_rows, Y, d};
+  return launch_umma_gemm<EpiScatterBf16, 256, false, kStages>(ta2, tb2, ta2, tb2, s2, e2, s);
+}
+
+cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const uint16_t* W_u,
+                           const uint16_t* W_g, const uint16_t* g_ovf, const float* u_ovf, float lambda,
+                           const int* ovf_rows, const int* n_ovf, int cap, int d, int f, uint16_t* duz_ovf,
+                           float* du_ovf, float* dz_ovf, float* dX, uint32_t* status, cudaStream_t s) {
+  if (cap <= 0) return cudaSuccess;
+  CUtensorMap ta, tb, tdu, tdz, twu, twg;
+  // dH = dY_ovf W_d: B = W_dt [f][d] (K-major)
+  if (!make_tmap_bf16(&ta, dy_ovf, d, cap, static_cast<uint64_t>(d) * 2, kBK, kBM) ||
+      !make_tmap_bf16(&tb, W_dt, d, f, static_cast<uint64_t>(d) * 2, kBK, 256) ||
+      // dX = dU W_u + dZ W_g: A segments are the two halves of duz, B = W_u / W_g as [K=f][N=d] (MN-major)
+      !make_tmap_bf16(&tdu, duz_ovf, f, cap, static_cast<uint64_t>(f) * 4, kBK, kBM) ||
+      !make_tmap_bf16(&tdz, duz_ovf + f, f, cap, static_cast<uint64_t>(f) * 4, kBK, kBM) ||
+      !make_tmap_bf16(&twu, W_u, d, f, static_cast<uint64_t>(d) * 2, 64, kBK) ||
+      !make_tmap_bf16(&twg, W_g, d, f, static_cast<uint64_t>(d) * 2, 64, kBK))
+    return cudaErrorInvalidValue;
+  GemmShape s1{cap, n_ovf, f, d, 0, status};
+  EpiBwdDH::Args e1{g_ovf, u_ovf, duz_ovf, du_ovf, dz_ovf, lambda, f};
+  cudaError_t e = launch_umma_gemm<EpiBwdDH, 256, false, kStages>(ta, tb, ta, tb, s1, e1, s);
+  if (e != cudaSuccess) return e;
+  GemmShape s2{cap, n_ovf, d, f, f, status};
+  EpiScatterF32::Args e2{ovf_rows, dX, d};
+  return launch_umma_gemm<EpiScatterF32, 256, true, kStages>(tdu, twu, tdz, twg, s2, e2, s);
+}
+
+}  // namespace twell

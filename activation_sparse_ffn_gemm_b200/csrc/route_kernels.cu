@@ -1,0 +1,214 @@
+// route_kernels.cu — routing of rows between the compact ELL store and the
+// dense backup block, and the small data-movement kernels around it.
+//
+// "Sakana AI и NVIDIA представили TwELL — формат и CUDA-ядра ...", paragraph 2:
+// a hybrid format dynamically routes rows either to a compact ELL matrix or to
+// a dense backup for overflows; paragraph 4: the maximum nonzeros per row can
+// be far above the mean. A row overflows when any of its tiles holds more than
+// K actives. Overflow rows are listed in ascending row order (a deterministic
+// scan), and each listed row is rebuilt densely from its ELL tiles plus the
+// dense slices that the gate epilogue spilled for its overflowing tiles.
+#include "twell_internal.cuh"
+
+namespace twell {
+
+namespace {
+
+constexpr int kScanThreads = 1024;
+constexpr int kScanItems = 16;
+
+// row_ovf[i] = any_t(count[i][t] > K); one warp per row.
+__global__ void row_flags_kernel(const uint16_t* __restrict__ count, int M, int T, int K,
+                                 uint8_t* __restrict__ row_ovf) {
+  const int lane = threadIdx.x & 31;
+  const long warp0 = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long nwarps = (static_cast<long>(gridDim.x) * blockDim.x) >> 5;
+  for (long row = warp0; row < M; row += nwarps) {
+    bool any = false;
+    for (int t = lane; t < T; t += 32) any |= count[row * T + t] > K;
+    any = __any_sync(0xFFFFFFFFu, any);
+    if (lane == 0) row_ovf[row] = any ? 1 : 0;
+  }
+}
+
+// Single-block ascending compaction of flagged rows. Writes ovf_rows[0..min(n, cap)),
+// n_ovf[0] = min(n, cap), n_ovf[1] = n, and sets the capacity bit when n > cap.
+__global__ void __launch_bounds__(kScanThreads) ovf_scan_kernel(const uint8_t* __restrict__ row_ovf, int M,
+                                                                 int cap, int* __restrict__ ovf_rows,
+                                                                 int* __restrict__ n_ovf, uint32_t* status) {
+  __shared__ int warp_tot[kScanThreads / 32];
+  __shared__ int carry_s;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  if (tid == 0) carry_s = 0;
+  __syncthreads();
+  for (long base = 0; base < M; base += static_cast<long>(kScanThreads) * kScanItems) {
+    const long r0 = base + static_cast<long>(tid) * kScanItems;
+    uint8_t f[kScanItems];
+    if (r0 + kScanItems <= M) {
+      const uint4 v = *reinterpret_cast<const uint4*>(row_ovf + r0);
+      const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < kScanItems; ++e) f[e] = (ww[e / 4] >> (8 * (e % 4))) & 0xFFu;
+    } else {
+#pragma unroll
+      for (int e = 0; e < kScanItems; ++e) f[e] = (r0 + e < M) ? row_ovf[r0 + e] : 0;
+    }
+    int mine = 0;
+#pragma unroll
+    for (int e = 0; e < kScanItems; ++e) mine += f[e] != 0;
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_tot[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+      int t = warp_tot[lane];
+      int ti = t;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, ti, o);
+        if (lane >= o) ti += v;
+      }
+      warp_tot[lane] = ti - t;  // exclusive prefix over warps
+    }
+    __syncthreads();
+    int pos = carry_s + warp_tot[w] + incl - mine;
+#pragma unroll
+    for (int e = 0; e < kScanItems; ++e) {
+      if (f[e]) {
+        if (pos < cap) ovf_rows[pos] = static_cast<int>(r0 + e);
+        ++pos;
+      }
+    }
+    __syncthreads();
+    if (tid == kScanThreads - 1) carry_s = pos;
+    __syncthreads();
+  }
+  if (tid == 0) {
+    const int n = carry_s;
+    n_ovf[0] = n < cap ? n : cap;
+    n_ovf[1] = n;
+    if (n > cap) set_status(status, TWELL_STATUS_OVERFLOW_CAP);
+  }
+}
+
+// Dense backup rows: for each stored overflow row, g_ovf[s] = bf16 ReLU(z) rebuilt
+// from the ELL slots (tiles with count <= K) and the spilled slices (count > K);
+// optionally x_ovf[s] = X[row]. One block per slot, grid-stride over slots.
+__global__ void ovf_gather_kernel(const int* __restrict__ n_ovf, const int* __restrict__ ovf_rows,
+                                  const uint16_t* __restrict__ count, const uint16_t* __restrict__ val,
+                                  const uint8_t* __restrict__ col, const uint16_t* __restrict__ spill, int f,
+                                  int K, uint16_t* __restrict__ g_ovf, const uint16_t* __restrict__ X, int d,
+                                  uint16_t* __restrict__ x_ovf) {
+  const int n = n_ovf[0];
+  const int T = f / kTn;
+  for (int sl = blockIdx.x; sl < n; sl += gridDim.x) {
+    const long row = ovf_rows[sl];
+    // 16 chunks of 8 columns per tile
+    for (int ch = threadIdx.x; ch < T * 16; ch += blockDim.x) {
+      const int t = ch >> 4, c0 = (ch & 15) * 8;
+      const int cnt = count[row * (f / kTn) + t];
+      uint4 out;
+      if (cnt > K) {
+        out = *reinterpret_cast<const uint4*>(spill + row * f + t * kTn + c0);
+      } else {
+        uint16_t e[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        const long base = (row * T + t) * K;
+        for (int s = 0; s < cnt; ++s) {
+          const int c = col[base + s];
+          if (c >= c0 && c < c0 + 8) e[c - c0] = val[base + s];
+        }
+        out = make_uint4(e[0] | (uint32_t(e[1]) << 16), e[2] | (uint32_t(e[3]) << 16), e[4] | (uint32_t(e[5]) << 16),
+                         e[6] | (uint32_t(e[7]) << 16));
+      }
+      *reinterpret_cast<uint4*>(g_ovf + static_cast<long>(sl) * f + t * kTn + c0) = out;
+    }
+    if (X != nullptr) {
+      const uint4* src = reinterpret_cast<const uint4*>(X + row * d);
+      uint4* dst = reinterpret_cast<uint4*>(x_ovf + static_cast<long>(sl) * d);
+      for (int q = threadIdx.x; q < d / 8; q += blockDim.x) dst[q] = src[q];
+    }
+  }
+}
+
+__global__ void gather_rows_kernel(const uint16_t* __restrict__ in, const int* __restrict__ rows,
+                                   const int* __restrict__ n_ovf, int d, uint16_t* __restrict__ out) {
+  const int n = n_ovf[0];
+  for (int sl = blockIdx.x; sl < n; sl += gridDim.x) {
+    const uint4* src = reinterpret_cast<const uint4*>(in + static_cast<long>(rows[sl]) * d);
+    uint4* dst = reinterpret_cast<uint4*>(out + static_cast<long>(sl) * d);
+    for (int q = threadIdx.x; q < d / 8; q += blockDim.x) dst[q] = src[q];
+  }
+}
+
+// out[c][r] = in[r][c] for a [rows][cols] bf16 matrix, 64 x 64 tiles through
+// shared memory (16-byte global accesses on both sides).
+__global__ void transpose_bf16_kernel(const uint16_t* __restrict__ in, int rows, int cols,
+                                      uint16_t* __restrict__ out) {
+  __shared__ uint16_t tile[64][64 + 2];
+  const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
+  const int tid = threadIdx.x;  // 256 threads: 64 rows x 8 chunks of 8
+  for (int i = tid; i < 64 * 8; i += 256) {
+    const int r = i >> 3, q = i & 7;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r0 + r < rows && c0 + q * 8 < cols)
+      v = *reinterpret_cast<const uint4*>(in + static_cast<long>(r0 + r) * cols + c0 + q * 8);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      tile[r][q * 8 + 2 * e] = w[e] & 0xFFFFu;
+      tile[r][q * 8 + 2 * e + 1] = w[e] >> 16;
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < 64 * 8; i += 256) {
+    const int c = i >> 3, q = i & 7;
+    if (c0 + c >= cols || r0 + q * 8 >= rows) continue;
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      w[e] = uint32_t(tile[q * 8 + 2 * e][c]) | (uint32_t(tile[q * 8 + 2 * e + 1][c]) << 16);
+    *reinterpret_cast<uint4*>(out + static_cast<long>(c0 + c) * rows + r0 + q * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_route(const uint16_t* count, const uint16_t* val, const uint8_t* col, const uint16_t* spill,
+                         int M, int f, int K, int cap, uint8_t* row_ovf, int* ovf_rows, int* n_ovf,
+                         uint16_t* g_ovf, const uint16_t* X, int d, uint16_t* x_ovf, uint32_t* status,
+                         cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  const int T = f / kTn;
+  const int warps_needed = M;
+  int blocks = (warps_needed + 7) / 8;
+  const int max_blocks = device_sm_count() * 16;
+  if (blocks > max_blocks) blocks = max_blocks;
+  row_flags_kernel<<<blocks, 256, 0, s>>>(count, M, T, K, row_ovf);
+  ovf_scan_kernel<<<1, kScanThreads, 0, s>>>(row_ovf, M, cap, ovf_rows, n_ovf, status);
+  if (cap > 0) {
+    int g = cap < device_sm_count() * 4 ? cap : device_sm_count() * 4;
+    ovf_gather_kernel<<<g, 256, 0, s>>>(n_ovf, ovf_rows, count, val, col, spill, f, K, g_ovf, X, d, x_ovf);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const uint16_t* in, const int* rows, const int* n_ovf, int cap, int d,
+                               uint16_t* out, cudaStream_t s) {
+  if (cap <= 0) return cudaSuccess;
+  int g = cap < device_sm_count() * 4 ? cap : device_sm_count() * 4;
+  gather_rows_kernel<<<g, 256, 0, s>>>(in, rows, n_ovf, d, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_bf16(const uint16_t* in, int rows, int cols, uint16_t* out, cudaStream_t s) {
+  if (rows <= 0 || cols <= 0) return cudaSuccess;
+  dim3 grid((cols + 63) / 64, (rows + 63) / 64);
+  transpose_bf16_kernel<<<grid, 256, 0, s>>>(in, rows, cols, out);
+  return cudaGetLastError();
+}
+
+}  // namespace twell

@@ -1,0 +1,313 @@
+// twell_api.cu — the extern "C" entry points of libtwell: argument validation,
+// workspace layout and the launch sequence of each call. Every step of every
+// call is one of this library's sm_100a kernels; nothing here computes on the
+// host and there is no alternative code path.
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
+#include "twell_internal.cuh"
+
+namespace twell {
+
+// ------------------------------------------------------------ host helpers
+
+int device_sm_count() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+  cache[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace
+
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                    uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || inner == 0 || outer == 0) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+namespace {
+
+constexpr size_t kWsAlign = 256;
+
+size_t align_up(size_t x) { return (x + kWsAlign - 1) & ~(kWsAlign - 1); }
+
+struct WsLayout {
+  size_t spill = 0, x_ovf = 0, h_ovf = 0, w_dt = 0;
+  size_t dy_ovf = 0, duz = 0, du_ovf = 0, dz_ovf = 0, du_ell = 0, dz_ell = 0, row_slot = 0, block_cnt = 0, unit_tot = 0, unit_ptr = 0,
+         csc_row = 0, csc_val = 0;
+  size_t total = 0;
+};
+
+WsLayout ws_layout(twell_op op, int64_t M, int64_t d, int64_t f, int64_t K, int64_t cap) {
+  WsLayout L;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t r = o;
+    o = align_up(o + bytes);
+    return r;
+  };
+  const int64_t T = f / kTn;
+  const int64_t cap1 = cap > 0 ? cap : 1;
+  if (op == TWELL_OP_PACK || op == TWELL_OP_FWD) L.spill = take(static_cast<size_t>(M * f * 2));
+  if (op == TWELL_OP_FWD) {
+    L.x_ovf = take(static_cast<size_t>(cap1 * d * 2));
+    L.h_ovf = take(static_cast<size_t>(cap1 * f * 2));
+    L.w_dt = take(static_cast<size_t>(f * d * 2));
+  }
+  if (op == TWELL_OP_BWD) {
+    L.w_dt = take(static_cast<size_t>(f * d * 2));
+    L.dy_ovf = take(static_cast<size_t>(cap1 * d * 2));
+    L.duz = take(static_cast<size_t>(cap1 * 2 * f * 2));
+    L.du_ovf = take(static_cast<size_t>(cap1 * f * 4));
+    L.dz_ovf = take(static_cast<size_t>(cap1 * f * 4));
+    L.du_ell = take(static_cast<size_t>(M * T * K * 4));
+    L.dz_ell = take(static_cast<size_t>(M * T * K * 4));
+    L.row_slot = take(static_cast<size_t>(M * 4));
+    const int64_t nrb = (M + kCscRows - 1) / kCscRows;
+    L.block_cnt = take(static_cast<size_t>(nrb * f * 4));
+    L.unit_tot = take(static_cast<size_t>(f * 4));
+    L.unit_ptr = take(static_cast<size_t>((f + 1) * 4));
+    // every active pair: at most T*K per ELL row and d_ff per dense row
+    const int64_t nnz_cap = (M - cap) * T * K + cap * f;
+    L.csc_row = take(static_cast<size_t>(nnz_cap * 4));
+    L.csc_val = take(static_cast<size_t>(nnz_cap * 16));
+  }
+  L.total = o;
+  return L;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Descriptor and shape checks. With M == 0 there is nothing to read or write,
+// so the per-row arrays may be null (empty tensors have no storage).
+twell_status check_hybrid(const twell_hybrid* h, int64_t d_model) {
+  if (!h) return TWELL_EINVAL;
+  const twell_status st = twell_query_support(h->M, d_model, h->d_ff, h->T_n, h->K, h->ovf_cap);
+  if (st != TWELL_OK) return st;
+  if (h->M == 0) return TWELL_OK;
+  const void* ptrs[] = {h->count, h->val, h->col, h->row_ovf, h->ovf_rows, h->n_ovf, h->g_ovf, h->status};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return TWELL_EINVAL;
+  if ((h->u_ell && !aligned16(h->u_ell)) || (h->u_ovf && !aligned16(h->u_ovf))) return TWELL_EINVAL;
+  return TWELL_OK;
+}
+
+twell_status check_ws(twell_op op, const twell_hybrid* h, int64_t d, void* ws, size_t ws_bytes) {
+  const size_t need = twell_workspace_bytes(op, h->M, d, h->d_ff, h->T_n, h->K, h->ovf_cap);
+  if (need == 0) return TWELL_OK;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kWsAlign - 1)) != 0 || ws_bytes < need) return TWELL_EWORKSPACE;
+  return TWELL_OK;
+}
+
+twell_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TWELL_OK : TWELL_ECUDA; }
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+twell_status run_pack(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_g, int64_t d, twell_hybrid* h,
+                      float* z_debug, void* ws, const WsLayout& L, const uint16_t* X_for_gather,
+                      uint16_t* x_ovf, cudaStream_t s) {
+  const int M = h->M, f = h->d_ff, K = h->K, cap = h->ovf_cap;
+  PackOut po{h->count, h->val, h->col, at<uint16_t>(ws, L.spill), z_debug};
+  cudaError_t e = launch_gate_pack(X, W_g, b_g, M, static_cast<int>(d), f, K, po, h->status, s);
+  if (e != cudaSuccess) return TWELL_ECUDA;
+  e = launch_route(h->count, h->val, h->col, po.spill, M, f, K, cap, h->row_ovf, h->ovf_rows, h->n_ovf, h->g_ovf,
+                   X_for_gather, static_cast<int>(d), x_ovf, h->status, s);
+  return cuda_status(e);
+}
+
+}  // namespace
+}  // namespace twell
+
+using namespace twell;
+
+extern "C" {
+
+const char* twell_status_string(twell_status s) {
+  switch (s) {
+    case TWELL_OK: return "ok";
+    case TWELL_EINVAL: return "invalid argument (null or misaligned pointer, bad descriptor)";
+    case TWELL_EUNSUPPORTED: return "unsupported shape";
+    case TWELL_EOVERFLOW_CAP: return "more overflow rows than ovf_cap";
+    case TWELL_ECUDA: return "CUDA call failed";
+    case TWELL_ETIMEOUT: return "device-side wait timed out";
+    case TWELL_EWORKSPACE: return "workspace too small or misaligned";
+  }
+  return "unknown status";
+}
+
+twell_status twell_query_support(int64_t M, int64_t d_model, int64_t d_ff, int64_t T_n, int64_t K,
+                                 int64_t ovf_cap) {
+  if (M < 0 || d_model <= 0 || d_ff <= 0 || T_n <= 0 || K <= 0 || ovf_cap < 0) return TWELL_EINVAL;
+  if (T_n != kTn) return TWELL_EUNSUPPORTED;
+  if (!(K == 8 || K == 16 || K == 32 || K == 64)) return TWELL_EUNSUPPORTED;
+  if (d_model % 64 != 0 || d_model > kMaxDModel) return TWELL_EUNSUPPORTED;
+  if (d_ff % kTn != 0 || d_ff > kMaxTiles * kTn) return TWELL_EUNSUPPORTED;
+  if (M > (int64_t(1) << 24) || ovf_cap > M) return TWELL_EUNSUPPORTED;
+  return TWELL_OK;
+}
+
+size_t twell_workspace_bytes(twell_op op, int64_t M, int64_t d_model, int64_t d_ff, int64_t T_n, int64_t K,
+                             int64_t ovf_cap) {
+  if (twell_query_support(M, d_model, d_ff, T_n, K, ovf_cap) != TWELL_OK) return 0;
+  if (op != TWELL_OP_PACK && op != TWELL_OP_FWD && op != TWELL_OP_BWD) return 0;
+  return ws_layout(op, M, d_model, d_ff, K, ovf_cap).total;
+}
+
+twell_status twell_transpose_wd(const uint16_t* W_d, int64_t d_model, int64_t d_ff, uint16_t* W_dt,
+                                twell_stream_t stream) {
+  if (!W_d || !W_dt || !aligned16(W_d) || !aligned16(W_dt) || d_model <= 0 || d_ff <= 0) return TWELL_EINVAL;
+  if (d_model % 64 != 0 || d_ff % 64 != 0 || d_model > kMaxDModel || d_ff > kMaxTiles * kTn)
+    return TWELL_EUNSUPPORTED;
+  return cuda_status(launch_transpose_bf16(W_d, static_cast<int>(d_model), static_cast<int>(d_ff), W_dt,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+twell_status twell_pack(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_g, int64_t d_model,
+                        twell_hybrid* h, float* z_debug, void* ws, size_t ws_bytes, twell_stream_t stream) {
+  twell_status st = check_hybrid(h, d_model);
+  if (st != TWELL_OK || h->M == 0) return st;
+  if (!X || !W_g || !b_g || !aligned16(X) || !aligned16(W_g) || !aligned16(b_g)) return TWELL_EINVAL;
+  if (z_debug && !aligned16(z_debug)) return TWELL_EINVAL;
+  st = check_ws(TWELL_OP_PACK, h, d_model, ws, ws_bytes);
+  if (st != TWELL_OK) return st;
+  if (h->M == 0) return TWELL_OK;
+  const WsLayout L = ws_layout(TWELL_OP_PACK, h->M, d_model, h->d_ff, h->K, h->ovf_cap);
+  return run_pack(X, W_g, b_g, d_model, h, z_debug, ws, L, nullptr, nullptr,
+                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+twell_status twell_ffn_fwd(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_g, const uint16_t* W_u,
+                           const uint16_t* W_d, const uint16_t* W_dt, int64_t d_model, uint16_t* Y,
+                           twell_hybrid* h, float* z_debug, void* ws, size_t ws_bytes, twell_stream_t stream) {
+  twell_status st = check_hybrid(h, d_model);
+  if (st != TWELL_OK || h->M == 0) return st;
+  const void* in[] = {X, W_g, b_g, W_u, W_d, Y};
+  for (const void* p : in)
+    if (!p || !aligned16(p)) return TWELL_EINVAL;
+  if ((W_dt && !aligned16(W_dt)) || (z_debug && !aligned16(z_debug))) return TWELL_EINVAL;
+  st = check_ws(TWELL_OP_FWD, h, d_model, ws, ws_bytes);
+  if (st != TWELL_OK) return st;
+  if (h->M == 0) return TWELL_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int M = h->M, d = static_cast<int>(d_model), f = h->d_ff, K = h->K, cap = h->ovf_cap;
+  const WsLayout L = ws_layout(TWELL_OP_FWD, M, d, f, K, cap);
+  const uint16_t* wdt = W_dt;
+  if (!wdt) {
+    uint16_t* t = at<uint16_t>(ws, L.w_dt);
+    if (launch_transpose_bf16(W_d, d, f, t, s) != cudaSuccess) return TWELL_ECUDA;
+    wdt = t;
+  }
+  uint16_t* x_ovf = at<uint16_t>(ws, L.x_ovf);
+  st = run_pack(X, W_g, b_g, d, h, z_debug, ws, L, X, x_ovf, s);
+  if (st != TWELL_OK) return st;
+  if (launch_ell_ffn_fwd(X, W_u, wdt, h->count, h->val, h->col, h->row_ovf, h->u_ell, Y, M, d, f, K, s) !=
+      cudaSuccess)
+    return TWELL_ECUDA;
+  return cuda_status(launch_ovf_fwd(x_ovf, W_u, W_d, h->g_ovf, h->ovf_rows, h->n_ovf, cap, d, f,
+                                    at<uint16_t>(ws, L.h_ovf), h->u_ovf, Y, h->status, s));
+}
+
+twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_t* W_u, const uint16_t* W_d,
+                           const uint16_t* W_dt, int64_t d_model, const twell_hybrid* h, const uint16_t* dY,
+                           float lambda, float* dX, float* dW_g, float* dW_u, float* dW_d, float* db_g, void* ws,
+                           size_t ws_bytes, twell_stream_t stream) {
+  twell_status st = check_hybrid(h, d_model);
+  if (st != TWELL_OK) return st;
+  const void* wout[] = {dW_g, dW_u, dW_d};
+  for (const void* p : wout)
+    if (!p || !aligned16(p)) return TWELL_EINVAL;
+  if (db_g && !aligned16(db_g)) return TWELL_EINVAL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int M = h->M, d = static_cast<int>(d_model), f = h->d_ff, K = h->K, cap = h->ovf_cap;
+  if (M > 0) {
+    const void* in[] = {X, W_g, W_u, W_d, dY, dX, h->u_ell, h->u_ovf};
+    for (const void* p : in)
+      if (!p || !aligned16(p)) return TWELL_EINVAL;
+    if (W_dt && !aligned16(W_dt)) return TWELL_EINVAL;
+    st = check_ws(TWELL_OP_BWD, h, d_model, ws, ws_bytes);
+    if (st != TWELL_OK) return st;
+  }
+  if (M == 0) {
+    // no tokens: every gradient is zero
+    cudaError_t e = cudaMemsetAsync(dW_g, 0, static_cast<size_t>(f) * d * 4, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dW_u, 0, static_cast<size_t>(f) * d * 4, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dW_d, 0, static_cast<size_t>(f) * d * 4, s);
+    if (e == cudaSuccess && db_g) e = cudaMemsetAsync(db_g, 0, static_cast<size_t>(f) * 4, s);
+    return cuda_status(e);
+  }
+  const WsLayout L = ws_layout(TWELL_OP_BWD, M, d, f, K, cap);
+  const uint16_t* wdt = W_dt;
+  if (!wdt) {
+    uint16_t* t = at<uint16_t>(ws, L.w_dt);
+    if (launch_transpose_bf16(W_d, d, f, t, s) != cudaSuccess) return TWELL_ECUDA;
+    wdt = t;
+  }
+  uint16_t* dy_ovf = at<uint16_t>(ws, L.dy_ovf);
+  uint16_t* duz = at<uint16_t>(ws, L.duz);
+  float* du_ell = at<float>(ws, L.du_ell);
+  float* dz_ell = at<float>(ws, L.dz_ell);
+  if (launch_gather_rows(dY, h->ovf_rows, h->n_ovf, cap, d, dy_ovf, s) != cudaSuccess) return TWELL_ECUDA;
+  if (launch_ell_ffn_bwd(dY, W_u, W_g, wdt, h->count, h->val, h->col, h->row_ovf, h->u_ell, lambda, du_ell, dz_ell,
+                         dX, M, d, f, K, s) != cudaSuccess)
+    return TWELL_ECUDA;
+  float* du_ovf = at<float>(ws, L.du_ovf);
+  float* dz_ovf = at<float>(ws, L.dz_ovf);
+  if (launch_ovf_bwd(dy_ovf, wdt, W_u, W_g, h->g_ovf, h->u_ovf, lambda, h->ovf_rows, h->n_ovf, cap, d, f, duz,
+                     du_ovf, dz_ovf, dX, h->status, s) != cudaSuccess)
+    return TWELL_ECUDA;
+  CscBuffers b{at<int>(ws, L.row_slot), at<int>(ws, L.block_cnt), at<int>(ws, L.unit_tot),
+               at<int>(ws, L.unit_ptr), at<int>(ws, L.csc_row), at<float4>(ws, L.csc_val)};
+  if (launch_build_csc(h->count, h->val, h->col, h->row_ovf, h->ovf_rows, h->n_ovf, h->g_ovf, h->u_ell, h->u_ovf,
+                       du_ell, dz_ell, du_ovf, dz_ovf, M, f, K, cap, b, s) != cudaSuccess)
+    return TWELL_ECUDA;
+  return cuda_status(launch_weight_grads(X, dY, b, d, f, dW_g, dW_u, dW_d, db_g, s));
+}
+
+twell_status twell_status_read(const twell_hybrid* h, uint32_t* out, int clear, twell_stream_t stream) {
+  if (!h || !h->status || !out) return TWELL_EINVAL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, h->status, sizeof v, cudaMemcpyDeviceToHost, s) != cudaSuccess) return TWELL_ECUDA;
+  if (clear && cudaMemsetAsync(h->status, 0, sizeof(uint32_t), s) != cudaSuccess) return TWELL_ECUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return TWELL_ECUDA;
+  *out = v;
+  return TWELL_OK;
+}
+
+}  // extern "C"

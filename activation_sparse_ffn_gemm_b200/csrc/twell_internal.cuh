@@ -1,0 +1,132 @@
+// twell_internal.cuh — declarations shared by the translation units of libtwell
+// (device helpers, the workspace/problem descriptors and the launchers). Not
+// part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "twell.h"
+
+namespace twell {
+
+constexpr int kTn = 128;           // TwELL tile width (columns of one GEMM N-tile half)
+constexpr int kMaxK = 64;          // widest ELL row per tile
+constexpr int kMaxTiles = 128;     // d_ff <= 16384
+constexpr int kMaxDModel = 16384;  // 128 threads x 16 chunks x 8 bf16
+
+// ------------------------------------------------------------ device helpers
+
+__device__ __forceinline__ void set_status(uint32_t* status, uint32_t bits) {
+  if (status) atomicOr(status, bits);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float x) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  return static_cast<uint32_t>(f32_to_bf16_bits(lo)) | (static_cast<uint32_t>(f32_to_bf16_bits(hi)) << 16);
+}
+
+// Eight bf16 (one uint4) -> eight floats.
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+  f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x);
+  f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+  f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z);
+  f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+}
+
+// ------------------------------------------------------------ host helpers
+
+int device_sm_count();
+
+// Encodes a 2-D bf16 tensor map (128-byte swizzle, zero fill out of bounds).
+// inner = contiguous extent (elements), outer = rows, row_bytes = row pitch.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                    uint32_t box_inner, uint32_t box_outer);
+
+// ------------------------------------------------------------ launchers
+// All launchers enqueue on `s` and return the launch error (cudaSuccess when
+// nothing needed launching).
+
+struct PackOut {
+  uint16_t* count;
+  uint16_t* val;
+  uint8_t* col;
+  uint16_t* spill;  // [M][f], written only at tiles with count > K
+  float* z_debug;   // nullable
+};
+
+// Gate GEMM z = X W_g^T + b_g with the ReLU + TwELL pack epilogue.
+cudaError_t launch_gate_pack(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_g, int M, int d, int f,
+                             int K, const PackOut& out, uint32_t* status, cudaStream_t s);
+
+// Row routing: flags, ascending overflow list, dense backup rows (and the
+// gathered X rows of overflow rows when x_ovf != nullptr).
+cudaError_t launch_route(const uint16_t* count, const uint16_t* val, const uint8_t* col, const uint16_t* spill,
+                         int M, int f, int K, int cap, uint8_t* row_ovf, int* ovf_rows, int* n_ovf,
+                         uint16_t* g_ovf, const uint16_t* X, int d, uint16_t* x_ovf, uint32_t* status,
+                         cudaStream_t s);
+
+// out[s][:] = in[rows[s]][:] for s < n_ovf[0] (bf16 rows of width d).
+cudaError_t launch_gather_rows(const uint16_t* in, const int* rows, const int* n_ovf, int cap, int d,
+                               uint16_t* out, cudaStream_t s);
+
+cudaError_t launch_transpose_bf16(const uint16_t* in, int rows, int cols, uint16_t* out, cudaStream_t s);
+
+// Fused sparse up + down over the ELL rows (overflow rows are skipped).
+cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
+                               const uint16_t* count, const uint16_t* val, const uint8_t* col,
+                               const uint8_t* row_ovf, float* u_ell, uint16_t* Y, int M, int d, int f, int K,
+                               cudaStream_t s);
+
+// Dense backup forward for overflow rows: H = bf16(G * (X_ovf W_u^T)) then
+// Y[ovf_rows] = bf16(H W_d^T).
+cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uint16_t* W_d,
+                           const uint16_t* g_ovf, const int* ovf_rows, const int* n_ovf, int cap, int d, int f,
+                           uint16_t* h_ovf, float* u_ovf, uint16_t* Y, uint32_t* status, cudaStream_t s);
+
+// Sparse backward over the ELL rows: dH at kept actives, dU, dZ (stored per
+// slot) and the rows of dX.
+cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const uint16_t* W_g,
+                               const uint16_t* W_dt, const uint16_t* count, const uint16_t* val,
+                               const uint8_t* col, const uint8_t* row_ovf, const float* u_ell, float lambda,
+                               float* du_ell, float* dz_ell, float* dX, int M, int d, int f, int K,
+                               cudaStream_t s);
+
+// Dense backup backward for overflow rows: dU, dZ (fp32, and bf16 [dU | dZ] as
+// the next GEMM's operand) from dH = dY_ovf W_d, then dX[ovf_rows] = dU W_u + dZ W_g.
+cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const uint16_t* W_u,
+                           const uint16_t* W_g, const uint16_t* g_ovf, const float* u_ovf, float lambda,
+                           const int* ovf_rows, const int* n_ovf, int cap, int d, int f, uint16_t* duz_ovf,
+                           float* du_ovf, float* dz_ovf, float* dX, uint32_t* status, cudaStream_t s);
+
+struct CscBuffers {
+  int* row_slot;   // [M]
+  int* block_cnt;  // [ceil(M/kCscRows)][f]
+  int* unit_tot;   // [f]
+  int* unit_ptr;   // [f+1]
+  int* csc_row;    // [nnz_cap]
+  float4* csc_val; // [nnz_cap]: (h, dU, dZ, 0)
+};
+constexpr int kCscRows = 64;
+
+// Unit-major list of every active (row, unit) pair of the hybrid format, in
+// ascending row order per unit, with h, dU and dZ attached.
+cudaError_t launch_build_csc(const uint16_t* count, const uint16_t* val, const uint8_t* col,
+                             const uint8_t* row_ovf, const int* ovf_rows, const int* n_ovf, const uint16_t* g_ovf,
+                             const float* u_ell, const float* u_ovf, const float* du_ell, const float* dz_ell,
+                             const float* du_ovf, const float* dz_ovf, int M, int f, int K, int cap,
+                             const CscBuffers& b, cudaStream_t s);
+
+// dW_u = dU^T X, dW_g = dZ^T X, dW_d = dY^T H, db_g = column sums of dZ.
+cudaError_t launch_weight_grads(const uint16_t* X, const uint16_t* dY, const CscBuffers& b, int d, int f,
+                                float* dW_g, float* dW_u, float* dW_d, float* db_g, cudaStream_t s);
+
+}  // namespace twell

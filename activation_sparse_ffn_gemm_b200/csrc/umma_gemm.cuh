@@ -1,0 +1,294 @@
+// umma_gemm.cuh — persistent, warp-specialised bf16 GEMM for sm_100a:
+//   C[M x N] = sum over K segments of A_s[M x K_s] * B_s^T, fp32 accumulation
+// with a pluggable epilogue that reads the accumulator straight from tensor
+// memory. A is K-major (rows of A contiguous along K); B is either K-major
+// ([N][K], like nn.Linear weights) or MN-major ([K][N]).
+//
+// Roles inside one 192-thread CTA (one CTA per SM):
+//   warp 0      TMA producer: 128-byte-swizzled A/B tiles into a STAGES-deep
+//               shared-memory ring, completion tracked by transaction bytes
+//   warp 1      tensor-memory allocation and the single thread that issues
+//               tcgen05.mma (128 x BN x 16 per instruction) and commits
+//   warps 2..5  epilogue: tcgen05.ld of the 128 x BN fp32 accumulator, one
+//               accumulator row per thread, then Epi::run
+// The accumulator is double-buffered in tensor memory (2 x BN columns), so the
+// epilogue of tile i overlaps the main loop of tile i+1. Tiles are visited in
+// groups of 16 M-blocks so that concurrently resident CTAs share A and B
+// panels in L2. Rows may be a device-side count (M_dev), so the dense backup
+// GEMMs need no host synchronisation to learn how many rows overflowed.
+//
+// Every wait is bounded (sm100.cuh); a CTA that gives up sets
+// TWELL_STATUS_TIMEOUT, lets the other roles unwind, waits for its own
+// outstanding copies and MMAs, frees its tensor memory and returns.
+#pragma once
+
+#include "sm100.cuh"
+#include "twell_internal.cuh"
+
+namespace twell {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;  // 64 bf16 = 128 bytes: one swizzle row
+constexpr int kGemmThreads = 192;
+constexpr int kGroupM = 16;
+
+struct GemmShape {
+  int M;             // static bound on rows of A / C
+  const int* M_dev;  // nullable: rows processed = min(*M_dev, M)
+  int N;             // columns of C
+  int K0;            // K extent of segment 0 (multiple of kBK)
+  int K1;            // K extent of segment 1 (0: single segment)
+  uint32_t* status;
+};
+
+template <int BN, int STAGES>
+struct GemmLayout {
+  static constexpr int A_BYTES = kBM * kBK * 2;
+  static constexpr int B_BYTES = BN * kBK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int NBAR = 2 * STAGES + 5;  // full, empty, tmem_full[2], tmem_empty[2], drain
+  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int EPI_OFF = (MISC_OFF + 16 + 127) / 128 * 128;
+  static constexpr int TMEM_COLS = 2 * BN;
+};
+
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
+  const int per_group = kGroupM * num_n;
+  const int group = tile / per_group;
+  const int first_m = group * kGroupM;
+  const int gm = min(kGroupM, num_m - first_m);
+  const int within = tile - group * per_group;
+  mb = first_m + within % gm;
+  nb = within / gm;
+}
+
+template <class Epi, int BN, bool B_MN, int STAGES>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                     const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                     const GemmShape shp, const typename Epi::Args ea) {
+  using L = GemmLayout<BN, STAGES>;
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "UMMA N tile");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+  int* m_eff_s = reinterpret_cast<int*>(smem + L::MISC_OFF + 8);
+  uint8_t* epi_smem = smem + L::EPI_OFF;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    int m = shp.M;
+    if (shp.M_dev) {
+      const int v = *shp.M_dev;
+      m = v < m ? v : m;
+      m = m < 0 ? 0 : m;
+    }
+    *m_eff_s = m;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA0);
+    prefetch_tensormap(&tmB0);
+    if (shp.K1 > 0) {
+      prefetch_tensormap(&tmA1);
+      prefetch_tensormap(&tmB1);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int M_eff = *m_eff_s;
+
+  const int num_m = (M_eff + kBM - 1) / kBM;
+  const int num_n = (shp.N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int nk0 = shp.K0 / kBK;
+  const int nk = nk0 + shp.K1 / kBK;
+
+  auto fail = [&]() {
+    *abort_flag = 1;
+    set_status(shp.status, TWELL_STATUS_TIMEOUT);
+  };
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0;      // stages with a load issued
+      uint32_t issued_par = 0;  // phase parity of that load
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        int mb, nb;
+        tile_coords(tile, num_m, num_n, mb, nb);
+        const int m0 = mb * kBM, n0 = nb * BN;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+            fail();
+            ok = false;
+            break;
+          }
+          uint8_t* sA = smem + stage * L::STAGE_BYTES;
+          uint8_t* sB = sA + L::A_BYTES;
+          mbar_arrive_expect_tx(&full[stage], L::STAGE_BYTES);
+          const bool seg1 = kb >= nk0;
+          const CUtensorMap* mA = seg1 ? &tmA1 : &tmA0;
+          const CUtensorMap* mB = seg1 ? &tmB1 : &tmB0;
+          const int k = (seg1 ? kb - nk0 : kb) * kBK;
+          tma_load_2d(sA, mA, &full[stage], k, m0);
+          if (!B_MN) {
+            tma_load_2d(sB, mB, &full[stage], k, n0);
+          } else {
+#pragma unroll
+            for (int q = 0; q < BN / 64; ++q) tma_load_2d(sB + q * (64 * kBK * 2), mB, &full[stage], n0 + 64 * q, k);
+          }
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // wait (bounded) for the copies this thread started, then unwind
+        int never = 0;
+        for (int s = 0; s < STAGES; ++s)
+          if (issued & (1u << s)) (void)mbar_wait(&full[s], (issued_par >> s) & 1u, &never);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // -------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, false, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true, any = false;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
+          fail();
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+            fail();
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + stage * L::STAGE_BYTES);
+          const uint32_t b_base = a_base + L::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t adesc = sdesc_sw128(a_base + kk * 32, 16, 1024);
+            const uint64_t bdesc = B_MN ? sdesc_sw128(b_base + kk * 2048, 64 * kBK * 2, 1024)
+                                        : sdesc_sw128(b_base + kk * 32, 16, 1024);
+            umma_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          any = true;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok && any) {
+        int never = 0;
+        umma_commit(drain);
+        (void)mbar_wait(drain, 0, &never);
+      }
+    }
+    __syncwarp();
+  } else {
+    // --------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;  // tensor-memory lane quarter this warp may access
+    const int r = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      int mb, nb;
+      tile_coords(tile, num_m, num_n, mb, nb);
+      const bool got = mbar_wait(&tfull[acc], acc_phase, abort_flag);
+      if (!got) {
+        fail();
+        break;
+      }
+      tc_fence_after();
+      __syncwarp();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      Epi::run(ea, mb * kBM, nb * BN, M_eff, shp.N, r, taddr, epi_smem);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::TMEM_COLS);
+  }
+}
+
+template <class Epi, int BN, int STAGES>
+constexpr int gemm_smem_bytes() {
+  return 1024 + GemmLayout<BN, STAGES>::EPI_OFF + Epi::SMEM_BYTES;
+}
+
+// Launches the GEMM on min(#SMs, tiles) persistent CTAs. The static row bound
+// shp.M sizes the grid; rows beyond *M_dev are skipped by the device.
+template <class Epi, int BN, bool B_MN, int STAGES>
+cudaError_t launch_umma_gemm(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
+                             const CUtensorMap& b1, const GemmShape& shp, const typename Epi::Args& ea,
+                             cudaStream_t s) {
+  constexpr int smem = gemm_smem_bytes<Epi, BN, STAGES>();
+  static_assert(smem <= 232448, "shared memory budget");
+  auto kern = umma_gemm_kernel<Epi, BN, B_MN, STAGES>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const long tiles = static_cast<long>((shp.M + kBM - 1) / kBM) * ((shp.N + BN - 1) / BN);
+  if (tiles <= 0) return cudaSuccess;
+  const int grid = static_cast<int>(tiles < device_sm_count() ? tiles : device_sm_count());
+  kern<<<grid, kGemmThreads, smem, s>>>(a0, b0, a1, b1, shp, ea);
+  return cudaGetLastError();
+}
+
+}  // namespace twell

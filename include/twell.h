@@ -1,0 +1,187 @@
+/*
+ * twell.h — C ABI of libtwell: the activation-sparse gated FFN hot path with
+ * TwELL (tile-wise ELLPACK) packing, for NVIDIA B200 (sm_100a).
+ *
+ * Sources of the method (news pages; they print no code and no kernel detail):
+ *   [aivizor]      "Sakana AI и NVIDIA представили TwELL — формат и CUDA-ядра,
+ *                  превращающие активную разреженность в реальные ускорения LLM"
+ *                  (edge.aivizor.me), paragraphs 1-4
+ *   [aimodelsnavi] "How TwELL by Sakana AI and NVIDIA Accelerates LLMs by 20%
+ *                  Using Unstructured Sparsity" (aimodelsnavi.com), sections
+ *                  "Technical Explanation" and "Core of TwELL"
+ *
+ * The block computed (gate / up / down projections, ReLU gate, gate bias):
+ *     z = X W_g^T + b_g      g = ReLU(z)      u = X W_u^T      h = g * u
+ *     Y = h W_d^T
+ * with an optional L1 term lambda * sum(g) on the gate activations in training
+ * ([aivizor] ¶1).
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are row-major device arrays. bf16 tensors are passed as uint16_t
+ *     bit patterns. Weights follow the nn.Linear layout: W_g, W_u are
+ *     [d_ff][d_model], W_d is [d_model][d_ff], b_g is [d_ff].
+ *   - Ownership: the caller allocates every buffer, including the workspace;
+ *     the library never allocates or frees device memory.
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream).
+ *     Argument and shape errors are reported synchronously and nothing is
+ *     enqueued. Device-side conditions (overflow capacity exceeded, a bounded
+ *     wait giving up) set bits in the caller's device status word, read with
+ *     twell_status_read.
+ *   - Base pointers must be 16-byte aligned; the workspace 256-byte aligned.
+ *   - Supported shapes: T_n == 128; K in {8, 16, 32, 64}; d_model a multiple
+ *     of 64 in [64, 16384]; d_ff a multiple of 128 in [128, 16384];
+ *     0 <= M <= 2^24; 0 <= ovf_cap <= M. Anything else returns
+ *     TWELL_EUNSUPPORTED. M == 0 is a valid no-op.
+ *   - No entry point keeps state between calls or falls back to another
+ *     implementation: every step runs in this library's sm_100a kernels.
+ */
+#ifndef TWELL_H
+#define TWELL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TWELL_API __attribute__((visibility("default")))
+#else
+#define TWELL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st* twell_stream_t;
+
+typedef enum twell_status {
+  TWELL_OK = 0,
+  TWELL_EINVAL = 1,         /* null or misaligned pointer, negative size, inconsistent descriptor */
+  TWELL_EUNSUPPORTED = 2,   /* shape outside the supported set above */
+  TWELL_EOVERFLOW_CAP = 3,  /* (device bit) more overflow rows than ovf_cap */
+  TWELL_ECUDA = 4,          /* a CUDA runtime or driver call failed */
+  TWELL_ETIMEOUT = 5,       /* (device bit) a bounded device-side wait gave up */
+  TWELL_EWORKSPACE = 6      /* workspace too small or misaligned */
+} twell_status;
+
+/* Device status word bits, set by kernels and read by twell_status_read. */
+#define TWELL_STATUS_OVERFLOW_CAP (1u << TWELL_EOVERFLOW_CAP)
+#define TWELL_STATUS_TIMEOUT (1u << TWELL_ETIMEOUT)
+
+/*
+ * The hybrid TwELL representation of g = ReLU(z) ([aivizor] ¶2: horizontal
+ * tiles of width T_n aligned with the matmul tile, nonzeros packed locally in
+ * each tile; the training format routes a row either to the compact ELL matrix
+ * or, if it overflows, to a dense backup; [aimodelsnavi] "Core of TwELL":
+ * ELLPACK applied per tile). All arrays are caller-owned device memory.
+ *
+ * Per (row i, tile t), T = d_ff / T_n:
+ *   count[i][t]   true number of units c in the tile with z > 0 (0..T_n), also when > K
+ *   val[i][t][s]  bf16 RNE of z for the s-th active unit in ascending column order,
+ *                 s < min(count, K); 0 in the unused slots
+ *   col[i][t][s]  in-tile column of that unit (0..T_n-1); 0 in the unused slots
+ * Row routing: row i is an overflow row (row_ovf[i] = 1) when some tile has
+ * count > K. Overflow rows are listed in ascending order in ovf_rows; the first
+ * ovf_cap of them get a dense row g_ovf[s][:] = bf16(ReLU(z[i][:])).
+ * n_ovf[0] = rows stored (min(flagged, ovf_cap)), n_ovf[1] = rows flagged.
+ * The ELL slots of an overflow row still hold its first K actives per tile.
+ *
+ * u_ell / u_ovf are written by twell_ffn_fwd when non-NULL and read by
+ * twell_ffn_bwd (which requires both): the up projection u at the kept ELL
+ * slots of non-overflow rows, and the dense u rows of stored overflow rows.
+ */
+typedef struct twell_hybrid {
+  int32_t M;         /* tokens (rows) */
+  int32_t d_ff;      /* hidden width */
+  int32_t T_n;       /* tile width (must be 128) */
+  int32_t K;         /* ELL slots per (row, tile) */
+  int32_t ovf_cap;   /* capacity of the dense backup block, in rows */
+  uint16_t* count;   /* [M][T] */
+  uint16_t* val;     /* [M][T][K] bf16 bits */
+  uint8_t* col;      /* [M][T][K] */
+  uint8_t* row_ovf;  /* [M] */
+  int32_t* ovf_rows; /* [max(ovf_cap,1)] */
+  int32_t* n_ovf;    /* [2] */
+  uint16_t* g_ovf;   /* [max(ovf_cap,1)][d_ff] bf16 bits */
+  float* u_ell;      /* [M][T][K], nullable */
+  float* u_ovf;      /* [max(ovf_cap,1)][d_ff], nullable */
+  uint32_t* status;  /* [1] device status word (TWELL_STATUS_* bits), never cleared by kernels */
+} twell_hybrid;
+
+/* Which call a workspace is sized for. */
+typedef enum twell_op { TWELL_OP_PACK = 0, TWELL_OP_FWD = 1, TWELL_OP_BWD = 2 } twell_op;
+
+/* Short English text for a status code (static storage). */
+TWELL_API const char* twell_status_string(twell_status s);
+
+/* Host-only check of a shape against the supported set; enqueues nothing. */
+TWELL_API twell_status twell_query_support(int64_t M, int64_t d_model, int64_t d_ff, int64_t T_n, int64_t K,
+                                 int64_t ovf_cap);
+
+/* Workspace bytes that `op` needs for this shape (0 for an unsupported shape).
+ * For TWELL_OP_FWD and TWELL_OP_BWD this includes room for a transposed W_d,
+ * used only when the caller passes W_dt == NULL. */
+TWELL_API size_t twell_workspace_bytes(twell_op op, int64_t M, int64_t d_model, int64_t d_ff, int64_t T_n,
+                             int64_t K, int64_t ovf_cap);
+
+/* W_dt[j][c] = W_d[c][j]: the down-projection weight stored unit-major
+ * ([d_ff][d_model]), so that the weights of one hidden unit are contiguous.
+ * Inference callers with fixed weights transpose once and pass W_dt to every
+ * call; training callers may pass W_dt == NULL and let each call transpose. */
+TWELL_API twell_status twell_transpose_wd(const uint16_t* W_d, int64_t d_model, int64_t d_ff, uint16_t* W_dt,
+                                twell_stream_t stream);
+
+/*
+ * Gate projection with the TwELL pack in its epilogue, then row routing
+ * ([aivizor] ¶2 places the packing inside the gate kernel's epilogue, so no
+ * separate conversion pass over a dense z exists).
+ *   X [M][d_model], W_g [d_ff][d_model], b_g [d_ff]  (bf16 bits)
+ *   h        descriptor (M, d_ff, T_n, K, ovf_cap, arrays) filled on the device;
+ *            u_ell / u_ovf are not touched
+ *   z_debug  nullable [M][d_ff] fp32: z = X W_g^T + b_g as the kernel computed it
+ *            (fp32 accumulation, then + b_g), for bit-exact checks of the pack
+ *   ws       workspace of twell_workspace_bytes(TWELL_OP_PACK, ...) bytes
+ */
+TWELL_API twell_status twell_pack(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_g, int64_t d_model,
+                        twell_hybrid* h, float* z_debug, void* ws, size_t ws_bytes,
+                        twell_stream_t stream);
+
+/*
+ * Forward pass of the sparse gated FFN ([aivizor] ¶2: a fused kernel reads the
+ * TwELL activations and performs the up and down projections without writing
+ * the hidden state to global memory; overflow rows take the dense backup path).
+ *   W_u [d_ff][d_model], W_d [d_model][d_ff], W_dt nullable [d_ff][d_model]
+ *   Y   [M][d_model] bf16 bits, fp32 accumulation. Rows routed to the dense
+ *       block beyond ovf_cap are not written (status bit OVERFLOW_CAP is set).
+ *   h   as in twell_pack; also writes u_ell / u_ovf when they are non-NULL
+ *   ws  workspace of twell_workspace_bytes(TWELL_OP_FWD, ...) bytes
+ */
+TWELL_API twell_status twell_ffn_fwd(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_g,
+                           const uint16_t* W_u, const uint16_t* W_d, const uint16_t* W_dt,
+                           int64_t d_model, uint16_t* Y, twell_hybrid* h, float* z_debug, void* ws,
+                           size_t ws_bytes, twell_stream_t stream);
+
+/*
+ * Backward pass over the hybrid format of a previous twell_ffn_fwd (which must
+ * have been given non-NULL u_ell and u_ovf), for L = sum(Y * dY) + lambda * sum(g):
+ *   dH_ij = dY_i . W_d[:, j] at active units;  dU = dH g;  dZ = (dH u + lambda) [z > 0]
+ *   dX = dU W_u + dZ W_g;  dW_d = dY^T H;  dW_u = dU^T X;  dW_g = dZ^T X;  db_g = sum_i dZ
+ *   dY [M][d_model] bf16 bits; dX [M][d_model], dW_g / dW_u [d_ff][d_model],
+ *   dW_d [d_model][d_ff], db_g [d_ff] (nullable): fp32, overwritten (not accumulated).
+ *   ws  workspace of twell_workspace_bytes(TWELL_OP_BWD, ...) bytes
+ */
+TWELL_API twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_t* W_u,
+                           const uint16_t* W_d, const uint16_t* W_dt, int64_t d_model,
+                           const twell_hybrid* h, const uint16_t* dY, float lambda, float* dX,
+                           float* dW_g, float* dW_u, float* dW_d, float* db_g, void* ws,
+                           size_t ws_bytes, twell_stream_t stream);
+
+/* Copies the device status word to *out after synchronizing `stream`; clears
+ * it when `clear` is non-zero. Returns TWELL_ECUDA if the copy fails. */
+TWELL_API twell_status twell_status_read(const twell_hybrid* h, uint32_t* out, int clear, twell_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TWELL_H */

@@ -11,6 +11,7 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
   ffn_fwd           pinned: brute-force loops, torch float64, closed forms
   ffn_fwd_hybrid    pinned: equals ffn_fwd (round_g=1) on the same active set
   ffn_bwd           pinned: torch float64 autograd, closed form of the L1 term
+  gmat input        pinned: with gmat = the oracle's own packed g, equals round_g
 """
 
 from __future__ import annotations
@@ -70,13 +71,13 @@ def lib():
                                         _i32, _u16p]
             L.oracle_ffn_fwd.restype = ctypes.c_int
             L.oracle_ffn_fwd.argtypes = [_u16p, _u16p, _u16p, _u16p, _u16p, _i64, _i64, _i64, _vp, _i64,
-                                         _vp, _i32, _f64p]
+                                         _vp, _i32, _vp, _f64p]
             L.oracle_ffn_fwd_hybrid.restype = ctypes.c_int
             L.oracle_ffn_fwd_hybrid.argtypes = [_u16p, _u16p, _u16p, _u16p, _u16p, _u8p, _u8p, _i32p, _i64,
                                                 _u16p, _i64, _i64, _i64, _i32, _i32, _f64p]
             L.oracle_ffn_bwd.restype = ctypes.c_int
             L.oracle_ffn_bwd.argtypes = [_u16p, _u16p, _u16p, _u16p, _u16p, _u16p, ctypes.c_double, _i64,
-                                         _i64, _i64, _vp, _i32, _f64p, _f64p, _f64p, _f64p, _vp]
+                                         _i64, _i64, _vp, _i32, _vp, _f64p, _f64p, _f64p, _f64p, _vp]
             _lib = L
     return _lib
 
@@ -165,8 +166,11 @@ def unpack(p: dict, f: int, T_n: int, K: int) -> np.ndarray:
     return G
 
 
-def ffn_fwd(X, W_g, b_g, W_u, W_d, rows=None, mask=None, round_g: bool = False) -> np.ndarray:
-    """Y = (ReLU(X W_g^T + b_g) * (X W_u^T)) W_d^T in float64 (rows subset optional)."""
+def ffn_fwd(X, W_g, b_g, W_u, W_d, rows=None, mask=None, round_g: bool = False, gmat=None) -> np.ndarray:
+    """Y = (ReLU(X W_g^T + b_g) * (X W_u^T)) W_d^T in float64 (rows subset optional).
+
+    mask [nrows, f] replaces the z > 0 test; gmat [nrows, f] (bf16 bits) gives g
+    itself (active where nonzero); round_g uses bf16(z) for g."""
     X, W_g, b_g, W_u, W_d = (_c(a, np.uint16) for a in (X, W_g, b_g, W_u, W_d))
     M, d = X.shape
     f = W_g.shape[0]
@@ -175,8 +179,11 @@ def ffn_fwd(X, W_g, b_g, W_u, W_d, rows=None, mask=None, round_g: bool = False) 
     m = None if mask is None else _c(mask, np.uint8)
     if m is not None and m.shape != (n, f):
         raise ValueError("mask must be [nrows, d_ff]")
+    gm = None if gmat is None else _c(gmat, np.uint16)
+    if gm is not None and gm.shape != (n, f):
+        raise ValueError("gmat must be [nrows, d_ff]")
     Y = np.empty((n, d), np.float64)
-    if lib().oracle_ffn_fwd(X, W_g, b_g, W_u, W_d, M, d, f, _ptr(r), n, _ptr(m), int(round_g), Y):
+    if lib().oracle_ffn_fwd(X, W_g, b_g, W_u, W_d, M, d, f, _ptr(r), n, _ptr(m), int(round_g), _ptr(gm), Y):
         raise MemoryError("oracle_ffn_fwd")
     return Y
 
@@ -201,17 +208,22 @@ def ffn_fwd_hybrid(X, W_u, W_d, p: dict, T_n: int, K: int) -> np.ndarray:
     return Y
 
 
-def ffn_bwd(X, W_g, b_g, W_u, W_d, dY, lam: float = 0.0, mask=None, round_g: bool = False) -> dict:
-    """Gradients of sum(Y * dY) + lam * sum(ReLU(z)): dX, dW_g, dW_u, dW_d, db_g (float64)."""
+def ffn_bwd(X, W_g, b_g, W_u, W_d, dY, lam: float = 0.0, mask=None, round_g: bool = False, gmat=None) -> dict:
+    """Gradients of sum(Y * dY) + lam * sum(ReLU(z)): dX, dW_g, dW_u, dW_d, db_g (float64).
+
+    mask / gmat / round_g as in ffn_fwd ([M, f])."""
     X, W_g, b_g, W_u, W_d, dY = (_c(a, np.uint16) for a in (X, W_g, b_g, W_u, W_d, dY))
     M, d = X.shape
     f = W_g.shape[0]
     m = None if mask is None else _c(mask, np.uint8)
     if m is not None and m.shape != (M, f):
         raise ValueError("mask must be [M, d_ff]")
+    gm = None if gmat is None else _c(gmat, np.uint16)
+    if gm is not None and gm.shape != (M, f):
+        raise ValueError("gmat must be [M, d_ff]")
     out = dict(dX=np.empty((M, d)), dW_g=np.empty((f, d)), dW_u=np.empty((f, d)), dW_d=np.empty((d, f)),
                db_g=np.empty(f))
-    rc = lib().oracle_ffn_bwd(X, W_g, b_g, W_u, W_d, dY, float(lam), M, d, f, _ptr(m), int(round_g),
+    rc = lib().oracle_ffn_bwd(X, W_g, b_g, W_u, W_d, dY, float(lam), M, d, f, _ptr(m), int(round_g), _ptr(gm),
                               out["dX"], out["dW_g"], out["dW_u"], out["dW_d"], _ptr(out["db_g"]))
     if rc:
         raise MemoryError("oracle_ffn_bwd")

@@ -257,13 +257,17 @@ void oracle_unpack(const uint16_t* count, const uint16_t* val, const uint8_t* co
  *   u_ij = x_i . W_u[j];  h_ij = g_ij u_ij;  Y_ic = sum_j h_ij W_d[c, j]  (j ascending)
  * mask, when given, is [nrows x f] bytes and replaces the z > 0 test (used to
  * evaluate the definition on another implementation's active set).
+ * gmat, when given, is [nrows x f] bf16 bits of g itself: active_ij = (gmat != 0)
+ * and g_ij = gmat_ij (used to evaluate the definition on the g values another
+ * implementation stored, i.e. with its z > 0 and bf16 rounding decisions).
  * Returns 0, or 1 on allocation failure. */
 int oracle_ffn_fwd(const uint16_t* X, const uint16_t* Wg, const uint16_t* bg, const uint16_t* Wu,
                    const uint16_t* Wd, int64_t M, int64_t d, int64_t f, const int32_t* rows,
-                   int64_t nrows, const uint8_t* mask, int32_t round_g, double* Y) {
+                   int64_t nrows, const uint8_t* mask, int32_t round_g, const uint16_t* gmat, double* Y) {
   if (!rows) nrows = M;
-  double* WgT = mask ? NULL : to_double_transposed(Wg, f, d);
-  double* Wgd = mask ? to_double(Wg, f * d) : NULL;
+  const int given = (mask != NULL) || (gmat != NULL);
+  double* WgT = given ? NULL : to_double_transposed(Wg, f, d);
+  double* Wgd = given ? to_double(Wg, f * d) : NULL;
   double* Wud = to_double(Wu, f * d);
   double* WdT = to_double_transposed(Wd, d, f); /* WdT[j*d + c] = W_d[c, j] */
   double* b = to_double(bg, f);
@@ -281,19 +285,22 @@ int oracle_ffn_fwd(const uint16_t* X, const uint16_t* Wg, const uint16_t* bg, co
         for (int64_t r = 0; r < nrows; ++r) {
           const int64_t i = rows ? rows[r] : r;
           oracle_bf16_to_double_array(X + i * d, x, d);
-          if (!mask) gate_row(x, WgT, b, d, f, z);
+          if (!given) gate_row(x, WgT, b, d, f, z);
           double* y = Y + r * d;
           for (int64_t c = 0; c < d; ++c) y[c] = 0.0;
           for (int64_t j = 0; j < f; ++j) {
             double zj;
-            if (mask) {
+            if (gmat) {
+              if (gmat[r * f + j] == 0) continue;
+              zj = oracle_bf16_to_double(gmat[r * f + j]);
+            } else if (mask) {
               if (!mask[r * f + j]) continue;
               zj = dot(x, Wgd + j * d, d) + b[j];
             } else {
               zj = z[j];
               if (!(zj > 0.0)) continue;
             }
-            const double g = round_g ? oracle_bf16_to_double(oracle_bf16_round(zj)) : zj;
+            const double g = (round_g && !gmat) ? oracle_bf16_to_double(oracle_bf16_round(zj)) : zj;
             const double u = dot(x, Wud + j * d, d);
             const double h = g * u;
             const double* w = WdT + j * d;
@@ -380,12 +387,14 @@ int oracle_ffn_fwd_hybrid(const uint16_t* X, const uint16_t* Wu, const uint16_t*
  *   dW_d[c, j] = sum_i dY_ic h_ij;  dW_u[j, k] = sum_i dU_ij x_ik
  *   dW_g[j, k] = sum_i dZ_ij x_ik;  db_g[j] = sum_i dZ_ij   (i ascending)
  * mask [M x f] (nullable) replaces the z > 0 test as in oracle_ffn_fwd; round_g
- * uses bf16(z) for g. db_g may be NULL. Returns 0, or 1 on allocation failure. */
+ * uses bf16(z) for g; gmat [M x f] (nullable) gives g itself as in
+ * oracle_ffn_fwd. db_g may be NULL. Returns 0, or 1 on allocation failure. */
 int oracle_ffn_bwd(const uint16_t* X, const uint16_t* Wg, const uint16_t* bg, const uint16_t* Wu,
                    const uint16_t* Wd, const uint16_t* dY, double lambda, int64_t M, int64_t d,
-                   int64_t f, const uint8_t* mask, int32_t round_g, double* dX, double* dWg,
-                   double* dWu, double* dWd, double* dbg) {
-  double* WgT = mask ? NULL : to_double_transposed(Wg, f, d);
+                   int64_t f, const uint8_t* mask, int32_t round_g, const uint16_t* gmat, double* dX,
+                   double* dWg, double* dWu, double* dWd, double* dbg) {
+  const int given = (mask != NULL) || (gmat != NULL);
+  double* WgT = given ? NULL : to_double_transposed(Wg, f, d);
   double* Wgd = to_double(Wg, f * d);
   double* Wud = to_double(Wu, f * d);
   double* WdT = to_double_transposed(Wd, d, f);
@@ -394,7 +403,7 @@ int oracle_ffn_bwd(const uint16_t* X, const uint16_t* Wg, const uint16_t* bg, co
   int64_t* nact = (int64_t*)calloc((size_t)(M > 0 ? M : 1), sizeof(int64_t));
   int32_t** act_j = (int32_t**)calloc((size_t)(M > 0 ? M : 1), sizeof(int32_t*));
   double** act_v = (double**)calloc((size_t)(M > 0 ? M : 1), sizeof(double*));
-  int err = ((!mask && !WgT) || !Wgd || !Wud || !WdT || !b || !nact || !act_j || !act_v);
+  int err = ((!given && !WgT) || !Wgd || !Wud || !WdT || !b || !nact || !act_j || !act_v);
   if (!err) {
 #pragma omp parallel
     {
@@ -409,9 +418,10 @@ int oracle_ffn_bwd(const uint16_t* X, const uint16_t* Wg, const uint16_t* bg, co
         for (int64_t i = 0; i < M; ++i) {
           oracle_bf16_to_double_array(X + i * d, x, d);
           oracle_bf16_to_double_array(dY + i * d, dy, d);
-          if (!mask) gate_row(x, WgT, b, d, f, z);
+          if (!given) gate_row(x, WgT, b, d, f, z);
           int64_t n = 0;
-          for (int64_t j = 0; j < f; ++j) n += mask ? (mask[i * f + j] != 0) : (z[j] > 0.0);
+          for (int64_t j = 0; j < f; ++j)
+            n += gmat ? (gmat[i * f + j] != 0) : mask ? (mask[i * f + j] != 0) : (z[j] > 0.0);
           nact[i] = n;
           act_j[i] = (int32_t*)malloc((size_t)(n > 0 ? n : 1) * sizeof(int32_t));
           act_v[i] = (double*)malloc((size_t)(n > 0 ? 3 * n : 1) * sizeof(double));
@@ -425,14 +435,17 @@ int oracle_ffn_bwd(const uint16_t* X, const uint16_t* Wg, const uint16_t* bg, co
           int64_t a = 0;
           for (int64_t j = 0; j < f; ++j) {
             double zj;
-            if (mask) {
+            if (gmat) {
+              if (gmat[i * f + j] == 0) continue;
+              zj = oracle_bf16_to_double(gmat[i * f + j]);
+            } else if (mask) {
               if (!mask[i * f + j]) continue;
               zj = dot(x, Wgd + j * d, d) + b[j];
             } else {
               zj = z[j];
               if (!(zj > 0.0)) continue;
             }
-            const double g = round_g ? oracle_bf16_to_double(oracle_bf16_round(zj)) : zj;
+            const double g = (round_g && !gmat) ? oracle_bf16_to_double(oracle_bf16_round(zj)) : zj;
             const double u = dot(x, Wud + j * d, d);
             const double dh = dot(dy, WdT + j * d, d);
             const double du = dh * g;

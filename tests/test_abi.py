@@ -1,0 +1,103 @@
+"""The C ABI on a host without a GPU: the library loads, exports every entry point
+that include/twell.h declares, and its host-only checks answer as documented.
+None of these calls reaches the GPU (they return before any CUDA call)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "twell.h")
+
+
+@pytest.fixture(scope="module")
+def tw():
+    from activation_sparse_ffn_gemm_b200 import build
+
+    build.build()
+    import activation_sparse_ffn_gemm_b200 as tw
+
+    return tw
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(twell_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("twell_pack", "twell_ffn_fwd", "twell_ffn_bwd", "twell_workspace_bytes", "twell_status_read"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(tw):
+    L = tw.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), f"{name} is declared in twell.h but not exported"
+    # nothing else is exported with the twell_ prefix besides the declared API
+    out = os.popen(f"nm -D --defined-only {tw.LIB_PATH}").read()
+    exported = set(re.findall(r"\bT (twell_[a-z_0-9]+)\b", out))
+    assert exported == set(declared_functions())
+
+
+def test_hybrid_struct_matches_header(tw):
+    # five int32 fields, 4 bytes of padding, ten pointers
+    assert ctypes.sizeof(tw.TwellHybrid) == 24 + 10 * 8
+    assert tw.TwellHybrid.count.offset == 24
+
+
+def test_query_support(tw):
+    ok = tw.query_support
+    assert ok(4096, 2048, 8192, 128, 8, 4096) == 0
+    assert ok(0, 2048, 8192, 128, 8, 0) == 0
+    assert ok(16384, 4096, 14336, 128, 64, 100) == 0
+    assert ok(4096, 2048, 8192, 64, 8, 0) == 2      # T_n must be 128
+    assert ok(4096, 2048, 8192, 128, 12, 0) == 2    # K not in {8,16,32,64}
+    assert ok(4096, 2000, 8192, 128, 8, 0) == 2     # d_model % 64
+    assert ok(4096, 2048, 8000, 128, 8, 0) == 2     # d_ff % 128
+    assert ok(4096, 2048, 32768, 128, 8, 0) == 2    # d_ff too wide
+    assert ok(10, 2048, 8192, 128, 8, 11) == 2      # ovf_cap > M
+    assert ok(-1, 2048, 8192, 128, 8, 0) == 1
+    assert tw.lib().twell_status_string(6).decode().startswith("workspace")
+
+
+def test_workspace_sizes(tw):
+    M, d, f, K = 4096, 2048, 8192, 8
+    pack = tw.workspace_bytes(tw.OP_PACK, M, d, f, 128, K, M)
+    fwd = tw.workspace_bytes(tw.OP_FWD, M, d, f, 128, K, M)
+    bwd = tw.workspace_bytes(tw.OP_BWD, M, d, f, 128, K, M)
+    assert pack >= M * f * 2 and fwd > pack and bwd > f * d * 2
+    assert tw.workspace_bytes(tw.OP_FWD, M, d, f, 64, K, M) == 0
+    assert tw.workspace_bytes(7, M, d, f, 128, K, M) == 0
+
+
+def test_host_side_errors(tw):
+    L = tw.lib()
+    h = tw.TwellHybrid(64, 1024, 128, 8, 64, *([None] * 10))
+    # null descriptor, null arrays, unsupported shape, missing workspace
+    assert L.twell_pack(None, None, None, 256, None, None, None, 0, None) == 1
+    assert L.twell_pack(None, None, None, 256, ctypes.byref(h), None, None, 0, None) == 1
+    bad = tw.TwellHybrid(64, 1024, 64, 8, 64, *([None] * 10))
+    assert L.twell_pack(None, None, None, 256, ctypes.byref(bad), None, None, 0, None) == 2
+    fake = 1 << 20  # aligned non-null addresses; never dereferenced by these checks
+    h2 = tw.TwellHybrid(64, 1024, 128, 8, 64, *([fake] * 10))
+    p = ctypes.c_void_p(fake)
+    assert L.twell_pack(p, p, p, 256, ctypes.byref(h2), None, None, 0, None) == 6
+    assert L.twell_pack(p, p, p, 256, ctypes.byref(h2), None, ctypes.c_void_p(fake + 8), 1 << 30, None) == 6
+    mis = ctypes.c_void_p(fake + 2)
+    assert L.twell_ffn_fwd(mis, p, p, p, p, None, 256, p, ctypes.byref(h2), None, None, 0, None) == 1
+    # empty batch forward: nothing to do, nothing touched
+    h0 = tw.TwellHybrid(0, 1024, 128, 8, 0, *([None] * 10))
+    assert L.twell_ffn_fwd(None, None, None, None, None, None, 256, None, ctypes.byref(h0), None, None, 0, None) == 0
+    assert L.twell_transpose_wd(None, 256, 1024, None, None) == 1
+
+
+def test_missing_library_fails_loudly(tw, monkeypatch):
+    monkeypatch.setattr(tw, "_lib", None)
+    monkeypatch.setattr(tw, "LIB_PATH", os.path.join(ROOT, "does_not_exist", "libtwell.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        tw.lib()

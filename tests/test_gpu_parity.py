@@ -1,0 +1,232 @@
+"""GPU parity of the sm_100a path against the fp64 CPU oracle, through the C ABI.
+
+Small cases compare every output element; the full-size workloads compare the
+pack on every row and Y on a seeded sample of rows plus every overflow row, and
+the training workload's gradients on full tensors. Tolerances are stated in
+tests/twell_testlib.py.
+"""
+
+import json
+import os
+
+import numpy as np
+import pytest
+
+from synthetic import WORKLOADS, Workload, make_inputs
+from twell_testlib import (assert_active_set, assert_matches_oracle, assert_pack_equal, bits_of, f32_of_bits,
+                           gpu_gmat, state_to_numpy, to_dev)
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.fixture(scope="module")
+def tw():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import activation_sparse_ffn_gemm_b200 as tw
+
+    tw.lib()
+    return tw
+
+
+def _dev(inp):
+    return {k: to_dev(v) for k, v in inp.items() if k != "meta"}
+
+
+def _run_fwd(tw, inp, w, cap=None, save=True):
+    D = _dev(inp)
+    Y, st, z = tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], T_n=w.T_n, K=w.K, ovf_cap=cap,
+                          save_for_backward=save, z_debug=True)
+    torch.cuda.synchronize()
+    return D, Y, st, z
+
+
+def _check_fwd(orc, inp, w, Y, st, z, rows=None, cap=None):
+    """Pack bit-exact (all rows), active set and Y (all rows or the given sample)."""
+    M, f = inp["X"].shape[0], inp["W_g"].shape[0]
+    zg = z.cpu().numpy()
+    p_gpu = state_to_numpy(st)
+    p_ref = orc.pack(zg.astype(np.float64), w.T_n, w.K, cap=cap)
+    assert_pack_equal(p_gpu, p_ref)
+    expect = 8 if p_ref["n_ovf_total"] > p_ref["n_ovf"] else 0  # TWELL_STATUS_OVERFLOW_CAP
+    assert st.read_status() == expect
+    if rows is None:
+        rows = np.arange(M, dtype=np.int32)
+    z64 = orc.gate(inp["X"], inp["W_g"], inp["b_g"], rows=rows)
+    flips = assert_active_set(zg[rows], z64, float(np.sqrt(np.mean(z64 ** 2))))
+    args = (inp["X"], inp["W_g"], inp["b_g"], inp["W_u"], inp["W_d"])
+    G = gpu_gmat(p_gpu, M, f, w.T_n, w.K)
+    y_stored = orc.ffn_fwd(*args, rows=rows, gmat=G[rows])
+    y_plain = orc.ffn_fwd(*args, rows=rows)
+    yg = f32_of_bits(bits_of(Y))[rows]
+    stats = assert_matches_oracle(yg, y_stored, y_plain, "Y", bf16_out=True)
+    return p_gpu, flips, stats
+
+
+def _check_bwd(orc, inp, g, G, lam, name):
+    args = (inp["X"], inp["W_g"], inp["b_g"], inp["W_u"], inp["W_d"], inp["dY"], lam)
+    ref_s = orc.ffn_bwd(*args, gmat=G)
+    ref_p = orc.ffn_bwd(*args, mask=(G != 0).astype(np.uint8))
+    for k in ("dX", "dW_g", "dW_u", "dW_d", "db_g"):
+        assert_matches_oracle(g[k].cpu().numpy(), ref_s[k], ref_p[k], f"{name} {k} lambda={lam}")
+
+
+CASES = {
+    # name: (M, d, f, K, activity, row_scale, seed)
+    "tiny": (64, 256, 1024, 16, 0.03, "none", 0),
+    "ragged": (300, 192, 384, 8, 0.05, "lognormal", 1),
+    "ragged_k16": (389, 320, 640, 16, 0.06, "lognormal", 2),
+    "k32": (257, 512, 1024, 32, 0.1, "lognormal", 3),
+    "k64": (130, 256, 2048, 64, 0.2, "lognormal", 4),
+    "one_row": (1, 128, 256, 8, 0.3, "none", 5),
+    "multi_tile": (700, 1024, 2048, 8, 0.01, "lognormal", 6),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_fwd_bwd_small(tw, orc, name):
+    M, d, f, K, act, rs, seed = CASES[name]
+    w = Workload(name, M, d, f, 128, K, act, row_scale=rs, training=True, seed=seed)
+    inp = make_inputs(w)
+    D, Y, st, z = _run_fwd(tw, inp, w)
+    p, flips, _ = _check_fwd(orc, inp, w, Y, st, z)
+    for lam in (0.0, 1e-3):
+        g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=lam)
+        torch.cuda.synchronize()
+        _check_bwd(orc, inp, g, gpu_gmat(p, M, f, 128, K), lam, name)
+
+
+def test_degenerate_all_inactive(tw, orc):
+    w = Workload("off", 200, 256, 512, 128, 8, 0.01, training=True)
+    inp = make_inputs(w)
+    inp["b_g"][:] = 0xC6C0  # bf16 -24576: no unit can be active
+    D, Y, st, z = _run_fwd(tw, inp, w)
+    assert not st.count.any().item() and st.n_overflow() == (0, 0)
+    assert not Y.float().abs().sum().item()
+    g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=0.5)
+    for k, v in g.items():
+        assert not v.abs().sum().item(), k
+
+
+def test_degenerate_all_active_dense_path(tw, orc):
+    """b >> 0: every unit active, every row overflows K < T_n, everything runs dense."""
+    w = Workload("on", 150, 256, 384, 128, 8, 0.01, training=True, seed=9)
+    inp = make_inputs(w)
+    inp["b_g"][:] = 0x4120  # bf16 10.0
+    D, Y, st, z = _run_fwd(tw, inp, w)
+    p, _, _ = _check_fwd(orc, inp, w, Y, st, z)
+    assert p["n_ovf"] == 150 and p["row_ovf"].all()
+    g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=1e-3)
+    _check_bwd(orc, inp, g, gpu_gmat(p, 150, 384, 128, 8), 1e-3, "all-active")
+
+
+def test_overflow_capacity_exceeded(tw, orc):
+    w = Workload("cap", 256, 256, 512, 128, 8, 0.15, row_scale="lognormal", seed=3)
+    inp = make_inputs(w)
+    Z = orc.gate(inp["X"], inp["W_g"], inp["b_g"])
+    n_flag = orc.pack(Z, 128, 8)["n_ovf_total"]
+    assert n_flag >= 4
+    cap = n_flag // 2
+    D = _dev(inp)
+    st, z = tw.pack(D["X"], D["W_g"], D["b_g"], T_n=128, K=8, ovf_cap=cap, z_debug=True)
+    torch.cuda.synchronize()
+    p_ref = orc.pack(z.cpu().numpy().astype(np.float64), 128, 8, cap=cap)
+    assert_pack_equal(state_to_numpy(st), p_ref)
+    assert st.n_overflow() == (cap, p_ref["n_ovf_total"])
+    assert st.read_status(clear=True) == tw.STATUS_OVERFLOW_CAP
+    assert st.read_status() == 0
+
+
+def test_empty_batch(tw):
+    d, f = 256, 512
+    X = torch.empty((0, d), dtype=torch.bfloat16, device="cuda")
+    W = torch.randn((f, d), device="cuda").bfloat16()
+    Wd = torch.randn((d, f), device="cuda").bfloat16()
+    b = torch.zeros(f, device="cuda").bfloat16()
+    Y, st = tw.ffn_fwd(X, W, b, W, Wd, K=8)
+    g = tw.ffn_bwd(X, W, W, Wd, st, X, lam=0.1)
+    torch.cuda.synchronize()
+    assert Y.shape == (0, d)
+    for k in ("dW_g", "dW_u", "dW_d", "db_g"):
+        assert not g[k].abs().sum().item()
+
+
+def test_deterministic(tw):
+    w = Workload("det", 300, 512, 1024, 128, 8, 0.05, row_scale="lognormal", training=True, seed=11)
+    D = _dev(make_inputs(w))
+    outs = []
+    for _ in range(2):
+        Y, st = tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], K=8)
+        g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=1e-3)
+        torch.cuda.synchronize()
+        outs.append([Y.clone()] + [g[k].clone() for k in sorted(g)])
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
+def test_prepared_wdt_matches(tw):
+    w = Workload("wdt", 256, 512, 1024, 128, 8, 0.03, training=True, seed=12)
+    D = _dev(make_inputs(w))
+    Wdt = tw.transpose_wd(D["W_d"])
+    assert torch.equal(Wdt, D["W_d"].t().contiguous())
+    Y1, st1 = tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], K=8)
+    Y2, st2 = tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], K=8, W_dt=Wdt)
+    g1 = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st1, D["dY"], lam=0.0)
+    g2 = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st2, D["dY"], lam=0.0, W_dt=Wdt)
+    torch.cuda.synchronize()
+    assert torch.equal(Y1, Y2)
+    for k in g1:
+        assert torch.equal(g1[k], g2[k]), k
+
+
+# ------------------------------------------------------------ full-size workloads
+
+
+def _sample_rows(M, n, seed, extra=()):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(M, size=min(n, M), replace=False).tolist()) | set(int(r) for r in extra)
+    return np.array(sorted(rows), dtype=np.int32)
+
+
+def test_uniform_full_size(tw, orc):
+    """Inference forward, uniform 1% activity, M=4096 d=2048 d_ff=8192 K=8 (no overflow rows)."""
+    w = WORKLOADS["uniform"]
+    with open(os.path.join(GOLDEN, "uniform_seed.json")) as fh:
+        seed = json.load(fh)["seed"]
+    inp = make_inputs(w, seed=seed)
+    D, Y, st, z = _run_fwd(tw, inp, w, save=False)
+    rows = _sample_rows(w.M, 256, 0)
+    p, flips, stats = _check_fwd(orc, inp, w, Y, st, z, rows=rows)
+    assert p["n_ovf_total"] == 0
+
+
+def test_heavy_tail_full_size(tw, orc):
+    """Inference forward, lognormal row scale, M=16384 d=4096 d_ff=14336 K=8: exercises the dense backup."""
+    w = WORKLOADS["heavy"]
+    inp = make_inputs(w)
+    D, Y, st, z = _run_fwd(tw, inp, w, save=False)
+    p = state_to_numpy(st)
+    assert p["n_ovf"] > 0
+    cnt = p["count"].astype(np.float64)
+    assert cnt.max() / cnt.mean() >= 10
+    rng = np.random.default_rng(1)
+    ovf_sample = rng.choice(p["ovf_rows"], size=min(64, p["n_ovf"]), replace=False)
+    rows = _sample_rows(w.M, 128, 1, extra=ovf_sample)
+    _check_fwd(orc, inp, w, Y, st, z, rows=rows)
+
+
+def test_train_full_size(tw, orc):
+    """Training step, M=8192 d=2048 d_ff=8192 K=8, lambda in {0, 1e-3}; gradients on full tensors."""
+    w = WORKLOADS["train"]
+    inp = make_inputs(w)
+    D, Y, st, z = _run_fwd(tw, inp, w)
+    rows = _sample_rows(w.M, 256, 2)
+    p, _, _ = _check_fwd(orc, inp, w, Y, st, z, rows=rows)
+    G = gpu_gmat(p, w.M, w.d_ff, w.T_n, w.K)
+    for lam in (0.0, 1e-3):
+        g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=lam)
+        torch.cuda.synchronize()
+        _check_bwd(orc, inp, g, G, lam, "train")

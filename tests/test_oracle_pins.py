@@ -336,3 +336,28 @@ def test_bwd_special_and_mask(orc):
     b = orc.ffn_bwd(X, Wg, bg, Wu, Wd, dY, 0.01, mask=mask)
     for k in a:
         assert np.array_equal(a[k], b[k]), k
+
+
+def test_gmat_input_equals_stored_g_definition(orc):
+    """g given explicitly (the packed, bf16-rounded ReLU(z)) reproduces round_g exactly,
+    and a perturbed g moves the result the way the definition says."""
+    rng = np.random.default_rng(21)
+    X, Wg, bg, Wu, Wd, dY = _problem(21, 16, 64, 256, -0.6)
+    Z = orc.gate(X, Wg, bg)
+    G = orc.unpack(orc.pack(Z, 128, 8), 256, 128, 8)
+    assert np.array_equal(orc.ffn_fwd(X, Wg, bg, Wu, Wd, gmat=G), orc.ffn_fwd(X, Wg, bg, Wu, Wd, round_g=True))
+    a = orc.ffn_bwd(X, Wg, bg, Wu, Wd, dY, 0.01, gmat=G)
+    b = orc.ffn_bwd(X, Wg, bg, Wu, Wd, dY, 0.01, round_g=True)
+    for k in a:
+        assert np.array_equal(a[k], b[k]), k
+    # doubling one stored g doubles that unit's contribution to Y (torch, float64)
+    i, j = [int(v) for v in np.argwhere(G != 0)[0]]
+    G2 = G.copy()
+    G2[i, j] = bf16_bits_from_f64(2 * _f64(G[i:i + 1, j:j + 1]))[0, 0]
+    x, wu, wd = _f64(X), _f64(Wu), _f64(Wd)
+    delta = _f64(G[i:i + 1, j:j + 1])[0, 0] * (x[i] @ wu[j]) * wd[:, j]
+    y1 = orc.ffn_fwd(X, Wg, bg, Wu, Wd, gmat=G)
+    y2 = orc.ffn_fwd(X, Wg, bg, Wu, Wd, gmat=G2)
+    assert np.abs(y2[i] - y1[i] - delta).max() < 1e-12
+    rows = np.array([3, 0], np.int32)
+    assert np.array_equal(orc.ffn_fwd(X, Wg, bg, Wu, Wd, rows=rows, gmat=G[rows]), y1[rows])
