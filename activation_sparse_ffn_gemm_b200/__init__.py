@@ -37,6 +37,10 @@ class TwellError(RuntimeError):
         super().__init__(f"{what}: {_STATUS_NAMES.get(code, code)} ({lib().twell_status_string(code).decode()})")
 
 
+class TwellTraceRec(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("ms", ctypes.c_float)]
+
+
 class TwellHybrid(ctypes.Structure):
     """Mirror of struct twell_hybrid."""
 
@@ -75,6 +79,12 @@ def lib():
             L.twell_ffn_bwd.restype = ctypes.c_int
             L.twell_ffn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, ctypes.POINTER(TwellHybrid), _vp,
                                         ctypes.c_float, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+            L.twell_launch_count.restype = ctypes.c_uint64
+            L.twell_launch_count.argtypes = []
+            L.twell_trace_enable.restype = None
+            L.twell_trace_enable.argtypes = [ctypes.c_int]
+            L.twell_trace_collect.restype = ctypes.c_int
+            L.twell_trace_collect.argtypes = [ctypes.POINTER(TwellTraceRec), ctypes.c_int]
             L.twell_status_read.restype = ctypes.c_int
             L.twell_status_read.argtypes = [ctypes.POINTER(TwellHybrid), ctypes.POINTER(ctypes.c_uint32),
                                             ctypes.c_int, _vp]
@@ -100,6 +110,22 @@ def _bf16(t: torch.Tensor, name: str) -> torch.Tensor:
     if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
         raise TypeError(f"{name} must be a contiguous CUDA bfloat16 tensor")
     return t
+
+
+def launch_count() -> int:
+    """Kernels this library has launched in the process so far."""
+    return int(lib().twell_launch_count())
+
+
+def trace_enable(on: bool = True) -> None:
+    lib().twell_trace_enable(1 if on else 0)
+
+
+def trace_collect(max_recs: int = 1 << 16) -> list:
+    """[(kernel name, ms), ...] for the launches recorded since the last collect."""
+    buf = (TwellTraceRec * max_recs)()
+    n = lib().twell_trace_collect(buf, max_recs)
+    return [(buf[i].name.decode(), float(buf[i].ms)) for i in range(min(n, max_recs))]
 
 
 def query_support(M, d_model, d_ff, T_n, K, ovf_cap) -> int:

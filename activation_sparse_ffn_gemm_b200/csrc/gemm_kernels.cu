@@ -328,7 +328,7 @@ cudaError_t launch_gate_pack(const uint16_t* X, const uint16_t* W_g, const uint1
     return cudaErrorInvalidValue;
   GemmShape shp{M, nullptr, f, d, 0, status};
   EpiTwell::Args ea{b_g, out.count, out.val, out.col, out.spill, out.z_debug, f / kTn, K, f};
-  return launch_umma_gemm<EpiTwell, 256, false, kStages>(ta, tb, ta, tb, shp, ea, s);
+  return launch_umma_gemm<EpiTwell, 256, false, kStages>("gate_pack_gemm", ta, tb, ta, tb, shp, ea, s);
 }
 
 cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uint16_t* W_d,
@@ -343,11 +343,11 @@ cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uin
     return cudaErrorInvalidValue;
   GemmShape s1{cap, n_ovf, f, d, 0, status};
   EpiGateMul::Args e1{g_ovf, h_ovf, u_ovf, f};
-  cudaError_t e = launch_umma_gemm<EpiGateMul, 256, false, kStages>(ta, tb, ta, tb, s1, e1, s);
+  cudaError_t e = launch_umma_gemm<EpiGateMul, 256, false, kStages>("ovf_up_gemm", ta, tb, ta, tb, s1, e1, s);
   if (e != cudaSuccess) return e;
   GemmShape s2{cap, n_ovf, d, f, 0, status};
   EpiScatterBf16::Args e2{ovf_rows, Y, d};
-  return launch_umma_gemm<EpiScatterBf16, 256, false, kStages>(ta2, tb2, ta2, tb2, s2, e2, s);
+  return launch_umma_gemm<EpiScatterBf16, 256, false, kStages>("ovf_down_gemm", ta2, tb2, ta2, tb2, s2, e2, s);
 }
 
 cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const uint16_t* W_u,
@@ -367,11 +367,11 @@ cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const u
     return cudaErrorInvalidValue;
   GemmShape s1{cap, n_ovf, f, d, 0, status};
   EpiBwdDH::Args e1{g_ovf, u_ovf, duz_ovf, du_ovf, dz_ovf, lambda, f};
-  cudaError_t e = launch_umma_gemm<EpiBwdDH, 256, false, kStages>(ta, tb, ta, tb, s1, e1, s);
+  cudaError_t e = launch_umma_gemm<EpiBwdDH, 256, false, kStages>("ovf_dh_gemm", ta, tb, ta, tb, s1, e1, s);
   if (e != cudaSuccess) return e;
   GemmShape s2{cap, n_ovf, d, f, f, status};
   EpiScatterF32::Args e2{ovf_rows, dX, d};
-  return launch_umma_gemm<EpiScatterF32, 256, true, kStages>(tdu, twu, tdz, twg, s2, e2, s);
+  return launch_umma_gemm<EpiScatterF32, 256, true, kStages>("ovf_dx_gemm", tdu, twu, tdz, twg, s2, e2, s);
 }
 
 }  // namespace twell

@@ -1,0 +1,331 @@
+// pairlist_kernels.cu — weight gradients over the hybrid format.
+//
+// dW_u = dU^T X, dW_g = dZ^T X, dW_d = dY^T H and db_g = column sums of dZ are
+// sums over the active (row, unit) pairs, taken unit by unit. A unit-major
+// (CSC) list of every active pair of the hybrid format — the ELL slots of
+// non-overflow rows and the nonzeros of the dense backup rows — is built in
+// ascending row order per unit (per-chunk counts, a scan over chunks, a scan
+// over units and an ordered fill), with h, dU and dZ attached; then for each
+// unit j
+//   dW_u[j] = sum_i dU_ij x_i,  dW_g[j] = sum_i dZ_ij x_i,
+//   dW_d[:, j] = sum_i h_ij dY_i,  db_g[j] = sum_i dZ_ij
+// in that fixed order, so the result is the same on every run.
+#include "trace.cuh"
+#include "twell_internal.cuh"
+
+namespace twell {
+
+namespace {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+// ------------------------------------------------------------------- CSC
+
+__global__ void row_slot_kernel(const int* __restrict__ ovf_rows, const int* __restrict__ n_ovf,
+                                int* __restrict__ row_slot) {
+  const int n = n_ovf[0];
+  for (int s = blockIdx.x * blockDim.x + threadIdx.x; s < n; s += gridDim.x * blockDim.x) row_slot[ovf_rows[s]] = s;
+}
+
+// The CSC is built per (unit tile t, chunk of kCscRows rows) with a counting
+// sort that keeps rows ascending inside each unit's list. Rows are taken in
+// groups of 32 (one per lane); each group records, per in-tile unit c, the
+// bitmask of its lanes (rows) activating c. A row's rank among the earlier rows
+// of its group with the same unit is then a popcount of that mask below its
+// lane, and group and chunk offsets come from prefix sums of the popcounts.
+
+// In-tile columns active for row r in tile t: the ELL slots of a non-overflow
+// row, or the nonzeros of its dense backup row; calls fn(c, ell_slot_or_-1).
+template <typename Fn>
+__device__ __forceinline__ void for_row_entries(long r, int t, int T, int K, int f, const uint16_t* __restrict__ count,
+                                                const uint8_t* __restrict__ col, const uint8_t* __restrict__ row_ovf,
+                                                const int* __restrict__ row_slot, const uint16_t* __restrict__ g_ovf,
+                                                Fn&& fn) {
+  if (!row_ovf[r]) {
+    const int c0 = count[r * T + t];
+    const int n = c0 < K ? c0 : K;
+    const long base = (r * T + t) * K;
+    for (int s = 0; s < n; ++s) fn(static_cast<int>(col[base + s]), base + s);
+  } else {
+    const int sl = row_slot[r];
+    if (sl < 0) return;
+    const uint4* gp = reinterpret_cast<const uint4*>(g_ovf + static_cast<long>(sl) * f + t * kTn);
+    for (int q = 0; q < kTn / 8; ++q) {
+      const uint4 v = gp[q];
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t bits = (w4[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+        if (bits) fn(q * 8 + e, -1L);
+      }
+    }
+  }
+}
+
+constexpr int kCscGroups = kCscRows / 32;
+
+__global__ void __launch_bounds__(256) csc_count_kernel(const uint16_t* __restrict__ count,
+                                                        const uint8_t* __restrict__ col,
+                                                        const uint8_t* __restrict__ row_ovf,
+                                                        const int* __restrict__ row_slot,
+                                                        const uint16_t* __restrict__ g_ovf, int M, int f, int K,
+                                                        int* __restrict__ chunk_cnt) {
+  __shared__ uint32_t mask[8][kTn];
+  __shared__ int cnt_s[kTn];
+  const int t = blockIdx.x, chunk = blockIdx.y, T = f / kTn;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x < kTn) cnt_s[threadIdx.x] = 0;
+  __syncthreads();
+  for (int g = w; g < kCscGroups; g += 8) {
+    const long r = static_cast<long>(chunk) * kCscRows + g * 32 + lane;
+#pragma unroll
+    for (int q = 0; q < kTn / 32; ++q) mask[w][lane + 32 * q] = 0u;
+    __syncwarp();
+    if (r < M)
+      for_row_entries(r, t, T, K, f, count, col, row_ovf, row_slot, g_ovf,
+                      [&](int c, long) { atomicOr(&mask[w][c], 1u << lane); });
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < kTn / 32; ++q) {
+      const int v = __popc(mask[w][lane + 32 * q]);
+      if (v) atomicAdd(&cnt_s[lane + 32 * q], v);
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+  if (threadIdx.x < kTn) chunk_cnt[static_cast<long>(chunk) * f + t * kTn + threadIdx.x] = cnt_s[threadIdx.x];
+}
+
+// Per unit: exclusive scan over the row blocks (in place) and the unit total.
+__global__ void csc_colscan_kernel(int* __restrict__ block_cnt, int nrb, int f, int* __restrict__ unit_tot) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= f) return;
+  int run = 0;
+  for (int rb = 0; rb < nrb; ++rb) {
+    const long o = static_cast<long>(rb) * f + j;
+    const int c = block_cnt[o];
+    block_cnt[o] = run;
+    run += c;
+  }
+  unit_tot[j] = run;
+}
+
+// Single block: unit_ptr = exclusive scan of unit_tot, unit_ptr[f] = total.
+__global__ void __launch_bounds__(1024) csc_unit_scan_kernel(const int* __restrict__ unit_tot, int f,
+                                                             int* __restrict__ unit_ptr) {
+  __shared__ int wsum[32];
+  __shared__ int carry;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < f; base += 1024) {
+    const int j = base + tid;
+    const int v = j < f ? unit_tot[j] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (lane == 31) wsum[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+      const int t = wsum[lane];
+      int ti = t;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int q = __shfl_up_sync(0xFFFFFFFFu, ti, o);
+        if (lane >= o) ti += q;
+      }
+      wsum[lane] = ti - t;
+    }
+    __syncthreads();
+    const int excl = carry + wsum[w] + incl - v;
+    if (j < f) unit_ptr[j] = excl;
+    __syncthreads();
+    if (tid == 1023) carry = excl + v;
+    __syncthreads();
+  }
+  if (tid == 0) unit_ptr[f] = carry;
+}
+
+__global__ void __launch_bounds__(256) csc_fill_kernel(
+    const uint16_t* __restrict__ count, const uint16_t* __restrict__ val, const uint8_t* __restrict__ col,
+    const uint8_t* __restrict__ row_ovf, const int* __restrict__ row_slot, const uint16_t* __restrict__ g_ovf,
+    const float* __restrict__ u_ell, const float* __restrict__ u_ovf, const float* __restrict__ du_ell,
+    const float* __restrict__ dz_ell, const float* __restrict__ du_ovf, const float* __restrict__ dz_ovf,
+    const int* __restrict__ chunk_base, const int* __restrict__ unit_ptr, int M, int f, int K,
+    int* __restrict__ csc_row, float4* __restrict__ csc_val) {
+  __shared__ uint32_t mask[kCscGroups][kTn];
+  __shared__ int gbase[kCscGroups][kTn];
+  const int t = blockIdx.x, chunk = blockIdx.y, T = f / kTn;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int g = w; g < kCscGroups; g += 8) {
+    const long r = static_cast<long>(chunk) * kCscRows + g * 32 + lane;
+#pragma unroll
+    for (int q = 0; q < kTn / 32; ++q) mask[g][lane + 32 * q] = 0u;
+    __syncwarp();
+    if (r < M)
+      for_row_entries(r, t, T, K, f, count, col, row_ovf, row_slot, g_ovf,
+                      [&](int c, long) { atomicOr(&mask[g][c], 1u << lane); });
+  }
+  __syncthreads();
+  if (threadIdx.x < kTn) {
+    const int j = t * kTn + threadIdx.x;
+    int run = unit_ptr[j] + chunk_base[static_cast<long>(chunk) * f + j];
+    for (int g = 0; g < kCscGroups; ++g) {
+      gbase[g][threadIdx.x] = run;
+      run += __popc(mask[g][threadIdx.x]);
+    }
+  }
+  __syncthreads();
+  const uint32_t below = (1u << lane) - 1u;
+  for (int g = w; g < kCscGroups; g += 8) {
+    const long r = static_cast<long>(chunk) * kCscRows + g * 32 + lane;
+    if (r >= M) continue;
+    const int sl = row_ovf[r] ? row_slot[r] : -1;
+    for_row_entries(r, t, T, K, f, count, col, row_ovf, row_slot, g_ovf, [&](int c, long slot) {
+      const int p = gbase[g][c] + __popc(mask[g][c] & below);
+      float4 v;
+      if (slot >= 0) {
+        const float gv = __uint_as_float(static_cast<uint32_t>(val[slot]) << 16);
+        v = make_float4(gv * u_ell[slot], du_ell[slot], dz_ell[slot], 0.f);
+      } else {
+        const long o = static_cast<long>(sl) * f + t * kTn + c;
+        const float gv = __uint_as_float(static_cast<uint32_t>(g_ovf[o]) << 16);
+        v = make_float4(gv * u_ovf[o], du_ovf[o], dz_ovf[o], 0.f);
+      }
+      csc_row[p] = static_cast<int>(r);
+      csc_val[p] = v;
+    });
+  }
+}
+
+// One warp per unit, 8 consecutive units per CTA, one 16-byte chunk (8
+// columns) per lane: a CTA covers a 256-column slice. The unit's list is read
+// 32 entries at a time, one entry per lane in a single coalesced load, and the
+// entries are handed out with shuffles, so the row loads of kWgBatch pairs can
+// be issued back to back without waiting on their indices. dW_d[:, j] is
+// transposed through shared memory so that each output row gets 8 consecutive
+// units (32 bytes).
+constexpr int kWgBatch = 4;
+constexpr int kWgCols = 256;
+
+__global__ void __launch_bounds__(256, 3) wgrad_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ dY,
+                                                    const int* __restrict__ unit_ptr, const int* __restrict__ csc_row,
+                                                    const float4* __restrict__ csc_val, int d, int f,
+                                                    float* __restrict__ dWg, float* __restrict__ dWu,
+                                                    float* __restrict__ dWd, float* __restrict__ dbg) {
+  __shared__ float s_dwd[kWgCols][9];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.x * 8 + w;
+  const int c0 = blockIdx.y * kWgCols;
+  const int cidx = (c0 >> 3) + lane;
+  const bool cval = cidx < (d >> 3);
+  float au[8], ag[8], ad[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) au[e] = ag[e] = ad[e] = 0.f;
+  float db = 0.f;
+  const int p0 = unit_ptr[j], p1 = unit_ptr[j + 1];
+  for (int pb = p0; pb < p1; pb += 32) {
+    const int n = min(32, p1 - pb);
+    const int my_row = lane < n ? csc_row[pb + lane] : 0;
+    const float4 my_v = lane < n ? csc_val[pb + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+    db += my_v.z;
+    for (int b0 = 0; b0 < n; b0 += kWgBatch) {
+      uint4 xv[kWgBatch], dv[kWgBatch];
+      float ch[kWgBatch], cu[kWgBatch], cz[kWgBatch];
+#pragma unroll
+      for (int b = 0; b < kWgBatch; ++b) {
+        const int src = b0 + b < n ? b0 + b : b0;
+        const long r = __shfl_sync(0xFFFFFFFFu, my_row, src);
+        const float h = __shfl_sync(0xFFFFFFFFu, my_v.x, src);
+        const float du = __shfl_sync(0xFFFFFFFFu, my_v.y, src);
+        const float dz = __shfl_sync(0xFFFFFFFFu, my_v.z, src);
+        const bool in = b0 + b < n;
+        ch[b] = in ? h : 0.f;
+        cu[b] = in ? du : 0.f;
+        cz[b] = in ? dz : 0.f;
+        if (cval) {
+          xv[b] = __ldg(reinterpret_cast<const uint4*>(X + r * d) + cidx);
+          dv[b] = __ldg(reinterpret_cast<const uint4*>(dY + r * d) + cidx);
+        } else {
+          xv[b] = dv[b] = make_uint4(0, 0, 0, 0);
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < kWgBatch; ++b) {
+        float xf[8], df[8];
+        unpack8(xv[b], xf);
+        unpack8(dv[b], df);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          au[e] = fmaf(cu[b], xf[e], au[e]);
+          ag[e] = fmaf(cz[b], xf[e], ag[e]);
+          ad[e] = fmaf(ch[b], df[e], ad[e]);
+        }
+      }
+    }
+  }
+  db = warp_sum(db);
+  if (cval) {
+    float4* pu = reinterpret_cast<float4*>(dWu + static_cast<long>(j) * d) + 2 * cidx;
+    float4* pg = reinterpret_cast<float4*>(dWg + static_cast<long>(j) * d) + 2 * cidx;
+    pu[0] = make_float4(au[0], au[1], au[2], au[3]);
+    pu[1] = make_float4(au[4], au[5], au[6], au[7]);
+    pg[0] = make_float4(ag[0], ag[1], ag[2], ag[3]);
+    pg[1] = make_float4(ag[4], ag[5], ag[6], ag[7]);
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) s_dwd[lane * 8 + e][w] = ad[e];
+  if (blockIdx.y == 0 && lane == 0 && dbg != nullptr) dbg[j] = db;
+  __syncthreads();
+  const int cc = c0 + threadIdx.x;
+  if (cc < d) {
+    float4* pd = reinterpret_cast<float4*>(dWd + static_cast<long>(cc) * f + blockIdx.x * 8);
+    pd[0] = make_float4(s_dwd[threadIdx.x][0], s_dwd[threadIdx.x][1], s_dwd[threadIdx.x][2], s_dwd[threadIdx.x][3]);
+    pd[1] = make_float4(s_dwd[threadIdx.x][4], s_dwd[threadIdx.x][5], s_dwd[threadIdx.x][6], s_dwd[threadIdx.x][7]);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_build_csc(const uint16_t* count, const uint16_t* val, const uint8_t* col,
+                             const uint8_t* row_ovf, const int* ovf_rows, const int* n_ovf, const uint16_t* g_ovf,
+                             const float* u_ell, const float* u_ovf, const float* du_ell, const float* dz_ell,
+                             const float* du_ovf, const float* dz_ovf, int M, int f, int K, int cap,
+                             const CscBuffers& b, cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  cudaError_t e = cudaMemsetAsync(b.row_slot, 0xFF, static_cast<size_t>(M) * sizeof(int), s);
+  if (e != cudaSuccess) return e;
+  if (cap > 0) {
+    const int g = (cap + 255) / 256 < 1024 ? (cap + 255) / 256 : 1024;
+    TWELL_LAUNCH("row_slot", s, row_slot_kernel<<<g, 256, 0, s>>>(ovf_rows, n_ovf, b.row_slot));
+  }
+  const int nch = (M + kCscRows - 1) / kCscRows;
+  const int T = f / kTn;
+  TWELL_LAUNCH("csc_count", s,
+               csc_count_kernel<<<dim3(T, nch), 256, 0, s>>>(count, col, row_ovf, b.row_slot, g_ovf, M, f, K,
+                                                            b.block_cnt));
+  TWELL_LAUNCH("csc_colscan", s, csc_colscan_kernel<<<(f + 255) / 256, 256, 0, s>>>(b.block_cnt, nch, f, b.unit_tot));
+  TWELL_LAUNCH("csc_unit_scan", s, csc_unit_scan_kernel<<<1, 1024, 0, s>>>(b.unit_tot, f, b.unit_ptr));
+  TWELL_LAUNCH("csc_fill", s,
+               csc_fill_kernel<<<dim3(T, nch), 256, 0, s>>>(count, val, col, row_ovf, b.row_slot, g_ovf, u_ell, u_ovf,
+                                                           du_ell, dz_ell, du_ovf, dz_ovf, b.block_cnt, b.unit_ptr, M,
+                                                           f, K, b.csc_row, b.csc_val));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_weight_grads(const uint16_t* X, const uint16_t* dY, const CscBuffers& b, int d, int f,
+                                float* dW_g, float* dW_u, float* dW_d, float* db_g, cudaStream_t s) {
+  dim3 grid(f / 8, (d + kWgCols - 1) / kWgCols);
+  TWELL_LAUNCH("weight_grads", s,
+               wgrad_kernel<<<grid, 256, 0, s>>>(X, dY, b.unit_ptr, b.csc_row, b.csc_val, d, f, dW_g, dW_u, dW_d, db_g));
+  return cudaGetLastError();
+}
+
+}  // namespace twell

@@ -8,6 +8,7 @@
 // K actives. Overflow rows are listed in ascending row order (a deterministic
 // scan), and each listed row is rebuilt densely from its ELL tiles plus the
 // dense slices that the gate epilogue spilled for its overflowing tiles.
+#include "trace.cuh"
 #include "twell_internal.cuh"
 
 namespace twell {
@@ -187,11 +188,12 @@ cudaError_t launch_route(const uint16_t* count, const uint16_t* val, const uint8
   int blocks = (warps_needed + 7) / 8;
   const int max_blocks = device_sm_count() * 16;
   if (blocks > max_blocks) blocks = max_blocks;
-  row_flags_kernel<<<blocks, 256, 0, s>>>(count, M, T, K, row_ovf);
-  ovf_scan_kernel<<<1, kScanThreads, 0, s>>>(row_ovf, M, cap, ovf_rows, n_ovf, status);
+  TWELL_LAUNCH("row_flags", s, row_flags_kernel<<<blocks, 256, 0, s>>>(count, M, T, K, row_ovf));
+  TWELL_LAUNCH("ovf_scan", s, ovf_scan_kernel<<<1, kScanThreads, 0, s>>>(row_ovf, M, cap, ovf_rows, n_ovf, status));
   if (cap > 0) {
     int g = cap < device_sm_count() * 4 ? cap : device_sm_count() * 4;
-    ovf_gather_kernel<<<g, 256, 0, s>>>(n_ovf, ovf_rows, count, val, col, spill, f, K, g_ovf, X, d, x_ovf);
+    TWELL_LAUNCH("ovf_gather", s,
+                 ovf_gather_kernel<<<g, 256, 0, s>>>(n_ovf, ovf_rows, count, val, col, spill, f, K, g_ovf, X, d, x_ovf));
   }
   return cudaGetLastError();
 }
@@ -200,14 +202,14 @@ cudaError_t launch_gather_rows(const uint16_t* in, const int* rows, const int* n
                                uint16_t* out, cudaStream_t s) {
   if (cap <= 0) return cudaSuccess;
   int g = cap < device_sm_count() * 4 ? cap : device_sm_count() * 4;
-  gather_rows_kernel<<<g, 256, 0, s>>>(in, rows, n_ovf, d, out);
+  TWELL_LAUNCH("gather_rows", s, gather_rows_kernel<<<g, 256, 0, s>>>(in, rows, n_ovf, d, out));
   return cudaGetLastError();
 }
 
 cudaError_t launch_transpose_bf16(const uint16_t* in, int rows, int cols, uint16_t* out, cudaStream_t s) {
   if (rows <= 0 || cols <= 0) return cudaSuccess;
   dim3 grid((cols + 63) / 64, (rows + 63) / 64);
-  transpose_bf16_kernel<<<grid, 256, 0, s>>>(in, rows, cols, out);
+  TWELL_LAUNCH("transpose_wd", s, transpose_bf16_kernel<<<grid, 256, 0, s>>>(in, rows, cols, out));
   return cudaGetLastError();
 }
 

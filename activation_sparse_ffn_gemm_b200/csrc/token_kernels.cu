@@ -1,0 +1,455 @@
+// token_kernels.cu — per-token CUDA-core kernels over the TwELL (ELL) rows.
+//
+// Forward: "Sakana AI и NVIDIA представили TwELL — формат и CUDA-ядра ...",
+// paragraph 2: a fused kernel reads TwELL activations and performs the up and
+// down projections at once, never writing the hidden state to global memory.
+// For each token row i and each kept active unit j (value g_ij):
+//   u_ij = x_i . W_u[j]            (x_i in registers, W_u[j] gathered)
+//   h_ij = g_ij u_ij               (shared memory only)
+//   Y_i  = sum_j h_ij W_d[:, j]    (W_d gathered unit-major from W_dt[j])
+// Backward over the same rows (same page, paragraph 2: training runs on the
+// hybrid format): dH_ij = dY_i . W_d[:, j], dU = dH g, dZ = dH u + lambda,
+// dX_i = sum_j dU_ij W_u[j] + dZ_ij W_g[j]; dU and dZ are kept per slot for the
+// weight gradients.
+//
+// The work is a stream of weight-row gathers from L2 (each active pair reads
+// whole d-wide rows), so the kernels are organised to keep many independent
+// 16-byte loads in flight with few instructions per byte:
+//   * a token is owned by a group of W warps (W = 1 for d <= 2048); each lane
+//     holds C 16-byte chunks of the row (x or dY packed as bf16, Y or dX as
+//     fp32), so a unit's row is one C-deep burst of coalesced loads per lane;
+//   * units are processed B at a time (all B*C loads issued before any use);
+//   * no CTA-wide barrier: a single-warp group synchronises with __syncwarp,
+//     wider groups with a named barrier of their own.
+// Overflow rows are skipped (the dense backup path owns them).
+#include "trace.cuh"
+#include "twell_internal.cuh"
+
+namespace twell {
+
+namespace {
+
+constexpr int kTokWarps = 8;   // warps per CTA
+constexpr int kListCap = 256;  // list entries per chunk and group
+
+template <int C, int W>
+struct TokCfg {
+  static constexpr int G = kTokWarps / W;  // token groups per CTA
+  static constexpr int B = C >= 8 ? 2 : (C >= 4 ? 4 : 8);
+  static constexpr int GT = W * 32;        // threads per group
+};
+
+struct GroupSmem {
+  int off[kMaxTiles];  // exclusive offsets of the kept entries per tile
+  int tot;
+  int j[kListCap];     // unit of each entry
+  float c[kListCap];   // coefficient (g, then h; or dU)
+  float c2[kListCap];  // second coefficient (u, then dZ) in the backward
+  int slot[kListCap];  // t * K + s
+};
+
+template <int W>
+__device__ __forceinline__ void group_sync(int grp) {
+  if (W == 1) {
+    __syncwarp();
+  } else {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(W * 32) : "memory");
+  }
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+// Kept-entry offsets of `row` over its T tiles, computed by warp 0 of the group.
+__device__ __forceinline__ void row_offsets(const uint16_t* __restrict__ count, long row, int T, int K, int lane,
+                                            GroupSmem& g) {
+  int run = 0;
+  for (int t0 = 0; t0 < T; t0 += 32) {
+    const int t = t0 + lane;
+    int c = 0;
+    if (t < T) {
+      c = count[row * T + t];
+      c = c < K ? c : K;
+    }
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (t < T) g.off[t] = run + incl - c;
+    run += __shfl_sync(0xFFFFFFFFu, incl, 31);
+  }
+  if (lane == 0) g.tot = run;
+}
+
+__device__ __forceinline__ void entry_of(const int* off, int T, int e, int& t, int& sl) {
+  int lo = 0, hi = T - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (off[mid] <= e) lo = mid;
+    else hi = mid - 1;
+  }
+  t = lo;
+  sl = e - off[lo];
+}
+
+// dot of C packed-bf16 chunks (register operand) with C chunks of a row.
+template <int C>
+__device__ __forceinline__ float dot_chunks(const uint4 (&a)[C], const uint4 (&w)[C]) {
+  float s = 0.f;
+#pragma unroll
+  for (int c = 0; c < C; ++c) {
+    const uint32_t av[4] = {a[c].x, a[c].y, a[c].z, a[c].w};
+    const uint32_t wv[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      s = fmaf(bf16_lo(av[e]), bf16_lo(wv[e]), s);
+      s = fmaf(bf16_hi(av[e]), bf16_hi(wv[e]), s);
+    }
+  }
+  return s;
+}
+
+template <int C>
+__device__ __forceinline__ void axpy_chunks(float a, const uint4 (&w)[C], float (&y)[C][8]) {
+#pragma unroll
+  for (int c = 0; c < C; ++c) {
+    float f[8];
+    unpack8(w[c], f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[c][e] = fmaf(a, f[e], y[c][e]);
+  }
+}
+
+// Chunk q of this lane: index (wi*32 + lane) + W*32*q into the row's d/8 chunks.
+template <int C, int W>
+__device__ __forceinline__ void load_row(const uint16_t* __restrict__ base, int first, int nch, uint4 (&v)[C]) {
+  const uint4* p = reinterpret_cast<const uint4*>(base);
+#pragma unroll
+  for (int q = 0; q < C; ++q) {
+    const int idx = first + W * 32 * q;
+    v[q] = idx < nch ? __ldg(p + idx) : make_uint4(0, 0, 0, 0);
+  }
+}
+
+// Phases of one list chunk [e0, e0 + ne) of a token row, shared by the two
+// kernels below. `g` is the token group's shared memory.
+
+__device__ __forceinline__ void build_list(GroupSmem& g, long row, int T, int K, int e0, int ne, int gtid, int GT,
+                                           const uint16_t* __restrict__ val, const uint8_t* __restrict__ col,
+                                           const float* __restrict__ u_ell) {
+  for (int e = gtid; e < ne; e += GT) {
+    int t, sl;
+    entry_of(g.off, T, e0 + e, t, sl);
+    const long base = (row * T + t) * K + sl;
+    g.j[e] = t * kTn + col[base];
+    g.c[e] = __uint_as_float(static_cast<uint32_t>(val[base]) << 16);
+    if (u_ell) g.c2[e] = u_ell[base];
+    g.slot[e] = t * K + sl;
+  }
+}
+
+// Dot products of a register-resident row (xp) with the gathered rows Wr[j] of
+// the listed units; the full dots land in out[e] (W == 1) or as per-warp
+// partials in part[wi][e] (W > 1).
+template <int C, int W, int B>
+__device__ __forceinline__ void gather_dots(const GroupSmem& g, int ne, const uint4 (&xp)[C],
+                                            const uint16_t* __restrict__ Wr, int d, int first, int nch, int lane,
+                                            float* out, float* part_w) {
+  for (int k = 0; k < ne; k += B) {
+    uint4 wv[B][C];
+#pragma unroll
+    for (int q = 0; q < B; ++q) load_row<C, W>(Wr + static_cast<long>(g.j[min(k + q, ne - 1)]) * d, first, nch, wv[q]);
+#pragma unroll
+    for (int q = 0; q < B; ++q) {
+      const float s = warp_sum(dot_chunks<C>(xp, wv[q]));
+      if (lane == 0 && k + q < ne) (W == 1 ? out : part_w)[k + q] = s;
+    }
+  }
+}
+
+// y += sum over listed units of coef[e] * Wr[j_e].
+template <int C, int W, int B>
+__device__ __forceinline__ void gather_axpy(const GroupSmem& g, int ne, const float* coef,
+                                            const uint16_t* __restrict__ Wr, int d, int first, int nch,
+                                            float (&y)[C][8]) {
+  for (int k = 0; k < ne; k += B) {
+    uint4 wv[B][C];
+    float h[B];
+#pragma unroll
+    for (int q = 0; q < B; ++q) {
+      const bool in = k + q < ne;
+      h[q] = in ? coef[k + q] : 0.f;
+      load_row<C, W>(Wr + static_cast<long>(g.j[in ? k + q : k]) * d, first, nch, wv[q]);
+    }
+#pragma unroll
+    for (int q = 0; q < B; ++q) axpy_chunks<C>(h[q], wv[q], y);
+  }
+}
+
+template <int C>
+__device__ __forceinline__ void zero_acc(float (&y)[C][8]) {
+#pragma unroll
+  for (int q = 0; q < C; ++q)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[q][e] = 0.f;
+}
+
+// LONG = false: rows whose kept entries fit one list (the common case): the
+// row operand (x or dY) and the accumulators (Y or dX) are never live together,
+// which keeps these kernels at two CTAs per SM. LONG = true: the rare rows with
+// more entries, processed in list chunks with the accumulators kept live.
+template <int C, int W, bool LONG>
+__global__ void __launch_bounds__(kTokWarps * 32, LONG ? 1 : 2) ell_fwd_kernel(
+    const uint16_t* __restrict__ X, const uint16_t* __restrict__ Wu, const uint16_t* __restrict__ Wdt,
+    const uint16_t* __restrict__ count, const uint16_t* __restrict__ val, const uint8_t* __restrict__ col,
+    const uint8_t* __restrict__ row_ovf, float* __restrict__ u_ell, uint16_t* __restrict__ Y, int M, int d, int T,
+    int K) {
+  using Cfg = TokCfg<C, W>;
+  constexpr int B = Cfg::B;
+  __shared__ GroupSmem gs[Cfg::G];
+  __shared__ float part[Cfg::G][W > 1 ? W : 1][kListCap];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = warp / W, wi = warp % W, gtid = wi * 32 + lane;
+  GroupSmem& g = gs[grp];
+  const int nch = d >> 3;
+  const int first = gtid;
+
+  // u = x . W_u[j] for the listed units, then h = g u in g.c (u saved when asked)
+  auto up = [&](long row, int ne) {
+    {
+      uint4 xp[C];
+      load_row<C, W>(X + row * d, first, nch, xp);
+      gather_dots<C, W, B>(g, ne, xp, Wu, d, first, nch, lane, g.c2, part[grp][wi]);
+    }
+    group_sync<W>(grp);
+    for (int e = gtid; e < ne; e += Cfg::GT) {
+      float u = g.c2[e];
+      if (W > 1) {
+        u = 0.f;
+#pragma unroll
+        for (int w = 0; w < W; ++w) u += part[grp][w][e];
+      }
+      g.c[e] *= u;
+      if (u_ell) u_ell[row * T * K + g.slot[e]] = u;
+    }
+    group_sync<W>(grp);
+  };
+  auto store = [&](long row, const float (&y)[C][8]) {
+    uint4* yr = reinterpret_cast<uint4*>(Y + row * d);
+#pragma unroll
+    for (int q = 0; q < C; ++q) {
+      const int idx = first + W * 32 * q;
+      if (idx < nch)
+        yr[idx] = make_uint4(pack_bf16x2(y[q][0], y[q][1]), pack_bf16x2(y[q][2], y[q][3]),
+                             pack_bf16x2(y[q][4], y[q][5]), pack_bf16x2(y[q][6], y[q][7]));
+    }
+  };
+
+  for (long row = static_cast<long>(blockIdx.x) * Cfg::G + grp; row < M; row += static_cast<long>(gridDim.x) * Cfg::G) {
+    if (row_ovf[row]) continue;
+    if (wi == 0) row_offsets(count, row, T, K, lane, g);
+    group_sync<W>(grp);
+    const int total = g.tot;
+    if ((total > kListCap) == LONG) {
+      if constexpr (!LONG) {
+        build_list(g, row, T, K, 0, total, gtid, Cfg::GT, val, col, nullptr);
+        group_sync<W>(grp);
+        up(row, total);
+        float y[C][8];
+        zero_acc<C>(y);
+        gather_axpy<C, W, B>(g, total, g.c, Wdt, d, first, nch, y);
+        store(row, y);
+      } else {
+        float y[C][8];
+        zero_acc<C>(y);
+        for (int e0 = 0; e0 < total; e0 += kListCap) {
+          const int ne = min(kListCap, total - e0);
+          build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, nullptr);
+          group_sync<W>(grp);
+          up(row, ne);
+          gather_axpy<C, W, B>(g, ne, g.c, Wdt, d, first, nch, y);
+          group_sync<W>(grp);
+        }
+        store(row, y);
+      }
+    }
+    group_sync<W>(grp);  // warp 0 rewrites the offsets for the next row
+  }
+}
+
+template <int C, int W, bool LONG>
+__global__ void __launch_bounds__(kTokWarps * 32, LONG ? 1 : 2) ell_bwd_kernel(
+    const uint16_t* __restrict__ dY, const uint16_t* __restrict__ Wu, const uint16_t* __restrict__ Wg,
+    const uint16_t* __restrict__ Wdt, const uint16_t* __restrict__ count, const uint16_t* __restrict__ val,
+    const uint8_t* __restrict__ col, const uint8_t* __restrict__ row_ovf, const float* __restrict__ u_ell,
+    float lambda, float* __restrict__ du_ell, float* __restrict__ dz_ell, float* __restrict__ dX, int M, int d,
+    int T, int K) {
+  using Cfg = TokCfg<C, W>;
+  constexpr int B = Cfg::B;
+  constexpr int B2 = B > 1 ? B / 2 : 1;  // two rows (W_u, W_g) per unit in the dX phase
+  __shared__ GroupSmem gs[Cfg::G];
+  __shared__ float part[Cfg::G][W > 1 ? W : 1][kListCap];
+  __shared__ float dhv[Cfg::G][kListCap];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = warp / W, wi = warp % W, gtid = wi * 32 + lane;
+  GroupSmem& g = gs[grp];
+  const int nch = d >> 3;
+  const int first = gtid;
+
+  // dH = dY_i . W_d[:, j] for the listed units, then dU (in g.c) and dZ (in g.c2)
+  auto dh_phase = [&](long row, int ne) {
+    {
+      uint4 dyp[C];
+      load_row<C, W>(dY + row * d, first, nch, dyp);
+      gather_dots<C, W, B>(g, ne, dyp, Wdt, d, first, nch, lane, dhv[grp], part[grp][wi]);
+    }
+    group_sync<W>(grp);
+    for (int e = gtid; e < ne; e += Cfg::GT) {
+      float s = dhv[grp][e];
+      if (W > 1) {
+        s = 0.f;
+#pragma unroll
+        for (int w = 0; w < W; ++w) s += part[grp][w][e];
+      }
+      const float du = s * g.c[e];
+      const float dz = fmaf(s, g.c2[e], lambda);
+      g.c[e] = du;
+      g.c2[e] = dz;
+      du_ell[row * T * K + g.slot[e]] = du;
+      dz_ell[row * T * K + g.slot[e]] = dz;
+    }
+    group_sync<W>(grp);
+  };
+  auto dx_phase = [&](int ne, float (&dx)[C][8]) {
+    gather_axpy<C, W, B2>(g, ne, g.c, Wu, d, first, nch, dx);
+    gather_axpy<C, W, B2>(g, ne, g.c2, Wg, d, first, nch, dx);
+  };
+  auto store = [&](long row, const float (&dx)[C][8]) {
+    float4* xr = reinterpret_cast<float4*>(dX + row * d);
+#pragma unroll
+    for (int q = 0; q < C; ++q) {
+      const int idx = first + W * 32 * q;
+      if (idx < nch) {
+        xr[2 * idx] = make_float4(dx[q][0], dx[q][1], dx[q][2], dx[q][3]);
+        xr[2 * idx + 1] = make_float4(dx[q][4], dx[q][5], dx[q][6], dx[q][7]);
+      }
+    }
+  };
+
+  for (long row = static_cast<long>(blockIdx.x) * Cfg::G + grp; row < M; row += static_cast<long>(gridDim.x) * Cfg::G) {
+    if (row_ovf[row]) continue;
+    if (wi == 0) row_offsets(count, row, T, K, lane, g);
+    group_sync<W>(grp);
+    const int total = g.tot;
+    if ((total > kListCap) == LONG) {
+      if constexpr (!LONG) {
+        build_list(g, row, T, K, 0, total, gtid, Cfg::GT, val, col, u_ell);
+        group_sync<W>(grp);
+        dh_phase(row, total);
+        float dx[C][8];
+        zero_acc<C>(dx);
+        dx_phase(total, dx);
+        store(row, dx);
+      } else {
+        float dx[C][8];
+        zero_acc<C>(dx);
+        for (int e0 = 0; e0 < total; e0 += kListCap) {
+          const int ne = min(kListCap, total - e0);
+          build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, u_ell);
+          group_sync<W>(grp);
+          dh_phase(row, ne);
+          dx_phase(ne, dx);
+          group_sync<W>(grp);
+        }
+        store(row, dx);
+      }
+    }
+    group_sync<W>(grp);  // warp 0 rewrites the offsets for the next row
+  }
+}
+
+// Chunks per lane C and warps per token W for a row of d bf16 (d/8 chunks).
+void tok_shape(int d, int& C, int& W) {
+  const int nch = d / 8;
+  if (nch <= 32) C = 1, W = 1;
+  else if (nch <= 64) C = 2, W = 1;
+  else if (nch <= 128) C = 4, W = 1;
+  else if (nch <= 256) C = 8, W = 1;
+  else if (nch <= 512) C = 8, W = 2;
+  else if (nch <= 1024) C = 8, W = 4;
+  else C = 8, W = 8;
+}
+
+int tok_grid(int M, int G) {
+  const long need = (static_cast<long>(M) + G - 1) / G;
+  const long cap = static_cast<long>(device_sm_count()) * 8;
+  return static_cast<int>(need < cap ? need : cap);
+}
+
+// Rows whose kept entries exceed one list are rare; the second pass only reads
+// the per-tile counts of the rows it skips.
+template <int C, int W, typename... A>
+void launch_fwd_cw(int M, cudaStream_t s, A... a) {
+  const int grid = tok_grid(M, TokCfg<C, W>::G);
+  TWELL_LAUNCH("ell_updown", s, ell_fwd_kernel<C, W, false><<<grid, kTokWarps * 32, 0, s>>>(a...));
+  TWELL_LAUNCH("ell_updown_long", s, ell_fwd_kernel<C, W, true><<<grid, kTokWarps * 32, 0, s>>>(a...));
+}
+
+template <int C, int W, typename... A>
+void launch_bwd_cw(int M, cudaStream_t s, A... a) {
+  const int grid = tok_grid(M, TokCfg<C, W>::G);
+  TWELL_LAUNCH("ell_bwd", s, ell_bwd_kernel<C, W, false><<<grid, kTokWarps * 32, 0, s>>>(a...));
+  TWELL_LAUNCH("ell_bwd_long", s, ell_bwd_kernel<C, W, true><<<grid, kTokWarps * 32, 0, s>>>(a...));
+}
+
+}  // namespace
+
+cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
+                               const uint16_t* count, const uint16_t* val, const uint8_t* col,
+                               const uint8_t* row_ovf, float* u_ell, uint16_t* Y, int M, int d, int f, int K,
+                               cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  int C, W;
+  tok_shape(d, C, W);
+  const int T = f / kTn;
+#define TWELL_FWD(CC, WW) launch_fwd_cw<CC, WW>(M, s, X, W_u, W_dt, count, val, col, row_ovf, u_ell, Y, M, d, T, K)
+  if (W == 1 && C == 1) TWELL_FWD(1, 1);
+  else if (W == 1 && C == 2) TWELL_FWD(2, 1);
+  else if (W == 1 && C == 4) TWELL_FWD(4, 1);
+  else if (W == 1) TWELL_FWD(8, 1);
+  else if (W == 2) TWELL_FWD(8, 2);
+  else if (W == 4) TWELL_FWD(8, 4);
+  else TWELL_FWD(8, 8);
+#undef TWELL_FWD
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const uint16_t* W_g,
+                               const uint16_t* W_dt, const uint16_t* count, const uint16_t* val,
+                               const uint8_t* col, const uint8_t* row_ovf, const float* u_ell, float lambda,
+                               float* du_ell, float* dz_ell, float* dX, int M, int d, int f, int K,
+                               cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  int C, W;
+  tok_shape(d, C, W);
+  const int T = f / kTn;
+#define TWELL_BWD(CC, WW)                                                                                      \
+  launch_bwd_cw<CC, WW>(M, s, dY, W_u, W_g, W_dt, count, val, col, row_ovf, u_ell, lambda, du_ell, dz_ell, dX, \
+                        M, d, T, K)
+  if (W == 1 && C == 1) TWELL_BWD(1, 1);
+  else if (W == 1 && C == 2) TWELL_BWD(2, 1);
+  else if (W == 1 && C == 4) TWELL_BWD(4, 1);
+  else if (W == 1) TWELL_BWD(8, 1);
+  else if (W == 2) TWELL_BWD(8, 2);
+  else if (W == 4) TWELL_BWD(8, 4);
+  else TWELL_BWD(8, 8);
+#undef TWELL_BWD
+  return cudaGetLastError();
+}
+
+}  // namespace twell

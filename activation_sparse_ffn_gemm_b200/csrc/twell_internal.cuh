@@ -109,13 +109,13 @@ cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const u
 
 struct CscBuffers {
   int* row_slot;   // [M]
-  int* block_cnt;  // [ceil(M/kCscRows)][f]
+  int* block_cnt;  // [ceil(M/kCscRows)][f] per-chunk counts, then their exclusive scan
   int* unit_tot;   // [f]
   int* unit_ptr;   // [f+1]
   int* csc_row;    // [nnz_cap]
   float4* csc_val; // [nnz_cap]: (h, dU, dZ, 0)
 };
-constexpr int kCscRows = 64;
+constexpr int kCscRows = 256;  // rows per chunk of the pair-list build
 
 // Unit-major list of every active (row, unit) pair of the hybrid format, in
 // ascending row order per unit, with h, dU and dZ attached.

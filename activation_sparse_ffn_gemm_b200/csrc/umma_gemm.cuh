@@ -23,6 +23,7 @@
 #pragma once
 
 #include "sm100.cuh"
+#include "trace.cuh"
 #include "twell_internal.cuh"
 
 namespace twell {
@@ -276,7 +277,7 @@ constexpr int gemm_smem_bytes() {
 // Launches the GEMM on min(#SMs, tiles) persistent CTAs. The static row bound
 // shp.M sizes the grid; rows beyond *M_dev are skipped by the device.
 template <class Epi, int BN, bool B_MN, int STAGES>
-cudaError_t launch_umma_gemm(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
+cudaError_t launch_umma_gemm(const char* name, const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
                              const CUtensorMap& b1, const GemmShape& shp, const typename Epi::Args& ea,
                              cudaStream_t s) {
   constexpr int smem = gemm_smem_bytes<Epi, BN, STAGES>();
@@ -287,7 +288,7 @@ cudaError_t launch_umma_gemm(const CUtensorMap& a0, const CUtensorMap& b0, const
   const long tiles = static_cast<long>((shp.M + kBM - 1) / kBM) * ((shp.N + BN - 1) / BN);
   if (tiles <= 0) return cudaSuccess;
   const int grid = static_cast<int>(tiles < device_sm_count() ? tiles : device_sm_count());
-  kern<<<grid, kGemmThreads, smem, s>>>(a0, b0, a1, b1, shp, ea);
+  TWELL_LAUNCH(name, s, kern<<<grid, kGemmThreads, smem, s>>>(a0, b0, a1, b1, shp, ea));
   return cudaGetLastError();
 }
 

@@ -1,0 +1,501 @@
+#!/usr/bin/env python
+"""Throughput of the TwELL activation-sparse gated FFN training step on B200.
+
+One step = the whole hot path over one batch: W_d transposed for the step's
+weights, the gate GEMM with the TwELL pack epilogue, row routing, the sparse
+up+down for ELL rows and the dense backup for overflow rows, then the backward
+over the hybrid format (L1 term on the gate activations). Workload: the uniform
+1%-activity inference shape (M=4096 tokens, d_model=2048, d_ff=8192, T_n=128,
+K=8) run as a training step, synthetic seeded data, inputs resident in HBM.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Prints one JSON line (rank 0). With N > 1 (torchrun) every rank runs its own
+replica of the batch; the time is the max over ranks and the value counts the
+tokens of all ranks (weak scaling; the path has no exchange step).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse FFN tokens/s fwd & fwd+bwd at 99% sparsity vs dense; % of roofline"
+L2_FLUSH_BYTES = 256 << 20
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["twell", "reference"], default="twell")
+    p.add_argument("--lam", type=float, default=1e-3)
+    p.add_argument("--cpu-seconds", type=float, default=8.0, help="target CPU work of the oracle baseline sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-dense", action="store_true")
+    p.add_argument("--no-trace", action="store_true")
+    return p.parse_args()
+
+
+def reduce_max(x: float, dist=None, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    if dist is None:
+        return x
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_env():
+    return int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def workload():
+    from synthetic import WORKLOADS
+
+    w = WORKLOADS["uniform"]
+    with open(os.path.join(ROOT, "tests", "golden", "uniform_seed.json")) as fh:
+        seed = json.load(fh)["seed"]
+    return w, seed
+
+
+def workload_desc(w, seed):
+    return (f"uniform i.i.d. {w.activity:.0%} activity: M={w.M} tokens, d_model={w.d_model}, d_ff={w.d_ff}, "
+            f"T_n={w.T_n}, K={w.K}, seed {seed} (no overflowing row), run as a training step")
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        time.sleep(0.25)
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------ algorithmic work
+
+
+def kernel_work(name, M, d, f, T, K, kept, pairs):
+    """Algorithmic flops (tensor-bound kernels) or bytes (memory-bound) of one launch.
+
+    kept = stored slots of ELL rows, pairs = all active (row, unit) pairs."""
+    if name == "gate_pack_gemm":
+        return "tensor", 2.0 * M * d * f
+    if name == "ell_updown":
+        return "hbm", (2 * M * d            # X
+                       + M * T * (2 + 3 * K)  # TwELL count/val/col
+                       + 4 * kept             # u written
+                       + 2 * M * d            # Y written
+                       + 2 * 2 * f * d)       # W_u, W_dt read once
+    if name == "ell_bwd":
+        return "hbm", (2 * M * d + M * T * (2 + 3 * K) + 4 * kept + 8 * kept + 4 * M * d + 3 * 2 * f * d)
+    if name == "weight_grads":
+        return "hbm", (2 * 2 * M * d + 20 * pairs + 3 * 4 * f * d + 4 * f)
+    if name == "transpose_wd":
+        return "hbm", 2 * 2 * f * d
+    if name in ("csc_count", "csc_fill"):
+        return "hbm", M * T * (2 + K) + (20 * pairs if name == "csc_fill" else 0)
+    return None, None
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "activation_sparse_ffn_gemm_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as fh:
+            h.update(fn.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it matches this source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        d = json.load(fh)
+    rec = d.get("kernels", {}).get(kernel)
+    if not rec or d.get("source_sha") != source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------ CPU oracle
+
+
+def cpu_baseline(inp, lam, target_s):
+    """The fp64 oracle as it stands, forward + backward on a bounded sample of token rows."""
+    import numpy as np
+
+    from oracle import oracle as O
+
+    O.build()
+    M = inp["X"].shape[0]
+
+    def run(n):
+        rows = np.arange(n)
+        t0 = time.perf_counter()
+        O.ffn_fwd(inp["X"], inp["W_g"], inp["b_g"], inp["W_u"], inp["W_d"], rows=rows.astype(np.int32))
+        O.ffn_bwd(inp["X"][:n], inp["W_g"], inp["b_g"], inp["W_u"], inp["W_d"], inp["dY"][:n], lam)
+        return time.perf_counter() - t0
+
+    n = 32
+    t = run(n)
+    if t < target_s / 4:
+        n = int(min(M, max(n, n * target_s / max(t, 1e-3))))
+        t = run(n)
+    return {"value": n / t, "unit": "tokens/s", "cores": O.get_threads(), "kind": "oracle",
+            "sample": f"first {n} of {M} token rows, forward + backward (weight gradients over the sample), "
+                      f"{t:.1f} s"}, n, t
+
+
+# --------------------------------------------------------------- arms
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import numpy as np
+
+    from oracle import oracle as O
+    from synthetic import make_inputs
+
+    w, seed = workload()
+    inp = make_inputs(w, seed=seed, with_dY=True)
+    O.build()
+    # each step: the oracle's forward + backward on a bounded sample of rows
+    probe = cpu_baseline(inp, args.lam, target_s=max(1.0, 60.0 / max(1, args.steps + args.warmup)))
+    n = probe[1]
+    rows = np.arange(n, dtype=np.int32)
+
+    def step():
+        O.ffn_fwd(inp["X"], inp["W_g"], inp["b_g"], inp["W_u"], inp["W_d"], rows=rows)
+        O.ffn_bwd(inp["X"][:n], inp["W_g"], inp["b_g"], inp["W_u"], inp["W_d"], inp["dY"][:n], args.lam)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / max(1, args.steps)
+    value = n / dt
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": workload_desc(w, seed), "sample_rows_per_step": n,
+                   "reference": "fp64 CPU oracle (oracle/twell_oracle.c), OpenMP over rows"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": O.get_threads(), "kind": "oracle",
+                         "sample": f"first {n} of {w.M} token rows per step, forward + backward"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_twell(args, world, rank, local):
+    import numpy as np
+    import torch
+
+    import activation_sparse_ffn_gemm_b200 as tw
+    from synthetic import make_inputs
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        return reduce_max(x, dist, dev)
+
+    w, seed = workload()
+    inp = make_inputs(w, seed=seed, with_dY=True)
+
+    def dev_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    X, W_g, b_g, W_u, W_d, dY = (dev_bf16(inp[k]) for k in ("X", "W_g", "b_g", "W_u", "W_d", "dY"))
+    M, d, f, K, T = w.M, w.d_model, w.d_ff, w.K, w.d_ff // w.T_n
+    cap = M
+    st = tw.HybridState(M, f, w.T_n, K, cap, dev, with_u=True)
+    wsf = tw.workspace(tw.OP_FWD, M, d, f, w.T_n, K, cap, dev)
+    wsb = tw.workspace(tw.OP_BWD, M, d, f, w.T_n, K, cap, dev)
+    Wdt = torch.empty((f, d), dtype=torch.bfloat16, device=dev)
+    Y = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
+    grads = dict(dX=torch.empty((M, d), device=dev), dW_g=torch.empty((f, d), device=dev),
+                 dW_u=torch.empty((f, d), device=dev), dW_d=torch.empty((d, f), device=dev),
+                 db_g=torch.empty(f, device=dev))
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd():
+        tw.transpose_wd(W_d, out=Wdt)
+        tw.ffn_fwd(X, W_g, b_g, W_u, W_d, T_n=w.T_n, K=K, W_dt=Wdt, state=st, ws=wsf, Y=Y)
+
+    def bwd():
+        tw.ffn_bwd(X, W_g, W_u, W_d, st, dY, lam=args.lam, W_dt=Wdt, ws=wsb, out=grads)
+
+    def timed(n, body, mid=None):
+        """Per-step CUDA events on the launching stream, L2 flushed before each step."""
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+               torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        barrier()
+        torch.cuda.synchronize(dev)
+        for e0, e1, e2 in ev:
+            flush.zero_()
+            e0.record(stream)
+            body(e1)
+            e2.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        tot = [a.elapsed_time(c) for a, _, c in ev]
+        first = [a.elapsed_time(b) for a, b, _ in ev]
+        return sum(tot) / n, sum(first) / n
+
+    def train_step(e_mid):
+        fwd()
+        e_mid.record(stream)
+        bwd()
+
+    for _ in range(max(3, args.warmup)):
+        train_step(torch.cuda.Event())
+    torch.cuda.synchronize(dev)
+    assert st.read_status() == 0, "device status word set during warm-up"
+    nst, nfl = st.n_overflow()
+    activity = float(st.count.sum().item()) / (M * f)
+    cnt = st.count.float()
+
+    launches0 = tw.launch_count()
+    with ClockSampler(local) as clk:
+        ms_step, ms_fwd = timed(args.steps, train_step)
+    launches = tw.launch_count() - launches0
+    ms_step = max_over_ranks(ms_step)
+    ms_fwd = max_over_ranks(ms_fwd)
+
+    # per-kernel breakdown: the same steps again with event tracing
+    breakdown = {}
+    if not args.no_trace:
+        tw.trace_collect()
+        tw.trace_enable(True)
+        timed(args.steps, train_step)
+        tw.trace_enable(False)
+        for name, ms in tw.trace_collect():
+            b = breakdown.setdefault(name, {"launches": 0, "ms": 0.0})
+            b["launches"] += 1
+            b["ms"] += ms
+        for b in breakdown.values():
+            b["ms_per_launch"] = b["ms"] / b["launches"]
+            b["ms_per_step"] = b["ms"] / args.steps
+
+    # e2e: inputs from pinned host memory each step, Y read back each step
+    hX = torch.empty((M, d), dtype=torch.bfloat16, pin_memory=True)
+    hdY = torch.empty((M, d), dtype=torch.bfloat16, pin_memory=True)
+    hY = torch.empty((M, d), dtype=torch.bfloat16, pin_memory=True)
+    hX.copy_(X.cpu())
+    hdY.copy_(dY.cpu())
+
+    def e2e_step(e_mid):
+        X.copy_(hX, non_blocking=True)
+        dY.copy_(hdY, non_blocking=True)
+        train_step(e_mid)
+        hY.copy_(Y, non_blocking=True)
+
+    ms_e2e, _ = timed(args.steps, e2e_step)
+    ms_e2e = max_over_ranks(ms_e2e)
+    assert st.read_status() == 0, "device status word set during timing"
+
+    # dense bf16 comparison point (torch / cuBLAS), same protocol
+    dense = None
+    if not args.no_dense:
+        Wg_r, Wu_r, Wd_r = (t.clone().requires_grad_() for t in (W_g, W_u, W_d))
+        Xr = X.clone().requires_grad_()
+
+        def dense_fwd(e_mid):
+            with torch.no_grad():
+                (torch.relu(X @ W_g.T + b_g) * (X @ W_u.T)) @ W_d.T
+            e_mid.record(stream)
+
+        def dense_fb(e_mid):
+            z = Xr @ Wg_r.T + b_g
+            g = torch.relu(z)
+            y = (g * (Xr @ Wu_r.T)) @ Wd_r.T
+            (y.float() * dY.float()).sum().add(g.float().sum() * args.lam).backward()
+            Xr.grad = Wg_r.grad = Wu_r.grad = Wd_r.grad = None
+            e_mid.record(stream)
+
+        for _ in range(3):
+            dense_fwd(torch.cuda.Event())
+            dense_fb(torch.cuda.Event())
+        dm_f, _ = timed(args.steps, dense_fwd)
+        dm_fb, _ = timed(args.steps, dense_fb)
+        dm_f, dm_fb = max_over_ranks(dm_f), max_over_ranks(dm_fb)
+        dense = {"fwd_tokens_per_s": M * world / (dm_f / 1e3), "fwd_bwd_tokens_per_s": M * world / (dm_fb / 1e3),
+                 "fwd_ms": dm_f, "fwd_bwd_ms": dm_fb, "impl": "torch bf16 matmuls (cuBLAS), autograd backward"}
+
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    ell_rows = (st.row_ovf[:M] == 0).unsqueeze(1)
+    kept = int((torch.minimum(st.count.int(), torch.tensor(K, device=dev)) * ell_rows).sum().item())
+    pairs = int(st.count.int().sum().item())
+    roofline = None
+    if breakdown:
+        top = max(breakdown, key=lambda k: breakdown[k]["ms"])
+        bound, work = kernel_work(top, M, d, f, T, K, kept, pairs)
+        b = breakdown[top]
+        if bound == "tensor":
+            peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+            achieved = work / (b["ms_per_launch"] / 1e3) / 1e12
+            unit = "TFLOP/s"
+        elif bound == "hbm":
+            peak = peaks["hbm_gbs"]
+            achieved = work / (b["ms_per_launch"] / 1e3) / 1e9
+            unit = "GB/s"
+        else:
+            peak = achieved = None
+            unit = None
+        roofline = {"kernel": top, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                    "frac": (achieved / peak) if achieved and peak else None,
+                    "traffic": committed_traffic(top),
+                    "peak_source": f"{peak_src} ({'sustained bf16' if bound == 'tensor' else 'HBM copy'}, "
+                                   "MEASURED_PEAKS.json)",
+                    "work_per_launch": work,
+                    "share_of_step": b["ms_per_step"] / ms_step if ms_step else None}
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        cpu, _, _ = cpu_baseline(inp, args.lam, args.cpu_seconds)
+
+    tokens = M * world
+    line = {
+        "metric": METRIC,
+        "value": tokens / (ms_step / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": workload_desc(w, seed), "global_batch": tokens, "lambda_l1": args.lam,
+                   "l2": "flushed before every timed step (256 MiB device write, outside the events)",
+                   "accumulation": "fp32", "ovf_cap": cap, "parallelism": f"replicas x{world}"},
+        "fwd": {"tokens_per_s": tokens / (ms_fwd / 1e3), "ms": ms_fwd},
+        "dense_bf16": dense,
+        "speedup_vs_dense": ({"fwd": dense["fwd_ms"] / ms_fwd, "fwd_bwd": dense["fwd_bwd_ms"] / ms_step}
+                             if dense else None),
+        "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": 2 * M * d * 2,
+                "d2h_bytes_per_step": M * d * 2},
+        "gpu_launches": launches,
+        "roofline": roofline,
+        "kernels": {k: {"launches_per_step": v["launches"] / args.steps, "ms_per_step": v["ms_per_step"]}
+                    for k, v in sorted(breakdown.items(), key=lambda kv: -kv[1]["ms"])},
+        "sparsity": {"activity": activity, "overflow_rows": nfl, "max_count": float(cnt.max().item()),
+                     "mean_count": float(cnt.mean().item())},
+        "clocks": clk.summary(),
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+    else:
+        run_twell(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -180,6 +180,27 @@ TWELL_API twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, con
  * it when `clear` is non-zero. Returns TWELL_ECUDA if the copy fails. */
 TWELL_API twell_status twell_status_read(const twell_hybrid* h, uint32_t* out, int clear, twell_stream_t stream);
 
+/*
+ * Launch accounting and per-kernel timing (no counterpart on the pages; a
+ * runtime aid for measuring where a call spends its time without a profiler).
+ *   twell_launch_count   number of kernels this library has launched in the
+ *                        process so far (monotonic; thread-safe)
+ *   twell_trace_enable   while on, every kernel launch is bracketed by two CUDA
+ *                        events recorded on its stream (adds two event records
+ *                        per kernel; off by default)
+ *   twell_trace_collect  waits for the recorded events, writes up to max_recs
+ *                        records (kernel name, duration in ms) to out (nullable),
+ *                        forgets them and returns how many there were
+ */
+typedef struct twell_trace_rec {
+  char name[32];
+  float ms;
+} twell_trace_rec;
+
+TWELL_API uint64_t twell_launch_count(void);
+TWELL_API void twell_trace_enable(int on);
+TWELL_API int twell_trace_collect(twell_trace_rec* out, int max_recs);
+
 #ifdef __cplusplus
 }
 #endif
