@@ -73,6 +73,8 @@ def lib():
             L.twell_transpose_wd.argtypes = [_vp, _i64, _i64, _vp, _vp]
             L.twell_pack.restype = ctypes.c_int
             L.twell_pack.argtypes = [_vp, _vp, _vp, _i64, ctypes.POINTER(TwellHybrid), _vp, _vp, ctypes.c_size_t, _vp]
+            L.twell_pack_noalloc.restype = ctypes.c_int
+            L.twell_pack_noalloc.argtypes = [_vp, _vp, _vp, _i64, ctypes.POINTER(TwellHybrid), _vp, _vp]
             L.twell_ffn_fwd.restype = ctypes.c_int
             L.twell_ffn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, ctypes.POINTER(TwellHybrid), _vp,
                                         _vp, ctypes.c_size_t, _vp]
@@ -200,6 +202,25 @@ def pack(X, W_g, b_g, T_n: int = 128, K: int = 8, ovf_cap: Optional[int] = None,
         ws = workspace(OP_PACK, M, d, f, T_n, K, st.ovf_cap, X.device)
     _check(lib().twell_pack(_ptr(X), _ptr(W_g), _ptr(b_g), d, ctypes.byref(st.c), _ptr(z), _ptr(ws), ws.numel(),
                             _stream(stream)), "twell_pack")
+    return st, z
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def pack_noalloc(X, W_g, b_g, T_n: int = 128, K: int = 8, ovf_cap: Optional[int] = None, z_debug: bool = False,
+                 state: Optional[HybridState] = None, stream=None):
+    """twell_pack_noalloc: the same result as pack() without a workspace; the
+    library's own fixed scratch is used instead (M * d_ff * 2 bytes at most
+    NOALLOC_SCRATCH_BYTES). Returns (state, z or None)."""
+    for t, n in ((X, "X"), (W_g, "W_g"), (b_g, "b_g")):
+        _bf16(t, n)
+    M, d = X.shape
+    f = W_g.shape[0]
+    st = state or HybridState(M, f, T_n, K, ovf_cap, X.device, with_u=False)
+    z = torch.empty((M, f), dtype=torch.float32, device=X.device) if z_debug else None
+    _check(lib().twell_pack_noalloc(_ptr(X), _ptr(W_g), _ptr(b_g), d, ctypes.byref(st.c), _ptr(z), _stream(stream)),
+           "twell_pack_noalloc")
     return st, z
 
 

@@ -147,6 +147,34 @@ TWELL_API twell_status twell_pack(const uint16_t* X, const uint16_t* W_g, const 
                         twell_stream_t stream);
 
 /*
+ * twell_pack without a workspace argument (the pages have no counterpart; this
+ * is an integration aid). It is meant for callers that may not allocate device
+ * memory: code embedded in a host application whose allocator owns all of the
+ * device memory (a plug-in handed only its inputs and outputs), or a latency-
+ * critical loop where a cudaMalloc, which can synchronise the device, is not
+ * acceptable. It computes exactly what twell_pack computes.
+ *   Scratch: the only scratch twell_pack needs, the dense slices spilled for
+ *   tiles with more than K actives, lives in a file-scope device array of
+ *   TWELL_NOALLOC_SCRATCH_BYTES that the library owns; every device that loads
+ *   the library keeps it until the process exits. Nothing is allocated or
+ *   freed by the call, by the library or by any library it calls.
+ *   Limit: M * d_ff * 2 <= TWELL_NOALLOC_SCRATCH_BYTES (M * d_ff <= 8,388,608);
+ *   larger shapes return TWELL_EWORKSPACE and enqueue nothing.
+ *   Set-up: the first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with the caller's current device, which must be the
+ *   device of `stream`); make that first call before any stream capture.
+ *   Sharing: all calls share the one array and the array keeps whatever the
+ *   last call left in it. A call writes every scratch slice before it reads it,
+ *   so nothing has to start at zero; but calls whose execution overlaps on the
+ *   GPU (for example on two streams) race on the array and must be serialised.
+ */
+#define TWELL_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+TWELL_API twell_status twell_pack_noalloc(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_g,
+                                          int64_t d_model, twell_hybrid* h, float* z_debug,
+                                          twell_stream_t stream);
+
+/*
  * Forward pass of the sparse gated FFN ([aivizor] ¶2: a fused kernel reads the
  * TwELL activations and performs the up and down projections without writing
  * the hidden state to global memory; overflow rows take the dense backup path).
