@@ -206,50 +206,50 @@ __global__ void __launch_bounds__(256) csc_fill_kernel(
 }
 
 // One warp per unit, 8 consecutive units per CTA, one 16-byte chunk (8
-// columns) per lane: a CTA covers a 256-column slice. The unit's list is read
-// 32 entries at a time, one entry per lane in a single coalesced load, and the
-// entries are handed out with shuffles, so the row loads of kWgBatch pairs can
-// be issued back to back without waiting on their indices. dW_d[:, j] is
-// transposed through shared memory so that each output row gets 8 consecutive
-// units (32 bytes).
+// columns) per lane: a CTA covers a 256-column slice. The warp stages its
+// unit's list 32 entries at a time in shared memory (one coalesced load), so
+// the x and dY loads of kWgBatch pairs are issued back to back; entries come
+// from shared-memory broadcasts. Accumulation uses the two-lane FMA. dW_d[:, j]
+// is transposed through shared memory so that each output row gets 8
+// consecutive units (32 bytes).
 constexpr int kWgBatch = 4;
 constexpr int kWgCols = 256;
 
-__global__ void __launch_bounds__(256, 3) wgrad_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ dY,
-                                                    const int* __restrict__ unit_ptr, const int* __restrict__ csc_row,
-                                                    const float4* __restrict__ csc_val, int d, int f,
-                                                    float* __restrict__ dWg, float* __restrict__ dWu,
-                                                    float* __restrict__ dWd, float* __restrict__ dbg) {
+__global__ void __launch_bounds__(256, 3) wgrad_kernel(const uint16_t* __restrict__ X,
+                                                       const uint16_t* __restrict__ dY,
+                                                       const int* __restrict__ unit_ptr,
+                                                       const int* __restrict__ csc_row,
+                                                       const float4* __restrict__ csc_val, int d, int f,
+                                                       float* __restrict__ dWg, float* __restrict__ dWu,
+                                                       float* __restrict__ dWd, float* __restrict__ dbg) {
   __shared__ float s_dwd[kWgCols][9];
+  __shared__ int s_row[8][32];
+  __shared__ float4 s_val[8][32];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = blockIdx.x * 8 + w;
   const int c0 = blockIdx.y * kWgCols;
   const int cidx = (c0 >> 3) + lane;
   const bool cval = cidx < (d >> 3);
-  float au[8], ag[8], ad[8];
+  float2 au[4], ag[4], ad[4];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) au[e] = ag[e] = ad[e] = 0.f;
+  for (int e = 0; e < 4; ++e) au[e] = ag[e] = ad[e] = make_float2(0.f, 0.f);
   float db = 0.f;
   const int p0 = unit_ptr[j], p1 = unit_ptr[j + 1];
   for (int pb = p0; pb < p1; pb += 32) {
     const int n = min(32, p1 - pb);
-    const int my_row = lane < n ? csc_row[pb + lane] : 0;
-    const float4 my_v = lane < n ? csc_val[pb + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
-    db += my_v.z;
+    __syncwarp();
+    if (lane < n) {
+      s_row[w][lane] = csc_row[pb + lane];
+      const float4 v = csc_val[pb + lane];
+      s_val[w][lane] = v;
+      db += v.z;
+    }
+    __syncwarp();
     for (int b0 = 0; b0 < n; b0 += kWgBatch) {
       uint4 xv[kWgBatch], dv[kWgBatch];
-      float ch[kWgBatch], cu[kWgBatch], cz[kWgBatch];
 #pragma unroll
       for (int b = 0; b < kWgBatch; ++b) {
-        const int src = b0 + b < n ? b0 + b : b0;
-        const long r = __shfl_sync(0xFFFFFFFFu, my_row, src);
-        const float h = __shfl_sync(0xFFFFFFFFu, my_v.x, src);
-        const float du = __shfl_sync(0xFFFFFFFFu, my_v.y, src);
-        const float dz = __shfl_sync(0xFFFFFFFFu, my_v.z, src);
-        const bool in = b0 + b < n;
-        ch[b] = in ? h : 0.f;
-        cu[b] = in ? du : 0.f;
-        cz[b] = in ? dz : 0.f;
+        const long r = s_row[w][min(b0 + b, n - 1)];
         if (cval) {
           xv[b] = __ldg(reinterpret_cast<const uint4*>(X + r * d) + cidx);
           dv[b] = __ldg(reinterpret_cast<const uint4*>(dY + r * d) + cidx);
@@ -259,14 +259,16 @@ __global__ void __launch_bounds__(256, 3) wgrad_kernel(const uint16_t* __restric
       }
 #pragma unroll
       for (int b = 0; b < kWgBatch; ++b) {
-        float xf[8], df[8];
-        unpack8(xv[b], xf);
-        unpack8(dv[b], df);
+        const float4 v = b0 + b < n ? s_val[w][b0 + b] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float2 h2 = make_float2(v.x, v.x), u2 = make_float2(v.y, v.y), z2 = make_float2(v.z, v.z);
+        const uint32_t xw[4] = {xv[b].x, xv[b].y, xv[b].z, xv[b].w};
+        const uint32_t dw[4] = {dv[b].x, dv[b].y, dv[b].z, dv[b].w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          au[e] = fmaf(cu[b], xf[e], au[e]);
-          ag[e] = fmaf(cz[b], xf[e], ag[e]);
-          ad[e] = fmaf(ch[b], df[e], ad[e]);
+        for (int e = 0; e < 4; ++e) {
+          const float2 xf = bf16x2_to_f2(xw[e]);
+          au[e] = fma2(u2, xf, au[e]);
+          ag[e] = fma2(z2, xf, ag[e]);
+          ad[e] = fma2(h2, bf16x2_to_f2(dw[e]), ad[e]);
         }
       }
     }
@@ -275,13 +277,16 @@ __global__ void __launch_bounds__(256, 3) wgrad_kernel(const uint16_t* __restric
   if (cval) {
     float4* pu = reinterpret_cast<float4*>(dWu + static_cast<long>(j) * d) + 2 * cidx;
     float4* pg = reinterpret_cast<float4*>(dWg + static_cast<long>(j) * d) + 2 * cidx;
-    pu[0] = make_float4(au[0], au[1], au[2], au[3]);
-    pu[1] = make_float4(au[4], au[5], au[6], au[7]);
-    pg[0] = make_float4(ag[0], ag[1], ag[2], ag[3]);
-    pg[1] = make_float4(ag[4], ag[5], ag[6], ag[7]);
+    pu[0] = make_float4(au[0].x, au[0].y, au[1].x, au[1].y);
+    pu[1] = make_float4(au[2].x, au[2].y, au[3].x, au[3].y);
+    pg[0] = make_float4(ag[0].x, ag[0].y, ag[1].x, ag[1].y);
+    pg[1] = make_float4(ag[2].x, ag[2].y, ag[3].x, ag[3].y);
   }
 #pragma unroll
-  for (int e = 0; e < 8; ++e) s_dwd[lane * 8 + e][w] = ad[e];
+  for (int e = 0; e < 4; ++e) {
+    s_dwd[lane * 8 + 2 * e][w] = ad[e].x;
+    s_dwd[lane * 8 + 2 * e + 1][w] = ad[e].y;
+  }
   if (blockIdx.y == 0 && lane == 0 && dbg != nullptr) dbg[j] = db;
   __syncthreads();
   const int cc = c0 + threadIdx.x;

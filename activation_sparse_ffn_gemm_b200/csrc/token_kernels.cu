@@ -20,7 +20,10 @@
 //     fp32), so a unit's row is one C-deep burst of coalesced loads per lane;
 //   * units are processed B at a time (all B*C loads issued before any use);
 //   * no CTA-wide barrier: a single-warp group synchronises with __syncwarp,
-//     wider groups with a named barrier of their own.
+//     wider groups with a named barrier of their own;
+//   * token rows are handed out dynamically (an atomic counter per launch),
+//     so groups that finish early take more rows and no CTA waits on a slow
+//     neighbour.
 // Overflow rows are skipped (the dense backup path owns them).
 #include "trace.cuh"
 #include "twell_internal.cuh"
@@ -29,12 +32,13 @@ namespace twell {
 
 namespace {
 
-constexpr int kTokWarps = 8;   // warps per CTA
+constexpr int kTokWarps = 4;   // warps per CTA (more when one token needs more)
 constexpr int kListCap = 256;  // list entries per chunk and group
 
 template <int C, int W>
 struct TokCfg {
-  static constexpr int G = kTokWarps / W;  // token groups per CTA
+  static constexpr int WARPS = W > kTokWarps ? W : kTokWarps;  // warps per CTA
+  static constexpr int G = WARPS / W;                           // token groups per CTA
   static constexpr int B = C >= 8 ? 2 : (C >= 4 ? 4 : 8);
   static constexpr int GT = W * 32;        // threads per group
 };
@@ -97,43 +101,58 @@ __device__ __forceinline__ void entry_of(const int* off, int T, int e, int& t, i
   sl = e - off[lo];
 }
 
-// dot of C packed-bf16 chunks (register operand) with C chunks of a row.
+// dot of C packed-bf16 chunks (register operand) with C chunks of a row, in
+// four independent two-lane accumulators (no dependent FMA chain).
 template <int C>
 __device__ __forceinline__ float dot_chunks(const uint4 (&a)[C], const uint4 (&w)[C]) {
-  float s = 0.f;
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
   for (int c = 0; c < C; ++c) {
     const uint32_t av[4] = {a[c].x, a[c].y, a[c].z, a[c].w};
     const uint32_t wv[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      s = fmaf(bf16_lo(av[e]), bf16_lo(wv[e]), s);
-      s = fmaf(bf16_hi(av[e]), bf16_hi(wv[e]), s);
-    }
+    for (int e = 0; e < 4; ++e) acc[e] = fma2(bf16x2_to_f2(av[e]), bf16x2_to_f2(wv[e]), acc[e]);
   }
-  return s;
+  return ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
 }
 
+// y += a * w over C chunks; y is held as pairs for the two-lane FMA.
 template <int C>
-__device__ __forceinline__ void axpy_chunks(float a, const uint4 (&w)[C], float (&y)[C][8]) {
+__device__ __forceinline__ void axpy_chunks(float a, const uint4 (&w)[C], float2 (&y)[C][4]) {
+  const float2 a2 = make_float2(a, a);
 #pragma unroll
   for (int c = 0; c < C; ++c) {
-    float f[8];
-    unpack8(w[c], f);
+    const uint32_t wv[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
 #pragma unroll
-    for (int e = 0; e < 8; ++e) y[c][e] = fmaf(a, f[e], y[c][e]);
+    for (int e = 0; e < 4; ++e) y[c][e] = fma2(a2, bf16x2_to_f2(wv[e]), y[c][e]);
   }
 }
 
-// Chunk q of this lane: index (wi*32 + lane) + W*32*q into the row's d/8 chunks.
-template <int C, int W>
+// Chunk q of this lane: index (wi*32 + lane) + W*32*q into the row's d/8
+// chunks. EXACT: the row is exactly W*32*C chunks long, no bounds test needed.
+template <int C, int W, bool EXACT>
 __device__ __forceinline__ void load_row(const uint16_t* __restrict__ base, int first, int nch, uint4 (&v)[C]) {
   const uint4* p = reinterpret_cast<const uint4*>(base);
 #pragma unroll
   for (int q = 0; q < C; ++q) {
     const int idx = first + W * 32 * q;
-    v[q] = idx < nch ? __ldg(p + idx) : make_uint4(0, 0, 0, 0);
+    v[q] = (EXACT || idx < nch) ? __ldg(p + idx) : make_uint4(0, 0, 0, 0);
   }
+}
+
+// Next token row for the group (W warps): claimed by one lane, shared by all.
+template <int W>
+__device__ __forceinline__ long next_row(int* ctr, int grp, int wi, int lane, int* s_row) {
+  int r = 0;
+  if (W == 1) {
+    if (lane == 0) r = atomicAdd(ctr, 1);
+    return __shfl_sync(0xFFFFFFFFu, r, 0);
+  }
+  if (wi == 0 && lane == 0) s_row[grp] = atomicAdd(ctr, 1);
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(W * 32) : "memory");
+  r = s_row[grp];
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(W * 32) : "memory");
+  return r;
 }
 
 // Phases of one list chunk [e0, e0 + ne) of a token row, shared by the two
@@ -156,14 +175,15 @@ __device__ __forceinline__ void build_list(GroupSmem& g, long row, int T, int K,
 // Dot products of a register-resident row (xp) with the gathered rows Wr[j] of
 // the listed units; the full dots land in out[e] (W == 1) or as per-warp
 // partials in part[wi][e] (W > 1).
-template <int C, int W, int B>
+template <int C, int W, int B, bool EXACT>
 __device__ __forceinline__ void gather_dots(const GroupSmem& g, int ne, const uint4 (&xp)[C],
                                             const uint16_t* __restrict__ Wr, int d, int first, int nch, int lane,
                                             float* out, float* part_w) {
   for (int k = 0; k < ne; k += B) {
     uint4 wv[B][C];
 #pragma unroll
-    for (int q = 0; q < B; ++q) load_row<C, W>(Wr + static_cast<long>(g.j[min(k + q, ne - 1)]) * d, first, nch, wv[q]);
+    for (int q = 0; q < B; ++q)
+      load_row<C, W, EXACT>(Wr + static_cast<long>(g.j[min(k + q, ne - 1)]) * d, first, nch, wv[q]);
 #pragma unroll
     for (int q = 0; q < B; ++q) {
       const float s = warp_sum(dot_chunks<C>(xp, wv[q]));
@@ -173,10 +193,10 @@ __device__ __forceinline__ void gather_dots(const GroupSmem& g, int ne, const ui
 }
 
 // y += sum over listed units of coef[e] * Wr[j_e].
-template <int C, int W, int B>
+template <int C, int W, int B, bool EXACT>
 __device__ __forceinline__ void gather_axpy(const GroupSmem& g, int ne, const float* coef,
                                             const uint16_t* __restrict__ Wr, int d, int first, int nch,
-                                            float (&y)[C][8]) {
+                                            float2 (&y)[C][4]) {
   for (int k = 0; k < ne; k += B) {
     uint4 wv[B][C];
     float h[B];
@@ -184,7 +204,7 @@ __device__ __forceinline__ void gather_axpy(const GroupSmem& g, int ne, const fl
     for (int q = 0; q < B; ++q) {
       const bool in = k + q < ne;
       h[q] = in ? coef[k + q] : 0.f;
-      load_row<C, W>(Wr + static_cast<long>(g.j[in ? k + q : k]) * d, first, nch, wv[q]);
+      load_row<C, W, EXACT>(Wr + static_cast<long>(g.j[in ? k + q : k]) * d, first, nch, wv[q]);
     }
 #pragma unroll
     for (int q = 0; q < B; ++q) axpy_chunks<C>(h[q], wv[q], y);
@@ -192,27 +212,28 @@ __device__ __forceinline__ void gather_axpy(const GroupSmem& g, int ne, const fl
 }
 
 template <int C>
-__device__ __forceinline__ void zero_acc(float (&y)[C][8]) {
+__device__ __forceinline__ void zero_acc(float2 (&y)[C][4]) {
 #pragma unroll
   for (int q = 0; q < C; ++q)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) y[q][e] = 0.f;
+    for (int e = 0; e < 4; ++e) y[q][e] = make_float2(0.f, 0.f);
 }
 
 // LONG = false: rows whose kept entries fit one list (the common case): the
 // row operand (x or dY) and the accumulators (Y or dX) are never live together,
 // which keeps these kernels at two CTAs per SM. LONG = true: the rare rows with
 // more entries, processed in list chunks with the accumulators kept live.
-template <int C, int W, bool LONG>
-__global__ void __launch_bounds__(kTokWarps * 32, LONG ? 1 : 2) ell_fwd_kernel(
+template <int C, int W, bool LONG, bool EXACT>
+__global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, LONG ? 1 : 512 / (TokCfg<C, W>::WARPS * 32)) ell_fwd_kernel(
     const uint16_t* __restrict__ X, const uint16_t* __restrict__ Wu, const uint16_t* __restrict__ Wdt,
     const uint16_t* __restrict__ count, const uint16_t* __restrict__ val, const uint8_t* __restrict__ col,
     const uint8_t* __restrict__ row_ovf, float* __restrict__ u_ell, uint16_t* __restrict__ Y, int M, int d, int T,
-    int K) {
+    int K, int* __restrict__ ctr) {
   using Cfg = TokCfg<C, W>;
   constexpr int B = Cfg::B;
   __shared__ GroupSmem gs[Cfg::G];
   __shared__ float part[Cfg::G][W > 1 ? W : 1][kListCap];
+  __shared__ int s_next[Cfg::G];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = warp / W, wi = warp % W, gtid = wi * 32 + lane;
   GroupSmem& g = gs[grp];
@@ -223,8 +244,8 @@ __global__ void __launch_bounds__(kTokWarps * 32, LONG ? 1 : 2) ell_fwd_kernel(
   auto up = [&](long row, int ne) {
     {
       uint4 xp[C];
-      load_row<C, W>(X + row * d, first, nch, xp);
-      gather_dots<C, W, B>(g, ne, xp, Wu, d, first, nch, lane, g.c2, part[grp][wi]);
+      load_row<C, W, EXACT>(X + row * d, first, nch, xp);
+      gather_dots<C, W, B, EXACT>(g, ne, xp, Wu, d, first, nch, lane, g.c2, part[grp][wi]);
     }
     group_sync<W>(grp);
     for (int e = gtid; e < ne; e += Cfg::GT) {
@@ -239,18 +260,20 @@ __global__ void __launch_bounds__(kTokWarps * 32, LONG ? 1 : 2) ell_fwd_kernel(
     }
     group_sync<W>(grp);
   };
-  auto store = [&](long row, const float (&y)[C][8]) {
+  auto store = [&](long row, const float2 (&y)[C][4]) {
     uint4* yr = reinterpret_cast<uint4*>(Y + row * d);
 #pragma unroll
     for (int q = 0; q < C; ++q) {
       const int idx = first + W * 32 * q;
       if (idx < nch)
-        yr[idx] = make_uint4(pack_bf16x2(y[q][0], y[q][1]), pack_bf16x2(y[q][2], y[q][3]),
-                             pack_bf16x2(y[q][4], y[q][5]), pack_bf16x2(y[q][6], y[q][7]));
+        yr[idx] = make_uint4(pack_bf16x2(y[q][0].x, y[q][0].y), pack_bf16x2(y[q][1].x, y[q][1].y),
+                             pack_bf16x2(y[q][2].x, y[q][2].y), pack_bf16x2(y[q][3].x, y[q][3].y));
     }
   };
 
-  for (long row = static_cast<long>(blockIdx.x) * Cfg::G + grp; row < M; row += static_cast<long>(gridDim.x) * Cfg::G) {
+  for (;;) {
+    const long row = next_row<W>(ctr, grp, wi, lane, s_next);
+    if (row >= M) break;
     if (row_ovf[row]) continue;
     if (wi == 0) row_offsets(count, row, T, K, lane, g);
     group_sync<W>(grp);
@@ -260,19 +283,19 @@ __global__ void __launch_bounds__(kTokWarps * 32, LONG ? 1 : 2) ell_fwd_kernel(
         build_list(g, row, T, K, 0, total, gtid, Cfg::GT, val, col, nullptr);
         group_sync<W>(grp);
         up(row, total);
-        float y[C][8];
+        float2 y[C][4];
         zero_acc<C>(y);
-        gather_axpy<C, W, B>(g, total, g.c, Wdt, d, first, nch, y);
+        gather_axpy<C, W, B, EXACT>(g, total, g.c, Wdt, d, first, nch, y);
         store(row, y);
       } else {
-        float y[C][8];
+        float2 y[C][4];
         zero_acc<C>(y);
         for (int e0 = 0; e0 < total; e0 += kListCap) {
           const int ne = min(kListCap, total - e0);
           build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, nullptr);
           group_sync<W>(grp);
           up(row, ne);
-          gather_axpy<C, W, B>(g, ne, g.c, Wdt, d, first, nch, y);
+          gather_axpy<C, W, B, EXACT>(g, ne, g.c, Wdt, d, first, nch, y);
           group_sync<W>(grp);
         }
         store(row, y);
@@ -282,19 +305,20 @@ __global__ void __launch_bounds__(kTokWarps * 32, LONG ? 1 : 2) ell_fwd_kernel(
   }
 }
 
-template <int C, int W, bool LONG>
-__global__ void __launch_bounds__(kTokWarps * 32, LONG ? 1 : 2) ell_bwd_kernel(
+template <int C, int W, bool LONG, bool EXACT>
+__global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, LONG ? 1 : 512 / (TokCfg<C, W>::WARPS * 32)) ell_bwd_kernel(
     const uint16_t* __restrict__ dY, const uint16_t* __restrict__ Wu, const uint16_t* __restrict__ Wg,
     const uint16_t* __restrict__ Wdt, const uint16_t* __restrict__ count, const uint16_t* __restrict__ val,
     const uint8_t* __restrict__ col, const uint8_t* __restrict__ row_ovf, const float* __restrict__ u_ell,
     float lambda, float* __restrict__ du_ell, float* __restrict__ dz_ell, float* __restrict__ dX, int M, int d,
-    int T, int K) {
+    int T, int K, int* __restrict__ ctr) {
   using Cfg = TokCfg<C, W>;
   constexpr int B = Cfg::B;
   constexpr int B2 = B > 1 ? B / 2 : 1;  // two rows (W_u, W_g) per unit in the dX phase
   __shared__ GroupSmem gs[Cfg::G];
   __shared__ float part[Cfg::G][W > 1 ? W : 1][kListCap];
   __shared__ float dhv[Cfg::G][kListCap];
+  __shared__ int s_next[Cfg::G];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = warp / W, wi = warp % W, gtid = wi * 32 + lane;
   GroupSmem& g = gs[grp];
@@ -305,8 +329,8 @@ __global__ void __launch_bounds__(kTokWarps * 32, LONG ? 1 : 2) ell_bwd_kernel(
   auto dh_phase = [&](long row, int ne) {
     {
       uint4 dyp[C];
-      load_row<C, W>(dY + row * d, first, nch, dyp);
-      gather_dots<C, W, B>(g, ne, dyp, Wdt, d, first, nch, lane, dhv[grp], part[grp][wi]);
+      load_row<C, W, EXACT>(dY + row * d, first, nch, dyp);
+      gather_dots<C, W, B, EXACT>(g, ne, dyp, Wdt, d, first, nch, lane, dhv[grp], part[grp][wi]);
     }
     group_sync<W>(grp);
     for (int e = gtid; e < ne; e += Cfg::GT) {
@@ -325,23 +349,25 @@ __global__ void __launch_bounds__(kTokWarps * 32, LONG ? 1 : 2) ell_bwd_kernel(
     }
     group_sync<W>(grp);
   };
-  auto dx_phase = [&](int ne, float (&dx)[C][8]) {
-    gather_axpy<C, W, B2>(g, ne, g.c, Wu, d, first, nch, dx);
-    gather_axpy<C, W, B2>(g, ne, g.c2, Wg, d, first, nch, dx);
+  auto dx_phase = [&](int ne, float2 (&dx)[C][4]) {
+    gather_axpy<C, W, B2, EXACT>(g, ne, g.c, Wu, d, first, nch, dx);
+    gather_axpy<C, W, B2, EXACT>(g, ne, g.c2, Wg, d, first, nch, dx);
   };
-  auto store = [&](long row, const float (&dx)[C][8]) {
+  auto store = [&](long row, const float2 (&dx)[C][4]) {
     float4* xr = reinterpret_cast<float4*>(dX + row * d);
 #pragma unroll
     for (int q = 0; q < C; ++q) {
       const int idx = first + W * 32 * q;
       if (idx < nch) {
-        xr[2 * idx] = make_float4(dx[q][0], dx[q][1], dx[q][2], dx[q][3]);
-        xr[2 * idx + 1] = make_float4(dx[q][4], dx[q][5], dx[q][6], dx[q][7]);
+        xr[2 * idx] = make_float4(dx[q][0].x, dx[q][0].y, dx[q][1].x, dx[q][1].y);
+        xr[2 * idx + 1] = make_float4(dx[q][2].x, dx[q][2].y, dx[q][3].x, dx[q][3].y);
       }
     }
   };
 
-  for (long row = static_cast<long>(blockIdx.x) * Cfg::G + grp; row < M; row += static_cast<long>(gridDim.x) * Cfg::G) {
+  for (;;) {
+    const long row = next_row<W>(ctr, grp, wi, lane, s_next);
+    if (row >= M) break;
     if (row_ovf[row]) continue;
     if (wi == 0) row_offsets(count, row, T, K, lane, g);
     group_sync<W>(grp);
@@ -351,12 +377,12 @@ __global__ void __launch_bounds__(kTokWarps * 32, LONG ? 1 : 2) ell_bwd_kernel(
         build_list(g, row, T, K, 0, total, gtid, Cfg::GT, val, col, u_ell);
         group_sync<W>(grp);
         dh_phase(row, total);
-        float dx[C][8];
+        float2 dx[C][4];
         zero_acc<C>(dx);
         dx_phase(total, dx);
         store(row, dx);
       } else {
-        float dx[C][8];
+        float2 dx[C][4];
         zero_acc<C>(dx);
         for (int e0 = 0; e0 < total; e0 += kListCap) {
           const int ne = min(kListCap, total - e0);
@@ -387,24 +413,27 @@ void tok_shape(int d, int& C, int& W) {
 
 int tok_grid(int M, int G) {
   const long need = (static_cast<long>(M) + G - 1) / G;
-  const long cap = static_cast<long>(device_sm_count()) * 8;
+  const long cap = static_cast<long>(device_sm_count()) * 4;  // about the resident CTAs; rows are claimed dynamically
   return static_cast<int>(need < cap ? need : cap);
 }
 
 // Rows whose kept entries exceed one list are rare; the second pass only reads
-// the per-tile counts of the rows it skips.
-template <int C, int W, typename... A>
-void launch_fwd_cw(int M, cudaStream_t s, A... a) {
+// the per-tile counts of the rows it skips. ctr[0], ctr[1]: the row counters
+// of the two passes (zero on entry).
+template <int C, int W, bool EXACT, typename... A>
+void launch_fwd_cw(int M, int* ctr, cudaStream_t s, A... a) {
   const int grid = tok_grid(M, TokCfg<C, W>::G);
-  TWELL_LAUNCH("ell_updown", s, ell_fwd_kernel<C, W, false><<<grid, kTokWarps * 32, 0, s>>>(a...));
-  TWELL_LAUNCH("ell_updown_long", s, ell_fwd_kernel<C, W, true><<<grid, kTokWarps * 32, 0, s>>>(a...));
+  constexpr int threads = TokCfg<C, W>::WARPS * 32;
+  TWELL_LAUNCH("ell_updown", s, ell_fwd_kernel<C, W, false, EXACT><<<grid, threads, 0, s>>>(a..., ctr));
+  TWELL_LAUNCH("ell_updown_long", s, ell_fwd_kernel<C, W, true, EXACT><<<grid, threads, 0, s>>>(a..., ctr + 1));
 }
 
-template <int C, int W, typename... A>
-void launch_bwd_cw(int M, cudaStream_t s, A... a) {
+template <int C, int W, bool EXACT, typename... A>
+void launch_bwd_cw(int M, int* ctr, cudaStream_t s, A... a) {
   const int grid = tok_grid(M, TokCfg<C, W>::G);
-  TWELL_LAUNCH("ell_bwd", s, ell_bwd_kernel<C, W, false><<<grid, kTokWarps * 32, 0, s>>>(a...));
-  TWELL_LAUNCH("ell_bwd_long", s, ell_bwd_kernel<C, W, true><<<grid, kTokWarps * 32, 0, s>>>(a...));
+  constexpr int threads = TokCfg<C, W>::WARPS * 32;
+  TWELL_LAUNCH("ell_bwd", s, ell_bwd_kernel<C, W, false, EXACT><<<grid, threads, 0, s>>>(a..., ctr));
+  TWELL_LAUNCH("ell_bwd_long", s, ell_bwd_kernel<C, W, true, EXACT><<<grid, threads, 0, s>>>(a..., ctr + 1));
 }
 
 }  // namespace
@@ -412,12 +441,17 @@ void launch_bwd_cw(int M, cudaStream_t s, A... a) {
 cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
                                const uint16_t* count, const uint16_t* val, const uint8_t* col,
                                const uint8_t* row_ovf, float* u_ell, uint16_t* Y, int M, int d, int f, int K,
-                               cudaStream_t s) {
+                               int* ctr, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
+  cudaError_t e = cudaMemsetAsync(ctr, 0, 2 * sizeof(int), s);
+  if (e != cudaSuccess) return e;
   int C, W;
   tok_shape(d, C, W);
   const int T = f / kTn;
-#define TWELL_FWD(CC, WW) launch_fwd_cw<CC, WW>(M, s, X, W_u, W_dt, count, val, col, row_ovf, u_ell, Y, M, d, T, K)
+  const bool exact = d / 8 == W * 32 * C;
+#define TWELL_FWD(CC, WW)                                                                                   \
+  (exact ? launch_fwd_cw<CC, WW, true>(M, ctr, s, X, W_u, W_dt, count, val, col, row_ovf, u_ell, Y, M, d, T, K) \
+         : launch_fwd_cw<CC, WW, false>(M, ctr, s, X, W_u, W_dt, count, val, col, row_ovf, u_ell, Y, M, d, T, K))
   if (W == 1 && C == 1) TWELL_FWD(1, 1);
   else if (W == 1 && C == 2) TWELL_FWD(2, 1);
   else if (W == 1 && C == 4) TWELL_FWD(4, 1);
@@ -432,15 +466,20 @@ cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uin
 cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const uint16_t* W_g,
                                const uint16_t* W_dt, const uint16_t* count, const uint16_t* val,
                                const uint8_t* col, const uint8_t* row_ovf, const float* u_ell, float lambda,
-                               float* du_ell, float* dz_ell, float* dX, int M, int d, int f, int K,
+                               float* du_ell, float* dz_ell, float* dX, int M, int d, int f, int K, int* ctr,
                                cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
+  cudaError_t e = cudaMemsetAsync(ctr, 0, 2 * sizeof(int), s);
+  if (e != cudaSuccess) return e;
   int C, W;
   tok_shape(d, C, W);
   const int T = f / kTn;
-#define TWELL_BWD(CC, WW)                                                                                      \
-  launch_bwd_cw<CC, WW>(M, s, dY, W_u, W_g, W_dt, count, val, col, row_ovf, u_ell, lambda, du_ell, dz_ell, dX, \
-                        M, d, T, K)
+  const bool exact = d / 8 == W * 32 * C;
+#define TWELL_BWD(CC, WW)                                                                                        \
+  (exact ? launch_bwd_cw<CC, WW, true>(M, ctr, s, dY, W_u, W_g, W_dt, count, val, col, row_ovf, u_ell, lambda,    \
+                                       du_ell, dz_ell, dX, M, d, T, K)                                          \
+         : launch_bwd_cw<CC, WW, false>(M, ctr, s, dY, W_u, W_g, W_dt, count, val, col, row_ovf, u_ell, lambda,   \
+                                        du_ell, dz_ell, dX, M, d, T, K))
   if (W == 1 && C == 1) TWELL_BWD(1, 1);
   else if (W == 1 && C == 2) TWELL_BWD(2, 1);
   else if (W == 1 && C == 4) TWELL_BWD(4, 1);

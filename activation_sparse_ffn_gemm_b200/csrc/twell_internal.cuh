@@ -34,6 +34,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return static_cast<uint32_t>(f32_to_bf16_bits(lo)) | (static_cast<uint32_t>(f32_to_bf16_bits(hi)) << 16);
 }
 
+// Packed two-lane fp32 arithmetic (sm_100 executes one instruction per pair).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(reinterpret_cast<unsigned long long&>(d))
+      : "l"(reinterpret_cast<const unsigned long long&>(a)), "l"(reinterpret_cast<const unsigned long long&>(b)),
+        "l"(reinterpret_cast<const unsigned long long&>(c)));
+  return d;
+}
+
+// bf16x2 word -> (low, high) as fp32.
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
 // Eight bf16 (one uint4) -> eight floats.
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
   f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x);
@@ -81,10 +96,11 @@ cudaError_t launch_gather_rows(const uint16_t* in, const int* rows, const int* n
 cudaError_t launch_transpose_bf16(const uint16_t* in, int rows, int cols, uint16_t* out, cudaStream_t s);
 
 // Fused sparse up + down over the ELL rows (overflow rows are skipped).
+// ctr: two ints of device scratch (row counters), zeroed by the launcher.
 cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
                                const uint16_t* count, const uint16_t* val, const uint8_t* col,
                                const uint8_t* row_ovf, float* u_ell, uint16_t* Y, int M, int d, int f, int K,
-                               cudaStream_t s);
+                               int* ctr, cudaStream_t s);
 
 // Dense backup forward for overflow rows: H = bf16(G * (X_ovf W_u^T)) then
 // Y[ovf_rows] = bf16(H W_d^T).
@@ -97,7 +113,7 @@ cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uin
 cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const uint16_t* W_g,
                                const uint16_t* W_dt, const uint16_t* count, const uint16_t* val,
                                const uint8_t* col, const uint8_t* row_ovf, const float* u_ell, float lambda,
-                               float* du_ell, float* dz_ell, float* dX, int M, int d, int f, int K,
+                               float* du_ell, float* dz_ell, float* dX, int M, int d, int f, int K, int* ctr,
                                cudaStream_t s);
 
 // Dense backup backward for overflow rows: dU, dZ (fp32, and bf16 [dU | dZ] as
