@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, LONG ? 1 : 512 / (To
     const uint16_t* __restrict__ X, const uint16_t* __restrict__ Wu, const uint16_t* __restrict__ Wdt,
     const uint16_t* __restrict__ count, const uint16_t* __restrict__ val, const uint8_t* __restrict__ col,
     const uint8_t* __restrict__ row_ovf, float* __restrict__ u_ell, uint16_t* __restrict__ Y, int M, int d, int T,
-    int K, int* __restrict__ ctr) {
+    int K, int* __restrict__ ctr, int* __restrict__ long_rows) {
   using Cfg = TokCfg<C, W>;
   constexpr int B = Cfg::B;
   __shared__ GroupSmem gs[Cfg::G];
@@ -271,13 +271,22 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, LONG ? 1 : 512 / (To
     }
   };
 
+  // short pass: rows 0..M-1 in claim order; rows too long for one list are
+  // appended to long_rows (count in ctr[2]) for the long pass, which walks
+  // that list only.
   for (;;) {
-    const long row = next_row<W>(ctr, grp, wi, lane, s_next);
-    if (row >= M) break;
-    if (row_ovf[row]) continue;
+    long row = next_row<W>(LONG ? ctr + 1 : ctr, grp, wi, lane, s_next);
+    if (LONG) {
+      if (row >= ctr[2]) break;
+      row = long_rows[row];
+    } else {
+      if (row >= M) break;
+      if (row_ovf[row]) continue;
+    }
     if (wi == 0) row_offsets(count, row, T, K, lane, g);
     group_sync<W>(grp);
     const int total = g.tot;
+    if (!LONG && total > kListCap && wi == 0 && lane == 0) long_rows[atomicAdd(ctr + 2, 1)] = static_cast<int>(row);
     if ((total > kListCap) == LONG) {
       if constexpr (!LONG) {
         build_list(g, row, T, K, 0, total, gtid, Cfg::GT, val, col, nullptr);
@@ -311,7 +320,7 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, LONG ? 1 : 512 / (To
     const uint16_t* __restrict__ Wdt, const uint16_t* __restrict__ count, const uint16_t* __restrict__ val,
     const uint8_t* __restrict__ col, const uint8_t* __restrict__ row_ovf, const float* __restrict__ u_ell,
     float lambda, float* __restrict__ du_ell, float* __restrict__ dz_ell, float* __restrict__ dX, int M, int d,
-    int T, int K, int* __restrict__ ctr) {
+    int T, int K, int* __restrict__ ctr, int* __restrict__ long_rows) {
   using Cfg = TokCfg<C, W>;
   constexpr int B = Cfg::B;
   constexpr int B2 = B > 1 ? B / 2 : 1;  // two rows (W_u, W_g) per unit in the dX phase
@@ -365,13 +374,22 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, LONG ? 1 : 512 / (To
     }
   };
 
+  // short pass: rows 0..M-1 in claim order; rows too long for one list are
+  // appended to long_rows (count in ctr[2]) for the long pass, which walks
+  // that list only.
   for (;;) {
-    const long row = next_row<W>(ctr, grp, wi, lane, s_next);
-    if (row >= M) break;
-    if (row_ovf[row]) continue;
+    long row = next_row<W>(LONG ? ctr + 1 : ctr, grp, wi, lane, s_next);
+    if (LONG) {
+      if (row >= ctr[2]) break;
+      row = long_rows[row];
+    } else {
+      if (row >= M) break;
+      if (row_ovf[row]) continue;
+    }
     if (wi == 0) row_offsets(count, row, T, K, lane, g);
     group_sync<W>(grp);
     const int total = g.tot;
+    if (!LONG && total > kListCap && wi == 0 && lane == 0) long_rows[atomicAdd(ctr + 2, 1)] = static_cast<int>(row);
     if ((total > kListCap) == LONG) {
       if constexpr (!LONG) {
         build_list(g, row, T, K, 0, total, gtid, Cfg::GT, val, col, u_ell);
@@ -417,23 +435,25 @@ int tok_grid(int M, int G) {
   return static_cast<int>(need < cap ? need : cap);
 }
 
-// Rows whose kept entries exceed one list are rare; the second pass only reads
-// the per-tile counts of the rows it skips. ctr[0], ctr[1]: the row counters
-// of the two passes (zero on entry).
+// Rows whose kept entries exceed one list are rare; the short pass lists them
+// and the long pass takes only those. ctr[0], ctr[1]: row counters of the two
+// passes; ctr[2]: number of listed long rows (all zero on entry).
 template <int C, int W, bool EXACT, typename... A>
-void launch_fwd_cw(int M, int* ctr, cudaStream_t s, A... a) {
-  const int grid = tok_grid(M, TokCfg<C, W>::G);
+void launch_fwd_cw(int M, int* ctr, int* long_rows, cudaStream_t s, A... a) {
   constexpr int threads = TokCfg<C, W>::WARPS * 32;
-  TWELL_LAUNCH("ell_updown", s, ell_fwd_kernel<C, W, false, EXACT><<<grid, threads, 0, s>>>(a..., ctr));
-  TWELL_LAUNCH("ell_updown_long", s, ell_fwd_kernel<C, W, true, EXACT><<<grid, threads, 0, s>>>(a..., ctr + 1));
+  TWELL_LAUNCH("ell_updown", s,
+               ell_fwd_kernel<C, W, false, EXACT><<<tok_grid(M, TokCfg<C, W>::G), threads, 0, s>>>(a..., ctr, long_rows));
+  TWELL_LAUNCH("ell_updown_long", s,
+               ell_fwd_kernel<C, W, true, EXACT><<<device_sm_count(), threads, 0, s>>>(a..., ctr, long_rows));
 }
 
 template <int C, int W, bool EXACT, typename... A>
-void launch_bwd_cw(int M, int* ctr, cudaStream_t s, A... a) {
-  const int grid = tok_grid(M, TokCfg<C, W>::G);
+void launch_bwd_cw(int M, int* ctr, int* long_rows, cudaStream_t s, A... a) {
   constexpr int threads = TokCfg<C, W>::WARPS * 32;
-  TWELL_LAUNCH("ell_bwd", s, ell_bwd_kernel<C, W, false, EXACT><<<grid, threads, 0, s>>>(a..., ctr));
-  TWELL_LAUNCH("ell_bwd_long", s, ell_bwd_kernel<C, W, true, EXACT><<<grid, threads, 0, s>>>(a..., ctr + 1));
+  TWELL_LAUNCH("ell_bwd", s,
+               ell_bwd_kernel<C, W, false, EXACT><<<tok_grid(M, TokCfg<C, W>::G), threads, 0, s>>>(a..., ctr, long_rows));
+  TWELL_LAUNCH("ell_bwd_long", s,
+               ell_bwd_kernel<C, W, true, EXACT><<<device_sm_count(), threads, 0, s>>>(a..., ctr, long_rows));
 }
 
 }  // namespace
@@ -441,17 +461,19 @@ void launch_bwd_cw(int M, int* ctr, cudaStream_t s, A... a) {
 cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
                                const uint16_t* count, const uint16_t* val, const uint8_t* col,
                                const uint8_t* row_ovf, float* u_ell, uint16_t* Y, int M, int d, int f, int K,
-                               int* ctr, cudaStream_t s) {
+                               int* ctr, int* long_rows, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
-  cudaError_t e = cudaMemsetAsync(ctr, 0, 2 * sizeof(int), s);
+  cudaError_t e = cudaMemsetAsync(ctr, 0, 3 * sizeof(int), s);
   if (e != cudaSuccess) return e;
   int C, W;
   tok_shape(d, C, W);
   const int T = f / kTn;
   const bool exact = d / 8 == W * 32 * C;
 #define TWELL_FWD(CC, WW)                                                                                   \
-  (exact ? launch_fwd_cw<CC, WW, true>(M, ctr, s, X, W_u, W_dt, count, val, col, row_ovf, u_ell, Y, M, d, T, K) \
-         : launch_fwd_cw<CC, WW, false>(M, ctr, s, X, W_u, W_dt, count, val, col, row_ovf, u_ell, Y, M, d, T, K))
+  (exact ? launch_fwd_cw<CC, WW, true>(M, ctr, long_rows, s, X, W_u, W_dt, count, val, col, row_ovf, u_ell, Y, M, d, \
+                                       T, K)                                                                    \
+         : launch_fwd_cw<CC, WW, false>(M, ctr, long_rows, s, X, W_u, W_dt, count, val, col, row_ovf, u_ell, Y, M, \
+                                        d, T, K))
   if (W == 1 && C == 1) TWELL_FWD(1, 1);
   else if (W == 1 && C == 2) TWELL_FWD(2, 1);
   else if (W == 1 && C == 4) TWELL_FWD(4, 1);
@@ -467,18 +489,18 @@ cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const ui
                                const uint16_t* W_dt, const uint16_t* count, const uint16_t* val,
                                const uint8_t* col, const uint8_t* row_ovf, const float* u_ell, float lambda,
                                float* du_ell, float* dz_ell, float* dX, int M, int d, int f, int K, int* ctr,
-                               cudaStream_t s) {
+                               int* long_rows, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
-  cudaError_t e = cudaMemsetAsync(ctr, 0, 2 * sizeof(int), s);
+  cudaError_t e = cudaMemsetAsync(ctr, 0, 3 * sizeof(int), s);
   if (e != cudaSuccess) return e;
   int C, W;
   tok_shape(d, C, W);
   const int T = f / kTn;
   const bool exact = d / 8 == W * 32 * C;
 #define TWELL_BWD(CC, WW)                                                                                        \
-  (exact ? launch_bwd_cw<CC, WW, true>(M, ctr, s, dY, W_u, W_g, W_dt, count, val, col, row_ovf, u_ell, lambda,    \
+  (exact ? launch_bwd_cw<CC, WW, true>(M, ctr, long_rows, s, dY, W_u, W_g, W_dt, count, val, col, row_ovf, u_ell, lambda,    \
                                        du_ell, dz_ell, dX, M, d, T, K)                                          \
-         : launch_bwd_cw<CC, WW, false>(M, ctr, s, dY, W_u, W_g, W_dt, count, val, col, row_ovf, u_ell, lambda,   \
+         : launch_bwd_cw<CC, WW, false>(M, ctr, long_rows, s, dY, W_u, W_g, W_dt, count, val, col, row_ovf, u_ell, lambda,   \
                                         du_ell, dz_ell, dX, M, d, T, K))
   if (W == 1 && C == 1) TWELL_BWD(1, 1);
   else if (W == 1 && C == 2) TWELL_BWD(2, 1);

@@ -86,6 +86,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  // rows to process; a CTA without tiles leaves before touching tensor memory
+  if (threadIdx.x == 0) {
+    int m = shp.M;
+    if (shp.M_dev) {
+      const int v = *shp.M_dev;
+      m = v < m ? v : m;
+      m = m < 0 ? 0 : m;
+    }
+    *m_eff_s = m;
+  }
+  __syncthreads();
+  if (static_cast<long>(blockIdx.x) >= static_cast<long>((*m_eff_s + kBM - 1) / kBM) * ((shp.N + BN - 1) / BN)) return;
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -97,13 +110,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
-    int m = shp.M;
-    if (shp.M_dev) {
-      const int v = *shp.M_dev;
-      m = v < m ? v : m;
-      m = m < 0 ? 0 : m;
-    }
-    *m_eff_s = m;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
