@@ -101,56 +101,69 @@ __global__ void __launch_bounds__(256) csc_count_kernel(const uint16_t* __restri
 }
 
 // Per unit: exclusive scan over the row blocks (in place) and the unit total.
+// Loads of a batch are issued before its stores so they overlap.
+constexpr int kColScanBatch = 16;
 __global__ void csc_colscan_kernel(int* __restrict__ block_cnt, int nrb, int f, int* __restrict__ unit_tot) {
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= f) return;
   int run = 0;
-  for (int rb = 0; rb < nrb; ++rb) {
-    const long o = static_cast<long>(rb) * f + j;
-    const int c = block_cnt[o];
-    block_cnt[o] = run;
-    run += c;
+  for (int rb0 = 0; rb0 < nrb; rb0 += kColScanBatch) {
+    int c[kColScanBatch];
+#pragma unroll
+    for (int q = 0; q < kColScanBatch; ++q)
+      c[q] = rb0 + q < nrb ? block_cnt[static_cast<long>(rb0 + q) * f + j] : 0;
+#pragma unroll
+    for (int q = 0; q < kColScanBatch; ++q) {
+      if (rb0 + q < nrb) block_cnt[static_cast<long>(rb0 + q) * f + j] = run;
+      run += c[q];
+    }
   }
   unit_tot[j] = run;
 }
 
 // Single block: unit_ptr = exclusive scan of unit_tot, unit_ptr[f] = total.
+// Thread t owns the consecutive units [t*per, (t+1)*per), per = ceil(f/1024)
+// <= kMaxTiles*kTn/1024; one block-wide scan of the per-thread sums.
+constexpr int kUnitScanPer = kMaxTiles * kTn / 1024;
 __global__ void __launch_bounds__(1024) csc_unit_scan_kernel(const int* __restrict__ unit_tot, int f,
                                                              int* __restrict__ unit_ptr) {
   __shared__ int wsum[32];
-  __shared__ int carry;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  if (tid == 0) carry = 0;
+  const int per = (f + 1023) / 1024;
+  const int j0 = tid * per;
+  int v[kUnitScanPer];
+  int tot = 0;
+#pragma unroll
+  for (int q = 0; q < kUnitScanPer; ++q) {
+    v[q] = (q < per && j0 + q < f) ? unit_tot[j0 + q] : 0;
+    tot += v[q];
+  }
+  int incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) wsum[w] = incl;
   __syncthreads();
-  for (int base = 0; base < f; base += 1024) {
-    const int j = base + tid;
-    const int v = j < f ? unit_tot[j] : 0;
-    int incl = v;
+  if (w == 0) {
+    const int t = wsum[lane];
+    int ti = t;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-      if (lane >= o) incl += t;
+      const int q = __shfl_up_sync(0xFFFFFFFFu, ti, o);
+      if (lane >= o) ti += q;
     }
-    if (lane == 31) wsum[w] = incl;
-    __syncthreads();
-    if (w == 0) {
-      const int t = wsum[lane];
-      int ti = t;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int q = __shfl_up_sync(0xFFFFFFFFu, ti, o);
-        if (lane >= o) ti += q;
-      }
-      wsum[lane] = ti - t;
-    }
-    __syncthreads();
-    const int excl = carry + wsum[w] + incl - v;
-    if (j < f) unit_ptr[j] = excl;
-    __syncthreads();
-    if (tid == 1023) carry = excl + v;
-    __syncthreads();
+    wsum[lane] = ti - t;
   }
-  if (tid == 0) unit_ptr[f] = carry;
+  __syncthreads();
+  int run = wsum[w] + incl - tot;
+#pragma unroll
+  for (int q = 0; q < kUnitScanPer; ++q) {
+    if (q < per && j0 + q < f) unit_ptr[j0 + q] = run;
+    run += v[q];
+  }
+  if (tid == 1023) unit_ptr[f] = run;
 }
 
 __global__ void __launch_bounds__(256) csc_fill_kernel(

@@ -23,7 +23,12 @@
 //     wider groups with a named barrier of their own;
 //   * token rows are handed out dynamically (an atomic counter per launch),
 //     so groups that finish early take more rows and no CTA waits on a slow
-//     neighbour.
+//     neighbour;
+//   * a row's kept entries are processed in list chunks of kTokListCap; the
+//     row operand (x or dY) and the accumulators (Y or dX) are never live
+//     together, and between chunks the fp32 accumulators rest in global
+//     memory (a scratch row for Y, dX itself for dX), so rows of any length
+//     run at the same register budget.
 // Overflow rows are skipped (the dense backup path owns them).
 #include "trace.cuh"
 #include "twell_internal.cuh"
@@ -32,8 +37,8 @@ namespace twell {
 
 namespace {
 
-constexpr int kTokWarps = 4;   // warps per CTA (more when one token needs more)
-constexpr int kListCap = 256;  // list entries per chunk and group
+constexpr int kTokWarps = 4;            // warps per CTA (more when one token needs more)
+constexpr int kListCap = kTokListCap;   // list entries per chunk and group
 
 template <int C, int W>
 struct TokCfg {
@@ -50,6 +55,7 @@ struct GroupSmem {
   float c[kListCap];   // coefficient (g, then h; or dU)
   float c2[kListCap];  // second coefficient (u, then dZ) in the backward
   int slot[kListCap];  // t * K + s
+  int row;             // the token row being processed (re-read instead of kept live)
 };
 
 template <int W>
@@ -219,16 +225,47 @@ __device__ __forceinline__ void zero_acc(float2 (&y)[C][4]) {
     for (int e = 0; e < 4; ++e) y[q][e] = make_float2(0.f, 0.f);
 }
 
-// LONG = false: rows whose kept entries fit one list (the common case): the
-// row operand (x or dY) and the accumulators (Y or dX) are never live together,
-// which keeps these kernels at two CTAs per SM. LONG = true: the rare rows with
-// more entries, processed in list chunks with the accumulators kept live.
-template <int C, int W, bool LONG, bool EXACT>
-__global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, LONG ? 1 : 512 / (TokCfg<C, W>::WARPS * 32)) ell_fwd_kernel(
+// Plain (coherent) loads: the accumulator rows are written by this kernel.
+template <int C, int W, bool EXACT>
+__device__ __forceinline__ void load_acc(const float* __restrict__ acc, int first, int nch, float2 (&y)[C][4]) {
+  const float4* p = reinterpret_cast<const float4*>(acc);
+#pragma unroll
+  for (int q = 0; q < C; ++q) {
+    const int idx = first + W * 32 * q;
+    if (EXACT || idx < nch) {
+      const float4 a = p[2 * idx], b = p[2 * idx + 1];
+      y[q][0] = make_float2(a.x, a.y);
+      y[q][1] = make_float2(a.z, a.w);
+      y[q][2] = make_float2(b.x, b.y);
+      y[q][3] = make_float2(b.z, b.w);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) y[q][e] = make_float2(0.f, 0.f);
+    }
+  }
+}
+
+template <int C, int W, bool EXACT>
+__device__ __forceinline__ void store_acc(float* __restrict__ acc, int first, int nch, const float2 (&y)[C][4]) {
+  float4* p = reinterpret_cast<float4*>(acc);
+#pragma unroll
+  for (int q = 0; q < C; ++q) {
+    const int idx = first + W * 32 * q;
+    if (EXACT || idx < nch) {
+      p[2 * idx] = make_float4(y[q][0].x, y[q][0].y, y[q][1].x, y[q][1].y);
+      p[2 * idx + 1] = make_float4(y[q][2].x, y[q][2].y, y[q][3].x, y[q][3].y);
+    }
+  }
+}
+
+// yacc: [M][d] fp32 scratch for the partial Y of rows longer than one list
+// (unused, may be null, when every row fits one list).
+template <int C, int W, bool EXACT>
+__global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>::WARPS * 32)) ell_fwd_kernel(
     const uint16_t* __restrict__ X, const uint16_t* __restrict__ Wu, const uint16_t* __restrict__ Wdt,
     const uint16_t* __restrict__ count, const uint16_t* __restrict__ val, const uint8_t* __restrict__ col,
     const uint8_t* __restrict__ row_ovf, float* __restrict__ u_ell, uint16_t* __restrict__ Y, int M, int d, int T,
-    int K, int* __restrict__ ctr, int* __restrict__ long_rows) {
+    int K, int* __restrict__ ctr, float* __restrict__ yacc) {
   using Cfg = TokCfg<C, W>;
   constexpr int B = Cfg::B;
   __shared__ GroupSmem gs[Cfg::G];
@@ -265,62 +302,45 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, LONG ? 1 : 512 / (To
 #pragma unroll
     for (int q = 0; q < C; ++q) {
       const int idx = first + W * 32 * q;
-      if (idx < nch)
+      if (EXACT || idx < nch)
         yr[idx] = make_uint4(pack_bf16x2(y[q][0].x, y[q][0].y), pack_bf16x2(y[q][1].x, y[q][1].y),
                              pack_bf16x2(y[q][2].x, y[q][2].y), pack_bf16x2(y[q][3].x, y[q][3].y));
     }
   };
 
-  // short pass: rows 0..M-1 in claim order; rows too long for one list are
-  // appended to long_rows (count in ctr[2]) for the long pass, which walks
-  // that list only.
   for (;;) {
-    long row = next_row<W>(LONG ? ctr + 1 : ctr, grp, wi, lane, s_next);
-    if (LONG) {
-      if (row >= ctr[2]) break;
-      row = long_rows[row];
-    } else {
-      if (row >= M) break;
-      if (row_ovf[row]) continue;
-    }
+    const long row = next_row<W>(ctr, grp, wi, lane, s_next);
+    if (row >= M) break;
+    if (row_ovf[row]) continue;
     if (wi == 0) row_offsets(count, row, T, K, lane, g);
+    if (gtid == 0) g.row = static_cast<int>(row);
     group_sync<W>(grp);
-    const int total = g.tot;
-    if (!LONG && total > kListCap && wi == 0 && lane == 0) long_rows[atomicAdd(ctr + 2, 1)] = static_cast<int>(row);
-    if ((total > kListCap) == LONG) {
-      if constexpr (!LONG) {
-        build_list(g, row, T, K, 0, total, gtid, Cfg::GT, val, col, nullptr);
-        group_sync<W>(grp);
-        up(row, total);
-        float2 y[C][4];
-        zero_acc<C>(y);
-        gather_axpy<C, W, B, EXACT>(g, total, g.c, Wdt, d, first, nch, y);
-        store(row, y);
-      } else {
-        float2 y[C][4];
-        zero_acc<C>(y);
-        for (int e0 = 0; e0 < total; e0 += kListCap) {
-          const int ne = min(kListCap, total - e0);
-          build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, nullptr);
-          group_sync<W>(grp);
-          up(row, ne);
-          gather_axpy<C, W, B, EXACT>(g, ne, g.c, Wdt, d, first, nch, y);
-          group_sync<W>(grp);
-        }
-        store(row, y);
-      }
-    }
-    group_sync<W>(grp);  // warp 0 rewrites the offsets for the next row
+    int e0 = 0;
+    do {  // at least once: a row with no kept entry still writes Y = 0
+      const long row = g.row;
+      const int ne = min(kListCap, g.tot - e0);
+      build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, nullptr);
+      group_sync<W>(grp);
+      up(row, ne);
+      float2 y[C][4];
+      if (e0 == 0) zero_acc<C>(y);
+      else load_acc<C, W, EXACT>(yacc + row * d, first, nch, y);
+      gather_axpy<C, W, B, EXACT>(g, ne, g.c, Wdt, d, first, nch, y);
+      e0 += kListCap;
+      if (e0 >= g.tot) store(row, y);
+      else store_acc<C, W, EXACT>(yacc + row * d, first, nch, y);
+      group_sync<W>(grp);  // the list is rebuilt for the next chunk or row
+    } while (e0 < g.tot);
   }
 }
 
-template <int C, int W, bool LONG, bool EXACT>
-__global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, LONG ? 1 : 512 / (TokCfg<C, W>::WARPS * 32)) ell_bwd_kernel(
+template <int C, int W, bool EXACT>
+__global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>::WARPS * 32)) ell_bwd_kernel(
     const uint16_t* __restrict__ dY, const uint16_t* __restrict__ Wu, const uint16_t* __restrict__ Wg,
     const uint16_t* __restrict__ Wdt, const uint16_t* __restrict__ count, const uint16_t* __restrict__ val,
     const uint8_t* __restrict__ col, const uint8_t* __restrict__ row_ovf, const float* __restrict__ u_ell,
     float lambda, float* __restrict__ du_ell, float* __restrict__ dz_ell, float* __restrict__ dX, int M, int d,
-    int T, int K, int* __restrict__ ctr, int* __restrict__ long_rows) {
+    int T, int K, int* __restrict__ ctr) {
   using Cfg = TokCfg<C, W>;
   constexpr int B = Cfg::B;
   constexpr int B2 = B > 1 ? B / 2 : 1;  // two rows (W_u, W_g) per unit in the dX phase
@@ -358,62 +378,29 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, LONG ? 1 : 512 / (To
     }
     group_sync<W>(grp);
   };
-  auto dx_phase = [&](int ne, float2 (&dx)[C][4]) {
-    gather_axpy<C, W, B2, EXACT>(g, ne, g.c, Wu, d, first, nch, dx);
-    gather_axpy<C, W, B2, EXACT>(g, ne, g.c2, Wg, d, first, nch, dx);
-  };
-  auto store = [&](long row, const float2 (&dx)[C][4]) {
-    float4* xr = reinterpret_cast<float4*>(dX + row * d);
-#pragma unroll
-    for (int q = 0; q < C; ++q) {
-      const int idx = first + W * 32 * q;
-      if (idx < nch) {
-        xr[2 * idx] = make_float4(dx[q][0].x, dx[q][0].y, dx[q][1].x, dx[q][1].y);
-        xr[2 * idx + 1] = make_float4(dx[q][2].x, dx[q][2].y, dx[q][3].x, dx[q][3].y);
-      }
-    }
-  };
 
-  // short pass: rows 0..M-1 in claim order; rows too long for one list are
-  // appended to long_rows (count in ctr[2]) for the long pass, which walks
-  // that list only.
   for (;;) {
-    long row = next_row<W>(LONG ? ctr + 1 : ctr, grp, wi, lane, s_next);
-    if (LONG) {
-      if (row >= ctr[2]) break;
-      row = long_rows[row];
-    } else {
-      if (row >= M) break;
-      if (row_ovf[row]) continue;
-    }
+    const long row = next_row<W>(ctr, grp, wi, lane, s_next);
+    if (row >= M) break;
+    if (row_ovf[row]) continue;
     if (wi == 0) row_offsets(count, row, T, K, lane, g);
     group_sync<W>(grp);
-    const int total = g.tot;
-    if (!LONG && total > kListCap && wi == 0 && lane == 0) long_rows[atomicAdd(ctr + 2, 1)] = static_cast<int>(row);
-    if ((total > kListCap) == LONG) {
-      if constexpr (!LONG) {
-        build_list(g, row, T, K, 0, total, gtid, Cfg::GT, val, col, u_ell);
-        group_sync<W>(grp);
-        dh_phase(row, total);
-        float2 dx[C][4];
-        zero_acc<C>(dx);
-        dx_phase(total, dx);
-        store(row, dx);
-      } else {
-        float2 dx[C][4];
-        zero_acc<C>(dx);
-        for (int e0 = 0; e0 < total; e0 += kListCap) {
-          const int ne = min(kListCap, total - e0);
-          build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, u_ell);
-          group_sync<W>(grp);
-          dh_phase(row, ne);
-          dx_phase(ne, dx);
-          group_sync<W>(grp);
-        }
-        store(row, dx);
-      }
-    }
-    group_sync<W>(grp);  // warp 0 rewrites the offsets for the next row
+    float* dxr = dX + row * d;
+    int e0 = 0;
+    do {  // at least once: a row with no kept entry still writes dX = 0
+      const int ne = min(kListCap, g.tot - e0);
+      build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, u_ell);
+      group_sync<W>(grp);
+      dh_phase(row, ne);
+      float2 dx[C][4];
+      if (e0 == 0) zero_acc<C>(dx);
+      else load_acc<C, W, EXACT>(dxr, first, nch, dx);
+      gather_axpy<C, W, B2, EXACT>(g, ne, g.c, Wu, d, first, nch, dx);
+      gather_axpy<C, W, B2, EXACT>(g, ne, g.c2, Wg, d, first, nch, dx);
+      store_acc<C, W, EXACT>(dxr, first, nch, dx);
+      e0 += kListCap;
+      group_sync<W>(grp);  // the list is rebuilt for the next chunk or row
+    } while (e0 < g.tot);
   }
 }
 
@@ -435,25 +422,18 @@ int tok_grid(int M, int G) {
   return static_cast<int>(need < cap ? need : cap);
 }
 
-// Rows whose kept entries exceed one list are rare; the short pass lists them
-// and the long pass takes only those. ctr[0], ctr[1]: row counters of the two
-// passes; ctr[2]: number of listed long rows (all zero on entry).
 template <int C, int W, bool EXACT, typename... A>
-void launch_fwd_cw(int M, int* ctr, int* long_rows, cudaStream_t s, A... a) {
+void launch_fwd_cw(int M, cudaStream_t s, A... a) {
   constexpr int threads = TokCfg<C, W>::WARPS * 32;
   TWELL_LAUNCH("ell_updown", s,
-               ell_fwd_kernel<C, W, false, EXACT><<<tok_grid(M, TokCfg<C, W>::G), threads, 0, s>>>(a..., ctr, long_rows));
-  TWELL_LAUNCH("ell_updown_long", s,
-               ell_fwd_kernel<C, W, true, EXACT><<<device_sm_count(), threads, 0, s>>>(a..., ctr, long_rows));
+               ell_fwd_kernel<C, W, EXACT><<<tok_grid(M, TokCfg<C, W>::G), threads, 0, s>>>(a...));
 }
 
 template <int C, int W, bool EXACT, typename... A>
-void launch_bwd_cw(int M, int* ctr, int* long_rows, cudaStream_t s, A... a) {
+void launch_bwd_cw(int M, cudaStream_t s, A... a) {
   constexpr int threads = TokCfg<C, W>::WARPS * 32;
   TWELL_LAUNCH("ell_bwd", s,
-               ell_bwd_kernel<C, W, false, EXACT><<<tok_grid(M, TokCfg<C, W>::G), threads, 0, s>>>(a..., ctr, long_rows));
-  TWELL_LAUNCH("ell_bwd_long", s,
-               ell_bwd_kernel<C, W, true, EXACT><<<device_sm_count(), threads, 0, s>>>(a..., ctr, long_rows));
+               ell_bwd_kernel<C, W, EXACT><<<tok_grid(M, TokCfg<C, W>::G), threads, 0, s>>>(a...));
 }
 
 }  // namespace
@@ -461,19 +441,19 @@ void launch_bwd_cw(int M, int* ctr, int* long_rows, cudaStream_t s, A... a) {
 cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
                                const uint16_t* count, const uint16_t* val, const uint8_t* col,
                                const uint8_t* row_ovf, float* u_ell, uint16_t* Y, int M, int d, int f, int K,
-                               int* ctr, int* long_rows, cudaStream_t s) {
+                               int* ctr, float* yacc, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
-  cudaError_t e = cudaMemsetAsync(ctr, 0, 3 * sizeof(int), s);
+  cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
   int C, W;
   tok_shape(d, C, W);
   const int T = f / kTn;
   const bool exact = d / 8 == W * 32 * C;
 #define TWELL_FWD(CC, WW)                                                                                   \
-  (exact ? launch_fwd_cw<CC, WW, true>(M, ctr, long_rows, s, X, W_u, W_dt, count, val, col, row_ovf, u_ell, Y, M, d, \
-                                       T, K)                                                                    \
-         : launch_fwd_cw<CC, WW, false>(M, ctr, long_rows, s, X, W_u, W_dt, count, val, col, row_ovf, u_ell, Y, M, \
-                                        d, T, K))
+  (exact ? launch_fwd_cw<CC, WW, true>(M, s, X, W_u, W_dt, count, val, col, row_ovf, u_ell, Y, M, d, T, K, ctr, \
+                                       yacc)                                                                     \
+         : launch_fwd_cw<CC, WW, false>(M, s, X, W_u, W_dt, count, val, col, row_ovf, u_ell, Y, M, d, T, K, ctr,  \
+                                        yacc))
   if (W == 1 && C == 1) TWELL_FWD(1, 1);
   else if (W == 1 && C == 2) TWELL_FWD(2, 1);
   else if (W == 1 && C == 4) TWELL_FWD(4, 1);
@@ -489,19 +469,19 @@ cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const ui
                                const uint16_t* W_dt, const uint16_t* count, const uint16_t* val,
                                const uint8_t* col, const uint8_t* row_ovf, const float* u_ell, float lambda,
                                float* du_ell, float* dz_ell, float* dX, int M, int d, int f, int K, int* ctr,
-                               int* long_rows, cudaStream_t s) {
+                               cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
-  cudaError_t e = cudaMemsetAsync(ctr, 0, 3 * sizeof(int), s);
+  cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
   int C, W;
   tok_shape(d, C, W);
   const int T = f / kTn;
   const bool exact = d / 8 == W * 32 * C;
 #define TWELL_BWD(CC, WW)                                                                                        \
-  (exact ? launch_bwd_cw<CC, WW, true>(M, ctr, long_rows, s, dY, W_u, W_g, W_dt, count, val, col, row_ovf, u_ell, lambda,    \
-                                       du_ell, dz_ell, dX, M, d, T, K)                                          \
-         : launch_bwd_cw<CC, WW, false>(M, ctr, long_rows, s, dY, W_u, W_g, W_dt, count, val, col, row_ovf, u_ell, lambda,   \
-                                        du_ell, dz_ell, dX, M, d, T, K))
+  (exact ? launch_bwd_cw<CC, WW, true>(M, s, dY, W_u, W_g, W_dt, count, val, col, row_ovf, u_ell, lambda, du_ell,  \
+                                       dz_ell, dX, M, d, T, K, ctr)                                              \
+         : launch_bwd_cw<CC, WW, false>(M, s, dY, W_u, W_g, W_dt, count, val, col, row_ovf, u_ell, lambda, du_ell, \
+                                        dz_ell, dX, M, d, T, K, ctr))
   if (W == 1 && C == 1) TWELL_BWD(1, 1);
   else if (W == 1 && C == 2) TWELL_BWD(2, 1);
   else if (W == 1 && C == 4) TWELL_BWD(4, 1);

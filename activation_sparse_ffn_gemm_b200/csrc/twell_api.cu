@@ -64,9 +64,12 @@ constexpr size_t kWsAlign = 256;
 
 size_t align_up(size_t x) { return (x + kWsAlign - 1) & ~(kWsAlign - 1); }
 
+// Rows of this shape can hold more kept entries than one token-kernel list.
+bool rows_can_exceed_list(int64_t f, int64_t K) { return (f / kTn) * K > kTokListCap; }
+
 struct WsLayout {
-  size_t ctr = 0;        // row counters of the token kernels
-  size_t long_rows = 0;  // rows too long for one list of the token kernels
+  size_t ctr = 0;   // row counter of the token kernels
+  size_t yacc = 0;  // fp32 partial Y of rows longer than one list of the token kernels
   size_t spill = 0, x_ovf = 0, h_ovf = 0, w_dt = 0;
   size_t dy_ovf = 0, duz = 0, du_ovf = 0, dz_ovf = 0, du_ell = 0, dz_ell = 0, row_slot = 0, block_cnt = 0, unit_tot = 0, unit_ptr = 0,
          csc_row = 0, csc_val = 0;
@@ -83,10 +86,8 @@ WsLayout ws_layout(twell_op op, int64_t M, int64_t d, int64_t f, int64_t K, int6
   };
   const int64_t T = f / kTn;
   const int64_t cap1 = cap > 0 ? cap : 1;
-  if (op == TWELL_OP_FWD || op == TWELL_OP_BWD) {
-    L.ctr = take(64);
-    L.long_rows = take(static_cast<size_t>(M * 4));
-  }
+  if (op == TWELL_OP_FWD || op == TWELL_OP_BWD) L.ctr = take(64);
+  if (op == TWELL_OP_FWD && rows_can_exceed_list(f, K)) L.yacc = take(static_cast<size_t>(M * d * 4));
   if (op == TWELL_OP_PACK || op == TWELL_OP_FWD) L.spill = take(static_cast<size_t>(M * f * 2));
   if (op == TWELL_OP_FWD) {
     L.x_ovf = take(static_cast<size_t>(cap1 * d * 2));
@@ -243,7 +244,7 @@ twell_status twell_ffn_fwd(const uint16_t* X, const uint16_t* W_g, const uint16_
   st = run_pack(X, W_g, b_g, d, h, z_debug, ws, L, X, x_ovf, s);
   if (st != TWELL_OK) return st;
   if (launch_ell_ffn_fwd(X, W_u, wdt, h->count, h->val, h->col, h->row_ovf, h->u_ell, Y, M, d, f, K,
-                         at<int>(ws, L.ctr), at<int>(ws, L.long_rows), s) != cudaSuccess)
+                         at<int>(ws, L.ctr), rows_can_exceed_list(f, K) ? at<float>(ws, L.yacc) : nullptr, s) != cudaSuccess)
     return TWELL_ECUDA;
   return cuda_status(launch_ovf_fwd(x_ovf, W_u, W_d, h->g_ovf, h->ovf_rows, h->n_ovf, cap, d, f,
                                     at<uint16_t>(ws, L.h_ovf), h->u_ovf, Y, h->status, s));
@@ -290,7 +291,7 @@ twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_
   float* dz_ell = at<float>(ws, L.dz_ell);
   if (launch_gather_rows(dY, h->ovf_rows, h->n_ovf, cap, d, dy_ovf, s) != cudaSuccess) return TWELL_ECUDA;
   if (launch_ell_ffn_bwd(dY, W_u, W_g, wdt, h->count, h->val, h->col, h->row_ovf, h->u_ell, lambda, du_ell, dz_ell,
-                         dX, M, d, f, K, at<int>(ws, L.ctr), at<int>(ws, L.long_rows), s) != cudaSuccess)
+                         dX, M, d, f, K, at<int>(ws, L.ctr), s) != cudaSuccess)
     return TWELL_ECUDA;
   float* du_ovf = at<float>(ws, L.du_ovf);
   float* dz_ovf = at<float>(ws, L.dz_ovf);

@@ -16,6 +16,7 @@ constexpr int kTn = 128;           // TwELL tile width (columns of one GEMM N-ti
 constexpr int kMaxK = 64;          // widest ELL row per tile
 constexpr int kMaxTiles = 128;     // d_ff <= 16384
 constexpr int kMaxDModel = 16384;  // 128 threads x 16 chunks x 8 bf16
+constexpr int kTokListCap = 256;   // kept entries per list chunk of the token kernels
 
 // ------------------------------------------------------------ device helpers
 
@@ -96,12 +97,13 @@ cudaError_t launch_gather_rows(const uint16_t* in, const int* rows, const int* n
 cudaError_t launch_transpose_bf16(const uint16_t* in, int rows, int cols, uint16_t* out, cudaStream_t s);
 
 // Fused sparse up + down over the ELL rows (overflow rows are skipped).
-// ctr: three ints of device scratch (row counters), zeroed by the launcher;
-// long_rows: M ints of device scratch (rows too long for one list).
+// ctr: one int of device scratch (the row counter), zeroed by the launcher;
+// yacc: [M][d] fp32 scratch for rows with more than kTokListCap kept entries
+// (may be null when (d_ff / kTn) * K <= kTokListCap).
 cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
                                const uint16_t* count, const uint16_t* val, const uint8_t* col,
                                const uint8_t* row_ovf, float* u_ell, uint16_t* Y, int M, int d, int f, int K,
-                               int* ctr, int* long_rows, cudaStream_t s);
+                               int* ctr, float* yacc, cudaStream_t s);
 
 // Dense backup forward for overflow rows: H = bf16(G * (X_ovf W_u^T)) then
 // Y[ovf_rows] = bf16(H W_d^T).
@@ -115,7 +117,7 @@ cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const ui
                                const uint16_t* W_dt, const uint16_t* count, const uint16_t* val,
                                const uint8_t* col, const uint8_t* row_ovf, const float* u_ell, float lambda,
                                float* du_ell, float* dz_ell, float* dX, int M, int d, int f, int K, int* ctr,
-                               int* long_rows, cudaStream_t s);
+                               cudaStream_t s);
 
 // Dense backup backward for overflow rows: dU, dZ (fp32, and bf16 [dU | dZ] as
 // the next GEMM's operand) from dH = dY_ovf W_d, then dX[ovf_rows] = dU W_u + dZ W_g.

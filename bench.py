@@ -9,6 +9,13 @@ over the hybrid format (L1 term on the gate activations). Workload: the uniform
 K=8) run as a training step, synthetic seeded data, inputs resident in HBM.
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+    python bench.py --sweep [--steps K --warmup W]
+
+--sweep times the forward and forward+backward of TwELL and of the dense bf16
+FFN over token counts M in {512, 2048, 8192, 32768, 65536} and mean sparsity in
+{90, 95, 99, 99.5, 99.9}% at d_model=4096, d_ff=14336, with per-token
+lognormal(0, 0.75) row scaling, K = max(8, 2^ceil(log2(4 p T_n))), one JSON
+line per point (1 GPU).
 
 Prints one JSON line (rank 0). With N > 1 (torchrun) every rank runs its own
 replica of the batch; the time is the max over ranks and the value counts the
@@ -47,6 +54,10 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--no-trace", action="store_true")
+    p.add_argument("--sweep", action="store_true",
+                   help="token-count x sparsity sweep at d_model=4096, d_ff=14336 (one JSON line per point)")
+    p.add_argument("--sweep-m", default="512,2048,8192,32768,65536")
+    p.add_argument("--sweep-sparsity", default="0.9,0.95,0.99,0.995,0.999")
     return p.parse_args()
 
 
@@ -488,10 +499,113 @@ def run_twell(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- sweep
+
+
+def run_sweep(args, local):
+    """Forward and forward+backward time of TwELL and dense bf16 per (M, sparsity) point."""
+    import torch
+
+    import activation_sparse_ffn_gemm_b200 as tw
+    from synthetic import gate_bias_for_activity, sweep_k
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    d, f, T_n, sigma = 4096, 14336, 128, 0.75
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    steps, warm = max(1, args.steps), max(3, args.warmup)
+
+    def timed(body):
+        for _ in range(warm):
+            body()
+        torch.cuda.synchronize(dev)
+        tot = 0.0
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            body()
+            e1.record(stream)
+            e1.synchronize()
+            tot += e0.elapsed_time(e1)
+        return tot / steps
+
+    for sp in (float(v) for v in args.sweep_sparsity.split(",")):
+        p = 1.0 - sp
+        K = sweep_k(p, T_n)
+        bias = gate_bias_for_activity(p, "lognormal", sigma)
+        for M in (int(v) for v in args.sweep_m.split(",")):
+            g = torch.Generator(device=dev)
+            g.manual_seed(1000003 * M + int(round(sp * 1e4)))
+            rs = torch.exp(sigma * torch.randn(M, 1, device=dev, generator=g))
+            X = (torch.randn(M, d, device=dev, generator=g) * rs).to(torch.bfloat16)
+            W_g = (torch.randn(f, d, device=dev, generator=g) / math.sqrt(d)).to(torch.bfloat16)
+            W_u = (torch.randn(f, d, device=dev, generator=g) / math.sqrt(d)).to(torch.bfloat16)
+            W_d = (torch.randn(d, f, device=dev, generator=g) / math.sqrt(f)).to(torch.bfloat16)
+            dY = torch.randn(M, d, device=dev, generator=g).to(torch.bfloat16)
+            b_g = torch.full((f,), bias, device=dev).to(torch.bfloat16)
+            st = tw.HybridState(M, f, T_n, K, M, dev, with_u=True)
+            wsf = tw.workspace(tw.OP_FWD, M, d, f, T_n, K, M, dev)
+            wsb = tw.workspace(tw.OP_BWD, M, d, f, T_n, K, M, dev)
+            Wdt = torch.empty((f, d), dtype=torch.bfloat16, device=dev)
+            Y = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
+            grads = dict(dX=torch.empty((M, d), device=dev), dW_g=torch.empty((f, d), device=dev),
+                         dW_u=torch.empty((f, d), device=dev), dW_d=torch.empty((d, f), device=dev),
+                         db_g=torch.empty(f, device=dev))
+
+            def fwd():
+                tw.transpose_wd(W_d, out=Wdt)
+                tw.ffn_fwd(X, W_g, b_g, W_u, W_d, T_n=T_n, K=K, W_dt=Wdt, state=st, ws=wsf, Y=Y)
+
+            def fwd_bwd():
+                fwd()
+                tw.ffn_bwd(X, W_g, W_u, W_d, st, dY, lam=args.lam, W_dt=Wdt, ws=wsb, out=grads)
+
+            t_fwd = timed(fwd)
+            t_fb = timed(fwd_bwd)
+            assert st.read_status() == 0, "device status word set"
+            n_ovf = st.n_overflow()[1]
+            cnt = st.count.float()
+            activity = float(cnt.sum().item()) / (M * f)
+            ratio = float(cnt.max().item()) / max(float(cnt.mean().item()), 1e-30)
+            del st, wsf, wsb, grads, Wdt, Y
+
+            Wg_r, Wu_r, Wd_r = (t.clone().requires_grad_() for t in (W_g, W_u, W_d))
+            Xr = X.clone().requires_grad_()
+
+            def dense_fwd():
+                with torch.no_grad():
+                    (torch.relu(X @ W_g.T + b_g) * (X @ W_u.T)) @ W_d.T
+
+            def dense_fb():
+                z = Xr @ Wg_r.T + b_g
+                gg = torch.relu(z)
+                y = (gg * (Xr @ Wu_r.T)) @ Wd_r.T
+                (y.float() * dY.float()).sum().add(gg.float().sum() * args.lam).backward()
+                Xr.grad = Wg_r.grad = Wu_r.grad = Wd_r.grad = None
+
+            t_dfwd = timed(dense_fwd)
+            t_dfb = timed(dense_fb)
+            del Wg_r, Wu_r, Wd_r, Xr, X, W_g, W_u, W_d, dY, b_g, rs
+            torch.cuda.empty_cache()
+            print(json.dumps({
+                "point": {"M": M, "sparsity": sp, "d_model": d, "d_ff": f, "T_n": T_n, "K": K},
+                "twell": {"fwd_ms": t_fwd, "fwd_bwd_ms": t_fb, "fwd_tokens_per_s": M / (t_fwd / 1e3),
+                          "fwd_bwd_tokens_per_s": M / (t_fb / 1e3)},
+                "dense_bf16": {"fwd_ms": t_dfwd, "fwd_bwd_ms": t_dfb},
+                "speedup_vs_dense": {"fwd": t_dfwd / t_fwd, "fwd_bwd": t_dfb / t_fb},
+                "measured": {"activity": activity, "overflow_rows": n_ovf, "max_over_mean_count": ratio},
+                "steps": steps, "warmup": warm, "data": "synthetic (seeded torch CUDA generator)",
+                "l2": "flushed before every timed step"}), flush=True)
+
+
 def main():
     args = parse_args()
     world, rank, local = dist_env()
-    if args.impl == "reference":
+    if args.sweep:
+        run_sweep(args, local)
+    elif args.impl == "reference":
         run_reference(args, world, rank)
     else:
         run_twell(args, world, rank, local)

@@ -83,6 +83,11 @@ CASES = {
     "k64": (130, 256, 2048, 64, 0.2, "lognormal", 4),
     "one_row": (1, 128, 256, 8, 0.3, "none", 5),
     "multi_tile": (700, 1024, 2048, 8, 0.01, "lognormal", 6),
+    # rows of ~400 kept entries (the long-row pass) with two warps per token
+    "long_rows_w2": (96, 4096, 4096, 32, 0.1, "none", 7),
+    # four and eight warps per token (d_model / 8 chunks of 16 bytes > 512)
+    "wide_d_w4": (40, 8192, 1024, 16, 0.05, "none", 8),
+    "widest_d_w8": (24, 16384, 512, 8, 0.03, "none", 10),
 }
 
 
