@@ -47,7 +47,7 @@ class TwellHybrid(ctypes.Structure):
     _fields_ = [("M", ctypes.c_int32), ("d_ff", ctypes.c_int32), ("T_n", ctypes.c_int32), ("K", ctypes.c_int32),
                 ("ovf_cap", ctypes.c_int32), ("count", _vp), ("val", _vp), ("col", _vp), ("row_ovf", _vp),
                 ("ovf_rows", _vp), ("n_ovf", _vp), ("g_ovf", _vp), ("u_ell", _vp), ("u_ovf", _vp),
-                ("status", _vp)]
+                ("status", _vp), ("row_plan", _vp)]
 
 
 _lock = threading.Lock()
@@ -67,6 +67,8 @@ def lib():
             L.twell_status_string.argtypes = [ctypes.c_int]
             L.twell_query_support.restype = ctypes.c_int
             L.twell_query_support.argtypes = [_i64] * 6
+            L.twell_plan_ints.restype = ctypes.c_size_t
+            L.twell_plan_ints.argtypes = [_i64] * 4
             L.twell_workspace_bytes.restype = ctypes.c_size_t
             L.twell_workspace_bytes.argtypes = [ctypes.c_int] + [_i64] * 6
             L.twell_transpose_wd.restype = ctypes.c_int
@@ -165,10 +167,12 @@ class HybridState:
         self.u_ell = torch.empty((M, T, K), dtype=torch.float32, device=dev) if with_u else None
         self.u_ovf = torch.empty((cap1, d_ff), dtype=torch.float32, device=dev) if with_u else None
         self.status = torch.zeros(4, dtype=torch.int32, device=dev)
+        self.row_plan = torch.zeros(max(int(lib().twell_plan_ints(M, d_ff, T_n, K)), 1), dtype=torch.int32,
+                                    device=dev)
         self.c = TwellHybrid(M, d_ff, T_n, K, cap, *(
             (t.data_ptr() if t is not None else None) for t in
             (self.count, self.val, self.col, self.row_ovf, self.ovf_rows, self.n_ovf, self.g_ovf, self.u_ell,
-             self.u_ovf, self.status)))
+             self.u_ovf, self.status, self.row_plan)))
 
     def read_status(self, clear: bool = False, stream=None) -> int:
         out = ctypes.c_uint32(0)

@@ -18,17 +18,99 @@ namespace {
 constexpr int kScanThreads = 1024;
 constexpr int kScanItems = 16;
 
-// row_ovf[i] = any_t(count[i][t] > K); one warp per row.
+// row_ovf[i] = any_t(count[i][t] > K), and the row's kept entries
+// kept[i] = sum_t min(count[i][t], K) (-1 for an overflow row); one warp per row.
 __global__ void row_flags_kernel(const uint16_t* __restrict__ count, int M, int T, int K,
-                                 uint8_t* __restrict__ row_ovf) {
+                                 uint8_t* __restrict__ row_ovf, int* __restrict__ kept) {
   const int lane = threadIdx.x & 31;
   const long warp0 = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long nwarps = (static_cast<long>(gridDim.x) * blockDim.x) >> 5;
   for (long row = warp0; row < M; row += nwarps) {
     bool any = false;
-    for (int t = lane; t < T; t += 32) any |= count[row * T + t] > K;
+    int n = 0;
+    for (int t = lane; t < T; t += 32) {
+      const int c = count[row * T + t];
+      any |= c > K;
+      n += c < K ? c : K;
+    }
     any = __any_sync(0xFFFFFFFFu, any);
-    if (lane == 0) row_ovf[row] = any ? 1 : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xFFFFFFFFu, n, o);
+    if (lane == 0) {
+      row_ovf[row] = any ? 1 : 0;
+      kept[row] = any ? -1 : n;
+    }
+  }
+}
+
+// Single block: the row plan of the token kernels (layout in twell_internal.cuh).
+// Reads the kept counts parked in the turnstile words, sizes the pieces
+// S = clamp(ceil(total / groups), kPieceMin, kTokListCap), lists the pieces
+// (max(1, ceil(kept / S)) per non-overflow row, none for overflow rows) and
+// zeroes the turnstile words. Thread t owns the consecutive rows
+// [t * per, (t + 1) * per): it reads its counts before it zeroes them.
+__global__ void __launch_bounds__(kScanThreads) plan_kernel(int* __restrict__ plan, int M, int groups) {
+  __shared__ long long red[kScanThreads / 32];
+  __shared__ int warp_tot[kScanThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  int* kept = plan + kPlanHdr;
+  int* pieces = plan + kPlanHdr + M;
+  const long per = (static_cast<long>(M) + kScanThreads - 1) / kScanThreads;
+  const long r0 = tid * per, r1 = r0 + per < M ? r0 + per : M;
+  long long tot = 0;
+  for (long r = r0; r < r1; ++r) {
+    const int v = kept[r];
+    tot += v > 0 ? v : 0;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xFFFFFFFFu, tot, o);
+  if (lane == 0) red[w] = tot;
+  __syncthreads();
+  long long total = 0;
+  for (int q = 0; q < kScanThreads / 32; ++q) total += red[q];
+  const long long g = groups > 0 ? groups : 1;
+  long long sz = (total + g - 1) / g;
+  sz = sz < kPieceMin ? kPieceMin : (sz > kTokListCap ? kTokListCap : sz);
+  const int S = static_cast<int>(sz);
+  int mine = 0;
+  for (long r = r0; r < r1; ++r) {
+    const int v = kept[r];
+    mine += v < 0 ? 0 : (v > 0 ? (v + S - 1) / S : 1);
+  }
+  int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) warp_tot[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    const int t = warp_tot[lane];
+    int ti = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int q = __shfl_up_sync(0xFFFFFFFFu, ti, o);
+      if (lane >= o) ti += q;
+    }
+    warp_tot[lane] = ti;  // inclusive
+  }
+  __syncthreads();
+  int base = (w > 0 ? warp_tot[w - 1] : 0) + incl - mine;
+  for (long r = r0; r < r1; ++r) {
+    const int v = kept[r];
+    const int P = v < 0 ? 0 : (v > 0 ? (v + S - 1) / S : 1);
+    for (int q = 0; q < P; ++q, ++base) {
+      pieces[2L * base] = static_cast<int>(r);
+      pieces[2L * base + 1] = q;
+    }
+    kept[r] = 0;
+  }
+  if (tid == 0) {
+    plan[0] = warp_tot[kScanThreads / 32 - 1];
+    plan[1] = S;
+    plan[2] = static_cast<int>(total < 0x7FFFFFFFLL ? total : 0x7FFFFFFFLL);
+    plan[3] = 0;
   }
 }
 
@@ -180,16 +262,17 @@ __global__ void transpose_bf16_kernel(const uint16_t* __restrict__ in, int rows,
 
 cudaError_t launch_route(const uint16_t* count, const uint16_t* val, const uint8_t* col, const uint16_t* spill,
                          int M, int f, int K, int cap, uint8_t* row_ovf, int* ovf_rows, int* n_ovf,
-                         uint16_t* g_ovf, const uint16_t* X, int d, uint16_t* x_ovf, uint32_t* status,
-                         cudaStream_t s) {
+                         uint16_t* g_ovf, const uint16_t* X, int d, uint16_t* x_ovf, int* plan, int groups,
+                         uint32_t* status, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   const int T = f / kTn;
   const int warps_needed = M;
   int blocks = (warps_needed + 7) / 8;
   const int max_blocks = device_sm_count() * 16;
   if (blocks > max_blocks) blocks = max_blocks;
-  TWELL_LAUNCH("row_flags", s, row_flags_kernel<<<blocks, 256, 0, s>>>(count, M, T, K, row_ovf));
+  TWELL_LAUNCH("row_flags", s, row_flags_kernel<<<blocks, 256, 0, s>>>(count, M, T, K, row_ovf, plan + kPlanHdr));
   TWELL_LAUNCH("ovf_scan", s, ovf_scan_kernel<<<1, kScanThreads, 0, s>>>(row_ovf, M, cap, ovf_rows, n_ovf, status));
+  TWELL_LAUNCH("row_plan", s, plan_kernel<<<1, kScanThreads, 0, s>>>(plan, M, groups));
   if (cap > 0) {
     int g = cap < device_sm_count() * 4 ? cap : device_sm_count() * 4;
     TWELL_LAUNCH("ovf_gather", s,

@@ -21,15 +21,18 @@
 //   * units are processed B at a time (all B*C loads issued before any use);
 //   * no CTA-wide barrier: a single-warp group synchronises with __syncwarp,
 //     wider groups with a named barrier of their own;
-//   * token rows are handed out dynamically (an atomic counter per launch),
-//     so groups that finish early take more rows and no CTA waits on a slow
-//     neighbour;
-//   * a row's kept entries are processed in list chunks of kTokListCap; the
-//     row operand (x or dY) and the accumulators (Y or dX) are never live
-//     together, and between chunks the fp32 accumulators rest in global
-//     memory (a scratch row for Y, dX itself for dX), so rows of any length
-//     run at the same register budget.
-// Overflow rows are skipped (the dense backup path owns them).
+//   * work is handed out dynamically (an atomic counter per launch) as the
+//     pieces of the row plan: a row's kept entries split into pieces of at
+//     most S entries, S sized so that the pieces spread over all resident
+//     token groups (the heavy rows of a batch are split, light rows stay
+//     whole), so no group is left with one long row at the end;
+//   * the row operand (x or dY) and the accumulators (Y or dX) are never live
+//     together; the pieces of one row add their fp32 partial sums into a
+//     global accumulator row (a scratch row for Y, dX itself for dX) one after
+//     another in piece order, through a per-row turnstile, so the result is
+//     the same on every run.
+// Overflow rows have no pieces (the dense backup path owns them).
+#include "sm100.cuh"
 #include "trace.cuh"
 #include "twell_internal.cuh"
 
@@ -55,7 +58,7 @@ struct GroupSmem {
   float c[kListCap];   // coefficient (g, then h; or dU)
   float c2[kListCap];  // second coefficient (u, then dZ) in the backward
   int slot[kListCap];  // t * K + s
-  int row;             // the token row being processed (re-read instead of kept live)
+  int row, q, P;       // the piece being processed (re-read instead of kept live)
 };
 
 template <int W>
@@ -225,22 +228,17 @@ __device__ __forceinline__ void zero_acc(float2 (&y)[C][4]) {
     for (int e = 0; e < 4; ++e) y[q][e] = make_float2(0.f, 0.f);
 }
 
-// Plain (coherent) loads: the accumulator rows are written by this kernel.
+// y += the fp32 row at acc (loaded through L2: it was written by another CTA).
 template <int C, int W, bool EXACT>
-__device__ __forceinline__ void load_acc(const float* __restrict__ acc, int first, int nch, float2 (&y)[C][4]) {
+__device__ __forceinline__ void add_acc(const float* __restrict__ acc, int first, int nch, float2 (&y)[C][4]) {
   const float4* p = reinterpret_cast<const float4*>(acc);
 #pragma unroll
   for (int q = 0; q < C; ++q) {
     const int idx = first + W * 32 * q;
     if (EXACT || idx < nch) {
-      const float4 a = p[2 * idx], b = p[2 * idx + 1];
-      y[q][0] = make_float2(a.x, a.y);
-      y[q][1] = make_float2(a.z, a.w);
-      y[q][2] = make_float2(b.x, b.y);
-      y[q][3] = make_float2(b.z, b.w);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) y[q][e] = make_float2(0.f, 0.f);
+      const float4 a = __ldcg(p + 2 * idx), b = __ldcg(p + 2 * idx + 1);
+      y[q][0].x += a.x; y[q][0].y += a.y; y[q][1].x += a.z; y[q][1].y += a.w;
+      y[q][2].x += b.x; y[q][2].y += b.y; y[q][3].x += b.z; y[q][3].y += b.w;
     }
   }
 }
@@ -258,14 +256,67 @@ __device__ __forceinline__ void store_acc(float* __restrict__ acc, int first, in
   }
 }
 
-// yacc: [M][d] fp32 scratch for the partial Y of rows longer than one list
-// (unused, may be null, when every row fits one list).
+// Turnstile of one row: the group holding piece q waits until the row's turn
+// word equals q (pieces q' < q have added their partials), bounded by
+// kWaitLimitNs; on expiry it records TWELL_STATUS_TIMEOUT and goes on.
+// Progress: pieces are handed out in order, so piece q-1 belongs to a group
+// that is already running (or has finished), and piece 0 never waits.
+template <int W>
+__device__ __forceinline__ void turn_wait(const int* turn, int row, int q, int grp, int gtid, uint32_t* status) {
+  if (gtid == 0 && q > 0) {
+    const volatile int* t = turn + row;
+    if (*t != q) {
+      const uint64_t t0 = globaltimer_ns();
+      while (*t != q) {
+        __nanosleep(100);
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          set_status(status, TWELL_STATUS_TIMEOUT);
+          break;
+        }
+      }
+    }
+    __threadfence();
+  }
+  group_sync<W>(grp);
+}
+
+// Publishes this piece's accumulator stores and passes the turn on (back to 0
+// after the last piece, so the word is 0 again between launches).
+template <int W>
+__device__ __forceinline__ void turn_pass(int* turn, int row, int q, int P, int grp, int gtid) {
+  __threadfence();
+  group_sync<W>(grp);
+  if (gtid == 0) atomicExch(turn + row, q + 1 == P ? 0 : q + 1);
+}
+
+// Reads piece p of the plan into the group's shared memory (row, q, P) with
+// the row's kept-entry offsets; returns false when the plan is exhausted.
+template <int W>
+__device__ __forceinline__ bool next_piece(int* ctr, const int* plan, int M, const uint16_t* __restrict__ count, int T,
+                                           int K, int grp, int wi, int lane, int* s_next, GroupSmem& g) {
+  const int np = plan[0], S = plan[1];
+  const int p = static_cast<int>(next_row<W>(ctr, grp, wi, lane, s_next));
+  if (p >= np) return false;
+  const int* pieces = plan + kPlanHdr + M;
+  const int row = pieces[2 * p], q = pieces[2 * p + 1];
+  if (wi == 0) row_offsets(count, row, T, K, lane, g);
+  if (wi == 0 && lane == 0) {
+    const int n = g.tot;
+    g.row = row;
+    g.q = q;
+    g.P = n > 0 ? (n + S - 1) / S : 1;
+  }
+  group_sync<W>(grp);
+  return true;
+}
+
+// yacc: [M][d] fp32 accumulator rows for rows split into several pieces.
 template <int C, int W, bool EXACT>
 __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>::WARPS * 32)) ell_fwd_kernel(
     const uint16_t* __restrict__ X, const uint16_t* __restrict__ Wu, const uint16_t* __restrict__ Wdt,
     const uint16_t* __restrict__ count, const uint16_t* __restrict__ val, const uint8_t* __restrict__ col,
-    const uint8_t* __restrict__ row_ovf, float* __restrict__ u_ell, uint16_t* __restrict__ Y, int M, int d, int T,
-    int K, int* __restrict__ ctr, float* __restrict__ yacc) {
+    int* __restrict__ plan, float* __restrict__ u_ell, uint16_t* __restrict__ Y, int M, int d, int T, int K,
+    int* __restrict__ ctr, float* __restrict__ yacc, uint32_t* status) {
   using Cfg = TokCfg<C, W>;
   constexpr int B = Cfg::B;
   __shared__ GroupSmem gs[Cfg::G];
@@ -276,6 +327,7 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
   GroupSmem& g = gs[grp];
   const int nch = d >> 3;
   const int first = gtid;
+  int* turn = plan + kPlanHdr;
 
   // u = x . W_u[j] for the listed units, then h = g u in g.c (u saved when asked)
   auto up = [&](long row, int ne) {
@@ -308,29 +360,31 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
     }
   };
 
-  for (;;) {
-    const long row = next_row<W>(ctr, grp, wi, lane, s_next);
-    if (row >= M) break;
-    if (row_ovf[row]) continue;
-    if (wi == 0) row_offsets(count, row, T, K, lane, g);
-    if (gtid == 0) g.row = static_cast<int>(row);
+  while (next_piece<W>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g)) {
+    const long row = g.row;
+    const int S = plan[1];
+    const int e0 = g.q * S;
+    const int ne = max(0, min(S, g.tot - e0));
+    build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, nullptr);
     group_sync<W>(grp);
-    int e0 = 0;
-    do {  // at least once: a row with no kept entry still writes Y = 0
-      const long row = g.row;
-      const int ne = min(kListCap, g.tot - e0);
-      build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, nullptr);
-      group_sync<W>(grp);
-      up(row, ne);
-      float2 y[C][4];
-      if (e0 == 0) zero_acc<C>(y);
-      else load_acc<C, W, EXACT>(yacc + row * d, first, nch, y);
-      gather_axpy<C, W, B, EXACT>(g, ne, g.c, Wdt, d, first, nch, y);
-      e0 += kListCap;
-      if (e0 >= g.tot) store(row, y);
-      else store_acc<C, W, EXACT>(yacc + row * d, first, nch, y);
-      group_sync<W>(grp);  // the list is rebuilt for the next chunk or row
-    } while (e0 < g.tot);
+    up(row, ne);
+    float2 y[C][4];
+    zero_acc<C>(y);
+    gather_axpy<C, W, B, EXACT>(g, ne, g.c, Wdt, d, first, nch, y);
+    {
+      const int rw = g.row, q = g.q, P = g.P;
+      if (P == 1) {
+        store(rw, y);
+      } else {
+        float* acc = yacc + static_cast<long>(rw) * d;
+        turn_wait<W>(turn, rw, q, grp, gtid, status);
+        if (q > 0) add_acc<C, W, EXACT>(acc, first, nch, y);
+        if (q + 1 == P) store(rw, y);
+        else store_acc<C, W, EXACT>(acc, first, nch, y);
+        turn_pass<W>(turn, rw, q, P, grp, gtid);
+      }
+    }
+    group_sync<W>(grp);  // the group's shared memory is rewritten for the next piece
   }
 }
 
@@ -338,9 +392,9 @@ template <int C, int W, bool EXACT>
 __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>::WARPS * 32)) ell_bwd_kernel(
     const uint16_t* __restrict__ dY, const uint16_t* __restrict__ Wu, const uint16_t* __restrict__ Wg,
     const uint16_t* __restrict__ Wdt, const uint16_t* __restrict__ count, const uint16_t* __restrict__ val,
-    const uint8_t* __restrict__ col, const uint8_t* __restrict__ row_ovf, const float* __restrict__ u_ell,
-    float lambda, float* __restrict__ du_ell, float* __restrict__ dz_ell, float* __restrict__ dX, int M, int d,
-    int T, int K, int* __restrict__ ctr) {
+    const uint8_t* __restrict__ col, int* __restrict__ plan, const float* __restrict__ u_ell, float lambda,
+    float* __restrict__ du_ell, float* __restrict__ dz_ell, float* __restrict__ dX, int M, int d, int T, int K,
+    int* __restrict__ ctr, uint32_t* status) {
   using Cfg = TokCfg<C, W>;
   constexpr int B = Cfg::B;
   constexpr int B2 = B > 1 ? B / 2 : 1;  // two rows (W_u, W_g) per unit in the dX phase
@@ -353,6 +407,7 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
   GroupSmem& g = gs[grp];
   const int nch = d >> 3;
   const int first = gtid;
+  int* turn = plan + kPlanHdr;
 
   // dH = dY_i . W_d[:, j] for the listed units, then dU (in g.c) and dZ (in g.c2)
   auto dh_phase = [&](long row, int ne) {
@@ -379,28 +434,31 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
     group_sync<W>(grp);
   };
 
-  for (;;) {
-    const long row = next_row<W>(ctr, grp, wi, lane, s_next);
-    if (row >= M) break;
-    if (row_ovf[row]) continue;
-    if (wi == 0) row_offsets(count, row, T, K, lane, g);
+  while (next_piece<W>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g)) {
+    const long row = g.row;
+    const int S = plan[1];
+    const int e0 = g.q * S;
+    const int ne = max(0, min(S, g.tot - e0));
+    build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, u_ell);
     group_sync<W>(grp);
-    float* dxr = dX + row * d;
-    int e0 = 0;
-    do {  // at least once: a row with no kept entry still writes dX = 0
-      const int ne = min(kListCap, g.tot - e0);
-      build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, u_ell);
-      group_sync<W>(grp);
-      dh_phase(row, ne);
-      float2 dx[C][4];
-      if (e0 == 0) zero_acc<C>(dx);
-      else load_acc<C, W, EXACT>(dxr, first, nch, dx);
-      gather_axpy<C, W, B2, EXACT>(g, ne, g.c, Wu, d, first, nch, dx);
-      gather_axpy<C, W, B2, EXACT>(g, ne, g.c2, Wg, d, first, nch, dx);
-      store_acc<C, W, EXACT>(dxr, first, nch, dx);
-      e0 += kListCap;
-      group_sync<W>(grp);  // the list is rebuilt for the next chunk or row
-    } while (e0 < g.tot);
+    dh_phase(row, ne);
+    float2 dx[C][4];
+    zero_acc<C>(dx);
+    gather_axpy<C, W, B2, EXACT>(g, ne, g.c, Wu, d, first, nch, dx);
+    gather_axpy<C, W, B2, EXACT>(g, ne, g.c2, Wg, d, first, nch, dx);
+    {
+      const int rw = g.row, q = g.q, P = g.P;
+      float* acc = dX + static_cast<long>(rw) * d;
+      if (P == 1) {
+        store_acc<C, W, EXACT>(acc, first, nch, dx);
+      } else {
+        turn_wait<W>(turn, rw, q, grp, gtid, status);
+        if (q > 0) add_acc<C, W, EXACT>(acc, first, nch, dx);
+        store_acc<C, W, EXACT>(acc, first, nch, dx);
+        turn_pass<W>(turn, rw, q, P, grp, gtid);
+      }
+    }
+    group_sync<W>(grp);  // the group's shared memory is rewritten for the next piece
   }
 }
 
@@ -438,10 +496,17 @@ void launch_bwd_cw(int M, cudaStream_t s, A... a) {
 
 }  // namespace
 
+int tok_groups(int M, int d) {
+  int C, W;
+  tok_shape(d, C, W);
+  const int G = (W > kTokWarps ? W : kTokWarps) / W;
+  return tok_grid(M, G) * G;
+}
+
 cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
-                               const uint16_t* count, const uint16_t* val, const uint8_t* col,
-                               const uint8_t* row_ovf, float* u_ell, uint16_t* Y, int M, int d, int f, int K,
-                               int* ctr, float* yacc, cudaStream_t s) {
+                               const uint16_t* count, const uint16_t* val, const uint8_t* col, int* plan,
+                               float* u_ell, uint16_t* Y, int M, int d, int f, int K, int* ctr, float* yacc,
+                               uint32_t* status, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
@@ -450,10 +515,10 @@ cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uin
   const int T = f / kTn;
   const bool exact = d / 8 == W * 32 * C;
 #define TWELL_FWD(CC, WW)                                                                                   \
-  (exact ? launch_fwd_cw<CC, WW, true>(M, s, X, W_u, W_dt, count, val, col, row_ovf, u_ell, Y, M, d, T, K, ctr, \
-                                       yacc)                                                                     \
-         : launch_fwd_cw<CC, WW, false>(M, s, X, W_u, W_dt, count, val, col, row_ovf, u_ell, Y, M, d, T, K, ctr,  \
-                                        yacc))
+  (exact ? launch_fwd_cw<CC, WW, true>(M, s, X, W_u, W_dt, count, val, col, plan, u_ell, Y, M, d, T, K, ctr, yacc, \
+                                       status)                                                                     \
+         : launch_fwd_cw<CC, WW, false>(M, s, X, W_u, W_dt, count, val, col, plan, u_ell, Y, M, d, T, K, ctr, yacc, \
+                                        status))
   if (W == 1 && C == 1) TWELL_FWD(1, 1);
   else if (W == 1 && C == 2) TWELL_FWD(2, 1);
   else if (W == 1 && C == 4) TWELL_FWD(4, 1);
@@ -467,8 +532,8 @@ cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uin
 
 cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const uint16_t* W_g,
                                const uint16_t* W_dt, const uint16_t* count, const uint16_t* val,
-                               const uint8_t* col, const uint8_t* row_ovf, const float* u_ell, float lambda,
-                               float* du_ell, float* dz_ell, float* dX, int M, int d, int f, int K, int* ctr,
+                               const uint8_t* col, int* plan, const float* u_ell, float lambda, float* du_ell,
+                               float* dz_ell, float* dX, int M, int d, int f, int K, int* ctr, uint32_t* status,
                                cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
@@ -478,10 +543,10 @@ cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const ui
   const int T = f / kTn;
   const bool exact = d / 8 == W * 32 * C;
 #define TWELL_BWD(CC, WW)                                                                                        \
-  (exact ? launch_bwd_cw<CC, WW, true>(M, s, dY, W_u, W_g, W_dt, count, val, col, row_ovf, u_ell, lambda, du_ell,  \
-                                       dz_ell, dX, M, d, T, K, ctr)                                              \
-         : launch_bwd_cw<CC, WW, false>(M, s, dY, W_u, W_g, W_dt, count, val, col, row_ovf, u_ell, lambda, du_ell, \
-                                        dz_ell, dX, M, d, T, K, ctr))
+  (exact ? launch_bwd_cw<CC, WW, true>(M, s, dY, W_u, W_g, W_dt, count, val, col, plan, u_ell, lambda, du_ell,  \
+                                       dz_ell, dX, M, d, T, K, ctr, status)                                    \
+         : launch_bwd_cw<CC, WW, false>(M, s, dY, W_u, W_g, W_dt, count, val, col, plan, u_ell, lambda, du_ell, \
+                                        dz_ell, dX, M, d, T, K, ctr, status))
   if (W == 1 && C == 1) TWELL_BWD(1, 1);
   else if (W == 1 && C == 2) TWELL_BWD(2, 1);
   else if (W == 1 && C == 4) TWELL_BWD(4, 1);

@@ -64,12 +64,9 @@ constexpr size_t kWsAlign = 256;
 
 size_t align_up(size_t x) { return (x + kWsAlign - 1) & ~(kWsAlign - 1); }
 
-// Rows of this shape can hold more kept entries than one token-kernel list.
-bool rows_can_exceed_list(int64_t f, int64_t K) { return (f / kTn) * K > kTokListCap; }
-
 struct WsLayout {
   size_t ctr = 0;   // row counter of the token kernels
-  size_t yacc = 0;  // fp32 partial Y of rows longer than one list of the token kernels
+  size_t yacc = 0;  // fp32 accumulator rows of rows split into several pieces
   size_t spill = 0, x_ovf = 0, h_ovf = 0, w_dt = 0;
   size_t dy_ovf = 0, duz = 0, du_ovf = 0, dz_ovf = 0, du_ell = 0, dz_ell = 0, row_slot = 0, block_cnt = 0, unit_tot = 0, unit_ptr = 0,
          csc_row = 0, csc_val = 0;
@@ -87,7 +84,7 @@ WsLayout ws_layout(twell_op op, int64_t M, int64_t d, int64_t f, int64_t K, int6
   const int64_t T = f / kTn;
   const int64_t cap1 = cap > 0 ? cap : 1;
   if (op == TWELL_OP_FWD || op == TWELL_OP_BWD) L.ctr = take(64);
-  if (op == TWELL_OP_FWD && rows_can_exceed_list(f, K)) L.yacc = take(static_cast<size_t>(M * d * 4));
+  if (op == TWELL_OP_FWD) L.yacc = take(static_cast<size_t>(M * d * 4));
   if (op == TWELL_OP_PACK || op == TWELL_OP_FWD) L.spill = take(static_cast<size_t>(M * f * 2));
   if (op == TWELL_OP_FWD) {
     L.x_ovf = take(static_cast<size_t>(cap1 * d * 2));
@@ -125,7 +122,8 @@ twell_status check_hybrid(const twell_hybrid* h, int64_t d_model) {
   const twell_status st = twell_query_support(h->M, d_model, h->d_ff, h->T_n, h->K, h->ovf_cap);
   if (st != TWELL_OK) return st;
   if (h->M == 0) return TWELL_OK;
-  const void* ptrs[] = {h->count, h->val, h->col, h->row_ovf, h->ovf_rows, h->n_ovf, h->g_ovf, h->status};
+  const void* ptrs[] = {h->count, h->val, h->col, h->row_ovf, h->ovf_rows, h->n_ovf, h->g_ovf, h->status,
+                        h->row_plan};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return TWELL_EINVAL;
   if ((h->u_ell && !aligned16(h->u_ell)) || (h->u_ovf && !aligned16(h->u_ovf))) return TWELL_EINVAL;
@@ -154,7 +152,8 @@ twell_status run_pack(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_
   cudaError_t e = launch_gate_pack(X, W_g, b_g, M, static_cast<int>(d), f, K, po, h->status, s);
   if (e != cudaSuccess) return TWELL_ECUDA;
   e = launch_route(h->count, h->val, h->col, po.spill, M, f, K, cap, h->row_ovf, h->ovf_rows, h->n_ovf, h->g_ovf,
-                   X_for_gather, static_cast<int>(d), x_ovf, h->status, s);
+                   X_for_gather, static_cast<int>(d), x_ovf, h->row_plan, tok_groups(M, static_cast<int>(d)),
+                   h->status, s);
   return cuda_status(e);
 }
 
@@ -187,6 +186,11 @@ twell_status twell_query_support(int64_t M, int64_t d_model, int64_t d_ff, int64
   if (d_ff % kTn != 0 || d_ff > kMaxTiles * kTn) return TWELL_EUNSUPPORTED;
   if (M > (int64_t(1) << 24) || ovf_cap > M) return TWELL_EUNSUPPORTED;
   return TWELL_OK;
+}
+
+size_t twell_plan_ints(int64_t M, int64_t d_ff, int64_t T_n, int64_t K) {
+  if (M < 0 || T_n != kTn || d_ff <= 0 || d_ff % kTn != 0 || K <= 0) return 0;
+  return static_cast<size_t>(plan_ints(M, d_ff / kTn, K));
 }
 
 size_t twell_workspace_bytes(twell_op op, int64_t M, int64_t d_model, int64_t d_ff, int64_t T_n, int64_t K,
@@ -243,8 +247,8 @@ twell_status twell_ffn_fwd(const uint16_t* X, const uint16_t* W_g, const uint16_
   uint16_t* x_ovf = at<uint16_t>(ws, L.x_ovf);
   st = run_pack(X, W_g, b_g, d, h, z_debug, ws, L, X, x_ovf, s);
   if (st != TWELL_OK) return st;
-  if (launch_ell_ffn_fwd(X, W_u, wdt, h->count, h->val, h->col, h->row_ovf, h->u_ell, Y, M, d, f, K,
-                         at<int>(ws, L.ctr), rows_can_exceed_list(f, K) ? at<float>(ws, L.yacc) : nullptr, s) != cudaSuccess)
+  if (launch_ell_ffn_fwd(X, W_u, wdt, h->count, h->val, h->col, h->row_plan, h->u_ell, Y, M, d, f, K,
+                         at<int>(ws, L.ctr), at<float>(ws, L.yacc), h->status, s) != cudaSuccess)
     return TWELL_ECUDA;
   return cuda_status(launch_ovf_fwd(x_ovf, W_u, W_d, h->g_ovf, h->ovf_rows, h->n_ovf, cap, d, f,
                                     at<uint16_t>(ws, L.h_ovf), h->u_ovf, Y, h->status, s));
@@ -290,8 +294,8 @@ twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_
   float* du_ell = at<float>(ws, L.du_ell);
   float* dz_ell = at<float>(ws, L.dz_ell);
   if (launch_gather_rows(dY, h->ovf_rows, h->n_ovf, cap, d, dy_ovf, s) != cudaSuccess) return TWELL_ECUDA;
-  if (launch_ell_ffn_bwd(dY, W_u, W_g, wdt, h->count, h->val, h->col, h->row_ovf, h->u_ell, lambda, du_ell, dz_ell,
-                         dX, M, d, f, K, at<int>(ws, L.ctr), s) != cudaSuccess)
+  if (launch_ell_ffn_bwd(dY, W_u, W_g, wdt, h->count, h->val, h->col, h->row_plan, h->u_ell, lambda, du_ell,
+                         dz_ell, dX, M, d, f, K, at<int>(ws, L.ctr), h->status, s) != cudaSuccess)
     return TWELL_ECUDA;
   float* du_ovf = at<float>(ws, L.du_ovf);
   float* dz_ovf = at<float>(ws, L.dz_ovf);

@@ -18,6 +18,22 @@ constexpr int kMaxTiles = 128;     // d_ff <= 16384
 constexpr int kMaxDModel = 16384;  // 128 threads x 16 chunks x 8 bf16
 constexpr int kTokListCap = 256;   // kept entries per list chunk of the token kernels
 
+// Row plan (twell_hybrid::row_plan, int32): the work of the token kernels as
+// pieces of at most S kept entries of one non-overflow row.
+//   [0] number of pieces, [1] S, [2] kept entries of non-overflow rows, [3] 0
+//   [kPlanHdr, kPlanHdr + M)  per-row turnstile words (0 between launches;
+//                             the routing step parks the kept counts there)
+//   then (row, q) int pairs, piece q of row, ascending rows then q
+// S = clamp(ceil(kept / resident groups), kPieceMin, kTokListCap), so the
+// pieces number at most M + max(groups, M * T * K / kTokListCap).
+constexpr int kPlanHdr = 4;
+constexpr int kPieceMin = 32;
+constexpr long kPlanGroupsCap = 65536;  // bound on resident token groups of any device
+inline long plan_ints(long M, long T, long K) {
+  const long spill = (M * T * K + kTokListCap - 1) / kTokListCap;
+  return kPlanHdr + M + 2 * (M + (spill > kPlanGroupsCap ? spill : kPlanGroupsCap));
+}
+
 // ------------------------------------------------------------ device helpers
 
 __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bits) {
@@ -84,11 +100,16 @@ cudaError_t launch_gate_pack(const uint16_t* X, const uint16_t* W_g, const uint1
                              int K, const PackOut& out, uint32_t* status, cudaStream_t s);
 
 // Row routing: flags, ascending overflow list, dense backup rows (and the
-// gathered X rows of overflow rows when x_ovf != nullptr).
+// gathered X rows of overflow rows when x_ovf != nullptr), and the row plan of
+// the token kernels for `groups` resident token groups.
 cudaError_t launch_route(const uint16_t* count, const uint16_t* val, const uint8_t* col, const uint16_t* spill,
                          int M, int f, int K, int cap, uint8_t* row_ovf, int* ovf_rows, int* n_ovf,
-                         uint16_t* g_ovf, const uint16_t* X, int d, uint16_t* x_ovf, uint32_t* status,
-                         cudaStream_t s);
+                         uint16_t* g_ovf, const uint16_t* X, int d, uint16_t* x_ovf, int* plan, int groups,
+                         uint32_t* status, cudaStream_t s);
+
+// Resident token groups of the token kernels for M rows of width d (the
+// launch shape they use); sizes the pieces of the row plan.
+int tok_groups(int M, int d);
 
 // out[s][:] = in[rows[s]][:] for s < n_ovf[0] (bf16 rows of width d).
 cudaError_t launch_gather_rows(const uint16_t* in, const int* rows, const int* n_ovf, int cap, int d,
@@ -96,14 +117,13 @@ cudaError_t launch_gather_rows(const uint16_t* in, const int* rows, const int* n
 
 cudaError_t launch_transpose_bf16(const uint16_t* in, int rows, int cols, uint16_t* out, cudaStream_t s);
 
-// Fused sparse up + down over the ELL rows (overflow rows are skipped).
-// ctr: one int of device scratch (the row counter), zeroed by the launcher;
-// yacc: [M][d] fp32 scratch for rows with more than kTokListCap kept entries
-// (may be null when (d_ff / kTn) * K <= kTokListCap).
+// Fused sparse up + down over the pieces of the row plan (ELL rows only).
+// ctr: one int of device scratch (the piece counter), zeroed by the launcher;
+// yacc: [M][d] fp32 accumulator rows for rows split into several pieces.
 cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
-                               const uint16_t* count, const uint16_t* val, const uint8_t* col,
-                               const uint8_t* row_ovf, float* u_ell, uint16_t* Y, int M, int d, int f, int K,
-                               int* ctr, float* yacc, cudaStream_t s);
+                               const uint16_t* count, const uint16_t* val, const uint8_t* col, int* plan,
+                               float* u_ell, uint16_t* Y, int M, int d, int f, int K, int* ctr, float* yacc,
+                               uint32_t* status, cudaStream_t s);
 
 // Dense backup forward for overflow rows: H = bf16(G * (X_ovf W_u^T)) then
 // Y[ovf_rows] = bf16(H W_d^T).
@@ -111,12 +131,12 @@ cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uin
                            const uint16_t* g_ovf, const int* ovf_rows, const int* n_ovf, int cap, int d, int f,
                            uint16_t* h_ovf, float* u_ovf, uint16_t* Y, uint32_t* status, cudaStream_t s);
 
-// Sparse backward over the ELL rows: dH at kept actives, dU, dZ (stored per
-// slot) and the rows of dX.
+// Sparse backward over the pieces of the row plan: dH at kept actives, dU,
+// dZ (stored per slot) and the rows of dX.
 cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const uint16_t* W_g,
                                const uint16_t* W_dt, const uint16_t* count, const uint16_t* val,
-                               const uint8_t* col, const uint8_t* row_ovf, const float* u_ell, float lambda,
-                               float* du_ell, float* dz_ell, float* dX, int M, int d, int f, int K, int* ctr,
+                               const uint8_t* col, int* plan, const float* u_ell, float lambda, float* du_ell,
+                               float* dz_ell, float* dX, int M, int d, int f, int K, int* ctr, uint32_t* status,
                                cudaStream_t s);
 
 // Dense backup backward for overflow rows: dU, dZ (fp32, and bf16 [dU | dZ] as

@@ -56,7 +56,8 @@ extern "C" TWELL_API twell_status twell_pack_noalloc(const uint16_t* X, const ui
   if (static_cast<uint64_t>(h->M) * static_cast<uint64_t>(h->d_ff) * sizeof(uint16_t) >
       static_cast<uint64_t>(TWELL_NOALLOC_SCRATCH_BYTES))
     return TWELL_EWORKSPACE;
-  const void* ptrs[] = {X, W_g, b_g, h->count, h->val, h->col, h->row_ovf, h->ovf_rows, h->n_ovf, h->g_ovf, h->status};
+  const void* ptrs[] = {X,          W_g,         b_g,      h->count, h->val,    h->col,
+                        h->row_ovf, h->ovf_rows, h->n_ovf, h->g_ovf, h->status, h->row_plan};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return TWELL_EINVAL;
   if (z_debug && !aligned16(z_debug)) return TWELL_EINVAL;
@@ -68,7 +69,7 @@ extern "C" TWELL_API twell_status twell_pack_noalloc(const uint16_t* X, const ui
   PackOut po{h->count, h->val, h->col, scratch, z_debug};
   if (launch_gate_pack(X, W_g, b_g, M, d, f, K, po, h->status, s) != cudaSuccess) return TWELL_ECUDA;
   if (launch_route(h->count, h->val, h->col, scratch, M, f, K, h->ovf_cap, h->row_ovf, h->ovf_rows, h->n_ovf,
-                   h->g_ovf, nullptr, d, nullptr, h->status, s) != cudaSuccess)
+                   h->g_ovf, nullptr, d, nullptr, h->row_plan, tok_groups(M, d), h->status, s) != cudaSuccess)
     return TWELL_ECUDA;
   return TWELL_OK;
 }

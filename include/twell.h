@@ -89,6 +89,15 @@ typedef enum twell_status {
  * u_ell / u_ovf are written by twell_ffn_fwd when non-NULL and read by
  * twell_ffn_bwd (which requires both): the up projection u at the kept ELL
  * slots of non-overflow rows, and the dense u rows of stored overflow rows.
+ *
+ * row_plan ([twell_plan_ints(M, d_ff, T_n, K)] int32, zero-filled by the
+ * caller when allocated) is the schedule of the sparse kernels, written by the
+ * routing step of twell_pack / twell_ffn_fwd and read by twell_ffn_fwd and
+ * twell_ffn_bwd: the kept entries of every non-overflow row split into pieces
+ * of at most S entries, S sized from the batch's total so that heavy rows are
+ * spread over the whole GPU. Its contents are internal; the library leaves its
+ * per-row turnstile words at zero between calls. The same d_model must be used
+ * for the pack and the passes that read the plan.
  */
 typedef struct twell_hybrid {
   int32_t M;         /* tokens (rows) */
@@ -106,6 +115,7 @@ typedef struct twell_hybrid {
   float* u_ell;      /* [M][T][K], nullable */
   float* u_ovf;      /* [max(ovf_cap,1)][d_ff], nullable */
   uint32_t* status;  /* [1] device status word (TWELL_STATUS_* bits), never cleared by kernels */
+  int32_t* row_plan; /* [twell_plan_ints(M, d_ff, T_n, K)], zero-filled at allocation */
 } twell_hybrid;
 
 /* Which call a workspace is sized for. */
@@ -117,6 +127,10 @@ TWELL_API const char* twell_status_string(twell_status s);
 /* Host-only check of a shape against the supported set; enqueues nothing. */
 TWELL_API twell_status twell_query_support(int64_t M, int64_t d_model, int64_t d_ff, int64_t T_n, int64_t K,
                                  int64_t ovf_cap);
+
+/* Elements (int32) of twell_hybrid::row_plan for this shape (0 for an invalid
+ * one): 4 + M + 2 * (M + max(65536, ceil(M * (d_ff / T_n) * K / 256))). */
+TWELL_API size_t twell_plan_ints(int64_t M, int64_t d_ff, int64_t T_n, int64_t K);
 
 /* Workspace bytes that `op` needs for this shape (0 for an unsupported shape).
  * For TWELL_OP_FWD and TWELL_OP_BWD this includes room for a transposed W_d,

@@ -45,9 +45,20 @@ def test_library_exports_every_declared_symbol(tw):
 
 
 def test_hybrid_struct_matches_header(tw):
-    # five int32 fields, 4 bytes of padding, ten pointers
-    assert ctypes.sizeof(tw.TwellHybrid) == 24 + 10 * 8
+    # five int32 fields, 4 bytes of padding, eleven pointers
+    assert ctypes.sizeof(tw.TwellHybrid) == 24 + 11 * 8
     assert tw.TwellHybrid.count.offset == 24
+    assert tw.TwellHybrid.row_plan.offset == 24 + 10 * 8
+
+
+def test_plan_ints(tw):
+    L = tw.lib()
+    # 4 + M + 2 * (M + max(65536, ceil(M * T * K / 256)))
+    assert L.twell_plan_ints(4096, 8192, 128, 8) == 4 + 4096 + 2 * (4096 + 65536)
+    big = 65536 * 112 * 64 // 256
+    assert L.twell_plan_ints(65536, 14336, 128, 64) == 4 + 65536 + 2 * (65536 + big)
+    assert L.twell_plan_ints(0, 8192, 128, 8) == 4 + 2 * 65536
+    assert L.twell_plan_ints(16, 8192, 64, 8) == 0
 
 
 def test_query_support(tw):
@@ -77,21 +88,21 @@ def test_workspace_sizes(tw):
 
 def test_host_side_errors(tw):
     L = tw.lib()
-    h = tw.TwellHybrid(64, 1024, 128, 8, 64, *([None] * 10))
+    h = tw.TwellHybrid(64, 1024, 128, 8, 64, *([None] * 11))
     # null descriptor, null arrays, unsupported shape, missing workspace
     assert L.twell_pack(None, None, None, 256, None, None, None, 0, None) == 1
     assert L.twell_pack(None, None, None, 256, ctypes.byref(h), None, None, 0, None) == 1
-    bad = tw.TwellHybrid(64, 1024, 64, 8, 64, *([None] * 10))
+    bad = tw.TwellHybrid(64, 1024, 64, 8, 64, *([None] * 11))
     assert L.twell_pack(None, None, None, 256, ctypes.byref(bad), None, None, 0, None) == 2
     fake = 1 << 20  # aligned non-null addresses; never dereferenced by these checks
-    h2 = tw.TwellHybrid(64, 1024, 128, 8, 64, *([fake] * 10))
+    h2 = tw.TwellHybrid(64, 1024, 128, 8, 64, *([fake] * 11))
     p = ctypes.c_void_p(fake)
     assert L.twell_pack(p, p, p, 256, ctypes.byref(h2), None, None, 0, None) == 6
     assert L.twell_pack(p, p, p, 256, ctypes.byref(h2), None, ctypes.c_void_p(fake + 8), 1 << 30, None) == 6
     mis = ctypes.c_void_p(fake + 2)
     assert L.twell_ffn_fwd(mis, p, p, p, p, None, 256, p, ctypes.byref(h2), None, None, 0, None) == 1
     # empty batch forward: nothing to do, nothing touched
-    h0 = tw.TwellHybrid(0, 1024, 128, 8, 0, *([None] * 10))
+    h0 = tw.TwellHybrid(0, 1024, 128, 8, 0, *([None] * 11))
     assert L.twell_ffn_fwd(None, None, None, None, None, None, 256, None, ctypes.byref(h0), None, None, 0, None) == 0
     assert L.twell_transpose_wd(None, 256, 1024, None, None) == 1
 

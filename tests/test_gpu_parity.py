@@ -13,8 +13,8 @@ import numpy as np
 import pytest
 
 from synthetic import WORKLOADS, Workload, make_inputs
-from twell_testlib import (assert_active_set, assert_matches_oracle, assert_pack_equal, bits_of, f32_of_bits,
-                           gpu_gmat, state_to_numpy, to_dev)
+from twell_testlib import (assert_active_set, assert_matches_oracle, assert_pack_equal, assert_plan_valid, bits_of,
+                           f32_of_bits, gpu_gmat, state_to_numpy, to_dev)
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -91,6 +91,11 @@ CASES = {
 }
 
 
+# cases whose plan splits some rows into several pieces (the ordered
+# accumulation across pieces is exercised)
+SPLIT_CASES = ("k64", "long_rows_w2", "multi_tile")
+
+
 @pytest.mark.parametrize("name", sorted(CASES))
 def test_fwd_bwd_small(tw, orc, name):
     M, d, f, K, act, rs, seed = CASES[name]
@@ -98,10 +103,14 @@ def test_fwd_bwd_small(tw, orc, name):
     inp = make_inputs(w)
     D, Y, st, z = _run_fwd(tw, inp, w)
     p, flips, _ = _check_fwd(orc, inp, w, Y, st, z)
+    plan = assert_plan_valid(st)
+    if name in SPLIT_CASES:
+        assert plan["split_rows"] > 0, "this case should split rows into several pieces"
     for lam in (0.0, 1e-3):
         g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=lam)
         torch.cuda.synchronize()
         _check_bwd(orc, inp, g, gpu_gmat(p, M, f, 128, K), lam, name)
+        assert_plan_valid(st)
 
 
 def test_degenerate_all_inactive(tw, orc):
@@ -206,6 +215,7 @@ def test_uniform_full_size(tw, orc):
     rows = _sample_rows(w.M, 256, 0)
     p, flips, stats = _check_fwd(orc, inp, w, Y, st, z, rows=rows)
     assert p["n_ovf_total"] == 0
+    assert assert_plan_valid(st)["split_rows"] == 0  # 1% i.i.d. rows are short: one piece each
 
 
 def test_heavy_tail_full_size(tw, orc):
@@ -219,7 +229,12 @@ def test_heavy_tail_full_size(tw, orc):
     assert cnt.max() / cnt.mean() >= 10
     rng = np.random.default_rng(1)
     ovf_sample = rng.choice(p["ovf_rows"], size=min(64, p["n_ovf"]), replace=False)
-    rows = _sample_rows(w.M, 128, 1, extra=ovf_sample)
+    plan = assert_plan_valid(st)
+    assert plan["split_rows"] > 0  # the heavy ELL rows are split into pieces
+    pieces = st.row_plan.cpu().numpy()[4 + w.M:4 + w.M + 2 * plan["pieces"]].reshape(-1, 2)
+    split = np.unique(pieces[pieces[:, 1] == 1, 0])
+    split_sample = rng.choice(split, size=min(32, split.size), replace=False)
+    rows = _sample_rows(w.M, 128, 1, extra=np.concatenate([ovf_sample, split_sample]))
     _check_fwd(orc, inp, w, Y, st, z, rows=rows)
 
 

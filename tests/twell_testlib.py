@@ -63,6 +63,29 @@ def assert_pack_equal(gpu: dict, ref: dict) -> None:
     assert np.array_equal(gpu["g_ovf"][:n], ref["g_ovf"][:n]), "dense backup rows differ"
 
 
+def assert_plan_valid(st, groups_hint=None) -> dict:
+    """The row plan of the sparse kernels, checked on the host from the pack.
+
+    Every non-overflow row appears as pieces q = 0..P-1 with P = max(1,
+    ceil(kept / S)), rows ascending; overflow rows have no piece; S lies in
+    [32, 256]; every turnstile word is back at zero between passes.
+    """
+    plan = st.row_plan.cpu().numpy()
+    M, K = st.M, st.K
+    npieces, S, total = int(plan[0]), int(plan[1]), int(plan[2])
+    count = st.count.cpu().numpy().view(np.uint16).astype(np.int64)
+    row_ovf = st.row_ovf.cpu().numpy()[:M]
+    kept = np.minimum(count, K).sum(axis=1)
+    assert 32 <= S <= 256, S
+    assert total == int(kept[row_ovf == 0].sum())
+    assert not plan[4:4 + M].any(), "turnstile words must be zero between passes"
+    pieces = plan[4 + M:4 + M + 2 * npieces].reshape(-1, 2)
+    want = [(r, q) for r in range(M) if not row_ovf[r]
+            for q in range(max(1, -(-int(kept[r]) // S)))]
+    assert [tuple(x) for x in pieces.tolist()] == want
+    return dict(pieces=npieces, S=S, total=total, split_rows=int(sum(1 for r, q in want if q == 1)))
+
+
 def gpu_mask(p: dict, M: int, f: int, T_n: int, K: int) -> np.ndarray:
     """Active set [M, f] as the GPU's hybrid representation records it."""
     T = f // T_n
