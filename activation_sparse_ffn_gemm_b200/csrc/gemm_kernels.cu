@@ -55,6 +55,7 @@ struct EpiTwell {
   };
   // per-thread slot staging: K bf16 values + K column bytes (K <= 64)
   static constexpr int SMEM_BYTES = 128 * kMaxK * 3;
+  static constexpr bool kSplitK = false;
 
   __device__ static void run(const Args& a, int m0, int n0, int M_eff, int /*N*/, int r, uint32_t taddr,
                              uint8_t* smem) {
@@ -152,7 +153,35 @@ struct EpiTwell {
   }
 };
 
+// The dense-backup epilogues are element-wise: apply8 handles eight columns
+// [n, n + 8) of accumulator row `row` (a valid row). run() feeds it from
+// tensor memory; the split-K reduction feeds it the summed partials.
+template <class Epi>
+__device__ __forceinline__ void run_apply8(const typename Epi::Args& a, int m0, int n0, int M_eff, int N, int r,
+                                           uint32_t taddr) {
+  const int row = m0 + r;
+  const bool valid = row < M_eff;
+#pragma unroll 1
+  for (int ch = 0; ch < 8; ++ch) {
+    const int n = n0 + ch * 32;
+    if (n >= N) break;
+    uint32_t v[32];
+    __syncwarp();
+    tmem_ld_32x32b_x32(taddr + ch * 32, v);
+    tmem_wait_ld();
+    if (!valid) continue;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float acc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = __uint_as_float(v[q * 8 + e]);
+      Epi::apply8(a, row, n + q * 8, acc);
+    }
+  }
+}
+
 // ---------------------------------------- dense backup forward, first GEMM
+// u = X_ovf W_u^T (accumulator); H = bf16(g * u); u kept in fp32 when asked.
 struct EpiGateMul {
   struct Args {
     const uint16_t* g;  // [cap][f] bf16 ReLU(z)
@@ -161,39 +190,24 @@ struct EpiGateMul {
     int f;
   };
   static constexpr int SMEM_BYTES = 0;
-  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
-    const int row = m0 + r;
-    const bool valid = row < M_eff;
-#pragma unroll 1
-    for (int ch = 0; ch < 8; ++ch) {
-      const int n = n0 + ch * 32;
-      if (n >= N) break;
-      uint32_t v[32];
-      __syncwarp();
-      tmem_ld_32x32b_x32(taddr + ch * 32, v);
-      tmem_wait_ld();
-      if (!valid) continue;
-      const size_t off = static_cast<size_t>(row) * a.f + n;
-      const uint4* gp = reinterpret_cast<const uint4*>(a.g + off);
-      uint4* hp = reinterpret_cast<uint4*>(a.H + off);
+  static constexpr bool kSplitK = true;
+  __device__ static void apply8(const Args& a, int row, int n, const float (&u)[8]) {
+    const size_t off = static_cast<size_t>(row) * a.f + n;
+    float g8[8];
+    unpack8(*reinterpret_cast<const uint4*>(a.g + off), g8);
+    float h[8];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float g8[8];
-        unpack8(gp[q], g8);
-        float h[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) h[e] = g8[e] * __uint_as_float(v[q * 8 + e]);
-        hp[q] = make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]), pack_bf16x2(h[4], h[5]),
-                           pack_bf16x2(h[6], h[7]));
-      }
-      if (a.u_save) {
-        float4* up = reinterpret_cast<float4*>(a.u_save + off);
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          up[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
-                              __uint_as_float(v[4 * q + 3]));
-      }
+    for (int e = 0; e < 8; ++e) h[e] = g8[e] * u[e];
+    *reinterpret_cast<uint4*>(a.H + off) = make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]),
+                                                      pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
+    if (a.u_save) {
+      float4* up = reinterpret_cast<float4*>(a.u_save + off);
+      up[0] = make_float4(u[0], u[1], u[2], u[3]);
+      up[1] = make_float4(u[4], u[5], u[6], u[7]);
     }
+  }
+  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
+    run_apply8<EpiGateMul>(a, m0, n0, M_eff, N, r, taddr);
   }
 };
 
@@ -205,27 +219,13 @@ struct EpiScatterBf16 {
     int ld;
   };
   static constexpr int SMEM_BYTES = 0;
+  static constexpr bool kSplitK = true;
+  __device__ static void apply8(const Args& a, int row, int n, const float (&v)[8]) {
+    *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(a.rows[row]) * a.ld + n) =
+        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+  }
   __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
-    const int row = m0 + r;
-    const bool valid = row < M_eff;
-    const int dst = valid ? a.rows[row] : 0;
-#pragma unroll 1
-    for (int ch = 0; ch < 8; ++ch) {
-      const int n = n0 + ch * 32;
-      if (n >= N) break;
-      uint32_t v[32];
-      __syncwarp();
-      tmem_ld_32x32b_x32(taddr + ch * 32, v);
-      tmem_wait_ld();
-      if (!valid) continue;
-      uint4* p = reinterpret_cast<uint4*>(a.out + static_cast<size_t>(dst) * a.ld + n);
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        p[q] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
-                          pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
-                          pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
-                          pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
-    }
+    run_apply8<EpiScatterBf16>(a, m0, n0, M_eff, N, r, taddr);
   }
 };
 
@@ -236,29 +236,20 @@ struct EpiScatterF32 {
     int ld;
   };
   static constexpr int SMEM_BYTES = 0;
+  static constexpr bool kSplitK = true;
+  __device__ static void apply8(const Args& a, int row, int n, const float (&v)[8]) {
+    float4* p = reinterpret_cast<float4*>(a.out + static_cast<size_t>(a.rows[row]) * a.ld + n);
+    p[0] = make_float4(v[0], v[1], v[2], v[3]);
+    p[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
   __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
-    const int row = m0 + r;
-    const bool valid = row < M_eff;
-    const int dst = valid ? a.rows[row] : 0;
-#pragma unroll 1
-    for (int ch = 0; ch < 8; ++ch) {
-      const int n = n0 + ch * 32;
-      if (n >= N) break;
-      uint32_t v[32];
-      __syncwarp();
-      tmem_ld_32x32b_x32(taddr + ch * 32, v);
-      tmem_wait_ld();
-      if (!valid) continue;
-      float4* p = reinterpret_cast<float4*>(a.out + static_cast<size_t>(dst) * a.ld + n);
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        p[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
-                           __uint_as_float(v[4 * q + 3]));
-    }
+    run_apply8<EpiScatterF32>(a, m0, n0, M_eff, N, r, taddr);
   }
 };
 
 // -------------------------------------- dense backup backward, dH epilogue
+// dH (accumulator) -> dU = dH g, dZ = (dH u + lambda) [g > 0], as fp32 (weight
+// gradients) and bf16 [dU | dZ] (the dX GEMM's operand).
 struct EpiBwdDH {
   struct Args {
     const uint16_t* g;  // [cap][f]
@@ -270,48 +261,34 @@ struct EpiBwdDH {
     int f;
   };
   static constexpr int SMEM_BYTES = 0;
-  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
-    const int row = m0 + r;
-    const bool valid = row < M_eff;
-#pragma unroll 1
-    for (int ch = 0; ch < 8; ++ch) {
-      const int n = n0 + ch * 32;
-      if (n >= N) break;
-      uint32_t v[32];
-      __syncwarp();
-      tmem_ld_32x32b_x32(taddr + ch * 32, v);
-      tmem_wait_ld();
-      if (!valid) continue;
-      const size_t off = static_cast<size_t>(row) * a.f + n;
-      const uint4* gp = reinterpret_cast<const uint4*>(a.g + off);
-      const float4* up = reinterpret_cast<const float4*>(a.u + off);
-      uint4* dup = reinterpret_cast<uint4*>(a.duz + static_cast<size_t>(row) * 2 * a.f + n);
-      uint4* dzp = reinterpret_cast<uint4*>(a.duz + static_cast<size_t>(row) * 2 * a.f + a.f + n);
+  static constexpr bool kSplitK = true;
+  __device__ static void apply8(const Args& a, int row, int n, const float (&dh)[8]) {
+    const size_t off = static_cast<size_t>(row) * a.f + n;
+    float g8[8];
+    unpack8(*reinterpret_cast<const uint4*>(a.g + off), g8);
+    const float4 u0 = reinterpret_cast<const float4*>(a.u + off)[0];
+    const float4 u1 = reinterpret_cast<const float4*>(a.u + off)[1];
+    const float u8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    float du[8], dz[8];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float g8[8];
-        unpack8(gp[q], g8);
-        const float4 u0 = up[2 * q], u1 = up[2 * q + 1];
-        const float u8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-        float du[8], dz[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float dh = __uint_as_float(v[q * 8 + e]);
-          du[e] = dh * g8[e];
-          dz[e] = g8[e] > 0.f ? fmaf(dh, u8[e], a.lambda) : 0.f;
-        }
-        dup[q] = make_uint4(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]), pack_bf16x2(du[4], du[5]),
-                            pack_bf16x2(du[6], du[7]));
-        float4* du32 = reinterpret_cast<float4*>(a.du + off) + 2 * q;
-        float4* dz32 = reinterpret_cast<float4*>(a.dz + off) + 2 * q;
-        du32[0] = make_float4(du[0], du[1], du[2], du[3]);
-        du32[1] = make_float4(du[4], du[5], du[6], du[7]);
-        dz32[0] = make_float4(dz[0], dz[1], dz[2], dz[3]);
-        dz32[1] = make_float4(dz[4], dz[5], dz[6], dz[7]);
-        dzp[q] = make_uint4(pack_bf16x2(dz[0], dz[1]), pack_bf16x2(dz[2], dz[3]), pack_bf16x2(dz[4], dz[5]),
-                            pack_bf16x2(dz[6], dz[7]));
-      }
+    for (int e = 0; e < 8; ++e) {
+      du[e] = dh[e] * g8[e];
+      dz[e] = g8[e] > 0.f ? fmaf(dh[e], u8[e], a.lambda) : 0.f;
     }
+    uint16_t* drow = a.duz + static_cast<size_t>(row) * 2 * a.f;
+    *reinterpret_cast<uint4*>(drow + n) = make_uint4(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]),
+                                                     pack_bf16x2(du[4], du[5]), pack_bf16x2(du[6], du[7]));
+    *reinterpret_cast<uint4*>(drow + a.f + n) = make_uint4(pack_bf16x2(dz[0], dz[1]), pack_bf16x2(dz[2], dz[3]),
+                                                           pack_bf16x2(dz[4], dz[5]), pack_bf16x2(dz[6], dz[7]));
+    float4* du32 = reinterpret_cast<float4*>(a.du + off);
+    float4* dz32 = reinterpret_cast<float4*>(a.dz + off);
+    du32[0] = make_float4(du[0], du[1], du[2], du[3]);
+    du32[1] = make_float4(du[4], du[5], du[6], du[7]);
+    dz32[0] = make_float4(dz[0], dz[1], dz[2], dz[3]);
+    dz32[1] = make_float4(dz[4], dz[5], dz[6], dz[7]);
+  }
+  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
+    run_apply8<EpiBwdDH>(a, m0, n0, M_eff, N, r, taddr);
   }
 };
 
@@ -331,9 +308,26 @@ cudaError_t launch_gate_pack(const uint16_t* X, const uint16_t* W_g, const uint1
   return launch_umma_gemm<EpiTwell, 256, false, kStages>("gate_pack_gemm", ta, tb, ta, tb, shp, ea, s);
 }
 
+namespace {
+// Split-K settings of a dense-backup GEMM with `cap` rows of capacity.
+void use_split(GemmShape& shp, const SplitKBuffers& sk, int cap) {
+  shp.partial = sk.partial;
+  shp.arrivals = sk.arrivals;
+  shp.split_rows = cap < kSplitRows ? cap : kSplitRows;
+  shp.split_max = kSplitMax;
+}
+}  // namespace
+
+size_t splitk_partial_floats(int cap, int d, int f) {
+  const size_t rows = static_cast<size_t>(cap < kSplitRows ? cap : kSplitRows);
+  return static_cast<size_t>(kSplitMax) * rows * static_cast<size_t>(d > f ? d : f);
+}
+size_t splitk_arrival_words() { return kSplitTiles; }
+
 cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uint16_t* W_d,
                            const uint16_t* g_ovf, const int* ovf_rows, const int* n_ovf, int cap, int d, int f,
-                           uint16_t* h_ovf, float* u_ovf, uint16_t* Y, uint32_t* status, cudaStream_t s) {
+                           uint16_t* h_ovf, float* u_ovf, uint16_t* Y, const SplitKBuffers& sk, uint32_t* status,
+                           cudaStream_t s) {
   if (cap <= 0) return cudaSuccess;
   CUtensorMap ta, tb, ta2, tb2;
   if (!make_tmap_bf16(&ta, x_ovf, d, cap, static_cast<uint64_t>(d) * 2, kBK, kBM) ||
@@ -342,10 +336,12 @@ cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uin
       !make_tmap_bf16(&tb2, W_d, f, d, static_cast<uint64_t>(f) * 2, kBK, 256))
     return cudaErrorInvalidValue;
   GemmShape s1{cap, n_ovf, f, d, 0, status};
+  use_split(s1, sk, cap);
   EpiGateMul::Args e1{g_ovf, h_ovf, u_ovf, f};
   cudaError_t e = launch_umma_gemm<EpiGateMul, 256, false, kStages>("ovf_up_gemm", ta, tb, ta, tb, s1, e1, s);
   if (e != cudaSuccess) return e;
   GemmShape s2{cap, n_ovf, d, f, 0, status};
+  use_split(s2, sk, cap);
   EpiScatterBf16::Args e2{ovf_rows, Y, d};
   return launch_umma_gemm<EpiScatterBf16, 256, false, kStages>("ovf_down_gemm", ta2, tb2, ta2, tb2, s2, e2, s);
 }
@@ -353,7 +349,8 @@ cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uin
 cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const uint16_t* W_u,
                            const uint16_t* W_g, const uint16_t* g_ovf, const float* u_ovf, float lambda,
                            const int* ovf_rows, const int* n_ovf, int cap, int d, int f, uint16_t* duz_ovf,
-                           float* du_ovf, float* dz_ovf, float* dX, uint32_t* status, cudaStream_t s) {
+                           float* du_ovf, float* dz_ovf, float* dX, const SplitKBuffers& sk, uint32_t* status,
+                           cudaStream_t s) {
   if (cap <= 0) return cudaSuccess;
   CUtensorMap ta, tb, tdu, tdz, twu, twg;
   // dH = dY_ovf W_d: B = W_dt [f][d] (K-major)
@@ -366,10 +363,12 @@ cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const u
       !make_tmap_bf16(&twg, W_g, d, f, static_cast<uint64_t>(d) * 2, 64, kBK))
     return cudaErrorInvalidValue;
   GemmShape s1{cap, n_ovf, f, d, 0, status};
+  use_split(s1, sk, cap);
   EpiBwdDH::Args e1{g_ovf, u_ovf, duz_ovf, du_ovf, dz_ovf, lambda, f};
   cudaError_t e = launch_umma_gemm<EpiBwdDH, 256, false, kStages>("ovf_dh_gemm", ta, tb, ta, tb, s1, e1, s);
   if (e != cudaSuccess) return e;
   GemmShape s2{cap, n_ovf, d, f, f, status};
+  use_split(s2, sk, cap);
   EpiScatterF32::Args e2{ovf_rows, dX, d};
   return launch_umma_gemm<EpiScatterF32, 256, true, kStages>("ovf_dx_gemm", tdu, twu, tdz, twg, s2, e2, s);
 }

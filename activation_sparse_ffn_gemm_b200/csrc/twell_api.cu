@@ -23,6 +23,15 @@ int device_sm_count() {
   return v;
 }
 
+unsigned long long next_gemm_epoch() {
+  static std::atomic<unsigned long long> next{1};
+  constexpr unsigned long long kMask = (1ull << 56) - 1;
+  for (;;) {
+    const unsigned long long e = next.fetch_add(1, std::memory_order_relaxed) & kMask;
+    if (e != 0) return e;
+  }
+}
+
 namespace {
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -67,6 +76,7 @@ size_t align_up(size_t x) { return (x + kWsAlign - 1) & ~(kWsAlign - 1); }
 struct WsLayout {
   size_t ctr = 0;   // row counter of the token kernels
   size_t yacc = 0;  // fp32 accumulator rows of rows split into several pieces
+  size_t sk_partial = 0, sk_arrivals = 0;  // split-K scratch of the dense-backup GEMMs
   size_t spill = 0, x_ovf = 0, h_ovf = 0, w_dt = 0;
   size_t dy_ovf = 0, duz = 0, du_ovf = 0, dz_ovf = 0, du_ell = 0, dz_ell = 0, row_slot = 0, block_cnt = 0, unit_tot = 0, unit_ptr = 0,
          csc_row = 0, csc_val = 0;
@@ -85,6 +95,10 @@ WsLayout ws_layout(twell_op op, int64_t M, int64_t d, int64_t f, int64_t K, int6
   const int64_t cap1 = cap > 0 ? cap : 1;
   if (op == TWELL_OP_FWD || op == TWELL_OP_BWD) L.ctr = take(64);
   if (op == TWELL_OP_FWD) L.yacc = take(static_cast<size_t>(M * d * 4));
+  if (op == TWELL_OP_FWD || op == TWELL_OP_BWD) {
+    L.sk_partial = take(splitk_partial_floats(static_cast<int>(cap1), static_cast<int>(d), static_cast<int>(f)) * 4);
+    L.sk_arrivals = take(splitk_arrival_words() * 8);
+  }
   if (op == TWELL_OP_PACK || op == TWELL_OP_FWD) L.spill = take(static_cast<size_t>(M * f * 2));
   if (op == TWELL_OP_FWD) {
     L.x_ovf = take(static_cast<size_t>(cap1 * d * 2));
@@ -250,8 +264,9 @@ twell_status twell_ffn_fwd(const uint16_t* X, const uint16_t* W_g, const uint16_
   if (launch_ell_ffn_fwd(X, W_u, wdt, h->count, h->val, h->col, h->row_plan, h->u_ell, Y, M, d, f, K,
                          at<int>(ws, L.ctr), at<float>(ws, L.yacc), h->status, s) != cudaSuccess)
     return TWELL_ECUDA;
+  const SplitKBuffers sk{at<float>(ws, L.sk_partial), at<unsigned long long>(ws, L.sk_arrivals)};
   return cuda_status(launch_ovf_fwd(x_ovf, W_u, W_d, h->g_ovf, h->ovf_rows, h->n_ovf, cap, d, f,
-                                    at<uint16_t>(ws, L.h_ovf), h->u_ovf, Y, h->status, s));
+                                    at<uint16_t>(ws, L.h_ovf), h->u_ovf, Y, sk, h->status, s));
 }
 
 twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_t* W_u, const uint16_t* W_d,
@@ -299,8 +314,9 @@ twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_
     return TWELL_ECUDA;
   float* du_ovf = at<float>(ws, L.du_ovf);
   float* dz_ovf = at<float>(ws, L.dz_ovf);
+  const SplitKBuffers sk{at<float>(ws, L.sk_partial), at<unsigned long long>(ws, L.sk_arrivals)};
   if (launch_ovf_bwd(dy_ovf, wdt, W_u, W_g, h->g_ovf, h->u_ovf, lambda, h->ovf_rows, h->n_ovf, cap, d, f, duz,
-                     du_ovf, dz_ovf, dX, h->status, s) != cudaSuccess)
+                     du_ovf, dz_ovf, dX, sk, h->status, s) != cudaSuccess)
     return TWELL_ECUDA;
   CscBuffers b{at<int>(ws, L.row_slot), at<int>(ws, L.block_cnt), at<int>(ws, L.unit_tot),
                at<int>(ws, L.unit_ptr), at<int>(ws, L.csc_row), at<float4>(ws, L.csc_val)};

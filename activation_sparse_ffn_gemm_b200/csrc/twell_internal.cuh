@@ -78,6 +78,9 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
 
 int device_sm_count();
 
+// Process-wide tag for one split-K GEMM launch (1 .. 2^56 - 1, never 0).
+unsigned long long next_gemm_epoch();
+
 // Encodes a 2-D bf16 tensor map (128-byte swizzle, zero fill out of bounds).
 // inner = contiguous extent (elements), outer = rows, row_bytes = row pitch.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
@@ -125,11 +128,21 @@ cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uin
                                float* u_ell, uint16_t* Y, int M, int d, int f, int K, int* ctr, float* yacc,
                                uint32_t* status, cudaStream_t s);
 
+// Split-K scratch of the dense-backup GEMMs (one GEMM at a time): fp32
+// partials and per-output-tile arrival words (any initial contents).
+struct SplitKBuffers {
+  float* partial;                // [splitk_partial_floats(cap, d, f)]
+  unsigned long long* arrivals;  // [splitk_arrival_words()]
+};
+size_t splitk_partial_floats(int cap, int d, int f);
+size_t splitk_arrival_words();
+
 // Dense backup forward for overflow rows: H = bf16(G * (X_ovf W_u^T)) then
 // Y[ovf_rows] = bf16(H W_d^T).
 cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uint16_t* W_d,
                            const uint16_t* g_ovf, const int* ovf_rows, const int* n_ovf, int cap, int d, int f,
-                           uint16_t* h_ovf, float* u_ovf, uint16_t* Y, uint32_t* status, cudaStream_t s);
+                           uint16_t* h_ovf, float* u_ovf, uint16_t* Y, const SplitKBuffers& sk, uint32_t* status,
+                           cudaStream_t s);
 
 // Sparse backward over the pieces of the row plan: dH at kept actives, dU,
 // dZ (stored per slot) and the rows of dX.
@@ -144,7 +157,8 @@ cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const ui
 cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const uint16_t* W_u,
                            const uint16_t* W_g, const uint16_t* g_ovf, const float* u_ovf, float lambda,
                            const int* ovf_rows, const int* n_ovf, int cap, int d, int f, uint16_t* duz_ovf,
-                           float* du_ovf, float* dz_ovf, float* dX, uint32_t* status, cudaStream_t s);
+                           float* du_ovf, float* dz_ovf, float* dX, const SplitKBuffers& sk, uint32_t* status,
+                           cudaStream_t s);
 
 struct CscBuffers {
   int* row_slot;   // [M]

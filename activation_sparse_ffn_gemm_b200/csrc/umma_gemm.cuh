@@ -16,6 +16,14 @@
 // groups of 16 M-blocks so that concurrently resident CTAs share A and B
 // panels in L2. Rows may be a device-side count (M_dev), so the dense backup
 // GEMMs need no host synchronisation to learn how many rows overflowed.
+// Split-K (when shp.partial is set): if the rows are few (M_eff <=
+// split_rows) and the output tiles cannot fill the GPU, the K blocks are split
+// into `split` ranges and each (tile, range) pair is its own work item. The
+// epilogue stores its fp32 partial sums and counts the tile's arrivals; the
+// CTA that arrives last adds the partials in range order and applies
+// Epi::apply8, so the result does not depend on which CTA finished when. The
+// arrival words carry a per-launch epoch, so stale words from earlier
+// launches (or uninitialised workspace) read as zero arrivals.
 //
 // Every wait is bounded (sm100.cuh); a CTA that gives up sets
 // TWELL_STATUS_TIMEOUT, lets the other roles unwind, waits for its own
@@ -40,7 +48,28 @@ struct GemmShape {
   int K0;            // K extent of segment 0 (multiple of kBK)
   int K1;            // K extent of segment 1 (0: single segment)
   uint32_t* status;
+  float* partial = nullptr;  // split-K partials [split_max][split_rows][N] fp32 (nullptr: no split-K)
+  int split_rows = 0;        // split-K only when the processed rows are at most this many
+  int split_max = 1;
+  unsigned long long* arrivals = nullptr;  // [kSplitTiles] per-output-tile arrival words
+  unsigned long long epoch = 0;            // this launch's tag (1 .. 2^56 - 1)
 };
+
+constexpr int kSplitMax = 8;
+constexpr int kSplitRows = 2 * 128;
+constexpr int kSplitMinKBlocks = 4;
+constexpr int kSplitMinWays = 4;  // a 2- or 3-way split measured no faster than none
+constexpr int kSplitTiles = (kSplitRows / 128) * (kMaxTiles * 128 / 64);  // output tiles of a split GEMM, BN >= 64
+
+// K-range count for M_eff rows on `grid` persistent CTAs (1: no split).
+__host__ __device__ inline int gemm_split(int M_eff, int N, int BN, int nk, const GemmShape& shp, int grid) {
+  if (shp.partial == nullptr || M_eff <= 0 || M_eff > shp.split_rows) return 1;
+  const int mn = ((M_eff + 127) / 128) * ((N + BN - 1) / BN);
+  int sp = grid / mn;
+  sp = sp < shp.split_max ? sp : shp.split_max;
+  sp = sp < nk / kSplitMinKBlocks ? sp : nk / kSplitMinKBlocks;
+  return sp >= kSplitMinWays ? sp : 1;
+}
 
 template <int BN, int STAGES>
 struct GemmLayout {
@@ -50,9 +79,28 @@ struct GemmLayout {
   static constexpr int NBAR = 2 * STAGES + 5;  // full, empty, tmem_full[2], tmem_empty[2], drain
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
-  static constexpr int EPI_OFF = (MISC_OFF + 16 + 127) / 128 * 128;
+  static constexpr int EPI_OFF = (MISC_OFF + 32 + 127) / 128 * 128;
   static constexpr int TMEM_COLS = 2 * BN;
 };
+
+// Barrier of the four epilogue warps with a bounded wait (a warp that left
+// its loop on a timeout must not strand the others): each warp adds one to a
+// shared counter; lane 0 waits until the counter reaches `gen` (advanced by 4
+// per use), or the CTA's abort flag is set, or kWaitLimitNs has passed.
+__device__ __forceinline__ void epi_bar(volatile int* cnt, int& gen, volatile int* abort_flag) {
+  gen += 4;
+  __threadfence_block();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) {
+    atomicAdd(const_cast<int*>(cnt), 1);
+    const uint64_t t0 = globaltimer_ns();
+    while (*cnt < gen) {
+      if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) break;
+    }
+  }
+  __syncwarp();
+  __threadfence_block();
+}
 
 __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
   const int per_group = kGroupM * num_n;
@@ -81,6 +129,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   int* m_eff_s = reinterpret_cast<int*>(smem + L::MISC_OFF + 8);
+  volatile int* last_s = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 12);
+  volatile int* epi_cnt = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 16);
   uint8_t* epi_smem = smem + L::EPI_OFF;
 
   const int warp = threadIdx.x >> 5;
@@ -97,7 +147,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     *m_eff_s = m;
   }
   __syncthreads();
-  if (static_cast<long>(blockIdx.x) >= static_cast<long>((*m_eff_s + kBM - 1) / kBM) * ((shp.N + BN - 1) / BN)) return;
+  const int nk = shp.K0 / kBK + shp.K1 / kBK;
+  const int split = gemm_split(*m_eff_s, shp.N, BN, nk, shp, gridDim.x);
+  if (static_cast<long>(blockIdx.x) >=
+      static_cast<long>((*m_eff_s + kBM - 1) / kBM) * ((shp.N + BN - 1) / BN) * split)
+    return;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -110,6 +164,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
+    *epi_cnt = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -132,9 +187,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int num_m = (M_eff + kBM - 1) / kBM;
   const int num_n = (shp.N + BN - 1) / BN;
-  const int num_tiles = num_m * num_n;
+  const int num_tiles = num_m * num_n * split;
   const int nk0 = shp.K0 / kBK;
-  const int nk = nk0 + shp.K1 / kBK;
+  // work item -> (output tile, K range [kb0, kb1)); split == 1: the whole K
+  auto item = [&](int tile, int& mb, int& nb, int& ks, int& kb0, int& kb1) {
+    ks = tile % split;
+    tile_coords(tile / split, num_m, num_n, mb, nb);
+    kb0 = static_cast<int>(static_cast<long>(ks) * nk / split);
+    kb1 = static_cast<int>(static_cast<long>(ks + 1) * nk / split);
+  };
 
   auto fail = [&]() {
     *abort_flag = 1;
@@ -150,10 +211,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t issued_par = 0;  // phase parity of that load
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        int mb, nb;
-        tile_coords(tile, num_m, num_n, mb, nb);
+        int mb, nb, ks, kb0, kb1;
+        item(tile, mb, nb, ks, kb0, kb1);
         const int m0 = mb * kBM, n0 = nb * BN;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             fail();
             ok = false;
@@ -199,6 +260,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true, any = false;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        int mb, nb, ks, kb0, kb1;
+        item(tile, mb, nb, ks, kb0, kb1);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
           fail();
           ok = false;
@@ -206,7 +269,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) {
             fail();
             ok = false;
@@ -220,7 +283,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint64_t adesc = sdesc_sw128(a_base + kk * 32, 16, 1024);
             const uint64_t bdesc = B_MN ? sdesc_sw128(b_base + kk * 2048, 64 * kBK * 2, 1024)
                                         : sdesc_sw128(b_base + kk * 32, 16, 1024);
-            umma_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            umma_bf16(d_tmem, adesc, bdesc, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
           }
           umma_commit(&empty[stage]);
           any = true;
@@ -245,11 +308,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // --------------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // tensor-memory lane quarter this warp may access
     const int r = quarter * 32 + lane;
+    int bar_gen = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      int mb, nb;
-      tile_coords(tile, num_m, num_n, mb, nb);
+      int mb, nb, ks, kb0, kb1;
+      item(tile, mb, nb, ks, kb0, kb1);
       const bool got = mbar_wait(&tfull[acc], acc_phase, abort_flag);
       if (!got) {
         fail();
@@ -258,7 +322,63 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       __syncwarp();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      Epi::run(ea, mb * kBM, nb * BN, M_eff, shp.N, r, taddr, epi_smem);
+      if (split == 1) {
+        Epi::run(ea, mb * kBM, nb * BN, M_eff, shp.N, r, taddr, epi_smem);
+      } else {
+        // fp32 partial of K range ks for this accumulator row
+        const int row = mb * kBM + r;
+#pragma unroll 1
+        for (int ch = 0; ch < BN / 32; ++ch) {
+          const int n = nb * BN + ch * 32;
+          if (n >= shp.N) break;
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(taddr + ch * 32, v);
+          tmem_wait_ld();
+          if (row >= M_eff) continue;
+          float4* p = reinterpret_cast<float4*>(shp.partial + (static_cast<size_t>(ks) * shp.split_rows + row) * shp.N + n);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            p[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
+                               __uint_as_float(v[4 * q + 3]));
+        }
+        if constexpr (Epi::kSplitK) {
+          // arrival: the last of the tile's `split` ranges reduces it
+          __threadfence();
+          epi_bar(epi_cnt, bar_gen, abort_flag);
+          if (threadIdx.x == 64) {
+            unsigned long long* w = shp.arrivals + (mb * num_n + nb);
+            unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(w), nw;
+            for (;;) {
+              nw = (cur >> 8) == shp.epoch ? cur + 1 : ((shp.epoch << 8) | 1ull);
+              const unsigned long long seen = atomicCAS(w, cur, nw);
+              if (seen == cur) break;
+              cur = seen;
+            }
+            const bool last = static_cast<int>(nw & 0xFFull) == split;
+            if (last) atomicExch(w, 0ull);
+            *last_s = last ? 1 : 0;
+          }
+          epi_bar(epi_cnt, bar_gen, abort_flag);
+          if (*last_s && row < M_eff) {
+            __threadfence();
+#pragma unroll 1
+            for (int c8 = 0; c8 < BN / 8; ++c8) {
+              const int n = nb * BN + c8 * 8;
+              if (n >= shp.N) break;
+              float accv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+              for (int k2 = 0; k2 < split; ++k2) {
+                const float4* p =
+                    reinterpret_cast<const float4*>(shp.partial + (static_cast<size_t>(k2) * shp.split_rows + row) * shp.N + n);
+                const float4 a = __ldcg(p), b = __ldcg(p + 1);
+                accv[0] += a.x; accv[1] += a.y; accv[2] += a.z; accv[3] += a.w;
+                accv[4] += b.x; accv[5] += b.y; accv[6] += b.z; accv[7] += b.w;
+              }
+              Epi::apply8(ea, row, n, accv);
+            }
+          }
+        }
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -293,8 +413,12 @@ cudaError_t launch_umma_gemm(const char* name, const CUtensorMap& a0, const CUte
   if (e != cudaSuccess) return e;
   const long tiles = static_cast<long>((shp.M + kBM - 1) / kBM) * ((shp.N + BN - 1) / BN);
   if (tiles <= 0) return cudaSuccess;
-  const int grid = static_cast<int>(tiles < device_sm_count() ? tiles : device_sm_count());
-  TWELL_LAUNCH(name, s, kern<<<grid, kGemmThreads, smem, s>>>(a0, b0, a1, b1, shp, ea));
+  const int sms = device_sm_count();
+  // with split-K the work items can outnumber the output tiles: one CTA per SM
+  const int grid = shp.partial ? sms : static_cast<int>(tiles < sms ? tiles : sms);
+  GemmShape shp2 = shp;
+  if (shp2.partial) shp2.epoch = next_gemm_epoch();
+  TWELL_LAUNCH(name, s, kern<<<grid, kGemmThreads, smem, s>>>(a0, b0, a1, b1, shp2, ea));
   return cudaGetLastError();
 }
 
