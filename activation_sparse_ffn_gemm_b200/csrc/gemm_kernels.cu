@@ -275,6 +275,7 @@ struct EpiBwdDH {
       du[e] = dh[e] * g8[e];
       dz[e] = g8[e] > 0.f ? fmaf(dh[e], u8[e], a.lambda) : 0.f;
     }
+
     uint16_t* drow = a.duz + static_cast<size_t>(row) * 2 * a.f;
     *reinterpret_cast<uint4*>(drow + n) = make_uint4(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]),
                                                      pack_bf16x2(du[4], du[5]), pack_bf16x2(du[6], du[7]));
@@ -289,6 +290,31 @@ struct EpiBwdDH {
   }
   __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
     run_apply8<EpiBwdDH>(a, m0, n0, M_eff, N, r, taddr);
+  }
+};
+
+// ------------------------------------------------- dense weight gradients
+// out[row][n..n+8) = acc: rows below m_split go to out0, the rest to out1
+// (row - m_split), both with leading dimension ld. The sparse weight-gradient
+// kernel then adds the ELL rows' sums, so the result is the same on every run.
+struct EpiStoreF32 {
+  struct Args {
+    float* out0;
+    float* out1;
+    int m_split;
+    int ld;
+  };
+  static constexpr int SMEM_BYTES = 0;
+  static constexpr bool kSplitK = false;
+  __device__ static void apply8(const Args& a, int row, int n, const float (&v)[8]) {
+    float* base = row < a.m_split ? a.out0 + static_cast<size_t>(row) * a.ld
+                                  : a.out1 + static_cast<size_t>(row - a.m_split) * a.ld;
+    float4* p = reinterpret_cast<float4*>(base + n);
+    p[0] = make_float4(v[0], v[1], v[2], v[3]);
+    p[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
+    run_apply8<EpiStoreF32>(a, m0, n0, M_eff, N, r, taddr);
   }
 };
 
@@ -371,6 +397,30 @@ cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const u
   use_split(s2, sk, cap);
   EpiScatterF32::Args e2{ovf_rows, dX, d};
   return launch_umma_gemm<EpiScatterF32, 256, true, kStages>("ovf_dx_gemm", tdu, twu, tdz, twg, s2, e2, s);
+}
+
+cudaError_t launch_dense_wgrad(const DenseWgradOperands& op, const int* k_rows, int cap, int d, int f, float* dW_g,
+                               float* dW_u, float* dW_d, uint32_t* status, cudaStream_t s) {
+  if (cap <= 0) return cudaSuccess;
+  const uint64_t rows = dense_wgrad_rows(cap);
+  CUtensorMap ta, tb, ta2, tb2;
+  // the contraction runs over the operand rows (hi rows, then lo rows): every operand is [K = rows][M or N]
+  if (!make_tmap_bf16(&ta, op.duz2, 2 * static_cast<uint64_t>(f), rows, static_cast<uint64_t>(f) * 4, 64, kBK) ||
+      !make_tmap_bf16(&tb, op.x2, d, rows, static_cast<uint64_t>(d) * 2, 64, kBK) ||
+      !make_tmap_bf16(&ta2, op.dy2, d, rows, static_cast<uint64_t>(d) * 2, 64, kBK) ||
+      !make_tmap_bf16(&tb2, op.h2, f, rows, static_cast<uint64_t>(f) * 2, 64, kBK))
+    return cudaErrorInvalidValue;
+  // [dW_u ; dW_g] (2 d_ff x d_model) = [dU | dZ]^T X_ovf
+  GemmShape s1{2 * f, nullptr, d, static_cast<int>(rows), 0, status};
+  s1.K_dev = k_rows;
+  EpiStoreF32::Args e1{dW_u, dW_g, f, d};
+  cudaError_t e = launch_umma_gemm<EpiStoreF32, 256, true, kStages, true>("dense_wgrad_ug", ta, tb, ta, tb, s1, e1, s);
+  if (e != cudaSuccess) return e;
+  // dW_d (d_model x d_ff) = dY_ovf^T H_ovf
+  GemmShape s2{d, nullptr, f, static_cast<int>(rows), 0, status};
+  s2.K_dev = k_rows;
+  EpiStoreF32::Args e2{dW_d, dW_d, d, f};
+  return launch_umma_gemm<EpiStoreF32, 256, true, kStages, true>("dense_wgrad_d", ta2, tb2, ta2, tb2, s2, e2, s);
 }
 
 }  // namespace twell

@@ -39,18 +39,20 @@ __global__ void row_slot_kernel(const int* __restrict__ ovf_rows, const int* __r
 // lane, and group and chunk offsets come from prefix sums of the popcounts.
 
 // In-tile columns active for row r in tile t: the ELL slots of a non-overflow
-// row, or the nonzeros of its dense backup row; calls fn(c, ell_slot_or_-1).
+// row, or the nonzeros of its dense backup row (none when the dense backup's
+// weight gradients run as dense GEMMs); calls fn(c, ell_slot_or_-1).
 template <typename Fn>
 __device__ __forceinline__ void for_row_entries(long r, int t, int T, int K, int f, const uint16_t* __restrict__ count,
                                                 const uint8_t* __restrict__ col, const uint8_t* __restrict__ row_ovf,
                                                 const int* __restrict__ row_slot, const uint16_t* __restrict__ g_ovf,
-                                                Fn&& fn) {
+                                                bool dense_ovf, Fn&& fn) {
   if (!row_ovf[r]) {
     const int c0 = count[r * T + t];
     const int n = c0 < K ? c0 : K;
     const long base = (r * T + t) * K;
     for (int s = 0; s < n; ++s) fn(static_cast<int>(col[base + s]), base + s);
   } else {
+    if (dense_ovf) return;
     const int sl = row_slot[r];
     if (sl < 0) return;
     const uint4* gp = reinterpret_cast<const uint4*>(g_ovf + static_cast<long>(sl) * f + t * kTn);
@@ -72,12 +74,14 @@ __global__ void __launch_bounds__(256) csc_count_kernel(const uint16_t* __restri
                                                         const uint8_t* __restrict__ col,
                                                         const uint8_t* __restrict__ row_ovf,
                                                         const int* __restrict__ row_slot,
-                                                        const uint16_t* __restrict__ g_ovf, int M, int f, int K,
+                                                        const uint16_t* __restrict__ g_ovf,
+                                                        const int* __restrict__ plan, int M, int f, int K,
                                                         int* __restrict__ chunk_cnt) {
   __shared__ uint32_t mask[8][kTn];
   __shared__ int cnt_s[kTn];
   const int t = blockIdx.x, chunk = blockIdx.y, T = f / kTn;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool dense_ovf = plan[3] != 0;
   if (threadIdx.x < kTn) cnt_s[threadIdx.x] = 0;
   __syncthreads();
   for (int g = w; g < kCscGroups; g += 8) {
@@ -86,7 +90,7 @@ __global__ void __launch_bounds__(256) csc_count_kernel(const uint16_t* __restri
     for (int q = 0; q < kTn / 32; ++q) mask[w][lane + 32 * q] = 0u;
     __syncwarp();
     if (r < M)
-      for_row_entries(r, t, T, K, f, count, col, row_ovf, row_slot, g_ovf,
+      for_row_entries(r, t, T, K, f, count, col, row_ovf, row_slot, g_ovf, dense_ovf,
                       [&](int c, long) { atomicOr(&mask[w][c], 1u << lane); });
     __syncwarp();
 #pragma unroll
@@ -171,19 +175,20 @@ __global__ void __launch_bounds__(256) csc_fill_kernel(
     const uint8_t* __restrict__ row_ovf, const int* __restrict__ row_slot, const uint16_t* __restrict__ g_ovf,
     const float* __restrict__ u_ell, const float* __restrict__ u_ovf, const float* __restrict__ du_ell,
     const float* __restrict__ dz_ell, const float* __restrict__ du_ovf, const float* __restrict__ dz_ovf,
-    const int* __restrict__ chunk_base, const int* __restrict__ unit_ptr, int M, int f, int K,
-    int* __restrict__ csc_row, float4* __restrict__ csc_val) {
+    const int* __restrict__ chunk_base, const int* __restrict__ unit_ptr, const int* __restrict__ plan, int M, int f,
+    int K, int* __restrict__ csc_row, float4* __restrict__ csc_val) {
   __shared__ uint32_t mask[kCscGroups][kTn];
   __shared__ int gbase[kCscGroups][kTn];
   const int t = blockIdx.x, chunk = blockIdx.y, T = f / kTn;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool dense_ovf = plan[3] != 0;
   for (int g = w; g < kCscGroups; g += 8) {
     const long r = static_cast<long>(chunk) * kCscRows + g * 32 + lane;
 #pragma unroll
     for (int q = 0; q < kTn / 32; ++q) mask[g][lane + 32 * q] = 0u;
     __syncwarp();
     if (r < M)
-      for_row_entries(r, t, T, K, f, count, col, row_ovf, row_slot, g_ovf,
+      for_row_entries(r, t, T, K, f, count, col, row_ovf, row_slot, g_ovf, dense_ovf,
                       [&](int c, long) { atomicOr(&mask[g][c], 1u << lane); });
   }
   __syncthreads();
@@ -201,7 +206,7 @@ __global__ void __launch_bounds__(256) csc_fill_kernel(
     const long r = static_cast<long>(chunk) * kCscRows + g * 32 + lane;
     if (r >= M) continue;
     const int sl = row_ovf[r] ? row_slot[r] : -1;
-    for_row_entries(r, t, T, K, f, count, col, row_ovf, row_slot, g_ovf, [&](int c, long slot) {
+    for_row_entries(r, t, T, K, f, count, col, row_ovf, row_slot, g_ovf, dense_ovf, [&](int c, long slot) {
       const int p = gbase[g][c] + __popc(mask[g][c] & below);
       float4 v;
       if (slot >= 0) {
@@ -233,8 +238,10 @@ __global__ void __launch_bounds__(256, 3) wgrad_kernel(const uint16_t* __restric
                                                        const int* __restrict__ unit_ptr,
                                                        const int* __restrict__ csc_row,
                                                        const float4* __restrict__ csc_val, int d, int f,
-                                                       float* __restrict__ dWg, float* __restrict__ dWu,
-                                                       float* __restrict__ dWd, float* __restrict__ dbg) {
+                                                       const float* __restrict__ db_extra,
+                                                       const int* __restrict__ accumulate, float* __restrict__ dWg,
+                                                       float* __restrict__ dWu, float* __restrict__ dWd,
+                                                       float* __restrict__ dbg) {
   __shared__ float s_dwd[kWgCols][9];
   __shared__ int s_row[8][32];
   __shared__ float4 s_val[8][32];
@@ -243,6 +250,19 @@ __global__ void __launch_bounds__(256, 3) wgrad_kernel(const uint16_t* __restric
   const int c0 = blockIdx.y * kWgCols;
   const int cidx = (c0 >> 3) + lane;
   const bool cval = cidx < (d >> 3);
+  // add to the dense GEMMs' result (written before this kernel) instead of
+  // overwriting: its lines are pulled into L2 now and read after the pair loop
+  const bool acc_old = accumulate != nullptr && *accumulate > 0;
+  float* pu_out = dWu + static_cast<long>(j) * d + 8 * cidx;
+  float* pg_out = dWg + static_cast<long>(j) * d + 8 * cidx;
+  float* pd_out = dWd + static_cast<long>(c0 + threadIdx.x) * f + blockIdx.x * 8;
+  if (acc_old) {
+    if (cval) {
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(pu_out));
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(pg_out));
+    }
+    if (c0 + static_cast<int>(threadIdx.x) < d) asm volatile("prefetch.global.L2 [%0];" ::"l"(pd_out));
+  }
   float2 au[4], ag[4], ad[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) au[e] = ag[e] = ad[e] = make_float2(0.f, 0.f);
@@ -288,35 +308,142 @@ __global__ void __launch_bounds__(256, 3) wgrad_kernel(const uint16_t* __restric
   }
   db = warp_sum(db);
   if (cval) {
-    float4* pu = reinterpret_cast<float4*>(dWu + static_cast<long>(j) * d) + 2 * cidx;
-    float4* pg = reinterpret_cast<float4*>(dWg + static_cast<long>(j) * d) + 2 * cidx;
-    pu[0] = make_float4(au[0].x, au[0].y, au[1].x, au[1].y);
-    pu[1] = make_float4(au[2].x, au[2].y, au[3].x, au[3].y);
-    pg[0] = make_float4(ag[0].x, ag[0].y, ag[1].x, ag[1].y);
-    pg[1] = make_float4(ag[2].x, ag[2].y, ag[3].x, ag[3].y);
+    float4* pu = reinterpret_cast<float4*>(pu_out);
+    float4* pg = reinterpret_cast<float4*>(pg_out);
+    float4 u0 = make_float4(au[0].x, au[0].y, au[1].x, au[1].y), u1 = make_float4(au[2].x, au[2].y, au[3].x, au[3].y);
+    float4 g0 = make_float4(ag[0].x, ag[0].y, ag[1].x, ag[1].y), g1 = make_float4(ag[2].x, ag[2].y, ag[3].x, ag[3].y);
+    if (acc_old) {
+      const float4 ou0 = pu[0], ou1 = pu[1], og0 = pg[0], og1 = pg[1];
+      u0 = make_float4(ou0.x + u0.x, ou0.y + u0.y, ou0.z + u0.z, ou0.w + u0.w);
+      u1 = make_float4(ou1.x + u1.x, ou1.y + u1.y, ou1.z + u1.z, ou1.w + u1.w);
+      g0 = make_float4(og0.x + g0.x, og0.y + g0.y, og0.z + g0.z, og0.w + g0.w);
+      g1 = make_float4(og1.x + g1.x, og1.y + g1.y, og1.z + g1.z, og1.w + g1.w);
+    }
+    pu[0] = u0;
+    pu[1] = u1;
+    pg[0] = g0;
+    pg[1] = g1;
   }
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     s_dwd[lane * 8 + 2 * e][w] = ad[e].x;
     s_dwd[lane * 8 + 2 * e + 1][w] = ad[e].y;
   }
-  if (blockIdx.y == 0 && lane == 0 && dbg != nullptr) dbg[j] = db;
+  if (blockIdx.y == 0 && lane == 0 && dbg != nullptr) dbg[j] = db_extra ? db + db_extra[j] : db;
   __syncthreads();
   const int cc = c0 + threadIdx.x;
   if (cc < d) {
-    float4* pd = reinterpret_cast<float4*>(dWd + static_cast<long>(cc) * f + blockIdx.x * 8);
-    pd[0] = make_float4(s_dwd[threadIdx.x][0], s_dwd[threadIdx.x][1], s_dwd[threadIdx.x][2], s_dwd[threadIdx.x][3]);
-    pd[1] = make_float4(s_dwd[threadIdx.x][4], s_dwd[threadIdx.x][5], s_dwd[threadIdx.x][6], s_dwd[threadIdx.x][7]);
+    float4* pd = reinterpret_cast<float4*>(pd_out);
+    float4 d0 = make_float4(s_dwd[threadIdx.x][0], s_dwd[threadIdx.x][1], s_dwd[threadIdx.x][2], s_dwd[threadIdx.x][3]);
+    float4 d1 = make_float4(s_dwd[threadIdx.x][4], s_dwd[threadIdx.x][5], s_dwd[threadIdx.x][6], s_dwd[threadIdx.x][7]);
+    if (acc_old) {
+      const float4 o0 = pd[0], o1 = pd[1];
+      d0 = make_float4(o0.x + d0.x, o0.y + d0.y, o0.z + d0.z, o0.w + d0.w);
+      d1 = make_float4(o1.x + d1.x, o1.y + d1.y, o1.z + d1.z, o1.w + d1.w);
+    }
+    pd[0] = d0;
+    pd[1] = d1;
+  }
+}
+
+// Operands of the dense weight gradients of the overflow rows (layout in
+// DenseWgradOperands), db_ovf[j] = sum over s < n of dZ[s][j] in ascending s,
+// and k_rows = np + n. When the plan keeps the overflow rows on the sparse
+// path, only k_rows = 0 and db_ovf = 0 are written. One block per operand row
+// pair (s, np + s), s < np.
+__device__ __forceinline__ void split_hi_lo(const float (&v)[8], uint4& hi, uint4& lo) {
+  float h[8], l[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    h[e] = __bfloat162float(__float2bfloat16_rn(v[e]));
+    l[e] = v[e] - h[e];  // exact in fp32
+  }
+  hi = make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]), pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
+  lo = make_uint4(pack_bf16x2(l[0], l[1]), pack_bf16x2(l[2], l[3]), pack_bf16x2(l[4], l[5]), pack_bf16x2(l[6], l[7]));
+}
+
+__global__ void ovf_operands_kernel(const int* __restrict__ n_ovf, const int* __restrict__ ovf_rows,
+                                    const int* __restrict__ plan, int d, int f, const uint16_t* __restrict__ X,
+                                    const uint16_t* __restrict__ dy_ovf, const float* __restrict__ du_ovf,
+                                    const float* __restrict__ dz_ovf, const uint16_t* __restrict__ g_ovf,
+                                    const float* __restrict__ u_ovf, DenseWgradOperands op, float* __restrict__ db_ovf,
+                                    int* __restrict__ k_rows) {
+  const bool dense = plan[3] != 0;
+  const int n = dense ? n_ovf[0] : 0;
+  const int np = (n + 63) / 64 * 64;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *k_rows = n > 0 ? np + n : 0;
+  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < f; j += gridDim.x * blockDim.x) {
+    float acc = 0.f;
+    for (int sl = 0; sl < n; ++sl) acc += dz_ovf[static_cast<long>(sl) * f + j];
+    db_ovf[j] = acc;
+  }
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  for (int sl = blockIdx.x; sl < np; sl += gridDim.x) {
+    const bool live = sl < n;
+    const long r_hi = sl, r_lo = static_cast<long>(np) + sl;
+    {
+      const uint4* xi = live ? reinterpret_cast<const uint4*>(X + static_cast<long>(ovf_rows[sl]) * d) : nullptr;
+      const uint4* yi = live ? reinterpret_cast<const uint4*>(dy_ovf + static_cast<long>(sl) * d) : nullptr;
+      uint4* xh = reinterpret_cast<uint4*>(op.x2 + r_hi * d);
+      uint4* xl = reinterpret_cast<uint4*>(op.x2 + r_lo * d);
+      uint4* yh = reinterpret_cast<uint4*>(op.dy2 + r_hi * d);
+      uint4* yl = reinterpret_cast<uint4*>(op.dy2 + r_lo * d);
+      for (int q = threadIdx.x; q < d / 8; q += blockDim.x) {
+        const uint4 xv = live ? xi[q] : z, yv = live ? yi[q] : z;
+        xh[q] = xv;
+        xl[q] = xv;
+        yh[q] = yv;
+        yl[q] = yv;
+      }
+    }
+    for (int q = threadIdx.x; q < f / 8; q += blockDim.x) {
+      uint4 uh = z, ul = z, zh = z, zl = z, hh = z, hl = z;
+      if (live) {
+        const long o = static_cast<long>(sl) * f + 8 * q;
+        float du[8], dz[8], h[8];
+        const float4 a0 = reinterpret_cast<const float4*>(du_ovf + o)[0], a1 = reinterpret_cast<const float4*>(du_ovf + o)[1];
+        const float4 b0 = reinterpret_cast<const float4*>(dz_ovf + o)[0], b1 = reinterpret_cast<const float4*>(dz_ovf + o)[1];
+        const float4 c0 = reinterpret_cast<const float4*>(u_ovf + o)[0], c1 = reinterpret_cast<const float4*>(u_ovf + o)[1];
+        float g8[8];
+        unpack8(*reinterpret_cast<const uint4*>(g_ovf + o), g8);
+        const float u8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        du[0] = a0.x; du[1] = a0.y; du[2] = a0.z; du[3] = a0.w; du[4] = a1.x; du[5] = a1.y; du[6] = a1.z; du[7] = a1.w;
+        dz[0] = b0.x; dz[1] = b0.y; dz[2] = b0.z; dz[3] = b0.w; dz[4] = b1.x; dz[5] = b1.y; dz[6] = b1.z; dz[7] = b1.w;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) h[e] = g8[e] * u8[e];  // h = g u in fp32, as on the sparse path
+        split_hi_lo(du, uh, ul);
+        split_hi_lo(dz, zh, zl);
+        split_hi_lo(h, hh, hl);
+      }
+      reinterpret_cast<uint4*>(op.duz2 + r_hi * 2 * f)[q] = uh;
+      reinterpret_cast<uint4*>(op.duz2 + r_lo * 2 * f)[q] = ul;
+      reinterpret_cast<uint4*>(op.duz2 + r_hi * 2 * f + f)[q] = zh;
+      reinterpret_cast<uint4*>(op.duz2 + r_lo * 2 * f + f)[q] = zl;
+      reinterpret_cast<uint4*>(op.h2 + r_hi * f)[q] = hh;
+      reinterpret_cast<uint4*>(op.h2 + r_lo * f)[q] = hl;
+    }
   }
 }
 
 }  // namespace
 
+cudaError_t launch_ovf_operands(const int* n_ovf, const int* ovf_rows, const int* plan, int cap, int d, int f,
+                                const uint16_t* X, const uint16_t* dy_ovf, const float* du_ovf, const float* dz_ovf,
+                                const uint16_t* g_ovf, const float* u_ovf, const DenseWgradOperands& op,
+                                float* db_ovf, int* k_rows, cudaStream_t s) {
+  if (cap <= 0) return cudaSuccess;
+  const int g = device_sm_count() * 2;
+  TWELL_LAUNCH("ovf_operands", s,
+               ovf_operands_kernel<<<g, 256, 0, s>>>(n_ovf, ovf_rows, plan, d, f, X, dy_ovf, du_ovf, dz_ovf, g_ovf,
+                                                     u_ovf, op, db_ovf, k_rows));
+  return cudaGetLastError();
+}
+
 cudaError_t launch_build_csc(const uint16_t* count, const uint16_t* val, const uint8_t* col,
                              const uint8_t* row_ovf, const int* ovf_rows, const int* n_ovf, const uint16_t* g_ovf,
                              const float* u_ell, const float* u_ovf, const float* du_ell, const float* dz_ell,
-                             const float* du_ovf, const float* dz_ovf, int M, int f, int K, int cap,
-                             const CscBuffers& b, cudaStream_t s) {
+                             const float* du_ovf, const float* dz_ovf, const int* plan, int M, int f, int K,
+                             int cap, const CscBuffers& b, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   cudaError_t e = cudaMemsetAsync(b.row_slot, 0xFF, static_cast<size_t>(M) * sizeof(int), s);
   if (e != cudaSuccess) return e;
@@ -327,22 +454,24 @@ cudaError_t launch_build_csc(const uint16_t* count, const uint16_t* val, const u
   const int nch = (M + kCscRows - 1) / kCscRows;
   const int T = f / kTn;
   TWELL_LAUNCH("csc_count", s,
-               csc_count_kernel<<<dim3(T, nch), 256, 0, s>>>(count, col, row_ovf, b.row_slot, g_ovf, M, f, K,
-                                                            b.block_cnt));
+               csc_count_kernel<<<dim3(T, nch), 256, 0, s>>>(count, col, row_ovf, b.row_slot, g_ovf, plan, M, f,
+                                                            K, b.block_cnt));
   TWELL_LAUNCH("csc_colscan", s, csc_colscan_kernel<<<(f + 255) / 256, 256, 0, s>>>(b.block_cnt, nch, f, b.unit_tot));
   TWELL_LAUNCH("csc_unit_scan", s, csc_unit_scan_kernel<<<1, 1024, 0, s>>>(b.unit_tot, f, b.unit_ptr));
   TWELL_LAUNCH("csc_fill", s,
                csc_fill_kernel<<<dim3(T, nch), 256, 0, s>>>(count, val, col, row_ovf, b.row_slot, g_ovf, u_ell, u_ovf,
-                                                           du_ell, dz_ell, du_ovf, dz_ovf, b.block_cnt, b.unit_ptr, M,
-                                                           f, K, b.csc_row, b.csc_val));
+                                                           du_ell, dz_ell, du_ovf, dz_ovf, b.block_cnt, b.unit_ptr, plan,
+                                                           M, f, K, b.csc_row, b.csc_val));
   return cudaGetLastError();
 }
 
 cudaError_t launch_weight_grads(const uint16_t* X, const uint16_t* dY, const CscBuffers& b, int d, int f,
-                                float* dW_g, float* dW_u, float* dW_d, float* db_g, cudaStream_t s) {
+                                const float* db_extra, const int* accumulate, float* dW_g, float* dW_u,
+                                float* dW_d, float* db_g, cudaStream_t s) {
   dim3 grid(f / 8, (d + kWgCols - 1) / kWgCols);
   TWELL_LAUNCH("weight_grads", s,
-               wgrad_kernel<<<grid, 256, 0, s>>>(X, dY, b.unit_ptr, b.csc_row, b.csc_val, d, f, dW_g, dW_u, dW_d, db_g));
+               wgrad_kernel<<<grid, 256, 0, s>>>(X, dY, b.unit_ptr, b.csc_row, b.csc_val, d, f, db_extra, accumulate,
+                                                 dW_g, dW_u, dW_d, db_g));
   return cudaGetLastError();
 }
 

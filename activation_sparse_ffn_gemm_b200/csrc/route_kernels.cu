@@ -19,7 +19,8 @@ constexpr int kScanThreads = 1024;
 constexpr int kScanItems = 16;
 
 // row_ovf[i] = any_t(count[i][t] > K), and the row's kept entries
-// kept[i] = sum_t min(count[i][t], K) (-1 for an overflow row); one warp per row.
+// kept[i] = sum_t min(count[i][t], K), or -(1 + sum_t count[i][t]) for an
+// overflow row; one warp per row.
 __global__ void row_flags_kernel(const uint16_t* __restrict__ count, int M, int T, int K,
                                  uint8_t* __restrict__ row_ovf, int* __restrict__ kept) {
   const int lane = threadIdx.x & 31;
@@ -27,18 +28,22 @@ __global__ void row_flags_kernel(const uint16_t* __restrict__ count, int M, int 
   const long nwarps = (static_cast<long>(gridDim.x) * blockDim.x) >> 5;
   for (long row = warp0; row < M; row += nwarps) {
     bool any = false;
-    int n = 0;
+    int n = 0, all = 0;
     for (int t = lane; t < T; t += 32) {
       const int c = count[row * T + t];
       any |= c > K;
       n += c < K ? c : K;
+      all += c;
     }
     any = __any_sync(0xFFFFFFFFu, any);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xFFFFFFFFu, n, o);
+    for (int o = 16; o > 0; o >>= 1) {
+      n += __shfl_xor_sync(0xFFFFFFFFu, n, o);
+      all += __shfl_xor_sync(0xFFFFFFFFu, all, o);
+    }
     if (lane == 0) {
       row_ovf[row] = any ? 1 : 0;
-      kept[row] = any ? -1 : n;
+      kept[row] = any ? -(1 + all) : n;
     }
   }
 }
@@ -49,25 +54,51 @@ __global__ void row_flags_kernel(const uint16_t* __restrict__ count, int M, int 
 // (max(1, ceil(kept / S)) per non-overflow row, none for overflow rows) and
 // zeroes the turnstile words. Thread t owns the consecutive rows
 // [t * per, (t + 1) * per): it reads its counts before it zeroes them.
-__global__ void __launch_bounds__(kScanThreads) plan_kernel(int* __restrict__ plan, int M, int groups) {
+// plan[3] = 1 when the weight gradients of the n overflow rows (P active
+// pairs) run as dense GEMMs instead of through the pair list, decided by a
+// cost model: the dense GEMMs contract 2 n rows (hi and lo parts) for
+// 12 d_ff d_model n flops and write the full gradients once more, the sparse
+// path gathers two d_model-wide rows per pair, which gives
+// P * 1000 > d_ff * (kDenseWgradPerRow * n + kDenseWgradFixed) with the
+// measured B200 rates of the two (tensor-core flops vs L2 row gathers, HBM
+// writes vs L2 row gathers).
+__global__ void __launch_bounds__(kScanThreads) plan_kernel(int* __restrict__ plan, int M, int f, int groups) {
   __shared__ long long red[kScanThreads / 32];
+  __shared__ long long red_ovf[kScanThreads / 32];
+  __shared__ long long red_rows[kScanThreads / 32];
   __shared__ int warp_tot[kScanThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   int* kept = plan + kPlanHdr;
   int* pieces = plan + kPlanHdr + M;
   const long per = (static_cast<long>(M) + kScanThreads - 1) / kScanThreads;
   const long r0 = tid * per, r1 = r0 + per < M ? r0 + per : M;
-  long long tot = 0;
+  long long tot = 0, tot_ovf = 0, n_ovf_rows = 0;
   for (long r = r0; r < r1; ++r) {
     const int v = kept[r];
-    tot += v > 0 ? v : 0;
+    if (v > 0) tot += v;
+    if (v < 0) {
+      tot_ovf += -1LL - v;
+      ++n_ovf_rows;
+    }
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xFFFFFFFFu, tot, o);
-  if (lane == 0) red[w] = tot;
+  for (int o = 16; o > 0; o >>= 1) {
+    tot += __shfl_xor_sync(0xFFFFFFFFu, tot, o);
+    tot_ovf += __shfl_xor_sync(0xFFFFFFFFu, tot_ovf, o);
+    n_ovf_rows += __shfl_xor_sync(0xFFFFFFFFu, n_ovf_rows, o);
+  }
+  if (lane == 0) {
+    red[w] = tot;
+    red_ovf[w] = tot_ovf;
+    red_rows[w] = n_ovf_rows;
+  }
   __syncthreads();
-  long long total = 0;
-  for (int q = 0; q < kScanThreads / 32; ++q) total += red[q];
+  long long total = 0, total_ovf = 0, rows_ovf = 0;
+  for (int q = 0; q < kScanThreads / 32; ++q) {
+    total += red[q];
+    total_ovf += red_ovf[q];
+    rows_ovf += red_rows[q];
+  }
   const long long g = groups > 0 ? groups : 1;
   long long sz = (total + g - 1) / g;
   sz = sz < kPieceMin ? kPieceMin : (sz > kTokListCap ? kTokListCap : sz);
@@ -110,7 +141,9 @@ __global__ void __launch_bounds__(kScanThreads) plan_kernel(int* __restrict__ pl
     plan[0] = warp_tot[kScanThreads / 32 - 1];
     plan[1] = S;
     plan[2] = static_cast<int>(total < 0x7FFFFFFFLL ? total : 0x7FFFFFFFLL);
-    plan[3] = 0;
+    plan[3] = rows_ovf > 0 && total_ovf * 1000 > static_cast<long long>(f) * (kDenseWgradPerRow * rows_ovf +
+                                                                              kDenseWgradFixed)
+                  ? 1 : 0;
   }
 }
 
@@ -272,7 +305,7 @@ cudaError_t launch_route(const uint16_t* count, const uint16_t* val, const uint8
   if (blocks > max_blocks) blocks = max_blocks;
   TWELL_LAUNCH("row_flags", s, row_flags_kernel<<<blocks, 256, 0, s>>>(count, M, T, K, row_ovf, plan + kPlanHdr));
   TWELL_LAUNCH("ovf_scan", s, ovf_scan_kernel<<<1, kScanThreads, 0, s>>>(row_ovf, M, cap, ovf_rows, n_ovf, status));
-  TWELL_LAUNCH("row_plan", s, plan_kernel<<<1, kScanThreads, 0, s>>>(plan, M, groups));
+  TWELL_LAUNCH("row_plan", s, plan_kernel<<<1, kScanThreads, 0, s>>>(plan, M, f, groups));
   if (cap > 0) {
     int g = cap < device_sm_count() * 4 ? cap : device_sm_count() * 4;
     TWELL_LAUNCH("ovf_gather", s,

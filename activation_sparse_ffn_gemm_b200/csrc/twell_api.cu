@@ -78,6 +78,7 @@ struct WsLayout {
   size_t yacc = 0;  // fp32 accumulator rows of rows split into several pieces
   size_t sk_partial = 0, sk_arrivals = 0;  // split-K scratch of the dense-backup GEMMs
   size_t spill = 0, x_ovf = 0, h_ovf = 0, w_dt = 0;
+  size_t x2 = 0, dy2 = 0, duz2 = 0, h2 = 0, db_ovf = 0, k_rows = 0;  // operands of the dense weight gradients
   size_t dy_ovf = 0, duz = 0, du_ovf = 0, dz_ovf = 0, du_ell = 0, dz_ell = 0, row_slot = 0, block_cnt = 0, unit_tot = 0, unit_ptr = 0,
          csc_row = 0, csc_val = 0;
   size_t total = 0;
@@ -111,6 +112,13 @@ WsLayout ws_layout(twell_op op, int64_t M, int64_t d, int64_t f, int64_t K, int6
     L.duz = take(static_cast<size_t>(cap1 * 2 * f * 2));
     L.du_ovf = take(static_cast<size_t>(cap1 * f * 4));
     L.dz_ovf = take(static_cast<size_t>(cap1 * f * 4));
+    const int64_t r2 = dense_wgrad_rows(cap1);
+    L.x2 = take(static_cast<size_t>(r2 * d * 2));
+    L.dy2 = take(static_cast<size_t>(r2 * d * 2));
+    L.duz2 = take(static_cast<size_t>(r2 * 2 * f * 2));
+    L.h2 = take(static_cast<size_t>(r2 * f * 2));
+    L.db_ovf = take(static_cast<size_t>(f * 4));
+    L.k_rows = take(64);
     L.du_ell = take(static_cast<size_t>(M * T * K * 4));
     L.dz_ell = take(static_cast<size_t>(M * T * K * 4));
     L.row_slot = take(static_cast<size_t>(M * 4));
@@ -315,15 +323,24 @@ twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_
   float* du_ovf = at<float>(ws, L.du_ovf);
   float* dz_ovf = at<float>(ws, L.dz_ovf);
   const SplitKBuffers sk{at<float>(ws, L.sk_partial), at<unsigned long long>(ws, L.sk_arrivals)};
+  const DenseWgradOperands dw{at<uint16_t>(ws, L.x2), at<uint16_t>(ws, L.dy2), at<uint16_t>(ws, L.duz2),
+                              at<uint16_t>(ws, L.h2)};
+  float* db_ovf = at<float>(ws, L.db_ovf);
+  int* k_rows = at<int>(ws, L.k_rows);
   if (launch_ovf_bwd(dy_ovf, wdt, W_u, W_g, h->g_ovf, h->u_ovf, lambda, h->ovf_rows, h->n_ovf, cap, d, f, duz,
                      du_ovf, dz_ovf, dX, sk, h->status, s) != cudaSuccess)
+    return TWELL_ECUDA;
+  if (launch_ovf_operands(h->n_ovf, h->ovf_rows, h->row_plan, cap, d, f, X, dy_ovf, du_ovf, dz_ovf, h->g_ovf,
+                          h->u_ovf, dw, db_ovf, k_rows, s) != cudaSuccess)
     return TWELL_ECUDA;
   CscBuffers b{at<int>(ws, L.row_slot), at<int>(ws, L.block_cnt), at<int>(ws, L.unit_tot),
                at<int>(ws, L.unit_ptr), at<int>(ws, L.csc_row), at<float4>(ws, L.csc_val)};
   if (launch_build_csc(h->count, h->val, h->col, h->row_ovf, h->ovf_rows, h->n_ovf, h->g_ovf, h->u_ell, h->u_ovf,
-                       du_ell, dz_ell, du_ovf, dz_ovf, M, f, K, cap, b, s) != cudaSuccess)
+                       du_ell, dz_ell, du_ovf, dz_ovf, h->row_plan, M, f, K, cap, b, s) != cudaSuccess)
     return TWELL_ECUDA;
-  return cuda_status(launch_weight_grads(X, dY, b, d, f, dW_g, dW_u, dW_d, db_g, s));
+  if (launch_dense_wgrad(dw, k_rows, cap, d, f, dW_g, dW_u, dW_d, h->status, s) != cudaSuccess) return TWELL_ECUDA;
+  return cuda_status(launch_weight_grads(X, dY, b, d, f, cap > 0 ? db_ovf : nullptr, cap > 0 ? k_rows : nullptr,
+                                         dW_g, dW_u, dW_d, db_g, s));
 }
 
 twell_status twell_status_read(const twell_hybrid* h, uint32_t* out, int clear, twell_stream_t stream) {

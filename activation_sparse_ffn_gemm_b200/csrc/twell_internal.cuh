@@ -20,13 +20,18 @@ constexpr int kTokListCap = 256;   // kept entries per list chunk of the token k
 
 // Row plan (twell_hybrid::row_plan, int32): the work of the token kernels as
 // pieces of at most S kept entries of one non-overflow row.
-//   [0] number of pieces, [1] S, [2] kept entries of non-overflow rows, [3] 0
+//   [0] number of pieces, [1] S, [2] kept entries of non-overflow rows,
+//   [3] 1 when the weight gradients of the overflow rows run as dense GEMMs
 //   [kPlanHdr, kPlanHdr + M)  per-row turnstile words (0 between launches;
 //                             the routing step parks the kept counts there)
 //   then (row, q) int pairs, piece q of row, ascending rows then q
 // S = clamp(ceil(kept / resident groups), kPieceMin, kTokListCap), so the
 // pieces number at most M + max(groups, M * T * K / kTokListCap).
 constexpr int kPlanHdr = 4;
+// Cost model of the dense weight gradients of overflow rows (plan[3]), in
+// thousandths of d_ff pairs: per overflow row and fixed.
+constexpr long long kDenseWgradPerRow = 24;
+constexpr long long kDenseWgradFixed = 12000;  // one more pass over the fp32 gradients, about 10 d_ff pair gathers
 constexpr int kPieceMin = 32;
 constexpr long kPlanGroupsCap = 65536;  // bound on resident token groups of any device
 inline long plan_ints(long M, long T, long K) {
@@ -160,6 +165,27 @@ cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const u
                            float* du_ovf, float* dz_ovf, float* dX, const SplitKBuffers& sk, uint32_t* status,
                            cudaStream_t s);
 
+// Operands of the dense weight gradients of the overflow rows, each with
+// dense_wgrad_rows(cap) rows of bf16: for the n stored overflow rows and
+// np = roundup(n, 64), rows [0, n) hold the "hi" part and rows [np, np + n)
+// the "lo" part, so that hi + lo carries a value to about 2^-16 (bf16 alone
+// loses too much where one heavy token dominates a gradient element); every
+// other row up to 2 np is zero. X and dY are exact in bf16 and appear twice.
+struct DenseWgradOperands {
+  uint16_t* x2;    // [rows][d]   X[ovf_rows[s]] (hi and lo halves equal)
+  uint16_t* dy2;   // [rows][d]   dY[ovf_rows[s]]
+  uint16_t* duz2;  // [rows][2f]  [dU | dZ] hi / lo
+  uint16_t* h2;    // [rows][f]   H = g u hi / lo
+};
+inline int64_t dense_wgrad_rows(int64_t cap) { return 2 * ((cap + 63) / 64 * 64); }
+
+// Weight gradients of the dense backup rows on the tensor cores, written
+// before the sparse kernel adds the ELL rows' sums: [dW_u ; dW_g] = [dU | dZ]^T X_ovf,
+// dW_d = dY_ovf^T H_ovf, contracting over the first *k_rows operand rows
+// (0: nothing is written).
+cudaError_t launch_dense_wgrad(const DenseWgradOperands& op, const int* k_rows, int cap, int d, int f, float* dW_g,
+                               float* dW_u, float* dW_d, uint32_t* status, cudaStream_t s);
+
 struct CscBuffers {
   int* row_slot;   // [M]
   int* block_cnt;  // [ceil(M/kCscRows)][f] per-chunk counts, then their exclusive scan
@@ -175,11 +201,25 @@ constexpr int kCscRows = 256;  // rows per chunk of the pair-list build
 cudaError_t launch_build_csc(const uint16_t* count, const uint16_t* val, const uint8_t* col,
                              const uint8_t* row_ovf, const int* ovf_rows, const int* n_ovf, const uint16_t* g_ovf,
                              const float* u_ell, const float* u_ovf, const float* du_ell, const float* dz_ell,
-                             const float* du_ovf, const float* dz_ovf, int M, int f, int K, int cap,
-                             const CscBuffers& b, cudaStream_t s);
+                             const float* du_ovf, const float* dz_ovf, const int* plan, int M, int f, int K,
+                             int cap, const CscBuffers& b, cudaStream_t s);
 
-// dW_u = dU^T X, dW_g = dZ^T X, dW_d = dY^T H, db_g = column sums of dZ.
+// After the dense backward: the operands of the dense weight gradients (from X,
+// the gathered dY rows, fp32 dU / dZ and g, u of the overflow rows), column
+// sums of dZ over the overflow rows (db_ovf) and the contraction length
+// k_rows = roundup(n, 64) + n (0 when the plan keeps the overflow rows on the
+// sparse path, and then db_ovf = 0).
+cudaError_t launch_ovf_operands(const int* n_ovf, const int* ovf_rows, const int* plan, int cap, int d, int f,
+                                const uint16_t* X, const uint16_t* dy_ovf, const float* du_ovf, const float* dz_ovf,
+                                const uint16_t* g_ovf, const float* u_ovf, const DenseWgradOperands& op,
+                                float* db_ovf, int* k_rows, cudaStream_t s);
+
+// dW_u = dU^T X, dW_g = dZ^T X, dW_d = dY^T H, db_g = column sums of dZ (plus
+// db_extra when non-null) over the pairs of the pair list; the weight
+// gradients are added to what dW_* hold when *accumulate > 0 (accumulate
+// nullable), else overwritten.
 cudaError_t launch_weight_grads(const uint16_t* X, const uint16_t* dY, const CscBuffers& b, int d, int f,
-                                float* dW_g, float* dW_u, float* dW_d, float* db_g, cudaStream_t s);
+                                const float* db_extra, const int* accumulate, float* dW_g, float* dW_u,
+                                float* dW_d, float* db_g, cudaStream_t s);
 
 }  // namespace twell

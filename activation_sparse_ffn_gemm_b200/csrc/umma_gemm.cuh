@@ -1,8 +1,8 @@
 // umma_gemm.cuh — persistent, warp-specialised bf16 GEMM for sm_100a:
 //   C[M x N] = sum over K segments of A_s[M x K_s] * B_s^T, fp32 accumulation
 // with a pluggable epilogue that reads the accumulator straight from tensor
-// memory. A is K-major (rows of A contiguous along K); B is either K-major
-// ([N][K], like nn.Linear weights) or MN-major ([K][N]).
+// memory. A is K-major ([M][K], rows of A contiguous along K) or MN-major
+// ([K][M]); B is K-major ([N][K], like nn.Linear weights) or MN-major ([K][N]).
 //
 // Roles inside one 192-thread CTA (one CTA per SM):
 //   warp 0      TMA producer: 128-byte-swizzled A/B tiles into a STAGES-deep
@@ -48,6 +48,8 @@ struct GemmShape {
   int K0;            // K extent of segment 0 (multiple of kBK)
   int K1;            // K extent of segment 1 (0: single segment)
   uint32_t* status;
+  const int* K_dev = nullptr;  // single segment only: K processed = min(*K_dev, K0), rounded up to kBK
+                               // (operand rows between *K_dev and the rounding must read as zero)
   float* partial = nullptr;  // split-K partials [split_max][split_rows][N] fp32 (nullptr: no split-K)
   int split_rows = 0;        // split-K only when the processed rows are at most this many
   int split_max = 1;
@@ -112,7 +114,7 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int&
   nb = within / gm;
 }
 
-template <class Epi, int BN, bool B_MN, int STAGES>
+template <class Epi, int BN, bool B_MN, int STAGES, bool A_MN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                      const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
@@ -131,6 +133,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   int* m_eff_s = reinterpret_cast<int*>(smem + L::MISC_OFF + 8);
   volatile int* last_s = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 12);
   volatile int* epi_cnt = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 16);
+  int* k0_eff_s = reinterpret_cast<int*>(smem + L::MISC_OFF + 20);
   uint8_t* epi_smem = smem + L::EPI_OFF;
 
   const int warp = threadIdx.x >> 5;
@@ -145,9 +148,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       m = m < 0 ? 0 : m;
     }
     *m_eff_s = m;
+    int k0 = shp.K0;
+    if (shp.K_dev) {
+      int kv = *shp.K_dev;
+      kv = kv < 0 ? 0 : (kv > k0 ? k0 : kv);
+      k0 = (kv + kBK - 1) / kBK * kBK;
+    }
+    *k0_eff_s = k0;
   }
   __syncthreads();
-  const int nk = shp.K0 / kBK + shp.K1 / kBK;
+  const int nk0 = *k0_eff_s / kBK;
+  const int nk = nk0 + shp.K1 / kBK;
+  if (nk == 0) return;  // nothing to contract (a device-side K of zero)
   const int split = gemm_split(*m_eff_s, shp.N, BN, nk, shp, gridDim.x);
   if (static_cast<long>(blockIdx.x) >=
       static_cast<long>((*m_eff_s + kBM - 1) / kBM) * ((shp.N + BN - 1) / BN) * split)
@@ -188,7 +200,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int num_m = (M_eff + kBM - 1) / kBM;
   const int num_n = (shp.N + BN - 1) / BN;
   const int num_tiles = num_m * num_n * split;
-  const int nk0 = shp.K0 / kBK;
   // work item -> (output tile, K range [kb0, kb1)); split == 1: the whole K
   auto item = [&](int tile, int& mb, int& nb, int& ks, int& kb0, int& kb1) {
     ks = tile % split;
@@ -227,7 +238,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const CUtensorMap* mA = seg1 ? &tmA1 : &tmA0;
           const CUtensorMap* mB = seg1 ? &tmB1 : &tmB0;
           const int k = (seg1 ? kb - nk0 : kb) * kBK;
-          tma_load_2d(sA, mA, &full[stage], k, m0);
+          if (!A_MN) {
+            tma_load_2d(sA, mA, &full[stage], k, m0);
+          } else {
+#pragma unroll
+            for (int q = 0; q < kBM / 64; ++q) tma_load_2d(sA + q * (64 * kBK * 2), mA, &full[stage], m0 + 64 * q, k);
+          }
           if (!B_MN) {
             tma_load_2d(sB, mB, &full[stage], k, n0);
           } else {
@@ -253,7 +269,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // -------------------------------------------------------------- MMA issue
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, false, B_MN);
+      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -280,7 +296,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t b_base = a_base + L::A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t adesc = sdesc_sw128(a_base + kk * 32, 16, 1024);
+            const uint64_t adesc = A_MN ? sdesc_sw128(a_base + kk * 2048, 64 * kBK * 2, 1024)
+                                        : sdesc_sw128(a_base + kk * 32, 16, 1024);
             const uint64_t bdesc = B_MN ? sdesc_sw128(b_base + kk * 2048, 64 * kBK * 2, 1024)
                                         : sdesc_sw128(b_base + kk * 32, 16, 1024);
             umma_bf16(d_tmem, adesc, bdesc, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
@@ -402,13 +419,13 @@ constexpr int gemm_smem_bytes() {
 
 // Launches the GEMM on min(#SMs, tiles) persistent CTAs. The static row bound
 // shp.M sizes the grid; rows beyond *M_dev are skipped by the device.
-template <class Epi, int BN, bool B_MN, int STAGES>
+template <class Epi, int BN, bool B_MN, int STAGES, bool A_MN = false>
 cudaError_t launch_umma_gemm(const char* name, const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
                              const CUtensorMap& b1, const GemmShape& shp, const typename Epi::Args& ea,
                              cudaStream_t s) {
   constexpr int smem = gemm_smem_bytes<Epi, BN, STAGES>();
   static_assert(smem <= 232448, "shared memory budget");
-  auto kern = umma_gemm_kernel<Epi, BN, B_MN, STAGES>;
+  auto kern = umma_gemm_kernel<Epi, BN, B_MN, STAGES, A_MN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const long tiles = static_cast<long>((shp.M + kBM - 1) / kBM) * ((shp.N + BN - 1) / BN);

@@ -94,6 +94,10 @@ CASES = {
 # cases whose plan splits some rows into several pieces (the ordered
 # accumulation across pieces is exercised)
 SPLIT_CASES = ("k64", "long_rows_w2", "multi_tile")
+# cases whose overflow rows pass the cost model of the dense weight gradients
+# (54 and 93 overflow rows: the contraction's zeroed tail rows matter); the
+# others keep their overflow rows in the pair list
+DENSE_WGRAD_CASES = ("k32", "ragged_k16")
 
 
 @pytest.mark.parametrize("name", sorted(CASES))
@@ -106,6 +110,7 @@ def test_fwd_bwd_small(tw, orc, name):
     plan = assert_plan_valid(st)
     if name in SPLIT_CASES:
         assert plan["split_rows"] > 0, "this case should split rows into several pieces"
+    assert plan["dense_wgrad"] == (name in DENSE_WGRAD_CASES)
     for lam in (0.0, 1e-3):
         g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=lam)
         torch.cuda.synchronize()
@@ -133,6 +138,7 @@ def test_degenerate_all_active_dense_path(tw, orc):
     D, Y, st, z = _run_fwd(tw, inp, w)
     p, _, _ = _check_fwd(orc, inp, w, Y, st, z)
     assert p["n_ovf"] == 150 and p["row_ovf"].all()
+    assert assert_plan_valid(st)["dense_wgrad"]
     g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=1e-3)
     _check_bwd(orc, inp, g, gpu_gmat(p, 150, 384, 128, 8), 1e-3, "all-active")
 

@@ -78,12 +78,18 @@ def assert_plan_valid(st, groups_hint=None) -> dict:
     kept = np.minimum(count, K).sum(axis=1)
     assert 32 <= S <= 256, S
     assert total == int(kept[row_ovf == 0].sum())
+    # weight gradients of the overflow rows as dense GEMMs when their P active pairs
+    # over n rows satisfy the cost model P * 1000 > d_ff * (24 n + 12000)
+    n_rows, pairs = int((row_ovf != 0).sum()), int(count[row_ovf != 0].sum())
+    dense = n_rows > 0 and pairs * 1000 > st.d_ff * (24 * n_rows + 12000)
+    assert int(plan[3]) == int(dense)
     assert not plan[4:4 + M].any(), "turnstile words must be zero between passes"
     pieces = plan[4 + M:4 + M + 2 * npieces].reshape(-1, 2)
     want = [(r, q) for r in range(M) if not row_ovf[r]
             for q in range(max(1, -(-int(kept[r]) // S)))]
     assert [tuple(x) for x in pieces.tolist()] == want
-    return dict(pieces=npieces, S=S, total=total, split_rows=int(sum(1 for r, q in want if q == 1)))
+    return dict(pieces=npieces, S=S, total=total, split_rows=int(sum(1 for r, q in want if q == 1)),
+                dense_wgrad=dense)
 
 
 def gpu_mask(p: dict, M: int, f: int, T_n: int, K: int) -> np.ndarray:
