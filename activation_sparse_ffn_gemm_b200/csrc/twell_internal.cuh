@@ -30,8 +30,14 @@ constexpr int kTokListCap = 256;   // kept entries per list chunk of the token k
 constexpr int kPlanHdr = 4;
 // Cost model of the dense weight gradients of overflow rows (plan[3]), in
 // thousandths of d_ff pairs: per overflow row and fixed.
-constexpr long long kDenseWgradPerRow = 24;
-constexpr long long kDenseWgradFixed = 12000;  // one more pass over the fp32 gradients, about 10 d_ff pair gathers
+#ifndef TWELL_DENSE_WGRAD_PER_ROW
+#define TWELL_DENSE_WGRAD_PER_ROW 24
+#endif
+#ifndef TWELL_DENSE_WGRAD_FIXED
+#define TWELL_DENSE_WGRAD_FIXED 30000  // one more pass over the fp32 gradients (measured break-even)
+#endif
+constexpr long long kDenseWgradPerRow = TWELL_DENSE_WGRAD_PER_ROW;
+constexpr long long kDenseWgradFixed = TWELL_DENSE_WGRAD_FIXED;
 constexpr int kPieceMin = 32;
 constexpr long kPlanGroupsCap = 65536;  // bound on resident token groups of any device
 inline long plan_ints(long M, long T, long K) {

@@ -88,16 +88,19 @@ CASES = {
     # four and eight warps per token (d_model / 8 chunks of 16 bytes > 512)
     "wide_d_w4": (40, 8192, 1024, 16, 0.05, "none", 8),
     "widest_d_w8": (24, 16384, 512, 8, 0.03, "none", 10),
+    # overflow rows dense enough that their weight gradients run as GEMMs
+    # (190 and 183 overflow rows: the contraction's zeroed tail rows matter)
+    "dense_wgrad": (300, 256, 512, 8, 0.12, "lognormal", 17),
+    "dense_wgrad_ragged": (260, 192, 384, 8, 0.15, "lognormal", 19),
 }
 
 
 # cases whose plan splits some rows into several pieces (the ordered
 # accumulation across pieces is exercised)
 SPLIT_CASES = ("k64", "long_rows_w2", "multi_tile")
-# cases whose overflow rows pass the cost model of the dense weight gradients
-# (54 and 93 overflow rows: the contraction's zeroed tail rows matter); the
-# others keep their overflow rows in the pair list
-DENSE_WGRAD_CASES = ("k32", "ragged_k16")
+# cases whose overflow rows pass the cost model of the dense weight gradients;
+# the others keep their overflow rows in the pair list
+DENSE_WGRAD_CASES = ("dense_wgrad", "dense_wgrad_ragged")
 
 
 @pytest.mark.parametrize("name", sorted(CASES))

@@ -79,9 +79,9 @@ def assert_plan_valid(st, groups_hint=None) -> dict:
     assert 32 <= S <= 256, S
     assert total == int(kept[row_ovf == 0].sum())
     # weight gradients of the overflow rows as dense GEMMs when their P active pairs
-    # over n rows satisfy the cost model P * 1000 > d_ff * (24 n + 12000)
+    # over n rows satisfy the cost model P * 1000 > d_ff * (24 n + 30000)
     n_rows, pairs = int((row_ovf != 0).sum()), int(count[row_ovf != 0].sum())
-    dense = n_rows > 0 and pairs * 1000 > st.d_ff * (24 * n_rows + 12000)
+    dense = n_rows > 0 and pairs * 1000 > st.d_ff * (24 * n_rows + 30000)
     assert int(plan[3]) == int(dense)
     assert not plan[4:4 + M].any(), "turnstile words must be zero between passes"
     pieces = plan[4 + M:4 + M + 2 * npieces].reshape(-1, 2)
