@@ -25,11 +25,6 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // ------------------------------------------------------------------- CSC
 
-__global__ void row_slot_kernel(const int* __restrict__ ovf_rows, const int* __restrict__ n_ovf,
-                                int* __restrict__ row_slot) {
-  const int n = n_ovf[0];
-  for (int s = blockIdx.x * blockDim.x + threadIdx.x; s < n; s += gridDim.x * blockDim.x) row_slot[ovf_rows[s]] = s;
-}
 
 // The CSC is built per (unit tile t, chunk of kCscRows rows) with a counting
 // sort that keeps rows ascending inside each unit's list. Rows are taken in
@@ -445,12 +440,6 @@ cudaError_t launch_build_csc(const uint16_t* count, const uint16_t* val, const u
                              const float* du_ovf, const float* dz_ovf, const int* plan, int M, int f, int K,
                              int cap, const CscBuffers& b, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
-  cudaError_t e = cudaMemsetAsync(b.row_slot, 0xFF, static_cast<size_t>(M) * sizeof(int), s);
-  if (e != cudaSuccess) return e;
-  if (cap > 0) {
-    const int g = (cap + 255) / 256 < 1024 ? (cap + 255) / 256 : 1024;
-    TWELL_LAUNCH("row_slot", s, row_slot_kernel<<<g, 256, 0, s>>>(ovf_rows, n_ovf, b.row_slot));
-  }
   const int nch = (M + kCscRows - 1) / kCscRows;
   const int T = f / kTn;
   TWELL_LAUNCH("csc_count", s,

@@ -16,7 +16,6 @@ namespace twell {
 namespace {
 
 constexpr int kScanThreads = 1024;
-constexpr int kScanItems = 16;
 
 // row_ovf[i] = any_t(count[i][t] > K), and the row's kept entries
 // kept[i] = sum_t min(count[i][t], K), or -(1 + sum_t count[i][t]) for an
@@ -48,166 +47,165 @@ __global__ void row_flags_kernel(const uint16_t* __restrict__ count, int M, int 
   }
 }
 
-// Single block: the row plan of the token kernels (layout in twell_internal.cuh).
-// Reads the kept counts parked in the turnstile words, sizes the pieces
-// S = clamp(ceil(total / groups), kPieceMin, kTokListCap), lists the pieces
-// (max(1, ceil(kept / S)) per non-overflow row, none for overflow rows) and
-// zeroes the turnstile words. Thread t owns the consecutive rows
-// [t * per, (t + 1) * per): it reads its counts before it zeroes them.
-// plan[3] = 1 when the weight gradients of the n overflow rows (P active
-// pairs) run as dense GEMMs instead of through the pair list, decided by a
-// cost model: the dense GEMMs contract 2 n rows (hi and lo parts) for
-// 12 d_ff d_model n flops and write the full gradients once more, the sparse
-// path gathers two d_model-wide rows per pair, which gives
-// P * 1000 > d_ff * (kDenseWgradPerRow * n + kDenseWgradFixed) with the
-// measured B200 rates of the two (tensor-core flops vs L2 row gathers, HBM
-// writes vs L2 row gathers).
-__global__ void __launch_bounds__(kScanThreads) plan_kernel(int* __restrict__ plan, int M, int f, int groups) {
-  __shared__ long long red[kScanThreads / 32];
-  __shared__ long long red_ovf[kScanThreads / 32];
-  __shared__ long long red_rows[kScanThreads / 32];
-  __shared__ int warp_tot[kScanThreads / 32];
+// Single block, after row_flags: the ascending list of overflow rows and the
+// row plan of the token kernels (layout in twell_internal.cuh), from the kept
+// counts parked in the turnstile words (negative for overflow rows).
+//   * ovf_rows[0..min(n, cap)), n_ovf = {min(n, cap), n}, the capacity bit when
+//     n > cap, and row_slot[i] = the dense slot of row i (-1 when none);
+//   * pieces: S = clamp(ceil(total / groups), kPieceMin, kTokListCap);
+//     max(1, ceil(kept / S)) pieces per non-overflow row, none for overflow rows;
+//   * plan[3] = 1 when the weight gradients of the n overflow rows (P active
+//     pairs) run as dense GEMMs instead of through the pair list, by a cost
+//     model calibrated on B200 (tensor-core GEMMs over 2 n rows plus one more
+//     pass over the fp32 gradients, against two d_model-wide L2 row gathers
+//     per pair): P * 1000 > d_ff * (kDenseWgradPerRow * n + kDenseWgradFixed);
+//   * every turnstile word is left at zero.
+// Rows go in tiles of kScanThreads * kPlanItems; thread t owns kPlanItems
+// consecutive rows of a tile (read before it writes them).
+constexpr int kPlanItems = 8;
+
+__device__ __forceinline__ void load_kept(const int* kept, long r0, int M, int (&v)[kPlanItems]) {
+  if (r0 + kPlanItems <= M) {
+    const int4 a = *reinterpret_cast<const int4*>(kept + r0), b = *reinterpret_cast<const int4*>(kept + r0 + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+#pragma unroll
+    for (int e = 0; e < kPlanItems; ++e) v[e] = r0 + e < M ? kept[r0 + e] : 0;
+  }
+}
+
+// Block-wide exclusive scan of two counts; returns the block totals.
+__device__ __forceinline__ int2 block_scan2(int a, int b, int& ea, int& eb, int2* warp_tot) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int ia = a, ib = b;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int ta = __shfl_up_sync(0xFFFFFFFFu, ia, o), tb = __shfl_up_sync(0xFFFFFFFFu, ib, o);
+    if (lane >= o) {
+      ia += ta;
+      ib += tb;
+    }
+  }
+  if (lane == 31) warp_tot[w] = make_int2(ia, ib);
+  __syncthreads();
+  if (w == 0) {
+    const int2 t = warp_tot[lane];
+    int xa = t.x, xb = t.y;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int ta = __shfl_up_sync(0xFFFFFFFFu, xa, o), tb = __shfl_up_sync(0xFFFFFFFFu, xb, o);
+      if (lane >= o) {
+        xa += ta;
+        xb += tb;
+      }
+    }
+    warp_tot[lane] = make_int2(xa, xb);  // inclusive over warps
+  }
+  __syncthreads();
+  const int2 before = w > 0 ? warp_tot[w - 1] : make_int2(0, 0);
+  ea = before.x + ia - a;
+  eb = before.y + ib - b;
+  const int2 tot = warp_tot[kScanThreads / 32 - 1];
+  __syncthreads();
+  return tot;
+}
+
+__global__ void __launch_bounds__(kScanThreads) route_plan_kernel(int* __restrict__ plan, int M, int f, int groups,
+                                                                  int cap, int* __restrict__ ovf_rows,
+                                                                  int* __restrict__ n_ovf, uint32_t* status) {
+  __shared__ long long red[3][kScanThreads / 32];
+  __shared__ int2 warp_tot[kScanThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   int* kept = plan + kPlanHdr;
-  int* pieces = plan + kPlanHdr + M;
-  const long per = (static_cast<long>(M) + kScanThreads - 1) / kScanThreads;
-  const long r0 = tid * per, r1 = r0 + per < M ? r0 + per : M;
-  long long tot = 0, tot_ovf = 0, n_ovf_rows = 0;
-  for (long r = r0; r < r1; ++r) {
-    const int v = kept[r];
-    if (v > 0) tot += v;
-    if (v < 0) {
-      tot_ovf += -1LL - v;
-      ++n_ovf_rows;
+  int* row_slot = plan + kPlanHdr + M;
+  int* pieces = plan + kPlanHdr + 2L * M;
+  constexpr long kTile = static_cast<long>(kScanThreads) * kPlanItems;
+
+  long long tot = 0, tot_ovf = 0, rows_ovf = 0;
+  for (long base = 0; base < M; base += kTile) {
+    int v[kPlanItems];
+    load_kept(kept, base + static_cast<long>(tid) * kPlanItems, M, v);
+#pragma unroll
+    for (int e = 0; e < kPlanItems; ++e) {
+      if (v[e] > 0) tot += v[e];
+      if (v[e] < 0) {
+        tot_ovf += -1LL - v[e];
+        ++rows_ovf;
+      }
     }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     tot += __shfl_xor_sync(0xFFFFFFFFu, tot, o);
     tot_ovf += __shfl_xor_sync(0xFFFFFFFFu, tot_ovf, o);
-    n_ovf_rows += __shfl_xor_sync(0xFFFFFFFFu, n_ovf_rows, o);
+    rows_ovf += __shfl_xor_sync(0xFFFFFFFFu, rows_ovf, o);
   }
   if (lane == 0) {
-    red[w] = tot;
-    red_ovf[w] = tot_ovf;
-    red_rows[w] = n_ovf_rows;
+    red[0][w] = tot;
+    red[1][w] = tot_ovf;
+    red[2][w] = rows_ovf;
   }
   __syncthreads();
-  long long total = 0, total_ovf = 0, rows_ovf = 0;
+  long long total = 0, total_ovf = 0, n_rows_ovf = 0;
   for (int q = 0; q < kScanThreads / 32; ++q) {
-    total += red[q];
-    total_ovf += red_ovf[q];
-    rows_ovf += red_rows[q];
+    total += red[0][q];
+    total_ovf += red[1][q];
+    n_rows_ovf += red[2][q];
   }
   const long long g = groups > 0 ? groups : 1;
   long long sz = (total + g - 1) / g;
   sz = sz < kPieceMin ? kPieceMin : (sz > kTokListCap ? kTokListCap : sz);
   const int S = static_cast<int>(sz);
-  int mine = 0;
-  for (long r = r0; r < r1; ++r) {
-    const int v = kept[r];
-    mine += v < 0 ? 0 : (v > 0 ? (v + S - 1) / S : 1);
-  }
-  int incl = mine;
+
+  int carry_o = 0, carry_p = 0;
+  for (long base = 0; base < M; base += kTile) {
+    const long r0 = base + static_cast<long>(tid) * kPlanItems;
+    int v[kPlanItems];
+    load_kept(kept, r0, M, v);
+    int mo = 0, mp = 0;
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-    if (lane >= o) incl += t;
-  }
-  if (lane == 31) warp_tot[w] = incl;
-  __syncthreads();
-  if (w == 0) {
-    const int t = warp_tot[lane];
-    int ti = t;
+    for (int e = 0; e < kPlanItems; ++e) {
+      if (r0 + e >= M) continue;
+      mo += v[e] < 0;
+      mp += v[e] < 0 ? 0 : (v[e] > 0 ? (v[e] + S - 1) / S : 1);
+    }
+    int eo, ep;
+    const int2 t = block_scan2(mo, mp, eo, ep, warp_tot);
+    int pos = carry_o + eo, pc = carry_p + ep;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int q = __shfl_up_sync(0xFFFFFFFFu, ti, o);
-      if (lane >= o) ti += q;
+    for (int e = 0; e < kPlanItems; ++e) {
+      const long r = r0 + e;
+      if (r >= M) continue;
+      int slot = -1;
+      if (v[e] < 0) {
+        if (pos < cap) {
+          ovf_rows[pos] = static_cast<int>(r);
+          slot = pos;
+        }
+        ++pos;
+      } else {
+        const int P = v[e] > 0 ? (v[e] + S - 1) / S : 1;
+        for (int q = 0; q < P; ++q, ++pc) {
+          pieces[2L * pc] = static_cast<int>(r);
+          pieces[2L * pc + 1] = q;
+        }
+      }
+      row_slot[r] = slot;
+      kept[r] = 0;
     }
-    warp_tot[lane] = ti;  // inclusive
-  }
-  __syncthreads();
-  int base = (w > 0 ? warp_tot[w - 1] : 0) + incl - mine;
-  for (long r = r0; r < r1; ++r) {
-    const int v = kept[r];
-    const int P = v < 0 ? 0 : (v > 0 ? (v + S - 1) / S : 1);
-    for (int q = 0; q < P; ++q, ++base) {
-      pieces[2L * base] = static_cast<int>(r);
-      pieces[2L * base + 1] = q;
-    }
-    kept[r] = 0;
+    carry_o += t.x;
+    carry_p += t.y;
   }
   if (tid == 0) {
-    plan[0] = warp_tot[kScanThreads / 32 - 1];
+    n_ovf[0] = carry_o < cap ? carry_o : cap;
+    n_ovf[1] = carry_o;
+    if (carry_o > cap) set_status(status, TWELL_STATUS_OVERFLOW_CAP);
+    plan[0] = carry_p;
     plan[1] = S;
     plan[2] = static_cast<int>(total < 0x7FFFFFFFLL ? total : 0x7FFFFFFFLL);
-    plan[3] = rows_ovf > 0 && total_ovf * 1000 > static_cast<long long>(f) * (kDenseWgradPerRow * rows_ovf +
-                                                                              kDenseWgradFixed)
+    plan[3] = n_rows_ovf > 0 && total_ovf * 1000 > static_cast<long long>(f) * (kDenseWgradPerRow * n_rows_ovf +
+                                                                                kDenseWgradFixed)
                   ? 1 : 0;
-  }
-}
-
-// Single-block ascending compaction of flagged rows. Writes ovf_rows[0..min(n, cap)),
-// n_ovf[0] = min(n, cap), n_ovf[1] = n, and sets the capacity bit when n > cap.
-__global__ void __launch_bounds__(kScanThreads) ovf_scan_kernel(const uint8_t* __restrict__ row_ovf, int M,
-                                                                 int cap, int* __restrict__ ovf_rows,
-                                                                 int* __restrict__ n_ovf, uint32_t* status) {
-  __shared__ int warp_tot[kScanThreads / 32];
-  __shared__ int carry_s;
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  if (tid == 0) carry_s = 0;
-  __syncthreads();
-  for (long base = 0; base < M; base += static_cast<long>(kScanThreads) * kScanItems) {
-    const long r0 = base + static_cast<long>(tid) * kScanItems;
-    uint8_t f[kScanItems];
-    if (r0 + kScanItems <= M) {
-      const uint4 v = *reinterpret_cast<const uint4*>(row_ovf + r0);
-      const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int e = 0; e < kScanItems; ++e) f[e] = (ww[e / 4] >> (8 * (e % 4))) & 0xFFu;
-    } else {
-#pragma unroll
-      for (int e = 0; e < kScanItems; ++e) f[e] = (r0 + e < M) ? row_ovf[r0 + e] : 0;
-    }
-    int mine = 0;
-#pragma unroll
-    for (int e = 0; e < kScanItems; ++e) mine += f[e] != 0;
-    int incl = mine;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    if (lane == 31) warp_tot[w] = incl;
-    __syncthreads();
-    if (w == 0) {
-      int t = warp_tot[lane];
-      int ti = t;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xFFFFFFFFu, ti, o);
-        if (lane >= o) ti += v;
-      }
-      warp_tot[lane] = ti - t;  // exclusive prefix over warps
-    }
-    __syncthreads();
-    int pos = carry_s + warp_tot[w] + incl - mine;
-#pragma unroll
-    for (int e = 0; e < kScanItems; ++e) {
-      if (f[e]) {
-        if (pos < cap) ovf_rows[pos] = static_cast<int>(r0 + e);
-        ++pos;
-      }
-    }
-    __syncthreads();
-    if (tid == kScanThreads - 1) carry_s = pos;
-    __syncthreads();
-  }
-  if (tid == 0) {
-    const int n = carry_s;
-    n_ovf[0] = n < cap ? n : cap;
-    n_ovf[1] = n;
-    if (n > cap) set_status(status, TWELL_STATUS_OVERFLOW_CAP);
   }
 }
 
@@ -304,8 +302,8 @@ cudaError_t launch_route(const uint16_t* count, const uint16_t* val, const uint8
   const int max_blocks = device_sm_count() * 16;
   if (blocks > max_blocks) blocks = max_blocks;
   TWELL_LAUNCH("row_flags", s, row_flags_kernel<<<blocks, 256, 0, s>>>(count, M, T, K, row_ovf, plan + kPlanHdr));
-  TWELL_LAUNCH("ovf_scan", s, ovf_scan_kernel<<<1, kScanThreads, 0, s>>>(row_ovf, M, cap, ovf_rows, n_ovf, status));
-  TWELL_LAUNCH("row_plan", s, plan_kernel<<<1, kScanThreads, 0, s>>>(plan, M, f, groups));
+  TWELL_LAUNCH("route_plan", s,
+               route_plan_kernel<<<1, kScanThreads, 0, s>>>(plan, M, f, groups, cap, ovf_rows, n_ovf, status));
   if (cap > 0) {
     int g = cap < device_sm_count() * 4 ? cap : device_sm_count() * 4;
     TWELL_LAUNCH("ovf_gather", s,

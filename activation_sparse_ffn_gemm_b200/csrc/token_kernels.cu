@@ -297,7 +297,7 @@ __device__ __forceinline__ bool next_piece(int* ctr, const int* plan, int M, con
   const int np = plan[0], S = plan[1];
   const int p = static_cast<int>(next_row<W>(ctr, grp, wi, lane, s_next));
   if (p >= np) return false;
-  const int* pieces = plan + kPlanHdr + M;
+  const int* pieces = plan + kPlanHdr + 2L * M;
   const int row = pieces[2 * p], q = pieces[2 * p + 1];
   if (wi == 0) row_offsets(count, row, T, K, lane, g);
   if (wi == 0 && lane == 0) {

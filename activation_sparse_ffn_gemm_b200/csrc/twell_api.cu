@@ -79,7 +79,7 @@ struct WsLayout {
   size_t sk_partial = 0, sk_arrivals = 0;  // split-K scratch of the dense-backup GEMMs
   size_t spill = 0, x_ovf = 0, h_ovf = 0, w_dt = 0;
   size_t x2 = 0, dy2 = 0, duz2 = 0, h2 = 0, db_ovf = 0, k_rows = 0;  // operands of the dense weight gradients
-  size_t dy_ovf = 0, duz = 0, du_ovf = 0, dz_ovf = 0, du_ell = 0, dz_ell = 0, row_slot = 0, block_cnt = 0, unit_tot = 0, unit_ptr = 0,
+  size_t dy_ovf = 0, duz = 0, du_ovf = 0, dz_ovf = 0, du_ell = 0, dz_ell = 0, block_cnt = 0, unit_tot = 0, unit_ptr = 0,
          csc_row = 0, csc_val = 0;
   size_t total = 0;
 };
@@ -121,7 +121,6 @@ WsLayout ws_layout(twell_op op, int64_t M, int64_t d, int64_t f, int64_t K, int6
     L.k_rows = take(64);
     L.du_ell = take(static_cast<size_t>(M * T * K * 4));
     L.dz_ell = take(static_cast<size_t>(M * T * K * 4));
-    L.row_slot = take(static_cast<size_t>(M * 4));
     const int64_t nrb = (M + kCscRows - 1) / kCscRows;
     L.block_cnt = take(static_cast<size_t>(nrb * f * 4));
     L.unit_tot = take(static_cast<size_t>(f * 4));
@@ -333,7 +332,7 @@ twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_
   if (launch_ovf_operands(h->n_ovf, h->ovf_rows, h->row_plan, cap, d, f, X, dy_ovf, du_ovf, dz_ovf, h->g_ovf,
                           h->u_ovf, dw, db_ovf, k_rows, s) != cudaSuccess)
     return TWELL_ECUDA;
-  CscBuffers b{at<int>(ws, L.row_slot), at<int>(ws, L.block_cnt), at<int>(ws, L.unit_tot),
+  CscBuffers b{h->row_plan + kPlanHdr + M, at<int>(ws, L.block_cnt), at<int>(ws, L.unit_tot),
                at<int>(ws, L.unit_ptr), at<int>(ws, L.csc_row), at<float4>(ws, L.csc_val)};
   if (launch_build_csc(h->count, h->val, h->col, h->row_ovf, h->ovf_rows, h->n_ovf, h->g_ovf, h->u_ell, h->u_ovf,
                        du_ell, dz_ell, du_ovf, dz_ovf, h->row_plan, M, f, K, cap, b, s) != cudaSuccess)

@@ -22,8 +22,9 @@ constexpr int kTokListCap = 256;   // kept entries per list chunk of the token k
 // pieces of at most S kept entries of one non-overflow row.
 //   [0] number of pieces, [1] S, [2] kept entries of non-overflow rows,
 //   [3] 1 when the weight gradients of the overflow rows run as dense GEMMs
-//   [kPlanHdr, kPlanHdr + M)  per-row turnstile words (0 between launches;
-//                             the routing step parks the kept counts there)
+//   [kPlanHdr, kPlanHdr + M)       per-row turnstile words (0 between launches;
+//                                  the routing step parks the kept counts there)
+//   [kPlanHdr + M, kPlanHdr + 2M)  row_slot: dense backup slot of each row, -1 if none
 //   then (row, q) int pairs, piece q of row, ascending rows then q
 // S = clamp(ceil(kept / resident groups), kPieceMin, kTokListCap), so the
 // pieces number at most M + max(groups, M * T * K / kTokListCap).
@@ -42,7 +43,7 @@ constexpr int kPieceMin = 32;
 constexpr long kPlanGroupsCap = 65536;  // bound on resident token groups of any device
 inline long plan_ints(long M, long T, long K) {
   const long spill = (M * T * K + kTokListCap - 1) / kTokListCap;
-  return kPlanHdr + M + 2 * (M + (spill > kPlanGroupsCap ? spill : kPlanGroupsCap));
+  return kPlanHdr + 2 * M + 2 * (M + (spill > kPlanGroupsCap ? spill : kPlanGroupsCap));
 }
 
 // ------------------------------------------------------------ device helpers
@@ -193,7 +194,7 @@ cudaError_t launch_dense_wgrad(const DenseWgradOperands& op, const int* k_rows, 
                                float* dW_u, float* dW_d, uint32_t* status, cudaStream_t s);
 
 struct CscBuffers {
-  int* row_slot;   // [M]
+  const int* row_slot;  // [M] dense backup slot of each row (-1: none), from the row plan
   int* block_cnt;  // [ceil(M/kCscRows)][f] per-chunk counts, then their exclusive scan
   int* unit_tot;   // [f]
   int* unit_ptr;   // [f+1]

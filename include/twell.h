@@ -129,7 +129,7 @@ TWELL_API twell_status twell_query_support(int64_t M, int64_t d_model, int64_t d
                                  int64_t ovf_cap);
 
 /* Elements (int32) of twell_hybrid::row_plan for this shape (0 for an invalid
- * one): 4 + M + 2 * (M + max(65536, ceil(M * (d_ff / T_n) * K / 256))). */
+ * one): 4 + 2 * M + 2 * (M + max(65536, ceil(M * (d_ff / T_n) * K / 256))). */
 TWELL_API size_t twell_plan_ints(int64_t M, int64_t d_ff, int64_t T_n, int64_t K);
 
 /* Workspace bytes that `op` needs for this shape (0 for an unsupported shape).

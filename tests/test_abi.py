@@ -53,10 +53,10 @@ def test_hybrid_struct_matches_header(tw):
 
 def test_plan_ints(tw):
     L = tw.lib()
-    # 4 + M + 2 * (M + max(65536, ceil(M * T * K / 256)))
-    assert L.twell_plan_ints(4096, 8192, 128, 8) == 4 + 4096 + 2 * (4096 + 65536)
+    # 4 + 2 M + 2 * (M + max(65536, ceil(M * T * K / 256)))
+    assert L.twell_plan_ints(4096, 8192, 128, 8) == 4 + 2 * 4096 + 2 * (4096 + 65536)
     big = 65536 * 112 * 64 // 256
-    assert L.twell_plan_ints(65536, 14336, 128, 64) == 4 + 65536 + 2 * (65536 + big)
+    assert L.twell_plan_ints(65536, 14336, 128, 64) == 4 + 2 * 65536 + 2 * (65536 + big)
     assert L.twell_plan_ints(0, 8192, 128, 8) == 4 + 2 * 65536
     assert L.twell_plan_ints(16, 8192, 64, 8) == 0
 

@@ -240,7 +240,7 @@ def test_heavy_tail_full_size(tw, orc):
     ovf_sample = rng.choice(p["ovf_rows"], size=min(64, p["n_ovf"]), replace=False)
     plan = assert_plan_valid(st)
     assert plan["split_rows"] > 0  # the heavy ELL rows are split into pieces
-    pieces = st.row_plan.cpu().numpy()[4 + w.M:4 + w.M + 2 * plan["pieces"]].reshape(-1, 2)
+    pieces = st.row_plan.cpu().numpy()[4 + 2 * w.M:4 + 2 * w.M + 2 * plan["pieces"]].reshape(-1, 2)
     split = np.unique(pieces[pieces[:, 1] == 1, 0])
     split_sample = rng.choice(split, size=min(32, split.size), replace=False)
     rows = _sample_rows(w.M, 128, 1, extra=np.concatenate([ovf_sample, split_sample]))

@@ -84,7 +84,12 @@ def assert_plan_valid(st, groups_hint=None) -> dict:
     dense = n_rows > 0 and pairs * 1000 > st.d_ff * (24 * n_rows + 30000)
     assert int(plan[3]) == int(dense)
     assert not plan[4:4 + M].any(), "turnstile words must be zero between passes"
-    pieces = plan[4 + M:4 + M + 2 * npieces].reshape(-1, 2)
+    slots = plan[4 + M:4 + 2 * M]
+    want_slot = np.full(M, -1)
+    ovf_list = st.ovf_rows.cpu().numpy()[:st.n_overflow()[0]]
+    want_slot[ovf_list] = np.arange(ovf_list.size)
+    assert np.array_equal(slots, want_slot), "row_slot: dense slot of each row"
+    pieces = plan[4 + 2 * M:4 + 2 * M + 2 * npieces].reshape(-1, 2)
     want = [(r, q) for r in range(M) if not row_ovf[r]
             for q in range(max(1, -(-int(kept[r]) // S)))]
     assert [tuple(x) for x in pieces.tolist()] == want
