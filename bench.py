@@ -185,24 +185,40 @@ def kernel_work(name, M, d, f, T, K, kept, pairs):
     return None, None
 
 
-def source_hash():
+# Source files that define each traced kernel's code (its own translation unit
+# and the headers it compiles in); a committed DRAM capture applies only while
+# these files are unchanged.
+KERNEL_SOURCES = {
+    "gate_pack_gemm": ("gemm_kernels.cu", "umma_gemm.cuh", "sm100.cuh", "twell_internal.cuh"),
+    "ell_updown": ("token_kernels.cu", "sm100.cuh", "twell_internal.cuh"),
+    "ell_bwd": ("token_kernels.cu", "sm100.cuh", "twell_internal.cuh"),
+    "weight_grads": ("pairlist_kernels.cu", "twell_internal.cuh"),
+    "csc_fill": ("pairlist_kernels.cu", "twell_internal.cuh"),
+    "transpose_wd": ("route_kernels.cu", "twell_internal.cuh"),
+}
+
+
+def source_hash(kernel):
+    files = KERNEL_SOURCES.get(kernel)
+    if not files:
+        return None
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "activation_sparse_ffn_gemm_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
+    for fn in files:
         with open(os.path.join(csrc, fn), "rb") as fh:
             h.update(fn.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
 def committed_traffic(kernel):
-    """DRAM bytes per launch from the committed ncu summary, if it matches this source."""
+    """DRAM bytes per launch from the committed ncu capture, if the kernel's sources still match."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as fh:
         d = json.load(fh)
     rec = d.get("kernels", {}).get(kernel)
-    if not rec or d.get("source_sha") != source_hash():
+    if not rec or rec.get("source_sha") != source_hash(kernel):
         return None
     return rec.get("dram_bytes_per_launch")
 
