@@ -99,43 +99,63 @@ __global__ void __launch_bounds__(256) csc_count_kernel(const uint16_t* __restri
   if (threadIdx.x < kTn) chunk_cnt[static_cast<long>(chunk) * f + t * kTn + threadIdx.x] = cnt_s[threadIdx.x];
 }
 
-// Per unit: exclusive scan over the row blocks (in place) and the unit total.
-// Loads of a batch are issued before its stores so they overlap.
+// Per unit j: exclusive scan over the row chunks (in place) and the unit
+// total; then unit_ptr = exclusive scan of the totals, unit_ptr[f] = total,
+// done by the block that finishes last (arrival words tagged with the
+// launch's epoch, so their initial contents do not matter). Loads of a batch
+// are issued before its stores so they overlap.
 constexpr int kColScanBatch = 16;
-__global__ void csc_colscan_kernel(int* __restrict__ block_cnt, int nrb, int f, int* __restrict__ unit_tot) {
+constexpr int kScanBlock = 1024;
+constexpr int kScanVec = kMaxTiles * kTn / (kScanBlock * 4);  // int4 of unit totals per thread, at most
+__global__ void __launch_bounds__(kScanBlock) csc_scan_kernel(int* __restrict__ block_cnt, int nrb, int f,
+                                                              int* __restrict__ unit_tot, int* __restrict__ unit_ptr,
+                                                              unsigned long long* __restrict__ arrive,
+                                                              unsigned long long epoch) {
+  __shared__ int last_s;
+  __shared__ int wsum[kScanBlock / 32];
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= f) return;
-  int run = 0;
-  for (int rb0 = 0; rb0 < nrb; rb0 += kColScanBatch) {
-    int c[kColScanBatch];
+  if (j < f) {
+    int run = 0;
+    for (int rb0 = 0; rb0 < nrb; rb0 += kColScanBatch) {
+      int c[kColScanBatch];
 #pragma unroll
-    for (int q = 0; q < kColScanBatch; ++q)
-      c[q] = rb0 + q < nrb ? block_cnt[static_cast<long>(rb0 + q) * f + j] : 0;
+      for (int q = 0; q < kColScanBatch; ++q)
+        c[q] = rb0 + q < nrb ? block_cnt[static_cast<long>(rb0 + q) * f + j] : 0;
 #pragma unroll
-    for (int q = 0; q < kColScanBatch; ++q) {
-      if (rb0 + q < nrb) block_cnt[static_cast<long>(rb0 + q) * f + j] = run;
-      run += c[q];
+      for (int q = 0; q < kColScanBatch; ++q) {
+        if (rb0 + q < nrb) block_cnt[static_cast<long>(rb0 + q) * f + j] = run;
+        run += c[q];
+      }
     }
+    unit_tot[j] = run;
   }
-  unit_tot[j] = run;
-}
-
-// Single block: unit_ptr = exclusive scan of unit_tot, unit_ptr[f] = total.
-// Thread t owns the consecutive units [t*per, (t+1)*per), per = ceil(f/1024)
-// <= kMaxTiles*kTn/1024; one block-wide scan of the per-thread sums.
-constexpr int kUnitScanPer = kMaxTiles * kTn / 1024;
-__global__ void __launch_bounds__(1024) csc_unit_scan_kernel(const int* __restrict__ unit_tot, int f,
-                                                             int* __restrict__ unit_ptr) {
-  __shared__ int wsum[32];
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(arrive), nw;
+    for (;;) {
+      nw = (cur >> 24) == epoch ? cur + 1 : ((epoch << 24) | 1ull);
+      const unsigned long long seen = atomicCAS(arrive, cur, nw);
+      if (seen == cur) break;
+      cur = seen;
+    }
+    last_s = static_cast<int>(nw & 0xFFFFFFull) == static_cast<int>(gridDim.x);
+  }
+  __syncthreads();
+  if (!last_s) return;
+  __threadfence();
+  // thread t owns the consecutive units [t * per, (t + 1) * per), per a
+  // multiple of 4 (d_ff is a multiple of 128), read and written as int4
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  const int per = (f + 1023) / 1024;
-  const int j0 = tid * per;
-  int v[kUnitScanPer];
+  const int per4 = (f + 4 * kScanBlock - 1) / (4 * kScanBlock);
+  const int j0 = tid * per4 * 4;
+  int4 v[kScanVec];
   int tot = 0;
 #pragma unroll
-  for (int q = 0; q < kUnitScanPer; ++q) {
-    v[q] = (q < per && j0 + q < f) ? unit_tot[j0 + q] : 0;
-    tot += v[q];
+  for (int q = 0; q < kScanVec; ++q) {
+    v[q] = make_int4(0, 0, 0, 0);
+    if (q < per4 && j0 + 4 * q < f) v[q] = __ldcg(reinterpret_cast<const int4*>(unit_tot + j0 + 4 * q));
+    tot += v[q].x + v[q].y + v[q].z + v[q].w;
   }
   int incl = tot;
 #pragma unroll
@@ -145,31 +165,29 @@ __global__ void __launch_bounds__(1024) csc_unit_scan_kernel(const int* __restri
   }
   if (lane == 31) wsum[w] = incl;
   __syncthreads();
-  if (w == 0) {
-    const int t = wsum[lane];
-    int ti = t;
+  int before = 0;
+  for (int q = 0; q < w; ++q) before += wsum[q];
+  int run = before + incl - tot;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int q = __shfl_up_sync(0xFFFFFFFFu, ti, o);
-      if (lane >= o) ti += q;
+  for (int q = 0; q < kScanVec; ++q) {
+    if (q < per4 && j0 + 4 * q < f) {
+      int4 o;
+      o.x = run;
+      o.y = o.x + v[q].x;
+      o.z = o.y + v[q].y;
+      o.w = o.z + v[q].z;
+      run = o.w + v[q].w;
+      *reinterpret_cast<int4*>(unit_ptr + j0 + 4 * q) = o;
     }
-    wsum[lane] = ti - t;
   }
-  __syncthreads();
-  int run = wsum[w] + incl - tot;
-#pragma unroll
-  for (int q = 0; q < kUnitScanPer; ++q) {
-    if (q < per && j0 + q < f) unit_ptr[j0 + q] = run;
-    run += v[q];
-  }
-  if (tid == 1023) unit_ptr[f] = run;
+  if (tid == kScanBlock - 1) unit_ptr[f] = run;
 }
 
 __global__ void __launch_bounds__(256) csc_fill_kernel(
     const uint16_t* __restrict__ count, const uint16_t* __restrict__ val, const uint8_t* __restrict__ col,
     const uint8_t* __restrict__ row_ovf, const int* __restrict__ row_slot, const uint16_t* __restrict__ g_ovf,
-    const float* __restrict__ u_ell, const float* __restrict__ u_ovf, const float* __restrict__ du_ell,
-    const float* __restrict__ dz_ell, const float* __restrict__ du_ovf, const float* __restrict__ dz_ovf,
+    const float* __restrict__ u_ovf, const float4* __restrict__ hdz_ell, const float* __restrict__ du_ovf,
+    const float* __restrict__ dz_ovf,
     const int* __restrict__ chunk_base, const int* __restrict__ unit_ptr, const int* __restrict__ plan, int M, int f,
     int K, int* __restrict__ csc_row, float4* __restrict__ csc_val) {
   __shared__ uint32_t mask[kCscGroups][kTn];
@@ -205,8 +223,7 @@ __global__ void __launch_bounds__(256) csc_fill_kernel(
       const int p = gbase[g][c] + __popc(mask[g][c] & below);
       float4 v;
       if (slot >= 0) {
-        const float gv = __uint_as_float(static_cast<uint32_t>(val[slot]) << 16);
-        v = make_float4(gv * u_ell[slot], du_ell[slot], dz_ell[slot], 0.f);
+        v = hdz_ell[slot];
       } else {
         const long o = static_cast<long>(sl) * f + t * kTn + c;
         const float gv = __uint_as_float(static_cast<uint32_t>(g_ovf[o]) << 16);
@@ -436,7 +453,7 @@ cudaError_t launch_ovf_operands(const int* n_ovf, const int* ovf_rows, const int
 
 cudaError_t launch_build_csc(const uint16_t* count, const uint16_t* val, const uint8_t* col,
                              const uint8_t* row_ovf, const int* ovf_rows, const int* n_ovf, const uint16_t* g_ovf,
-                             const float* u_ell, const float* u_ovf, const float* du_ell, const float* dz_ell,
+                             const float* u_ovf, const float4* hdz_ell,
                              const float* du_ovf, const float* dz_ovf, const int* plan, int M, int f, int K,
                              int cap, const CscBuffers& b, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
@@ -445,11 +462,12 @@ cudaError_t launch_build_csc(const uint16_t* count, const uint16_t* val, const u
   TWELL_LAUNCH("csc_count", s,
                csc_count_kernel<<<dim3(T, nch), 256, 0, s>>>(count, col, row_ovf, b.row_slot, g_ovf, plan, M, f,
                                                             K, b.block_cnt));
-  TWELL_LAUNCH("csc_colscan", s, csc_colscan_kernel<<<(f + 255) / 256, 256, 0, s>>>(b.block_cnt, nch, f, b.unit_tot));
-  TWELL_LAUNCH("csc_unit_scan", s, csc_unit_scan_kernel<<<1, 1024, 0, s>>>(b.unit_tot, f, b.unit_ptr));
+  TWELL_LAUNCH("csc_scan", s,
+               csc_scan_kernel<<<(f + kScanBlock - 1) / kScanBlock, kScanBlock, 0, s>>>(
+                   b.block_cnt, nch, f, b.unit_tot, b.unit_ptr, b.arrive, next_launch_epoch() & ((1ull << 40) - 1)));
   TWELL_LAUNCH("csc_fill", s,
-               csc_fill_kernel<<<dim3(T, nch), 256, 0, s>>>(count, val, col, row_ovf, b.row_slot, g_ovf, u_ell, u_ovf,
-                                                           du_ell, dz_ell, du_ovf, dz_ovf, b.block_cnt, b.unit_ptr, plan,
+               csc_fill_kernel<<<dim3(T, nch), 256, 0, s>>>(count, val, col, row_ovf, b.row_slot, g_ovf, u_ovf,
+                                                           hdz_ell, du_ovf, dz_ovf, b.block_cnt, b.unit_ptr, plan,
                                                            M, f, K, b.csc_row, b.csc_val));
   return cudaGetLastError();
 }

@@ -160,14 +160,14 @@ __global__ void __launch_bounds__(kScanThreads) route_plan_kernel(int* __restric
   int carry_o = 0, carry_p = 0;
   for (long base = 0; base < M; base += kTile) {
     const long r0 = base + static_cast<long>(tid) * kPlanItems;
-    int v[kPlanItems];
+    int v[kPlanItems], P[kPlanItems];
     load_kept(kept, r0, M, v);
     int mo = 0, mp = 0;
 #pragma unroll
     for (int e = 0; e < kPlanItems; ++e) {
-      if (r0 + e >= M) continue;
-      mo += v[e] < 0;
-      mp += v[e] < 0 ? 0 : (v[e] > 0 ? (v[e] + S - 1) / S : 1);
+      P[e] = (r0 + e >= M || v[e] < 0) ? 0 : (v[e] > 0 ? (v[e] + S - 1) / S : 1);
+      mo += r0 + e < M && v[e] < 0;
+      mp += P[e];
     }
     int eo, ep;
     const int2 t = block_scan2(mo, mp, eo, ep, warp_tot);
@@ -184,8 +184,7 @@ __global__ void __launch_bounds__(kScanThreads) route_plan_kernel(int* __restric
         }
         ++pos;
       } else {
-        const int P = v[e] > 0 ? (v[e] + S - 1) / S : 1;
-        for (int q = 0; q < P; ++q, ++pc) {
+        for (int q = 0; q < P[e]; ++q, ++pc) {
           pieces[2L * pc] = static_cast<int>(r);
           pieces[2L * pc + 1] = q;
         }

@@ -9,8 +9,8 @@
 //   Y_i  = sum_j h_ij W_d[:, j]    (W_d gathered unit-major from W_dt[j])
 // Backward over the same rows (same page, paragraph 2: training runs on the
 // hybrid format): dH_ij = dY_i . W_d[:, j], dU = dH g, dZ = dH u + lambda,
-// dX_i = sum_j dU_ij W_u[j] + dZ_ij W_g[j]; dU and dZ are kept per slot for the
-// weight gradients.
+// dX_i = sum_j dU_ij W_u[j] + dZ_ij W_g[j]; (h, dU, dZ) are kept per slot for
+// the weight gradients.
 //
 // The work is a stream of weight-row gathers from L2 (each active pair reads
 // whole d-wide rows), so the kernels are organised to keep many independent
@@ -393,8 +393,8 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
     const uint16_t* __restrict__ dY, const uint16_t* __restrict__ Wu, const uint16_t* __restrict__ Wg,
     const uint16_t* __restrict__ Wdt, const uint16_t* __restrict__ count, const uint16_t* __restrict__ val,
     const uint8_t* __restrict__ col, int* __restrict__ plan, const float* __restrict__ u_ell, float lambda,
-    float* __restrict__ du_ell, float* __restrict__ dz_ell, float* __restrict__ dX, int M, int d, int T, int K,
-    int* __restrict__ ctr, uint32_t* status) {
+    float4* __restrict__ hdz_ell, float* __restrict__ dX, int M, int d, int T, int K, int* __restrict__ ctr,
+    uint32_t* status) {
   using Cfg = TokCfg<C, W>;
   constexpr int B = Cfg::B;
   constexpr int B2 = B > 1 ? B / 2 : 1;  // two rows (W_u, W_g) per unit in the dX phase
@@ -424,12 +424,12 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
 #pragma unroll
         for (int w = 0; w < W; ++w) s += part[grp][w][e];
       }
-      const float du = s * g.c[e];
-      const float dz = fmaf(s, g.c2[e], lambda);
+      const float gv = g.c[e], uv = g.c2[e];
+      const float du = s * gv;
+      const float dz = fmaf(s, uv, lambda);
       g.c[e] = du;
       g.c2[e] = dz;
-      du_ell[row * T * K + g.slot[e]] = du;
-      dz_ell[row * T * K + g.slot[e]] = dz;
+      hdz_ell[row * T * K + g.slot[e]] = make_float4(gv * uv, du, dz, 0.f);
     }
     group_sync<W>(grp);
   };
@@ -532,8 +532,8 @@ cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uin
 
 cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const uint16_t* W_g,
                                const uint16_t* W_dt, const uint16_t* count, const uint16_t* val,
-                               const uint8_t* col, int* plan, const float* u_ell, float lambda, float* du_ell,
-                               float* dz_ell, float* dX, int M, int d, int f, int K, int* ctr, uint32_t* status,
+                               const uint8_t* col, int* plan, const float* u_ell, float lambda, float4* hdz_ell,
+                               float* dX, int M, int d, int f, int K, int* ctr, uint32_t* status,
                                cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
@@ -543,10 +543,10 @@ cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const ui
   const int T = f / kTn;
   const bool exact = d / 8 == W * 32 * C;
 #define TWELL_BWD(CC, WW)                                                                                        \
-  (exact ? launch_bwd_cw<CC, WW, true>(M, s, dY, W_u, W_g, W_dt, count, val, col, plan, u_ell, lambda, du_ell,  \
-                                       dz_ell, dX, M, d, T, K, ctr, status)                                    \
-         : launch_bwd_cw<CC, WW, false>(M, s, dY, W_u, W_g, W_dt, count, val, col, plan, u_ell, lambda, du_ell, \
-                                        dz_ell, dX, M, d, T, K, ctr, status))
+  (exact ? launch_bwd_cw<CC, WW, true>(M, s, dY, W_u, W_g, W_dt, count, val, col, plan, u_ell, lambda, hdz_ell, \
+                                       dX, M, d, T, K, ctr, status)                                           \
+         : launch_bwd_cw<CC, WW, false>(M, s, dY, W_u, W_g, W_dt, count, val, col, plan, u_ell, lambda, hdz_ell, \
+                                        dX, M, d, T, K, ctr, status))
   if (W == 1 && C == 1) TWELL_BWD(1, 1);
   else if (W == 1 && C == 2) TWELL_BWD(2, 1);
   else if (W == 1 && C == 4) TWELL_BWD(4, 1);

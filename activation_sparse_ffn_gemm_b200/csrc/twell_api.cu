@@ -23,7 +23,7 @@ int device_sm_count() {
   return v;
 }
 
-unsigned long long next_gemm_epoch() {
+unsigned long long next_launch_epoch() {
   static std::atomic<unsigned long long> next{1};
   constexpr unsigned long long kMask = (1ull << 56) - 1;
   for (;;) {
@@ -79,7 +79,7 @@ struct WsLayout {
   size_t sk_partial = 0, sk_arrivals = 0;  // split-K scratch of the dense-backup GEMMs
   size_t spill = 0, x_ovf = 0, h_ovf = 0, w_dt = 0;
   size_t x2 = 0, dy2 = 0, duz2 = 0, h2 = 0, db_ovf = 0, k_rows = 0;  // operands of the dense weight gradients
-  size_t dy_ovf = 0, duz = 0, du_ovf = 0, dz_ovf = 0, du_ell = 0, dz_ell = 0, block_cnt = 0, unit_tot = 0, unit_ptr = 0,
+  size_t dy_ovf = 0, duz = 0, du_ovf = 0, dz_ovf = 0, hdz_ell = 0, block_cnt = 0, unit_tot = 0, unit_ptr = 0, scan_arrive = 0,
          csc_row = 0, csc_val = 0;
   size_t total = 0;
 };
@@ -119,11 +119,11 @@ WsLayout ws_layout(twell_op op, int64_t M, int64_t d, int64_t f, int64_t K, int6
     L.h2 = take(static_cast<size_t>(r2 * f * 2));
     L.db_ovf = take(static_cast<size_t>(f * 4));
     L.k_rows = take(64);
-    L.du_ell = take(static_cast<size_t>(M * T * K * 4));
-    L.dz_ell = take(static_cast<size_t>(M * T * K * 4));
+    L.hdz_ell = take(static_cast<size_t>(M * T * K * 16));
     const int64_t nrb = (M + kCscRows - 1) / kCscRows;
     L.block_cnt = take(static_cast<size_t>(nrb * f * 4));
     L.unit_tot = take(static_cast<size_t>(f * 4));
+    L.scan_arrive = take(64);
     L.unit_ptr = take(static_cast<size_t>((f + 1) * 4));
     // every active pair: at most T*K per ELL row and d_ff per dense row
     const int64_t nnz_cap = (M - cap) * T * K + cap * f;
@@ -313,11 +313,10 @@ twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_
   }
   uint16_t* dy_ovf = at<uint16_t>(ws, L.dy_ovf);
   uint16_t* duz = at<uint16_t>(ws, L.duz);
-  float* du_ell = at<float>(ws, L.du_ell);
-  float* dz_ell = at<float>(ws, L.dz_ell);
+  float4* hdz_ell = at<float4>(ws, L.hdz_ell);
   if (launch_gather_rows(dY, h->ovf_rows, h->n_ovf, cap, d, dy_ovf, s) != cudaSuccess) return TWELL_ECUDA;
-  if (launch_ell_ffn_bwd(dY, W_u, W_g, wdt, h->count, h->val, h->col, h->row_plan, h->u_ell, lambda, du_ell,
-                         dz_ell, dX, M, d, f, K, at<int>(ws, L.ctr), h->status, s) != cudaSuccess)
+  if (launch_ell_ffn_bwd(dY, W_u, W_g, wdt, h->count, h->val, h->col, h->row_plan, h->u_ell, lambda, hdz_ell,
+                         dX, M, d, f, K, at<int>(ws, L.ctr), h->status, s) != cudaSuccess)
     return TWELL_ECUDA;
   float* du_ovf = at<float>(ws, L.du_ovf);
   float* dz_ovf = at<float>(ws, L.dz_ovf);
@@ -332,10 +331,11 @@ twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_
   if (launch_ovf_operands(h->n_ovf, h->ovf_rows, h->row_plan, cap, d, f, X, dy_ovf, du_ovf, dz_ovf, h->g_ovf,
                           h->u_ovf, dw, db_ovf, k_rows, s) != cudaSuccess)
     return TWELL_ECUDA;
-  CscBuffers b{h->row_plan + kPlanHdr + M, at<int>(ws, L.block_cnt), at<int>(ws, L.unit_tot),
-               at<int>(ws, L.unit_ptr), at<int>(ws, L.csc_row), at<float4>(ws, L.csc_val)};
-  if (launch_build_csc(h->count, h->val, h->col, h->row_ovf, h->ovf_rows, h->n_ovf, h->g_ovf, h->u_ell, h->u_ovf,
-                       du_ell, dz_ell, du_ovf, dz_ovf, h->row_plan, M, f, K, cap, b, s) != cudaSuccess)
+  CscBuffers b{h->row_plan + kPlanHdr + M,          at<int>(ws, L.block_cnt), at<int>(ws, L.unit_tot),
+               at<unsigned long long>(ws, L.scan_arrive), at<int>(ws, L.unit_ptr), at<int>(ws, L.csc_row),
+               at<float4>(ws, L.csc_val)};
+  if (launch_build_csc(h->count, h->val, h->col, h->row_ovf, h->ovf_rows, h->n_ovf, h->g_ovf, h->u_ovf,
+                       hdz_ell, du_ovf, dz_ovf, h->row_plan, M, f, K, cap, b, s) != cudaSuccess)
     return TWELL_ECUDA;
   if (launch_dense_wgrad(dw, k_rows, cap, d, f, dW_g, dW_u, dW_d, h->status, s) != cudaSuccess) return TWELL_ECUDA;
   return cuda_status(launch_weight_grads(X, dY, b, d, f, cap > 0 ? db_ovf : nullptr, cap > 0 ? k_rows : nullptr,

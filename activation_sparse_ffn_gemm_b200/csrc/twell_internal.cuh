@@ -90,8 +90,9 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
 
 int device_sm_count();
 
-// Process-wide tag for one split-K GEMM launch (1 .. 2^56 - 1, never 0).
-unsigned long long next_gemm_epoch();
+// Process-wide tag of one launch that counts block arrivals (1 .. 2^56 - 1,
+// never 0), so arrival words need no reset between launches.
+unsigned long long next_launch_epoch();
 
 // Encodes a 2-D bf16 tensor map (128-byte swizzle, zero fill out of bounds).
 // inner = contiguous extent (elements), outer = rows, row_bytes = row pitch.
@@ -157,11 +158,11 @@ cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uin
                            cudaStream_t s);
 
 // Sparse backward over the pieces of the row plan: dH at kept actives, dU,
-// dZ (stored per slot) and the rows of dX.
+// dZ, with (h = g u, dU, dZ, 0) stored per slot, and the rows of dX.
 cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const uint16_t* W_g,
                                const uint16_t* W_dt, const uint16_t* count, const uint16_t* val,
-                               const uint8_t* col, int* plan, const float* u_ell, float lambda, float* du_ell,
-                               float* dz_ell, float* dX, int M, int d, int f, int K, int* ctr, uint32_t* status,
+                               const uint8_t* col, int* plan, const float* u_ell, float lambda, float4* hdz_ell,
+                               float* dX, int M, int d, int f, int K, int* ctr, uint32_t* status,
                                cudaStream_t s);
 
 // Dense backup backward for overflow rows: dU, dZ (fp32, and bf16 [dU | dZ] as
@@ -197,6 +198,7 @@ struct CscBuffers {
   const int* row_slot;  // [M] dense backup slot of each row (-1: none), from the row plan
   int* block_cnt;  // [ceil(M/kCscRows)][f] per-chunk counts, then their exclusive scan
   int* unit_tot;   // [f]
+  unsigned long long* arrive;  // [1] arrival word of the scan (any initial contents)
   int* unit_ptr;   // [f+1]
   int* csc_row;    // [nnz_cap]
   float4* csc_val; // [nnz_cap]: (h, dU, dZ, 0)
@@ -207,7 +209,7 @@ constexpr int kCscRows = 256;  // rows per chunk of the pair-list build
 // ascending row order per unit, with h, dU and dZ attached.
 cudaError_t launch_build_csc(const uint16_t* count, const uint16_t* val, const uint8_t* col,
                              const uint8_t* row_ovf, const int* ovf_rows, const int* n_ovf, const uint16_t* g_ovf,
-                             const float* u_ell, const float* u_ovf, const float* du_ell, const float* dz_ell,
+                             const float* u_ovf, const float4* hdz_ell,
                              const float* du_ovf, const float* dz_ovf, const int* plan, int M, int f, int K,
                              int cap, const CscBuffers& b, cudaStream_t s);
 

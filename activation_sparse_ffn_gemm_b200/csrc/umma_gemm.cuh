@@ -434,7 +434,7 @@ cudaError_t launch_umma_gemm(const char* name, const CUtensorMap& a0, const CUte
   // with split-K the work items can outnumber the output tiles: one CTA per SM
   const int grid = shp.partial ? sms : static_cast<int>(tiles < sms ? tiles : sms);
   GemmShape shp2 = shp;
-  if (shp2.partial) shp2.epoch = next_gemm_epoch();
+  if (shp2.partial) shp2.epoch = next_launch_epoch();
   TWELL_LAUNCH(name, s, kern<<<grid, kGemmThreads, smem, s>>>(a0, b0, a1, b1, shp2, ea));
   return cudaGetLastError();
 }
