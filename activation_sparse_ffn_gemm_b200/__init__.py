@@ -24,6 +24,7 @@ LIB_PATH = os.path.join(_PKG, "libtwell.so")
 OP_PACK, OP_FWD, OP_BWD = 0, 1, 2
 STATUS_OVERFLOW_CAP = 1 << 3
 STATUS_TIMEOUT = 1 << 5
+STATUS_BAD_STATE = 1 << 1  # a tile-routed (inference) state given to the backward
 _STATUS_NAMES = {0: "TWELL_OK", 1: "TWELL_EINVAL", 2: "TWELL_EUNSUPPORTED", 3: "TWELL_EOVERFLOW_CAP",
                  4: "TWELL_ECUDA", 5: "TWELL_ETIMEOUT", 6: "TWELL_EWORKSPACE"}
 
@@ -80,6 +81,8 @@ def lib():
             L.twell_ffn_fwd.restype = ctypes.c_int
             L.twell_ffn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, ctypes.POINTER(TwellHybrid), _vp,
                                         _vp, ctypes.c_size_t, _vp]
+            L.twell_ffn_fwd_tiles.restype = ctypes.c_int
+            L.twell_ffn_fwd_tiles.argtypes = L.twell_ffn_fwd.argtypes
             L.twell_ffn_bwd.restype = ctypes.c_int
             L.twell_ffn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, ctypes.POINTER(TwellHybrid), _vp,
                                         ctypes.c_float, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
@@ -230,8 +233,12 @@ def pack_noalloc(X, W_g, b_g, T_n: int = 128, K: int = 8, ovf_cap: Optional[int]
 
 def ffn_fwd(X, W_g, b_g, W_u, W_d, T_n: int = 128, K: int = 8, ovf_cap: Optional[int] = None, W_dt=None,
             save_for_backward: bool = True, z_debug: bool = False, state: Optional[HybridState] = None,
-            ws: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None, stream=None):
-    """Sparse gated FFN forward. Returns (Y, state) or (Y, state, z) with z_debug."""
+            ws: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None, stream=None,
+            tile_routing: bool = False):
+    """Sparse gated FFN forward. Returns (Y, state) or (Y, state, z) with z_debug.
+
+    tile_routing: per-(row, tile) overflow routing (twell_ffn_fwd_tiles), an
+    inference-only state; otherwise the row-level hybrid (twell_ffn_fwd)."""
     for t, n in ((X, "X"), (W_g, "W_g"), (b_g, "b_g"), (W_u, "W_u"), (W_d, "W_d")):
         _bf16(t, n)
     M, d = X.shape
@@ -241,8 +248,10 @@ def ffn_fwd(X, W_g, b_g, W_u, W_d, T_n: int = 128, K: int = 8, ovf_cap: Optional
     z = torch.empty((M, f), dtype=torch.float32, device=X.device) if z_debug else None
     if ws is None:
         ws = workspace(OP_FWD, M, d, f, T_n, K, st.ovf_cap, X.device)
-    _check(lib().twell_ffn_fwd(_ptr(X), _ptr(W_g), _ptr(b_g), _ptr(W_u), _ptr(W_d), _ptr(W_dt), d, _ptr(Y),
-                               ctypes.byref(st.c), _ptr(z), _ptr(ws), ws.numel(), _stream(stream)), "twell_ffn_fwd")
+    fn = lib().twell_ffn_fwd_tiles if tile_routing else lib().twell_ffn_fwd
+    _check(fn(_ptr(X), _ptr(W_g), _ptr(b_g), _ptr(W_u), _ptr(W_d), _ptr(W_dt), d, _ptr(Y), ctypes.byref(st.c),
+              _ptr(z), _ptr(ws), ws.numel(), _stream(stream)),
+           "twell_ffn_fwd_tiles" if tile_routing else "twell_ffn_fwd")
     return (Y, st, z) if z_debug else (Y, st)
 
 

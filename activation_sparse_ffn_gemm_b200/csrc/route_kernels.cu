@@ -20,7 +20,8 @@ constexpr int kScanThreads = 1024;
 // row_ovf[i] = any_t(count[i][t] > K), and the row's kept entries
 // kept[i] = sum_t min(count[i][t], K), or -(1 + sum_t count[i][t]) for an
 // overflow row; one warp per row.
-__global__ void row_flags_kernel(const uint16_t* __restrict__ count, int M, int T, int K,
+// With tile-level routing no row overflows: row_ovf = 0, kept = every active unit.
+__global__ void row_flags_kernel(const uint16_t* __restrict__ count, int M, int T, int K, bool tiles,
                                  uint8_t* __restrict__ row_ovf, int* __restrict__ kept) {
   const int lane = threadIdx.x & 31;
   const long warp0 = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -40,6 +41,7 @@ __global__ void row_flags_kernel(const uint16_t* __restrict__ count, int M, int 
       n += __shfl_xor_sync(0xFFFFFFFFu, n, o);
       all += __shfl_xor_sync(0xFFFFFFFFu, all, o);
     }
+    if (tiles) any = false, n = all;
     if (lane == 0) {
       row_ovf[row] = any ? 1 : 0;
       kept[row] = any ? -(1 + all) : n;
@@ -111,7 +113,7 @@ __device__ __forceinline__ int2 block_scan2(int a, int b, int& ea, int& eb, int2
 }
 
 __global__ void __launch_bounds__(kScanThreads) route_plan_kernel(int* __restrict__ plan, int M, int f, int groups,
-                                                                  int cap, int* __restrict__ ovf_rows,
+                                                                  int cap, bool tiles, int* __restrict__ ovf_rows,
                                                                   int* __restrict__ n_ovf, uint32_t* status) {
   __shared__ long long red[3][kScanThreads / 32];
   __shared__ int2 warp_tot[kScanThreads / 32];
@@ -202,9 +204,10 @@ __global__ void __launch_bounds__(kScanThreads) route_plan_kernel(int* __restric
     plan[0] = carry_p;
     plan[1] = S;
     plan[2] = static_cast<int>(total < 0x7FFFFFFFLL ? total : 0x7FFFFFFFLL);
-    plan[3] = n_rows_ovf > 0 && total_ovf * 1000 > static_cast<long long>(f) * (kDenseWgradPerRow * n_rows_ovf +
-                                                                                kDenseWgradFixed)
-                  ? 1 : 0;
+    plan[3] = tiles ? -1
+                    : (n_rows_ovf > 0 && total_ovf * 1000 > static_cast<long long>(f) * (kDenseWgradPerRow * n_rows_ovf +
+                                                                                         kDenseWgradFixed)
+                           ? 1 : 0);
   }
 }
 
@@ -293,17 +296,17 @@ __global__ void transpose_bf16_kernel(const uint16_t* __restrict__ in, int rows,
 cudaError_t launch_route(const uint16_t* count, const uint16_t* val, const uint8_t* col, const uint16_t* spill,
                          int M, int f, int K, int cap, uint8_t* row_ovf, int* ovf_rows, int* n_ovf,
                          uint16_t* g_ovf, const uint16_t* X, int d, uint16_t* x_ovf, int* plan, int groups,
-                         uint32_t* status, cudaStream_t s) {
+                         bool tiles, uint32_t* status, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   const int T = f / kTn;
   const int warps_needed = M;
   int blocks = (warps_needed + 7) / 8;
   const int max_blocks = device_sm_count() * 16;
   if (blocks > max_blocks) blocks = max_blocks;
-  TWELL_LAUNCH("row_flags", s, row_flags_kernel<<<blocks, 256, 0, s>>>(count, M, T, K, row_ovf, plan + kPlanHdr));
+  TWELL_LAUNCH("row_flags", s, row_flags_kernel<<<blocks, 256, 0, s>>>(count, M, T, K, tiles, row_ovf, plan + kPlanHdr));
   TWELL_LAUNCH("route_plan", s,
-               route_plan_kernel<<<1, kScanThreads, 0, s>>>(plan, M, f, groups, cap, ovf_rows, n_ovf, status));
-  if (cap > 0) {
+               route_plan_kernel<<<1, kScanThreads, 0, s>>>(plan, M, f, groups, cap, tiles, ovf_rows, n_ovf, status));
+  if (cap > 0 && !tiles) {
     int g = cap < device_sm_count() * 4 ? cap : device_sm_count() * 4;
     TWELL_LAUNCH("ovf_gather", s,
                  ovf_gather_kernel<<<g, 256, 0, s>>>(n_ovf, ovf_rows, count, val, col, spill, f, K, g_ovf, X, d, x_ovf));

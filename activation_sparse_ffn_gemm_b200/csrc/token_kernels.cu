@@ -31,7 +31,10 @@
 //     global accumulator row (a scratch row for Y, dX itself for dX) one after
 //     another in piece order, through a per-row turnstile, so the result is
 //     the same on every run.
-// Overflow rows have no pieces (the dense backup path owns them).
+// Overflow rows have no pieces (the dense backup path owns them). With
+// tile-level routing (TILES) no row overflows: a tile with more than K actives
+// is read whole from the dense slice the gate epilogue spilled for it, so
+// every active unit of every row goes through these kernels.
 #include "sm100.cuh"
 #include "trace.cuh"
 #include "twell_internal.cuh"
@@ -57,7 +60,8 @@ struct GroupSmem {
   int j[kListCap];     // unit of each entry
   float c[kListCap];   // coefficient (g, then h; or dU)
   float c2[kListCap];  // second coefficient (u, then dZ) in the backward
-  int slot[kListCap];  // t * K + s
+  int slot[kListCap];  // t * K + s (-1 for an entry read from a spilled slice)
+  uint16_t tcnt[kMaxTiles];  // per-tile true counts (tile-level routing)
   int row, q, P;       // the piece being processed (re-read instead of kept live)
 };
 
@@ -76,7 +80,10 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Kept-entry offsets of `row` over its T tiles, computed by warp 0 of the group.
+// Entry offsets of `row` over its T tiles, computed by warp 0 of the group:
+// min(count, K) entries per tile (the ELL slots), or every active unit of the
+// tile with tile-level routing (TILES; the true counts are kept in g.tcnt).
+template <bool TILES>
 __device__ __forceinline__ void row_offsets(const uint16_t* __restrict__ count, long row, int T, int K, int lane,
                                             GroupSmem& g) {
   int run = 0;
@@ -85,7 +92,8 @@ __device__ __forceinline__ void row_offsets(const uint16_t* __restrict__ count, 
     int c = 0;
     if (t < T) {
       c = count[row * T + t];
-      c = c < K ? c : K;
+      if (TILES) g.tcnt[t] = static_cast<uint16_t>(c);
+      else c = c < K ? c : K;
     }
     int incl = c;
 #pragma unroll
@@ -178,6 +186,62 @@ __device__ __forceinline__ void build_list(GroupSmem& g, long row, int T, int K,
     g.c[e] = __uint_as_float(static_cast<uint32_t>(val[base]) << 16);
     if (u_ell) g.c2[e] = u_ell[base];
     g.slot[e] = t * K + sl;
+  }
+}
+
+// List entries [e0, e0 + ne) of `row` under tile-level routing: entries of
+// tiles with at most K actives come from the ELL slots; a tile with more is
+// read from its spilled dense slice (bf16 ReLU(z), 128 values) by one warp,
+// its nonzeros ranked by a warp prefix sum in column order. A unit with
+// 0 < z below the smallest bf16 is counted but has a zero slice value; its
+// leftover entries are filled with g = 0 (no contribution).
+__device__ __forceinline__ void build_list_tiles(GroupSmem& g, long row, int T, int K, int f, int e0, int ne, int gtid,
+                                                 int GT, int wi, int W, int lane,
+                                                 const uint16_t* __restrict__ val, const uint8_t* __restrict__ col,
+                                                 const uint16_t* __restrict__ spill) {
+  for (int e = gtid; e < ne; e += GT) {
+    int t, sl;
+    entry_of(g.off, T, e0 + e, t, sl);
+    if (g.tcnt[t] > K) continue;
+    const long base = (row * T + t) * K + sl;
+    g.j[e] = t * kTn + col[base];
+    g.c[e] = __uint_as_float(static_cast<uint32_t>(val[base]) << 16);
+    g.slot[e] = t * K + sl;
+  }
+  for (int t = wi; t < T; t += W) {
+    const int cnt = g.tcnt[t];
+    const int o = g.off[t];
+    if (cnt <= K || o >= e0 + ne || o + cnt <= e0) continue;
+    const uint2 v = *reinterpret_cast<const uint2*>(spill + row * f + t * kTn + lane * 4);
+    const uint32_t w4[2] = {v.x, v.y};
+    int nz = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) nz += ((w4[k >> 1] >> (16 * (k & 1))) & 0xFFFFu) != 0;
+    int incl = nz;
+#pragma unroll
+    for (int s = 1; s < 32; s <<= 1) {
+      const int x = __shfl_up_sync(0xFFFFFFFFu, incl, s);
+      if (lane >= s) incl += x;
+    }
+    int idx = o + incl - nz;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t bits = (w4[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+      if (!bits) continue;
+      if (idx >= e0 && idx < e0 + ne && idx < o + cnt) {
+        g.j[idx - e0] = t * kTn + lane * 4 + k;
+        g.c[idx - e0] = __uint_as_float(bits << 16);
+        g.slot[idx - e0] = -1;
+      }
+      ++idx;
+    }
+    const int found = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    for (int x = o + found + lane; x < o + cnt; x += 32)
+      if (x >= e0 && x < e0 + ne) {
+        g.j[x - e0] = t * kTn;
+        g.c[x - e0] = 0.f;
+        g.slot[x - e0] = -1;
+      }
   }
 }
 
@@ -291,7 +355,7 @@ __device__ __forceinline__ void turn_pass(int* turn, int row, int q, int P, int 
 
 // Reads piece p of the plan into the group's shared memory (row, q, P) with
 // the row's kept-entry offsets; returns false when the plan is exhausted.
-template <int W>
+template <int W, bool TILES>
 __device__ __forceinline__ bool next_piece(int* ctr, const int* plan, int M, const uint16_t* __restrict__ count, int T,
                                            int K, int grp, int wi, int lane, int* s_next, GroupSmem& g) {
   const int np = plan[0], S = plan[1];
@@ -299,7 +363,7 @@ __device__ __forceinline__ bool next_piece(int* ctr, const int* plan, int M, con
   if (p >= np) return false;
   const int* pieces = plan + kPlanHdr + 2L * M;
   const int row = pieces[2 * p], q = pieces[2 * p + 1];
-  if (wi == 0) row_offsets(count, row, T, K, lane, g);
+  if (wi == 0) row_offsets<TILES>(count, row, T, K, lane, g);
   if (wi == 0 && lane == 0) {
     const int n = g.tot;
     g.row = row;
@@ -311,12 +375,15 @@ __device__ __forceinline__ bool next_piece(int* ctr, const int* plan, int M, con
 }
 
 // yacc: [M][d] fp32 accumulator rows for rows split into several pieces.
-template <int C, int W, bool EXACT>
+// TILES: tile-level routing; spill holds the dense slices of tiles with more
+// than K actives (u is not saved: an inference-only state).
+template <int C, int W, bool EXACT, bool TILES>
 __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>::WARPS * 32)) ell_fwd_kernel(
     const uint16_t* __restrict__ X, const uint16_t* __restrict__ Wu, const uint16_t* __restrict__ Wdt,
     const uint16_t* __restrict__ count, const uint16_t* __restrict__ val, const uint8_t* __restrict__ col,
-    int* __restrict__ plan, float* __restrict__ u_ell, uint16_t* __restrict__ Y, int M, int d, int T, int K,
-    int* __restrict__ ctr, float* __restrict__ yacc, uint32_t* status) {
+    const uint16_t* __restrict__ spill, int* __restrict__ plan, float* __restrict__ u_ell,
+    uint16_t* __restrict__ Y, int M, int d, int T, int K, int* __restrict__ ctr, float* __restrict__ yacc,
+    uint32_t* status) {
   using Cfg = TokCfg<C, W>;
   constexpr int B = Cfg::B;
   __shared__ GroupSmem gs[Cfg::G];
@@ -360,12 +427,15 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
     }
   };
 
-  while (next_piece<W>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g)) {
+  while (next_piece<W, TILES>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g)) {
     const long row = g.row;
     const int S = plan[1];
     const int e0 = g.q * S;
     const int ne = max(0, min(S, g.tot - e0));
-    build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, nullptr);
+    if (TILES)
+      build_list_tiles(g, row, T, K, T * kTn, e0, ne, gtid, Cfg::GT, wi, W, lane, val, col, spill);
+    else
+      build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, nullptr);
     group_sync<W>(grp);
     up(row, ne);
     float2 y[C][4];
@@ -434,7 +504,11 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
     group_sync<W>(grp);
   };
 
-  while (next_piece<W>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g)) {
+  if (plan[3] < 0) {  // a tile-routed (inference) state cannot serve the backward
+    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, TWELL_STATUS_BAD_STATE);
+    return;
+  }
+  while (next_piece<W, false>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g)) {
     const long row = g.row;
     const int S = plan[1];
     const int e0 = g.q * S;
@@ -481,10 +555,14 @@ int tok_grid(int M, int G) {
 }
 
 template <int C, int W, bool EXACT, typename... A>
-void launch_fwd_cw(int M, cudaStream_t s, A... a) {
+void launch_fwd_cw(int M, bool tiles, cudaStream_t s, A... a) {
   constexpr int threads = TokCfg<C, W>::WARPS * 32;
-  TWELL_LAUNCH("ell_updown", s,
-               ell_fwd_kernel<C, W, EXACT><<<tok_grid(M, TokCfg<C, W>::G), threads, 0, s>>>(a...));
+  if (tiles)
+    TWELL_LAUNCH("ell_updown_tiles", s,
+                 (ell_fwd_kernel<C, W, EXACT, true><<<tok_grid(M, TokCfg<C, W>::G), threads, 0, s>>>(a...)));
+  else
+    TWELL_LAUNCH("ell_updown", s,
+                 (ell_fwd_kernel<C, W, EXACT, false><<<tok_grid(M, TokCfg<C, W>::G), threads, 0, s>>>(a...)));
 }
 
 template <int C, int W, bool EXACT, typename... A>
@@ -504,9 +582,10 @@ int tok_groups(int M, int d) {
 }
 
 cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
-                               const uint16_t* count, const uint16_t* val, const uint8_t* col, int* plan,
-                               float* u_ell, uint16_t* Y, int M, int d, int f, int K, int* ctr, float* yacc,
-                               uint32_t* status, cudaStream_t s) {
+                               const uint16_t* count, const uint16_t* val, const uint8_t* col,
+                               const uint16_t* spill, int* plan, float* u_ell, uint16_t* Y, int M, int d, int f,
+                               int K, int* ctr, float* yacc, uint32_t* status, cudaStream_t s) {
+  const bool tiles = spill != nullptr;
   if (M <= 0) return cudaSuccess;
   cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
@@ -515,10 +594,10 @@ cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uin
   const int T = f / kTn;
   const bool exact = d / 8 == W * 32 * C;
 #define TWELL_FWD(CC, WW)                                                                                   \
-  (exact ? launch_fwd_cw<CC, WW, true>(M, s, X, W_u, W_dt, count, val, col, plan, u_ell, Y, M, d, T, K, ctr, yacc, \
-                                       status)                                                                     \
-         : launch_fwd_cw<CC, WW, false>(M, s, X, W_u, W_dt, count, val, col, plan, u_ell, Y, M, d, T, K, ctr, yacc, \
-                                        status))
+  (exact ? launch_fwd_cw<CC, WW, true>(M, tiles, s, X, W_u, W_dt, count, val, col, spill, plan, u_ell, Y, M, d, T, \
+                                       K, ctr, yacc, status)                                                      \
+         : launch_fwd_cw<CC, WW, false>(M, tiles, s, X, W_u, W_dt, count, val, col, spill, plan, u_ell, Y, M, d,   \
+                                        T, K, ctr, yacc, status))
   if (W == 1 && C == 1) TWELL_FWD(1, 1);
   else if (W == 1 && C == 2) TWELL_FWD(2, 1);
   else if (W == 1 && C == 4) TWELL_FWD(4, 1);

@@ -167,14 +167,14 @@ T* at(void* ws, size_t off) {
 
 twell_status run_pack(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_g, int64_t d, twell_hybrid* h,
                       float* z_debug, void* ws, const WsLayout& L, const uint16_t* X_for_gather,
-                      uint16_t* x_ovf, cudaStream_t s) {
+                      uint16_t* x_ovf, bool tiles, cudaStream_t s) {
   const int M = h->M, f = h->d_ff, K = h->K, cap = h->ovf_cap;
   PackOut po{h->count, h->val, h->col, at<uint16_t>(ws, L.spill), z_debug};
   cudaError_t e = launch_gate_pack(X, W_g, b_g, M, static_cast<int>(d), f, K, po, h->status, s);
   if (e != cudaSuccess) return TWELL_ECUDA;
   e = launch_route(h->count, h->val, h->col, po.spill, M, f, K, cap, h->row_ovf, h->ovf_rows, h->n_ovf, h->g_ovf,
                    X_for_gather, static_cast<int>(d), x_ovf, h->row_plan, tok_groups(M, static_cast<int>(d)),
-                   h->status, s);
+                   tiles, h->status, s);
   return cuda_status(e);
 }
 
@@ -240,13 +240,20 @@ twell_status twell_pack(const uint16_t* X, const uint16_t* W_g, const uint16_t* 
   if (st != TWELL_OK) return st;
   if (h->M == 0) return TWELL_OK;
   const WsLayout L = ws_layout(TWELL_OP_PACK, h->M, d_model, h->d_ff, h->K, h->ovf_cap);
-  return run_pack(X, W_g, b_g, d_model, h, z_debug, ws, L, nullptr, nullptr,
+  return run_pack(X, W_g, b_g, d_model, h, z_debug, ws, L, nullptr, nullptr, false,
                   reinterpret_cast<cudaStream_t>(stream));
 }
 
-twell_status twell_ffn_fwd(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_g, const uint16_t* W_u,
-                           const uint16_t* W_d, const uint16_t* W_dt, int64_t d_model, uint16_t* Y,
-                           twell_hybrid* h, float* z_debug, void* ws, size_t ws_bytes, twell_stream_t stream) {
+}  // extern "C"
+
+namespace twell {
+namespace {
+
+// The forward shared by twell_ffn_fwd (row-level routing with the dense
+// backup) and twell_ffn_fwd_tiles (tile-level routing, inference only).
+twell_status ffn_fwd_impl(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_g, const uint16_t* W_u,
+                          const uint16_t* W_d, const uint16_t* W_dt, int64_t d_model, uint16_t* Y, twell_hybrid* h,
+                          float* z_debug, void* ws, size_t ws_bytes, bool tiles, twell_stream_t stream) {
   twell_status st = check_hybrid(h, d_model);
   if (st != TWELL_OK || h->M == 0) return st;
   const void* in[] = {X, W_g, b_g, W_u, W_d, Y};
@@ -266,14 +273,33 @@ twell_status twell_ffn_fwd(const uint16_t* X, const uint16_t* W_g, const uint16_
     wdt = t;
   }
   uint16_t* x_ovf = at<uint16_t>(ws, L.x_ovf);
-  st = run_pack(X, W_g, b_g, d, h, z_debug, ws, L, X, x_ovf, s);
+  st = run_pack(X, W_g, b_g, d, h, z_debug, ws, L, X, x_ovf, tiles, s);
   if (st != TWELL_OK) return st;
-  if (launch_ell_ffn_fwd(X, W_u, wdt, h->count, h->val, h->col, h->row_plan, h->u_ell, Y, M, d, f, K,
-                         at<int>(ws, L.ctr), at<float>(ws, L.yacc), h->status, s) != cudaSuccess)
+  if (launch_ell_ffn_fwd(X, W_u, wdt, h->count, h->val, h->col, tiles ? at<uint16_t>(ws, L.spill) : nullptr,
+                         h->row_plan, tiles ? nullptr : h->u_ell, Y, M, d, f, K, at<int>(ws, L.ctr),
+                         at<float>(ws, L.yacc), h->status, s) != cudaSuccess)
     return TWELL_ECUDA;
+  if (tiles) return TWELL_OK;
   const SplitKBuffers sk{at<float>(ws, L.sk_partial), at<unsigned long long>(ws, L.sk_arrivals)};
   return cuda_status(launch_ovf_fwd(x_ovf, W_u, W_d, h->g_ovf, h->ovf_rows, h->n_ovf, cap, d, f,
                                     at<uint16_t>(ws, L.h_ovf), h->u_ovf, Y, sk, h->status, s));
+}
+
+}  // namespace
+}  // namespace twell
+
+extern "C" {
+
+twell_status twell_ffn_fwd(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_g, const uint16_t* W_u,
+                           const uint16_t* W_d, const uint16_t* W_dt, int64_t d_model, uint16_t* Y,
+                           twell_hybrid* h, float* z_debug, void* ws, size_t ws_bytes, twell_stream_t stream) {
+  return ffn_fwd_impl(X, W_g, b_g, W_u, W_d, W_dt, d_model, Y, h, z_debug, ws, ws_bytes, false, stream);
+}
+
+twell_status twell_ffn_fwd_tiles(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_g, const uint16_t* W_u,
+                                 const uint16_t* W_d, const uint16_t* W_dt, int64_t d_model, uint16_t* Y,
+                                 twell_hybrid* h, float* z_debug, void* ws, size_t ws_bytes, twell_stream_t stream) {
+  return ffn_fwd_impl(X, W_g, b_g, W_u, W_d, W_dt, d_model, Y, h, z_debug, ws, ws_bytes, true, stream);
 }
 
 twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_t* W_u, const uint16_t* W_d,

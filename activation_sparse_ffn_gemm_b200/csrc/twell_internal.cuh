@@ -21,7 +21,8 @@ constexpr int kTokListCap = 256;   // kept entries per list chunk of the token k
 // Row plan (twell_hybrid::row_plan, int32): the work of the token kernels as
 // pieces of at most S kept entries of one non-overflow row.
 //   [0] number of pieces, [1] S, [2] kept entries of non-overflow rows,
-//   [3] 1 when the weight gradients of the overflow rows run as dense GEMMs
+//   [3] 1 when the weight gradients of the overflow rows run as dense GEMMs,
+//       -1 for a tile-routed (inference-only) plan
 //   [kPlanHdr, kPlanHdr + M)       per-row turnstile words (0 between launches;
 //                                  the routing step parks the kept counts there)
 //   [kPlanHdr + M, kPlanHdr + 2M)  row_slot: dense backup slot of each row, -1 if none
@@ -118,10 +119,12 @@ cudaError_t launch_gate_pack(const uint16_t* X, const uint16_t* W_g, const uint1
 // Row routing: flags, ascending overflow list, dense backup rows (and the
 // gathered X rows of overflow rows when x_ovf != nullptr), and the row plan of
 // the token kernels for `groups` resident token groups.
+// tiles: tile-level routing (no overflow rows; the plan counts every active
+// unit and is marked inference-only).
 cudaError_t launch_route(const uint16_t* count, const uint16_t* val, const uint8_t* col, const uint16_t* spill,
                          int M, int f, int K, int cap, uint8_t* row_ovf, int* ovf_rows, int* n_ovf,
                          uint16_t* g_ovf, const uint16_t* X, int d, uint16_t* x_ovf, int* plan, int groups,
-                         uint32_t* status, cudaStream_t s);
+                         bool tiles, uint32_t* status, cudaStream_t s);
 
 // Resident token groups of the token kernels for M rows of width d (the
 // launch shape they use); sizes the pieces of the row plan.
@@ -136,10 +139,12 @@ cudaError_t launch_transpose_bf16(const uint16_t* in, int rows, int cols, uint16
 // Fused sparse up + down over the pieces of the row plan (ELL rows only).
 // ctr: one int of device scratch (the piece counter), zeroed by the launcher;
 // yacc: [M][d] fp32 accumulator rows for rows split into several pieces.
+// spill: nullptr for row-level routing; for tile-level routing the dense
+// slices of tiles with more than K actives (and u_ell must be nullptr).
 cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
-                               const uint16_t* count, const uint16_t* val, const uint8_t* col, int* plan,
-                               float* u_ell, uint16_t* Y, int M, int d, int f, int K, int* ctr, float* yacc,
-                               uint32_t* status, cudaStream_t s);
+                               const uint16_t* count, const uint16_t* val, const uint8_t* col,
+                               const uint16_t* spill, int* plan, float* u_ell, uint16_t* Y, int M, int d, int f,
+                               int K, int* ctr, float* yacc, uint32_t* status, cudaStream_t s);
 
 // Split-K scratch of the dense-backup GEMMs (one GEMM at a time): fp32
 // partials and per-output-tile arrival words (any initial contents).

@@ -69,7 +69,7 @@ extern "C" TWELL_API twell_status twell_pack_noalloc(const uint16_t* X, const ui
   PackOut po{h->count, h->val, h->col, scratch, z_debug};
   if (launch_gate_pack(X, W_g, b_g, M, d, f, K, po, h->status, s) != cudaSuccess) return TWELL_ECUDA;
   if (launch_route(h->count, h->val, h->col, scratch, M, f, K, h->ovf_cap, h->row_ovf, h->ovf_rows, h->n_ovf,
-                   h->g_ovf, nullptr, d, nullptr, h->row_plan, tok_groups(M, d), h->status, s) != cudaSuccess)
+                   h->g_ovf, nullptr, d, nullptr, h->row_plan, tok_groups(M, d), false, h->status, s) != cudaSuccess)
     return TWELL_ECUDA;
   return TWELL_OK;
 }

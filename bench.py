@@ -585,7 +585,18 @@ def run_sweep(args, local):
             cnt = st.count.float()
             activity = float(cnt.sum().item()) / (M * f)
             ratio = float(cnt.max().item()) / max(float(cnt.mean().item()), 1e-30)
-            del st, wsf, wsb, grads, Wdt, Y
+            dense_wgrad = int(st.row_plan[3].item())
+
+            # the same forward with per-(row, tile) overflow routing (inference only)
+            st_t = tw.HybridState(M, f, T_n, K, M, dev, with_u=False)
+
+            def fwd_tiles():
+                tw.transpose_wd(W_d, out=Wdt)
+                tw.ffn_fwd(X, W_g, b_g, W_u, W_d, T_n=T_n, K=K, W_dt=Wdt, state=st_t, ws=wsf, Y=Y, tile_routing=True)
+
+            t_fwd_tiles = timed(fwd_tiles)
+            assert st_t.read_status() == 0, "device status word set"
+            del st, st_t, wsf, wsb, grads, Wdt, Y
 
             Wg_r, Wu_r, Wd_r = (t.clone().requires_grad_() for t in (W_g, W_u, W_d))
             Xr = X.clone().requires_grad_()
@@ -608,7 +619,8 @@ def run_sweep(args, local):
             print(json.dumps({
                 "point": {"M": M, "sparsity": sp, "d_model": d, "d_ff": f, "T_n": T_n, "K": K},
                 "twell": {"fwd_ms": t_fwd, "fwd_bwd_ms": t_fb, "fwd_tokens_per_s": M / (t_fwd / 1e3),
-                          "fwd_bwd_tokens_per_s": M / (t_fb / 1e3)},
+                          "fwd_bwd_tokens_per_s": M / (t_fb / 1e3), "dense_wgrad_for_overflow_rows": dense_wgrad},
+                "twell_tile_routing": {"fwd_ms": t_fwd_tiles, "fwd_tokens_per_s": M / (t_fwd_tiles / 1e3)},
                 "dense_bf16": {"fwd_ms": t_dfwd, "fwd_bwd_ms": t_dfb},
                 "speedup_vs_dense": {"fwd": t_dfwd / t_fwd, "fwd_bwd": t_dfb / t_fb},
                 "measured": {"activity": activity, "overflow_rows": n_ovf, "max_over_mean_count": ratio},

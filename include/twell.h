@@ -67,6 +67,9 @@ typedef enum twell_status {
 /* Device status word bits, set by kernels and read by twell_status_read. */
 #define TWELL_STATUS_OVERFLOW_CAP (1u << TWELL_EOVERFLOW_CAP)
 #define TWELL_STATUS_TIMEOUT (1u << TWELL_ETIMEOUT)
+/* The state given to a call cannot serve it (a tile-routed inference state
+ * passed to twell_ffn_bwd); the call wrote no result. */
+#define TWELL_STATUS_BAD_STATE (1u << TWELL_EINVAL)
 
 /*
  * The hybrid TwELL representation of g = ReLU(z) ([aivizor] ¶2: horizontal
@@ -202,6 +205,24 @@ TWELL_API twell_status twell_ffn_fwd(const uint16_t* X, const uint16_t* W_g, con
                            const uint16_t* W_u, const uint16_t* W_d, const uint16_t* W_dt,
                            int64_t d_model, uint16_t* Y, twell_hybrid* h, float* z_debug, void* ws,
                            size_t ws_bytes, twell_stream_t stream);
+
+/*
+ * Inference forward with per-(row, tile) overflow routing, the alternative to
+ * the row-level hybrid of twell_ffn_fwd ([aivizor] ¶2 routes overflowing rows
+ * to a dense backup; ¶4 notes that rows can hold far more nonzeros than the
+ * mean): no row goes dense; a tile with more than K actives keeps its count
+ * and its first K slots and is otherwise read whole from the dense slice the
+ * gate epilogue spilled for it, so the sparse kernel runs every active unit
+ * (an adaptive number of entries per tile). Same arguments and workspace as
+ * twell_ffn_fwd; Y is the same function of the inputs.
+ *   h   filled as by twell_pack except: row_ovf = 0 for every row, n_ovf = {0, 0},
+ *       g_ovf, u_ell and u_ovf untouched. The state serves inference only:
+ *       twell_ffn_bwd given it sets TWELL_STATUS_BAD_STATE and writes nothing.
+ */
+TWELL_API twell_status twell_ffn_fwd_tiles(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_g,
+                                 const uint16_t* W_u, const uint16_t* W_d, const uint16_t* W_dt,
+                                 int64_t d_model, uint16_t* Y, twell_hybrid* h, float* z_debug, void* ws,
+                                 size_t ws_bytes, twell_stream_t stream);
 
 /*
  * Backward pass over the hybrid format of a previous twell_ffn_fwd (which must

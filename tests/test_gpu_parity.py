@@ -259,3 +259,37 @@ def test_train_full_size(tw, orc):
         g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=lam)
         torch.cuda.synchronize()
         _check_bwd(orc, inp, g, G, lam, "train")
+
+
+@pytest.mark.parametrize("name", ["k32", "multi_tile", "ragged_k16", "tiny"])
+def test_tile_routing_forward(tw, orc, name):
+    """Per-(row, tile) overflow routing: every active unit runs sparsely (tiles
+    over K read from their spilled slice); Y matches the oracle with the GPU's
+    stored g = bf16(ReLU(z)) for every unit, no row is dense, and the state is
+    refused by the backward."""
+    M, d, f, K, act, rs, seed = CASES[name]
+    w = Workload(name, M, d, f, 128, K, act, row_scale=rs, training=True, seed=seed)
+    inp = make_inputs(w)
+    D = _dev(inp)
+    Y, st, z = tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], T_n=128, K=K, z_debug=True,
+                          tile_routing=True)
+    torch.cuda.synchronize()
+    zg = z.cpu().numpy()
+    p_gpu = state_to_numpy(st)
+    p_ref = orc.pack(zg.astype(np.float64), 128, K)
+    for k in ("count", "val", "col"):
+        assert np.array_equal(p_gpu[k], p_ref[k]), k
+    assert not p_gpu["row_ovf"].any() and st.n_overflow() == (0, 0)
+    assert st.read_status() == 0
+    plan = st.row_plan.cpu().numpy()
+    assert plan[3] == -1
+    counts = p_gpu["count"].astype(np.int64)
+    assert plan[2] == counts.sum()  # every active unit is listed
+    G = orc.bf16_round(np.maximum(zg.astype(np.float64), 0.0))
+    args = (inp["X"], inp["W_g"], inp["b_g"], inp["W_u"], inp["W_d"])
+    y_stored = orc.ffn_fwd(*args, gmat=G)
+    y_plain = orc.ffn_fwd(*args)
+    assert_matches_oracle(f32_of_bits(bits_of(Y)), y_stored, y_plain, f"{name} tile-routed Y", bf16_out=True)
+    # the inference-only state is refused by the backward, which writes nothing
+    tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=0.0)
+    assert st.read_status(clear=True) == tw.STATUS_BAD_STATE
