@@ -50,7 +50,7 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["twell", "reference"], default="twell")
     p.add_argument("--lam", type=float, default=1e-3)
-    p.add_argument("--cpu-seconds", type=float, default=8.0, help="target CPU work of the oracle baseline sample")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--no-trace", action="store_true")
@@ -198,6 +198,31 @@ KERNEL_SOURCES = {
 }
 
 
+def path_roofline(M, d, f, T, K, kept, n_ovf, peaks, ms_fwd, ms_step):
+    """Whole-step roofline: the time the step's algorithmic work takes at the
+    measured peaks (dense flops at the sustained bf16 rate, algorithmic bytes
+    at the HBM copy rate), against the measured times.
+
+    forward:  gate GEMM 2 M d f flops; dense backup 4 M_ovf d f flops; bytes:
+              X, TwELL (2 + 3K bytes per row tile), Y, u saved, W_u and W_dt
+              once, the W_d transpose (read + write)
+    backward: 12 d flops per kept pair (dH, dX, three weight gradients) and
+              12 M_ovf d f for dense rows; bytes: X, dY, TwELL, u, dX (fp32),
+              W_u, W_g, W_dt once, the three fp32 weight gradients written
+    """
+    P = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * 1e12
+    B = peaks["hbm_gbs"] * 1e9
+    tw_bytes = M * T * (2 + 3 * K)
+    f_flops = 2.0 * M * d * f + 4.0 * n_ovf * d * f
+    f_bytes = 2 * M * d + tw_bytes + 2 * M * d + 4 * kept + 2 * 2 * f * d + 2 * 2 * f * d
+    b_flops = 12.0 * d * kept + 12.0 * n_ovf * d * f
+    b_bytes = 2 * M * d + 2 * M * d + tw_bytes + 4 * kept + 4 * M * d + 3 * 2 * f * d + 3 * 4 * f * d
+    t_f = f_flops / P + f_bytes / B
+    t_s = t_f + b_flops / P + b_bytes / B
+    return {"fwd_ms": t_f * 1e3, "step_ms": t_s * 1e3, "fwd_frac": t_f * 1e3 / ms_fwd, "step_frac": t_s * 1e3 / ms_step,
+            "note": "algorithmic time at measured peaks (sustained bf16, HBM copy) / measured time"}
+
+
 def source_hash(kernel):
     files = KERNEL_SOURCES.get(kernel)
     if not files:
@@ -244,8 +269,10 @@ def cpu_baseline(inp, lam, target_s):
 
     n = 32
     t = run(n)
-    if t < target_s / 4:
-        n = int(min(M, max(n, n * target_s / max(t, 1e-3))))
+    for _ in range(3):  # grow the sample towards target_s (the oracle's cost is not quite linear in rows)
+        if t >= target_s / 2 or n >= M:
+            break
+        n = int(min(M, max(2 * n, n * target_s / max(t, 1e-3))))
         t = run(n)
     return {"value": n / t, "unit": "tokens/s", "cores": O.get_threads(), "kind": "oracle",
             "sample": f"first {n} of {M} token rows, forward + backward (weight gradients over the sample), "
@@ -505,6 +532,7 @@ def run_twell(args, world, rank, local):
                 "d2h_bytes_per_step": M * d * 2},
         "gpu_launches": launches,
         "roofline": roofline,
+        "path_roofline": path_roofline(M, d, f, T, K, kept, nst, peaks, ms_fwd, ms_step),
         "kernels": {k: {"launches_per_step": v["launches"] / args.steps, "ms_per_step": v["ms_per_step"]}
                     for k, v in sorted(breakdown.items(), key=lambda kv: -kv[1]["ms"])},
         "sparsity": {"activity": activity, "overflow_rows": nfl, "max_count": float(cnt.max().item()),

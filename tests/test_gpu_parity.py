@@ -293,3 +293,36 @@ def test_tile_routing_forward(tw, orc, name):
     # the inference-only state is refused by the backward, which writes nothing
     tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=0.0)
     assert st.read_status(clear=True) == tw.STATUS_BAD_STATE
+
+
+def test_turnstile_wait_gives_up(tw, orc):
+    """Failure detection without a GPU fault: a piece whose predecessor never
+    runs waits on its row's turnstile word, which nothing sets; the bounded
+    wait (2 s of %globaltimer) gives up, the kernel records
+    TWELL_STATUS_TIMEOUT and returns, and the context stays usable."""
+    w = Workload("turn", 64, 256, 1024, 128, 16, 0.05, training=True, seed=21)
+    inp = make_inputs(w)
+    D = _dev(inp)
+    Y, st = tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], K=16)
+    torch.cuda.synchronize()
+    assert st.read_status() == 0
+    kept0 = int(np.minimum(st.count[0].cpu().numpy().view(np.uint16), 16).sum())
+    assert kept0 >= 2
+    # plan: one piece, (row 0, q = 1) of a row cut into pieces of one entry;
+    # piece q = 0 is never handed out, so turn word 0 never reaches 1
+    M = st.M
+    plan = st.row_plan
+    plan[0] = 1
+    plan[1] = 1
+    plan[3] = 0
+    plan[4:4 + M] = 0
+    plan[4 + 2 * M:4 + 2 * M + 2] = torch.tensor([0, 1], dtype=torch.int32, device=plan.device)
+    torch.cuda.synchronize()
+    tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=0.0)
+    assert st.read_status(clear=True) & tw.STATUS_TIMEOUT
+    # the context is still usable: a fresh forward and backward run clean
+    Y2, st2 = tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], K=16)
+    g2 = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st2, D["dY"], lam=0.0)
+    torch.cuda.synchronize()
+    assert st2.read_status() == 0
+    assert torch.equal(Y2, Y)
