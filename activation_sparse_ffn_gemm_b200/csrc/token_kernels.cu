@@ -118,19 +118,33 @@ __device__ __forceinline__ void entry_of(const int* off, int T, int e, int& t, i
   sl = e - off[lo];
 }
 
+// acc_lo += lo(a) * lo(w), acc_hi += hi(a) * hi(w) for two bf16x2 words: the
+// mixed-precision FMA takes the bf16 halves as they are (exact in fp32) with
+// one fp32 rounding, the same result as converting first and then fmaf.
+__device__ __forceinline__ void fma_bf16x2_f32(uint32_t a, uint32_t w, float& acc_lo, float& acc_hi) {
+  asm("{\n\t.reg .b16 al, ah, wl, wh;\n\t"
+      "mov.b32 {al, ah}, %2;\n\t"
+      "mov.b32 {wl, wh}, %3;\n\t"
+      "fma.rn.f32.bf16 %0, al, wl, %0;\n\t"
+      "fma.rn.f32.bf16 %1, ah, wh, %1;\n\t}"
+      : "+f"(acc_lo), "+f"(acc_hi)
+      : "r"(a), "r"(w));
+}
+
 // dot of C packed-bf16 chunks (register operand) with C chunks of a row, in
-// four independent two-lane accumulators (no dependent FMA chain).
+// eight independent accumulators (no dependent FMA chain), summed in a fixed
+// tree.
 template <int C>
 __device__ __forceinline__ float dot_chunks(const uint4 (&a)[C], const uint4 (&w)[C]) {
-  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int c = 0; c < C; ++c) {
     const uint32_t av[4] = {a[c].x, a[c].y, a[c].z, a[c].w};
     const uint32_t wv[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc[e] = fma2(bf16x2_to_f2(av[e]), bf16x2_to_f2(wv[e]), acc[e]);
+    for (int e = 0; e < 4; ++e) fma_bf16x2_f32(av[e], wv[e], acc[2 * e], acc[2 * e + 1]);
   }
-  return ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
 // y += a * w over C chunks; y is held as pairs for the two-lane FMA.
