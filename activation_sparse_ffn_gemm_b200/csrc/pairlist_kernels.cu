@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(kScanBlock) csc_scan_kernel(int* __restrict__ 
 }
 
 __global__ void __launch_bounds__(256) csc_fill_kernel(
-    const uint16_t* __restrict__ count, const uint16_t* __restrict__ val, const uint8_t* __restrict__ col,
+    const uint16_t* __restrict__ count, const uint8_t* __restrict__ col,
     const uint8_t* __restrict__ row_ovf, const int* __restrict__ row_slot, const uint16_t* __restrict__ g_ovf,
     const float* __restrict__ u_ovf, const float4* __restrict__ hdz_ell, const float* __restrict__ du_ovf,
     const float* __restrict__ dz_ovf,
@@ -451,11 +451,10 @@ cudaError_t launch_ovf_operands(const int* n_ovf, const int* ovf_rows, const int
   return cudaGetLastError();
 }
 
-cudaError_t launch_build_csc(const uint16_t* count, const uint16_t* val, const uint8_t* col,
-                             const uint8_t* row_ovf, const int* ovf_rows, const int* n_ovf, const uint16_t* g_ovf,
-                             const float* u_ovf, const float4* hdz_ell,
-                             const float* du_ovf, const float* dz_ovf, const int* plan, int M, int f, int K,
-                             int cap, const CscBuffers& b, cudaStream_t s) {
+cudaError_t launch_build_csc(const uint16_t* count, const uint8_t* col, const uint8_t* row_ovf,
+                             const uint16_t* g_ovf, const float* u_ovf, const float4* hdz_ell, const float* du_ovf,
+                             const float* dz_ovf, const int* plan, int M, int f, int K, const CscBuffers& b,
+                             cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   const int nch = (M + kCscRows - 1) / kCscRows;
   const int T = f / kTn;
@@ -466,7 +465,7 @@ cudaError_t launch_build_csc(const uint16_t* count, const uint16_t* val, const u
                csc_scan_kernel<<<(f + kScanBlock - 1) / kScanBlock, kScanBlock, 0, s>>>(
                    b.block_cnt, nch, f, b.unit_tot, b.unit_ptr, b.arrive, next_launch_epoch() & ((1ull << 40) - 1)));
   TWELL_LAUNCH("csc_fill", s,
-               csc_fill_kernel<<<dim3(T, nch), 256, 0, s>>>(count, val, col, row_ovf, b.row_slot, g_ovf, u_ovf,
+               csc_fill_kernel<<<dim3(T, nch), 256, 0, s>>>(count, col, row_ovf, b.row_slot, g_ovf, u_ovf,
                                                            hdz_ell, du_ovf, dz_ovf, b.block_cnt, b.unit_ptr, plan,
                                                            M, f, K, b.csc_row, b.csc_val));
   return cudaGetLastError();

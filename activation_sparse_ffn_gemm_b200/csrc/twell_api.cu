@@ -360,8 +360,8 @@ twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_
   CscBuffers b{h->row_plan + kPlanHdr + M,          at<int>(ws, L.block_cnt), at<int>(ws, L.unit_tot),
                at<unsigned long long>(ws, L.scan_arrive), at<int>(ws, L.unit_ptr), at<int>(ws, L.csc_row),
                at<float4>(ws, L.csc_val)};
-  if (launch_build_csc(h->count, h->val, h->col, h->row_ovf, h->ovf_rows, h->n_ovf, h->g_ovf, h->u_ovf,
-                       hdz_ell, du_ovf, dz_ovf, h->row_plan, M, f, K, cap, b, s) != cudaSuccess)
+  if (launch_build_csc(h->count, h->col, h->row_ovf, h->g_ovf, h->u_ovf, hdz_ell, du_ovf, dz_ovf, h->row_plan, M, f,
+                       K, b, s) != cudaSuccess)
     return TWELL_ECUDA;
   if (launch_dense_wgrad(dw, k_rows, cap, d, f, dW_g, dW_u, dW_d, h->status, s) != cudaSuccess) return TWELL_ECUDA;
   return cuda_status(launch_weight_grads(X, dY, b, d, f, cap > 0 ? db_ovf : nullptr, cap > 0 ? k_rows : nullptr,

@@ -212,11 +212,10 @@ constexpr int kCscRows = 256;  // rows per chunk of the pair-list build
 
 // Unit-major list of every active (row, unit) pair of the hybrid format, in
 // ascending row order per unit, with h, dU and dZ attached.
-cudaError_t launch_build_csc(const uint16_t* count, const uint16_t* val, const uint8_t* col,
-                             const uint8_t* row_ovf, const int* ovf_rows, const int* n_ovf, const uint16_t* g_ovf,
-                             const float* u_ovf, const float4* hdz_ell,
-                             const float* du_ovf, const float* dz_ovf, const int* plan, int M, int f, int K,
-                             int cap, const CscBuffers& b, cudaStream_t s);
+cudaError_t launch_build_csc(const uint16_t* count, const uint8_t* col, const uint8_t* row_ovf,
+                             const uint16_t* g_ovf, const float* u_ovf, const float4* hdz_ell, const float* du_ovf,
+                             const float* dz_ovf, const int* plan, int M, int f, int K, const CscBuffers& b,
+                             cudaStream_t s);
 
 // After the dense backward: the operands of the dense weight gradients (from X,
 // the gathered dY rows, fp32 dU / dZ and g, u of the overflow rows), column
