@@ -235,119 +235,150 @@ __global__ void __launch_bounds__(256) csc_fill_kernel(
   }
 }
 
-// One warp per unit, 8 consecutive units per CTA, one 16-byte chunk (8
-// columns) per lane: a CTA covers a 256-column slice. The warp stages its
-// unit's list 32 entries at a time in shared memory (one coalesced load), so
-// the x and dY loads of kWgBatch pairs are issued back to back; entries come
-// from shared-memory broadcasts. Accumulation uses the two-lane FMA. dW_d[:, j]
-// is transposed through shared memory so that each output row gets 8
-// consecutive units (32 bytes).
+// A CTA covers 8 consecutive units and a 256-column slice; each lane owns one
+// 16-byte chunk (8 columns). Its 4 warps take the 8 units one at a time from a
+// shared counter, longest pair list first, so a long list does not leave the
+// other warps waiting at the CTA's end. A warp stages its unit's list 32
+// entries at a time in shared memory (one coalesced load), then issues the x
+// and dY loads of kWgBatch pairs back to back; entries come from
+// shared-memory broadcasts and accumulation uses the two-lane FMA. Each unit's
+// sums are taken in list order, whichever warp runs it, so the result is the
+// same on every run. dW_d[:, j] is transposed through shared memory so that
+// each output row gets 8 consecutive units (32 bytes).
 constexpr int kWgBatch = 4;
 constexpr int kWgCols = 256;
+constexpr int kWgUnits = 8;   // units per CTA
+constexpr int kWgWarps = 4;   // warps per CTA
 
-__global__ void __launch_bounds__(256, 3) wgrad_kernel(const uint16_t* __restrict__ X,
-                                                       const uint16_t* __restrict__ dY,
-                                                       const int* __restrict__ unit_ptr,
-                                                       const int* __restrict__ csc_row,
-                                                       const float4* __restrict__ csc_val, int d, int f,
-                                                       const float* __restrict__ db_extra,
-                                                       const int* __restrict__ accumulate, float* __restrict__ dWg,
-                                                       float* __restrict__ dWu, float* __restrict__ dWd,
-                                                       float* __restrict__ dbg) {
-  __shared__ float s_dwd[kWgCols][9];
-  __shared__ int s_row[8][32];
-  __shared__ float4 s_val[8][32];
+__global__ void __launch_bounds__(kWgWarps * 32, 6) wgrad_kernel(const uint16_t* __restrict__ X,
+                                                                 const uint16_t* __restrict__ dY,
+                                                                 const int* __restrict__ unit_ptr,
+                                                                 const int* __restrict__ csc_row,
+                                                                 const float4* __restrict__ csc_val, int d, int f,
+                                                                 const float* __restrict__ db_extra,
+                                                                 const int* __restrict__ accumulate,
+                                                                 float* __restrict__ dWg, float* __restrict__ dWu,
+                                                                 float* __restrict__ dWd, float* __restrict__ dbg) {
+  __shared__ float s_dwd[kWgCols][kWgUnits + 1];
+  __shared__ int s_row[kWgWarps][32];
+  __shared__ float4 s_val[kWgWarps][32];
+  __shared__ int s_order[kWgUnits];
+  __shared__ int s_next;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = blockIdx.x * 8 + w;
+  const int j0 = blockIdx.x * kWgUnits;
   const int c0 = blockIdx.y * kWgCols;
   const int cidx = (c0 >> 3) + lane;
   const bool cval = cidx < (d >> 3);
   // add to the dense GEMMs' result (written before this kernel) instead of
-  // overwriting: its lines are pulled into L2 now and read after the pair loop
+  // overwriting: its lines are pulled into L2 now and read after the pair loops
   const bool acc_old = accumulate != nullptr && *accumulate > 0;
-  float* pu_out = dWu + static_cast<long>(j) * d + 8 * cidx;
-  float* pg_out = dWg + static_cast<long>(j) * d + 8 * cidx;
-  float* pd_out = dWd + static_cast<long>(c0 + threadIdx.x) * f + blockIdx.x * 8;
-  if (acc_old) {
-    if (cval) {
+  if (threadIdx.x == 0) {
+    int len[kWgUnits];
+    for (int u = 0; u < kWgUnits; ++u) {
+      len[u] = unit_ptr[j0 + u + 1] - unit_ptr[j0 + u];
+      s_order[u] = u;
+    }
+    for (int u = 1; u < kWgUnits; ++u)  // insertion sort, longest first (ties: lower unit first)
+      for (int v = u; v > 0 && len[s_order[v]] > len[s_order[v - 1]]; --v) {
+        const int t = s_order[v];
+        s_order[v] = s_order[v - 1];
+        s_order[v - 1] = t;
+      }
+    s_next = 0;
+  }
+  if (acc_old)
+    for (int r = threadIdx.x; r < kWgCols; r += kWgWarps * 32)
+      if (c0 + r < d) asm volatile("prefetch.global.L2 [%0];" ::"l"(dWd + static_cast<long>(c0 + r) * f + j0));
+  __syncthreads();
+
+  for (;;) {
+    int u = 0;
+    if (lane == 0) u = atomicAdd(&s_next, 1);
+    u = __shfl_sync(0xFFFFFFFFu, u, 0);
+    if (u >= kWgUnits) break;
+    const int lu = s_order[u];
+    const int j = j0 + lu;
+    float* pu_out = dWu + static_cast<long>(j) * d + 8 * cidx;
+    float* pg_out = dWg + static_cast<long>(j) * d + 8 * cidx;
+    if (acc_old && cval) {
       asm volatile("prefetch.global.L2 [%0];" ::"l"(pu_out));
       asm volatile("prefetch.global.L2 [%0];" ::"l"(pg_out));
     }
-    if (c0 + static_cast<int>(threadIdx.x) < d) asm volatile("prefetch.global.L2 [%0];" ::"l"(pd_out));
-  }
-  float2 au[4], ag[4], ad[4];
+    float2 au[4], ag[4], ad[4];
 #pragma unroll
-  for (int e = 0; e < 4; ++e) au[e] = ag[e] = ad[e] = make_float2(0.f, 0.f);
-  float db = 0.f;
-  const int p0 = unit_ptr[j], p1 = unit_ptr[j + 1];
-  for (int pb = p0; pb < p1; pb += 32) {
-    const int n = min(32, p1 - pb);
-    __syncwarp();
-    if (lane < n) {
-      s_row[w][lane] = csc_row[pb + lane];
-      const float4 v = csc_val[pb + lane];
-      s_val[w][lane] = v;
-      db += v.z;
-    }
-    __syncwarp();
-    for (int b0 = 0; b0 < n; b0 += kWgBatch) {
-      uint4 xv[kWgBatch], dv[kWgBatch];
+    for (int e = 0; e < 4; ++e) au[e] = ag[e] = ad[e] = make_float2(0.f, 0.f);
+    float db = 0.f;
+    const int p0 = unit_ptr[j], p1 = unit_ptr[j + 1];
+    for (int pb = p0; pb < p1; pb += 32) {
+      const int n = min(32, p1 - pb);
+      __syncwarp();
+      if (lane < n) {
+        s_row[w][lane] = csc_row[pb + lane];
+        const float4 v = csc_val[pb + lane];
+        s_val[w][lane] = v;
+        db += v.z;
+      }
+      __syncwarp();
+      for (int b0 = 0; b0 < n; b0 += kWgBatch) {
+        uint4 xv[kWgBatch], dv[kWgBatch];
 #pragma unroll
-      for (int b = 0; b < kWgBatch; ++b) {
-        const long r = s_row[w][min(b0 + b, n - 1)];
-        if (cval) {
-          xv[b] = __ldg(reinterpret_cast<const uint4*>(X + r * d) + cidx);
-          dv[b] = __ldg(reinterpret_cast<const uint4*>(dY + r * d) + cidx);
-        } else {
-          xv[b] = dv[b] = make_uint4(0, 0, 0, 0);
+        for (int b = 0; b < kWgBatch; ++b) {
+          const long r = s_row[w][min(b0 + b, n - 1)];
+          if (cval) {
+            xv[b] = __ldg(reinterpret_cast<const uint4*>(X + r * d) + cidx);
+            dv[b] = __ldg(reinterpret_cast<const uint4*>(dY + r * d) + cidx);
+          } else {
+            xv[b] = dv[b] = make_uint4(0, 0, 0, 0);
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < kWgBatch; ++b) {
+          const float4 v = b0 + b < n ? s_val[w][b0 + b] : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float2 h2 = make_float2(v.x, v.x), u2 = make_float2(v.y, v.y), z2 = make_float2(v.z, v.z);
+          const uint32_t xw[4] = {xv[b].x, xv[b].y, xv[b].z, xv[b].w};
+          const uint32_t dw[4] = {dv[b].x, dv[b].y, dv[b].z, dv[b].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 xf = bf16x2_to_f2(xw[e]);
+            au[e] = fma2(u2, xf, au[e]);
+            ag[e] = fma2(z2, xf, ag[e]);
+            ad[e] = fma2(h2, bf16x2_to_f2(dw[e]), ad[e]);
+          }
         }
       }
-#pragma unroll
-      for (int b = 0; b < kWgBatch; ++b) {
-        const float4 v = b0 + b < n ? s_val[w][b0 + b] : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float2 h2 = make_float2(v.x, v.x), u2 = make_float2(v.y, v.y), z2 = make_float2(v.z, v.z);
-        const uint32_t xw[4] = {xv[b].x, xv[b].y, xv[b].z, xv[b].w};
-        const uint32_t dw[4] = {dv[b].x, dv[b].y, dv[b].z, dv[b].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 xf = bf16x2_to_f2(xw[e]);
-          au[e] = fma2(u2, xf, au[e]);
-          ag[e] = fma2(z2, xf, ag[e]);
-          ad[e] = fma2(h2, bf16x2_to_f2(dw[e]), ad[e]);
-        }
+    }
+    db = warp_sum(db);
+    if (cval) {
+      float4* pu = reinterpret_cast<float4*>(pu_out);
+      float4* pg = reinterpret_cast<float4*>(pg_out);
+      float4 u0 = make_float4(au[0].x, au[0].y, au[1].x, au[1].y), u1 = make_float4(au[2].x, au[2].y, au[3].x, au[3].y);
+      float4 g0 = make_float4(ag[0].x, ag[0].y, ag[1].x, ag[1].y), g1 = make_float4(ag[2].x, ag[2].y, ag[3].x, ag[3].y);
+      if (acc_old) {
+        const float4 ou0 = pu[0], ou1 = pu[1], og0 = pg[0], og1 = pg[1];
+        u0 = make_float4(ou0.x + u0.x, ou0.y + u0.y, ou0.z + u0.z, ou0.w + u0.w);
+        u1 = make_float4(ou1.x + u1.x, ou1.y + u1.y, ou1.z + u1.z, ou1.w + u1.w);
+        g0 = make_float4(og0.x + g0.x, og0.y + g0.y, og0.z + g0.z, og0.w + g0.w);
+        g1 = make_float4(og1.x + g1.x, og1.y + g1.y, og1.z + g1.z, og1.w + g1.w);
       }
+      pu[0] = u0;
+      pu[1] = u1;
+      pg[0] = g0;
+      pg[1] = g1;
     }
-  }
-  db = warp_sum(db);
-  if (cval) {
-    float4* pu = reinterpret_cast<float4*>(pu_out);
-    float4* pg = reinterpret_cast<float4*>(pg_out);
-    float4 u0 = make_float4(au[0].x, au[0].y, au[1].x, au[1].y), u1 = make_float4(au[2].x, au[2].y, au[3].x, au[3].y);
-    float4 g0 = make_float4(ag[0].x, ag[0].y, ag[1].x, ag[1].y), g1 = make_float4(ag[2].x, ag[2].y, ag[3].x, ag[3].y);
-    if (acc_old) {
-      const float4 ou0 = pu[0], ou1 = pu[1], og0 = pg[0], og1 = pg[1];
-      u0 = make_float4(ou0.x + u0.x, ou0.y + u0.y, ou0.z + u0.z, ou0.w + u0.w);
-      u1 = make_float4(ou1.x + u1.x, ou1.y + u1.y, ou1.z + u1.z, ou1.w + u1.w);
-      g0 = make_float4(og0.x + g0.x, og0.y + g0.y, og0.z + g0.z, og0.w + g0.w);
-      g1 = make_float4(og1.x + g1.x, og1.y + g1.y, og1.z + g1.z, og1.w + g1.w);
-    }
-    pu[0] = u0;
-    pu[1] = u1;
-    pg[0] = g0;
-    pg[1] = g1;
-  }
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    s_dwd[lane * 8 + 2 * e][w] = ad[e].x;
-    s_dwd[lane * 8 + 2 * e + 1][w] = ad[e].y;
+    for (int e = 0; e < 4; ++e) {
+      s_dwd[lane * 8 + 2 * e][lu] = ad[e].x;
+      s_dwd[lane * 8 + 2 * e + 1][lu] = ad[e].y;
+    }
+    if (blockIdx.y == 0 && lane == 0 && dbg != nullptr) dbg[j] = db_extra ? db + db_extra[j] : db;
   }
-  if (blockIdx.y == 0 && lane == 0 && dbg != nullptr) dbg[j] = db_extra ? db + db_extra[j] : db;
   __syncthreads();
-  const int cc = c0 + threadIdx.x;
-  if (cc < d) {
-    float4* pd = reinterpret_cast<float4*>(pd_out);
-    float4 d0 = make_float4(s_dwd[threadIdx.x][0], s_dwd[threadIdx.x][1], s_dwd[threadIdx.x][2], s_dwd[threadIdx.x][3]);
-    float4 d1 = make_float4(s_dwd[threadIdx.x][4], s_dwd[threadIdx.x][5], s_dwd[threadIdx.x][6], s_dwd[threadIdx.x][7]);
+  for (int r = threadIdx.x; r < kWgCols; r += kWgWarps * 32) {
+    const int cc = c0 + r;
+    if (cc >= d) continue;
+    float4* pd = reinterpret_cast<float4*>(dWd + static_cast<long>(cc) * f + j0);
+    float4 d0 = make_float4(s_dwd[r][0], s_dwd[r][1], s_dwd[r][2], s_dwd[r][3]);
+    float4 d1 = make_float4(s_dwd[r][4], s_dwd[r][5], s_dwd[r][6], s_dwd[r][7]);
     if (acc_old) {
       const float4 o0 = pd[0], o1 = pd[1];
       d0 = make_float4(o0.x + d0.x, o0.y + d0.y, o0.z + d0.z, o0.w + d0.w);
@@ -474,9 +505,9 @@ cudaError_t launch_build_csc(const uint16_t* count, const uint8_t* col, const ui
 cudaError_t launch_weight_grads(const uint16_t* X, const uint16_t* dY, const CscBuffers& b, int d, int f,
                                 const float* db_extra, const int* accumulate, float* dW_g, float* dW_u,
                                 float* dW_d, float* db_g, cudaStream_t s) {
-  dim3 grid(f / 8, (d + kWgCols - 1) / kWgCols);
+  dim3 grid(f / kWgUnits, (d + kWgCols - 1) / kWgCols);
   TWELL_LAUNCH("weight_grads", s,
-               wgrad_kernel<<<grid, 256, 0, s>>>(X, dY, b.unit_ptr, b.csc_row, b.csc_val, d, f, db_extra, accumulate,
+               wgrad_kernel<<<grid, kWgWarps * 32, 0, s>>>(X, dY, b.unit_ptr, b.csc_row, b.csc_val, d, f, db_extra, accumulate,
                                                  dW_g, dW_u, dW_d, db_g));
   return cudaGetLastError();
 }
