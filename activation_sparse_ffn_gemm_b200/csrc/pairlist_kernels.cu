@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(256) csc_fill_kernel(
 // sums are taken in list order, whichever warp runs it, so the result is the
 // same on every run. dW_d[:, j] is transposed through shared memory so that
 // each output row gets 8 consecutive units (32 bytes).
-constexpr int kWgBatch = 4;
+constexpr int kWgBatch = 4;  // pairs whose row loads are issued together (2, 6, 8 measured slower)
 constexpr int kWgCols = 256;
 constexpr int kWgUnits = 8;   // units per CTA
 constexpr int kWgWarps = 4;   // warps per CTA

@@ -92,6 +92,9 @@ CASES = {
     # (190 and 183 overflow rows: the contraction's zeroed tail rows matter)
     "dense_wgrad": (300, 256, 512, 8, 0.12, "lognormal", 17),
     "dense_wgrad_ragged": (260, 192, 384, 8, 0.15, "lognormal", 19),
+    # 170 overflow rows of a heavy-tailed batch: split-K dense backup GEMMs,
+    # overflow pairs kept in the pair list
+    "heavy_small": (1024, 1024, 4096, 8, 0.02, "lognormal", 23),
 }
 
 
