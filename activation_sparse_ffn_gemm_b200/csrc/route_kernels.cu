@@ -260,34 +260,48 @@ __global__ void gather_rows_kernel(const uint16_t* __restrict__ in, const int* _
   }
 }
 
-// out[c][r] = in[r][c] for a [rows][cols] bf16 matrix, 64 x 64 tiles through
-// shared memory (16-byte global accesses on both sides).
-__global__ void transpose_bf16_kernel(const uint16_t* __restrict__ in, int rows, int cols,
-                                      uint16_t* __restrict__ out) {
-  __shared__ uint16_t tile[64][64 + 2];
-  const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
-  const int tid = threadIdx.x;  // 256 threads: 64 rows x 8 chunks of 8
-  for (int i = tid; i < 64 * 8; i += 256) {
-    const int r = i >> 3, q = i & 7;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r0 + r < rows && c0 + q * 8 < cols)
-      v = *reinterpret_cast<const uint4*>(in + static_cast<long>(r0 + r) * cols + c0 + q * 8);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+// out[c][r] = in[r][c] for a [rows][cols] bf16 matrix (rows, cols multiples of
+// 8). A CTA moves a 64-row x 128-column tile: every thread first issues its four
+// 16-byte loads (256 contiguous bytes per input row), then parks them in shared
+// memory as 32-bit words, each holding a column pair of one row. The word
+// column is XOR-swizzled by the row's octet so that both the 16-byte stores and
+// the column reads are free of bank conflicts. Each thread then reads eight rows
+// of one column pair and writes two 16-byte output chunks (columns 2p and 2p+1).
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(const uint16_t* __restrict__ in, int rows, int cols,
+                                                            uint16_t* __restrict__ out) {
+  constexpr int TR = 64, TC = 128, WPR = TC / 2;  // words per tile row
+  __shared__ __align__(16) uint32_t tile[TR * WPR];
+  const int r0 = blockIdx.y * TR, c0 = blockIdx.x * TC;
+  const int tid = threadIdx.x;
+  const auto swz = [](int r, int j) { return r * WPR + (j ^ (((r >> 3) & 7) << 2)); };
+  uint4 v[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      tile[r][q * 8 + 2 * e] = w[e] & 0xFFFFu;
-      tile[r][q * 8 + 2 * e + 1] = w[e] >> 16;
-    }
+  for (int k = 0; k < 4; ++k) {  // chunk i: row i / 16, columns 8 (i % 16) ..
+    const int i = tid + 256 * k, r = i >> 4, q = i & 15;
+    v[k] = make_uint4(0, 0, 0, 0);
+    if (r0 + r < rows && c0 + q * 8 < cols)
+      v[k] = __ldg(reinterpret_cast<const uint4*>(in + static_cast<long>(r0 + r) * cols + c0 + q * 8));
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int i = tid + 256 * k, r = i >> 4, q = i & 15;
+    *reinterpret_cast<uint4*>(&tile[swz(r, 4 * q)]) = v[k];
   }
   __syncthreads();
-  for (int i = tid; i < 64 * 8; i += 256) {
-    const int c = i >> 3, q = i & 7;
-    if (c0 + c >= cols || r0 + q * 8 >= rows) continue;
-    uint32_t w[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
-      w[e] = uint32_t(tile[q * 8 + 2 * e][c]) | (uint32_t(tile[q * 8 + 2 * e + 1][c]) << 16);
-    *reinterpret_cast<uint4*>(out + static_cast<long>(c0 + c) * rows + r0 + q * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+  for (int k = 0; k < 2; ++k) {  // task i: row octet i % 8, column pair i / 8
+    const int i = tid + 256 * k, o = i & 7, p = i >> 3;
+    uint32_t w[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) w[e] = tile[swz(8 * o + e, p)];
+    const uint4 lo = make_uint4(__byte_perm(w[0], w[1], 0x5410), __byte_perm(w[2], w[3], 0x5410),
+                                __byte_perm(w[4], w[5], 0x5410), __byte_perm(w[6], w[7], 0x5410));
+    const uint4 hi = make_uint4(__byte_perm(w[0], w[1], 0x7632), __byte_perm(w[2], w[3], 0x7632),
+                                __byte_perm(w[4], w[5], 0x7632), __byte_perm(w[6], w[7], 0x7632));
+    const int c = c0 + 2 * p, r = r0 + 8 * o;
+    if (r >= rows) continue;
+    if (c < cols) *reinterpret_cast<uint4*>(out + static_cast<long>(c) * rows + r) = lo;
+    if (c + 1 < cols) *reinterpret_cast<uint4*>(out + static_cast<long>(c + 1) * rows + r) = hi;
   }
 }
 
@@ -324,7 +338,7 @@ cudaError_t launch_gather_rows(const uint16_t* in, const int* rows, const int* n
 
 cudaError_t launch_transpose_bf16(const uint16_t* in, int rows, int cols, uint16_t* out, cudaStream_t s) {
   if (rows <= 0 || cols <= 0) return cudaSuccess;
-  dim3 grid((cols + 63) / 64, (rows + 63) / 64);
+  dim3 grid((cols + 127) / 128, (rows + 63) / 64);
   TWELL_LAUNCH("transpose_wd", s, transpose_bf16_kernel<<<grid, 256, 0, s>>>(in, rows, cols, out));
   return cudaGetLastError();
 }
