@@ -486,6 +486,21 @@ def run_twell(args, world, rank, local):
     assert torch.equal(hY[(args.steps - 1) % 2].to(dev), Y), "end-to-end result differs from the resident run"
     assert st.read_status() == 0, "device status word set during timing"
 
+    def copy_ms(body, reps=5):
+        """Mean time of one step's host<->device copies alone (no compute), for context."""
+        body()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            body()
+        e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    ms_h2d = copy_ms(lambda: (Xb[1].copy_(hX, non_blocking=True), dYb[1].copy_(hdY, non_blocking=True)))
+    ms_d2h = copy_ms(lambda: hY[1].copy_(Yb[0], non_blocking=True))
+
     # dense bf16 comparison point (torch / cuBLAS), same protocol
     dense = None
     if not args.no_dense:
@@ -574,6 +589,7 @@ def run_twell(args, world, rank, local):
                              if dense else None),
         "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": 2 * M * d * 2,
                 "d2h_bytes_per_step": M * d * 2, "ms_per_step": ms_e2e,
+                "copy_alone_ms": {"h2d": ms_h2d, "d2h": ms_d2h},
                 "copies": "pinned host X and dY in and Y out every step, on two copy streams, overlapping the "
                           "neighbouring steps' compute (double-buffered device inputs and outputs)"},
         "gpu_launches": launches,

@@ -13,4 +13,5 @@ from .workloads import (  # noqa: F401
     gate_bias_for_activity,
     make_inputs,
     sweep_k,
+    sweep_workload,
 )

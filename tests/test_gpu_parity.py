@@ -12,7 +12,7 @@ import os
 import numpy as np
 import pytest
 
-from synthetic import WORKLOADS, Workload, make_inputs
+from synthetic import WORKLOADS, Workload, make_inputs, sweep_workload
 from twell_testlib import (assert_active_set, assert_matches_oracle, assert_pack_equal, assert_plan_valid, bits_of,
                            f32_of_bits, gpu_gmat, state_to_numpy, to_dev)
 
@@ -262,6 +262,28 @@ def test_train_full_size(tw, orc):
         g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=lam)
         torch.cuda.synchronize()
         _check_bwd(orc, inp, g, G, lam, "train")
+
+
+@pytest.mark.parametrize("M,activity,bwd", [(2048, 0.1, False), (512, 0.001, False), (64, 0.1, True),
+                                              (96, 0.05, True)])
+def test_sweep_points(tw, orc, M, activity, bwd):
+    """Points of the d_model=4096, d_ff=14336 lognormal sweep (K = 64, 8, 64, 32):
+    pack on all rows and Y on a sample plus every overflow row; for the small-M
+    points also the backward, every gradient on its full tensor."""
+    w = sweep_workload(M, activity)
+    inp = make_inputs(w)
+    D, Y, st, z = _run_fwd(tw, inp, w, save=bwd)
+    p = state_to_numpy(st)
+    extra = p["ovf_rows"][:p["n_ovf"]][:16]
+    rows = np.arange(M, dtype=np.int32) if bwd else _sample_rows(M, 64, 3, extra=extra)
+    p, _, _ = _check_fwd(orc, inp, w, Y, st, z, rows=rows)
+    assert_plan_valid(st)
+    if bwd:
+        G = gpu_gmat(p, M, w.d_ff, w.T_n, w.K)
+        g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=1e-3)
+        torch.cuda.synchronize()
+        assert st.read_status() == 0
+        _check_bwd(orc, inp, g, G, 1e-3, w.name)
 
 
 @pytest.mark.parametrize("name", ["k32", "multi_tile", "ragged_k16", "tiny"])
