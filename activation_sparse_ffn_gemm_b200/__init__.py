@@ -18,6 +18,8 @@ from typing import Optional
 
 import torch
 
+from .kchoice import CostModel, modelled_times, suggest_k  # noqa: F401
+
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libtwell.so")
 
@@ -92,6 +94,8 @@ def lib():
             L.twell_trace_enable.argtypes = [ctypes.c_int]
             L.twell_trace_collect.restype = ctypes.c_int
             L.twell_trace_collect.argtypes = [ctypes.POINTER(TwellTraceRec), ctypes.c_int]
+            L.twell_count_stats.restype = ctypes.c_int
+            L.twell_count_stats.argtypes = [ctypes.POINTER(TwellHybrid), _vp, _vp, _vp, _vp]
             L.twell_status_read.restype = ctypes.c_int
             L.twell_status_read.argtypes = [ctypes.POINTER(TwellHybrid), ctypes.POINTER(ctypes.c_uint32),
                                             ctypes.c_int, _vp]
@@ -186,6 +190,17 @@ class HybridState:
     def n_overflow(self) -> tuple[int, int]:
         v = self.n_ovf.cpu().tolist()
         return int(v[0]), int(v[1])
+
+
+def count_stats(state: HybridState, stream=None) -> dict:
+    """Count statistics of a packed batch (twell_count_stats): int64 CUDA tensors
+    rows_by_max, act_by_max, tiles_by_count of T_n + 1 bins each."""
+    n = state.T_n + 1
+    dev = state.count.device
+    out = {k: torch.empty(n, dtype=torch.int64, device=dev) for k in ("rows_by_max", "act_by_max", "tiles_by_count")}
+    _check(lib().twell_count_stats(ctypes.byref(state.c), _ptr(out["rows_by_max"]), _ptr(out["act_by_max"]),
+                                   _ptr(out["tiles_by_count"]), _stream(stream)), "twell_count_stats")
+    return out
 
 
 def transpose_wd(W_d: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

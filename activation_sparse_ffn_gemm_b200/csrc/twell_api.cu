@@ -6,6 +6,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "count_stats.cuh"
 #include "twell_internal.cuh"
 
 namespace twell {
@@ -366,6 +367,20 @@ twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_
   if (launch_dense_wgrad(dw, k_rows, cap, d, f, dW_g, dW_u, dW_d, h->status, s) != cudaSuccess) return TWELL_ECUDA;
   return cuda_status(launch_weight_grads(X, dY, b, d, f, cap > 0 ? db_ovf : nullptr, cap > 0 ? k_rows : nullptr,
                                          dW_g, dW_u, dW_d, db_g, s));
+}
+
+twell_status twell_count_stats(const twell_hybrid* h, int64_t* rows_by_max, int64_t* act_by_max,
+                               int64_t* tiles_by_count, twell_stream_t stream) {
+  if (!h || !rows_by_max || !act_by_max || !tiles_by_count) return TWELL_EINVAL;
+  for (const void* p : {static_cast<const void*>(rows_by_max), static_cast<const void*>(act_by_max),
+                        static_cast<const void*>(tiles_by_count)})
+    if ((reinterpret_cast<uintptr_t>(p) & 7) != 0) return TWELL_EINVAL;
+  // d_model plays no part here; the smallest supported one stands in for it
+  const twell_status st = twell_query_support(h->M, 64, h->d_ff, h->T_n, h->K, h->ovf_cap);
+  if (st != TWELL_OK) return st;
+  if (h->M > 0 && (!h->count || !aligned16(h->count))) return TWELL_EINVAL;
+  return cuda_status(launch_count_stats(h->count, h->M, h->d_ff / kTn, rows_by_max, act_by_max, tiles_by_count,
+                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
 twell_status twell_status_read(const twell_hybrid* h, uint32_t* out, int clear, twell_stream_t stream) {

@@ -1,0 +1,97 @@
+"""Choice of the ELL width K from the count statistics of a batch.
+
+The pages fix no K. [aivizor] paragraph 4 only warns that in training the
+largest number of nonzeros per row can be far above the mean, so one fixed K
+either wastes slots or sends many rows to the dense backup. This module turns
+the statistics of ``twell_count_stats`` (bins c = 0..T_n of per-row largest
+tile count, with those rows' active units, and of per-tile counts) into a
+modelled time per candidate K and returns the cheapest. A training loop calls
+it on one batch's statistics to set K for the next batches; an inference
+server calls it on a calibration batch.
+
+Row routing, candidate K:
+    rows(K)  = sum of rows_by_max[c] over c > K        (dense backup rows)
+    pairs(K) = sum of act_by_max[c] over c <= K        (units kept in ELL slots)
+    t(K) = a * d * pairs(K) + r * d * f * rows(K) + (bytes of the slots) / BW
+Tile routing (inference only), every active unit is gathered and each tile
+over K is read from its spilled dense slice:
+    t(K) = a * d * total + (bytes of the slots + 512 bytes per spilled tile) / BW
+with the slot bytes M * T * (2 + 3K) (count, values, columns), written by the
+gate epilogue and read back once.
+
+The coefficients are B200 measurements of this library: ``a`` is the time of
+one (token, unit) pair per d_model element in the sparse kernels (forward: the
+fused up+down; training adds the sparse backward, the pair list and the weight
+gradients), ``r`` the time per d_model * d_ff of one dense backup row on the
+tensor cores (4 flops per element in the forward, about 18 with the backward,
+whose dense weight gradients run on hi/lo operand pairs), ``BW`` the HBM copy
+rate.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Iterable, Mapping, Sequence
+
+import numpy as np
+
+CANDIDATES = (8, 16, 32, 64)
+
+
+@dataclass(frozen=True)
+class CostModel:
+    pair_fwd_s: float = 2.5e-13      # fused up+down, per pair per d_model element
+    pair_bwd_s: float = 8.0e-13      # sparse backward + pair list + weight gradients
+    dense_fwd_s: float = 4.0 / 1.0e15   # per row per d_model * d_ff: 4 flops at ~1 PFLOP/s
+    dense_bwd_s: float = 18.0 / 1.0e15  # dH, dX and the hi/lo dense weight gradients
+    hbm_bytes_s: float = 6.5e12
+
+
+def _np(stats: Mapping[str, object], key: str) -> np.ndarray:
+    v = stats[key]
+    if hasattr(v, "detach"):
+        v = v.detach().cpu().numpy()
+    return np.asarray(v, dtype=np.int64)
+
+
+def modelled_times(stats: Mapping[str, object], d_model: int, d_ff: int, T_n: int = 128,
+                   candidates: Iterable[int] = CANDIDATES, training: bool = True, routing: str = "rows",
+                   model: CostModel = CostModel()) -> dict:
+    """Modelled seconds per candidate K (see the module docstring)."""
+    if routing not in ("rows", "tiles"):
+        raise ValueError("routing is 'rows' or 'tiles'")
+    if training and routing == "tiles":
+        raise ValueError("tile routing is an inference-only format")
+    rows_by_max = _np(stats, "rows_by_max")
+    act_by_max = _np(stats, "act_by_max")
+    tiles_by_count = _np(stats, "tiles_by_count")
+    if not (rows_by_max.shape == act_by_max.shape == tiles_by_count.shape == (T_n + 1,)):
+        raise ValueError(f"statistics must have T_n + 1 = {T_n + 1} bins")
+    M = int(rows_by_max.sum())
+    T = d_ff // T_n
+    total = int(act_by_max.sum())
+    a = model.pair_fwd_s + (model.pair_bwd_s if training else 0.0)
+    r = model.dense_fwd_s + (model.dense_bwd_s if training else 0.0)
+    out = {}
+    for K in candidates:
+        K = int(K)
+        if not 1 <= K <= T_n:
+            raise ValueError(f"K={K} outside [1, T_n]")
+        slots = M * T * (2 + 3 * K)
+        if routing == "rows":
+            pairs = int(act_by_max[:K + 1].sum())
+            rows = int(rows_by_max[K + 1:].sum())
+            out[K] = a * d_model * pairs + r * d_model * d_ff * rows + slots / model.hbm_bytes_s
+        else:
+            spilled = int(tiles_by_count[K + 1:].sum())
+            out[K] = a * d_model * total + (slots + 512 * spilled) / model.hbm_bytes_s
+    return out
+
+
+def suggest_k(stats: Mapping[str, object], d_model: int, d_ff: int, T_n: int = 128,
+              candidates: Sequence[int] = CANDIDATES, training: bool = True, routing: str = "rows",
+              model: CostModel = CostModel()) -> tuple[int, dict]:
+    """The candidate K of least modelled time (the smaller K on a tie) and the table of times."""
+    times = modelled_times(stats, d_model, d_ff, T_n, candidates, training, routing, model)
+    best = min(sorted(times), key=lambda k: times[k])
+    return best, times

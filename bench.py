@@ -15,7 +15,9 @@ K=8) run as a training step, synthetic seeded data, inputs resident in HBM.
 FFN over token counts M in {512, 2048, 8192, 32768, 65536} and mean sparsity in
 {90, 95, 99, 99.5, 99.9}% at d_model=4096, d_ff=14336, with per-token
 lognormal(0, 0.75) row scaling, K = max(8, 2^ceil(log2(4 p T_n))), one JSON
-line per point (1 GPU).
+line per point (1 GPU). With --sweep-k 8,16,32,64 each point is timed for every
+listed K instead, next to the K that the batch's count statistics and the cost
+model of activation_sparse_ffn_gemm_b200.kchoice choose.
 
 Prints one JSON line (rank 0). With N > 1 (torchrun) every rank runs its own
 replica of the batch; the time is the max over ranks and the value counts the
@@ -58,6 +60,9 @@ def parse_args():
                    help="token-count x sparsity sweep at d_model=4096, d_ff=14336 (one JSON line per point)")
     p.add_argument("--sweep-m", default="512,2048,8192,32768,65536")
     p.add_argument("--sweep-sparsity", default="0.9,0.95,0.99,0.995,0.999")
+    p.add_argument("--sweep-k", default="",
+                   help="with --sweep: time every K of this list at each point (e.g. 8,16,32,64) next to the "
+                        "K chosen from the count statistics")
     return p.parse_args()
 
 
@@ -425,6 +430,19 @@ def run_twell(args, world, rank, local):
             b["ms_per_launch"] = b["ms"] / b["launches"]
             b["ms_per_step"] = b["ms"] / args.steps
 
+    # inference forward with fixed weights: W_d transposed once (outside the timed
+    # region, as an inference caller does), u not saved for a backward
+    st_inf = tw.HybridState(M, f, w.T_n, K, cap, dev, with_u=False)
+
+    def infer(e_mid):
+        tw.ffn_fwd(X, W_g, b_g, W_u, W_d, T_n=w.T_n, K=K, W_dt=Wdt, state=st_inf, ws=wsf, Y=Y)
+        e_mid.record(stream)
+
+    for _ in range(3):
+        infer(torch.cuda.Event())
+    ms_inf = max_over_ranks(timed(args.steps, infer)[0])
+    assert st_inf.read_status() == 0, "device status word set during the inference timing"
+
     # e2e: every step copies its inputs (X, dY) from pinned host memory and reads its
     # result Y back, inside the timed region. As a training loop that prefetches its
     # next batch does, the copies run on two copy streams (host->device, device->host)
@@ -583,9 +601,13 @@ def run_twell(args, world, rank, local):
         "config": {"workload": workload_desc(w, seed), "global_batch": tokens, "lambda_l1": args.lam,
                    "l2": "flushed before every timed step (256 MiB device write, outside the events)",
                    "accumulation": "fp32", "ovf_cap": cap, "parallelism": f"replicas x{world}"},
-        "fwd": {"tokens_per_s": tokens / (ms_fwd / 1e3), "ms": ms_fwd},
+        "fwd": {"tokens_per_s": tokens / (ms_fwd / 1e3), "ms": ms_fwd,
+                "note": "forward half of the training step (W_d transposed, u saved)"},
+        "fwd_inference": {"tokens_per_s": tokens / (ms_inf / 1e3), "ms": ms_inf,
+                          "note": "forward alone with fixed weights (W_dt prepared once, u not saved)"},
         "dense_bf16": dense,
-        "speedup_vs_dense": ({"fwd": dense["fwd_ms"] / ms_fwd, "fwd_bwd": dense["fwd_bwd_ms"] / ms_step}
+        "speedup_vs_dense": ({"fwd": dense["fwd_ms"] / ms_fwd, "fwd_inference": dense["fwd_ms"] / ms_inf,
+                              "fwd_bwd": dense["fwd_bwd_ms"] / ms_step}
                              if dense else None),
         "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": 2 * M * d * 2,
                 "d2h_bytes_per_step": M * d * 2, "ms_per_step": ms_e2e,
@@ -606,6 +628,97 @@ def run_twell(args, world, rank, local):
 
 
 # ---------------------------------------------------------------- sweep
+
+
+def _sweep_inputs(torch, dev, M, sp, d, f, sigma, bias):
+    """Seeded sweep-point inputs drawn on the device: X rows scaled by lognormal(0, sigma)."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000003 * M + int(round(sp * 1e4)))
+    rs = torch.exp(sigma * torch.randn(M, 1, device=dev, generator=g))
+    X = (torch.randn(M, d, device=dev, generator=g) * rs).to(torch.bfloat16)
+    W_g = (torch.randn(f, d, device=dev, generator=g) / math.sqrt(d)).to(torch.bfloat16)
+    W_u = (torch.randn(f, d, device=dev, generator=g) / math.sqrt(d)).to(torch.bfloat16)
+    W_d = (torch.randn(d, f, device=dev, generator=g) / math.sqrt(f)).to(torch.bfloat16)
+    dY = torch.randn(M, d, device=dev, generator=g).to(torch.bfloat16)
+    b_g = torch.full((f,), bias, device=dev).to(torch.bfloat16)
+    return X, W_g, W_u, W_d, dY, b_g, rs
+
+
+def run_ksweep(args, local):
+    """At each sweep point, the TwELL forward and forward+backward for every K of
+    --sweep-k, next to the K that the count statistics and the cost model
+    (activation_sparse_ffn_gemm_b200.kchoice) choose for training and inference."""
+    import torch
+
+    import activation_sparse_ffn_gemm_b200 as tw
+    from synthetic import gate_bias_for_activity
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    d, f, T_n, sigma = 4096, 14336, 128, 0.75
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    steps, warm = max(1, args.steps), max(3, args.warmup)
+    ks = [int(v) for v in args.sweep_k.split(",")]
+
+    def timed(body):
+        for _ in range(warm):
+            body()
+        torch.cuda.synchronize(dev)
+        tot = 0.0
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            body()
+            e1.record(stream)
+            e1.synchronize()
+            tot += e0.elapsed_time(e1)
+        return tot / steps
+
+    for sp in (float(v) for v in args.sweep_sparsity.split(",")):
+        bias = gate_bias_for_activity(1.0 - sp, "lognormal", sigma)
+        for M in (int(v) for v in args.sweep_m.split(",")):
+            X, W_g, W_u, W_d, dY, b_g, rs = _sweep_inputs(torch, dev, M, sp, d, f, sigma, bias)
+            Wdt = tw.transpose_wd(W_d)
+            Y = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
+            per_k, stats = {}, None
+            for K in ks:
+                st = tw.HybridState(M, f, T_n, K, M, dev, with_u=True)
+                wsf = tw.workspace(tw.OP_FWD, M, d, f, T_n, K, M, dev)
+                wsb = tw.workspace(tw.OP_BWD, M, d, f, T_n, K, M, dev)
+                grads = dict(dX=torch.empty((M, d), device=dev), dW_g=torch.empty((f, d), device=dev),
+                             dW_u=torch.empty((f, d), device=dev), dW_d=torch.empty((d, f), device=dev),
+                             db_g=torch.empty(f, device=dev))
+
+                def fwd():
+                    tw.ffn_fwd(X, W_g, b_g, W_u, W_d, T_n=T_n, K=K, W_dt=Wdt, state=st, ws=wsf, Y=Y)
+
+                def fwd_bwd():
+                    fwd()
+                    tw.ffn_bwd(X, W_g, W_u, W_d, st, dY, lam=args.lam, W_dt=Wdt, ws=wsb, out=grads)
+
+                t_fwd, t_fb = timed(fwd), timed(fwd_bwd)
+                assert st.read_status() == 0, "device status word set"
+                if stats is None:
+                    stats = {k: v.cpu().numpy() for k, v in tw.count_stats(st).items()}
+                per_k[K] = {"fwd_ms": t_fwd, "fwd_bwd_ms": t_fb, "overflow_rows": st.n_overflow()[1],
+                            "dense_wgrad_for_overflow_rows": int(st.row_plan[3].item())}
+                del st, wsf, wsb, grads
+            del X, W_g, W_u, W_d, dY, b_g, rs, Wdt, Y
+            torch.cuda.empty_cache()
+            k_train, m_train = tw.suggest_k(stats, d, f, T_n, ks, training=True)
+            k_inf, m_inf = tw.suggest_k(stats, d, f, T_n, ks, training=False)
+            print(json.dumps({
+                "point": {"M": M, "sparsity": sp, "d_model": d, "d_ff": f, "T_n": T_n},
+                "per_k": per_k,
+                "measured_best": {"fwd_bwd": min(per_k, key=lambda k: per_k[k]["fwd_bwd_ms"]),
+                                  "fwd": min(per_k, key=lambda k: per_k[k]["fwd_ms"])},
+                "suggested": {"fwd_bwd": k_train, "fwd": k_inf},
+                "modelled_ms": {"fwd_bwd": {k: v * 1e3 for k, v in m_train.items()},
+                                "fwd": {k: v * 1e3 for k, v in m_inf.items()}},
+                "steps": steps, "warmup": warm, "l2": "flushed before every timed step",
+                "data": "synthetic (seeded torch CUDA generator)"}), flush=True)
 
 
 def run_sweep(args, local):
@@ -642,15 +755,7 @@ def run_sweep(args, local):
         K = sweep_k(p, T_n)
         bias = gate_bias_for_activity(p, "lognormal", sigma)
         for M in (int(v) for v in args.sweep_m.split(",")):
-            g = torch.Generator(device=dev)
-            g.manual_seed(1000003 * M + int(round(sp * 1e4)))
-            rs = torch.exp(sigma * torch.randn(M, 1, device=dev, generator=g))
-            X = (torch.randn(M, d, device=dev, generator=g) * rs).to(torch.bfloat16)
-            W_g = (torch.randn(f, d, device=dev, generator=g) / math.sqrt(d)).to(torch.bfloat16)
-            W_u = (torch.randn(f, d, device=dev, generator=g) / math.sqrt(d)).to(torch.bfloat16)
-            W_d = (torch.randn(d, f, device=dev, generator=g) / math.sqrt(f)).to(torch.bfloat16)
-            dY = torch.randn(M, d, device=dev, generator=g).to(torch.bfloat16)
-            b_g = torch.full((f,), bias, device=dev).to(torch.bfloat16)
+            X, W_g, W_u, W_d, dY, b_g, rs = _sweep_inputs(torch, dev, M, sp, d, f, sigma, bias)
             st = tw.HybridState(M, f, T_n, K, M, dev, with_u=True)
             wsf = tw.workspace(tw.OP_FWD, M, d, f, T_n, K, M, dev)
             wsb = tw.workspace(tw.OP_BWD, M, d, f, T_n, K, M, dev)
@@ -721,7 +826,9 @@ def run_sweep(args, local):
 def main():
     args = parse_args()
     world, rank, local = dist_env()
-    if args.sweep:
+    if args.sweep and args.sweep_k:
+        run_ksweep(args, local)
+    elif args.sweep:
         run_sweep(args, local)
     elif args.impl == "reference":
         run_reference(args, world, rank)

@@ -239,6 +239,25 @@ TWELL_API twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, con
                            float* dW_g, float* dW_u, float* dW_d, float* db_g, void* ws,
                            size_t ws_bytes, twell_stream_t stream);
 
+/*
+ * Count statistics of a packed batch, for choosing the ELL width K of later
+ * batches ([aivizor] ¶4: in training the largest number of nonzeros per row
+ * can exceed the mean by a large factor). Read from h->count, which keeps the
+ * true per-tile counts 0..T_n. With bins c = 0..T_n:
+ *   rows_by_max[c]     rows whose largest tile count is c
+ *   act_by_max[c]      active units of those rows (summed over their tiles)
+ *   tiles_by_count[c]  (row, tile) pairs holding c active units
+ * Under row routing with width K the rows of bins c > K are the dense backup
+ * rows and the rest keep all their units in ELL slots; under tile routing the
+ * tiles of bins c > K are read from their spilled slices.
+ * The three outputs are caller-owned device int64 arrays of T_n + 1 entries
+ * (8-byte aligned), overwritten; asynchronous on `stream`. Integer sums: the
+ * same result on every run. Errors: TWELL_EINVAL (null or misaligned pointer),
+ * TWELL_EUNSUPPORTED (descriptor shape), TWELL_ECUDA (launch failure).
+ */
+TWELL_API twell_status twell_count_stats(const twell_hybrid* h, int64_t* rows_by_max, int64_t* act_by_max,
+                                         int64_t* tiles_by_count, twell_stream_t stream);
+
 /* Copies the device status word to *out after synchronizing `stream`; clears
  * it when `clear` is non-zero. Returns TWELL_ECUDA if the copy fails. */
 TWELL_API twell_status twell_status_read(const twell_hybrid* h, uint32_t* out, int clear, twell_stream_t stream);

@@ -8,6 +8,7 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
   bf16_round        pinned: torch's float32->bfloat16 RNE cast, hand-made ties
   gate              pinned: brute-force loops, torch float64 matmul
   pack / unpack     pinned: round trip, invariants, hand-built identity-gate case
+  count_stats       pinned: hand-counted bins, brute-force loops, sum invariants
   ffn_fwd           pinned: brute-force loops, torch float64, closed forms
   ffn_fwd_hybrid    pinned: equals ffn_fwd (round_g=1) on the same active set
   ffn_bwd           pinned: torch float64 autograd, closed form of the L1 term
@@ -150,6 +151,24 @@ def pack(Z, T_n: int, K: int, cap=None) -> dict:
     out["ovf_rows"] = out["ovf_rows"][:cap]
     out["g_ovf"] = out["g_ovf"][:cap]
     return out
+
+
+def count_stats(count, T_n: int) -> dict:
+    """Count statistics of a packed batch from its true per-tile counts [M, T]
+    (the definitions of twell_count_stats): rows binned by their largest tile
+    count, those rows' active units summed in the same bins, and (row, tile)
+    pairs binned by count; T_n + 1 bins each."""
+    c = np.asarray(count).astype(np.int64)
+    if c.ndim != 2 or (c.size and (c.min() < 0 or c.max() > T_n)):
+        raise ValueError("count must be [M, T] with entries in [0, T_n]")
+    M = c.shape[0]
+    mx = c.max(axis=1) if c.shape[1] else np.zeros(M, np.int64)
+    act = c.sum(axis=1)
+    act_by_max = np.zeros(T_n + 1, np.int64)
+    np.add.at(act_by_max, mx, act)
+    return {"rows_by_max": np.bincount(mx, minlength=T_n + 1).astype(np.int64),
+            "act_by_max": act_by_max,
+            "tiles_by_count": np.bincount(c.ravel(), minlength=T_n + 1).astype(np.int64)}
 
 
 def unpack(p: dict, f: int, T_n: int, K: int) -> np.ndarray:

@@ -264,6 +264,33 @@ def test_train_full_size(tw, orc):
         _check_bwd(orc, inp, g, G, lam, "train")
 
 
+@pytest.mark.parametrize("name", ["tiny", "ragged", "heavy_small", "one_row", "k64"])
+def test_count_stats(tw, orc, name):
+    """twell_count_stats bit-exact against the oracle's statistics of its own pack
+    of the GPU's z; the rows above K are the routed overflow rows, the actives
+    of the other rows are the plan's kept total; the K choice runs on them."""
+    M, d, f, K, act, rs, seed = CASES[name]
+    w = Workload(name, M, d, f, 128, K, act, row_scale=rs, training=True, seed=seed)
+    inp = make_inputs(w)
+    D, Y, st, z = _run_fwd(tw, inp, w)
+    gs = {k: v.cpu().numpy() for k, v in tw.count_stats(st).items()}
+    p_ref = orc.pack(z.cpu().numpy().astype(np.float64), 128, K)
+    ref = orc.count_stats(p_ref["count"], 128)
+    for k in ref:
+        assert np.array_equal(gs[k], ref[k]), k
+    assert gs["rows_by_max"][K + 1:].sum() == st.n_overflow()[1]
+    assert gs["act_by_max"][:K + 1].sum() == int(st.row_plan[2].item())
+    best, times = tw.suggest_k(gs, d, f)
+    assert best in times and len(times) == 4
+
+
+def test_count_stats_empty_batch(tw):
+    st = tw.HybridState(0, 256, 128, 8, 0, "cuda")
+    out = tw.count_stats(st)
+    torch.cuda.synchronize()
+    assert all(v.shape == (129,) and int(v.abs().sum().item()) == 0 for v in out.values())
+
+
 @pytest.mark.parametrize("M,activity,bwd", [(2048, 0.1, False), (512, 0.001, False), (64, 0.1, True),
                                               (96, 0.05, True)])
 def test_sweep_points(tw, orc, M, activity, bwd):

@@ -1,0 +1,83 @@
+"""Host logic of the ELL-width choice (activation_sparse_ffn_gemm_b200.kchoice):
+the modelled time of each candidate K against values worked out by hand."""
+
+import numpy as np
+import pytest
+
+from activation_sparse_ffn_gemm_b200.kchoice import CostModel, modelled_times, suggest_k
+
+T_n = 128
+
+
+def _stats(rows_by_max, act_by_max, tiles_by_count):
+    out = {}
+    for k, v in (("rows_by_max", rows_by_max), ("act_by_max", act_by_max), ("tiles_by_count", tiles_by_count)):
+        a = np.zeros(T_n + 1, np.int64)
+        for c, n in v.items():
+            a[c] = n
+        out[k] = a
+    return out
+
+
+# unit coefficients, so each term can be read off: pair = 1 s per d element,
+# dense row = 10 s per d*f element, 1 byte/s
+UNIT = CostModel(pair_fwd_s=1.0, pair_bwd_s=0.0, dense_fwd_s=10.0, dense_bwd_s=0.0, hbm_bytes_s=1.0)
+
+
+def test_row_routing_terms_by_hand():
+    # 3 rows with largest count 5 (30 actives), 1 row with 20 (40 actives); T = 2 tiles
+    st = _stats({5: 3, 20: 1}, {5: 30, 20: 40}, {5: 3, 3: 3, 20: 1, 1: 1})
+    t = modelled_times(st, d_model=2, d_ff=256, candidates=(8, 32), training=False, model=UNIT)
+    M, T = 4, 2
+    # K=8: 30 pairs sparse, 1 row dense; K=32: all 70 pairs sparse, no dense row
+    assert t[8] == 1.0 * 2 * 30 + 10.0 * 2 * 256 * 1 + M * T * (2 + 3 * 8)
+    assert t[32] == 1.0 * 2 * 70 + M * T * (2 + 3 * 32)
+    best, times = suggest_k(st, d_model=2, d_ff=256, candidates=(8, 32), training=False, model=UNIT)
+    assert best == 32 and times == t
+
+
+def test_tile_routing_terms_by_hand():
+    st = _stats({5: 3, 20: 1}, {5: 30, 20: 40}, {5: 3, 3: 3, 20: 1, 1: 1})
+    t = modelled_times(st, d_model=2, d_ff=256, candidates=(4, 8), training=False, routing="tiles", model=UNIT)
+    # every active unit gathered; spilled tiles: count > 4 -> 4 tiles (three 5s, one 20); > 8 -> 1
+    assert t[4] == 1.0 * 2 * 70 + 4 * 2 * (2 + 3 * 4) + 512 * 4
+    assert t[8] == 1.0 * 2 * 70 + 4 * 2 * (2 + 3 * 8) + 512 * 1
+    with pytest.raises(ValueError):
+        modelled_times(st, 2, 256, training=True, routing="tiles")
+
+
+def test_training_adds_backward_terms():
+    st = _stats({10: 2}, {10: 12}, {10: 2, 1: 2})
+    m = CostModel(pair_fwd_s=1.0, pair_bwd_s=2.0, dense_fwd_s=4.0, dense_bwd_s=5.0, hbm_bytes_s=1e30)
+    t_inf = modelled_times(st, 1, 256, candidates=(8, 16), training=False, model=m)
+    t_trn = modelled_times(st, 1, 256, candidates=(8, 16), training=True, model=m)
+    assert t_inf[8] == pytest.approx(4.0 * 256 * 2) and t_trn[8] == pytest.approx(9.0 * 256 * 2)
+    assert t_inf[16] == pytest.approx(1.0 * 12) and t_trn[16] == pytest.approx(3.0 * 12)
+
+
+def test_no_overflow_prefers_smallest_k_and_ties_go_small():
+    st = _stats({3: 100}, {3: 500}, {3: 100, 0: 100})
+    best, times = suggest_k(st, 2048, 256)
+    assert best == 8 and times[8] < times[16] < times[32] < times[64]
+    free = CostModel(pair_fwd_s=0.0, pair_bwd_s=0.0, dense_fwd_s=0.0, dense_bwd_s=0.0, hbm_bytes_s=1e300)
+    assert suggest_k(st, 2048, 256, model=free)[0] == 8
+
+
+def test_heavy_rows_trade_slots_for_dense_rows():
+    """Rows with many actives go dense at a small K when a dense row is cheap next
+    to their gathers, and stay sparse at a large K when it is not."""
+    st = _stats({4: 1000, 40: 10}, {4: 3000, 40: 10 * 2000}, {4: 1000, 40: 10, 0: 1010 * 111})
+    d, f = 4096, 14336
+    cheap_dense = CostModel(pair_fwd_s=1e-12, pair_bwd_s=0.0, dense_fwd_s=1e-17, dense_bwd_s=0.0)
+    dear_dense = CostModel(pair_fwd_s=1e-12, pair_bwd_s=0.0, dense_fwd_s=1e-12, dense_bwd_s=0.0)
+    assert suggest_k(st, d, f, training=False, model=cheap_dense)[0] == 8
+    assert suggest_k(st, d, f, training=False, model=dear_dense)[0] == 64
+
+
+def test_rejects_bad_statistics():
+    st = _stats({3: 1}, {3: 3}, {3: 1})
+    st["rows_by_max"] = st["rows_by_max"][:-1]
+    with pytest.raises(ValueError):
+        suggest_k(st, 64, 128)
+    with pytest.raises(ValueError):
+        modelled_times(_stats({3: 1}, {3: 3}, {3: 1}), 64, 128, candidates=(0,))

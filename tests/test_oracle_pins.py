@@ -361,3 +361,56 @@ def test_gmat_input_equals_stored_g_definition(orc):
     assert np.abs(y2[i] - y1[i] - delta).max() < 1e-12
     rows = np.array([3, 0], np.int32)
     assert np.array_equal(orc.ffn_fwd(X, Wg, bg, Wu, Wd, rows=rows, gmat=G[rows]), y1[rows])
+
+
+def test_count_stats_hand_counted(orc):
+    """Bins counted by hand for a 3-row, 2-tile batch with T_n = 4."""
+    count = np.array([[1, 3], [0, 0], [4, 2]], dtype=np.uint16)
+    st = orc.count_stats(count, 4)
+    # largest tile counts 3, 0, 4; row sums 4, 0, 6; tile counts 1, 3, 0, 0, 4, 2
+    assert st["rows_by_max"].tolist() == [1, 0, 0, 1, 1]
+    assert st["act_by_max"].tolist() == [0, 0, 0, 4, 6]
+    assert st["tiles_by_count"].tolist() == [2, 1, 1, 1, 1]
+    empty = orc.count_stats(np.zeros((0, 5), np.uint16), 128)
+    assert all(v.shape == (129,) and not v.any() for v in empty.values())
+    with pytest.raises(ValueError):
+        orc.count_stats(np.array([[5]], np.uint16), 4)
+
+
+def test_count_stats_brute_force_and_sums(orc):
+    """Plain loops over rows and tiles on random counts, plus the sum identities
+    (rows, actives and tiles are each counted once) and the link to routing:
+    the rows of bins above K are exactly the rows the oracle's pack routes to
+    the dense backup."""
+    rng = np.random.default_rng(11)
+    M, T, T_n = 57, 6, 128
+    count = np.minimum(rng.geometric(0.3, size=(M, T)) - 1 + (rng.random((M, T)) < 0.05) * 40, T_n).astype(np.uint16)
+    st = orc.count_stats(count, T_n)
+    rows = [0] * (T_n + 1)
+    act = [0] * (T_n + 1)
+    tiles = [0] * (T_n + 1)
+    for i in range(M):
+        m = 0
+        s = 0
+        for t in range(T):
+            c = int(count[i, t])
+            tiles[c] += 1
+            m = max(m, c)
+            s += c
+        rows[m] += 1
+        act[m] += s
+    assert st["rows_by_max"].tolist() == rows
+    assert st["act_by_max"].tolist() == act
+    assert st["tiles_by_count"].tolist() == tiles
+    assert st["rows_by_max"].sum() == M and st["tiles_by_count"].sum() == M * T
+    assert st["act_by_max"].sum() == count.astype(np.int64).sum()
+    assert (np.arange(T_n + 1) * st["tiles_by_count"]).sum() == count.astype(np.int64).sum()
+    # a dense Z whose tile counts are `count`: the first c columns of each tile positive
+    Z = -np.ones((M, T * T_n))
+    for i in range(M):
+        for t in range(T):
+            Z[i, t * T_n:t * T_n + int(count[i, t])] = 1.0
+    for K in (8, 16, 32):
+        p = orc.pack(Z, T_n, K)
+        assert np.array_equal(p["count"], count)
+        assert p["n_ovf_total"] == st["rows_by_max"][K + 1:].sum()
