@@ -66,7 +66,7 @@ def lib():
             L.oracle_gate.restype = ctypes.c_int
             L.oracle_gate.argtypes = [_u16p, _u16p, _u16p, _i64, _i64, _i64, _vp, _i64, _f64p]
             L.oracle_pack.restype = ctypes.c_int
-            L.oracle_pack.argtypes = [_f64p, _i64, _i64, _i32, _i32, _i64, _u16p, _u16p, _u8p, _u8p,
+            L.oracle_pack.argtypes = [_f64p, _i64, _i64, _i32, _i32, _i64, _i64, _u16p, _u16p, _u8p, _u8p,
                                       _i32p, ctypes.POINTER(ctypes.c_int64), _u16p]
             L.oracle_unpack.argtypes = [_u16p, _u16p, _u8p, _u8p, _i32p, _i64, _u16p, _i64, _i64, _i32,
                                         _i32, _u16p]
@@ -127,8 +127,9 @@ def gate(X, W_g, b_g, rows=None) -> np.ndarray:
     return Z
 
 
-def pack(Z, T_n: int, K: int, cap=None) -> dict:
-    """TwELL + hybrid routing of a dense float64 Z [M, f]."""
+def pack(Z, T_n: int, K: int, cap=None, dense_min: int = 0) -> dict:
+    """TwELL + hybrid routing of a dense float64 Z [M, f]; with dense_min > 0 a
+    row with at least that many active units is also routed to the dense backup."""
     Z = _c(Z, np.float64)
     M, f = Z.shape
     if f % T_n or not (1 <= T_n <= 256) or K < 1:
@@ -141,7 +142,7 @@ def pack(Z, T_n: int, K: int, cap=None) -> dict:
         ovf_rows=np.zeros(max(cap, 1), np.int32), g_ovf=np.zeros((max(cap, 1), f), np.uint16),
     )
     n = ctypes.c_int64(0)
-    rc = lib().oracle_pack(Z, M, f, T_n, K, cap, out["count"], out["val"], out["col"], out["row_ovf"],
+    rc = lib().oracle_pack(Z, M, f, T_n, K, cap, int(dense_min), out["count"], out["val"], out["col"], out["row_ovf"],
                            out["ovf_rows"], ctypes.byref(n), out["g_ovf"])
     if rc == 1:
         raise ValueError("oracle_pack rejected the shape")
@@ -153,22 +154,26 @@ def pack(Z, T_n: int, K: int, cap=None) -> dict:
     return out
 
 
-def count_stats(count, T_n: int) -> dict:
+def count_stats(count, T_n: int, dense_min: int = 0) -> dict:
     """Count statistics of a packed batch from its true per-tile counts [M, T]
-    (the definitions of twell_count_stats): rows binned by their largest tile
-    count, those rows' active units summed in the same bins, and (row, tile)
-    pairs binned by count; T_n + 1 bins each."""
+    (the definitions of twell_count_stats), T_n + 2 bins each: rows binned by
+    their largest tile count c (bin c), and those rows' active units summed in
+    the same bins, except that with dense_min > 0 a row with at least dense_min
+    active units goes to bin T_n + 1; (row, tile) pairs binned by count (bin
+    T_n + 1 stays empty)."""
     c = np.asarray(count).astype(np.int64)
     if c.ndim != 2 or (c.size and (c.min() < 0 or c.max() > T_n)):
         raise ValueError("count must be [M, T] with entries in [0, T_n]")
     M = c.shape[0]
-    mx = c.max(axis=1) if c.shape[1] else np.zeros(M, np.int64)
     act = c.sum(axis=1)
-    act_by_max = np.zeros(T_n + 1, np.int64)
-    np.add.at(act_by_max, mx, act)
-    return {"rows_by_max": np.bincount(mx, minlength=T_n + 1).astype(np.int64),
+    b = c.max(axis=1) if c.shape[1] else np.zeros(M, np.int64)
+    if dense_min > 0:
+        b = np.where(act >= dense_min, T_n + 1, b)
+    act_by_max = np.zeros(T_n + 2, np.int64)
+    np.add.at(act_by_max, b, act)
+    return {"rows_by_max": np.bincount(b, minlength=T_n + 2).astype(np.int64),
             "act_by_max": act_by_max,
-            "tiles_by_count": np.bincount(c.ravel(), minlength=T_n + 1).astype(np.int64)}
+            "tiles_by_count": np.bincount(c.ravel(), minlength=T_n + 2).astype(np.int64)}
 
 
 def unpack(p: dict, f: int, T_n: int, K: int) -> np.ndarray:

@@ -183,14 +183,16 @@ int oracle_gate(const uint16_t* X, const uint16_t* Wg, const uint16_t* bg, int64
  *   count[i,t] = #{c : Z[i, t*T_n + c] > 0}
  *   the first min(count, K) active c in ascending order fill slots 0.. with
  *   val = bf16(Z), col = c; the remaining slots are (0, 0).
- * Row i overflows (row_ovf[i] = 1) when some tile has count > K. Overflow rows
+ * Row i overflows (row_ovf[i] = 1) when some tile has count > K, or, with
+ * dense_min > 0, when its active units (the sum of its counts) number at least
+ * dense_min (rows whose gathers cost more than a dense row). Overflow rows
  * are listed in ascending order in ovf_rows; the first `cap` of them get a dense
  * row g_ovf[s, :] = bf16(ReLU(Z[i, :])) (bits 0 where Z <= 0).
  * *n_ovf_total receives the number of overflow rows. Returns 0, 3 when that
  * number exceeds cap (rows beyond cap are counted but not stored), or 1 when
  * the shape is not packable (in-tile columns are bytes, so 1 <= T_n <= 256,
  * and d_ff must be a whole number of tiles). */
-int oracle_pack(const double* Z, int64_t M, int64_t f, int32_t T_n, int32_t K, int64_t cap,
+int oracle_pack(const double* Z, int64_t M, int64_t f, int32_t T_n, int32_t K, int64_t cap, int64_t dense_min,
                 uint16_t* count, uint16_t* val, uint8_t* col, uint8_t* row_ovf, int32_t* ovf_rows,
                 int64_t* n_ovf_total, uint16_t* g_ovf) {
   if (T_n < 1 || T_n > 256 || K < 1 || f % T_n != 0) return 1;
@@ -198,6 +200,7 @@ int oracle_pack(const double* Z, int64_t M, int64_t f, int32_t T_n, int32_t K, i
   int64_t n = 0;
   for (int64_t i = 0; i < M; ++i) {
     int ovf = 0;
+    int64_t active = 0;
     for (int64_t t = 0; t < T; ++t) {
       const double* z = Z + i * f + t * T_n;
       uint16_t* v = val + (i * T + t) * K;
@@ -212,7 +215,9 @@ int oracle_pack(const double* Z, int64_t M, int64_t f, int32_t T_n, int32_t K, i
       }
       count[i * T + t] = (uint16_t)cnt;
       if (cnt > K) ovf = 1;
+      active += cnt;
     }
+    if (dense_min > 0 && active >= dense_min) ovf = 1;
     row_ovf[i] = (uint8_t)ovf;
     if (ovf) {
       if (n < cap) {

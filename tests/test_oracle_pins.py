@@ -189,6 +189,15 @@ def test_pack_roundtrip_and_invariants(orc, T_n, K):
     assert p["n_ovf"] == rows.size and np.array_equal(p["ovf_rows"][: rows.size], rows)
     if K >= T_n:
         assert p["n_ovf"] == 0
+    # with a row threshold, rows of many actives also go dense; same round trip
+    dm = int(np.median(cnt.sum(1))) + 1
+    q = orc.pack(Z, T_n, K, dense_min=dm)
+    want = (cnt > K).any(1) | (cnt.sum(1) >= dm)
+    assert np.array_equal(q["row_ovf"].astype(bool), want) and want.sum() > (cnt > K).any(1).sum() - 1
+    assert np.array_equal(q["ovf_rows"][:q["n_ovf"]], np.nonzero(want)[0])
+    assert np.array_equal(orc.unpack(q, f, T_n, K), G)
+    for k in ("count", "val", "col"):
+        assert np.array_equal(q[k], p[k])
 
 
 def test_pack_single_tile_is_row_ellpack(orc):
@@ -368,11 +377,16 @@ def test_count_stats_hand_counted(orc):
     count = np.array([[1, 3], [0, 0], [4, 2]], dtype=np.uint16)
     st = orc.count_stats(count, 4)
     # largest tile counts 3, 0, 4; row sums 4, 0, 6; tile counts 1, 3, 0, 0, 4, 2
-    assert st["rows_by_max"].tolist() == [1, 0, 0, 1, 1]
-    assert st["act_by_max"].tolist() == [0, 0, 0, 4, 6]
-    assert st["tiles_by_count"].tolist() == [2, 1, 1, 1, 1]
+    assert st["rows_by_max"].tolist() == [1, 0, 0, 1, 1, 0]
+    assert st["act_by_max"].tolist() == [0, 0, 0, 4, 6, 0]
+    assert st["tiles_by_count"].tolist() == [2, 1, 1, 1, 1, 0]
+    # rows with at least 5 active units (the third, 6) go to the last bin
+    st = orc.count_stats(count, 4, dense_min=5)
+    assert st["rows_by_max"].tolist() == [1, 0, 0, 1, 0, 1]
+    assert st["act_by_max"].tolist() == [0, 0, 0, 4, 0, 6]
+    assert st["tiles_by_count"].tolist() == [2, 1, 1, 1, 1, 0]
     empty = orc.count_stats(np.zeros((0, 5), np.uint16), 128)
-    assert all(v.shape == (129,) and not v.any() for v in empty.values())
+    assert all(v.shape == (130,) and not v.any() for v in empty.values())
     with pytest.raises(ValueError):
         orc.count_stats(np.array([[5]], np.uint16), 4)
 
@@ -385,32 +399,41 @@ def test_count_stats_brute_force_and_sums(orc):
     rng = np.random.default_rng(11)
     M, T, T_n = 57, 6, 128
     count = np.minimum(rng.geometric(0.3, size=(M, T)) - 1 + (rng.random((M, T)) < 0.05) * 40, T_n).astype(np.uint16)
-    st = orc.count_stats(count, T_n)
-    rows = [0] * (T_n + 1)
-    act = [0] * (T_n + 1)
-    tiles = [0] * (T_n + 1)
-    for i in range(M):
-        m = 0
-        s = 0
-        for t in range(T):
-            c = int(count[i, t])
-            tiles[c] += 1
-            m = max(m, c)
-            s += c
-        rows[m] += 1
-        act[m] += s
-    assert st["rows_by_max"].tolist() == rows
-    assert st["act_by_max"].tolist() == act
-    assert st["tiles_by_count"].tolist() == tiles
-    assert st["rows_by_max"].sum() == M and st["tiles_by_count"].sum() == M * T
-    assert st["act_by_max"].sum() == count.astype(np.int64).sum()
-    assert (np.arange(T_n + 1) * st["tiles_by_count"]).sum() == count.astype(np.int64).sum()
+    for dense_min in (0, 40):
+        st = orc.count_stats(count, T_n, dense_min)
+        rows = [0] * (T_n + 2)
+        act = [0] * (T_n + 2)
+        tiles = [0] * (T_n + 2)
+        for i in range(M):
+            m = 0
+            s = 0
+            for t in range(T):
+                c = int(count[i, t])
+                tiles[c] += 1
+                m = max(m, c)
+                s += c
+            if dense_min and s >= dense_min:
+                m = T_n + 1
+            rows[m] += 1
+            act[m] += s
+        assert st["rows_by_max"].tolist() == rows
+        assert st["act_by_max"].tolist() == act
+        assert st["tiles_by_count"].tolist() == tiles
+        assert st["rows_by_max"].sum() == M and st["tiles_by_count"].sum() == M * T
+        assert st["act_by_max"].sum() == count.astype(np.int64).sum()
+        assert (np.arange(T_n + 2) * st["tiles_by_count"]).sum() == count.astype(np.int64).sum()
+    assert 0 < st["rows_by_max"][T_n + 1] < M  # the threshold splits this batch
     # a dense Z whose tile counts are `count`: the first c columns of each tile positive
     Z = -np.ones((M, T * T_n))
     for i in range(M):
         for t in range(T):
             Z[i, t * T_n:t * T_n + int(count[i, t])] = 1.0
     for K in (8, 16, 32):
-        p = orc.pack(Z, T_n, K)
-        assert np.array_equal(p["count"], count)
-        assert p["n_ovf_total"] == st["rows_by_max"][K + 1:].sum()
+        for dense_min in (0, 40):
+            st = orc.count_stats(count, T_n, dense_min)
+            p = orc.pack(Z, T_n, K, dense_min=dense_min)
+            assert np.array_equal(p["count"], count)
+            assert p["n_ovf_total"] == st["rows_by_max"][K + 1:].sum()
+            flagged = (count.max(axis=1) > K) | ((count.astype(np.int64).sum(axis=1) >= dense_min) & (dense_min > 0))
+            assert np.array_equal(p["row_ovf"].astype(bool), flagged)
+            assert np.array_equal(p["ovf_rows"][:p["n_ovf"]], np.flatnonzero(flagged))
