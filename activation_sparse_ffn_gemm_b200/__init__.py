@@ -18,7 +18,7 @@ from typing import Optional
 
 import torch
 
-from .kchoice import CostModel, modelled_times, suggest_k  # noqa: F401
+from .kchoice import CostModel, dense_min_for, modelled_times, suggest_k  # noqa: F401
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libtwell.so")
@@ -48,9 +48,9 @@ class TwellHybrid(ctypes.Structure):
     """Mirror of struct twell_hybrid."""
 
     _fields_ = [("M", ctypes.c_int32), ("d_ff", ctypes.c_int32), ("T_n", ctypes.c_int32), ("K", ctypes.c_int32),
-                ("ovf_cap", ctypes.c_int32), ("count", _vp), ("val", _vp), ("col", _vp), ("row_ovf", _vp),
-                ("ovf_rows", _vp), ("n_ovf", _vp), ("g_ovf", _vp), ("u_ell", _vp), ("u_ovf", _vp),
-                ("status", _vp), ("row_plan", _vp)]
+                ("ovf_cap", ctypes.c_int32), ("dense_min", ctypes.c_int32), ("count", _vp), ("val", _vp),
+                ("col", _vp), ("row_ovf", _vp), ("ovf_rows", _vp), ("n_ovf", _vp), ("g_ovf", _vp), ("u_ell", _vp),
+                ("u_ovf", _vp), ("status", _vp), ("row_plan", _vp)]
 
 
 _lock = threading.Lock()
@@ -158,12 +158,14 @@ class HybridState:
     """Device buffers of one hybrid TwELL representation (see struct twell_hybrid)."""
 
     def __init__(self, M: int, d_ff: int, T_n: int = 128, K: int = 8, ovf_cap: Optional[int] = None,
-                 device=None, with_u: bool = True):
+                 device=None, with_u: bool = True, dense_min: int = 0):
+        """dense_min > 0 also routes rows with at least that many active units to
+        the dense backup (kchoice.dense_min_for gives the measured break-even)."""
         dev = torch.device(device or "cuda")
         T = d_ff // T_n
         cap = M if ovf_cap is None else int(ovf_cap)
         cap1 = max(cap, 1)
-        self.M, self.d_ff, self.T_n, self.K, self.ovf_cap = M, d_ff, T_n, K, cap
+        self.M, self.d_ff, self.T_n, self.K, self.ovf_cap, self.dense_min = M, d_ff, T_n, K, cap, int(dense_min)
         self.count = torch.empty((M, T), dtype=torch.int16, device=dev)
         self.val = torch.empty((M, T, K), dtype=torch.bfloat16, device=dev)
         self.col = torch.empty((M, T, K), dtype=torch.uint8, device=dev)
@@ -176,7 +178,7 @@ class HybridState:
         self.status = torch.zeros(4, dtype=torch.int32, device=dev)
         self.row_plan = torch.zeros(max(int(lib().twell_plan_ints(M, d_ff, T_n, K)), 1), dtype=torch.int32,
                                     device=dev)
-        self.c = TwellHybrid(M, d_ff, T_n, K, cap, *(
+        self.c = TwellHybrid(M, d_ff, T_n, K, cap, int(dense_min), *(
             (t.data_ptr() if t is not None else None) for t in
             (self.count, self.val, self.col, self.row_ovf, self.ovf_rows, self.n_ovf, self.g_ovf, self.u_ell,
              self.u_ovf, self.status, self.row_plan)))
@@ -194,8 +196,9 @@ class HybridState:
 
 def count_stats(state: HybridState, stream=None) -> dict:
     """Count statistics of a packed batch (twell_count_stats): int64 CUDA tensors
-    rows_by_max, act_by_max, tiles_by_count of T_n + 1 bins each."""
-    n = state.T_n + 1
+    rows_by_max, act_by_max, tiles_by_count of T_n + 2 bins each (bin T_n + 1:
+    rows routed dense by the state's dense_min)."""
+    n = state.T_n + 2
     dev = state.count.device
     out = {k: torch.empty(n, dtype=torch.int64, device=dev) for k in ("rows_by_max", "act_by_max", "tiles_by_count")}
     _check(lib().twell_count_stats(ctypes.byref(state.c), _ptr(out["rows_by_max"]), _ptr(out["act_by_max"]),
@@ -212,13 +215,13 @@ def transpose_wd(W_d: torch.Tensor, out: Optional[torch.Tensor] = None, stream=N
 
 
 def pack(X, W_g, b_g, T_n: int = 128, K: int = 8, ovf_cap: Optional[int] = None, z_debug: bool = False,
-         state: Optional[HybridState] = None, ws: Optional[torch.Tensor] = None, stream=None):
+         state: Optional[HybridState] = None, ws: Optional[torch.Tensor] = None, stream=None, dense_min: int = 0):
     """Gate GEMM + TwELL pack + row routing. Returns (state, z or None)."""
     for t, n in ((X, "X"), (W_g, "W_g"), (b_g, "b_g")):
         _bf16(t, n)
     M, d = X.shape
     f = W_g.shape[0]
-    st = state or HybridState(M, f, T_n, K, ovf_cap, X.device, with_u=False)
+    st = state or HybridState(M, f, T_n, K, ovf_cap, X.device, with_u=False, dense_min=dense_min)
     z = torch.empty((M, f), dtype=torch.float32, device=X.device) if z_debug else None
     if ws is None:
         ws = workspace(OP_PACK, M, d, f, T_n, K, st.ovf_cap, X.device)
@@ -231,7 +234,7 @@ NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def pack_noalloc(X, W_g, b_g, T_n: int = 128, K: int = 8, ovf_cap: Optional[int] = None, z_debug: bool = False,
-                 state: Optional[HybridState] = None, stream=None):
+                 state: Optional[HybridState] = None, stream=None, dense_min: int = 0):
     """twell_pack_noalloc: the same result as pack() without a workspace; the
     library's own fixed scratch is used instead (M * d_ff * 2 bytes at most
     NOALLOC_SCRATCH_BYTES). Returns (state, z or None)."""
@@ -239,7 +242,7 @@ def pack_noalloc(X, W_g, b_g, T_n: int = 128, K: int = 8, ovf_cap: Optional[int]
         _bf16(t, n)
     M, d = X.shape
     f = W_g.shape[0]
-    st = state or HybridState(M, f, T_n, K, ovf_cap, X.device, with_u=False)
+    st = state or HybridState(M, f, T_n, K, ovf_cap, X.device, with_u=False, dense_min=dense_min)
     z = torch.empty((M, f), dtype=torch.float32, device=X.device) if z_debug else None
     _check(lib().twell_pack_noalloc(_ptr(X), _ptr(W_g), _ptr(b_g), d, ctypes.byref(st.c), _ptr(z), _stream(stream)),
            "twell_pack_noalloc")
@@ -249,16 +252,18 @@ def pack_noalloc(X, W_g, b_g, T_n: int = 128, K: int = 8, ovf_cap: Optional[int]
 def ffn_fwd(X, W_g, b_g, W_u, W_d, T_n: int = 128, K: int = 8, ovf_cap: Optional[int] = None, W_dt=None,
             save_for_backward: bool = True, z_debug: bool = False, state: Optional[HybridState] = None,
             ws: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None, stream=None,
-            tile_routing: bool = False):
+            tile_routing: bool = False, dense_min: int = 0):
     """Sparse gated FFN forward. Returns (Y, state) or (Y, state, z) with z_debug.
 
     tile_routing: per-(row, tile) overflow routing (twell_ffn_fwd_tiles), an
-    inference-only state; otherwise the row-level hybrid (twell_ffn_fwd)."""
+    inference-only state; otherwise the row-level hybrid (twell_ffn_fwd).
+    dense_min: for a state made here, rows with at least this many active
+    units also go to the dense backup (0: only rows with a tile over K)."""
     for t, n in ((X, "X"), (W_g, "W_g"), (b_g, "b_g"), (W_u, "W_u"), (W_d, "W_d")):
         _bf16(t, n)
     M, d = X.shape
     f = W_g.shape[0]
-    st = state or HybridState(M, f, T_n, K, ovf_cap, X.device, with_u=save_for_backward)
+    st = state or HybridState(M, f, T_n, K, ovf_cap, X.device, with_u=save_for_backward, dense_min=dense_min)
     Y = torch.empty((M, d), dtype=torch.bfloat16, device=X.device) if Y is None else Y
     z = torch.empty((M, f), dtype=torch.float32, device=X.device) if z_debug else None
     if ws is None:

@@ -5,14 +5,15 @@
 // to the dense backup).
 //
 // From the true per-tile counts (0..T_n, kept even when a tile holds more than
-// K), with bins c = 0..T_n:
-//   rows_by_max[c]    rows whose largest tile count is c
-//   act_by_max[c]     active units of those rows
-//   tiles_by_count[c] (row, tile) pairs holding c active units
-// Under row routing with width K, the rows with largest count > K are the
-// dense backup rows and the others keep all their units in ELL slots; under
-// tile routing, tiles with count > K are read from their spilled slices. The
-// sums are of integers, so the result is the same on every run.
+// K), with bins c = 0..T_n + 1:
+//   rows_by_max[c]    rows whose largest tile count is c; a row with at least
+//                     dense_min active units (dense_min > 0) goes to bin T_n + 1
+//   act_by_max[c]     active units of the rows of bin c
+//   tiles_by_count[c] (row, tile) pairs holding c active units (bin T_n + 1 empty)
+// Under row routing with width K, the rows of bins c > K are the dense backup
+// rows and the others keep all their units in ELL slots; under tile routing,
+// tiles with count > K are read from their spilled slices. The sums are of
+// integers, so the result is the same on every run.
 #include "count_stats.cuh"
 #include "trace.cuh"
 #include "twell_internal.cuh"
@@ -21,11 +22,12 @@ namespace twell {
 
 namespace {
 
-constexpr int kBins = kTn + 1;
+constexpr int kBins = kTn + 2;
 
 // One warp per row (grid-stride), lanes over the row's tiles. Equal tile
 // counts within a warp are merged with a match before the shared-memory add.
 __global__ void __launch_bounds__(256) count_stats_kernel(const uint16_t* __restrict__ count, int M, int T,
+                                                          int dense_min,
                                                           unsigned long long* __restrict__ rows_by_max,
                                                           unsigned long long* __restrict__ act_by_max,
                                                           unsigned long long* __restrict__ tiles_by_count) {
@@ -53,9 +55,10 @@ __global__ void __launch_bounds__(256) count_stats_kernel(const uint16_t* __rest
       mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
       sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
     }
+    const int bin = dense_min > 0 && sum >= dense_min ? kTn + 1 : mx;
     if (lane == 0) {
-      atomicAdd(&s_rows[mx], 1ull);
-      atomicAdd(&s_act[mx], static_cast<unsigned long long>(sum));
+      atomicAdd(&s_rows[bin], 1ull);
+      atomicAdd(&s_act[bin], static_cast<unsigned long long>(sum));
     }
   }
   __syncthreads();
@@ -68,8 +71,8 @@ __global__ void __launch_bounds__(256) count_stats_kernel(const uint16_t* __rest
 
 }  // namespace
 
-cudaError_t launch_count_stats(const uint16_t* count, int M, int T, int64_t* rows_by_max, int64_t* act_by_max,
-                               int64_t* tiles_by_count, cudaStream_t s) {
+cudaError_t launch_count_stats(const uint16_t* count, int M, int T, int dense_min, int64_t* rows_by_max,
+                               int64_t* act_by_max, int64_t* tiles_by_count, cudaStream_t s) {
   const size_t bytes = sizeof(int64_t) * kBins;
   cudaError_t e = cudaMemsetAsync(rows_by_max, 0, bytes, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(act_by_max, 0, bytes, s);
@@ -79,7 +82,7 @@ cudaError_t launch_count_stats(const uint16_t* count, int M, int T, int64_t* row
   const int max_blocks = device_sm_count() * 8;
   if (blocks > max_blocks) blocks = max_blocks;
   TWELL_LAUNCH("count_stats", s,
-               count_stats_kernel<<<blocks, 256, 0, s>>>(count, M, T,
+               count_stats_kernel<<<blocks, 256, 0, s>>>(count, M, T, dense_min,
                                                          reinterpret_cast<unsigned long long*>(rows_by_max),
                                                          reinterpret_cast<unsigned long long*>(act_by_max),
                                                          reinterpret_cast<unsigned long long*>(tiles_by_count)));

@@ -6,9 +6,9 @@
 
 namespace twell {
 
-// rows_by_max, act_by_max, tiles_by_count: device arrays of kTn + 1 int64
+// rows_by_max, act_by_max, tiles_by_count: device arrays of kTn + 2 int64
 // entries each, overwritten (see twell_count_stats in include/twell.h).
-cudaError_t launch_count_stats(const uint16_t* count, int M, int T, int64_t* rows_by_max, int64_t* act_by_max,
-                               int64_t* tiles_by_count, cudaStream_t s);
+cudaError_t launch_count_stats(const uint16_t* count, int M, int T, int dense_min, int64_t* rows_by_max,
+                               int64_t* act_by_max, int64_t* tiles_by_count, cudaStream_t s);
 
 }  // namespace twell

@@ -17,11 +17,12 @@ namespace {
 
 constexpr int kScanThreads = 1024;
 
-// row_ovf[i] = any_t(count[i][t] > K), and the row's kept entries
+// row_ovf[i] = any_t(count[i][t] > K), or (dense_min > 0) the row has at
+// least dense_min active units; the row's kept entries
 // kept[i] = sum_t min(count[i][t], K), or -(1 + sum_t count[i][t]) for an
 // overflow row; one warp per row.
 // With tile-level routing no row overflows: row_ovf = 0, kept = every active unit.
-__global__ void row_flags_kernel(const uint16_t* __restrict__ count, int M, int T, int K, bool tiles,
+__global__ void row_flags_kernel(const uint16_t* __restrict__ count, int M, int T, int K, int dense_min, bool tiles,
                                  uint8_t* __restrict__ row_ovf, int* __restrict__ kept) {
   const int lane = threadIdx.x & 31;
   const long warp0 = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -41,6 +42,7 @@ __global__ void row_flags_kernel(const uint16_t* __restrict__ count, int M, int 
       n += __shfl_xor_sync(0xFFFFFFFFu, n, o);
       all += __shfl_xor_sync(0xFFFFFFFFu, all, o);
     }
+    any |= dense_min > 0 && all >= dense_min;
     if (tiles) any = false, n = all;
     if (lane == 0) {
       row_ovf[row] = any ? 1 : 0;
@@ -308,7 +310,7 @@ __global__ void __launch_bounds__(256) transpose_bf16_kernel(const uint16_t* __r
 }  // namespace
 
 cudaError_t launch_route(const uint16_t* count, const uint16_t* val, const uint8_t* col, const uint16_t* spill,
-                         int M, int f, int K, int cap, uint8_t* row_ovf, int* ovf_rows, int* n_ovf,
+                         int M, int f, int K, int dense_min, int cap, uint8_t* row_ovf, int* ovf_rows, int* n_ovf,
                          uint16_t* g_ovf, const uint16_t* X, int d, uint16_t* x_ovf, int* plan, int groups,
                          bool tiles, uint32_t* status, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
@@ -317,7 +319,8 @@ cudaError_t launch_route(const uint16_t* count, const uint16_t* val, const uint8
   int blocks = (warps_needed + 7) / 8;
   const int max_blocks = device_sm_count() * 16;
   if (blocks > max_blocks) blocks = max_blocks;
-  TWELL_LAUNCH("row_flags", s, row_flags_kernel<<<blocks, 256, 0, s>>>(count, M, T, K, tiles, row_ovf, plan + kPlanHdr));
+  TWELL_LAUNCH("row_flags", s, row_flags_kernel<<<blocks, 256, 0, s>>>(count, M, T, K, dense_min, tiles, row_ovf,
+                                                                       plan + kPlanHdr));
   TWELL_LAUNCH("route_plan", s,
                route_plan_kernel<<<1, kScanThreads, 0, s>>>(plan, M, f, groups, cap, tiles, ovf_rows, n_ovf, status));
   if (cap > 0 && !tiles) {

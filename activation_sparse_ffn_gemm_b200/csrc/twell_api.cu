@@ -143,6 +143,7 @@ twell_status check_hybrid(const twell_hybrid* h, int64_t d_model) {
   if (!h) return TWELL_EINVAL;
   const twell_status st = twell_query_support(h->M, d_model, h->d_ff, h->T_n, h->K, h->ovf_cap);
   if (st != TWELL_OK) return st;
+  if (h->dense_min < 0) return TWELL_EINVAL;
   if (h->M == 0) return TWELL_OK;
   const void* ptrs[] = {h->count, h->val, h->col, h->row_ovf, h->ovf_rows, h->n_ovf, h->g_ovf, h->status,
                         h->row_plan};
@@ -173,7 +174,7 @@ twell_status run_pack(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_
   PackOut po{h->count, h->val, h->col, at<uint16_t>(ws, L.spill), z_debug};
   cudaError_t e = launch_gate_pack(X, W_g, b_g, M, static_cast<int>(d), f, K, po, h->status, s);
   if (e != cudaSuccess) return TWELL_ECUDA;
-  e = launch_route(h->count, h->val, h->col, po.spill, M, f, K, cap, h->row_ovf, h->ovf_rows, h->n_ovf, h->g_ovf,
+  e = launch_route(h->count, h->val, h->col, po.spill, M, f, K, h->dense_min, cap, h->row_ovf, h->ovf_rows, h->n_ovf, h->g_ovf,
                    X_for_gather, static_cast<int>(d), x_ovf, h->row_plan, tok_groups(M, static_cast<int>(d)),
                    tiles, h->status, s);
   return cuda_status(e);
@@ -379,8 +380,9 @@ twell_status twell_count_stats(const twell_hybrid* h, int64_t* rows_by_max, int6
   const twell_status st = twell_query_support(h->M, 64, h->d_ff, h->T_n, h->K, h->ovf_cap);
   if (st != TWELL_OK) return st;
   if (h->M > 0 && (!h->count || !aligned16(h->count))) return TWELL_EINVAL;
-  return cuda_status(launch_count_stats(h->count, h->M, h->d_ff / kTn, rows_by_max, act_by_max, tiles_by_count,
-                                        reinterpret_cast<cudaStream_t>(stream)));
+  if (h->dense_min < 0) return TWELL_EINVAL;
+  return cuda_status(launch_count_stats(h->count, h->M, h->d_ff / kTn, h->dense_min, rows_by_max, act_by_max,
+                                        tiles_by_count, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 twell_status twell_status_read(const twell_hybrid* h, uint32_t* out, int clear, twell_stream_t stream) {

@@ -122,7 +122,7 @@ cudaError_t launch_gate_pack(const uint16_t* X, const uint16_t* W_g, const uint1
 // tiles: tile-level routing (no overflow rows; the plan counts every active
 // unit and is marked inference-only).
 cudaError_t launch_route(const uint16_t* count, const uint16_t* val, const uint8_t* col, const uint16_t* spill,
-                         int M, int f, int K, int cap, uint8_t* row_ovf, int* ovf_rows, int* n_ovf,
+                         int M, int f, int K, int dense_min, int cap, uint8_t* row_ovf, int* ovf_rows, int* n_ovf,
                          uint16_t* g_ovf, const uint16_t* X, int d, uint16_t* x_ovf, int* plan, int groups,
                          bool tiles, uint32_t* status, cudaStream_t s);
 

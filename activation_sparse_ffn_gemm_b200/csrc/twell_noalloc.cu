@@ -52,6 +52,7 @@ extern "C" TWELL_API twell_status twell_pack_noalloc(const uint16_t* X, const ui
   if (!h) return TWELL_EINVAL;
   const twell_status st = twell_query_support(h->M, d_model, h->d_ff, h->T_n, h->K, h->ovf_cap);
   if (st != TWELL_OK) return st;
+  if (h->dense_min < 0) return TWELL_EINVAL;
   if (h->M == 0) return TWELL_OK;
   if (static_cast<uint64_t>(h->M) * static_cast<uint64_t>(h->d_ff) * sizeof(uint16_t) >
       static_cast<uint64_t>(TWELL_NOALLOC_SCRATCH_BYTES))
@@ -68,8 +69,9 @@ extern "C" TWELL_API twell_status twell_pack_noalloc(const uint16_t* X, const ui
   const int M = h->M, d = static_cast<int>(d_model), f = h->d_ff, K = h->K;
   PackOut po{h->count, h->val, h->col, scratch, z_debug};
   if (launch_gate_pack(X, W_g, b_g, M, d, f, K, po, h->status, s) != cudaSuccess) return TWELL_ECUDA;
-  if (launch_route(h->count, h->val, h->col, scratch, M, f, K, h->ovf_cap, h->row_ovf, h->ovf_rows, h->n_ovf,
-                   h->g_ovf, nullptr, d, nullptr, h->row_plan, tok_groups(M, d), false, h->status, s) != cudaSuccess)
+  if (launch_route(h->count, h->val, h->col, scratch, M, f, K, h->dense_min, h->ovf_cap, h->row_ovf, h->ovf_rows,
+                   h->n_ovf, h->g_ovf, nullptr, d, nullptr, h->row_plan, tok_groups(M, d), false, h->status,
+                   s) != cudaSuccess)
     return TWELL_ECUDA;
   return TWELL_OK;
 }

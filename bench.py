@@ -15,7 +15,9 @@ K=8) run as a training step, synthetic seeded data, inputs resident in HBM.
 FFN over token counts M in {512, 2048, 8192, 32768, 65536} and mean sparsity in
 {90, 95, 99, 99.5, 99.9}% at d_model=4096, d_ff=14336, with per-token
 lognormal(0, 0.75) row scaling, K = max(8, 2^ceil(log2(4 p T_n))), one JSON
-line per point (1 GPU). With --sweep-k 8,16,32,64 each point is timed for every
+line per point (1 GPU). Each point also times adaptive routing: the dense-row
+threshold of the cost model and the K chosen from the batch's count statistics
+(activation_sparse_ffn_gemm_b200.kchoice). With --sweep-k 8,16,32,64 each point is timed for every
 listed K instead, next to the K that the batch's count statistics and the cost
 model of activation_sparse_ffn_gemm_b200.kchoice choose.
 
@@ -791,7 +793,32 @@ def run_sweep(args, local):
 
             t_fwd_tiles = timed(fwd_tiles)
             assert st_t.read_status() == 0, "device status word set"
-            del st, st_t, wsf, wsb, grads, Wdt, Y
+            del st, st_t, wsf, wsb
+
+            # adaptive routing: the cost model's dense-row threshold and the K that the
+            # batch's count statistics choose (kchoice), for training and for inference
+            adaptive = {}
+            for mode, training in (("fwd_bwd", True), ("fwd", False)):
+                dm = tw.dense_min_for(d, f, training)
+                probe = tw.HybridState(M, f, T_n, 8, M, dev, with_u=False, dense_min=dm)
+                tw.pack(X, W_g, b_g, T_n=T_n, K=8, state=probe)
+                K_a = tw.suggest_k(tw.count_stats(probe), d, f, T_n, training=training)[0]
+                del probe
+                st_a = tw.HybridState(M, f, T_n, K_a, M, dev, with_u=training, dense_min=dm)
+                wsf_a = tw.workspace(tw.OP_FWD, M, d, f, T_n, K_a, M, dev)
+                wsb_a = tw.workspace(tw.OP_BWD, M, d, f, T_n, K_a, M, dev) if training else None
+
+                def body():
+                    tw.transpose_wd(W_d, out=Wdt)
+                    tw.ffn_fwd(X, W_g, b_g, W_u, W_d, T_n=T_n, K=K_a, W_dt=Wdt, state=st_a, ws=wsf_a, Y=Y)
+                    if training:
+                        tw.ffn_bwd(X, W_g, W_u, W_d, st_a, dY, lam=args.lam, W_dt=Wdt, ws=wsb_a, out=grads)
+
+                adaptive[mode] = {"ms": timed(body), "K": K_a, "dense_min": dm,
+                                  "overflow_rows": st_a.n_overflow()[1]}
+                assert st_a.read_status() == 0, "device status word set"
+                del st_a, wsf_a, wsb_a
+            del grads, Wdt, Y
 
             Wg_r, Wu_r, Wd_r = (t.clone().requires_grad_() for t in (W_g, W_u, W_d))
             Xr = X.clone().requires_grad_()
@@ -816,8 +843,11 @@ def run_sweep(args, local):
                 "twell": {"fwd_ms": t_fwd, "fwd_bwd_ms": t_fb, "fwd_tokens_per_s": M / (t_fwd / 1e3),
                           "fwd_bwd_tokens_per_s": M / (t_fb / 1e3), "dense_wgrad_for_overflow_rows": dense_wgrad},
                 "twell_tile_routing": {"fwd_ms": t_fwd_tiles, "fwd_tokens_per_s": M / (t_fwd_tiles / 1e3)},
+                "twell_adaptive": adaptive,
                 "dense_bf16": {"fwd_ms": t_dfwd, "fwd_bwd_ms": t_dfb},
-                "speedup_vs_dense": {"fwd": t_dfwd / t_fwd, "fwd_bwd": t_dfb / t_fb},
+                "speedup_vs_dense": {"fwd": t_dfwd / t_fwd, "fwd_bwd": t_dfb / t_fb,
+                                     "adaptive_fwd": t_dfwd / adaptive["fwd"]["ms"],
+                                     "adaptive_fwd_bwd": t_dfb / adaptive["fwd_bwd"]["ms"]},
                 "measured": {"activity": activity, "overflow_rows": n_ovf, "max_over_mean_count": ratio},
                 "steps": steps, "warmup": warm, "data": "synthetic (seeded torch CUDA generator)",
                 "l2": "flushed before every timed step"}), flush=True)

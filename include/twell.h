@@ -84,7 +84,11 @@ typedef enum twell_status {
  *                 s < min(count, K); 0 in the unused slots
  *   col[i][t][s]  in-tile column of that unit (0..T_n-1); 0 in the unused slots
  * Row routing: row i is an overflow row (row_ovf[i] = 1) when some tile has
- * count > K. Overflow rows are listed in ascending order in ovf_rows; the first
+ * count > K, or, when dense_min > 0, when its active units (sum over its tiles
+ * of count) number at least dense_min. The second rule is this library's
+ * addition to the pages' overflow routing: it sends rows whose gathers would
+ * cost more than a dense row to the dense backup (results are the same either
+ * way; kchoice.py derives the threshold from measured costs). Overflow rows are listed in ascending order in ovf_rows; the first
  * ovf_cap of them get a dense row g_ovf[s][:] = bf16(ReLU(z[i][:])).
  * n_ovf[0] = rows stored (min(flagged, ovf_cap)), n_ovf[1] = rows flagged.
  * The ELL slots of an overflow row still hold its first K actives per tile.
@@ -108,6 +112,7 @@ typedef struct twell_hybrid {
   int32_t T_n;       /* tile width (must be 128) */
   int32_t K;         /* ELL slots per (row, tile) */
   int32_t ovf_cap;   /* capacity of the dense backup block, in rows */
+  int32_t dense_min; /* 0, or route rows with at least this many active units dense */
   uint16_t* count;   /* [M][T] */
   uint16_t* val;     /* [M][T][K] bf16 bits */
   uint8_t* col;      /* [M][T][K] */
@@ -243,17 +248,21 @@ TWELL_API twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, con
  * Count statistics of a packed batch, for choosing the ELL width K of later
  * batches ([aivizor] ¶4: in training the largest number of nonzeros per row
  * can exceed the mean by a large factor). Read from h->count, which keeps the
- * true per-tile counts 0..T_n. With bins c = 0..T_n:
- *   rows_by_max[c]     rows whose largest tile count is c
- *   act_by_max[c]      active units of those rows (summed over their tiles)
- *   tiles_by_count[c]  (row, tile) pairs holding c active units
+ * true per-tile counts 0..T_n. With bins c = 0..T_n + 1:
+ *   rows_by_max[c]     rows whose largest tile count is c, except that a row
+ *                      with at least h->dense_min active units (when
+ *                      dense_min > 0) is counted in bin T_n + 1
+ *   act_by_max[c]      active units of the rows of bin c (summed over tiles)
+ *   tiles_by_count[c]  (row, tile) pairs holding c active units (bin T_n + 1
+ *                      stays 0)
  * Under row routing with width K the rows of bins c > K are the dense backup
  * rows and the rest keep all their units in ELL slots; under tile routing the
  * tiles of bins c > K are read from their spilled slices.
- * The three outputs are caller-owned device int64 arrays of T_n + 1 entries
+ * The three outputs are caller-owned device int64 arrays of T_n + 2 entries
  * (8-byte aligned), overwritten; asynchronous on `stream`. Integer sums: the
- * same result on every run. Errors: TWELL_EINVAL (null or misaligned pointer),
- * TWELL_EUNSUPPORTED (descriptor shape), TWELL_ECUDA (launch failure).
+ * same result on every run. Errors: TWELL_EINVAL (null or misaligned pointer,
+ * negative dense_min), TWELL_EUNSUPPORTED (descriptor shape), TWELL_ECUDA
+ * (launch failure).
  */
 TWELL_API twell_status twell_count_stats(const twell_hybrid* h, int64_t* rows_by_max, int64_t* act_by_max,
                                          int64_t* tiles_by_count, twell_stream_t stream);

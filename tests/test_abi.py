@@ -44,11 +44,26 @@ def test_library_exports_every_declared_symbol(tw):
     assert exported == set(declared_functions())
 
 
-def test_hybrid_struct_matches_header(tw):
-    # five int32 fields, 4 bytes of padding, eleven pointers
+def test_hybrid_struct_matches_header(tw, tmp_path):
+    # six int32 fields, eleven pointers
     assert ctypes.sizeof(tw.TwellHybrid) == 24 + 11 * 8
+    assert tw.TwellHybrid.dense_min.offset == 20
     assert tw.TwellHybrid.count.offset == 24
     assert tw.TwellHybrid.row_plan.offset == 24 + 10 * 8
+    # the header's own layout, as a C compiler sees it
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "twell.h"\n'
+                   'int main(void) { printf("%zu", sizeof(twell_hybrid)); '
+                   'printf(" %zu %zu %zu %zu\\n", offsetof(twell_hybrid, ovf_cap), offsetof(twell_hybrid, dense_min), '
+                   'offsetof(twell_hybrid, count), offsetof(twell_hybrid, row_plan)); return 0; }\n')
+    exe = tmp_path / "layout"
+    rc = os.system(f"gcc -std=c11 -I{os.path.join(ROOT, 'include')} -o {exe} {src}")
+    assert rc == 0
+    got = [int(v) for v in os.popen(str(exe)).read().split()]
+    fields = dict(tw.TwellHybrid._fields_)
+    assert got == [ctypes.sizeof(tw.TwellHybrid), tw.TwellHybrid.ovf_cap.offset, tw.TwellHybrid.dense_min.offset,
+                   tw.TwellHybrid.count.offset, tw.TwellHybrid.row_plan.offset]
+    assert "dense_min" in fields
 
 
 def test_plan_ints(tw):
@@ -88,23 +103,33 @@ def test_workspace_sizes(tw):
 
 def test_host_side_errors(tw):
     L = tw.lib()
-    h = tw.TwellHybrid(64, 1024, 128, 8, 64, *([None] * 11))
+    h = tw.TwellHybrid(64, 1024, 128, 8, 64, 0, *([None] * 11))
     # null descriptor, null arrays, unsupported shape, missing workspace
     assert L.twell_pack(None, None, None, 256, None, None, None, 0, None) == 1
     assert L.twell_pack(None, None, None, 256, ctypes.byref(h), None, None, 0, None) == 1
-    bad = tw.TwellHybrid(64, 1024, 64, 8, 64, *([None] * 11))
+    bad = tw.TwellHybrid(64, 1024, 64, 8, 64, 0, *([None] * 11))
     assert L.twell_pack(None, None, None, 256, ctypes.byref(bad), None, None, 0, None) == 2
     fake = 1 << 20  # aligned non-null addresses; never dereferenced by these checks
-    h2 = tw.TwellHybrid(64, 1024, 128, 8, 64, *([fake] * 11))
+    h2 = tw.TwellHybrid(64, 1024, 128, 8, 64, 0, *([fake] * 11))
     p = ctypes.c_void_p(fake)
     assert L.twell_pack(p, p, p, 256, ctypes.byref(h2), None, None, 0, None) == 6
     assert L.twell_pack(p, p, p, 256, ctypes.byref(h2), None, ctypes.c_void_p(fake + 8), 1 << 30, None) == 6
     mis = ctypes.c_void_p(fake + 2)
     assert L.twell_ffn_fwd(mis, p, p, p, p, None, 256, p, ctypes.byref(h2), None, None, 0, None) == 1
     # empty batch forward: nothing to do, nothing touched
-    h0 = tw.TwellHybrid(0, 1024, 128, 8, 0, *([None] * 11))
+    h0 = tw.TwellHybrid(0, 1024, 128, 8, 0, 0, *([None] * 11))
     assert L.twell_ffn_fwd(None, None, None, None, None, None, 256, None, ctypes.byref(h0), None, None, 0, None) == 0
     assert L.twell_transpose_wd(None, 256, 1024, None, None) == 1
+    # a negative row threshold is refused before anything is enqueued
+    hn = tw.TwellHybrid(64, 1024, 128, 8, 64, -1, *([fake] * 11))
+    assert L.twell_pack(p, p, p, 256, ctypes.byref(hn), None, p, 1 << 30, None) == 1
+    assert L.twell_pack_noalloc(p, p, p, 256, ctypes.byref(hn), None, None) == 1
+    # count statistics: null or misaligned outputs, bad threshold, unsupported shape
+    assert L.twell_count_stats(ctypes.byref(h2), None, p, p, None) == 1
+    assert L.twell_count_stats(ctypes.byref(h2), p, ctypes.c_void_p(fake + 4), p, None) == 1
+    assert L.twell_count_stats(ctypes.byref(hn), p, p, p, None) == 1
+    assert L.twell_count_stats(ctypes.byref(bad), p, p, p, None) == 2
+    assert L.twell_count_stats(None, p, p, p, None) == 1
 
 
 def test_missing_library_fails_loudly(tw, monkeypatch):

@@ -36,10 +36,10 @@ def _dev(inp):
     return {k: to_dev(v) for k, v in inp.items() if k != "meta"}
 
 
-def _run_fwd(tw, inp, w, cap=None, save=True):
+def _run_fwd(tw, inp, w, cap=None, save=True, dense_min=0):
     D = _dev(inp)
     Y, st, z = tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], T_n=w.T_n, K=w.K, ovf_cap=cap,
-                          save_for_backward=save, z_debug=True)
+                          save_for_backward=save, z_debug=True, dense_min=dense_min)
     torch.cuda.synchronize()
     return D, Y, st, z
 
@@ -49,7 +49,7 @@ def _check_fwd(orc, inp, w, Y, st, z, rows=None, cap=None):
     M, f = inp["X"].shape[0], inp["W_g"].shape[0]
     zg = z.cpu().numpy()
     p_gpu = state_to_numpy(st)
-    p_ref = orc.pack(zg.astype(np.float64), w.T_n, w.K, cap=cap)
+    p_ref = orc.pack(zg.astype(np.float64), w.T_n, w.K, cap=cap, dense_min=st.dense_min)
     assert_pack_equal(p_gpu, p_ref)
     expect = 8 if p_ref["n_ovf_total"] > p_ref["n_ovf"] else 0  # TWELL_STATUS_OVERFLOW_CAP
     assert st.read_status() == expect
@@ -282,13 +282,44 @@ def test_count_stats(tw, orc, name):
     assert gs["act_by_max"][:K + 1].sum() == int(st.row_plan[2].item())
     best, times = tw.suggest_k(gs, d, f)
     assert best in times and len(times) == 4
+    # with a row threshold, rows of at least dense_min actives move to the last bin
+    dm = max(1, int(np.median(p_ref["count"].astype(np.int64).sum(1))))
+    st.c.dense_min = dm
+    gs = {k: v.cpu().numpy() for k, v in tw.count_stats(st).items()}
+    ref = orc.count_stats(p_ref["count"], 128, dense_min=dm)
+    for k in ref:
+        assert np.array_equal(gs[k], ref[k]), k
+
+
+@pytest.mark.parametrize("name,frac", [("heavy_small", 0.5), ("ragged", 0.3), ("k64", 0.6)])
+def test_dense_min_routing(tw, orc, name, frac):
+    """Rows with at least dense_min active units go to the dense backup as well
+    (threshold at a quantile of the row totals): pack bit-exact against the
+    oracle's pack with the same rule, Y and every gradient against the oracle."""
+    M, d, f, K, act, rs, seed = CASES[name]
+    w = Workload(name, M, d, f, 128, K, act, row_scale=rs, training=True, seed=seed)
+    inp = make_inputs(w)
+    D0, Y0, st0, z0 = _run_fwd(tw, inp, w)
+    totals = st0.count.cpu().numpy().view(np.uint16).astype(np.int64).sum(1)
+    dm = max(1, int(np.quantile(totals, 1.0 - frac)))
+    D, Y, st, z = _run_fwd(tw, inp, w, dense_min=dm)
+    n_plain, n_thr = st0.n_overflow()[1], st.n_overflow()[1]
+    assert n_thr == int(((st0.count.cpu().numpy().view(np.uint16) > K).any(1) | (totals >= dm)).sum())
+    assert n_thr > n_plain
+    p, _, _ = _check_fwd(orc, inp, w, Y, st, z)
+    assert_plan_valid(st)
+    for lam in (0.0, 1e-3):
+        g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=lam)
+        torch.cuda.synchronize()
+        _check_bwd(orc, inp, g, gpu_gmat(p, M, f, 128, K), lam, f"{name} dense_min={dm}")
+    assert st.read_status() == 0
 
 
 def test_count_stats_empty_batch(tw):
     st = tw.HybridState(0, 256, 128, 8, 0, "cuda")
     out = tw.count_stats(st)
     torch.cuda.synchronize()
-    assert all(v.shape == (129,) and int(v.abs().sum().item()) == 0 for v in out.values())
+    assert all(v.shape == (130,) and int(v.abs().sum().item()) == 0 for v in out.values())
 
 
 @pytest.mark.parametrize("M,activity,bwd", [(2048, 0.1, False), (512, 0.001, False), (64, 0.1, True),

@@ -4,7 +4,7 @@ the modelled time of each candidate K against values worked out by hand."""
 import numpy as np
 import pytest
 
-from activation_sparse_ffn_gemm_b200.kchoice import CostModel, modelled_times, suggest_k
+from activation_sparse_ffn_gemm_b200.kchoice import CostModel, dense_min_for, modelled_times, suggest_k
 
 T_n = 128
 
@@ -12,7 +12,7 @@ T_n = 128
 def _stats(rows_by_max, act_by_max, tiles_by_count):
     out = {}
     for k, v in (("rows_by_max", rows_by_max), ("act_by_max", act_by_max), ("tiles_by_count", tiles_by_count)):
-        a = np.zeros(T_n + 1, np.int64)
+        a = np.zeros(T_n + 2, np.int64)
         for c, n in v.items():
             a[c] = n
         out[k] = a
@@ -32,6 +32,10 @@ def test_row_routing_terms_by_hand():
     # K=8: 30 pairs sparse, 1 row dense; K=32: all 70 pairs sparse, no dense row
     assert t[8] == 1.0 * 2 * 30 + 10.0 * 2 * 256 * 1 + M * T * (2 + 3 * 8)
     assert t[32] == 1.0 * 2 * 70 + M * T * (2 + 3 * 32)
+    # a row routed dense by the threshold (bin T_n + 1) is dense at every K
+    st2 = _stats({5: 3, T_n + 1: 1}, {5: 30, T_n + 1: 40}, {5: 3, 3: 3, 20: 1, 1: 1})
+    t2 = modelled_times(st2, d_model=2, d_ff=256, candidates=(8, 32), training=False, model=UNIT)
+    assert t2[8] == t[8] and t2[32] == 1.0 * 2 * 30 + 10.0 * 2 * 256 * 1 + M * T * (2 + 3 * 32)
     best, times = suggest_k(st, d_model=2, d_ff=256, candidates=(8, 32), training=False, model=UNIT)
     assert best == 32 and times == t
 
@@ -81,3 +85,17 @@ def test_rejects_bad_statistics():
         suggest_k(st, 64, 128)
     with pytest.raises(ValueError):
         modelled_times(_stats({3: 1}, {3: 3}, {3: 1}), 64, 128, candidates=(0,))
+
+
+def test_dense_min_break_even():
+    m = CostModel(pair_fwd_s=2.0, pair_bwd_s=3.0, dense_fwd_s=1.0, dense_bwd_s=4.0)
+    # ceil(r * d_ff / a): inference 1 * 256 / 2, training 5 * 256 / 5
+    assert dense_min_for(64, 256, training=False, model=m) == 128
+    assert dense_min_for(64, 256, training=True, model=m) == 256
+    # the measured coefficients: weights in L2 at d_model=2048, d_ff=8192, from HBM at 4096 x 14336
+    assert CostModel.for_shape(2048, 8192).pair_fwd_s < CostModel.for_shape(4096, 14336).pair_fwd_s
+    for d, f in ((2048, 8192), (4096, 14336)):
+        for training in (False, True):
+            a = dense_min_for(d, f, training)
+            # about 1-3% of the row active: above the 1% rows of the uniform workload's mean
+            assert 0.01 * f < a < 0.03 * f, (d, f, training, a)
