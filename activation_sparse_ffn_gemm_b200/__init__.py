@@ -297,3 +297,6 @@ def ffn_bwd(X, W_g, W_u, W_d, state: HybridState, dY, lam: float = 0.0, W_dt=Non
                                _ptr(out["dW_d"]), _ptr(out.get("db_g")), _ptr(ws), ws.numel(), _stream(stream)),
            "twell_ffn_bwd")
     return out
+
+
+from .autograd import TwellFFNFunction, twell_ffn  # noqa: E402,F401

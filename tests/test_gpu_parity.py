@@ -315,6 +315,32 @@ def test_dense_min_routing(tw, orc, name, frac):
     assert st.read_status() == 0
 
 
+def test_autograd_function(tw, orc):
+    """twell_ffn under autograd: the same Y as twell_ffn_fwd and the same
+    gradients as twell_ffn_bwd (rounded to the inputs' bf16), for a 3-D input,
+    with the L1 term and a row threshold; and Y against the oracle."""
+    M, d, f, K, act, rs, seed = CASES["ragged"]
+    w = Workload("ragged", M, d, f, 128, K, act, row_scale=rs, training=True, seed=seed)
+    inp = make_inputs(w)
+    D = _dev(inp)
+    dm = 20
+    Y_ref, st = tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], K=K, dense_min=dm)
+    g_ref = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=1e-3)
+    leaves = {k: D[k].clone().requires_grad_() for k in ("X", "W_g", "b_g", "W_u", "W_d")}
+    X3 = leaves["X"].view(2, M // 2, d)
+    Y = tw.twell_ffn(X3, leaves["W_g"], leaves["b_g"], leaves["W_u"], leaves["W_d"], K=K, lam=1e-3, dense_min=dm)
+    assert Y.shape == (2, M // 2, d) and torch.equal(Y.reshape(M, d), Y_ref)
+    (Y.float() * D["dY"].view(2, M // 2, d).float()).sum().backward()
+    torch.cuda.synchronize()
+    for k, gk in (("X", "dX"), ("W_g", "dW_g"), ("b_g", "db_g"), ("W_u", "dW_u"), ("W_d", "dW_d")):
+        assert leaves[k].grad.dtype == torch.bfloat16
+        assert torch.equal(leaves[k].grad, g_ref[gk].to(torch.bfloat16)), k
+    args = (inp["X"], inp["W_g"], inp["b_g"], inp["W_u"], inp["W_d"])
+    G = gpu_gmat(state_to_numpy(st), M, f, 128, K)
+    assert_matches_oracle(f32_of_bits(bits_of(Y_ref)), orc.ffn_fwd(*args, gmat=G), orc.ffn_fwd(*args),
+                          "autograd Y", bf16_out=True)
+
+
 def test_count_stats_empty_batch(tw):
     st = tw.HybridState(0, 256, 128, 8, 0, "cuda")
     out = tw.count_stats(st)
