@@ -377,21 +377,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             *last_s = last ? 1 : 0;
           }
           epi_bar(epi_cnt, bar_gen, abort_flag);
-          if (*last_s && row < M_eff) {
+          if (*last_s) {
+            // the tile's (row, 8-column chunk) items spread over the 128 epilogue
+            // threads (consecutive threads on consecutive chunks of a row), each
+            // issuing its `split` partial loads together; per element the
+            // partials are still added in range order 0, 1, ...
             __threadfence();
+            const int rows_here = min(kBM, M_eff - mb * kBM);
+            const int items = rows_here * (BN / 8);
 #pragma unroll 1
-            for (int c8 = 0; c8 < BN / 8; ++c8) {
-              const int n = nb * BN + c8 * 8;
-              if (n >= shp.N) break;
-              float accv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-              for (int k2 = 0; k2 < split; ++k2) {
-                const float4* p =
-                    reinterpret_cast<const float4*>(shp.partial + (static_cast<size_t>(k2) * shp.split_rows + row) * shp.N + n);
-                const float4 a = __ldcg(p), b = __ldcg(p + 1);
-                accv[0] += a.x; accv[1] += a.y; accv[2] += a.z; accv[3] += a.w;
-                accv[4] += b.x; accv[5] += b.y; accv[6] += b.z; accv[7] += b.w;
+            for (int it = r; it < items; it += kBM) {
+              const int row2 = mb * kBM + it / (BN / 8);
+              const int n = nb * BN + (it % (BN / 8)) * 8;
+              if (n >= shp.N) continue;
+              float4 pa[kSplitMax], pb[kSplitMax];
+#pragma unroll
+              for (int k2 = 0; k2 < kSplitMax; ++k2) {
+                if (k2 < split) {
+                  const float4* p = reinterpret_cast<const float4*>(
+                      shp.partial + (static_cast<size_t>(k2) * shp.split_rows + row2) * shp.N + n);
+                  pa[k2] = __ldcg(p);
+                  pb[k2] = __ldcg(p + 1);
+                }
               }
-              Epi::apply8(ea, row, n, accv);
+              float accv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+              for (int k2 = 0; k2 < kSplitMax; ++k2) {
+                if (k2 < split) {
+                  accv[0] += pa[k2].x; accv[1] += pa[k2].y; accv[2] += pa[k2].z; accv[3] += pa[k2].w;
+                  accv[4] += pb[k2].x; accv[5] += pb[k2].y; accv[6] += pb[k2].z; accv[7] += pb[k2].w;
+                }
+              }
+              Epi::apply8(ea, row2, n, accv);
             }
           }
         }
