@@ -55,8 +55,15 @@ struct GemmShape {
   int split_max = 1;
   unsigned long long* arrivals = nullptr;  // [kSplitTiles] per-output-tile arrival words
   unsigned long long epoch = 0;            // this launch's tag (1 .. 2^56 - 1)
+  // CUDA-core path for at most kGemvRows processed rows (single segment only;
+  // nullptr: none): C[i][n] = sum_k gv_a[i * lda + k] * gv_b[n * ldb + k], both
+  // K-contiguous bf16 in global memory, each 8-column group through Epi::apply8
+  const uint16_t* gv_a = nullptr;
+  const uint16_t* gv_b = nullptr;
+  int lda = 0, ldb = 0;
 };
 
+constexpr int kGemvRows = 8;
 constexpr int kSplitMax = 8;
 constexpr int kSplitRows = 2 * 128;
 constexpr int kSplitMinKBlocks = 4;
@@ -114,6 +121,83 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int&
   nb = within / gm;
 }
 
+// The rows-times-matrix product of a GEMM with at most kGemvRows rows: a tensor-
+// core tile would be 128 rows of which almost all are padding, and its K-split
+// pipeline is latency-bound, while this streams each row of B once from HBM.
+// Column groups of 8 are dealt to the CTAs round robin; a CTA's six warps take
+// the group's 256-element K chunks round robin (lane l holds elements l*8 ..
+// l*8+7 of a chunk, so a warp reads 512 contiguous bytes of each row); per
+// (row, column) the lanes' sums meet by shuffles, the warps' sums in shared
+// memory, added in warp order by thread i for row i, which applies Epi::apply8.
+// The order of every sum is fixed, so the result is the same on every run.
+template <class Epi>
+__device__ __forceinline__ void gemv_rows(const GemmShape& shp, const typename Epi::Args& ea, int M_eff,
+                                          float* red) {
+  constexpr int W = kGemmThreads / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int K = shp.K0, N = shp.N;
+  const int nchunks = (K + 255) / 256;
+  for (int n0 = blockIdx.x * 8; n0 < N; n0 += gridDim.x * 8) {
+    float acc[kGemvRows][8];
+#pragma unroll
+    for (int i = 0; i < kGemvRows; ++i)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[i][c] = 0.f;
+    for (int q = warp; q < nchunks; q += W) {
+      const int k = q * 256 + lane * 8;  // K is a multiple of 64, so k < K means k + 8 <= K
+      if (k >= K) continue;
+      uint4 b[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        b[c] = n0 + c < N ? __ldg(reinterpret_cast<const uint4*>(shp.gv_b + static_cast<size_t>(n0 + c) * shp.ldb + k))
+                          : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int i = 0; i < kGemvRows; ++i) {
+        if (i >= M_eff) break;
+        const uint4 a = __ldg(reinterpret_cast<const uint4*>(shp.gv_a + static_cast<size_t>(i) * shp.lda + k));
+        const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t bv[4] = {b[c].x, b[c].y, b[c].z, b[c].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+                "mov.b32 {al, ah}, %1;\n\t"
+                "mov.b32 {bl, bh}, %2;\n\t"
+                "fma.rn.f32.bf16 %0, al, bl, %0;\n\t"
+                "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+                : "+f"(acc[i][c])
+                : "r"(av[e]), "r"(bv[e]));
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kGemvRows; ++i) {
+      if (i >= M_eff) break;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float v = acc[i][c];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        if (lane == 0) red[(warp * kGemvRows + i) * 8 + c] = v;
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < M_eff) {
+      float v[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float t = 0.f;
+        for (int w = 0; w < W; ++w) t += red[(w * kGemvRows + threadIdx.x) * 8 + c];
+        v[c] = t;
+      }
+      Epi::apply8(ea, threadIdx.x, n0, v);
+    }
+    __syncthreads();
+  }
+}
+
 template <class Epi, int BN, bool B_MN, int STAGES, bool A_MN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
@@ -160,6 +244,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int nk0 = *k0_eff_s / kBK;
   const int nk = nk0 + shp.K1 / kBK;
   if (nk == 0) return;  // nothing to contract (a device-side K of zero)
+  if constexpr (Epi::kSplitK) {
+    if (shp.gv_b != nullptr && shp.K1 == 0 && shp.K_dev == nullptr && *m_eff_s <= kGemvRows) {
+      if (*m_eff_s > 0) gemv_rows<Epi>(shp, ea, *m_eff_s, reinterpret_cast<float*>(smem));
+      return;
+    }
+  }
   const int split = gemm_split(*m_eff_s, shp.N, BN, nk, shp, gridDim.x);
   if (static_cast<long>(blockIdx.x) >=
       static_cast<long>((*m_eff_s + kBM - 1) / kBM) * ((shp.N + BN - 1) / BN) * split)

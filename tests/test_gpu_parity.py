@@ -95,6 +95,10 @@ CASES = {
     # 170 overflow rows of a heavy-tailed batch: split-K dense backup GEMMs,
     # overflow pairs kept in the pair list
     "heavy_small": (1024, 1024, 4096, 8, 0.02, "lognormal", 23),
+    # 8 and 9 overflow rows: the dense backup's CUDA-core path (at most 8 rows)
+    # and, one row more, the tensor-core split-K path
+    "ovf_rows_8": (384, 512, 2048, 8, 0.02, "none", 30),
+    "ovf_rows_9": (384, 512, 2048, 8, 0.02, "none", 41),
 }
 
 
@@ -113,6 +117,8 @@ def test_fwd_bwd_small(tw, orc, name):
     inp = make_inputs(w)
     D, Y, st, z = _run_fwd(tw, inp, w)
     p, flips, _ = _check_fwd(orc, inp, w, Y, st, z)
+    if name.startswith("ovf_rows_"):
+        assert p["n_ovf"] == int(name.rsplit("_", 1)[1])
     plan = assert_plan_valid(st)
     if name in SPLIT_CASES:
         assert plan["split_rows"] > 0, "this case should split rows into several pieces"
