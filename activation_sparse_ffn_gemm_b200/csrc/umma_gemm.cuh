@@ -124,33 +124,38 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int&
 // The rows-times-matrix product of a GEMM with at most kGemvRows rows: a tensor-
 // core tile would be 128 rows of which almost all are padding, and its K-split
 // pipeline is latency-bound, while this streams each row of B once from HBM.
-// Column groups of 8 are dealt to the CTAs round robin; a CTA's six warps take
-// the group's 256-element K chunks round robin (lane l holds elements l*8 ..
-// l*8+7 of a chunk, so a warp reads 512 contiguous bytes of each row); per
-// (row, column) the lanes' sums meet by shuffles, the warps' sums in shared
-// memory, added in warp order by thread i for row i, which applies Epi::apply8.
+// Work is 8-column groups (one Epi::apply8 per row); lane l holds elements
+// l*8 .. l*8+7 of each 256-element K chunk, so a warp reads 512 contiguous
+// bytes of a row per load, and kGemvBatch chunks of the group's 8 rows are
+// loaded before any is used (enough bytes in flight to stream from HBM).
+//   * K <= kGemvWarpK: a warp owns whole groups (dealt over all warps of the
+//     grid); its lanes' sums meet by shuffles and lane i applies row i.
+//   * larger K: a CTA owns a group (dealt over the CTAs), its warps take the
+//     chunk batches round robin, and their sums meet in shared memory, added
+//     in warp order by thread i for row i.
 // The order of every sum is fixed, so the result is the same on every run.
-template <class Epi>
-__device__ __forceinline__ void gemv_rows(const GemmShape& shp, const typename Epi::Args& ea, int M_eff,
-                                          float* red) {
-  constexpr int W = kGemmThreads / 32;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+constexpr int kGemvBatch = 4;
+constexpr int kGemvWarpK = 4096;
+
+template <int U>
+__device__ __forceinline__ void gemv_chunks(const GemmShape& shp, int M_eff, int n0, int q0, int qstep, int nchunks,
+                                            int lane, float (&acc)[kGemvRows][8]) {
   const int K = shp.K0, N = shp.N;
-  const int nchunks = (K + 255) / 256;
-  for (int n0 = blockIdx.x * 8; n0 < N; n0 += gridDim.x * 8) {
-    float acc[kGemvRows][8];
+  for (int q = q0; q < nchunks; q += qstep * U) {
+    uint4 b[U][8];
 #pragma unroll
-    for (int i = 0; i < kGemvRows; ++i)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[i][c] = 0.f;
-    for (int q = warp; q < nchunks; q += W) {
-      const int k = q * 256 + lane * 8;  // K is a multiple of 64, so k < K means k + 8 <= K
-      if (k >= K) continue;
-      uint4 b[8];
+    for (int u = 0; u < U; ++u) {
+      const int k = (q + u * qstep) * 256 + lane * 8;  // K is a multiple of 64: k < K means k + 8 <= K
 #pragma unroll
       for (int c = 0; c < 8; ++c)
-        b[c] = n0 + c < N ? __ldg(reinterpret_cast<const uint4*>(shp.gv_b + static_cast<size_t>(n0 + c) * shp.ldb + k))
-                          : make_uint4(0, 0, 0, 0);
+        b[u][c] = (k < K && n0 + c < N)
+                      ? __ldg(reinterpret_cast<const uint4*>(shp.gv_b + static_cast<size_t>(n0 + c) * shp.ldb + k))
+                      : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int k = (q + u * qstep) * 256 + lane * 8;
+      if (k >= K) continue;
 #pragma unroll
       for (int i = 0; i < kGemvRows; ++i) {
         if (i >= M_eff) break;
@@ -158,7 +163,7 @@ __device__ __forceinline__ void gemv_rows(const GemmShape& shp, const typename E
         const uint32_t av[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          const uint32_t bv[4] = {b[c].x, b[c].y, b[c].z, b[c].w};
+          const uint32_t bv[4] = {b[u][c].x, b[u][c].y, b[u][c].z, b[u][c].w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
@@ -172,6 +177,46 @@ __device__ __forceinline__ void gemv_rows(const GemmShape& shp, const typename E
         }
       }
     }
+  }
+}
+
+template <class Epi>
+__device__ __forceinline__ void gemv_rows(const GemmShape& shp, const typename Epi::Args& ea, int M_eff,
+                                          float* red) {
+  constexpr int W = kGemmThreads / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int K = shp.K0, N = shp.N;
+  const int nchunks = (K + 255) / 256;
+  float acc[kGemvRows][8];
+  if (K <= kGemvWarpK) {
+    for (int n0 = (blockIdx.x * W + warp) * 8; n0 < N; n0 += gridDim.x * W * 8) {
+#pragma unroll
+      for (int i = 0; i < kGemvRows; ++i)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[i][c] = 0.f;
+      gemv_chunks<kGemvBatch>(shp, M_eff, n0, 0, 1, nchunks, lane, acc);
+#pragma unroll
+      for (int i = 0; i < kGemvRows; ++i) {
+        if (i >= M_eff) break;
+        float v[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float t = acc[i][c];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
+          v[c] = t;
+        }
+        if (lane == i) Epi::apply8(ea, i, n0, v);
+      }
+    }
+    return;
+  }
+  for (int n0 = blockIdx.x * 8; n0 < N; n0 += gridDim.x * 8) {
+#pragma unroll
+    for (int i = 0; i < kGemvRows; ++i)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[i][c] = 0.f;
+    gemv_chunks<2>(shp, M_eff, n0, warp, W, nchunks, lane, acc);
 #pragma unroll
     for (int i = 0; i < kGemvRows; ++i) {
       if (i >= M_eff) break;
