@@ -342,14 +342,6 @@ void use_split(GemmShape& shp, const SplitKBuffers& sk, int cap) {
   shp.split_rows = cap < kSplitRows ? cap : kSplitRows;
   shp.split_max = kSplitMax;
 }
-// A GEMM of at most kGemvRows rows runs on the CUDA cores: a [rows][K] and b [N][K],
-// K-contiguous with row strides lda and ldb (elements).
-void use_gemv(GemmShape& shp, const uint16_t* a, int lda, const uint16_t* b, int ldb) {
-  shp.gv_a = a;
-  shp.lda = lda;
-  shp.gv_b = b;
-  shp.ldb = ldb;
-}
 }  // namespace
 
 size_t splitk_partial_floats(int cap, int d, int f) {
@@ -371,13 +363,11 @@ cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uin
     return cudaErrorInvalidValue;
   GemmShape s1{cap, n_ovf, f, d, 0, status};
   use_split(s1, sk, cap);
-  use_gemv(s1, x_ovf, d, W_u, d);
   EpiGateMul::Args e1{g_ovf, h_ovf, u_ovf, f};
   cudaError_t e = launch_umma_gemm<EpiGateMul, 256, false, kStages>("ovf_up_gemm", ta, tb, ta, tb, s1, e1, s);
   if (e != cudaSuccess) return e;
   GemmShape s2{cap, n_ovf, d, f, 0, status};
   use_split(s2, sk, cap);
-  use_gemv(s2, h_ovf, f, W_d, f);
   EpiScatterBf16::Args e2{ovf_rows, Y, d};
   return launch_umma_gemm<EpiScatterBf16, 256, false, kStages>("ovf_down_gemm", ta2, tb2, ta2, tb2, s2, e2, s);
 }
@@ -400,7 +390,6 @@ cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const u
     return cudaErrorInvalidValue;
   GemmShape s1{cap, n_ovf, f, d, 0, status};
   use_split(s1, sk, cap);
-  use_gemv(s1, dy_ovf, d, W_dt, d);
   EpiBwdDH::Args e1{g_ovf, u_ovf, duz_ovf, du_ovf, dz_ovf, lambda, f};
   cudaError_t e = launch_umma_gemm<EpiBwdDH, 256, false, kStages>("ovf_dh_gemm", ta, tb, ta, tb, s1, e1, s);
   if (e != cudaSuccess) return e;

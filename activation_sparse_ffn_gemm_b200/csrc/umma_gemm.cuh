@@ -55,15 +55,8 @@ struct GemmShape {
   int split_max = 1;
   unsigned long long* arrivals = nullptr;  // [kSplitTiles] per-output-tile arrival words
   unsigned long long epoch = 0;            // this launch's tag (1 .. 2^56 - 1)
-  // CUDA-core path for at most kGemvRows processed rows (single segment only;
-  // nullptr: none): C[i][n] = sum_k gv_a[i * lda + k] * gv_b[n * ldb + k], both
-  // K-contiguous bf16 in global memory, each 8-column group through Epi::apply8
-  const uint16_t* gv_a = nullptr;
-  const uint16_t* gv_b = nullptr;
-  int lda = 0, ldb = 0;
 };
 
-constexpr int kGemvRows = 8;
 constexpr int kSplitMax = 8;
 constexpr int kSplitRows = 2 * 128;
 constexpr int kSplitMinKBlocks = 4;
@@ -121,128 +114,6 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int&
   nb = within / gm;
 }
 
-// The rows-times-matrix product of a GEMM with at most kGemvRows rows: a tensor-
-// core tile would be 128 rows of which almost all are padding, and its K-split
-// pipeline is latency-bound, while this streams each row of B once from HBM.
-// Work is 8-column groups (one Epi::apply8 per row); lane l holds elements
-// l*8 .. l*8+7 of each 256-element K chunk, so a warp reads 512 contiguous
-// bytes of a row per load, and kGemvBatch chunks of the group's 8 rows are
-// loaded before any is used (enough bytes in flight to stream from HBM).
-//   * K <= kGemvWarpK: a warp owns whole groups (dealt over all warps of the
-//     grid); its lanes' sums meet by shuffles and lane i applies row i.
-//   * larger K: a CTA owns a group (dealt over the CTAs), its warps take the
-//     chunk batches round robin, and their sums meet in shared memory, added
-//     in warp order by thread i for row i.
-// The order of every sum is fixed, so the result is the same on every run.
-constexpr int kGemvBatch = 4;
-constexpr int kGemvWarpK = 4096;
-
-template <int U>
-__device__ __forceinline__ void gemv_chunks(const GemmShape& shp, int M_eff, int n0, int q0, int qstep, int nchunks,
-                                            int lane, float (&acc)[kGemvRows][8]) {
-  const int K = shp.K0, N = shp.N;
-  for (int q = q0; q < nchunks; q += qstep * U) {
-    uint4 b[U][8];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int k = (q + u * qstep) * 256 + lane * 8;  // K is a multiple of 64: k < K means k + 8 <= K
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        b[u][c] = (k < K && n0 + c < N)
-                      ? __ldg(reinterpret_cast<const uint4*>(shp.gv_b + static_cast<size_t>(n0 + c) * shp.ldb + k))
-                      : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int k = (q + u * qstep) * 256 + lane * 8;
-      if (k >= K) continue;
-#pragma unroll
-      for (int i = 0; i < kGemvRows; ++i) {
-        if (i >= M_eff) break;
-        const uint4 a = __ldg(reinterpret_cast<const uint4*>(shp.gv_a + static_cast<size_t>(i) * shp.lda + k));
-        const uint32_t av[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t bv[4] = {b[u][c].x, b[u][c].y, b[u][c].z, b[u][c].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
-                "mov.b32 {al, ah}, %1;\n\t"
-                "mov.b32 {bl, bh}, %2;\n\t"
-                "fma.rn.f32.bf16 %0, al, bl, %0;\n\t"
-                "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
-                : "+f"(acc[i][c])
-                : "r"(av[e]), "r"(bv[e]));
-          }
-        }
-      }
-    }
-  }
-}
-
-template <class Epi>
-__device__ __forceinline__ void gemv_rows(const GemmShape& shp, const typename Epi::Args& ea, int M_eff,
-                                          float* red) {
-  constexpr int W = kGemmThreads / 32;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int K = shp.K0, N = shp.N;
-  const int nchunks = (K + 255) / 256;
-  float acc[kGemvRows][8];
-  if (K <= kGemvWarpK) {
-    for (int n0 = (blockIdx.x * W + warp) * 8; n0 < N; n0 += gridDim.x * W * 8) {
-#pragma unroll
-      for (int i = 0; i < kGemvRows; ++i)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[i][c] = 0.f;
-      gemv_chunks<kGemvBatch>(shp, M_eff, n0, 0, 1, nchunks, lane, acc);
-#pragma unroll
-      for (int i = 0; i < kGemvRows; ++i) {
-        if (i >= M_eff) break;
-        float v[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          float t = acc[i][c];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
-          v[c] = t;
-        }
-        if (lane == i) Epi::apply8(ea, i, n0, v);
-      }
-    }
-    return;
-  }
-  for (int n0 = blockIdx.x * 8; n0 < N; n0 += gridDim.x * 8) {
-#pragma unroll
-    for (int i = 0; i < kGemvRows; ++i)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[i][c] = 0.f;
-    gemv_chunks<2>(shp, M_eff, n0, warp, W, nchunks, lane, acc);
-#pragma unroll
-    for (int i = 0; i < kGemvRows; ++i) {
-      if (i >= M_eff) break;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float v = acc[i][c];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-        if (lane == 0) red[(warp * kGemvRows + i) * 8 + c] = v;
-      }
-    }
-    __syncthreads();
-    if (threadIdx.x < M_eff) {
-      float v[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float t = 0.f;
-        for (int w = 0; w < W; ++w) t += red[(w * kGemvRows + threadIdx.x) * 8 + c];
-        v[c] = t;
-      }
-      Epi::apply8(ea, threadIdx.x, n0, v);
-    }
-    __syncthreads();
-  }
-}
-
 template <class Epi, int BN, bool B_MN, int STAGES, bool A_MN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
@@ -289,12 +160,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int nk0 = *k0_eff_s / kBK;
   const int nk = nk0 + shp.K1 / kBK;
   if (nk == 0) return;  // nothing to contract (a device-side K of zero)
-  if constexpr (Epi::kSplitK) {
-    if (shp.gv_b != nullptr && shp.K1 == 0 && shp.K_dev == nullptr && *m_eff_s <= kGemvRows) {
-      if (*m_eff_s > 0) gemv_rows<Epi>(shp, ea, *m_eff_s, reinterpret_cast<float*>(smem));
-      return;
-    }
-  }
   const int split = gemm_split(*m_eff_s, shp.N, BN, nk, shp, gridDim.x);
   if (static_cast<long>(blockIdx.x) >=
       static_cast<long>((*m_eff_s + kBM - 1) / kBM) * ((shp.N + BN - 1) / BN) * split)

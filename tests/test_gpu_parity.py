@@ -95,8 +95,7 @@ CASES = {
     # 170 overflow rows of a heavy-tailed batch: split-K dense backup GEMMs,
     # overflow pairs kept in the pair list
     "heavy_small": (1024, 1024, 4096, 8, 0.02, "lognormal", 23),
-    # 8 and 9 overflow rows: the dense backup's CUDA-core path (at most 8 rows)
-    # and, one row more, the tensor-core split-K path
+    # 8 and 9 overflow rows: split-K dense backup GEMMs of a few rows
     "ovf_rows_8": (384, 512, 2048, 8, 0.02, "none", 30),
     "ovf_rows_9": (384, 512, 2048, 8, 0.02, "none", 41),
 }
