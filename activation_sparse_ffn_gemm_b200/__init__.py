@@ -171,13 +171,16 @@ class HybridState:
         self.col = torch.empty((M, T, K), dtype=torch.uint8, device=dev)
         self.row_ovf = torch.empty(max(M, 1), dtype=torch.uint8, device=dev)
         self.ovf_rows = torch.empty(cap1, dtype=torch.int32, device=dev)
-        self.n_ovf = torch.zeros(2, dtype=torch.int32, device=dev)
+        # n_ovf, the status word and the row plan start at zero: one buffer, one fill,
+        # each part 16-byte aligned
+        n_plan = max(int(lib().twell_plan_ints(M, d_ff, T_n, K)), 1)
+        self._zeroed = torch.zeros(8 + n_plan, dtype=torch.int32, device=dev)
+        self.n_ovf = self._zeroed[0:2]
         self.g_ovf = torch.empty((cap1, d_ff), dtype=torch.bfloat16, device=dev)
         self.u_ell = torch.empty((M, T, K), dtype=torch.float32, device=dev) if with_u else None
         self.u_ovf = torch.empty((cap1, d_ff), dtype=torch.float32, device=dev) if with_u else None
-        self.status = torch.zeros(4, dtype=torch.int32, device=dev)
-        self.row_plan = torch.zeros(max(int(lib().twell_plan_ints(M, d_ff, T_n, K)), 1), dtype=torch.int32,
-                                    device=dev)
+        self.status = self._zeroed[4:8]
+        self.row_plan = self._zeroed[8:]
         self.c = TwellHybrid(M, d_ff, T_n, K, cap, int(dense_min), *(
             (t.data_ptr() if t is not None else None) for t in
             (self.count, self.val, self.col, self.row_ovf, self.ovf_rows, self.n_ovf, self.g_ovf, self.u_ell,

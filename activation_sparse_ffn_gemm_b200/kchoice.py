@@ -19,6 +19,14 @@ Row routing, candidate K:
     rows(K)  = sum of rows_by_max[c] over c > K        (dense backup rows)
     pairs(K) = sum of act_by_max[c] over c <= K        (units kept in ELL slots)
     t(K) = a * d * pairs(K) + r * d * f * rows(K) + (bytes of the slots) / BW
+           + [rows(K) > 0] * (fixed cost of the dense backup GEMMs)
+The fixed cost is what the backup GEMMs take beyond their empty launch as soon
+as one row overflows: per GEMM a launch and one pass over its weight matrix
+(the forward has two, the backward two more, dX with two matrices). The model
+takes a lower bound, 3 us plus the matrix at the HBM copy rate; B200 measured
+16-28 us per GEMM for a single row at d_model=2048, d_ff=8192. A bound keeps
+the heavy-tailed batches, where the model's pair cost is itself low for long
+rows, on the measured best K.
 Tile routing (inference only), every active unit is gathered and each tile
 over K is read from its spilled dense slice:
     t(K) = a * d * total + (bytes of the slots + 512 bytes per spilled tile) / BW
@@ -56,6 +64,15 @@ class CostModel:
     dense_fwd_s: float = 6.5e-15     # per dense row per d_model * d_ff element, forward
     dense_bwd_s: float = 1.04e-14    # the same, backward
     hbm_bytes_s: float = 6.5e12
+    gemm_launch_s: float = 3e-6        # a dense backup GEMM with any row, beyond its empty launch
+    weight_stream_bytes_s: float = 6.5e12  # one pass over a weight matrix by a few-row GEMM (bound)
+
+    def dense_fixed_s(self, d_model: int, d_ff: int, training: bool) -> float:
+        """Cost of the dense backup GEMMs as soon as one row overflows: up and
+        down in the forward, dH and dX (two weight matrices) in the backward."""
+        w = 2.0 * d_model * d_ff / self.weight_stream_bytes_s
+        fwd = 2 * (self.gemm_launch_s + w)
+        return fwd + ((self.gemm_launch_s + w) + (self.gemm_launch_s + 2 * w) if training else 0.0)
 
     @classmethod
     def for_shape(cls, d_model: int, d_ff: int) -> "CostModel":
@@ -110,7 +127,8 @@ def modelled_times(stats: Mapping[str, object], d_model: int, d_ff: int, T_n: in
         if routing == "rows":
             pairs = int(act_by_max[:K + 1].sum())
             rows = int(rows_by_max[K + 1:].sum())
-            out[K] = a * d_model * pairs + r * d_model * d_ff * rows + slots / model.hbm_bytes_s
+            out[K] = (a * d_model * pairs + r * d_model * d_ff * rows + slots / model.hbm_bytes_s
+                      + (model.dense_fixed_s(d_model, d_ff, training) if rows > 0 else 0.0))
         else:
             spilled = int(tiles_by_count[K + 1:].sum())
             out[K] = a * d_model * total + (slots + 512 * spilled) / model.hbm_bytes_s

@@ -899,8 +899,10 @@ def run_block(args, local):
     def dense_ffn(t):
         return (torch.relu(t @ W_g.T + b_g) * (t @ W_u.T)) @ W_d.T
 
-    def twell(t):
-        return tw.twell_ffn(t, W_g, b_g, W_u, W_d, K=K, lam=args.lam)
+    def twell_k(k_):
+        def ffn(t):
+            return tw.twell_ffn(t, W_g, b_g, W_u, W_d, K=k_, lam=args.lam)
+        return ffn
 
     def timed(body):
         for _ in range(max(3, args.warmup)):
@@ -932,21 +934,35 @@ def run_block(args, local):
         return body
 
     with torch.no_grad():
-        hn = rms(block(x, lambda t: torch.zeros_like(t)), n2)  # the FFN input of this block
-        activity = float(((hn.reshape(M, d) @ W_g.T + b_g) > 0).float().mean().item())
+        hn = rms(block(x, lambda t: torch.zeros_like(t)), n2).reshape(M, d)  # the FFN input of this block
+        activity = float(((hn @ W_g.T + b_g) > 0).float().mean().item())
+        # adaptive K: the count statistics of this batch's pack and the cost model (kchoice)
+        probe = tw.HybridState(M, f, 128, K, M, dev, with_u=False)
+        tw.pack(hn.contiguous(), W_g.detach(), b_g.detach(), T_n=128, K=K, state=probe)
+        stats = tw.count_stats(probe)
+        k_train = tw.suggest_k(stats, d, f, training=True)[0]
+        k_inf = tw.suggest_k(stats, d, f, training=False)[0]
+        overflow_k8 = probe.n_overflow()[1]
+        del probe
     res = {}
-    for name, ffn in (("dense_ffn", dense_ffn), ("twell_ffn", twell)):
-        res[name] = {"fwd_ms": timed(fwd(ffn)), "fwd_bwd_ms": timed(train(ffn))}
+    arms = (("dense_ffn", dense_ffn, dense_ffn), ("twell_ffn_k8", twell_k(K), twell_k(K)),
+            ("twell_ffn_adaptive_k", twell_k(k_inf), twell_k(k_train)))
+    for name, ffn_inf, ffn_train in arms:
+        res[name] = {"fwd_ms": timed(fwd(ffn_inf)), "fwd_bwd_ms": timed(train(ffn_train))}
         res[name]["fwd_tokens_per_s"] = M / (res[name]["fwd_ms"] / 1e3)
         res[name]["fwd_bwd_tokens_per_s"] = M / (res[name]["fwd_bwd_ms"] / 1e3)
+    res["twell_ffn_adaptive_k"]["K"] = {"fwd": k_inf, "fwd_bwd": k_train}
     print(json.dumps({
         "workload": f"pre-norm transformer block, batch {B} x seq {S} (M={M} tokens), d_model={d}, {heads} heads, "
-                    f"causal SDPA attention (torch), gated ReLU FFN d_ff={f}; TwELL FFN with T_n=128, K={K}, "
-                    f"L1 lambda={args.lam}",
+                    f"causal SDPA attention (torch), gated ReLU FFN d_ff={f}; TwELL FFN with T_n=128, K={K} or the "
+                    f"K chosen from the batch's count statistics, L1 lambda={args.lam}",
         "ffn_gate_activity": activity,
+        "ffn_overflow_rows_at_k8": overflow_k8,
         "block": res,
-        "speedup_vs_dense_block": {"fwd": res["dense_ffn"]["fwd_ms"] / res["twell_ffn"]["fwd_ms"],
-                                   "fwd_bwd": res["dense_ffn"]["fwd_bwd_ms"] / res["twell_ffn"]["fwd_bwd_ms"]},
+        "speedup_vs_dense_block": {
+            arm: {"fwd": res["dense_ffn"]["fwd_ms"] / res[arm]["fwd_ms"],
+                  "fwd_bwd": res["dense_ffn"]["fwd_bwd_ms"] / res[arm]["fwd_bwd_ms"]}
+            for arm in ("twell_ffn_k8", "twell_ffn_adaptive_k")},
         "steps": args.steps, "warmup": max(3, args.warmup), "l2": "flushed before every timed step",
         "data": "synthetic (random weights, seeded torch CUDA generator)"}), flush=True)
 

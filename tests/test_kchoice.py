@@ -21,7 +21,8 @@ def _stats(rows_by_max, act_by_max, tiles_by_count):
 
 # unit coefficients, so each term can be read off: pair = 1 s per d element,
 # dense row = 10 s per d*f element, 1 byte/s
-UNIT = CostModel(pair_fwd_s=1.0, pair_bwd_s=0.0, dense_fwd_s=10.0, dense_bwd_s=0.0, hbm_bytes_s=1.0)
+UNIT = CostModel(pair_fwd_s=1.0, pair_bwd_s=0.0, dense_fwd_s=10.0, dense_bwd_s=0.0, hbm_bytes_s=1.0,
+                 gemm_launch_s=0.0, weight_stream_bytes_s=1e300)
 
 
 def test_row_routing_terms_by_hand():
@@ -52,7 +53,8 @@ def test_tile_routing_terms_by_hand():
 
 def test_training_adds_backward_terms():
     st = _stats({10: 2}, {10: 12}, {10: 2, 1: 2})
-    m = CostModel(pair_fwd_s=1.0, pair_bwd_s=2.0, dense_fwd_s=4.0, dense_bwd_s=5.0, hbm_bytes_s=1e30)
+    m = CostModel(pair_fwd_s=1.0, pair_bwd_s=2.0, dense_fwd_s=4.0, dense_bwd_s=5.0, hbm_bytes_s=1e30,
+                  gemm_launch_s=0.0, weight_stream_bytes_s=1e300)
     t_inf = modelled_times(st, 1, 256, candidates=(8, 16), training=False, model=m)
     t_trn = modelled_times(st, 1, 256, candidates=(8, 16), training=True, model=m)
     assert t_inf[8] == pytest.approx(4.0 * 256 * 2) and t_trn[8] == pytest.approx(9.0 * 256 * 2)
@@ -63,7 +65,8 @@ def test_no_overflow_prefers_smallest_k_and_ties_go_small():
     st = _stats({3: 100}, {3: 500}, {3: 100, 0: 100})
     best, times = suggest_k(st, 2048, 256)
     assert best == 8 and times[8] < times[16] < times[32] < times[64]
-    free = CostModel(pair_fwd_s=0.0, pair_bwd_s=0.0, dense_fwd_s=0.0, dense_bwd_s=0.0, hbm_bytes_s=1e300)
+    free = CostModel(pair_fwd_s=0.0, pair_bwd_s=0.0, dense_fwd_s=0.0, dense_bwd_s=0.0, hbm_bytes_s=1e300,
+                     gemm_launch_s=0.0, weight_stream_bytes_s=1e300)
     assert suggest_k(st, 2048, 256, model=free)[0] == 8
 
 
@@ -72,7 +75,8 @@ def test_heavy_rows_trade_slots_for_dense_rows():
     to their gathers, and stay sparse at a large K when it is not."""
     st = _stats({4: 1000, 40: 10}, {4: 3000, 40: 10 * 2000}, {4: 1000, 40: 10, 0: 1010 * 111})
     d, f = 4096, 14336
-    cheap_dense = CostModel(pair_fwd_s=1e-12, pair_bwd_s=0.0, dense_fwd_s=1e-17, dense_bwd_s=0.0)
+    cheap_dense = CostModel(pair_fwd_s=1e-12, pair_bwd_s=0.0, dense_fwd_s=1e-17, dense_bwd_s=0.0, gemm_launch_s=0.0,
+                            weight_stream_bytes_s=1e300)
     dear_dense = CostModel(pair_fwd_s=1e-12, pair_bwd_s=0.0, dense_fwd_s=1e-12, dense_bwd_s=0.0)
     assert suggest_k(st, d, f, training=False, model=cheap_dense)[0] == 8
     assert suggest_k(st, d, f, training=False, model=dear_dense)[0] == 64
@@ -99,3 +103,22 @@ def test_dense_min_break_even():
             a = dense_min_for(d, f, training)
             # about 1-3% of the row active: above the 1% rows of the uniform workload's mean
             assert 0.01 * f < a < 0.03 * f, (d, f, training, a)
+
+
+def test_fixed_cost_of_the_first_overflow_row():
+    """One overflowing row at K=8 costs the backup GEMMs' fixed time; K=16 keeps it in ELL
+    slots for a few more slot bytes, so the uniform 1% batch picks K=16."""
+    m = CostModel(pair_fwd_s=1.0, pair_bwd_s=0.0, dense_fwd_s=0.0, dense_bwd_s=0.0, hbm_bytes_s=1.0,
+                  gemm_launch_s=3.0, weight_stream_bytes_s=2.0)
+    # fixed: forward 2 * (3 + 2*d*f/2) = 2 * (3 + 512) with d=2, f=256
+    assert m.dense_fixed_s(2, 256, False) == 2 * (3 + 512)
+    assert m.dense_fixed_s(2, 256, True) == 2 * (3 + 512) + (3 + 512) + (3 + 1024)
+    st = _stats({5: 3, 12: 1}, {5: 30, 12: 40}, {5: 3, 3: 3, 12: 1, 1: 1})
+    t = modelled_times(st, 2, 256, candidates=(8, 16), training=False, model=m)
+    assert t[8] == 1.0 * 2 * 30 + 4 * 2 * (2 + 3 * 8) + 2 * (3 + 512)
+    assert t[16] == 1.0 * 2 * 70 + 4 * 2 * (2 + 3 * 16)
+    # with the measured coefficients: 4095 rows of largest count <= 8, one row at 9
+    M, f, d = 4096, 8192, 2048
+    st = _stats({6: 4095, 9: 1}, {6: 4095 * 82, 9: 90}, {1: M * 64})
+    assert suggest_k(st, d, f, training=True)[0] == 16
+    assert suggest_k(st, d, f, training=False)[0] == 16
