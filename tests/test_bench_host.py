@@ -1,0 +1,106 @@
+"""Host logic of bench.py, without a GPU: the clock sampler's summary (with a
+fake NVML), the algorithmic work per kernel, the whole-step roofline and the
+committed DRAM-traffic records."""
+
+import json
+import sys
+import time
+import types
+
+import pytest
+
+import bench
+
+
+class _FakeNVML(types.ModuleType):
+    NVML_CLOCK_SM = 1
+
+    def __init__(self, clocks, reasons):
+        super().__init__("pynvml")
+        self.clocks, self.reasons, self.i = clocks, reasons, 0
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlDeviceGetHandleByUUID(self, uuid):
+        raise RuntimeError("no CUDA device here")
+
+    def nvmlDeviceGetHandleByIndex(self, index):
+        return ("gpu", index)
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        v = self.clocks[min(self.i, len(self.clocks) - 1)]
+        return v
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        r = self.reasons[min(self.i, len(self.reasons) - 1)]
+        self.i += 1
+        return r
+
+
+def test_clock_sampler_polls_nvml(monkeypatch):
+    fake = _FakeNVML([1800, 1950, 1965, 1965, 1965], [0, 0x4, 0, 0, 0])
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    with bench.ClockSampler(0) as clk:
+        t0 = time.time()
+        while len(clk.samples) < 5 and time.time() - t0 < 5:
+            time.sleep(0.005)
+    s = clk.summary()
+    assert s["source"].startswith("nvml") and s["samples"] >= 5
+    assert s["sm_max_mhz"] == 1965.0 and s["sm_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_sampler_reasons_by_bit():
+    clk = bench.ClockSampler(0)
+    clk.nvml = object()
+    clk.max_mhz = 1965.0
+    clk.samples = [(1300.0, 0x8 | 0x40), (1310.0, 0x20), (1320.0, 0)]
+    s = clk.summary()
+    assert s["sm_mhz"] == 1310.0
+    assert s["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"]
+
+
+def test_kernel_work_by_hand():
+    M, d, f, T, K, kept, pairs = 4, 8, 256, 2, 8, 10, 12
+    assert bench.kernel_work("gate_pack_gemm", M, d, f, T, K, kept, pairs) == ("tensor", 2.0 * 4 * 8 * 256)
+    # X + TwELL + u + Y + W_u and W_dt once
+    assert bench.kernel_work("ell_updown", M, d, f, T, K, kept, pairs) == (
+        "hbm", 2 * 32 + 4 * 2 * 26 + 40 + 2 * 32 + 4 * 256 * 8)
+    # X, TwELL, u, (dU, dZ) per slot, dX fp32, three weight matrices once
+    assert bench.kernel_work("ell_bwd", M, d, f, T, K, kept, pairs) == (
+        "hbm", 2 * 32 + 4 * 2 * 26 + 40 + 80 + 4 * 32 + 6 * 256 * 8)
+    assert bench.kernel_work("transpose_wd", M, d, f, T, K, kept, pairs) == ("hbm", 4 * 256 * 8)
+    assert bench.kernel_work("row_flags", M, d, f, T, K, kept, pairs) == (None, None)
+
+
+def test_path_roofline_fractions():
+    peaks = {"hbm_gbs": 1000.0, "bf16_tflops": 2.0, "bf16_tflops_sustained": 1.0}
+    r = bench.path_roofline(M=128, d=64, f=256, T=2, K=8, kept=100, n_ovf=0, peaks=peaks, ms_fwd=2.0, ms_step=5.0)
+    assert r["step_ms"] > r["fwd_ms"] > 0
+    assert r["fwd_frac"] == pytest.approx(r["fwd_ms"] / 2.0) and r["step_frac"] == pytest.approx(r["step_ms"] / 5.0)
+    # the gate GEMM's flops at the sustained rate are part of the forward's floor
+    assert r["fwd_ms"] >= 2.0 * 128 * 64 * 256 / 1e12 * 1e3
+
+
+def test_committed_traffic_follows_the_sources(monkeypatch):
+    with open(bench.os.path.join(bench.ROOT, "profiles", "dram_traffic.json")) as fh:
+        rec = json.load(fh)["kernels"]
+    for k, v in rec.items():
+        got = bench.committed_traffic(k)
+        if v["source_sha"] == bench.source_hash(k):
+            assert got == v["dram_bytes_per_launch"]
+        else:
+            assert got is None
+    monkeypatch.setattr(bench, "source_hash", lambda kernel: "changed")
+    assert all(bench.committed_traffic(k) is None for k in rec)
+
+
+def test_workload_is_the_uniform_shape_with_the_golden_seed():
+    w, seed = bench.workload()
+    assert (w.M, w.d_model, w.d_ff, w.T_n, w.K, w.activity) == (4096, 2048, 8192, 128, 8, 0.01)
+    with open(bench.os.path.join(bench.ROOT, "tests", "golden", "uniform_seed.json")) as fh:
+        assert seed == json.load(fh)["seed"]
