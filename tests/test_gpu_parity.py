@@ -95,6 +95,9 @@ CASES = {
     # 170 overflow rows of a heavy-tailed batch: split-K dense backup GEMMs,
     # overflow pairs kept in the pair list
     "heavy_small": (1024, 1024, 4096, 8, 0.02, "lognormal", 23),
+    # the supported extremes: d_ff = 16384 (128 tiles), d_model = 64
+    "max_d_ff": (40, 256, 16384, 8, 0.02, "none", 31),
+    "min_d_model": (50, 64, 256, 8, 0.05, "lognormal", 32),
     # 8 and 9 overflow rows: split-K dense backup GEMMs of a few rows
     "ovf_rows_8": (384, 512, 2048, 8, 0.02, "none", 30),
     "ovf_rows_9": (384, 512, 2048, 8, 0.02, "none", 41),
