@@ -221,7 +221,8 @@ TWELL_API twell_status twell_ffn_fwd(const uint16_t* X, const uint16_t* W_g, con
  * (an adaptive number of entries per tile). Same arguments and workspace as
  * twell_ffn_fwd; Y is the same function of the inputs.
  *   h   filled as by twell_pack except: row_ovf = 0 for every row, n_ovf = {0, 0},
- *       g_ovf, u_ell and u_ovf untouched. The state serves inference only:
+ *       g_ovf, u_ell and u_ovf untouched (h->dense_min plays no part: no row
+ *       goes dense under tile routing). The state serves inference only:
  *       twell_ffn_bwd given it sets TWELL_STATUS_BAD_STATE and writes nothing.
  */
 TWELL_API twell_status twell_ffn_fwd_tiles(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_g,
