@@ -235,30 +235,34 @@ __global__ void __launch_bounds__(256) csc_fill_kernel(
   }
 }
 
-// A CTA covers 8 consecutive units and a 256-column slice; each lane owns one
-// 16-byte chunk (8 columns). Its 4 warps take the 8 units one at a time from a
-// shared counter, longest pair list first, so a long list does not leave the
-// other warps waiting at the CTA's end. A warp stages its unit's list 32
-// entries at a time in shared memory (one coalesced load), then issues the x
-// and dY loads of kWgBatch pairs back to back; entries come from
-// shared-memory broadcasts and accumulation uses the two-lane FMA. Each unit's
-// sums are taken in list order, whichever warp runs it, so the result is the
-// same on every run. dW_d[:, j] is transposed through shared memory so that
-// each output row gets 8 consecutive units (32 bytes).
-constexpr int kWgBatch = 4;  // pairs whose row loads are issued together (2, 6, 8 measured slower)
-constexpr int kWgCols = 256;
+// A CTA covers 8 consecutive units and a kWgCols-column slice; each lane owns
+// kWgChunks 16-byte chunks (8 columns each, 256 columns apart). Its 4 warps
+// take the 8 units one at a time from a shared counter, longest pair list
+// first, so a long list does not leave the other warps waiting at the CTA's
+// end. A warp stages its unit's list 32 entries at a time in shared memory
+// (one coalesced load), then issues the x and dY loads of kWgBatch pairs back
+// to back; entries come from shared-memory broadcasts and accumulation uses the
+// two-lane FMA. Each unit's sums are taken in list order, whichever warp runs
+// it, so the result is the same on every run. dW_d[:, j] is transposed through
+// shared memory so that each output row gets 8 consecutive units (32 bytes).
+constexpr int kWgBatch = 4;   // pairs whose row loads are issued together (2, 6, 8 measured slower)
+constexpr int kWgChunks = 2;  // 16-byte chunks per lane and row: per-pair work amortised over 2 chunks
+constexpr int kWgCols = 256 * kWgChunks;
 constexpr int kWgUnits = 8;   // units per CTA
 constexpr int kWgWarps = 4;   // warps per CTA
+constexpr int kWgMinBlocks = kWgChunks == 1 ? 6 : 4;
 
-__global__ void __launch_bounds__(kWgWarps * 32, 6) wgrad_kernel(const uint16_t* __restrict__ X,
-                                                                 const uint16_t* __restrict__ dY,
-                                                                 const int* __restrict__ unit_ptr,
-                                                                 const int* __restrict__ csc_row,
-                                                                 const float4* __restrict__ csc_val, int d, int f,
-                                                                 const float* __restrict__ db_extra,
-                                                                 const int* __restrict__ accumulate,
-                                                                 float* __restrict__ dWg, float* __restrict__ dWu,
-                                                                 float* __restrict__ dWd, float* __restrict__ dbg) {
+__global__ void __launch_bounds__(kWgWarps * 32, kWgMinBlocks) wgrad_kernel(const uint16_t* __restrict__ X,
+                                                                            const uint16_t* __restrict__ dY,
+                                                                            const int* __restrict__ unit_ptr,
+                                                                            const int* __restrict__ csc_row,
+                                                                            const float4* __restrict__ csc_val, int d,
+                                                                            int f, const float* __restrict__ db_extra,
+                                                                            const int* __restrict__ accumulate,
+                                                                            float* __restrict__ dWg,
+                                                                            float* __restrict__ dWu,
+                                                                            float* __restrict__ dWd,
+                                                                            float* __restrict__ dbg) {
   __shared__ float s_dwd[kWgCols][kWgUnits + 1];
   __shared__ int s_row[kWgWarps][32];
   __shared__ float4 s_val[kWgWarps][32];
@@ -267,8 +271,13 @@ __global__ void __launch_bounds__(kWgWarps * 32, 6) wgrad_kernel(const uint16_t*
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j0 = blockIdx.x * kWgUnits;
   const int c0 = blockIdx.y * kWgCols;
-  const int cidx = (c0 >> 3) + lane;
-  const bool cval = cidx < (d >> 3);
+  int cidx[kWgChunks];
+  bool cval[kWgChunks];
+#pragma unroll
+  for (int q = 0; q < kWgChunks; ++q) {
+    cidx[q] = (c0 >> 3) + lane + 32 * q;
+    cval[q] = cidx[q] < (d >> 3);
+  }
   // add to the dense GEMMs' result (written before this kernel) instead of
   // overwriting: its lines are pulled into L2 now and read after the pair loops
   const bool acc_old = accumulate != nullptr && *accumulate > 0;
@@ -298,15 +307,19 @@ __global__ void __launch_bounds__(kWgWarps * 32, 6) wgrad_kernel(const uint16_t*
     if (u >= kWgUnits) break;
     const int lu = s_order[u];
     const int j = j0 + lu;
-    float* pu_out = dWu + static_cast<long>(j) * d + 8 * cidx;
-    float* pg_out = dWg + static_cast<long>(j) * d + 8 * cidx;
-    if (acc_old && cval) {
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(pu_out));
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(pg_out));
-    }
-    float2 au[4], ag[4], ad[4];
+    if (acc_old) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) au[e] = ag[e] = ad[e] = make_float2(0.f, 0.f);
+      for (int q = 0; q < kWgChunks; ++q)
+        if (cval[q]) {
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(dWu + static_cast<long>(j) * d + 8 * cidx[q]));
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(dWg + static_cast<long>(j) * d + 8 * cidx[q]));
+        }
+    }
+    float2 au[kWgChunks][4], ag[kWgChunks][4], ad[kWgChunks][4];
+#pragma unroll
+    for (int q = 0; q < kWgChunks; ++q)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) au[q][e] = ag[q][e] = ad[q][e] = make_float2(0.f, 0.f);
     float db = 0.f;
     const int p0 = unit_ptr[j], p1 = unit_ptr[j + 1];
     for (int pb = p0; pb < p1; pb += 32) {
@@ -320,55 +333,66 @@ __global__ void __launch_bounds__(kWgWarps * 32, 6) wgrad_kernel(const uint16_t*
       }
       __syncwarp();
       for (int b0 = 0; b0 < n; b0 += kWgBatch) {
-        uint4 xv[kWgBatch], dv[kWgBatch];
+        uint4 xv[kWgBatch][kWgChunks], dv[kWgBatch][kWgChunks];
 #pragma unroll
         for (int b = 0; b < kWgBatch; ++b) {
           const long r = s_row[w][min(b0 + b, n - 1)];
-          if (cval) {
-            xv[b] = __ldg(reinterpret_cast<const uint4*>(X + r * d) + cidx);
-            dv[b] = __ldg(reinterpret_cast<const uint4*>(dY + r * d) + cidx);
-          } else {
-            xv[b] = dv[b] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int q = 0; q < kWgChunks; ++q) {
+            if (cval[q]) {
+              xv[b][q] = __ldg(reinterpret_cast<const uint4*>(X + r * d) + cidx[q]);
+              dv[b][q] = __ldg(reinterpret_cast<const uint4*>(dY + r * d) + cidx[q]);
+            } else {
+              xv[b][q] = dv[b][q] = make_uint4(0, 0, 0, 0);
+            }
           }
         }
 #pragma unroll
         for (int b = 0; b < kWgBatch; ++b) {
           const float4 v = b0 + b < n ? s_val[w][b0 + b] : make_float4(0.f, 0.f, 0.f, 0.f);
           const float2 h2 = make_float2(v.x, v.x), u2 = make_float2(v.y, v.y), z2 = make_float2(v.z, v.z);
-          const uint32_t xw[4] = {xv[b].x, xv[b].y, xv[b].z, xv[b].w};
-          const uint32_t dw[4] = {dv[b].x, dv[b].y, dv[b].z, dv[b].w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 xf = bf16x2_to_f2(xw[e]);
-            au[e] = fma2(u2, xf, au[e]);
-            ag[e] = fma2(z2, xf, ag[e]);
-            ad[e] = fma2(h2, bf16x2_to_f2(dw[e]), ad[e]);
+          for (int q = 0; q < kWgChunks; ++q) {
+            const uint32_t xw[4] = {xv[b][q].x, xv[b][q].y, xv[b][q].z, xv[b][q].w};
+            const uint32_t dw[4] = {dv[b][q].x, dv[b][q].y, dv[b][q].z, dv[b][q].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 xf = bf16x2_to_f2(xw[e]);
+              au[q][e] = fma2(u2, xf, au[q][e]);
+              ag[q][e] = fma2(z2, xf, ag[q][e]);
+              ad[q][e] = fma2(h2, bf16x2_to_f2(dw[e]), ad[q][e]);
+            }
           }
         }
       }
     }
     db = warp_sum(db);
-    if (cval) {
-      float4* pu = reinterpret_cast<float4*>(pu_out);
-      float4* pg = reinterpret_cast<float4*>(pg_out);
-      float4 u0 = make_float4(au[0].x, au[0].y, au[1].x, au[1].y), u1 = make_float4(au[2].x, au[2].y, au[3].x, au[3].y);
-      float4 g0 = make_float4(ag[0].x, ag[0].y, ag[1].x, ag[1].y), g1 = make_float4(ag[2].x, ag[2].y, ag[3].x, ag[3].y);
-      if (acc_old) {
-        const float4 ou0 = pu[0], ou1 = pu[1], og0 = pg[0], og1 = pg[1];
-        u0 = make_float4(ou0.x + u0.x, ou0.y + u0.y, ou0.z + u0.z, ou0.w + u0.w);
-        u1 = make_float4(ou1.x + u1.x, ou1.y + u1.y, ou1.z + u1.z, ou1.w + u1.w);
-        g0 = make_float4(og0.x + g0.x, og0.y + g0.y, og0.z + g0.z, og0.w + g0.w);
-        g1 = make_float4(og1.x + g1.x, og1.y + g1.y, og1.z + g1.z, og1.w + g1.w);
-      }
-      pu[0] = u0;
-      pu[1] = u1;
-      pg[0] = g0;
-      pg[1] = g1;
-    }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      s_dwd[lane * 8 + 2 * e][lu] = ad[e].x;
-      s_dwd[lane * 8 + 2 * e + 1][lu] = ad[e].y;
+    for (int q = 0; q < kWgChunks; ++q) {
+      if (cval[q]) {
+        float4* pu = reinterpret_cast<float4*>(dWu + static_cast<long>(j) * d + 8 * cidx[q]);
+        float4* pg = reinterpret_cast<float4*>(dWg + static_cast<long>(j) * d + 8 * cidx[q]);
+        float4 u0 = make_float4(au[q][0].x, au[q][0].y, au[q][1].x, au[q][1].y);
+        float4 u1 = make_float4(au[q][2].x, au[q][2].y, au[q][3].x, au[q][3].y);
+        float4 g0 = make_float4(ag[q][0].x, ag[q][0].y, ag[q][1].x, ag[q][1].y);
+        float4 g1 = make_float4(ag[q][2].x, ag[q][2].y, ag[q][3].x, ag[q][3].y);
+        if (acc_old) {
+          const float4 ou0 = pu[0], ou1 = pu[1], og0 = pg[0], og1 = pg[1];
+          u0 = make_float4(ou0.x + u0.x, ou0.y + u0.y, ou0.z + u0.z, ou0.w + u0.w);
+          u1 = make_float4(ou1.x + u1.x, ou1.y + u1.y, ou1.z + u1.z, ou1.w + u1.w);
+          g0 = make_float4(og0.x + g0.x, og0.y + g0.y, og0.z + g0.z, og0.w + g0.w);
+          g1 = make_float4(og1.x + g1.x, og1.y + g1.y, og1.z + g1.z, og1.w + g1.w);
+        }
+        pu[0] = u0;
+        pu[1] = u1;
+        pg[0] = g0;
+        pg[1] = g1;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        s_dwd[256 * q + lane * 8 + 2 * e][lu] = ad[q][e].x;
+        s_dwd[256 * q + lane * 8 + 2 * e + 1][lu] = ad[q][e].y;
+      }
     }
     if (blockIdx.y == 0 && lane == 0 && dbg != nullptr) dbg[j] = db_extra ? db + db_extra[j] : db;
   }
