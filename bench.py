@@ -351,7 +351,8 @@ def run_reference(args, world, rank):
     inp = make_inputs(w, seed=seed, with_dY=True)
     O.build()
     # each step: the oracle's forward + backward on a bounded sample of rows
-    probe = cpu_baseline(inp, args.lam, target_s=max(1.0, 60.0 / max(1, args.steps + args.warmup)))
+    # the whole run is sized to about 5 x --cpu-seconds (60 s by default) of oracle work
+    probe = cpu_baseline(inp, args.lam, target_s=max(0.05, 5.0 * args.cpu_seconds / max(1, args.steps + args.warmup)))
     n = probe[1]
     rows = np.arange(n, dtype=np.int32)
 

@@ -104,3 +104,23 @@ def test_workload_is_the_uniform_shape_with_the_golden_seed():
     assert (w.M, w.d_model, w.d_ff, w.T_n, w.K, w.activity) == (4096, 2048, 8192, 128, 8, 0.01)
     with open(bench.os.path.join(bench.ROOT, "tests", "golden", "uniform_seed.json")) as fh:
         assert seed == json.load(fh)["seed"]
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` (the fp64 oracle on the host cores) prints one JSON
+    line with the contract's keys; a tiny --cpu-seconds keeps the sample small."""
+    import subprocess
+
+    out = subprocess.run([sys.executable, bench.os.path.join(bench.ROOT, "bench.py"), "--impl", "reference",
+                          "--steps", "1", "--warmup", "0", "--cpu-seconds", "0.05"],
+                         capture_output=True, text=True, timeout=600, cwd=bench.ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"]
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
