@@ -122,3 +122,27 @@ def test_fixed_cost_of_the_first_overflow_row():
     st = _stats({6: 4095, 9: 1}, {6: 4095 * 82, 9: 90}, {1: M * 64})
     assert suggest_k(st, d, f, training=True)[0] == 16
     assert suggest_k(st, d, f, training=False)[0] == 16
+
+
+def test_choice_from_oracle_statistics(orc):
+    """End to end on the host: the oracle packs a uniform 1% batch (the uniform
+    workload's shape of d_ff) in which a few rows overflow K=8 but none overflows
+    K=16; its statistics make suggest_k pick 16 (the backup GEMMs' fixed cost
+    outweighs the wider slots). A 4% batch, whose rows are past the break-even of a
+    dense row, keeps K=8 and sends its overflowing rows dense. With a row threshold
+    of 1 every row with an active unit lands in the threshold bin."""
+    rng = np.random.default_rng(3)
+    M, d, f = 4096, 2048, 8192
+    Z = rng.standard_normal((M, f)) - 2.326  # 1% active, 1.3 per 128-wide tile
+    p8, p16 = orc.pack(Z, T_n, 8), orc.pack(Z, T_n, 16)
+    assert p8["n_ovf_total"] > 0 and p16["n_ovf_total"] == 0
+    st = orc.count_stats(p8["count"], T_n)
+    assert st["rows_by_max"][9:].sum() == p8["n_ovf_total"]
+    best, times = suggest_k(st, d, f, training=True)
+    assert best == 16 and times[16] < times[8]
+    dense = orc.count_stats(p8["count"], T_n, dense_min=1)
+    assert dense["rows_by_max"][T_n + 1] == M - int((p8["count"].sum(1) == 0).sum())
+    Z4 = rng.standard_normal((512, f)) - 1.75  # 4% active: 330 per row, above the break-even
+    st4 = orc.count_stats(orc.pack(Z4, T_n, 8)["count"], T_n)
+    assert dense_min_for(d, f, training=True) < 330
+    assert suggest_k(st4, d, f, training=True)[0] == 8
