@@ -216,10 +216,19 @@ size_t twell_plan_ints(int64_t M, int64_t d_ff, int64_t T_n, int64_t K) {
   return static_cast<size_t>(plan_ints(M, d_ff / kTn, K));
 }
 
+// The pair list of the weight gradients addresses its entries with 32-bit
+// positions: at most (M - ovf_cap) * T * K entries from ELL rows and ovf_cap *
+// d_ff from dense rows.
+static bool pair_list_fits(int64_t M, int64_t d_ff, int64_t K, int64_t ovf_cap) {
+  const int64_t T = d_ff / kTn;
+  return (M - ovf_cap) * T * K + ovf_cap * d_ff <= static_cast<int64_t>(INT32_MAX);
+}
+
 size_t twell_workspace_bytes(twell_op op, int64_t M, int64_t d_model, int64_t d_ff, int64_t T_n, int64_t K,
                              int64_t ovf_cap) {
   if (twell_query_support(M, d_model, d_ff, T_n, K, ovf_cap) != TWELL_OK) return 0;
   if (op != TWELL_OP_PACK && op != TWELL_OP_FWD && op != TWELL_OP_BWD) return 0;
+  if (op == TWELL_OP_BWD && !pair_list_fits(M, d_ff, K, ovf_cap)) return 0;
   return ws_layout(op, M, d_model, d_ff, K, ovf_cap).total;
 }
 
@@ -310,6 +319,7 @@ twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_
                            size_t ws_bytes, twell_stream_t stream) {
   twell_status st = check_hybrid(h, d_model);
   if (st != TWELL_OK) return st;
+  if (!pair_list_fits(h->M, h->d_ff, h->K, h->ovf_cap)) return TWELL_EUNSUPPORTED;
   const void* wout[] = {dW_g, dW_u, dW_d};
   for (const void* p : wout)
     if (!p || !aligned16(p)) return TWELL_EINVAL;

@@ -238,6 +238,10 @@ TWELL_API twell_status twell_ffn_fwd_tiles(const uint16_t* X, const uint16_t* W_
  *   dY [M][d_model] bf16 bits; dX [M][d_model], dW_g / dW_u [d_ff][d_model],
  *   dW_d [d_model][d_ff], db_g [d_ff] (nullable): fp32, overwritten (not accumulated).
  *   ws  workspace of twell_workspace_bytes(TWELL_OP_BWD, ...) bytes
+ * TWELL_EUNSUPPORTED (and a zero TWELL_OP_BWD workspace size) when the weight
+ * gradients' pair list could exceed 2^31 - 1 entries, i.e. when
+ * (M - ovf_cap) * (d_ff / T_n) * K + ovf_cap * d_ff > 2^31 - 1 (its positions
+ * are 32-bit); a smaller ovf_cap or a split batch fits.
  */
 TWELL_API twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_t* W_u,
                            const uint16_t* W_d, const uint16_t* W_dt, int64_t d_model,

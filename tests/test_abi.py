@@ -137,3 +137,21 @@ def test_missing_library_fails_loudly(tw, monkeypatch):
     monkeypatch.setattr(tw, "LIB_PATH", os.path.join(ROOT, "does_not_exist", "libtwell.so"))
     with pytest.raises(RuntimeError, match="missing"):
         tw.lib()
+
+
+def test_pair_list_bound(tw):
+    """The weight gradients' pair list has 32-bit positions: a backward whose list
+    could pass 2^31 - 1 entries is refused before anything is enqueued, and its
+    workspace size is reported as 0 (the forward is unaffected)."""
+    L = tw.lib()
+    M, d, f, K = 1 << 18, 2048, 14336, 8
+    assert (M - M) * (f // 128) * K + M * f > 2 ** 31 - 1
+    assert tw.workspace_bytes(tw.OP_BWD, M, d, f, 128, K, M) == 0
+    assert tw.workspace_bytes(tw.OP_FWD, M, d, f, 128, K, M) > 0
+    assert tw.workspace_bytes(tw.OP_BWD, M, d, f, 128, K, 0) > 0  # 2^18 * 112 * 8 entries fit
+    assert tw.workspace_bytes(tw.OP_BWD, 65536, 4096, 14336, 128, 8, 65536) > 0  # the sweep's largest
+    fake = 1 << 20
+    p = ctypes.c_void_p(fake)
+    h = tw.TwellHybrid(M, f, 128, K, M, 0, *([fake] * 11))
+    assert L.twell_ffn_bwd(p, p, p, p, None, d, ctypes.byref(h), p, ctypes.c_float(0.0), p, p, p, p, None, p,
+                           1 << 40, None) == 2
