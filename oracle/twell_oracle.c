@@ -473,38 +473,63 @@ int oracle_ffn_bwd(const uint16_t* X, const uint16_t* Wg, const uint16_t* bg, co
     }
   }
   if (!err) {
-    /* weight gradients: i ascending for every output element (serial) */
+    /* weight gradients: for every output element the terms are added in
+     * ascending i, exactly as a loop over i would add them; the units are
+     * independent, so they are spread over threads after the per-row active
+     * lists are regrouped by unit (i ascending inside each unit's list). */
+    int64_t* uptr = (int64_t*)calloc((size_t)(f + 1), sizeof(int64_t));
+    int64_t tot = 0;
+    for (int64_t i = 0; i < M; ++i) tot += nact[i];
+    int64_t* urow = (int64_t*)malloc((size_t)(tot > 0 ? tot : 1) * sizeof(int64_t));
+    double* uval = (double*)malloc((size_t)(tot > 0 ? 3 * tot : 1) * sizeof(double));
     double* dWdT = (double*)calloc((size_t)(f * d), sizeof(double));
-    double* x = (double*)malloc((size_t)d * sizeof(double));
-    double* dy = (double*)malloc((size_t)d * sizeof(double));
-    if (!dWdT || !x || !dy) {
+    double* Xd = to_double(X, M * d);
+    double* dYd = to_double(dY, M * d);
+    if (!uptr || !urow || !uval || !dWdT || !Xd || !dYd) {
       err = 1;
     } else {
-      memset(dWg, 0, (size_t)(f * d) * sizeof(double));
-      memset(dWu, 0, (size_t)(f * d) * sizeof(double));
-      if (dbg) memset(dbg, 0, (size_t)f * sizeof(double));
-      for (int64_t i = 0; i < M; ++i) {
-        if (nact[i] == 0) continue;
-        oracle_bf16_to_double_array(X + i * d, x, d);
-        oracle_bf16_to_double_array(dY + i * d, dy, d);
-        for (int64_t a = 0; a < nact[i]; ++a) {
-          const int64_t j = act_j[i][a];
-          const double h = act_v[i][3 * a + 0], du = act_v[i][3 * a + 1], dz = act_v[i][3 * a + 2];
+      for (int64_t i = 0; i < M; ++i)
+        for (int64_t a = 0; a < nact[i]; ++a) uptr[act_j[i][a] + 1] += 1;
+      for (int64_t j = 0; j < f; ++j) uptr[j + 1] += uptr[j];
+      int64_t* fill = (int64_t*)malloc((size_t)(f > 0 ? f : 1) * sizeof(int64_t));
+      if (!fill) {
+        err = 1;
+      } else {
+        memcpy(fill, uptr, (size_t)f * sizeof(int64_t));
+        for (int64_t i = 0; i < M; ++i)
+          for (int64_t a = 0; a < nact[i]; ++a) {
+            const int64_t p = fill[act_j[i][a]]++;
+            urow[p] = i;
+            uval[3 * p + 0] = act_v[i][3 * a + 0];
+            uval[3 * p + 1] = act_v[i][3 * a + 1];
+            uval[3 * p + 2] = act_v[i][3 * a + 2];
+          }
+        free(fill);
+#pragma omp parallel for schedule(dynamic, 4)
+        for (int64_t j = 0; j < f; ++j) {
           double* gu = dWu + j * d;
           double* gg = dWg + j * d;
           double* gd = dWdT + j * d;
-          for (int64_t k = 0; k < d; ++k) {
-            gu[k] += du * x[k];
-            gg[k] += dz * x[k];
-            gd[k] += h * dy[k];
+          for (int64_t k = 0; k < d; ++k) { gu[k] = 0.0; gg[k] = 0.0; }
+          double db = 0.0;
+          for (int64_t p = uptr[j]; p < uptr[j + 1]; ++p) {
+            const double* x = Xd + urow[p] * d;
+            const double* dy = dYd + urow[p] * d;
+            const double h = uval[3 * p + 0], du = uval[3 * p + 1], dz = uval[3 * p + 2];
+            for (int64_t k = 0; k < d; ++k) {
+              gu[k] += du * x[k];
+              gg[k] += dz * x[k];
+              gd[k] += h * dy[k];
+            }
+            db += dz;
           }
-          if (dbg) dbg[j] += dz;
+          if (dbg) dbg[j] = db;
         }
+        for (int64_t j = 0; j < f; ++j)
+          for (int64_t c = 0; c < d; ++c) dWd[c * f + j] = dWdT[j * d + c];
       }
-      for (int64_t j = 0; j < f; ++j)
-        for (int64_t c = 0; c < d; ++c) dWd[c * f + j] = dWdT[j * d + c];
     }
-    free(dWdT); free(x); free(dy);
+    free(uptr); free(urow); free(uval); free(dWdT); free(Xd); free(dYd);
   }
   if (act_j) for (int64_t i = 0; i < M; ++i) free(act_j[i]);
   if (act_v) for (int64_t i = 0; i < M; ++i) free(act_v[i]);
