@@ -11,6 +11,7 @@ is raised.
 
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -22,13 +23,16 @@ from .kchoice import CostModel, dense_min_for, modelled_times, suggest_k  # noqa
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libtwell.so")
+# the same library compiled with -DTWELL_BOUNDS (index checks, STATUS_BOUNDS); see bounds_checked()
+BOUNDS_LIB_PATH = os.path.join(_PKG, "libtwell_bounds.so")
 
 OP_PACK, OP_FWD, OP_BWD = 0, 1, 2
 STATUS_OVERFLOW_CAP = 1 << 3
 STATUS_TIMEOUT = 1 << 5
 STATUS_BAD_STATE = 1 << 1  # a tile-routed (inference) state given to the backward
+STATUS_BOUNDS = 1 << 7  # bounds-checked build only: an index read from a buffer was out of range
 _STATUS_NAMES = {0: "TWELL_OK", 1: "TWELL_EINVAL", 2: "TWELL_EUNSUPPORTED", 3: "TWELL_EOVERFLOW_CAP",
-                 4: "TWELL_ECUDA", 5: "TWELL_ETIMEOUT", 6: "TWELL_EWORKSPACE"}
+                 4: "TWELL_ECUDA", 5: "TWELL_ETIMEOUT", 6: "TWELL_EWORKSPACE", 7: "TWELL_EBOUNDS"}
 
 _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -53,19 +57,22 @@ class TwellHybrid(ctypes.Structure):
                 ("u_ovf", _vp), ("status", _vp), ("row_plan", _vp)]
 
 
-_lock = threading.Lock()
-_lib = None
+_lock = threading.RLock()
+_libs = {}
+_use_bounds = 0
 
 
 def lib():
-    """Loads libtwell.so (built in-tree by activation_sparse_ffn_gemm_b200.build)."""
-    global _lib
+    """Loads libtwell.so (built in-tree by activation_sparse_ffn_gemm_b200.build),
+    or libtwell_bounds.so inside a bounds_checked() block."""
     with _lock:
-        if _lib is None:
-            if not os.path.exists(LIB_PATH):
-                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+        path = BOUNDS_LIB_PATH if _use_bounds else LIB_PATH
+        L = _libs.get(path)
+        if L is None:
+            if not os.path.exists(path):
+                raise RuntimeError(f"{path} is missing: build it with "
                                    "`python -m activation_sparse_ffn_gemm_b200.build`")
-            L = ctypes.CDLL(LIB_PATH)
+            L = ctypes.CDLL(path)
             L.twell_status_string.restype = ctypes.c_char_p
             L.twell_status_string.argtypes = [ctypes.c_int]
             L.twell_query_support.restype = ctypes.c_int
@@ -96,11 +103,32 @@ def lib():
             L.twell_trace_collect.argtypes = [ctypes.POINTER(TwellTraceRec), ctypes.c_int]
             L.twell_count_stats.restype = ctypes.c_int
             L.twell_count_stats.argtypes = [ctypes.POINTER(TwellHybrid), _vp, _vp, _vp, _vp]
+            L.twell_test_withhold_epilogue_arrival.restype = None
+            L.twell_test_withhold_epilogue_arrival.argtypes = [ctypes.c_int]
             L.twell_status_read.restype = ctypes.c_int
             L.twell_status_read.argtypes = [ctypes.POINTER(TwellHybrid), ctypes.POINTER(ctypes.c_uint32),
                                             ctypes.c_int, _vp]
-            _lib = L
-    return _lib
+            _libs[path] = L
+    return L
+
+
+@contextlib.contextmanager
+def bounds_checked():
+    """Within the block every call of this binding runs in libtwell_bounds.so, the
+    library compiled with index checks: each index a kernel reads from a buffer
+    (in-tile column, piece row, overflow row, dense slot, pair-list row and
+    position) is checked against the extent it addresses, and an index out of
+    range sets STATUS_BOUNDS in the state's status word instead of being used.
+    Results are otherwise those of libtwell.so (the checks change no arithmetic).
+    A test and debugging aid (compute-sanitizer stands in for nothing here)."""
+    global _use_bounds
+    with _lock:
+        _use_bounds += 1
+    try:
+        yield lib()
+    finally:
+        with _lock:
+            _use_bounds -= 1
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -128,6 +156,14 @@ def launch_count() -> int:
     return int(lib().twell_launch_count())
 
 
+def test_withhold_epilogue_arrival(launches: int) -> None:
+    """Failure-detection test aid (twell_test_withhold_epilogue_arrival): the next
+    `launches` split-capable dense-backup GEMM launches run with one epilogue warp
+    that never reaches the split-K barrier, so its bounded wait runs out and the
+    kernel sets TWELL_STATUS_TIMEOUT."""
+    lib().twell_test_withhold_epilogue_arrival(int(launches))
+
+
 def trace_enable(on: bool = True) -> None:
     lib().twell_trace_enable(1 if on else 0)
 
@@ -147,10 +183,15 @@ def workspace_bytes(op: int, M: int, d_model: int, d_ff: int, T_n: int, K: int, 
     return int(lib().twell_workspace_bytes(op, M, d_model, d_ff, T_n, K, ovf_cap))
 
 
-def workspace(op: int, M: int, d_model: int, d_ff: int, T_n: int, K: int, ovf_cap: int, device=None) -> torch.Tensor:
+def workspace(op: int, M: int, d_model: int, d_ff: int, T_n: int, K: int, ovf_cap: int, device=None,
+              alloc=None) -> torch.Tensor:
+    """Workspace of `op` for this shape; alloc(shape, dtype), when given, supplies
+    the (256-byte aligned) memory instead of torch.empty on `device`."""
     n = workspace_bytes(op, M, d_model, d_ff, T_n, K, ovf_cap)
     if n == 0 and query_support(M, d_model, d_ff, T_n, K, ovf_cap) != 0:
         _check(query_support(M, d_model, d_ff, T_n, K, ovf_cap), "workspace")
+    if alloc is not None:
+        return alloc((max(n, 256),), torch.uint8)
     return torch.empty(max(n, 256), dtype=torch.uint8, device=device or "cuda")
 
 
@@ -158,27 +199,33 @@ class HybridState:
     """Device buffers of one hybrid TwELL representation (see struct twell_hybrid)."""
 
     def __init__(self, M: int, d_ff: int, T_n: int = 128, K: int = 8, ovf_cap: Optional[int] = None,
-                 device=None, with_u: bool = True, dense_min: int = 0):
+                 device=None, with_u: bool = True, dense_min: int = 0, alloc=None):
         """dense_min > 0 also routes rows with at least that many active units to
-        the dense backup (kchoice.dense_min_for gives the measured break-even)."""
+        the dense backup (kchoice.dense_min_for gives the measured break-even).
+        alloc(shape, dtype), when given, supplies each array's (16-byte aligned)
+        memory instead of torch.empty on `device`."""
         dev = torch.device(device or "cuda")
+        if alloc is None:
+            def alloc(shape, dtype):
+                return torch.empty(shape, dtype=dtype, device=dev)
         T = d_ff // T_n
         cap = M if ovf_cap is None else int(ovf_cap)
         cap1 = max(cap, 1)
         self.M, self.d_ff, self.T_n, self.K, self.ovf_cap, self.dense_min = M, d_ff, T_n, K, cap, int(dense_min)
-        self.count = torch.empty((M, T), dtype=torch.int16, device=dev)
-        self.val = torch.empty((M, T, K), dtype=torch.bfloat16, device=dev)
-        self.col = torch.empty((M, T, K), dtype=torch.uint8, device=dev)
-        self.row_ovf = torch.empty(max(M, 1), dtype=torch.uint8, device=dev)
-        self.ovf_rows = torch.empty(cap1, dtype=torch.int32, device=dev)
+        self.count = alloc((M, T), torch.int16)
+        self.val = alloc((M, T, K), torch.bfloat16)
+        self.col = alloc((M, T, K), torch.uint8)
+        self.row_ovf = alloc((max(M, 1),), torch.uint8)
+        self.ovf_rows = alloc((cap1,), torch.int32)
         # n_ovf, the status word and the row plan start at zero: one buffer, one fill,
         # each part 16-byte aligned
         n_plan = max(int(lib().twell_plan_ints(M, d_ff, T_n, K)), 1)
-        self._zeroed = torch.zeros(8 + n_plan, dtype=torch.int32, device=dev)
+        self._zeroed = alloc((8 + n_plan,), torch.int32)
+        self._zeroed.zero_()
         self.n_ovf = self._zeroed[0:2]
-        self.g_ovf = torch.empty((cap1, d_ff), dtype=torch.bfloat16, device=dev)
-        self.u_ell = torch.empty((M, T, K), dtype=torch.float32, device=dev) if with_u else None
-        self.u_ovf = torch.empty((cap1, d_ff), dtype=torch.float32, device=dev) if with_u else None
+        self.g_ovf = alloc((cap1, d_ff), torch.bfloat16)
+        self.u_ell = alloc((M, T, K), torch.float32) if with_u else None
+        self.u_ovf = alloc((cap1, d_ff), torch.float32) if with_u else None
         self.status = self._zeroed[4:8]
         self.row_plan = self._zeroed[8:]
         self.c = TwellHybrid(M, d_ff, T_n, K, cap, int(dense_min), *(

@@ -214,14 +214,18 @@ struct EpiGateMul {
 // ----------------------------- row-scatter epilogues (bf16 out / fp32 out)
 struct EpiScatterBf16 {
   struct Args {
-    const int* rows;  // destination row of each GEMM row
+    const int* rows;  // destination row of each GEMM row (< rows_out)
     uint16_t* out;
     int ld;
+    int rows_out;
+    uint32_t* status;
   };
   static constexpr int SMEM_BYTES = 0;
   static constexpr bool kSplitK = true;
   __device__ static void apply8(const Args& a, int row, int n, const float (&v)[8]) {
-    *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(a.rows[row]) * a.ld + n) =
+    const int dst = a.rows[row];
+    if (!in_bounds(dst >= 0 && dst < a.rows_out, a.status)) return;
+    *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(dst) * a.ld + n) =
         make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
   }
   __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
@@ -231,14 +235,18 @@ struct EpiScatterBf16 {
 
 struct EpiScatterF32 {
   struct Args {
-    const int* rows;
+    const int* rows;  // destination row of each GEMM row (< rows_out)
     float* out;
     int ld;
+    int rows_out;
+    uint32_t* status;
   };
   static constexpr int SMEM_BYTES = 0;
   static constexpr bool kSplitK = true;
   __device__ static void apply8(const Args& a, int row, int n, const float (&v)[8]) {
-    float4* p = reinterpret_cast<float4*>(a.out + static_cast<size_t>(a.rows[row]) * a.ld + n);
+    const int dst = a.rows[row];
+    if (!in_bounds(dst >= 0 && dst < a.rows_out, a.status)) return;
+    float4* p = reinterpret_cast<float4*>(a.out + static_cast<size_t>(dst) * a.ld + n);
     p[0] = make_float4(v[0], v[1], v[2], v[3]);
     p[1] = make_float4(v[4], v[5], v[6], v[7]);
   }
@@ -351,7 +359,7 @@ size_t splitk_partial_floats(int cap, int d, int f) {
 size_t splitk_arrival_words() { return kSplitTiles; }
 
 cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uint16_t* W_d,
-                           const uint16_t* g_ovf, const int* ovf_rows, const int* n_ovf, int cap, int d, int f,
+                           const uint16_t* g_ovf, const int* ovf_rows, const int* n_ovf, int cap, int M, int d, int f,
                            uint16_t* h_ovf, float* u_ovf, uint16_t* Y, const SplitKBuffers& sk, uint32_t* status,
                            cudaStream_t s) {
   if (cap <= 0) return cudaSuccess;
@@ -368,13 +376,13 @@ cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uin
   if (e != cudaSuccess) return e;
   GemmShape s2{cap, n_ovf, d, f, 0, status};
   use_split(s2, sk, cap);
-  EpiScatterBf16::Args e2{ovf_rows, Y, d};
+  EpiScatterBf16::Args e2{ovf_rows, Y, d, M, status};
   return launch_umma_gemm<EpiScatterBf16, 256, false, kStages>("ovf_down_gemm", ta2, tb2, ta2, tb2, s2, e2, s);
 }
 
 cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const uint16_t* W_u,
                            const uint16_t* W_g, const uint16_t* g_ovf, const float* u_ovf, float lambda,
-                           const int* ovf_rows, const int* n_ovf, int cap, int d, int f, uint16_t* duz_ovf,
+                           const int* ovf_rows, const int* n_ovf, int cap, int M, int d, int f, uint16_t* duz_ovf,
                            float* du_ovf, float* dz_ovf, float* dX, const SplitKBuffers& sk, uint32_t* status,
                            cudaStream_t s) {
   if (cap <= 0) return cudaSuccess;
@@ -395,7 +403,7 @@ cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const u
   if (e != cudaSuccess) return e;
   GemmShape s2{cap, n_ovf, d, f, f, status};
   use_split(s2, sk, cap);
-  EpiScatterF32::Args e2{ovf_rows, dX, d};
+  EpiScatterF32::Args e2{ovf_rows, dX, d, M, status};
   return launch_umma_gemm<EpiScatterF32, 256, true, kStages>("ovf_dx_gemm", tdu, twu, tdz, twg, s2, e2, s);
 }
 

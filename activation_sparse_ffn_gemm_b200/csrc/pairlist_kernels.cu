@@ -40,16 +40,19 @@ template <typename Fn>
 __device__ __forceinline__ void for_row_entries(long r, int t, int T, int K, int f, const uint16_t* __restrict__ count,
                                                 const uint8_t* __restrict__ col, const uint8_t* __restrict__ row_ovf,
                                                 const int* __restrict__ row_slot, const uint16_t* __restrict__ g_ovf,
-                                                bool dense_ovf, Fn&& fn) {
+                                                bool dense_ovf, int cap, uint32_t* status, Fn&& fn) {
   if (!row_ovf[r]) {
     const int c0 = count[r * T + t];
     const int n = c0 < K ? c0 : K;
     const long base = (r * T + t) * K;
-    for (int s = 0; s < n; ++s) fn(static_cast<int>(col[base + s]), base + s);
+    for (int s = 0; s < n; ++s) {
+      const int c = col[base + s];
+      if (in_bounds(c < kTn, status)) fn(c, base + s);
+    }
   } else {
     if (dense_ovf) return;
     const int sl = row_slot[r];
-    if (sl < 0) return;
+    if (sl < 0 || !in_bounds(sl < cap, status)) return;
     const uint4* gp = reinterpret_cast<const uint4*>(g_ovf + static_cast<long>(sl) * f + t * kTn);
     for (int q = 0; q < kTn / 8; ++q) {
       const uint4 v = gp[q];
@@ -70,8 +73,8 @@ __global__ void __launch_bounds__(256) csc_count_kernel(const uint16_t* __restri
                                                         const uint8_t* __restrict__ row_ovf,
                                                         const int* __restrict__ row_slot,
                                                         const uint16_t* __restrict__ g_ovf,
-                                                        const int* __restrict__ plan, int M, int f, int K,
-                                                        int* __restrict__ chunk_cnt) {
+                                                        const int* __restrict__ plan, int M, int f, int K, int cap,
+                                                        int* __restrict__ chunk_cnt, uint32_t* status) {
   __shared__ uint32_t mask[8][kTn];
   __shared__ int cnt_s[kTn];
   const int t = blockIdx.x, chunk = blockIdx.y, T = f / kTn;
@@ -85,7 +88,7 @@ __global__ void __launch_bounds__(256) csc_count_kernel(const uint16_t* __restri
     for (int q = 0; q < kTn / 32; ++q) mask[w][lane + 32 * q] = 0u;
     __syncwarp();
     if (r < M)
-      for_row_entries(r, t, T, K, f, count, col, row_ovf, row_slot, g_ovf, dense_ovf,
+      for_row_entries(r, t, T, K, f, count, col, row_ovf, row_slot, g_ovf, dense_ovf, cap, status,
                       [&](int c, long) { atomicOr(&mask[w][c], 1u << lane); });
     __syncwarp();
 #pragma unroll
@@ -189,7 +192,7 @@ __global__ void __launch_bounds__(256) csc_fill_kernel(
     const float* __restrict__ u_ovf, const float4* __restrict__ hdz_ell, const float* __restrict__ du_ovf,
     const float* __restrict__ dz_ovf,
     const int* __restrict__ chunk_base, const int* __restrict__ unit_ptr, const int* __restrict__ plan, int M, int f,
-    int K, int* __restrict__ csc_row, float4* __restrict__ csc_val) {
+    int K, int cap, long long nnz_cap, int* __restrict__ csc_row, float4* __restrict__ csc_val, uint32_t* status) {
   __shared__ uint32_t mask[kCscGroups][kTn];
   __shared__ int gbase[kCscGroups][kTn];
   const int t = blockIdx.x, chunk = blockIdx.y, T = f / kTn;
@@ -201,7 +204,7 @@ __global__ void __launch_bounds__(256) csc_fill_kernel(
     for (int q = 0; q < kTn / 32; ++q) mask[g][lane + 32 * q] = 0u;
     __syncwarp();
     if (r < M)
-      for_row_entries(r, t, T, K, f, count, col, row_ovf, row_slot, g_ovf, dense_ovf,
+      for_row_entries(r, t, T, K, f, count, col, row_ovf, row_slot, g_ovf, dense_ovf, cap, status,
                       [&](int c, long) { atomicOr(&mask[g][c], 1u << lane); });
   }
   __syncthreads();
@@ -219,8 +222,9 @@ __global__ void __launch_bounds__(256) csc_fill_kernel(
     const long r = static_cast<long>(chunk) * kCscRows + g * 32 + lane;
     if (r >= M) continue;
     const int sl = row_ovf[r] ? row_slot[r] : -1;
-    for_row_entries(r, t, T, K, f, count, col, row_ovf, row_slot, g_ovf, dense_ovf, [&](int c, long slot) {
+    for_row_entries(r, t, T, K, f, count, col, row_ovf, row_slot, g_ovf, dense_ovf, cap, status, [&](int c, long slot) {
       const int p = gbase[g][c] + __popc(mask[g][c] & below);
+      if (!in_bounds(p >= 0 && p < nnz_cap, status)) return;
       float4 v;
       if (slot >= 0) {
         v = hdz_ell[slot];
@@ -256,8 +260,10 @@ __global__ void __launch_bounds__(kWgWarps * 32, kWgMinBlocks) wgrad_kernel(cons
                                                                             const uint16_t* __restrict__ dY,
                                                                             const int* __restrict__ unit_ptr,
                                                                             const int* __restrict__ csc_row,
-                                                                            const float4* __restrict__ csc_val, int d,
-                                                                            int f, const float* __restrict__ db_extra,
+                                                                            const float4* __restrict__ csc_val, int M,
+                                                                            long long nnz_cap, int d, int f,
+                                                                            uint32_t* status,
+                                                                            const float* __restrict__ db_extra,
                                                                             const int* __restrict__ accumulate,
                                                                             float* __restrict__ dWg,
                                                                             float* __restrict__ dWu,
@@ -321,13 +327,16 @@ __global__ void __launch_bounds__(kWgWarps * 32, kWgMinBlocks) wgrad_kernel(cons
 #pragma unroll
       for (int e = 0; e < 4; ++e) au[q][e] = ag[q][e] = ad[q][e] = make_float2(0.f, 0.f);
     float db = 0.f;
-    const int p0 = unit_ptr[j], p1 = unit_ptr[j + 1];
+    int p0 = unit_ptr[j], p1 = unit_ptr[j + 1];
+    if (!in_bounds(p0 >= 0 && p0 <= p1 && p1 <= nnz_cap, status)) p0 = p1 = 0;
     for (int pb = p0; pb < p1; pb += 32) {
       const int n = min(32, p1 - pb);
       __syncwarp();
       if (lane < n) {
-        s_row[w][lane] = csc_row[pb + lane];
-        const float4 v = csc_val[pb + lane];
+        const int r = csc_row[pb + lane];
+        const bool ok = in_bounds(r >= 0 && r < M, status);
+        s_row[w][lane] = ok ? r : 0;
+        const float4 v = ok ? csc_val[pb + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
         s_val[w][lane] = v;
         db += v.z;
       }
@@ -430,13 +439,15 @@ __device__ __forceinline__ void split_hi_lo(const float (&v)[8], uint4& hi, uint
 }
 
 __global__ void ovf_operands_kernel(const int* __restrict__ n_ovf, const int* __restrict__ ovf_rows,
-                                    const int* __restrict__ plan, int d, int f, const uint16_t* __restrict__ X,
+                                    const int* __restrict__ plan, int cap, int M, int d, int f, uint32_t* status,
+                                    const uint16_t* __restrict__ X,
                                     const uint16_t* __restrict__ dy_ovf, const float* __restrict__ du_ovf,
                                     const float* __restrict__ dz_ovf, const uint16_t* __restrict__ g_ovf,
                                     const float* __restrict__ u_ovf, DenseWgradOperands op, float* __restrict__ db_ovf,
                                     int* __restrict__ k_rows) {
   const bool dense = plan[3] != 0;
-  const int n = dense ? n_ovf[0] : 0;
+  int n = dense ? n_ovf[0] : 0;
+  if (!in_bounds(n <= cap, status)) n = cap;
   const int np = (n + 63) / 64 * 64;
   if (blockIdx.x == 0 && threadIdx.x == 0) *k_rows = n > 0 ? np + n : 0;
   for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < f; j += gridDim.x * blockDim.x) {
@@ -446,10 +457,11 @@ __global__ void ovf_operands_kernel(const int* __restrict__ n_ovf, const int* __
   }
   const uint4 z = make_uint4(0, 0, 0, 0);
   for (int sl = blockIdx.x; sl < np; sl += gridDim.x) {
-    const bool live = sl < n;
+    const int src_row = sl < n ? ovf_rows[sl] : 0;
+    const bool live = sl < n && in_bounds(src_row >= 0 && src_row < M, status);
     const long r_hi = sl, r_lo = static_cast<long>(np) + sl;
     {
-      const uint4* xi = live ? reinterpret_cast<const uint4*>(X + static_cast<long>(ovf_rows[sl]) * d) : nullptr;
+      const uint4* xi = live ? reinterpret_cast<const uint4*>(X + static_cast<long>(src_row) * d) : nullptr;
       const uint4* yi = live ? reinterpret_cast<const uint4*>(dy_ovf + static_cast<long>(sl) * d) : nullptr;
       uint4* xh = reinterpret_cast<uint4*>(op.x2 + r_hi * d);
       uint4* xl = reinterpret_cast<uint4*>(op.x2 + r_lo * d);
@@ -494,15 +506,15 @@ __global__ void ovf_operands_kernel(const int* __restrict__ n_ovf, const int* __
 
 }  // namespace
 
-cudaError_t launch_ovf_operands(const int* n_ovf, const int* ovf_rows, const int* plan, int cap, int d, int f,
+cudaError_t launch_ovf_operands(const int* n_ovf, const int* ovf_rows, const int* plan, int cap, int M, int d, int f,
                                 const uint16_t* X, const uint16_t* dy_ovf, const float* du_ovf, const float* dz_ovf,
                                 const uint16_t* g_ovf, const float* u_ovf, const DenseWgradOperands& op,
-                                float* db_ovf, int* k_rows, cudaStream_t s) {
+                                float* db_ovf, int* k_rows, uint32_t* status, cudaStream_t s) {
   if (cap <= 0) return cudaSuccess;
   const int g = device_sm_count() * 2;
   TWELL_LAUNCH("ovf_operands", s,
-               ovf_operands_kernel<<<g, 256, 0, s>>>(n_ovf, ovf_rows, plan, d, f, X, dy_ovf, du_ovf, dz_ovf, g_ovf,
-                                                     u_ovf, op, db_ovf, k_rows));
+               ovf_operands_kernel<<<g, 256, 0, s>>>(n_ovf, ovf_rows, plan, cap, M, d, f, status, X, dy_ovf, du_ovf, dz_ovf,
+                                                     g_ovf, u_ovf, op, db_ovf, k_rows));
   return cudaGetLastError();
 }
 
@@ -515,14 +527,14 @@ cudaError_t launch_build_csc(const uint16_t* count, const uint8_t* col, const ui
   const int T = f / kTn;
   TWELL_LAUNCH("csc_count", s,
                csc_count_kernel<<<dim3(T, nch), 256, 0, s>>>(count, col, row_ovf, b.row_slot, g_ovf, plan, M, f,
-                                                            K, b.block_cnt));
+                                                            K, b.cap, b.block_cnt, b.status));
   TWELL_LAUNCH("csc_scan", s,
                csc_scan_kernel<<<(f + kScanBlock - 1) / kScanBlock, kScanBlock, 0, s>>>(
                    b.block_cnt, nch, f, b.unit_tot, b.unit_ptr, b.arrive, next_launch_epoch() & ((1ull << 40) - 1)));
   TWELL_LAUNCH("csc_fill", s,
                csc_fill_kernel<<<dim3(T, nch), 256, 0, s>>>(count, col, row_ovf, b.row_slot, g_ovf, u_ovf,
                                                            hdz_ell, du_ovf, dz_ovf, b.block_cnt, b.unit_ptr, plan,
-                                                           M, f, K, b.csc_row, b.csc_val));
+                                                           M, f, K, b.cap, b.nnz_cap, b.csc_row, b.csc_val, b.status));
   return cudaGetLastError();
 }
 
@@ -531,8 +543,9 @@ cudaError_t launch_weight_grads(const uint16_t* X, const uint16_t* dY, const Csc
                                 float* dW_d, float* db_g, cudaStream_t s) {
   dim3 grid(f / kWgUnits, (d + kWgCols - 1) / kWgCols);
   TWELL_LAUNCH("weight_grads", s,
-               wgrad_kernel<<<grid, kWgWarps * 32, 0, s>>>(X, dY, b.unit_ptr, b.csc_row, b.csc_val, d, f, db_extra, accumulate,
-                                                 dW_g, dW_u, dW_d, db_g));
+               wgrad_kernel<<<grid, kWgWarps * 32, 0, s>>>(X, dY, b.unit_ptr, b.csc_row, b.csc_val, b.M, b.nnz_cap, d, f,
+                                                           b.status,
+                                                           db_extra, accumulate, dW_g, dW_u, dW_d, db_g));
   return cudaGetLastError();
 }
 

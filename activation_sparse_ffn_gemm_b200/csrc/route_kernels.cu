@@ -218,13 +218,15 @@ __global__ void __launch_bounds__(kScanThreads) route_plan_kernel(int* __restric
 // optionally x_ovf[s] = X[row]. One block per slot, grid-stride over slots.
 __global__ void ovf_gather_kernel(const int* __restrict__ n_ovf, const int* __restrict__ ovf_rows,
                                   const uint16_t* __restrict__ count, const uint16_t* __restrict__ val,
-                                  const uint8_t* __restrict__ col, const uint16_t* __restrict__ spill, int f,
-                                  int K, uint16_t* __restrict__ g_ovf, const uint16_t* __restrict__ X, int d,
-                                  uint16_t* __restrict__ x_ovf) {
-  const int n = n_ovf[0];
+                                  const uint8_t* __restrict__ col, const uint16_t* __restrict__ spill, int M, int f,
+                                  int K, int cap, uint16_t* __restrict__ g_ovf, const uint16_t* __restrict__ X, int d,
+                                  uint16_t* __restrict__ x_ovf, uint32_t* status) {
+  int n = n_ovf[0];
+  if (!in_bounds(n <= cap, status)) n = cap;
   const int T = f / kTn;
   for (int sl = blockIdx.x; sl < n; sl += gridDim.x) {
     const long row = ovf_rows[sl];
+    if (!in_bounds(row >= 0 && row < M, status)) continue;
     // 16 chunks of 8 columns per tile
     for (int ch = threadIdx.x; ch < T * 16; ch += blockDim.x) {
       const int t = ch >> 4, c0 = (ch & 15) * 8;
@@ -253,10 +255,14 @@ __global__ void ovf_gather_kernel(const int* __restrict__ n_ovf, const int* __re
 }
 
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ in, const int* __restrict__ rows,
-                                   const int* __restrict__ n_ovf, int d, uint16_t* __restrict__ out) {
-  const int n = n_ovf[0];
+                                   const int* __restrict__ n_ovf, int cap, int M, int d, uint16_t* __restrict__ out,
+                                   uint32_t* status) {
+  int n = n_ovf[0];
+  if (!in_bounds(n <= cap, status)) n = cap;
   for (int sl = blockIdx.x; sl < n; sl += gridDim.x) {
-    const uint4* src = reinterpret_cast<const uint4*>(in + static_cast<long>(rows[sl]) * d);
+    const int r = rows[sl];
+    if (!in_bounds(r >= 0 && r < M, status)) continue;
+    const uint4* src = reinterpret_cast<const uint4*>(in + static_cast<long>(r) * d);
     uint4* dst = reinterpret_cast<uint4*>(out + static_cast<long>(sl) * d);
     for (int q = threadIdx.x; q < d / 8; q += blockDim.x) dst[q] = src[q];
   }
@@ -326,16 +332,17 @@ cudaError_t launch_route(const uint16_t* count, const uint16_t* val, const uint8
   if (cap > 0 && !tiles) {
     int g = cap < device_sm_count() * 4 ? cap : device_sm_count() * 4;
     TWELL_LAUNCH("ovf_gather", s,
-                 ovf_gather_kernel<<<g, 256, 0, s>>>(n_ovf, ovf_rows, count, val, col, spill, f, K, g_ovf, X, d, x_ovf));
+                 ovf_gather_kernel<<<g, 256, 0, s>>>(n_ovf, ovf_rows, count, val, col, spill, M, f, K, cap, g_ovf, X,
+                                                     d, x_ovf, status));
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_gather_rows(const uint16_t* in, const int* rows, const int* n_ovf, int cap, int d,
-                               uint16_t* out, cudaStream_t s) {
+cudaError_t launch_gather_rows(const uint16_t* in, const int* rows, const int* n_ovf, int cap, int M, int d,
+                               uint16_t* out, uint32_t* status, cudaStream_t s) {
   if (cap <= 0) return cudaSuccess;
   int g = cap < device_sm_count() * 4 ? cap : device_sm_count() * 4;
-  TWELL_LAUNCH("gather_rows", s, gather_rows_kernel<<<g, 256, 0, s>>>(in, rows, n_ovf, d, out));
+  TWELL_LAUNCH("gather_rows", s, gather_rows_kernel<<<g, 256, 0, s>>>(in, rows, n_ovf, cap, M, d, out, status));
   return cudaGetLastError();
 }
 

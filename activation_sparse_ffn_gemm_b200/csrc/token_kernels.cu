@@ -191,13 +191,15 @@ __device__ __forceinline__ long next_row(int* ctr, int grp, int wi, int lane, in
 
 __device__ __forceinline__ void build_list(GroupSmem& g, long row, int T, int K, int e0, int ne, int gtid, int GT,
                                            const uint16_t* __restrict__ val, const uint8_t* __restrict__ col,
-                                           const float* __restrict__ u_ell) {
+                                           const float* __restrict__ u_ell, uint32_t* status) {
   for (int e = gtid; e < ne; e += GT) {
     int t, sl;
     entry_of(g.off, T, e0 + e, t, sl);
     const long base = (row * T + t) * K + sl;
-    g.j[e] = t * kTn + col[base];
-    g.c[e] = __uint_as_float(static_cast<uint32_t>(val[base]) << 16);
+    const int c = col[base];
+    const bool ok = in_bounds(c < kTn, status);
+    g.j[e] = t * kTn + (ok ? c : 0);
+    g.c[e] = ok ? __uint_as_float(static_cast<uint32_t>(val[base]) << 16) : 0.f;
     if (u_ell) g.c2[e] = u_ell[base];
     g.slot[e] = t * K + sl;
   }
@@ -212,14 +214,16 @@ __device__ __forceinline__ void build_list(GroupSmem& g, long row, int T, int K,
 __device__ __forceinline__ void build_list_tiles(GroupSmem& g, long row, int T, int K, int f, int e0, int ne, int gtid,
                                                  int GT, int wi, int W, int lane,
                                                  const uint16_t* __restrict__ val, const uint8_t* __restrict__ col,
-                                                 const uint16_t* __restrict__ spill) {
+                                                 const uint16_t* __restrict__ spill, uint32_t* status) {
   for (int e = gtid; e < ne; e += GT) {
     int t, sl;
     entry_of(g.off, T, e0 + e, t, sl);
     if (g.tcnt[t] > K) continue;
     const long base = (row * T + t) * K + sl;
-    g.j[e] = t * kTn + col[base];
-    g.c[e] = __uint_as_float(static_cast<uint32_t>(val[base]) << 16);
+    const int c = col[base];
+    const bool ok = in_bounds(c < kTn, status);
+    g.j[e] = t * kTn + (ok ? c : 0);
+    g.c[e] = ok ? __uint_as_float(static_cast<uint32_t>(val[base]) << 16) : 0.f;
     g.slot[e] = t * K + sl;
   }
   for (int t = wi; t < T; t += W) {
@@ -371,12 +375,18 @@ __device__ __forceinline__ void turn_pass(int* turn, int row, int q, int P, int 
 // the row's kept-entry offsets; returns false when the plan is exhausted.
 template <int W, bool TILES>
 __device__ __forceinline__ bool next_piece(int* ctr, const int* plan, int M, const uint16_t* __restrict__ count, int T,
-                                           int K, int grp, int wi, int lane, int* s_next, GroupSmem& g) {
+                                           int K, int grp, int wi, int lane, int* s_next, GroupSmem& g,
+                                           uint32_t* status) {
   const int np = plan[0], S = plan[1];
-  const int p = static_cast<int>(next_row<W>(ctr, grp, wi, lane, s_next));
-  if (p >= np) return false;
   const int* pieces = plan + kPlanHdr + 2L * M;
-  const int row = pieces[2 * p], q = pieces[2 * p + 1];
+  int p, row, q;
+  for (;;) {  // a piece whose row is out of range is skipped (bounds-checked build)
+    p = static_cast<int>(next_row<W>(ctr, grp, wi, lane, s_next));
+    if (p >= np) return false;
+    row = pieces[2 * p];
+    q = pieces[2 * p + 1];
+    if (in_bounds(row >= 0 && row < M && q >= 0, status)) break;
+  }
   if (wi == 0) row_offsets<TILES>(count, row, T, K, lane, g);
   if (wi == 0 && lane == 0) {
     const int n = g.tot;
@@ -441,15 +451,15 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
     }
   };
 
-  while (next_piece<W, TILES>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g)) {
+  while (next_piece<W, TILES>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g, status)) {
     const long row = g.row;
     const int S = plan[1];
     const int e0 = g.q * S;
     const int ne = max(0, min(S, g.tot - e0));
     if (TILES)
-      build_list_tiles(g, row, T, K, T * kTn, e0, ne, gtid, Cfg::GT, wi, W, lane, val, col, spill);
+      build_list_tiles(g, row, T, K, T * kTn, e0, ne, gtid, Cfg::GT, wi, W, lane, val, col, spill, status);
     else
-      build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, nullptr);
+      build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, nullptr, status);
     group_sync<W>(grp);
     up(row, ne);
     float2 y[C][4];
@@ -476,9 +486,9 @@ template <int C, int W, bool EXACT>
 __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>::WARPS * 32)) ell_bwd_kernel(
     const uint16_t* __restrict__ dY, const uint16_t* __restrict__ Wu, const uint16_t* __restrict__ Wg,
     const uint16_t* __restrict__ Wdt, const uint16_t* __restrict__ count, const uint16_t* __restrict__ val,
-    const uint8_t* __restrict__ col, int* __restrict__ plan, const float* __restrict__ u_ell, float lambda,
-    float4* __restrict__ hdz_ell, float* __restrict__ dX, int M, int d, int T, int K, int* __restrict__ ctr,
-    uint32_t* status) {
+    const uint8_t* __restrict__ col, int* __restrict__ plan, const int* __restrict__ n_ovf,
+    const float* __restrict__ u_ell, float lambda, float4* __restrict__ hdz_ell, float* __restrict__ dX, int M, int d,
+    int T, int K, int* __restrict__ ctr, uint32_t* status) {
   using Cfg = TokCfg<C, W>;
   constexpr int B = Cfg::B;
   constexpr int B2 = B > 1 ? B / 2 : 1;  // two rows (W_u, W_g) per unit in the dX phase
@@ -522,12 +532,16 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
     if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, TWELL_STATUS_BAD_STATE);
     return;
   }
-  while (next_piece<W, false>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g)) {
+  // overflow rows beyond the dense backup's capacity have no stored g or u: the
+  // backward leaves their dX rows unwritten and their pairs out of the weight
+  // gradients, and says so in the status word
+  if (blockIdx.x == 0 && threadIdx.x == 0 && n_ovf[1] > n_ovf[0]) set_status(status, TWELL_STATUS_OVERFLOW_CAP);
+  while (next_piece<W, false>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g, status)) {
     const long row = g.row;
     const int S = plan[1];
     const int e0 = g.q * S;
     const int ne = max(0, min(S, g.tot - e0));
-    build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, u_ell);
+    build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, u_ell, status);
     group_sync<W>(grp);
     dh_phase(row, ne);
     float2 dx[C][4];
@@ -625,8 +639,8 @@ cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uin
 
 cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const uint16_t* W_g,
                                const uint16_t* W_dt, const uint16_t* count, const uint16_t* val,
-                               const uint8_t* col, int* plan, const float* u_ell, float lambda, float4* hdz_ell,
-                               float* dX, int M, int d, int f, int K, int* ctr, uint32_t* status,
+                               const uint8_t* col, int* plan, const int* n_ovf, const float* u_ell, float lambda,
+                               float4* hdz_ell, float* dX, int M, int d, int f, int K, int* ctr, uint32_t* status,
                                cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
@@ -636,10 +650,10 @@ cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const ui
   const int T = f / kTn;
   const bool exact = d / 8 == W * 32 * C;
 #define TWELL_BWD(CC, WW)                                                                                        \
-  (exact ? launch_bwd_cw<CC, WW, true>(M, s, dY, W_u, W_g, W_dt, count, val, col, plan, u_ell, lambda, hdz_ell, \
-                                       dX, M, d, T, K, ctr, status)                                           \
-         : launch_bwd_cw<CC, WW, false>(M, s, dY, W_u, W_g, W_dt, count, val, col, plan, u_ell, lambda, hdz_ell, \
-                                        dX, M, d, T, K, ctr, status))
+  (exact ? launch_bwd_cw<CC, WW, true>(M, s, dY, W_u, W_g, W_dt, count, val, col, plan, n_ovf, u_ell, lambda,  \
+                                       hdz_ell, dX, M, d, T, K, ctr, status)                                    \
+         : launch_bwd_cw<CC, WW, false>(M, s, dY, W_u, W_g, W_dt, count, val, col, plan, n_ovf, u_ell, lambda, \
+                                        hdz_ell, dX, M, d, T, K, ctr, status))
   if (W == 1 && C == 1) TWELL_BWD(1, 1);
   else if (W == 1 && C == 2) TWELL_BWD(2, 1);
   else if (W == 1 && C == 4) TWELL_BWD(4, 1);

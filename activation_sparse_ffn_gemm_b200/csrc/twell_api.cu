@@ -34,6 +34,17 @@ unsigned long long next_launch_epoch() {
 }
 
 namespace {
+std::atomic<int> g_epi_withhold{0};
+}  // namespace
+
+bool take_epi_withhold() {
+  int v = g_epi_withhold.load(std::memory_order_relaxed);
+  while (v > 0)
+    if (g_epi_withhold.compare_exchange_weak(v, v - 1, std::memory_order_relaxed)) return true;
+  return false;
+}
+
+namespace {
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -292,7 +303,7 @@ twell_status ffn_fwd_impl(const uint16_t* X, const uint16_t* W_g, const uint16_t
     return TWELL_ECUDA;
   if (tiles) return TWELL_OK;
   const SplitKBuffers sk{at<float>(ws, L.sk_partial), at<unsigned long long>(ws, L.sk_arrivals)};
-  return cuda_status(launch_ovf_fwd(x_ovf, W_u, W_d, h->g_ovf, h->ovf_rows, h->n_ovf, cap, d, f,
+  return cuda_status(launch_ovf_fwd(x_ovf, W_u, W_d, h->g_ovf, h->ovf_rows, h->n_ovf, cap, M, d, f,
                                     at<uint16_t>(ws, L.h_ovf), h->u_ovf, Y, sk, h->status, s));
 }
 
@@ -352,9 +363,9 @@ twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_
   uint16_t* dy_ovf = at<uint16_t>(ws, L.dy_ovf);
   uint16_t* duz = at<uint16_t>(ws, L.duz);
   float4* hdz_ell = at<float4>(ws, L.hdz_ell);
-  if (launch_gather_rows(dY, h->ovf_rows, h->n_ovf, cap, d, dy_ovf, s) != cudaSuccess) return TWELL_ECUDA;
-  if (launch_ell_ffn_bwd(dY, W_u, W_g, wdt, h->count, h->val, h->col, h->row_plan, h->u_ell, lambda, hdz_ell,
-                         dX, M, d, f, K, at<int>(ws, L.ctr), h->status, s) != cudaSuccess)
+  if (launch_gather_rows(dY, h->ovf_rows, h->n_ovf, cap, M, d, dy_ovf, h->status, s) != cudaSuccess) return TWELL_ECUDA;
+  if (launch_ell_ffn_bwd(dY, W_u, W_g, wdt, h->count, h->val, h->col, h->row_plan, h->n_ovf, h->u_ell, lambda,
+                         hdz_ell, dX, M, d, f, K, at<int>(ws, L.ctr), h->status, s) != cudaSuccess)
     return TWELL_ECUDA;
   float* du_ovf = at<float>(ws, L.du_ovf);
   float* dz_ovf = at<float>(ws, L.dz_ovf);
@@ -363,15 +374,16 @@ twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_
                               at<uint16_t>(ws, L.h2)};
   float* db_ovf = at<float>(ws, L.db_ovf);
   int* k_rows = at<int>(ws, L.k_rows);
-  if (launch_ovf_bwd(dy_ovf, wdt, W_u, W_g, h->g_ovf, h->u_ovf, lambda, h->ovf_rows, h->n_ovf, cap, d, f, duz,
+  if (launch_ovf_bwd(dy_ovf, wdt, W_u, W_g, h->g_ovf, h->u_ovf, lambda, h->ovf_rows, h->n_ovf, cap, M, d, f, duz,
                      du_ovf, dz_ovf, dX, sk, h->status, s) != cudaSuccess)
     return TWELL_ECUDA;
-  if (launch_ovf_operands(h->n_ovf, h->ovf_rows, h->row_plan, cap, d, f, X, dy_ovf, du_ovf, dz_ovf, h->g_ovf,
-                          h->u_ovf, dw, db_ovf, k_rows, s) != cudaSuccess)
+  if (launch_ovf_operands(h->n_ovf, h->ovf_rows, h->row_plan, cap, M, d, f, X, dy_ovf, du_ovf, dz_ovf, h->g_ovf,
+                          h->u_ovf, dw, db_ovf, k_rows, h->status, s) != cudaSuccess)
     return TWELL_ECUDA;
-  CscBuffers b{h->row_plan + kPlanHdr + M,          at<int>(ws, L.block_cnt), at<int>(ws, L.unit_tot),
-               at<unsigned long long>(ws, L.scan_arrive), at<int>(ws, L.unit_ptr), at<int>(ws, L.csc_row),
-               at<float4>(ws, L.csc_val)};
+  const long long nnz_cap = static_cast<long long>(M - cap) * (f / kTn) * K + static_cast<long long>(cap) * f;
+  CscBuffers b{M, cap, nnz_cap, h->status, h->row_plan + kPlanHdr + M, at<int>(ws, L.block_cnt),
+               at<int>(ws, L.unit_tot), at<unsigned long long>(ws, L.scan_arrive), at<int>(ws, L.unit_ptr),
+               at<int>(ws, L.csc_row), at<float4>(ws, L.csc_val)};
   if (launch_build_csc(h->count, h->col, h->row_ovf, h->g_ovf, h->u_ovf, hdz_ell, du_ovf, dz_ovf, h->row_plan, M, f,
                        K, b, s) != cudaSuccess)
     return TWELL_ECUDA;
@@ -393,6 +405,10 @@ twell_status twell_count_stats(const twell_hybrid* h, int64_t* rows_by_max, int6
   if (h->dense_min < 0) return TWELL_EINVAL;
   return cuda_status(launch_count_stats(h->count, h->M, h->d_ff / kTn, h->dense_min, rows_by_max, act_by_max,
                                         tiles_by_count, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+void twell_test_withhold_epilogue_arrival(int launches) {
+  g_epi_withhold.store(launches > 0 ? launches : 0, std::memory_order_relaxed);
 }
 
 twell_status twell_status_read(const twell_hybrid* h, uint32_t* out, int clear, twell_stream_t stream) {

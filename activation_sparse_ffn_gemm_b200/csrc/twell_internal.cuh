@@ -53,6 +53,19 @@ __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bits) {
   if (status) atomicOr(status, bits);
 }
 
+// Index checks of the bounds-checked build (-DTWELL_BOUNDS): an index read from
+// a buffer is tested against the extent it addresses before the access it
+// steers; a failed test sets TWELL_STATUS_BOUNDS and the caller skips the
+// access. The regular build compiles every check to `true`.
+#ifdef TWELL_BOUNDS
+__device__ __forceinline__ bool in_bounds(bool ok, uint32_t* status) {
+  if (!ok) set_status(status, TWELL_STATUS_BOUNDS);
+  return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool in_bounds(bool, uint32_t*) { return true; }
+#endif
+
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
@@ -95,6 +108,10 @@ int device_sm_count();
 // never 0), so arrival words need no reset between launches.
 unsigned long long next_launch_epoch();
 
+// Test of the split-K epilogue's bounded barrier (twell_test_withhold_epilogue_arrival):
+// true for as many split-capable GEMM launches as the test asked for.
+bool take_epi_withhold();
+
 // Encodes a 2-D bf16 tensor map (128-byte swizzle, zero fill out of bounds).
 // inner = contiguous extent (elements), outer = rows, row_bytes = row pitch.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
@@ -130,9 +147,9 @@ cudaError_t launch_route(const uint16_t* count, const uint16_t* val, const uint8
 // launch shape they use); sizes the pieces of the row plan.
 int tok_groups(int M, int d);
 
-// out[s][:] = in[rows[s]][:] for s < n_ovf[0] (bf16 rows of width d).
-cudaError_t launch_gather_rows(const uint16_t* in, const int* rows, const int* n_ovf, int cap, int d,
-                               uint16_t* out, cudaStream_t s);
+// out[s][:] = in[rows[s]][:] for s < n_ovf[0] (bf16 rows of width d, M rows in `in`).
+cudaError_t launch_gather_rows(const uint16_t* in, const int* rows, const int* n_ovf, int cap, int M, int d,
+                               uint16_t* out, uint32_t* status, cudaStream_t s);
 
 cudaError_t launch_transpose_bf16(const uint16_t* in, int rows, int cols, uint16_t* out, cudaStream_t s);
 
@@ -158,23 +175,24 @@ size_t splitk_arrival_words();
 // Dense backup forward for overflow rows: H = bf16(G * (X_ovf W_u^T)) then
 // Y[ovf_rows] = bf16(H W_d^T).
 cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uint16_t* W_d,
-                           const uint16_t* g_ovf, const int* ovf_rows, const int* n_ovf, int cap, int d, int f,
+                           const uint16_t* g_ovf, const int* ovf_rows, const int* n_ovf, int cap, int M, int d, int f,
                            uint16_t* h_ovf, float* u_ovf, uint16_t* Y, const SplitKBuffers& sk, uint32_t* status,
                            cudaStream_t s);
 
 // Sparse backward over the pieces of the row plan: dH at kept actives, dU,
 // dZ, with (h = g u, dU, dZ, 0) stored per slot, and the rows of dX.
+// Sets TWELL_STATUS_OVERFLOW_CAP when the forward flagged more overflow rows than it stored.
 cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const uint16_t* W_g,
                                const uint16_t* W_dt, const uint16_t* count, const uint16_t* val,
-                               const uint8_t* col, int* plan, const float* u_ell, float lambda, float4* hdz_ell,
-                               float* dX, int M, int d, int f, int K, int* ctr, uint32_t* status,
+                               const uint8_t* col, int* plan, const int* n_ovf, const float* u_ell, float lambda,
+                               float4* hdz_ell, float* dX, int M, int d, int f, int K, int* ctr, uint32_t* status,
                                cudaStream_t s);
 
 // Dense backup backward for overflow rows: dU, dZ (fp32, and bf16 [dU | dZ] as
 // the next GEMM's operand) from dH = dY_ovf W_d, then dX[ovf_rows] = dU W_u + dZ W_g.
 cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const uint16_t* W_u,
                            const uint16_t* W_g, const uint16_t* g_ovf, const float* u_ovf, float lambda,
-                           const int* ovf_rows, const int* n_ovf, int cap, int d, int f, uint16_t* duz_ovf,
+                           const int* ovf_rows, const int* n_ovf, int cap, int M, int d, int f, uint16_t* duz_ovf,
                            float* du_ovf, float* dz_ovf, float* dX, const SplitKBuffers& sk, uint32_t* status,
                            cudaStream_t s);
 
@@ -200,6 +218,9 @@ cudaError_t launch_dense_wgrad(const DenseWgradOperands& op, const int* k_rows, 
                                float* dW_u, float* dW_d, uint32_t* status, cudaStream_t s);
 
 struct CscBuffers {
+  int M, cap;           // token rows; dense backup capacity (the extent of row_slot's values)
+  long long nnz_cap;    // entries csc_row / csc_val can hold
+  uint32_t* status;     // device status word (index checks of the bounds-checked build)
   const int* row_slot;  // [M] dense backup slot of each row (-1: none), from the row plan
   int* block_cnt;  // [ceil(M/kCscRows)][f] per-chunk counts, then their exclusive scan
   int* unit_tot;   // [f]
@@ -222,10 +243,10 @@ cudaError_t launch_build_csc(const uint16_t* count, const uint8_t* col, const ui
 // sums of dZ over the overflow rows (db_ovf) and the contraction length
 // k_rows = roundup(n, 64) + n (0 when the plan keeps the overflow rows on the
 // sparse path, and then db_ovf = 0).
-cudaError_t launch_ovf_operands(const int* n_ovf, const int* ovf_rows, const int* plan, int cap, int d, int f,
+cudaError_t launch_ovf_operands(const int* n_ovf, const int* ovf_rows, const int* plan, int cap, int M, int d, int f,
                                 const uint16_t* X, const uint16_t* dy_ovf, const float* du_ovf, const float* dz_ovf,
                                 const uint16_t* g_ovf, const float* u_ovf, const DenseWgradOperands& op,
-                                float* db_ovf, int* k_rows, cudaStream_t s);
+                                float* db_ovf, int* k_rows, uint32_t* status, cudaStream_t s);
 
 // dW_u = dU^T X, dW_g = dZ^T X, dW_d = dY^T H, db_g = column sums of dZ (plus
 // db_extra when non-null) over the pairs of the pair list; the weight

@@ -55,6 +55,7 @@ struct GemmShape {
   int split_max = 1;
   unsigned long long* arrivals = nullptr;  // [kSplitTiles] per-output-tile arrival words
   unsigned long long epoch = 0;            // this launch's tag (1 .. 2^56 - 1)
+  int withhold_epi_arrival = 0;  // test of the bounded epilogue barrier: one epilogue warp never arrives
 };
 
 constexpr int kSplitMax = 8;
@@ -89,19 +90,28 @@ struct GemmLayout {
 // its loop on a timeout must not strand the others): each warp adds one to a
 // shared counter; lane 0 waits until the counter reaches `gen` (advanced by 4
 // per use), or the CTA's abort flag is set, or kWaitLimitNs has passed.
-__device__ __forceinline__ void epi_bar(volatile int* cnt, int& gen, volatile int* abort_flag) {
+// Returns true, to every lane, only when all four warps arrived; on false the
+// caller records the timeout and leaves its tile loop without touching what
+// the other warps were to write. `withhold` (a test of this path) skips this
+// warp's arrival, so the wait runs out as it would behind a stalled warp.
+__device__ __forceinline__ bool epi_bar(volatile int* cnt, int& gen, volatile int* abort_flag, bool withhold = false) {
   gen += 4;
   __threadfence_block();
   __syncwarp();
+  int done = 1;
   if ((threadIdx.x & 31) == 0) {
-    atomicAdd(const_cast<int*>(cnt), 1);
+    if (!withhold) atomicAdd(const_cast<int*>(cnt), 1);
     const uint64_t t0 = globaltimer_ns();
     while (*cnt < gen) {
-      if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) break;
+      if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) {
+        done = 0;
+        break;
+      }
     }
   }
-  __syncwarp();
+  done = __shfl_sync(0xFFFFFFFFu, done, 0);
   __threadfence_block();
+  return done != 0;
 }
 
 __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
@@ -360,9 +370,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                __uint_as_float(v[4 * q + 3]));
         }
         if constexpr (Epi::kSplitK) {
-          // arrival: the last of the tile's `split` ranges reduces it
+          // arrival: the last of the tile's `split` ranges reduces it. A barrier
+          // that runs out means a warp of this CTA may not have stored its
+          // partial rows: the tile's arrival is not counted (no CTA reduces it)
+          // and the CTA unwinds with TWELL_STATUS_TIMEOUT.
           __threadfence();
-          epi_bar(epi_cnt, bar_gen, abort_flag);
+          if (!epi_bar(epi_cnt, bar_gen, abort_flag, shp.withhold_epi_arrival != 0 && quarter == 3)) {
+            fail();
+            break;
+          }
           if (threadIdx.x == 64) {
             unsigned long long* w = shp.arrivals + (mb * num_n + nb);
             unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(w), nw;
@@ -376,7 +392,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (last) atomicExch(w, 0ull);
             *last_s = last ? 1 : 0;
           }
-          epi_bar(epi_cnt, bar_gen, abort_flag);
+          if (!epi_bar(epi_cnt, bar_gen, abort_flag)) {
+            fail();
+            break;
+          }
           if (*last_s) {
             // the tile's (row, 8-column chunk) items spread over the 128 epilogue
             // threads (consecutive threads on consecutive chunks of a row), each
@@ -451,7 +470,10 @@ cudaError_t launch_umma_gemm(const char* name, const CUtensorMap& a0, const CUte
   // with split-K the work items can outnumber the output tiles: one CTA per SM
   const int grid = shp.partial ? sms : static_cast<int>(tiles < sms ? tiles : sms);
   GemmShape shp2 = shp;
-  if (shp2.partial) shp2.epoch = next_launch_epoch();
+  if (shp2.partial) {
+    shp2.epoch = next_launch_epoch();
+    shp2.withhold_epi_arrival = take_epi_withhold() ? 1 : 0;
+  }
   TWELL_LAUNCH(name, s, kern<<<grid, kGemmThreads, smem, s>>>(a0, b0, a1, b1, shp2, ea));
   return cudaGetLastError();
 }

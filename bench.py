@@ -4,9 +4,14 @@
 One step = the whole hot path over one batch: W_d transposed for the step's
 weights, the gate GEMM with the TwELL pack epilogue, row routing, the sparse
 up+down for ELL rows and the dense backup for overflow rows, then the backward
-over the hybrid format (L1 term on the gate activations). Workload: the uniform
-1%-activity inference shape (M=4096 tokens, d_model=2048, d_ff=8192, T_n=128,
-K=8) run as a training step, synthetic seeded data, inputs resident in HBM.
+over the hybrid format (L1 term on the gate activations). Workload: M=65536
+tokens, d_model=4096, d_ff=14336, T_n=128, K=8, 99% sparsity (1% target
+activity) with lognormal(0, 0.75) per-token row scaling, synthetic seeded data
+drawn on the host, inputs resident in HBM. The line also carries the forward
+half and the inference forward of that workload, the dense bf16 FFN on the
+same inputs, and two smaller workloads beside it (the uniform 1% inference
+forward at M=4096, d_model=2048, d_ff=8192, and the uniform training step at
+M=8192 of the same shape).
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
     python bench.py --sweep [--steps K --warmup W]
@@ -22,9 +27,12 @@ threshold of the cost model and the K chosen from the batch's count statistics
 listed K instead, next to the K that the batch's count statistics and the cost
 model of activation_sparse_ffn_gemm_b200.kchoice choose.
 
-Prints one JSON line (rank 0). With N > 1 (torchrun) every rank runs its own
-replica of the batch; the time is the max over ranks and the value counts the
-tokens of all ranks (weak scaling; the path has no exchange step).
+Prints one JSON line (rank 0). With N > 1 (torchrun) the step is the
+token-sharded (data-parallel) training step: every rank holds its own batch of
+tokens for the same weights and the weight gradients are summed over the ranks
+by NCCL all-reduce inside every timed step (activation_sparse_ffn_gemm_b200.sharded);
+the time is the max over ranks and the value counts the tokens of all ranks
+(weak scaling).
 """
 
 from __future__ import annotations
@@ -59,6 +67,9 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--no-trace", action="store_true")
+    p.add_argument("--workload", default=MAIN_WORKLOAD, choices=["large", "train", "heavy"],
+                   help="workload of the timed training step (synthetic.WORKLOADS)")
+    p.add_argument("--no-extra", action="store_true", help="skip the two smaller workloads of the line")
     p.add_argument("--sweep", action="store_true",
                    help="token-count x sparsity sweep at d_model=4096, d_ff=14336 (one JSON line per point)")
     p.add_argument("--sweep-m", default="512,2048,8192,32768,65536")
@@ -86,18 +97,36 @@ def dist_env():
     return int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0"))
 
 
-def workload():
+# the workload of the timed training step, and the smaller ones reported beside it
+MAIN_WORKLOAD = "large"
+OTHER_WORKLOADS = (("uniform_d2048_f8192_M4096_inference", "uniform", "infer"),
+                   ("uniform_d2048_f8192_M8192_training", "train", "train"))
+CPU_SLICE_ROWS = 256  # token rows of the CPU baseline's slice of the main workload
+
+
+def workload(name=MAIN_WORKLOAD):
     from synthetic import WORKLOADS
 
-    w = WORKLOADS["uniform"]
-    with open(os.path.join(ROOT, "tests", "golden", "uniform_seed.json")) as fh:
-        seed = json.load(fh)["seed"]
+    w = WORKLOADS[name]
+    seed = w.seed
+    if name == "uniform":
+        with open(os.path.join(ROOT, "tests", "golden", "uniform_seed.json")) as fh:
+            seed = json.load(fh)["seed"]
     return w, seed
 
 
-def workload_desc(w, seed):
-    return (f"uniform i.i.d. {w.activity:.0%} activity: M={w.M} tokens, d_model={w.d_model}, d_ff={w.d_ff}, "
-            f"T_n={w.T_n}, K={w.K}, seed {seed} (no overflowing row), run as a training step")
+def workload_desc(w, seed, mode="train"):
+    rows = (f"lognormal(0, {w.sigma:g}) per-token row scale" if w.row_scale == "lognormal"
+            else "i.i.d. activity across tokens")
+    what = "training step (forward + backward)" if mode == "train" else "inference forward"
+    return (f"{100.0 * (1.0 - w.activity):g}% sparsity ({100.0 * w.activity:g}% target activity), {rows}: "
+            f"M={w.M} tokens, d_model={w.d_model}, d_ff={w.d_ff}, T_n={w.T_n}, K={w.K}, seed {seed}, {what}")
+
+
+def ovf_cap_for(w):
+    """Dense-backup capacity of the timed runs: a quarter of the rows (the heavy-tailed
+    99% batches route about 10% of their rows dense; the status word is checked)."""
+    return max(1, w.M // 4)
 
 
 def load_peaks():
@@ -219,26 +248,40 @@ class ClockSampler:
 # ------------------------------------------------------ algorithmic work
 
 
-def kernel_work(name, M, d, f, T, K, kept, pairs):
+def kernel_work(name, M, d, f, T, K, kept, pairs, n_ovf=0, dense_wgrad=0):
     """Algorithmic flops (tensor-bound kernels) or bytes (memory-bound) of one launch.
 
-    kept = stored slots of ELL rows, pairs = all active (row, unit) pairs."""
+    kept = stored slots of ELL rows (all their active units), pairs = all active
+    (row, unit) pairs, n_ovf = stored dense backup rows, dense_wgrad = 1 when the
+    overflow rows' weight gradients run as GEMMs (their pairs then stay out of
+    the pair list). The dense backup GEMMs count the plain contraction (the
+    weight-gradient GEMMs run it twice, over hi and lo halves of their operand)."""
+    m_ell = M - n_ovf
+    listed = kept + (0 if dense_wgrad else pairs - kept)
     if name == "gate_pack_gemm":
         return "tensor", 2.0 * M * d * f
+    if name in ("ovf_up_gemm", "ovf_down_gemm", "ovf_dh_gemm", "dense_wgrad_d"):
+        return "tensor", 2.0 * n_ovf * d * f
+    if name in ("ovf_dx_gemm", "dense_wgrad_ug"):
+        return "tensor", 4.0 * n_ovf * d * f
     if name == "ell_updown":
-        return "hbm", (2 * M * d            # X
-                       + M * T * (2 + 3 * K)  # TwELL count/val/col
-                       + 4 * kept             # u written
-                       + 2 * M * d            # Y written
-                       + 2 * 2 * f * d)       # W_u, W_dt read once
+        return "hbm", (2 * m_ell * d            # X
+                       + m_ell * T * (2 + 3 * K)  # TwELL count/val/col
+                       + 4 * kept                 # u written
+                       + 2 * m_ell * d            # Y written
+                       + 2 * 2 * f * d)           # W_u, W_dt read once
     if name == "ell_bwd":
-        return "hbm", (2 * M * d + M * T * (2 + 3 * K) + 4 * kept + 8 * kept + 4 * M * d + 3 * 2 * f * d)
+        # dY, TwELL, u read; (h, dU, dZ) per slot written; dX (fp32) written; W_u, W_g, W_dt once
+        return "hbm", (2 * m_ell * d + m_ell * T * (2 + 3 * K) + 4 * kept + 16 * kept + 4 * m_ell * d
+                       + 3 * 2 * f * d)
     if name == "weight_grads":
-        return "hbm", (2 * 2 * M * d + 20 * pairs + 3 * 4 * f * d + 4 * f)
+        # X and dY rows once, the pair list (row + (h, dU, dZ)), three fp32 gradients written
+        # (and read back when the dense GEMMs wrote the overflow rows' part first), db_g
+        return "hbm", (2 * 2 * M * d + 20 * listed + (2 if dense_wgrad else 1) * 3 * 4 * f * d + 4 * f)
     if name == "transpose_wd":
         return "hbm", 2 * 2 * f * d
     if name in ("csc_count", "csc_fill"):
-        return "hbm", M * T * (2 + K) + (20 * pairs if name == "csc_fill" else 0)
+        return "hbm", M * T * (2 + K) + (20 * listed if name == "csc_fill" else 0)
     return None, None
 
 
@@ -292,14 +335,15 @@ def source_hash(kernel):
     return h.hexdigest()[:16]
 
 
-def committed_traffic(kernel):
-    """DRAM bytes per launch from the committed ncu capture, if the kernel's sources still match."""
+def committed_traffic(kernel, wname=MAIN_WORKLOAD):
+    """DRAM bytes per launch of `kernel` on workload `wname` from the committed ncu
+    capture, if the kernel's sources still match the ones captured."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as fh:
         d = json.load(fh)
-    rec = d.get("kernels", {}).get(kernel)
+    rec = d.get("workloads", {}).get(wname, {}).get("kernels", {}).get(kernel)
     if not rec or rec.get("source_sha") != source_hash(kernel):
         return None
     return rec.get("dram_bytes_per_launch")
@@ -308,29 +352,45 @@ def committed_traffic(kernel):
 # ------------------------------------------------------------ CPU oracle
 
 
-def cpu_baseline(inp, lam, target_s):
-    """The fp64 oracle as it stands, forward + backward on a bounded sample of token rows."""
+def _oracle_rows(O, inp, n, lam):
+    """One oracle step on the first n token rows: forward (Y of those rows) and
+    backward (dX of those rows, weight gradients over them); returns seconds."""
     import numpy as np
 
+    rows = np.arange(n, dtype=np.int32)
+    t0 = time.perf_counter()
+    O.ffn_fwd(inp["X"], inp["W_g"], inp["b_g"], inp["W_u"], inp["W_d"], rows=rows)
+    O.ffn_bwd(inp["X"][:n], inp["W_g"], inp["b_g"], inp["W_u"], inp["W_d"], inp["dY"][:n], lam)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline_slice(inp, lam, n):
+    """The fp64 oracle as it stands, forward + backward on a fixed slice of n token rows."""
     from oracle import oracle as O
 
     O.build()
     M = inp["X"].shape[0]
+    n = min(n, M)
+    t = _oracle_rows(O, inp, n, lam)
+    return {"value": n / t, "unit": "tokens/s", "cores": O.get_threads(), "kind": "oracle",
+            "sample": f"slice: first {n} of {M} token rows, forward + backward (weight gradients over the "
+                      f"slice), {t:.1f} s"}
 
-    def run(n):
-        rows = np.arange(n)
-        t0 = time.perf_counter()
-        O.ffn_fwd(inp["X"], inp["W_g"], inp["b_g"], inp["W_u"], inp["W_d"], rows=rows.astype(np.int32))
-        O.ffn_bwd(inp["X"][:n], inp["W_g"], inp["b_g"], inp["W_u"], inp["W_d"], inp["dY"][:n], lam)
-        return time.perf_counter() - t0
 
-    n = 32
-    t = run(n)
+def cpu_baseline(inp, lam, target_s):
+    """The fp64 oracle as it stands, forward + backward on a sample of token rows
+    sized towards target_s seconds; returns (line, rows, seconds)."""
+    from oracle import oracle as O
+
+    O.build()
+    M = inp["X"].shape[0]
+    n = 8
+    t = _oracle_rows(O, inp, n, lam)
     for _ in range(3):  # grow the sample towards target_s (the oracle's cost is not quite linear in rows)
         if t >= target_s / 2 or n >= M:
             break
         n = int(min(M, max(2 * n, n * target_s / max(t, 1e-3))))
-        t = run(n)
+        t = _oracle_rows(O, inp, n, lam)
     return {"value": n / t, "unit": "tokens/s", "cores": O.get_threads(), "kind": "oracle",
             "sample": f"first {n} of {M} token rows, forward + backward (weight gradients over the sample), "
                       f"{t:.1f} s"}, n, t
@@ -347,7 +407,7 @@ def run_reference(args, world, rank):
     from oracle import oracle as O
     from synthetic import make_inputs
 
-    w, seed = workload()
+    w, seed = workload(args.workload)
     inp = make_inputs(w, seed=seed, with_dY=True)
     O.build()
     # each step: the oracle's forward + backward on a bounded sample of rows
@@ -371,7 +431,7 @@ def run_reference(args, world, rank):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": workload_desc(w, seed), "sample_rows_per_step": n,
+        "config": {"workload": workload_desc(w, seed, "train"), "sample_rows_per_step": n,
                    "reference": "fp64 CPU oracle (oracle/twell_oracle.c), OpenMP over rows"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": O.get_threads(), "kind": "oracle",
                          "sample": f"first {n} of {w.M} token rows per step, forward + backward"},
@@ -380,11 +440,63 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def _dense_arm(torch, X, W_g, b_g, W_u, W_d, dY, lam, timed, train):
+    """The dense bf16 gated FFN in torch (cuBLAS) on the same inputs, in two forms:
+    three GEMMs, and one GEMM against the stacked [W_g; W_u] (the concatenation is
+    made once, outside the timed region, as a model storing the fused weight
+    would). The backward goes through autograd with the L1 term's gradient fed
+    in directly (lambda on every gate activation), so no extra reduction is timed.
+    Returns per-form times and the faster form for each measure."""
+    f = W_g.shape[0]
+    M = X.shape[0]
+    W_gu = torch.cat([W_g, W_u]).contiguous()
+
+    def fwd3(e_mid):
+        with torch.no_grad():
+            (torch.relu(X @ W_g.T + b_g) * (X @ W_u.T)) @ W_d.T
+        e_mid.record()
+
+    def fwd_fused(e_mid):
+        with torch.no_grad():
+            zu = X @ W_gu.T
+            (torch.relu(zu[:, :f] + b_g) * zu[:, f:]) @ W_d.T
+        e_mid.record()
+
+    res = {"fwd_ms": {"three_gemms": timed(fwd3), "fused_gate_up": timed(fwd_fused)}}
+    if train:
+        Xr = X.clone().requires_grad_()
+        Wg_r, Wu_r, Wd_r, Wgu_r = (t.clone().requires_grad_() for t in (W_g, W_u, W_d, W_gu))
+        lam_g = torch.full((1, 1), lam, dtype=torch.bfloat16, device=X.device).expand(M, f)
+
+        def fb3(e_mid):
+            g = torch.relu(Xr @ Wg_r.T + b_g)
+            y = (g * (Xr @ Wu_r.T)) @ Wd_r.T
+            torch.autograd.backward((y, g), (dY, lam_g))
+            Xr.grad = Wg_r.grad = Wu_r.grad = Wd_r.grad = None
+            e_mid.record()
+
+        def fb_fused(e_mid):
+            zu = Xr @ Wgu_r.T
+            g = torch.relu(zu[:, :f] + b_g)
+            y = (g * zu[:, f:]) @ Wd_r.T
+            torch.autograd.backward((y, g), (dY, lam_g))
+            Xr.grad = Wgu_r.grad = Wd_r.grad = None
+            e_mid.record()
+
+        res["fwd_bwd_ms"] = {"three_gemms": timed(fb3), "fused_gate_up": timed(fb_fused)}
+    for k in ("fwd_ms", "fwd_bwd_ms"):
+        if k in res:
+            best = min(res[k], key=res[k].get)
+            res[k.replace("_ms", "_best")] = {"form": best, "ms": res[k][best], "tokens_per_s": M / (res[k][best] / 1e3)}
+    return res
+
+
 def run_twell(args, world, rank, local):
     import numpy as np
     import torch
 
     import activation_sparse_ffn_gemm_b200 as tw
+    from activation_sparse_ffn_gemm_b200.sharded import allreduce_grads
     from synthetic import make_inputs
 
     torch.cuda.set_device(local)
@@ -404,35 +516,13 @@ def run_twell(args, world, rank, local):
     def max_over_ranks(x):
         return reduce_max(x, dist, dev)
 
-    w, seed = workload()
-    inp = make_inputs(w, seed=seed, with_dY=True)
-
-    def dev_bf16(a):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
-
-    X, W_g, b_g, W_u, W_d, dY = (dev_bf16(inp[k]) for k in ("X", "W_g", "b_g", "W_u", "W_d", "dY"))
-    M, d, f, K, T = w.M, w.d_model, w.d_ff, w.K, w.d_ff // w.T_n
-    cap = M
-    st = tw.HybridState(M, f, w.T_n, K, cap, dev, with_u=True)
-    wsf = tw.workspace(tw.OP_FWD, M, d, f, w.T_n, K, cap, dev)
-    wsb = tw.workspace(tw.OP_BWD, M, d, f, w.T_n, K, cap, dev)
-    Wdt = torch.empty((f, d), dtype=torch.bfloat16, device=dev)
-    Y = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
-    grads = dict(dX=torch.empty((M, d), device=dev), dW_g=torch.empty((f, d), device=dev),
-                 dW_u=torch.empty((f, d), device=dev), dW_d=torch.empty((d, f), device=dev),
-                 db_g=torch.empty(f, device=dev))
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def fwd():
-        tw.transpose_wd(W_d, out=Wdt)
-        tw.ffn_fwd(X, W_g, b_g, W_u, W_d, T_n=w.T_n, K=K, W_dt=Wdt, state=st, ws=wsf, Y=Y)
-
-    def bwd():
-        tw.ffn_bwd(X, W_g, W_u, W_d, st, dY, lam=args.lam, W_dt=Wdt, ws=wsb, out=grads)
-
-    def timed(n, body, mid=None):
-        """Per-step CUDA events on the launching stream, L2 flushed before each step."""
+    def timed_pair(n, body):
+        """Per-step CUDA events on the launching stream, L2 flushed before each
+        step (outside the events); returns the mean step time and the mean time
+        to the event the body records part-way (body(e_mid))."""
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
                torch.cuda.Event(enable_timing=True)) for _ in range(n)]
         barrier()
@@ -444,201 +534,245 @@ def run_twell(args, world, rank, local):
             e2.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        tot = [a.elapsed_time(c) for a, _, c in ev]
-        first = [a.elapsed_time(b) for a, b, _ in ev]
-        return sum(tot) / n, sum(first) / n
+        return sum(a.elapsed_time(c) for a, _, c in ev) / n, sum(a.elapsed_time(b) for a, b, _ in ev) / n
 
-    def train_step(e_mid):
-        fwd()
-        e_mid.record(stream)
-        bwd()
+    def warm_and_time(body):
+        for _ in range(max(3, args.warmup)):
+            body(torch.cuda.Event())
+        return max_over_ranks(timed_pair(args.steps, body)[0])
 
-    for _ in range(max(3, args.warmup)):
-        train_step(torch.cuda.Event())
-    torch.cuda.synchronize(dev)
-    assert st.read_status() == 0, "device status word set during warm-up"
-    nst, nfl = st.n_overflow()
-    activity = float(st.count.sum().item()) / (M * f)
-    cnt = st.count.float()
+    def dev_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    launches0 = tw.launch_count()
-    with ClockSampler(local) as clk:
-        ms_step, ms_fwd = timed(args.steps, train_step)
-    launches = tw.launch_count() - launches0
-    ms_step = max_over_ranks(ms_step)
-    ms_fwd = max_over_ranks(ms_fwd)
+    def measure(name, mode, full):
+        """Times one workload: mode "train" = forward + backward per step, "infer"
+        = the inference forward (W_dt prepared once, u not saved). `full` adds the
+        per-kernel trace, the inference forward of a training workload, the
+        end-to-end run with host copies, and the CPU baseline."""
+        w, seed = workload(name)
+        # with N ranks each rank holds its own tokens for the same weights (shard = rank)
+        inp = make_inputs(w, seed=seed, with_dY=True, shard=rank if world > 1 else 0)
+        X, W_g, b_g, W_u, W_d, dY = (dev_bf16(inp[k]) for k in ("X", "W_g", "b_g", "W_u", "W_d", "dY"))
+        M, d, f, K, T = w.M, w.d_model, w.d_ff, w.K, w.d_ff // w.T_n
+        cap = ovf_cap_for(w)
+        train = mode == "train"
+        st = tw.HybridState(M, f, w.T_n, K, cap, dev, with_u=train)
+        wsf = tw.workspace(tw.OP_FWD, M, d, f, w.T_n, K, cap, dev)
+        wsb = tw.workspace(tw.OP_BWD, M, d, f, w.T_n, K, cap, dev) if train else None
+        Wdt = torch.empty((f, d), dtype=torch.bfloat16, device=dev)
+        Y = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
+        grads = (dict(dX=torch.empty((M, d), device=dev), dW_g=torch.empty((f, d), device=dev),
+                      dW_u=torch.empty((f, d), device=dev), dW_d=torch.empty((d, f), device=dev),
+                      db_g=torch.empty(f, device=dev)) if train else None)
+        res = {"workload": workload_desc(w, seed, mode), "M": M, "ovf_cap": cap}
 
-    # per-kernel breakdown: the same steps again with event tracing
-    breakdown = {}
-    if not args.no_trace:
-        tw.trace_collect()
-        tw.trace_enable(True)
-        timed(args.steps, train_step)
-        tw.trace_enable(False)
-        for name, ms in tw.trace_collect():
-            b = breakdown.setdefault(name, {"launches": 0, "ms": 0.0})
-            b["launches"] += 1
-            b["ms"] += ms
-        for b in breakdown.values():
-            b["ms_per_launch"] = b["ms"] / b["launches"]
-            b["ms_per_step"] = b["ms"] / args.steps
-
-    # inference forward with fixed weights: W_d transposed once (outside the timed
-    # region, as an inference caller does), u not saved for a backward
-    st_inf = tw.HybridState(M, f, w.T_n, K, cap, dev, with_u=False)
-
-    def infer(e_mid):
-        tw.ffn_fwd(X, W_g, b_g, W_u, W_d, T_n=w.T_n, K=K, W_dt=Wdt, state=st_inf, ws=wsf, Y=Y)
-        e_mid.record(stream)
-
-    for _ in range(3):
-        infer(torch.cuda.Event())
-    ms_inf = max_over_ranks(timed(args.steps, infer)[0])
-    assert st_inf.read_status() == 0, "device status word set during the inference timing"
-
-    # e2e: every step copies its inputs (X, dY) from pinned host memory and reads its
-    # result Y back, inside the timed region. As a training loop that prefetches its
-    # next batch does, the copies run on two copy streams (host->device, device->host)
-    # into double-buffered device tensors, so step i+1's inputs and step i-1's result
-    # move while step i computes. The step's working set (weights, workspaces, state,
-    # gradients: about 0.6 GB) is far larger than L2, so no extra flush is inserted.
-    hX = torch.empty((M, d), dtype=torch.bfloat16, pin_memory=True)
-    hdY = torch.empty((M, d), dtype=torch.bfloat16, pin_memory=True)
-    hY = [torch.empty((M, d), dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
-    hX.copy_(X.cpu())
-    hdY.copy_(dY.cpu())
-    Xb, dYb, Yb = [X, torch.empty_like(X)], [dY, torch.empty_like(dY)], [Y, torch.empty_like(Y)]
-    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-
-    def e2e_run(n):
-        ev_in = [torch.cuda.Event() for _ in range(2)]
-        ev_done = [torch.cuda.Event() for _ in range(2)]
-        ev_out = [torch.cuda.Event() for _ in range(2)]
-        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier()
-        torch.cuda.synchronize(dev)
-        t0.record(stream)
-        up.wait_stream(stream)
-        down.wait_stream(stream)
-
-        def load(b):
-            with torch.cuda.stream(up):
-                Xb[b].copy_(hX, non_blocking=True)
-                dYb[b].copy_(hdY, non_blocking=True)
-                ev_in[b].record(up)
-
-        load(0)
-        for i in range(n):
-            b = i % 2
-            if i + 1 < n:
-                if i >= 1:
-                    up.wait_event(ev_done[1 - b])  # step i-1 has finished reading these buffers
-                load(1 - b)
-            stream.wait_event(ev_in[b])
-            if i >= 2:
-                stream.wait_event(ev_out[b])  # step i-2's result has left Yb[b]
+        def fwd_train():
             tw.transpose_wd(W_d, out=Wdt)
-            tw.ffn_fwd(Xb[b], W_g, b_g, W_u, W_d, T_n=w.T_n, K=K, W_dt=Wdt, state=st, ws=wsf, Y=Yb[b])
-            tw.ffn_bwd(Xb[b], W_g, W_u, W_d, st, dYb[b], lam=args.lam, W_dt=Wdt, ws=wsb, out=grads)
-            ev_done[b].record(stream)
-            down.wait_event(ev_done[b])
-            with torch.cuda.stream(down):
-                hY[b].copy_(Yb[b], non_blocking=True)
-                ev_out[b].record(down)
-        stream.wait_stream(down)
-        stream.wait_stream(up)
-        t1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier()
-        return t0.elapsed_time(t1) / n
+            tw.ffn_fwd(X, W_g, b_g, W_u, W_d, T_n=w.T_n, K=K, W_dt=Wdt, state=st, ws=wsf, Y=Y)
 
-    e2e_run(max(3, args.warmup))
-    ms_e2e = max_over_ranks(e2e_run(args.steps))
-    assert torch.equal(hY[(args.steps - 1) % 2].to(dev), Y), "end-to-end result differs from the resident run"
-    assert st.read_status() == 0, "device status word set during timing"
+        def bwd():
+            tw.ffn_bwd(X, W_g, W_u, W_d, st, dY, lam=args.lam, W_dt=Wdt, ws=wsb, out=grads)
+            allreduce_grads(grads)  # data parallel over ranks: weight gradients summed (NCCL); no-op on one rank
 
-    def copy_ms(body, reps=5):
-        """Mean time of one step's host<->device copies alone (no compute), for context."""
-        body()
+        def train_step(e_mid):
+            fwd_train()
+            e_mid.record(stream)
+            bwd()
+
+        def infer(st_i):
+            def body(e_mid):
+                tw.ffn_fwd(X, W_g, b_g, W_u, W_d, T_n=w.T_n, K=K, W_dt=Wdt, state=st_i, ws=wsf, Y=Y)
+                e_mid.record(stream)
+            return body
+
+        if not train:
+            tw.transpose_wd(W_d, out=Wdt)  # fixed weights: transposed once, outside the timed region
+        step = train_step if train else infer(st)
+        for _ in range(max(3, args.warmup)):
+            step(torch.cuda.Event())
         torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
+        assert st.read_status() == 0, f"device status word set during warm-up ({name})"
+        launches0 = tw.launch_count()
+        clk = ClockSampler(local) if full else None
+        if clk:
+            clk.__enter__()
+        ms_step, ms_mid = timed_pair(args.steps, step)
+        if clk:
+            clk.__exit__(None, None, None)
+        res["gpu_launches"] = tw.launch_count() - launches0
+        ms_step, ms_mid = max_over_ranks(ms_step), max_over_ranks(ms_mid)
+        assert st.read_status() == 0, f"device status word set during timing ({name})"
+        res["ms_step"] = ms_step
+        if train:
+            res["ms_fwd"] = ms_mid
+        cnt = st.count.float()
+        nst, nfl = st.n_overflow()
+        ell_rows = (st.row_ovf[:M] == 0).unsqueeze(1)
+        res["kept"] = int((torch.minimum(st.count.int(), torch.tensor(K, device=dev)) * ell_rows).sum().item())
+        res["pairs"] = int(st.count.int().sum().item())
+        res["n_ovf"] = nst
+        res["dense_wgrad"] = int(st.row_plan[3].item())
+        res["sparsity"] = {"activity": res["pairs"] / (M * f), "overflow_rows": nfl,
+                           "max_count": float(cnt.max().item()), "mean_count": float(cnt.mean().item()),
+                           "max_over_mean_count": float(cnt.max().item()) / max(float(cnt.mean().item()), 1e-30)}
+        res["shape"] = (M, d, f, T, K)
+        if full:
+            res["clocks"] = clk.summary()
+            # per-kernel breakdown: the same steps again with event tracing
+            breakdown = {}
+            if not args.no_trace:
+                tw.trace_collect()
+                tw.trace_enable(True)
+                timed_pair(args.steps, step)
+                tw.trace_enable(False)
+                for kname, ms in tw.trace_collect():
+                    b = breakdown.setdefault(kname, {"launches": 0, "ms": 0.0})
+                    b["launches"] += 1
+                    b["ms"] += ms
+                for b in breakdown.values():
+                    b["ms_per_launch"] = b["ms"] / b["launches"]
+                    b["ms_per_step"] = b["ms"] / args.steps
+            res["breakdown"] = breakdown
+            if train:
+                # the inference forward with fixed weights: W_d transposed once, u not saved
+                st_inf = tw.HybridState(M, f, w.T_n, K, cap, dev, with_u=False)
+                res["ms_infer"] = warm_and_time(infer(st_inf))
+                assert st_inf.read_status() == 0, "device status word set during the inference timing"
+                del st_inf
+            res["e2e"] = e2e(M, d, X, dY, Y, lambda Xi, dYi, Yi: (
+                tw.transpose_wd(W_d, out=Wdt),
+                tw.ffn_fwd(Xi, W_g, b_g, W_u, W_d, T_n=w.T_n, K=K, W_dt=Wdt, state=st, ws=wsf, Y=Yi),
+                tw.ffn_bwd(Xi, W_g, W_u, W_d, st, dYi, lam=args.lam, W_dt=Wdt, ws=wsb, out=grads),
+                allreduce_grads(grads)))
+            assert st.read_status() == 0, "device status word set during the end-to-end timing"
+        del st, wsf, wsb, Wdt, Y, grads
+        torch.cuda.empty_cache()
+        if not args.no_dense:
+            res["dense"] = _dense_arm(torch, X, W_g, b_g, W_u, W_d, dY, args.lam, warm_and_time, train)
+        del X, W_g, b_g, W_u, W_d, dY
+        torch.cuda.empty_cache()
+        if full and not args.no_cpu_baseline and world == 1 and rank == 0:
+            res["cpu_baseline"] = cpu_baseline_slice(inp, args.lam, CPU_SLICE_ROWS)
+        return res
+
+    def e2e(M, d, X, dY, Y, run_step):
+        """The same step end to end: every step copies its inputs (X, dY) from
+        pinned host memory and reads its result Y back, inside the timed region.
+        As a training loop that prefetches its next batch does, the copies run on
+        two copy streams (host->device, device->host) into double-buffered device
+        tensors, so step i+1's inputs and step i-1's result move while step i
+        computes. The step's working set is far larger than L2, so no extra flush
+        is inserted."""
+        hX = torch.empty((M, d), dtype=torch.bfloat16, pin_memory=True)
+        hdY = torch.empty((M, d), dtype=torch.bfloat16, pin_memory=True)
+        hY = [torch.empty((M, d), dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
+        hX.copy_(X.cpu())
+        hdY.copy_(dY.cpu())
+        Xb, dYb, Yb = [X, torch.empty_like(X)], [dY, torch.empty_like(dY)], [Y, torch.empty_like(Y)]
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+        def run(n):
+            ev_in = [torch.cuda.Event() for _ in range(2)]
+            ev_done = [torch.cuda.Event() for _ in range(2)]
+            ev_out = [torch.cuda.Event() for _ in range(2)]
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            barrier()
+            torch.cuda.synchronize(dev)
+            t0.record(stream)
+            up.wait_stream(stream)
+            down.wait_stream(stream)
+
+            def load(b):
+                with torch.cuda.stream(up):
+                    Xb[b].copy_(hX, non_blocking=True)
+                    dYb[b].copy_(hdY, non_blocking=True)
+                    ev_in[b].record(up)
+
+            load(0)
+            for i in range(n):
+                b = i % 2
+                if i + 1 < n:
+                    if i >= 1:
+                        up.wait_event(ev_done[1 - b])  # step i-1 has finished reading these buffers
+                    load(1 - b)
+                stream.wait_event(ev_in[b])
+                if i >= 2:
+                    stream.wait_event(ev_out[b])  # step i-2's result has left Yb[b]
+                run_step(Xb[b], dYb[b], Yb[b])
+                ev_done[b].record(stream)
+                down.wait_event(ev_done[b])
+                with torch.cuda.stream(down):
+                    hY[b].copy_(Yb[b], non_blocking=True)
+                    ev_out[b].record(down)
+            stream.wait_stream(down)
+            stream.wait_stream(up)
+            t1.record(stream)
+            torch.cuda.synchronize(dev)
+            barrier()
+            return t0.elapsed_time(t1) / n
+
+        run(max(3, args.warmup))
+        ms = max_over_ranks(run(args.steps))
+        assert torch.equal(hY[(args.steps - 1) % 2].to(dev), Y), "end-to-end result differs from the resident run"
+
+        def copy_ms(body, reps=5):
+            """Mean time of one step's host<->device copies alone (no compute), for context."""
             body()
-        e1.record(stream)
-        e1.synchronize()
-        return e0.elapsed_time(e1) / reps
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                body()
+            e1.record(stream)
+            e1.synchronize()
+            return e0.elapsed_time(e1) / reps
 
-    ms_h2d = copy_ms(lambda: (Xb[1].copy_(hX, non_blocking=True), dYb[1].copy_(hdY, non_blocking=True)))
-    ms_d2h = copy_ms(lambda: hY[1].copy_(Yb[0], non_blocking=True))
+        ms_h2d = copy_ms(lambda: (Xb[1].copy_(hX, non_blocking=True), dYb[1].copy_(hdY, non_blocking=True)))
+        ms_d2h = copy_ms(lambda: hY[1].copy_(Yb[0], non_blocking=True))
+        return {"ms_per_step": ms, "h2d_bytes_per_step": 2 * M * d * 2, "d2h_bytes_per_step": M * d * 2,
+                "copy_alone_ms": {"h2d": ms_h2d, "d2h": ms_d2h}}
 
-    # dense bf16 comparison point (torch / cuBLAS), same protocol
-    dense = None
-    if not args.no_dense:
-        Wg_r, Wu_r, Wd_r = (t.clone().requires_grad_() for t in (W_g, W_u, W_d))
-        Xr = X.clone().requires_grad_()
-
-        def dense_fwd(e_mid):
-            with torch.no_grad():
-                (torch.relu(X @ W_g.T + b_g) * (X @ W_u.T)) @ W_d.T
-            e_mid.record(stream)
-
-        def dense_fb(e_mid):
-            z = Xr @ Wg_r.T + b_g
-            g = torch.relu(z)
-            y = (g * (Xr @ Wu_r.T)) @ Wd_r.T
-            (y.float() * dY.float()).sum().add(g.float().sum() * args.lam).backward()
-            Xr.grad = Wg_r.grad = Wu_r.grad = Wd_r.grad = None
-            e_mid.record(stream)
-
-        for _ in range(3):
-            dense_fwd(torch.cuda.Event())
-            dense_fb(torch.cuda.Event())
-        dm_f, _ = timed(args.steps, dense_fwd)
-        dm_fb, _ = timed(args.steps, dense_fb)
-        dm_f, dm_fb = max_over_ranks(dm_f), max_over_ranks(dm_fb)
-        dense = {"fwd_tokens_per_s": M * world / (dm_f / 1e3), "fwd_bwd_tokens_per_s": M * world / (dm_fb / 1e3),
-                 "fwd_ms": dm_f, "fwd_bwd_ms": dm_fb, "impl": "torch bf16 matmuls (cuBLAS), autograd backward"}
+    main = measure(args.workload, "train", full=True)
+    others = {}
+    if not args.no_extra:
+        for key, wname, mode in OTHER_WORKLOADS:
+            if wname != args.workload:
+                others[key] = measure(wname, mode, full=False)
 
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:
         return
+    print(json.dumps(bench_line(args, world, main, others)), flush=True)
 
+
+def bench_line(args, world, main, others):
+    """The JSON line of the TwELL arm from the measurements (host arithmetic only)."""
     peaks, peak_src = load_peaks()
-    ell_rows = (st.row_ovf[:M] == 0).unsqueeze(1)
-    kept = int((torch.minimum(st.count.int(), torch.tensor(K, device=dev)) * ell_rows).sum().item())
-    pairs = int(st.count.int().sum().item())
-    roofline = None
-    if breakdown:
-        top = max(breakdown, key=lambda k: breakdown[k]["ms"])
-        bound, work = kernel_work(top, M, d, f, T, K, kept, pairs)
-        b = breakdown[top]
-        if bound == "tensor":
-            peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-            achieved = work / (b["ms_per_launch"] / 1e3) / 1e12
-            unit = "TFLOP/s"
-        elif bound == "hbm":
-            peak = peaks["hbm_gbs"]
-            achieved = work / (b["ms_per_launch"] / 1e3) / 1e9
-            unit = "GB/s"
-        else:
-            peak = achieved = None
-            unit = None
-        roofline = {"kernel": top, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                    "frac": (achieved / peak) if achieved and peak else None,
-                    "traffic": committed_traffic(top),
-                    "peak_source": f"{peak_src} ({'sustained bf16' if bound == 'tensor' else 'HBM copy'}, "
-                                   "MEASURED_PEAKS.json)",
-                    "work_per_launch": work,
-                    "share_of_step": b["ms_per_step"] / ms_step if ms_step else None}
-
-    cpu = None
-    if not args.no_cpu_baseline and world == 1:
-        cpu, _, _ = cpu_baseline(inp, args.lam, args.cpu_seconds)
-
+    M, d, f, T, K = main["shape"]
     tokens = M * world
-    line = {
+    ms_step, ms_fwd = main["ms_step"], main["ms_fwd"]
+    kernels, roofline = kernel_table(main["breakdown"], main, peaks, peak_src, args.steps, ms_step, args.workload)
+    dense = main.get("dense")
+    e = main["e2e"]
+
+    def summary(r, train):
+        out = {"workload": r["workload"], "ovf_cap": r["ovf_cap"], "sparsity": r["sparsity"]}
+        tok = r["M"] * world
+        if train:
+            out["fwd_bwd"] = {"tokens_per_s": tok / (r["ms_step"] / 1e3), "ms": r["ms_step"]}
+            out["fwd"] = {"tokens_per_s": tok / (r["ms_fwd"] / 1e3), "ms": r["ms_fwd"]}
+        else:
+            out["fwd_inference"] = {"tokens_per_s": tok / (r["ms_step"] / 1e3), "ms": r["ms_step"]}
+        dn = r.get("dense")
+        if dn:
+            out["dense_bf16"] = dn
+            out["speedup_vs_dense"] = ({"fwd": dn["fwd_best"]["ms"] / r["ms_fwd"],
+                                        "fwd_bwd": dn["fwd_bwd_best"]["ms"] / r["ms_step"]} if train else
+                                       {"fwd_inference": dn["fwd_best"]["ms"] / r["ms_step"]})
+        return out
+
+    return {
         "metric": METRIC,
         "value": tokens / (ms_step / 1e3),
         "unit": "tokens/s",
@@ -651,33 +785,66 @@ def run_twell(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": workload_desc(w, seed), "global_batch": tokens, "lambda_l1": args.lam,
-                   "l2": "flushed before every timed step (256 MiB device write, outside the events)",
-                   "accumulation": "fp32", "ovf_cap": cap, "parallelism": f"replicas x{world}"},
+        "config": {"workload": main["workload"], "global_batch": tokens, "lambda_l1": args.lam,
+                   "l2": "flushed before every timed step (256 MiB device write, outside the events); "
+                         "the step's inputs are also larger than L2",
+                   "accumulation": "fp32", "ovf_cap": main["ovf_cap"],
+                   "parallelism": (f"dp{world}: every rank its own {M} tokens, weight gradients summed over "
+                                   "ranks (NCCL all-reduce) inside each step" if world > 1 else "dp1")},
         "fwd": {"tokens_per_s": tokens / (ms_fwd / 1e3), "ms": ms_fwd,
                 "note": "forward half of the training step (W_d transposed, u saved)"},
-        "fwd_inference": {"tokens_per_s": tokens / (ms_inf / 1e3), "ms": ms_inf,
+        "fwd_inference": {"tokens_per_s": tokens / (main["ms_infer"] / 1e3), "ms": main["ms_infer"],
                           "note": "forward alone with fixed weights (W_dt prepared once, u not saved)"},
         "dense_bf16": dense,
-        "speedup_vs_dense": ({"fwd": dense["fwd_ms"] / ms_fwd, "fwd_inference": dense["fwd_ms"] / ms_inf,
-                              "fwd_bwd": dense["fwd_bwd_ms"] / ms_step}
-                             if dense else None),
-        "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": 2 * M * d * 2,
-                "d2h_bytes_per_step": M * d * 2, "ms_per_step": ms_e2e,
-                "copy_alone_ms": {"h2d": ms_h2d, "d2h": ms_d2h},
+        "speedup_vs_dense": ({"fwd": dense["fwd_best"]["ms"] / ms_fwd,
+                              "fwd_inference": dense["fwd_best"]["ms"] / main["ms_infer"],
+                              "fwd_bwd": dense["fwd_bwd_best"]["ms"] / ms_step} if dense else None),
+        "e2e": {"value": tokens / (e["ms_per_step"] / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": e["h2d_bytes_per_step"], "d2h_bytes_per_step": e["d2h_bytes_per_step"],
+                "ms_per_step": e["ms_per_step"], "copy_alone_ms": e["copy_alone_ms"],
                 "copies": "pinned host X and dY in and Y out every step, on two copy streams, overlapping the "
                           "neighbouring steps' compute (double-buffered device inputs and outputs)"},
-        "gpu_launches": launches,
+        "gpu_launches": main["gpu_launches"],
         "roofline": roofline,
-        "path_roofline": path_roofline(M, d, f, T, K, kept, nst, peaks, ms_fwd, ms_step),
-        "kernels": {k: {"launches_per_step": v["launches"] / args.steps, "ms_per_step": v["ms_per_step"]}
-                    for k, v in sorted(breakdown.items(), key=lambda kv: -kv[1]["ms"])},
-        "sparsity": {"activity": activity, "overflow_rows": nfl, "max_count": float(cnt.max().item()),
-                     "mean_count": float(cnt.mean().item())},
-        "clocks": clk.summary(),
-        "cpu_baseline": cpu,
+        "path_roofline": path_roofline(M, d, f, T, K, main["kept"], main["n_ovf"], peaks, ms_fwd, ms_step),
+        "kernels": kernels,
+        "sparsity": main["sparsity"],
+        "clocks": main["clocks"],
+        "cpu_baseline": main.get("cpu_baseline"),
+        "other_workloads": {k: summary(r, r.get("ms_fwd") is not None) for k, r in others.items()},
     }
-    print(json.dumps(line), flush=True)
+
+
+def kernel_table(breakdown, r, peaks, peak_src, steps, ms_step, wname):
+    """Per-kernel time per step from the event trace, with the algorithmic work
+    and roofline fraction of every kernel whose work is defined; and the
+    roofline object of the dominant kernel (the one with the most time)."""
+    M, d, f, T, K = r["shape"]
+    table = {}
+    for k, v in sorted(breakdown.items(), key=lambda kv: -kv[1]["ms"]):
+        row = {"launches_per_step": v["launches"] / steps, "ms_per_step": v["ms_per_step"]}
+        bound, work = kernel_work(k, M, d, f, T, K, r["kept"], r["pairs"], r["n_ovf"], r["dense_wgrad"])
+        if bound:
+            peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) if bound == "tensor" else peaks["hbm_gbs"]
+            achieved = work / (v["ms_per_launch"] / 1e3) / (1e12 if bound == "tensor" else 1e9)
+            row.update({"bound": bound, "work_per_launch": work, "achieved": achieved,
+                        "unit": "TFLOP/s" if bound == "tensor" else "GB/s", "frac": achieved / peak})
+        table[k] = row
+    roofline = None
+    if breakdown:
+        top = max(breakdown, key=lambda k: breakdown[k]["ms"])
+        row = table[top]
+        bound = row.get("bound")
+        peak = None
+        if bound:
+            peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) if bound == "tensor" else peaks["hbm_gbs"]
+        roofline = {"kernel": top, "bound": bound, "achieved": row.get("achieved"), "peak": peak,
+                    "unit": row.get("unit"), "frac": row.get("frac"), "traffic": committed_traffic(top, wname),
+                    "peak_source": f"{peak_src} ({'sustained bf16' if bound == 'tensor' else 'HBM copy'}, "
+                                   "MEASURED_PEAKS.json)",
+                    "work_per_launch": row.get("work_per_launch"),
+                    "share_of_step": breakdown[top]["ms_per_step"] / ms_step if ms_step else None}
+    return table, roofline
 
 
 # ---------------------------------------------------------------- sweep

@@ -61,7 +61,8 @@ typedef enum twell_status {
   TWELL_EOVERFLOW_CAP = 3,  /* (device bit) more overflow rows than ovf_cap */
   TWELL_ECUDA = 4,          /* a CUDA runtime or driver call failed */
   TWELL_ETIMEOUT = 5,       /* (device bit) a bounded device-side wait gave up */
-  TWELL_EWORKSPACE = 6      /* workspace too small or misaligned */
+  TWELL_EWORKSPACE = 6,     /* workspace too small or misaligned */
+  TWELL_EBOUNDS = 7         /* (device bit, bounds-checked build only) an index read from a buffer was out of range */
 } twell_status;
 
 /* Device status word bits, set by kernels and read by twell_status_read. */
@@ -70,6 +71,13 @@ typedef enum twell_status {
 /* The state given to a call cannot serve it (a tile-routed inference state
  * passed to twell_ffn_bwd); the call wrote no result. */
 #define TWELL_STATUS_BAD_STATE (1u << TWELL_EINVAL)
+/* Set only by the bounds-checked build of the library (libtwell_bounds.so,
+ * compiled with -DTWELL_BOUNDS): its kernels check every index they read from
+ * a buffer (a slot's in-tile column, a piece's row, an overflow row, a dense
+ * slot, a pair-list row or position) against the extent it addresses before the
+ * access it steers; an index out of range sets this bit and the access is
+ * skipped. The regular build never sets it and does not check. */
+#define TWELL_STATUS_BOUNDS (1u << TWELL_EBOUNDS)
 
 /*
  * The hybrid TwELL representation of g = ReLU(z) ([aivizor] ¶2: horizontal
@@ -178,13 +186,18 @@ TWELL_API twell_status twell_pack(const uint16_t* X, const uint16_t* W_g, const 
  *   Scratch: the only scratch twell_pack needs, the dense slices spilled for
  *   tiles with more than K actives, lives in a file-scope device array of
  *   TWELL_NOALLOC_SCRATCH_BYTES that the library owns; every device that loads
- *   the library keeps it until the process exits. Nothing is allocated or
- *   freed by the call, by the library or by any library it calls.
+ *   the library keeps it until the process exits. The call itself never calls
+ *   cudaMalloc, cudaFree or an allocating library routine.
  *   Limit: M * d_ff * 2 <= TWELL_NOALLOC_SCRATCH_BYTES (M * d_ff <= 8,388,608);
  *   larger shapes return TWELL_EWORKSPACE and enqueue nothing.
  *   Set-up: the first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress, with the caller's current device, which must be the
- *   device of `stream`); make that first call before any stream capture.
+ *   device of `stream`). Under CUDA's lazy module loading (the default since
+ *   CUDA 12.2) that lookup is also when the driver loads this code onto the
+ *   device and reserves the array's 16 MiB there, so the first call on each
+ *   device does take device memory: make it at set-up time, before a host
+ *   allocator claims the device's memory (else it can fail with TWELL_ECUDA)
+ *   and before any stream capture. Later calls on that device reserve nothing.
  *   Sharing: all calls share the one array and the array keeps whatever the
  *   last call left in it. A call writes every scratch slice before it reads it,
  *   so nothing has to start at zero; but calls whose execution overlaps on the
@@ -238,6 +251,11 @@ TWELL_API twell_status twell_ffn_fwd_tiles(const uint16_t* X, const uint16_t* W_
  *   dY [M][d_model] bf16 bits; dX [M][d_model], dW_g / dW_u [d_ff][d_model],
  *   dW_d [d_model][d_ff], db_g [d_ff] (nullable): fp32, overwritten (not accumulated).
  *   ws  workspace of twell_workspace_bytes(TWELL_OP_BWD, ...) bytes
+ * Overflow rows that the forward flagged but could not store (more than
+ * ovf_cap of them; the forward set TWELL_STATUS_OVERFLOW_CAP) have no stored g
+ * or u: their dX rows are not written (they keep whatever the buffer held),
+ * their pairs are left out of dW_g, dW_u, dW_d and db_g, and the backward sets
+ * TWELL_STATUS_OVERFLOW_CAP again. Every other row is computed as usual.
  * TWELL_EUNSUPPORTED (and a zero TWELL_OP_BWD workspace size) when the weight
  * gradients' pair list could exceed 2^31 - 1 entries, i.e. when
  * (M - ovf_cap) * (d_ff / T_n) * K + ovf_cap * d_ff > 2^31 - 1 (its positions
@@ -275,6 +293,22 @@ TWELL_API twell_status twell_count_stats(const twell_hybrid* h, int64_t* rows_by
 /* Copies the device status word to *out after synchronizing `stream`; clears
  * it when `clear` is non-zero. Returns TWELL_ECUDA if the copy fails. */
 TWELL_API twell_status twell_status_read(const twell_hybrid* h, uint32_t* out, int clear, twell_stream_t stream);
+
+/*
+ * Test of failure detection (no counterpart on the pages; a test aid). The
+ * dense-backup GEMMs of twell_ffn_fwd and twell_ffn_bwd may split their K
+ * range when few rows overflow; the four epilogue warps of such a GEMM meet at
+ * a bounded barrier before the tile's partial sums are counted and reduced.
+ * After this call, the next `launches` of those GEMMs (each launch that can
+ * split counts, whether or not it splits on the device) run with one epilogue
+ * warp that never arrives at that barrier, as if it had stalled: the wait runs
+ * out after its limit (2 s), the kernel sets TWELL_STATUS_TIMEOUT, counts no
+ * arrival for the tile (so no CTA reduces partial sums that may be missing),
+ * and unwinds; the rows that GEMM should have written are left unwritten.
+ * launches <= 0 cancels what is left. Nothing else changes; the context stays
+ * usable.
+ */
+TWELL_API void twell_test_withhold_epilogue_arrival(int launches);
 
 /*
  * Launch accounting and per-kernel timing (no counterpart on the pages; a

@@ -58,6 +58,9 @@ WORKLOADS = {
     "heavy": Workload("heavy", 16384, 4096, 14336, 128, 8, 0.01, row_scale="lognormal"),
     # one training step of a sparse FFN layer
     "train": Workload("train", 8192, 2048, 8192, 128, 8, 0.01, training=True),
+    # the largest single-GPU point of the d_model=4096, d_ff=14336 sweep at 99% sparsity,
+    # run as a training step (the throughput workload of bench.py)
+    "large": Workload("large", 65536, 4096, 14336, 128, 8, 0.01, row_scale="lognormal", training=True),
 }
 
 
@@ -82,9 +85,13 @@ def bf16_bits_from_f64(a: np.ndarray) -> np.ndarray:
     to the float32 pattern and truncates, which is round-half-to-even on finite values.
     """
     f32 = np.ascontiguousarray(a, dtype=np.float32)
-    u = f32.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return u.astype(np.uint16)
+    u = f32.view(np.uint32)
+    # finite patterns are at most 0xFF7FFFFF, so the sum below stays within 32 bits
+    r = (u >> 16) & 1
+    r += 0x7FFF
+    r += u
+    r >>= 16
+    return r.astype(np.uint16)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
@@ -126,9 +133,11 @@ def gate_bias_for_activity(activity: float, row_scale: str = "none", sigma: floa
 def _draw_rows(rng: np.random.Generator, rows: int, cols: int, scale: float,
                row_scale: Optional[np.ndarray] = None) -> np.ndarray:
     out = np.empty((rows, cols), dtype=np.uint16)
+    buf = np.empty((min(rows, _ROW_CHUNK), cols), dtype=np.float64)
     for r0 in range(0, rows, _ROW_CHUNK):
         r1 = min(rows, r0 + _ROW_CHUNK)
-        a = rng.standard_normal((r1 - r0, cols))
+        a = buf[: r1 - r0]
+        rng.standard_normal(out=a)
         if scale != 1.0:
             a *= scale
         if row_scale is not None:
@@ -138,34 +147,52 @@ def _draw_rows(rng: np.random.Generator, rows: int, cols: int, scale: float,
 
 
 def make_inputs(w: Workload, seed: Optional[int] = None, with_dY: Optional[bool] = None,
-                M: Optional[int] = None) -> dict:
+                M: Optional[int] = None, shard: int = 0) -> dict:
     """Draw one workload. Returns uint16 (bf16 bit) arrays and the recipe metadata.
 
     Keys: X [M, d], W_g [f, d], b_g [f], W_u [f, d], W_d [d, f], dY [M, d] (training),
     plus "meta" with the seed, the calibrated bias value (as float) and the shapes.
-    `M` overrides the token count (the weights do not depend on it).
+    `M` overrides the token count (the weights do not depend on it). `shard` > 0
+    draws another batch of tokens for the same weights (the per-token streams X,
+    s and dY come from the children of SeedSequence([seed, shard]); the weights
+    from the seed's own), as the ranks of a data-parallel step hold; shard 0 is
+    the plain draw.
     """
     seed = w.seed if seed is None else int(seed)
     with_dY = w.training if with_dY is None else bool(with_dY)
     M = w.M if M is None else int(M)
     d, f = w.d_model, w.d_ff
     streams = dict(zip(_STREAMS, np.random.SeedSequence(seed).spawn(len(_STREAMS))))
+    if shard:
+        tok = dict(zip(_STREAMS, np.random.SeedSequence([seed, int(shard)]).spawn(len(_STREAMS))))
+        streams.update({k: tok[k] for k in ("X", "s", "dY")})
     g = {k: np.random.Generator(np.random.PCG64(v)) for k, v in streams.items()}
 
     s = None
     if w.row_scale == "lognormal":
         s = np.exp(w.sigma * g["s"].standard_normal(M))
-    X = _draw_rows(g["X"], M, d, 1.0, s)
-    W_g = _draw_rows(g["W_g"], f, d, 1.0 / math.sqrt(d))
-    W_u = _draw_rows(g["W_u"], f, d, 1.0 / math.sqrt(d))
-    W_d = _draw_rows(g["W_d"], d, f, 1.0 / math.sqrt(f))
+    # each tensor has its own stream, so the draws run concurrently (numpy releases
+    # the GIL in bulk fills) and give the same values as drawing them one by one
+    jobs = {"X": (g["X"], M, d, 1.0, s), "W_g": (g["W_g"], f, d, 1.0 / math.sqrt(d)),
+            "W_u": (g["W_u"], f, d, 1.0 / math.sqrt(d)), "W_d": (g["W_d"], d, f, 1.0 / math.sqrt(f))}
+    if with_dY:
+        jobs["dY"] = (g["dY"], M, d, 1.0)
+    big = M * d + 3 * f * d > (1 << 24)
+    if big:
+        from concurrent.futures import ThreadPoolExecutor
+
+        with ThreadPoolExecutor(max_workers=len(jobs)) as ex:
+            futs = {k: ex.submit(_draw_rows, *a) for k, a in jobs.items()}
+            drawn = {k: fu.result() for k, fu in futs.items()}
+    else:
+        drawn = {k: _draw_rows(*a) for k, a in jobs.items()}
     b = gate_bias_for_activity(w.activity, w.row_scale, w.sigma)
     b_bits = bf16_bits_from_f64(np.full(f, b))
-    out = dict(X=X, W_g=W_g, b_g=b_bits, W_u=W_u, W_d=W_d)
+    out = dict(X=drawn["X"], W_g=drawn["W_g"], b_g=b_bits, W_u=drawn["W_u"], W_d=drawn["W_d"])
     if with_dY:
-        out["dY"] = _draw_rows(g["dY"], M, d, 1.0)
+        out["dY"] = drawn["dY"]
     out["meta"] = dict(
-        workload=w.name, seed=seed, M=M, d_model=d, d_ff=f, T_n=w.T_n, K=w.K,
+        workload=w.name, seed=seed, shard=int(shard), M=M, d_model=d, d_ff=f, T_n=w.T_n, K=w.K,
         target_activity=w.activity, row_scale=w.row_scale, sigma=w.sigma,
         b_g=float(bf16_bits_to_f32(b_bits[:1])[0]),
     )

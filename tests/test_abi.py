@@ -133,10 +133,23 @@ def test_host_side_errors(tw):
 
 
 def test_missing_library_fails_loudly(tw, monkeypatch):
-    monkeypatch.setattr(tw, "_lib", None)
+    monkeypatch.setattr(tw, "_libs", {})
     monkeypatch.setattr(tw, "LIB_PATH", os.path.join(ROOT, "does_not_exist", "libtwell.so"))
     with pytest.raises(RuntimeError, match="missing"):
         tw.lib()
+
+
+def test_bounds_checked_library_exports_the_same_symbols(tw):
+    """libtwell_bounds.so (the -DTWELL_BOUNDS build) exports exactly the header's
+    entry points too, and bounds_checked() routes the binding to it."""
+    out = os.popen(f"nm -D --defined-only {tw.BOUNDS_LIB_PATH}").read()
+    assert set(re.findall(r"\bT (twell_[a-z_0-9]+)\b", out)) == set(declared_functions())
+    plain = tw.lib()
+    with tw.bounds_checked() as L:
+        assert L is not plain and tw.lib() is L
+        assert tw.query_support(64, 256, 1024, 128, 8, 64) == 0
+    assert tw.lib() is plain
+    assert tw.STATUS_BOUNDS == 1 << 7
 
 
 def test_pair_list_bound(tw):

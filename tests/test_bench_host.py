@@ -70,9 +70,19 @@ def test_kernel_work_by_hand():
     # X + TwELL + u + Y + W_u and W_dt once
     assert bench.kernel_work("ell_updown", M, d, f, T, K, kept, pairs) == (
         "hbm", 2 * 32 + 4 * 2 * 26 + 40 + 2 * 32 + 4 * 256 * 8)
-    # X, TwELL, u, (dU, dZ) per slot, dX fp32, three weight matrices once
+    # dY, TwELL, u, (h, dU, dZ, 0) per slot, dX fp32, three weight matrices once
     assert bench.kernel_work("ell_bwd", M, d, f, T, K, kept, pairs) == (
-        "hbm", 2 * 32 + 4 * 2 * 26 + 40 + 80 + 4 * 32 + 6 * 256 * 8)
+        "hbm", 2 * 32 + 4 * 2 * 26 + 40 + 160 + 4 * 32 + 6 * 256 * 8)
+    # one overflow row: the ELL rows are the other three
+    assert bench.kernel_work("ell_updown", M, d, f, T, K, kept, pairs, n_ovf=1) == (
+        "hbm", 2 * 24 + 3 * 2 * 26 + 40 + 2 * 24 + 4 * 256 * 8)
+    assert bench.kernel_work("ovf_dx_gemm", M, d, f, T, K, kept, pairs, n_ovf=3) == ("tensor", 4.0 * 3 * 8 * 256)
+    assert bench.kernel_work("ovf_up_gemm", M, d, f, T, K, kept, pairs, n_ovf=3) == ("tensor", 2.0 * 3 * 8 * 256)
+    # the pair list holds the overflow rows' pairs unless their gradients run as GEMMs
+    sparse = bench.kernel_work("weight_grads", M, d, f, T, K, kept, pairs, n_ovf=1, dense_wgrad=0)[1]
+    dense = bench.kernel_work("weight_grads", M, d, f, T, K, kept, pairs, n_ovf=1, dense_wgrad=1)[1]
+    assert sparse == 4 * 32 + 20 * 12 + 12 * 256 * 8 + 4 * 256
+    assert dense == 4 * 32 + 20 * 10 + 24 * 256 * 8 + 4 * 256
     assert bench.kernel_work("transpose_wd", M, d, f, T, K, kept, pairs) == ("hbm", 4 * 256 * 8)
     assert bench.kernel_work("row_flags", M, d, f, T, K, kept, pairs) == (None, None)
 
@@ -88,22 +98,49 @@ def test_path_roofline_fractions():
 
 def test_committed_traffic_follows_the_sources(monkeypatch):
     with open(bench.os.path.join(bench.ROOT, "profiles", "dram_traffic.json")) as fh:
-        rec = json.load(fh)["kernels"]
-    for k, v in rec.items():
-        got = bench.committed_traffic(k)
-        if v["source_sha"] == bench.source_hash(k):
-            assert got == v["dram_bytes_per_launch"]
-        else:
-            assert got is None
+        wls = json.load(fh)["workloads"]
+    assert wls
+    for wname, wrec in wls.items():
+        for k, v in wrec["kernels"].items():
+            got = bench.committed_traffic(k, wname)
+            if v["source_sha"] == bench.source_hash(k):
+                assert got == v["dram_bytes_per_launch"]
+            else:
+                assert got is None
+    assert bench.committed_traffic("gate_pack_gemm", "no such workload") is None
     monkeypatch.setattr(bench, "source_hash", lambda kernel: "changed")
-    assert all(bench.committed_traffic(k) is None for k in rec)
+    assert all(bench.committed_traffic(k, wname) is None for wname, wrec in wls.items() for k in wrec["kernels"])
 
 
-def test_workload_is_the_uniform_shape_with_the_golden_seed():
+def test_workloads_of_the_line():
+    """The timed training step runs the largest single-GPU sweep point at 99% sparsity;
+    the uniform inference workload keeps its golden seed."""
     w, seed = bench.workload()
+    assert (w.M, w.d_model, w.d_ff, w.T_n, w.K, w.activity, w.row_scale) == (
+        65536, 4096, 14336, 128, 8, 0.01, "lognormal")
+    assert "M=65536" in bench.workload_desc(w, seed) and "99% sparsity" in bench.workload_desc(w, seed)
+    w, seed = bench.workload("uniform")
     assert (w.M, w.d_model, w.d_ff, w.T_n, w.K, w.activity) == (4096, 2048, 8192, 128, 8, 0.01)
     with open(bench.os.path.join(bench.ROOT, "tests", "golden", "uniform_seed.json")) as fh:
         assert seed == json.load(fh)["seed"]
+    assert bench.ovf_cap_for(w) == 1024
+
+
+def test_kernel_table_and_dominant_kernel():
+    """Per-kernel fractions from the event trace; the roofline object is the kernel with the most time."""
+    peaks = {"hbm_gbs": 1000.0, "bf16_tflops": 2.0, "bf16_tflops_sustained": 1.0}
+    r = {"shape": (128, 64, 256, 2, 8), "kept": 100, "pairs": 120, "n_ovf": 2, "dense_wgrad": 0}
+    bd = {"gate_pack_gemm": {"launches": 2, "ms": 4.0, "ms_per_launch": 2.0, "ms_per_step": 2.0},
+          "ell_updown": {"launches": 2, "ms": 1.0, "ms_per_launch": 0.5, "ms_per_step": 0.5},
+          "row_flags": {"launches": 2, "ms": 0.1, "ms_per_launch": 0.05, "ms_per_step": 0.05}}
+    table, roof = bench.kernel_table(bd, r, peaks, "measured", 2, 4.0, "large")
+    assert list(table) == ["gate_pack_gemm", "ell_updown", "row_flags"]
+    flops = 2.0 * 128 * 64 * 256
+    assert table["gate_pack_gemm"]["achieved"] == pytest.approx(flops / 2e-3 / 1e12)
+    assert table["gate_pack_gemm"]["frac"] == pytest.approx(flops / 2e-3 / 1e12 / 1.0)
+    assert "frac" not in table["row_flags"]
+    assert roof["kernel"] == "gate_pack_gemm" and roof["bound"] == "tensor" and roof["peak"] == 1.0
+    assert roof["share_of_step"] == pytest.approx(0.5)
 
 
 def test_reference_arm_prints_the_contract_line():
@@ -112,7 +149,7 @@ def test_reference_arm_prints_the_contract_line():
     import subprocess
 
     out = subprocess.run([sys.executable, bench.os.path.join(bench.ROOT, "bench.py"), "--impl", "reference",
-                          "--steps", "1", "--warmup", "0", "--cpu-seconds", "0.05"],
+                          "--workload", "train", "--steps", "1", "--warmup", "0", "--cpu-seconds", "0.05"],
                          capture_output=True, text=True, timeout=600, cwd=bench.ROOT)
     assert out.returncode == 0, out.stderr[-2000:]
     lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]

@@ -1,9 +1,11 @@
 """GPU parity of the sm_100a path against the fp64 CPU oracle, through the C ABI.
 
 Small cases compare every output element; the full-size workloads compare the
-pack on every row and Y on a seeded sample of rows plus every overflow row, and
-the training workload's gradients on full tensors. Tolerances are stated in
-tests/twell_testlib.py.
+pack on every row, the gate output element by element, and Y on every row (the
+uniform inference workload) or on a seeded sample of rows plus every overflow
+row (the heavy-tailed ones); the training workloads' gradients on full tensors.
+Tolerances are stated in tests/twell_testlib.py: the plain bounds on the
+uniform cases, the per-row reading on the lognormal ones.
 """
 
 import json
@@ -13,8 +15,8 @@ import numpy as np
 import pytest
 
 from synthetic import WORKLOADS, Workload, make_inputs, sweep_workload
-from twell_testlib import (assert_active_set, assert_matches_oracle, assert_pack_equal, assert_plan_valid, bits_of,
-                           f32_of_bits, gpu_gmat, state_to_numpy, to_dev)
+from twell_testlib import (assert_active_set, assert_gate_close, assert_matches_oracle, assert_pack_equal,
+                           assert_plan_valid, bits_of, f32_of_bits, gate_error_bound, gpu_gmat, state_to_numpy, to_dev)
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -45,7 +47,8 @@ def _run_fwd(tw, inp, w, cap=None, save=True, dense_min=0):
 
 
 def _check_fwd(orc, inp, w, Y, st, z, rows=None, cap=None):
-    """Pack bit-exact (all rows), active set and Y (all rows or the given sample)."""
+    """Pack bit-exact (all rows); gate z element by element, active set and Y
+    (all rows or the given sample)."""
     M, f = inp["X"].shape[0], inp["W_g"].shape[0]
     zg = z.cpu().numpy()
     p_gpu = state_to_numpy(st)
@@ -56,22 +59,30 @@ def _check_fwd(orc, inp, w, Y, st, z, rows=None, cap=None):
     if rows is None:
         rows = np.arange(M, dtype=np.int32)
     z64 = orc.gate(inp["X"], inp["W_g"], inp["b_g"], rows=rows)
+    assert_gate_close(zg[rows], z64, gate_error_bound(inp["X"], inp["W_g"], inp["b_g"], rows=rows))
     flips = assert_active_set(zg[rows], z64, float(np.sqrt(np.mean(z64 ** 2))))
     args = (inp["X"], inp["W_g"], inp["b_g"], inp["W_u"], inp["W_d"])
     G = gpu_gmat(p_gpu, M, f, w.T_n, w.K)
     y_stored = orc.ffn_fwd(*args, rows=rows, gmat=G[rows])
     y_plain = orc.ffn_fwd(*args, rows=rows)
     yg = f32_of_bits(bits_of(Y))[rows]
-    stats = assert_matches_oracle(yg, y_stored, y_plain, "Y", bf16_out=True)
+    stats = assert_matches_oracle(yg, y_stored, y_plain, "Y", bf16_out=True, per_row=w.row_scale == "lognormal")
     return p_gpu, flips, stats
 
 
-def _check_bwd(orc, inp, g, G, lam, name):
+def _check_bwd(orc, inp, g, G, lam, name, per_row, skip_rows=None):
+    """Every gradient on its full tensor (dX without the rows in skip_rows)."""
     args = (inp["X"], inp["W_g"], inp["b_g"], inp["W_u"], inp["W_d"], inp["dY"], lam)
     ref_s = orc.ffn_bwd(*args, gmat=G)
     ref_p = orc.ffn_bwd(*args, mask=(G != 0).astype(np.uint8))
+    keep = None
+    if skip_rows is not None and len(skip_rows):
+        keep = np.setdiff1d(np.arange(inp["X"].shape[0]), skip_rows)
     for k in ("dX", "dW_g", "dW_u", "dW_d", "db_g"):
-        assert_matches_oracle(g[k].cpu().numpy(), ref_s[k], ref_p[k], f"{name} {k} lambda={lam}")
+        a, rs, rp = g[k].cpu().numpy(), ref_s[k], ref_p[k]
+        if k == "dX" and keep is not None:
+            a, rs, rp = a[keep], rs[keep], rp[keep]
+        assert_matches_oracle(a, rs, rp, f"{name} {k} lambda={lam}", per_row=per_row)
 
 
 CASES = {
@@ -128,7 +139,7 @@ def test_fwd_bwd_small(tw, orc, name):
     for lam in (0.0, 1e-3):
         g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=lam)
         torch.cuda.synchronize()
-        _check_bwd(orc, inp, g, gpu_gmat(p, M, f, 128, K), lam, name)
+        _check_bwd(orc, inp, g, gpu_gmat(p, M, f, 128, K), lam, name, per_row=rs == "lognormal")
         assert_plan_valid(st)
 
 
@@ -154,7 +165,7 @@ def test_degenerate_all_active_dense_path(tw, orc):
     assert p["n_ovf"] == 150 and p["row_ovf"].all()
     assert assert_plan_valid(st)["dense_wgrad"]
     g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=1e-3)
-    _check_bwd(orc, inp, g, gpu_gmat(p, 150, 384, 128, 8), 1e-3, "all-active")
+    _check_bwd(orc, inp, g, gpu_gmat(p, 150, 384, 128, 8), 1e-3, "all-active", per_row=False)
 
 
 def test_overflow_capacity_exceeded(tw, orc):
@@ -226,14 +237,14 @@ def _sample_rows(M, n, seed, extra=()):
 
 
 def test_uniform_full_size(tw, orc):
-    """Inference forward, uniform 1% activity, M=4096 d=2048 d_ff=8192 K=8 (no overflow rows)."""
+    """Inference forward, uniform 1% activity, M=4096 d=2048 d_ff=8192 K=8 (no overflow rows):
+    the gate output and Y on every row."""
     w = WORKLOADS["uniform"]
     with open(os.path.join(GOLDEN, "uniform_seed.json")) as fh:
         seed = json.load(fh)["seed"]
     inp = make_inputs(w, seed=seed)
     D, Y, st, z = _run_fwd(tw, inp, w, save=False)
-    rows = _sample_rows(w.M, 256, 0)
-    p, flips, stats = _check_fwd(orc, inp, w, Y, st, z, rows=rows)
+    p, flips, stats = _check_fwd(orc, inp, w, Y, st, z)
     assert p["n_ovf_total"] == 0
     assert assert_plan_valid(st)["split_rows"] == 0  # 1% i.i.d. rows are short: one piece each
 
@@ -269,7 +280,7 @@ def test_train_full_size(tw, orc):
     for lam in (0.0, 1e-3):
         g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=lam)
         torch.cuda.synchronize()
-        _check_bwd(orc, inp, g, G, lam, "train")
+        _check_bwd(orc, inp, g, G, lam, "train", per_row=False)
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged", "heavy_small", "one_row", "k64"])
@@ -319,7 +330,7 @@ def test_dense_min_routing(tw, orc, name, frac):
     for lam in (0.0, 1e-3):
         g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=lam)
         torch.cuda.synchronize()
-        _check_bwd(orc, inp, g, gpu_gmat(p, M, f, 128, K), lam, f"{name} dense_min={dm}")
+        _check_bwd(orc, inp, g, gpu_gmat(p, M, f, 128, K), lam, f"{name} dense_min={dm}", per_row=rs == "lognormal")
     assert st.read_status() == 0
 
 
@@ -346,7 +357,7 @@ def test_autograd_function(tw, orc):
     args = (inp["X"], inp["W_g"], inp["b_g"], inp["W_u"], inp["W_d"])
     G = gpu_gmat(state_to_numpy(st), M, f, 128, K)
     assert_matches_oracle(f32_of_bits(bits_of(Y_ref)), orc.ffn_fwd(*args, gmat=G), orc.ffn_fwd(*args),
-                          "autograd Y", bf16_out=True)
+                          "autograd Y", bf16_out=True, per_row=rs == "lognormal")
 
 
 def test_count_stats_empty_batch(tw):
@@ -375,7 +386,7 @@ def test_sweep_points(tw, orc, M, activity, bwd):
         g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=1e-3)
         torch.cuda.synchronize()
         assert st.read_status() == 0
-        _check_bwd(orc, inp, g, G, 1e-3, w.name)
+        _check_bwd(orc, inp, g, G, 1e-3, w.name, per_row=True)
 
 
 @pytest.mark.parametrize("name", ["k32", "multi_tile", "ragged_k16", "tiny"])
@@ -406,7 +417,8 @@ def test_tile_routing_forward(tw, orc, name):
     args = (inp["X"], inp["W_g"], inp["b_g"], inp["W_u"], inp["W_d"])
     y_stored = orc.ffn_fwd(*args, gmat=G)
     y_plain = orc.ffn_fwd(*args)
-    assert_matches_oracle(f32_of_bits(bits_of(Y)), y_stored, y_plain, f"{name} tile-routed Y", bf16_out=True)
+    assert_matches_oracle(f32_of_bits(bits_of(Y)), y_stored, y_plain, f"{name} tile-routed Y", bf16_out=True,
+                          per_row=rs == "lognormal")
     # the inference-only state is refused by the backward, which writes nothing
     tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=0.0)
     assert st.read_status(clear=True) == tw.STATUS_BAD_STATE
@@ -443,3 +455,85 @@ def test_turnstile_wait_gives_up(tw, orc):
     torch.cuda.synchronize()
     assert st2.read_status() == 0
     assert torch.equal(Y2, Y)
+
+
+@pytest.mark.parametrize("activity", [0.01, 0.1])
+def test_sweep_scale_training(tw, orc, activity):
+    """A sweep point at full width: d_model=4096, d_ff=14336, M=8192 tokens with
+    lognormal row scaling, at 99% (K=8) and 90% (K=64) sparsity. The pack on every
+    row; the gate output and Y on a seeded sample of 256 rows plus every overflow
+    row; every gradient on its full tensor (lambda = 1e-3). Hundreds of rows
+    overflow, so the dense backup runs without split-K and the overflow rows'
+    weight gradients take the tensor-core path."""
+    w = sweep_workload(8192, activity)
+    inp = make_inputs(w)
+    D, Y, st, z = _run_fwd(tw, inp, w)
+    p = state_to_numpy(st)
+    assert p["n_ovf"] >= 64
+    plan = assert_plan_valid(st)
+    assert plan["dense_wgrad"]
+    rows = _sample_rows(w.M, 256, 5, extra=p["ovf_rows"][:p["n_ovf"]])
+    p, _, _ = _check_fwd(orc, inp, w, Y, st, z, rows=rows)
+    G = gpu_gmat(p, w.M, w.d_ff, w.T_n, w.K)
+    g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=1e-3)
+    torch.cuda.synchronize()
+    assert st.read_status() == 0
+    _check_bwd(orc, inp, g, G, 1e-3, w.name, per_row=True)
+
+
+def test_split_epilogue_barrier_gives_up(tw):
+    """Failure detection without a GPU fault: the split-K dense-backup GEMM of a
+    forward with 8 overflow rows runs with one epilogue warp that never reaches
+    the bounded barrier before the tile's partial sums are counted (the
+    library's test switch). The wait runs out after 2 s, the kernel sets
+    TWELL_STATUS_TIMEOUT and unwinds; the context stays usable, and the next
+    forward gives the clean result again."""
+    M, d, f, K, act, rs, seed = CASES["ovf_rows_8"]
+    w = Workload("ovf_rows_8", M, d, f, 128, K, act, row_scale=rs, seed=seed)
+    D = _dev(make_inputs(w))
+    Y0, st0 = tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], K=K)
+    torch.cuda.synchronize()
+    assert st0.read_status() == 0 and st0.n_overflow() == (8, 8)
+    try:
+        tw.test_withhold_epilogue_arrival(2)  # the forward's two dense-backup GEMMs; the second splits
+        Y1, st1 = tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], K=K)
+        torch.cuda.synchronize()
+    finally:
+        tw.test_withhold_epilogue_arrival(0)
+    assert st1.read_status(clear=True) & tw.STATUS_TIMEOUT
+    Y2, st2 = tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], K=K)
+    torch.cuda.synchronize()
+    assert st2.read_status() == 0
+    assert torch.equal(Y2, Y0)
+
+
+def test_backward_over_capacity(tw, orc):
+    """A forward that flagged more overflow rows than ovf_cap: the backward sets
+    TWELL_STATUS_OVERFLOW_CAP again, leaves the dX rows of the rows it could not
+    store untouched and their pairs out of the weight gradients; every other
+    gradient entry matches the oracle evaluated on the g the GPU stored (in which
+    those rows hold no active unit)."""
+    w = Workload("cap", 256, 256, 512, 128, 8, 0.15, row_scale="lognormal", training=True, seed=3)
+    inp = make_inputs(w)
+    n_flag = orc.pack(orc.gate(inp["X"], inp["W_g"], inp["b_g"]), 128, 8)["n_ovf_total"]
+    assert n_flag >= 4
+    cap = n_flag // 2
+    D = _dev(inp)
+    Y, st = tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], K=8, ovf_cap=cap)
+    torch.cuda.synchronize()
+    assert st.read_status(clear=True) == tw.STATUS_OVERFLOW_CAP
+    assert st.n_overflow() == (cap, n_flag)
+    M, d, f = w.M, w.d_model, w.d_ff
+    out = dict(dX=torch.full((M, d), 7.0, device="cuda"), dW_g=torch.empty((f, d), device="cuda"),
+               dW_u=torch.empty((f, d), device="cuda"), dW_d=torch.empty((d, f), device="cuda"),
+               db_g=torch.empty(f, device="cuda"))
+    g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=1e-3, out=out)
+    torch.cuda.synchronize()
+    assert st.read_status() == tw.STATUS_OVERFLOW_CAP
+    p = state_to_numpy(st)
+    unstored = np.setdiff1d(np.nonzero(p["row_ovf"])[0], p["ovf_rows"][:p["n_ovf"]])
+    assert unstored.size == n_flag - cap
+    assert bool((g["dX"][torch.from_numpy(unstored).cuda()] == 7.0).all())
+    G = gpu_gmat(p, M, f, 128, 8)
+    assert not G[unstored].any()
+    _check_bwd(orc, inp, g, G, 1e-3, "over capacity", per_row=True, skip_rows=unstored)
