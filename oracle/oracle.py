@@ -13,6 +13,10 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
   ffn_fwd_hybrid    pinned: equals ffn_fwd (round_g=1) on the same active set
   ffn_bwd           pinned: torch float64 autograd, closed form of the L1 term
   gmat input        pinned: with gmat = the oracle's own packed g, equals round_g
+  e4m3_value        pinned: torch's float8_e4m3fn reading of all 256 codes
+  e4m3_round        pinned: brute-force nearest code with the tie rule; torch's cast
+  quantize_e4m3     pinned: scale bounds, exact round trip, idempotence, a unit
+                    already on the grid, zero units, both layouts agree
 """
 
 from __future__ import annotations
@@ -61,6 +65,12 @@ def lib():
             L.oracle_bf16_round.argtypes = [ctypes.c_double]
             L.oracle_bf16_round_array.argtypes = [_f64p, _u16p, _i64]
             L.oracle_bf16_to_double_array.argtypes = [_u16p, _f64p, _i64]
+            L.oracle_e4m3_value.restype = ctypes.c_double
+            L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+            L.oracle_e4m3_round.restype = ctypes.c_uint8
+            L.oracle_e4m3_round.argtypes = [ctypes.c_double]
+            L.oracle_quantize_units.restype = None
+            L.oracle_quantize_units.argtypes = [_u16p, _i64, _i64, _i64, _i64, _u8p, _i32p, _u16p]
             L.oracle_set_threads.argtypes = [ctypes.c_int]
             L.oracle_get_threads.restype = ctypes.c_int
             L.oracle_gate.restype = ctypes.c_int
@@ -112,6 +122,34 @@ def bf16_to_f64(b) -> np.ndarray:
     out = np.empty(a.shape, np.float64)
     lib().oracle_bf16_to_double_array(a.reshape(-1), out.reshape(-1), a.size)
     return out
+
+
+def e4m3_value(code: int) -> float:
+    """Value of an FP8 E4M3 code (NaN for 0x7F / 0xFF)."""
+    return float(lib().oracle_e4m3_value(int(code) & 0xFF))
+
+
+def e4m3_round(x: float) -> int:
+    """Nearest E4M3 code of x, ties to even; |x| >= 448 saturates."""
+    return int(lib().oracle_e4m3_round(float(x)))
+
+
+def quantize_e4m3(W, unit_axis: int) -> dict:
+    """8-bit copy of a bf16 weight matrix, one power-of-two scale per hidden unit.
+
+    unit_axis = 0: units are rows (W_u [d_ff, d_model]); 1: units are columns
+    (W_d [d_model, d_ff]). Returns q [units, len] uint8 codes (unit-major), exp
+    [units] int32 (scale 2^exp) and deq: bf16 bits of the dequantised weights in
+    W's own layout."""
+    W = _c(W, np.uint16)
+    R, C = W.shape
+    units, length = (R, C) if unit_axis == 0 else (C, R)
+    su, sk = (C, 1) if unit_axis == 0 else (1, C)
+    q = np.empty((units, length), np.uint8)
+    e = np.empty(units, np.int32)
+    deq = np.empty_like(W)
+    lib().oracle_quantize_units(W, units, length, su, sk, q, e, deq)
+    return {"q": q, "exp": e, "deq": deq}
 
 
 def gate(X, W_g, b_g, rows=None) -> np.ndarray:

@@ -123,6 +123,81 @@ static double* to_double_transposed(const uint16_t* b, int64_t rows, int64_t col
   return d;
 }
 
+/* ------------------------------------------------------------- 8-bit weights */
+
+/* Combining the method with 8-bit quantisation is the pages' outlook
+ * ([aimodelsnavi] "Industry Impact", long-term impact). Reading taken here: the
+ * weights the sparse kernels gather (W_u and W_d) are stored per hidden unit j
+ * (row j of W_u, column j of W_d) as FP8 E4M3 codes with one power-of-two scale
+ * 2^e_j per unit and matrix. E4M3 (the OCP 8-bit floating-point format with a
+ * 4-bit exponent, bias 7, and a 3-bit mantissa; no infinities; code 0x7F/0xFF is
+ * NaN; largest finite value 448): code s eeee mmm is (-1)^s (8 + m) 2^(e - 10)
+ * for e >= 1 and (-1)^s m 2^-9 for e = 0.
+ *   e_j  = the smallest integer with max_k |w_jk| <= 448 * 2^e_j (0 for a zero unit)
+ *   q_jk = w_jk / 2^e_j rounded to the nearest E4M3 value, ties to even mantissa
+ *   w~_jk = value(q_jk) * 2^e_j, which has at most 4 significant bits and is
+ *          therefore a bf16 value exactly
+ * The FFN with 8-bit weights is the definition above evaluated on w~. */
+
+double oracle_e4m3_value(uint8_t code) {
+  const int s = code >> 7, e = (code >> 3) & 15, m = code & 7;
+  if (e == 15 && m == 7) return NAN;
+  const double v = e == 0 ? ldexp((double)m, -9) : ldexp((double)(8 + m), e - 10);
+  return s ? -v : v;
+}
+
+/* Nearest E4M3 code of x (ties to even); |x| > 448 saturates to +-448. Within a
+ * binade [2^k, 2^(k+1)), k >= -6, the E4M3 values are spaced 2^(k-3); below
+ * 2^-6 (the subnormals) they are spaced 2^-9. a / spacing is exact, nearbyint
+ * rounds it half to even (an even integer is an even mantissa), and a result
+ * of 2^(k+1) moves to the next binade with mantissa 0. */
+uint8_t oracle_e4m3_round(double x) {
+  if (isnan(x)) return 0x7F;
+  const uint8_t sign = signbit(x) ? 0x80 : 0;
+  const double a = fabs(x);
+  if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+  if (a == 0.0) return sign;
+  int E;
+  (void)frexp(a, &E); /* a in [2^(E-1), 2^E) */
+  const int k = E - 1;
+  const double spacing = k >= -6 ? ldexp(1.0, k - 3) : ldexp(1.0, -9);
+  const double r = nearbyint(a / spacing) * spacing;
+  if (r == 0.0) return sign;
+  if (r < ldexp(1.0, -6)) return (uint8_t)(sign | (int)ldexp(r, 9));
+  int E2;
+  (void)frexp(r, &E2);
+  const int k2 = E2 - 1;
+  const int m = (int)ldexp(r, 3 - k2) - 8;
+  return (uint8_t)(sign | ((k2 + 7) << 3) | m);
+}
+
+/* Quantises `units` units of `len` bf16 weights each; element k of unit j is
+ * W[j * su + k * sk]. Writes q[j * len + k] (unit-major codes), exps[j] = e_j and
+ * deq[j * su + k * sk] = bf16 bits of w~_jk (the input's layout). */
+void oracle_quantize_units(const uint16_t* W, int64_t units, int64_t len, int64_t su, int64_t sk, uint8_t* q,
+                           int32_t* exps, uint16_t* deq) {
+  for (int64_t j = 0; j < units; ++j) {
+    double amax = 0.0;
+    for (int64_t k = 0; k < len; ++k) {
+      const double v = fabs(oracle_bf16_to_double(W[j * su + k * sk]));
+      if (v > amax) amax = v;
+    }
+    int e = 0;
+    if (amax > 0.0) {
+      int E;
+      (void)frexp(amax, &E);
+      e = E - 12; /* 448 * 2^(E - 12) < 2^(E - 1) <= amax: start below the answer */
+      while (amax > ldexp(448.0, e)) ++e;
+    }
+    exps[j] = e;
+    for (int64_t k = 0; k < len; ++k) {
+      const uint8_t c = oracle_e4m3_round(ldexp(oracle_bf16_to_double(W[j * su + k * sk]), -e));
+      q[j * len + k] = c;
+      deq[j * su + k * sk] = oracle_bf16_round(ldexp(oracle_e4m3_value(c), e));
+    }
+  }
+}
+
 /* -------------------------------------------------------------------- gate */
 
 /* z_ij = sum_k x_ik W_g[j,k] (k ascending) + b_j for one row i.

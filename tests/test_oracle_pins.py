@@ -437,3 +437,95 @@ def test_count_stats_brute_force_and_sums(orc):
             flagged = (count.max(axis=1) > K) | ((count.astype(np.int64).sum(axis=1) >= dense_min) & (dense_min > 0))
             assert np.array_equal(p["row_ovf"].astype(bool), flagged)
             assert np.array_equal(p["ovf_rows"][:p["n_ovf"]], np.flatnonzero(flagged))
+
+
+# ------------------------------------------------------------- 8-bit weights
+
+
+def test_e4m3_values_match_torch(orc):
+    """All 256 E4M3 codes read as torch's float8_e4m3fn reads them (NaN codes aside)."""
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for c in range(256):
+        v = orc.e4m3_value(c)
+        if c & 0x7F == 0x7F:
+            assert math.isnan(v) and math.isnan(ref[c])
+        else:
+            assert v == ref[c] and math.copysign(1.0, v) == math.copysign(1.0, ref[c]), c
+    # the grid's landmarks
+    assert orc.e4m3_value(0x7E) == 448.0 and orc.e4m3_value(0x01) == 2.0 ** -9 and orc.e4m3_value(0x08) == 2.0 ** -6
+
+
+def _nearest_code(x, values):
+    """Brute force: the finite code nearest to x; on a tie the one with the even mantissa."""
+    best = None
+    for c, v in values:
+        dist = abs(v - x)
+        if best is None or dist < best[0] or (dist == best[0] and (c & 1) == 0 and (best[1] & 1) == 1):
+            best = (dist, c)
+    return best[1]
+
+
+def test_e4m3_round_brute_force_and_torch(orc):
+    """Nearest-even rounding to E4M3 against a brute-force search over the finite
+    codes (with both signs, ties, subnormals, the binade edges) and against torch's
+    float64 -> float8_e4m3fn cast."""
+    finite = [(c, orc.e4m3_value(c)) for c in range(256) if c & 0x7F != 0x7F]
+    pos = sorted({v for _, v in finite if v > 0})
+    xs = [0.0, 448.0, 2.0 ** -9, 2.0 ** -10, 3 * 2.0 ** -11, 2.0 ** -6, 1.0, 1.0625, 1.1875, 15.5, 240.0, 232.0,
+          447.0, 2.0 ** -7 * 0.99]
+    xs += [(a + b) / 2 for a, b in zip(pos, pos[1:])]  # every tie between neighbours
+    rng = np.random.default_rng(3)
+    xs += list(rng.uniform(0, 448, 400)) + list(np.exp(rng.uniform(np.log(2.0 ** -12), np.log(448), 400)))
+    for x in xs:
+        for sx in (x, -x):
+            got = orc.e4m3_round(sx)
+            want = _nearest_code(sx, [(c, v) for c, v in finite if (v > 0) == (sx > 0) or v == 0])
+            assert orc.e4m3_value(got) == orc.e4m3_value(want), (sx, got, want)
+    t = torch.tensor(xs + [-x for x in xs], dtype=torch.float64)
+    ref = t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([orc.e4m3_round(float(v)) for v in t], np.uint8)
+    assert np.array_equal(np.vectorize(orc.e4m3_value)(got), np.vectorize(orc.e4m3_value)(ref))
+    assert orc.e4m3_round(500.0) == 0x7E and orc.e4m3_round(-1e9) == 0xFE
+
+
+def test_quantize_units_scale_round_trip_idempotence(orc):
+    """Per unit: amax <= 448 * 2^e < 2 * amax (the smallest such e); the dequantised
+    weights are bf16 values equal to value(q) * 2^e; quantising them again gives the
+    same codes and exponents; the two layouts (units as rows / columns) agree."""
+    rng = np.random.default_rng(11)
+    W = _rand_bf16(rng, (37, 96), 1 / math.sqrt(96))
+    W[5] = 0  # a zero unit
+    W[6, :] = bf16_bits_from_f64(np.linspace(-3.0, 5.0, 96))  # a wider range
+    r = orc.quantize_e4m3(W, unit_axis=0)
+    q, e, deq = r["q"], r["exp"], r["deq"]
+    vals = np.vectorize(orc.e4m3_value)(q)
+    Wf = _f64(W)
+    for j in range(W.shape[0]):
+        amax = np.abs(Wf[j]).max()
+        if amax == 0:
+            assert e[j] == 0 and not q[j].any() and not deq[j].any()
+            continue
+        assert amax <= 448.0 * 2.0 ** e[j] and amax > 448.0 * 2.0 ** (e[j] - 1)
+        np.testing.assert_array_equal(_f64(deq[j]), vals[j] * 2.0 ** e[j])
+        # each code is the nearest grid point of the scaled weight
+        assert np.all(np.abs(vals[j] - Wf[j] / 2.0 ** e[j]) <= np.abs(
+            np.vectorize(orc.e4m3_value)((q[j] ^ 1) & 0xFF) - Wf[j] / 2.0 ** e[j]) + 1e-300)
+    again = orc.quantize_e4m3(deq, unit_axis=0)
+    assert np.array_equal(again["q"], q) and np.array_equal(again["exp"], e) and np.array_equal(again["deq"], deq)
+    cols = orc.quantize_e4m3(np.ascontiguousarray(W.T), unit_axis=1)
+    assert np.array_equal(cols["q"], q) and np.array_equal(cols["exp"], e)
+    assert np.array_equal(cols["deq"], np.ascontiguousarray(deq.T))
+
+
+def test_quantize_grid_unit_is_exact(orc):
+    """A unit whose weights already lie on the E4M3 grid times a power of two (with
+    the largest one at 448 * 2^e) comes back unchanged."""
+    e = -7
+    codes = np.array([0x7E, 0x01, 0x38, 0xBA, 0x08, 0x00, 0x55, 0xD0], np.uint8)
+    vals = np.array([orc.e4m3_value(c) for c in codes]) * 2.0 ** e
+    W = bf16_bits_from_f64(vals)[None, :]
+    r = orc.quantize_e4m3(W, unit_axis=0)
+    assert r["exp"][0] == e
+    assert np.array_equal(np.vectorize(orc.e4m3_value)(r["q"][0]) * 2.0 ** e, vals)
+    assert np.array_equal(r["deq"], W)
