@@ -92,6 +92,11 @@ def lib():
                                         _vp, ctypes.c_size_t, _vp]
             L.twell_ffn_fwd_tiles.restype = ctypes.c_int
             L.twell_ffn_fwd_tiles.argtypes = L.twell_ffn_fwd.argtypes
+            L.twell_quantize_e4m3_rows.restype = ctypes.c_int
+            L.twell_quantize_e4m3_rows.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp, _vp]
+            L.twell_ffn_fwd_e4m3.restype = ctypes.c_int
+            L.twell_ffn_fwd_e4m3.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp,
+                                             ctypes.POINTER(TwellHybrid), _vp, _vp, ctypes.c_size_t, _vp]
             L.twell_ffn_bwd.restype = ctypes.c_int
             L.twell_ffn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, ctypes.POINTER(TwellHybrid), _vp,
                                         ctypes.c_float, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
@@ -322,6 +327,53 @@ def ffn_fwd(X, W_g, b_g, W_u, W_d, T_n: int = 128, K: int = 8, ovf_cap: Optional
     _check(fn(_ptr(X), _ptr(W_g), _ptr(b_g), _ptr(W_u), _ptr(W_d), _ptr(W_dt), d, _ptr(Y), ctypes.byref(st.c),
               _ptr(z), _ptr(ws), ws.numel(), _stream(stream)),
            "twell_ffn_fwd_tiles" if tile_routing else "twell_ffn_fwd")
+    return (Y, st, z) if z_debug else (Y, st)
+
+
+def quantize_e4m3_rows(W, with_deq: bool = True, stream=None):
+    """twell_quantize_e4m3_rows: E4M3 codes [rows, len] (uint8), per-row scales
+    2^e [rows] (float32) and, with_deq, the dequantised bf16 rows."""
+    _bf16(W, "W")
+    rows, length = W.shape
+    q = torch.empty((rows, length), dtype=torch.uint8, device=W.device)
+    sc = torch.empty(rows, dtype=torch.float32, device=W.device)
+    deq = torch.empty_like(W) if with_deq else None
+    _check(lib().twell_quantize_e4m3_rows(_ptr(W), rows, length, _ptr(q), _ptr(sc), _ptr(deq), _stream(stream)),
+           "twell_quantize_e4m3_rows")
+    return q, sc, deq
+
+
+def quantize_weights(W_u, W_d, stream=None) -> dict:
+    """8-bit copies of the gathered weights for ffn_fwd_e4m3: W_u8 / s_u (rows of
+    W_u), W_dt8 / s_d (rows of W_d^T), and the dequantised bf16 W_u, W_d (the
+    weights the computed FFN uses)."""
+    W_u8, s_u, W_uq = quantize_e4m3_rows(W_u, stream=stream)
+    W_dt8, s_d, W_dtq = quantize_e4m3_rows(transpose_wd(W_d, stream=stream), stream=stream)
+    W_dq = torch.empty_like(W_d)
+    d, f = W_d.shape
+    # [d_ff][d_model] -> [d_model][d_ff]: the same transpose kernel with the roles of the extents swapped
+    _check(lib().twell_transpose_wd(_ptr(W_dtq), f, d, _ptr(W_dq), _stream(stream)), "twell_transpose_wd")
+    return dict(W_u8=W_u8, s_u=s_u, W_dt8=W_dt8, s_d=s_d, W_u=W_uq, W_d=W_dq)
+
+
+def ffn_fwd_e4m3(X, W_g, b_g, q8: dict, T_n: int = 128, K: int = 8, ovf_cap: Optional[int] = None,
+                 save_for_backward: bool = False, z_debug: bool = False, state: Optional[HybridState] = None,
+                 ws: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None, stream=None, dense_min: int = 0):
+    """twell_ffn_fwd_e4m3: the forward with the sparse kernel's gathers reading the
+    8-bit weights of q8 (from quantize_weights); the FFN computed is the one with
+    weights (W_g, q8["W_u"], q8["W_d"]). Returns (Y, state) or (Y, state, z)."""
+    for t, n in ((X, "X"), (W_g, "W_g"), (b_g, "b_g"), (q8["W_u"], "W_u"), (q8["W_d"], "W_d")):
+        _bf16(t, n)
+    M, d = X.shape
+    f = W_g.shape[0]
+    st = state or HybridState(M, f, T_n, K, ovf_cap, X.device, with_u=save_for_backward, dense_min=dense_min)
+    Y = torch.empty((M, d), dtype=torch.bfloat16, device=X.device) if Y is None else Y
+    z = torch.empty((M, f), dtype=torch.float32, device=X.device) if z_debug else None
+    if ws is None:
+        ws = workspace(OP_FWD, M, d, f, T_n, K, st.ovf_cap, X.device)
+    _check(lib().twell_ffn_fwd_e4m3(_ptr(X), _ptr(W_g), _ptr(b_g), _ptr(q8["W_u"]), _ptr(q8["W_d"]), _ptr(q8["W_u8"]),
+                                    _ptr(q8["s_u"]), _ptr(q8["W_dt8"]), _ptr(q8["s_d"]), d, _ptr(Y), ctypes.byref(st.c),
+                                    _ptr(z), _ptr(ws), ws.numel(), _stream(stream)), "twell_ffn_fwd_e4m3")
     return (Y, st, z) if z_debug else (Y, st)
 
 

@@ -271,11 +271,21 @@ twell_status twell_pack(const uint16_t* X, const uint16_t* W_g, const uint16_t* 
 namespace twell {
 namespace {
 
+// 8-bit copies of the gathered weights (twell_ffn_fwd_e4m3).
+struct Q8Weights {
+  const uint8_t* W_u8;
+  const float* s_u;
+  const uint8_t* W_dt8;
+  const float* s_d;
+};
+
 // The forward shared by twell_ffn_fwd (row-level routing with the dense
-// backup) and twell_ffn_fwd_tiles (tile-level routing, inference only).
+// backup), twell_ffn_fwd_tiles (tile-level routing, inference only) and
+// twell_ffn_fwd_e4m3 (row-level routing, 8-bit gathers when q8 is given).
 twell_status ffn_fwd_impl(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_g, const uint16_t* W_u,
                           const uint16_t* W_d, const uint16_t* W_dt, int64_t d_model, uint16_t* Y, twell_hybrid* h,
-                          float* z_debug, void* ws, size_t ws_bytes, bool tiles, twell_stream_t stream) {
+                          float* z_debug, void* ws, size_t ws_bytes, bool tiles, twell_stream_t stream,
+                          const Q8Weights* q8 = nullptr) {
   twell_status st = check_hybrid(h, d_model);
   if (st != TWELL_OK || h->M == 0) return st;
   const void* in[] = {X, W_g, b_g, W_u, W_d, Y};
@@ -289,7 +299,7 @@ twell_status ffn_fwd_impl(const uint16_t* X, const uint16_t* W_g, const uint16_t
   const int M = h->M, d = static_cast<int>(d_model), f = h->d_ff, K = h->K, cap = h->ovf_cap;
   const WsLayout L = ws_layout(TWELL_OP_FWD, M, d, f, K, cap);
   const uint16_t* wdt = W_dt;
-  if (!wdt) {
+  if (!wdt && !q8) {
     uint16_t* t = at<uint16_t>(ws, L.w_dt);
     if (launch_transpose_bf16(W_d, d, f, t, s) != cudaSuccess) return TWELL_ECUDA;
     wdt = t;
@@ -297,10 +307,13 @@ twell_status ffn_fwd_impl(const uint16_t* X, const uint16_t* W_g, const uint16_t
   uint16_t* x_ovf = at<uint16_t>(ws, L.x_ovf);
   st = run_pack(X, W_g, b_g, d, h, z_debug, ws, L, X, x_ovf, tiles, s);
   if (st != TWELL_OK) return st;
-  if (launch_ell_ffn_fwd(X, W_u, wdt, h->count, h->val, h->col, tiles ? at<uint16_t>(ws, L.spill) : nullptr,
-                         h->row_plan, tiles ? nullptr : h->u_ell, Y, M, d, f, K, at<int>(ws, L.ctr),
-                         at<float>(ws, L.yacc), h->status, s) != cudaSuccess)
-    return TWELL_ECUDA;
+  const cudaError_t ce =
+      q8 ? launch_ell_ffn_fwd_q8(X, q8->W_u8, q8->s_u, q8->W_dt8, q8->s_d, h->count, h->val, h->col, h->row_plan,
+                                 h->u_ell, Y, M, d, f, K, at<int>(ws, L.ctr), at<float>(ws, L.yacc), h->status, s)
+         : launch_ell_ffn_fwd(X, W_u, wdt, h->count, h->val, h->col, tiles ? at<uint16_t>(ws, L.spill) : nullptr,
+                              h->row_plan, tiles ? nullptr : h->u_ell, Y, M, d, f, K, at<int>(ws, L.ctr),
+                              at<float>(ws, L.yacc), h->status, s);
+  if (ce != cudaSuccess) return TWELL_ECUDA;
   if (tiles) return TWELL_OK;
   const SplitKBuffers sk{at<float>(ws, L.sk_partial), at<unsigned long long>(ws, L.sk_arrivals)};
   return cuda_status(launch_ovf_fwd(x_ovf, W_u, W_d, h->g_ovf, h->ovf_rows, h->n_ovf, cap, M, d, f,
@@ -322,6 +335,28 @@ twell_status twell_ffn_fwd_tiles(const uint16_t* X, const uint16_t* W_g, const u
                                  const uint16_t* W_d, const uint16_t* W_dt, int64_t d_model, uint16_t* Y,
                                  twell_hybrid* h, float* z_debug, void* ws, size_t ws_bytes, twell_stream_t stream) {
   return ffn_fwd_impl(X, W_g, b_g, W_u, W_d, W_dt, d_model, Y, h, z_debug, ws, ws_bytes, true, stream);
+}
+
+twell_status twell_quantize_e4m3_rows(const uint16_t* W, int64_t rows, int64_t len, uint8_t* q, float* scale,
+                                      uint16_t* deq, twell_stream_t stream) {
+  if (rows < 0 || len <= 0 || len % 16 != 0) return TWELL_EINVAL;
+  if (len > kMaxDModel || rows > (int64_t(1) << 24)) return TWELL_EUNSUPPORTED;
+  if (rows == 0) return TWELL_OK;
+  if (!W || !q || !scale || !aligned16(W) || !aligned16(q) || (deq && !aligned16(deq))) return TWELL_EINVAL;
+  return cuda_status(launch_quantize_rows(W, static_cast<int>(rows), static_cast<int>(len), q, scale, deq,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+twell_status twell_ffn_fwd_e4m3(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_g, const uint16_t* W_u,
+                                const uint16_t* W_d, const uint8_t* W_u8, const float* s_u, const uint8_t* W_dt8,
+                                const float* s_d, int64_t d_model, uint16_t* Y, twell_hybrid* h, float* z_debug,
+                                void* ws, size_t ws_bytes, twell_stream_t stream) {
+  const void* q[] = {W_u8, s_u, W_dt8, s_d};
+  if (h && h->M > 0)
+    for (const void* p : q)
+      if (!p || !aligned16(p)) return TWELL_EINVAL;
+  const Q8Weights q8{W_u8, s_u, W_dt8, s_d};
+  return ffn_fwd_impl(X, W_g, b_g, W_u, W_d, nullptr, d_model, Y, h, z_debug, ws, ws_bytes, false, stream, &q8);
 }
 
 twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_t* W_u, const uint16_t* W_d,

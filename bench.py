@@ -270,6 +270,9 @@ def kernel_work(name, M, d, f, T, K, kept, pairs, n_ovf=0, dense_wgrad=0):
                        + 4 * kept                 # u written
                        + 2 * m_ell * d            # Y written
                        + 2 * 2 * f * d)           # W_u, W_dt read once
+    if name == "ell_updown_q8":
+        # as ell_updown, with the two gathered weights read as 1-byte codes (plus a scale per unit)
+        return "hbm", (2 * m_ell * d + m_ell * T * (2 + 3 * K) + 4 * kept + 2 * m_ell * d + 2 * f * d + 2 * 4 * f)
     if name == "ell_bwd":
         # dY, TwELL, u read; (h, dU, dZ) per slot written; dX (fp32) written; W_u, W_g, W_dt once
         return "hbm", (2 * m_ell * d + m_ell * T * (2 + 3 * K) + 4 * kept + 16 * kept + 4 * m_ell * d
@@ -638,7 +641,20 @@ def run_twell(args, world, rank, local):
                 st_inf = tw.HybridState(M, f, w.T_n, K, cap, dev, with_u=False)
                 res["ms_infer"] = warm_and_time(infer(st_inf))
                 assert st_inf.read_status() == 0, "device status word set during the inference timing"
-                del st_inf
+                Y_ref = Y.clone()
+                # the same inference forward with the gathers reading 8-bit (E4M3) weights, quantised
+                # once outside the timed region; the FFN it computes uses the dequantised weights
+                q8 = tw.quantize_weights(W_u, W_d)
+                Yq = torch.empty_like(Y)
+
+                def infer_q8(e_mid):
+                    tw.ffn_fwd_e4m3(X, W_g, b_g, q8, T_n=w.T_n, K=K, state=st_inf, ws=wsf, Y=Yq)
+                    e_mid.record(stream)
+
+                res["ms_infer_e4m3"] = warm_and_time(infer_q8)
+                assert st_inf.read_status() == 0, "device status word set during the 8-bit inference timing"
+                res["e4m3_rel_l2"] = float((Yq.float() - Y_ref.float()).norm() / Y_ref.float().norm())
+                del st_inf, q8, Yq, Y_ref
             res["e2e"] = e2e(M, d, X, dY, Y, lambda Xi, dYi, Yi: (
                 tw.transpose_wd(W_d, out=Wdt),
                 tw.ffn_fwd(Xi, W_g, b_g, W_u, W_d, T_n=w.T_n, K=K, W_dt=Wdt, state=st, ws=wsf, Y=Yi),
@@ -795,6 +811,11 @@ def bench_line(args, world, main, others):
                 "note": "forward half of the training step (W_d transposed, u saved)"},
         "fwd_inference": {"tokens_per_s": tokens / (main["ms_infer"] / 1e3), "ms": main["ms_infer"],
                           "note": "forward alone with fixed weights (W_dt prepared once, u not saved)"},
+        "fwd_inference_e4m3": {"tokens_per_s": tokens / (main["ms_infer_e4m3"] / 1e3), "ms": main["ms_infer_e4m3"],
+                               "rel_l2_vs_bf16_weights": main["e4m3_rel_l2"],
+                               "note": "the inference forward with the sparse kernel gathering E4M3 weights (per-unit "
+                                       "power-of-two scales, quantised once); the FFN computed is the one with the "
+                                       "dequantised weights; rel_l2 is its Y against the bf16-weight Y"},
         "dense_bf16": dense,
         "speedup_vs_dense": ({"fwd": dense["fwd_best"]["ms"] / ms_fwd,
                               "fwd_inference": dense["fwd_best"]["ms"] / main["ms_infer"],

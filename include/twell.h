@@ -244,6 +244,45 @@ TWELL_API twell_status twell_ffn_fwd_tiles(const uint16_t* X, const uint16_t* W_
                                  size_t ws_bytes, twell_stream_t stream);
 
 /*
+ * 8-bit weights for the gathers ([aimodelsnavi] "Industry Impact" names the
+ * combination of the method with 8-bit quantisation as its long-term outlook).
+ * twell_quantize_e4m3_rows stores each row r of a bf16 matrix W [rows][len] as
+ * FP8 E4M3 codes (the OCP 8-bit format with a 4-bit exponent, bias 7, 3-bit
+ * mantissa, largest finite value 448) with one power-of-two scale per row:
+ *   scale[r] = 2^e_r, e_r the smallest integer with max_k |W[r][k]| <= 448 * 2^e_r
+ *              (2^0 for an all-zero row)
+ *   q[r][k]  = W[r][k] / 2^e_r rounded to the nearest E4M3 value, ties to even
+ *   deq[r][k] (nullable) = bf16 bits of q[r][k] * 2^e_r, which is exact (the
+ *              dequantised value has at most 4 significant bits)
+ * len must be a multiple of 16 in [16, 16384], rows in [0, 2^24]; W, q and deq
+ * 16-byte aligned, scale 4-byte aligned; all caller-owned device memory,
+ * asynchronous on `stream`. For the forward below: quantise W_u (rows = d_ff,
+ * len = d_model) and W_d^T (from twell_transpose_wd; rows = d_ff).
+ */
+TWELL_API twell_status twell_quantize_e4m3_rows(const uint16_t* W, int64_t rows, int64_t len, uint8_t* q,
+                                                float* scale, uint16_t* deq, twell_stream_t stream);
+
+/*
+ * twell_ffn_fwd with the fused sparse up+down kernel reading 8-bit weights: per
+ * active unit j it gathers row j of W_u8 (d_model codes, scale s_u[j]) and row j
+ * of W_dt8 (the codes of column j of W_d, scale s_d[j]) instead of 2 * d_model
+ * bf16 values, half the bytes. W_u and W_d are the dequantised bf16 weights
+ * (deq of the quantisation above, W_d in its [d_model][d_ff] layout): the gate
+ * GEMM takes W_g as it is and the dense backup GEMMs take W_u and W_d. Y is the
+ * FFN of X with weights (W_g, W_u, W_d), the function twell_ffn_fwd computes on
+ * the same arguments, up to fp32 rounding order. Inside the kernel the token
+ * row enters the dot products as f16 (exact for magnitudes in [2^-14, 65504];
+ * smaller values are rounded to f16's subnormal grid, larger ones saturate).
+ * Row-level routing only; arguments, descriptor, workspace (TWELL_OP_FWD) and
+ * errors as twell_ffn_fwd; u_ell / u_ovf are written when non-NULL.
+ */
+TWELL_API twell_status twell_ffn_fwd_e4m3(const uint16_t* X, const uint16_t* W_g, const uint16_t* b_g,
+                                          const uint16_t* W_u, const uint16_t* W_d, const uint8_t* W_u8,
+                                          const float* s_u, const uint8_t* W_dt8, const float* s_d, int64_t d_model,
+                                          uint16_t* Y, twell_hybrid* h, float* z_debug, void* ws, size_t ws_bytes,
+                                          twell_stream_t stream);
+
+/*
  * Backward pass over the hybrid format of a previous twell_ffn_fwd (which must
  * have been given non-NULL u_ell and u_ovf), for L = sum(Y * dY) + lambda * sum(g):
  *   dH_ij = dY_i . W_d[:, j] at active units;  dU = dH g;  dZ = (dH u + lambda) [z > 0]
