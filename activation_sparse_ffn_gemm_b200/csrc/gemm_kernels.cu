@@ -13,12 +13,19 @@
 //                 forward  H = bf16(g * (X_ovf W_u^T)),  Y[rows] = bf16(H W_d^T)
 //                 backward [dU | dZ] from dH = dY_ovf W_d,  dX[rows] = dU W_u + dZ W_g
 #include "umma_gemm.cuh"
+#include "umma_gemm_pair.cuh"
+
+// The gate GEMM runs on CTA pairs (umma_gemm_pair.cuh); 0 selects the one-CTA engine.
+#ifndef TWELL_PAIR_GEMM
+#define TWELL_PAIR_GEMM 1
+#endif
 
 namespace twell {
 
 namespace {
 
 constexpr int kStages = 4;
+constexpr int kPairStages = 6;  // 32 KB per stage on a CTA pair (A 128 x 64 and half of B)
 
 __device__ __forceinline__ void load_bias32(const uint16_t* b, float (&out)[32]) {
   const uint4* p = reinterpret_cast<const uint4*>(b);
@@ -334,12 +341,17 @@ cudaError_t launch_gate_pack(const uint16_t* X, const uint16_t* W_g, const uint1
                              int K, const PackOut& out, uint32_t* status, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   CUtensorMap ta, tb;
+  constexpr int b_rows = TWELL_PAIR_GEMM ? 128 : 256;  // B rows one CTA loads per K block
   if (!make_tmap_bf16(&ta, X, d, M, static_cast<uint64_t>(d) * 2, kBK, kBM) ||
-      !make_tmap_bf16(&tb, W_g, d, f, static_cast<uint64_t>(d) * 2, kBK, 256))
+      !make_tmap_bf16(&tb, W_g, d, f, static_cast<uint64_t>(d) * 2, kBK, b_rows))
     return cudaErrorInvalidValue;
   GemmShape shp{M, nullptr, f, d, 0, status};
   EpiTwell::Args ea{b_g, out.count, out.val, out.col, out.spill, out.z_debug, f / kTn, K, f};
+#if TWELL_PAIR_GEMM
+  return launch_umma_pair<EpiTwell, false, kPairStages>("gate_pack_gemm", ta, tb, ta, tb, shp, ea, s);
+#else
   return launch_umma_gemm<EpiTwell, 256, false, kStages>("gate_pack_gemm", ta, tb, ta, tb, shp, ea, s);
+#endif
 }
 
 namespace {
@@ -352,6 +364,31 @@ void use_split(GemmShape& shp, const SplitKBuffers& sk, int cap) {
 }
 }  // namespace
 
+// A dense-backup GEMM over a device-side row count of at most `cap` rows: the
+// one-CTA engine (split-K when few rows overflow) takes up to kSplitRows rows,
+// the CTA-pair engine takes more. When cap allows both, both are launched and
+// the one that does not own the count returns at once (no host synchronisation
+// learns the count). b_pair is B's tensor map with 128-row boxes for the pair
+// engine (the same map as b when B is MN-major).
+template <class Epi, bool B_MN, bool A_MN = false>
+cudaError_t launch_rows_gemm(const char* name, const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
+                             const CUtensorMap& b1, const CUtensorMap& b0_pair, const CUtensorMap& b1_pair,
+                             GemmShape shp, const typename Epi::Args& ea, int cap, cudaStream_t s) {
+#if TWELL_PAIR_GEMM
+  const bool pair = cap > kSplitRows;
+#else
+  const bool pair = false;
+#endif
+  GemmShape one = shp;
+  if (pair) one.max_rows = kSplitRows;
+  cudaError_t e = launch_umma_gemm<Epi, 256, B_MN, kStages, A_MN>(name, a0, b0, a1, b1, one, ea, s);
+  if (e != cudaSuccess || !pair) return e;
+  GemmShape two = shp;
+  two.partial = nullptr;
+  two.min_rows = kSplitRows;
+  return launch_umma_pair<Epi, B_MN, kPairStages, A_MN>(name, a0, b0_pair, a1, b1_pair, two, ea, s);
+}
+
 size_t splitk_partial_floats(int cap, int d, int f) {
   const size_t rows = static_cast<size_t>(cap < kSplitRows ? cap : kSplitRows);
   return static_cast<size_t>(kSplitMax) * rows * static_cast<size_t>(d > f ? d : f);
@@ -363,21 +400,23 @@ cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uin
                            uint16_t* h_ovf, float* u_ovf, uint16_t* Y, const SplitKBuffers& sk, uint32_t* status,
                            cudaStream_t s) {
   if (cap <= 0) return cudaSuccess;
-  CUtensorMap ta, tb, ta2, tb2;
+  CUtensorMap ta, tb, ta2, tb2, tbp, tb2p;
   if (!make_tmap_bf16(&ta, x_ovf, d, cap, static_cast<uint64_t>(d) * 2, kBK, kBM) ||
       !make_tmap_bf16(&tb, W_u, d, f, static_cast<uint64_t>(d) * 2, kBK, 256) ||
+      !make_tmap_bf16(&tbp, W_u, d, f, static_cast<uint64_t>(d) * 2, kBK, 128) ||
       !make_tmap_bf16(&ta2, h_ovf, f, cap, static_cast<uint64_t>(f) * 2, kBK, kBM) ||
-      !make_tmap_bf16(&tb2, W_d, f, d, static_cast<uint64_t>(f) * 2, kBK, 256))
+      !make_tmap_bf16(&tb2, W_d, f, d, static_cast<uint64_t>(f) * 2, kBK, 256) ||
+      !make_tmap_bf16(&tb2p, W_d, f, d, static_cast<uint64_t>(f) * 2, kBK, 128))
     return cudaErrorInvalidValue;
   GemmShape s1{cap, n_ovf, f, d, 0, status};
   use_split(s1, sk, cap);
   EpiGateMul::Args e1{g_ovf, h_ovf, u_ovf, f};
-  cudaError_t e = launch_umma_gemm<EpiGateMul, 256, false, kStages>("ovf_up_gemm", ta, tb, ta, tb, s1, e1, s);
+  cudaError_t e = launch_rows_gemm<EpiGateMul, false>("ovf_up_gemm", ta, tb, ta, tb, tbp, tbp, s1, e1, cap, s);
   if (e != cudaSuccess) return e;
   GemmShape s2{cap, n_ovf, d, f, 0, status};
   use_split(s2, sk, cap);
   EpiScatterBf16::Args e2{ovf_rows, Y, d, M, status};
-  return launch_umma_gemm<EpiScatterBf16, 256, false, kStages>("ovf_down_gemm", ta2, tb2, ta2, tb2, s2, e2, s);
+  return launch_rows_gemm<EpiScatterBf16, false>("ovf_down_gemm", ta2, tb2, ta2, tb2, tb2p, tb2p, s2, e2, cap, s);
 }
 
 cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const uint16_t* W_u,
@@ -386,10 +425,11 @@ cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const u
                            float* du_ovf, float* dz_ovf, float* dX, const SplitKBuffers& sk, uint32_t* status,
                            cudaStream_t s) {
   if (cap <= 0) return cudaSuccess;
-  CUtensorMap ta, tb, tdu, tdz, twu, twg;
+  CUtensorMap ta, tb, tbp, tdu, tdz, twu, twg;
   // dH = dY_ovf W_d: B = W_dt [f][d] (K-major)
   if (!make_tmap_bf16(&ta, dy_ovf, d, cap, static_cast<uint64_t>(d) * 2, kBK, kBM) ||
       !make_tmap_bf16(&tb, W_dt, d, f, static_cast<uint64_t>(d) * 2, kBK, 256) ||
+      !make_tmap_bf16(&tbp, W_dt, d, f, static_cast<uint64_t>(d) * 2, kBK, 128) ||
       // dX = dU W_u + dZ W_g: A segments are the two halves of duz, B = W_u / W_g as [K=f][N=d] (MN-major)
       !make_tmap_bf16(&tdu, duz_ovf, f, cap, static_cast<uint64_t>(f) * 4, kBK, kBM) ||
       !make_tmap_bf16(&tdz, duz_ovf + f, f, cap, static_cast<uint64_t>(f) * 4, kBK, kBM) ||
@@ -399,12 +439,12 @@ cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const u
   GemmShape s1{cap, n_ovf, f, d, 0, status};
   use_split(s1, sk, cap);
   EpiBwdDH::Args e1{g_ovf, u_ovf, duz_ovf, du_ovf, dz_ovf, lambda, f};
-  cudaError_t e = launch_umma_gemm<EpiBwdDH, 256, false, kStages>("ovf_dh_gemm", ta, tb, ta, tb, s1, e1, s);
+  cudaError_t e = launch_rows_gemm<EpiBwdDH, false>("ovf_dh_gemm", ta, tb, ta, tb, tbp, tbp, s1, e1, cap, s);
   if (e != cudaSuccess) return e;
   GemmShape s2{cap, n_ovf, d, f, f, status};
   use_split(s2, sk, cap);
   EpiScatterF32::Args e2{ovf_rows, dX, d, M, status};
-  return launch_umma_gemm<EpiScatterF32, 256, true, kStages>("ovf_dx_gemm", tdu, twu, tdz, twg, s2, e2, s);
+  return launch_rows_gemm<EpiScatterF32, true>("ovf_dx_gemm", tdu, twu, tdz, twg, twu, twg, s2, e2, cap, s);
 }
 
 cudaError_t launch_dense_wgrad(const DenseWgradOperands& op, const int* k_rows, int cap, int d, int f, float* dW_g,
@@ -422,13 +462,21 @@ cudaError_t launch_dense_wgrad(const DenseWgradOperands& op, const int* k_rows, 
   GemmShape s1{2 * f, nullptr, d, static_cast<int>(rows), 0, status};
   s1.K_dev = k_rows;
   EpiStoreF32::Args e1{dW_u, dW_g, f, d};
+#if TWELL_PAIR_GEMM
+  cudaError_t e = launch_umma_pair<EpiStoreF32, true, kPairStages, true>("dense_wgrad_ug", ta, tb, ta, tb, s1, e1, s);
+#else
   cudaError_t e = launch_umma_gemm<EpiStoreF32, 256, true, kStages, true>("dense_wgrad_ug", ta, tb, ta, tb, s1, e1, s);
+#endif
   if (e != cudaSuccess) return e;
   // dW_d (d_model x d_ff) = dY_ovf^T H_ovf
   GemmShape s2{d, nullptr, f, static_cast<int>(rows), 0, status};
   s2.K_dev = k_rows;
   EpiStoreF32::Args e2{dW_d, dW_d, d, f};
+#if TWELL_PAIR_GEMM
+  return launch_umma_pair<EpiStoreF32, true, kPairStages, true>("dense_wgrad_d", ta2, tb2, ta2, tb2, s2, e2, s);
+#else
   return launch_umma_gemm<EpiStoreF32, 256, true, kStages, true>("dense_wgrad_d", ta2, tb2, ta2, tb2, s2, e2, s);
+#endif
 }
 
 }  // namespace twell

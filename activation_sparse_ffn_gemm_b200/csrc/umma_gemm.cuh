@@ -56,6 +56,8 @@ struct GemmShape {
   unsigned long long* arrivals = nullptr;  // [kSplitTiles] per-output-tile arrival words
   unsigned long long epoch = 0;            // this launch's tag (1 .. 2^56 - 1)
   int withhold_epi_arrival = 0;  // test of the bounded epilogue barrier: one epilogue warp never arrives
+  int max_rows = 0;  // one-CTA engine: nothing to do when more rows than this are processed (0: no bound)
+  int min_rows = 0;  // CTA-pair engine: nothing to do unless more rows than this are processed
 };
 
 constexpr int kSplitMax = 8;
@@ -171,6 +173,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int nk = nk0 + shp.K1 / kBK;
   if (nk == 0) return;  // nothing to contract (a device-side K of zero)
   const int split = gemm_split(*m_eff_s, shp.N, BN, nk, shp, gridDim.x);
+  if (shp.max_rows > 0 && *m_eff_s > shp.max_rows) return;  // the pair engine owns this row count
   if (static_cast<long>(blockIdx.x) >=
       static_cast<long>((*m_eff_s + kBM - 1) / kBM) * ((shp.N + BN - 1) / BN) * split)
     return;
