@@ -263,20 +263,40 @@ struct EpiScatterF32 {
 };
 
 // -------------------------------------- dense backup backward, dH epilogue
-// dH (accumulator) -> dU = dH g, dZ = (dH u + lambda) [g > 0], as fp32 (weight
-// gradients) and bf16 [dU | dZ] (the dX GEMM's operand).
+// dH (accumulator) -> dU = dH g, dZ = (dH u + lambda) [g > 0] for dense row s:
+//   duz_hi[s]  = bf16 [dU | dZ]          (the dX GEMM's A operand; also the "hi"
+//                                         part of the weight-gradient operand)
+// and, for the weight gradients of the dense rows,
+//   when they run as GEMMs (plan[3] != 0): the "lo" parts duz_lo[s] =
+//     bf16([dU | dZ] - hi) and the hi / lo parts of H = g u, h_hi[s], h_lo[s]
+//     (hi + lo carries each value to about 2^-16 of it);
+//   otherwise the fp32 dU and dZ rows that the pair list takes.
 struct EpiBwdDH {
   struct Args {
     const uint16_t* g;  // [cap][f]
     const float* u;     // [cap][f]
-    uint16_t* duz;      // [cap][2f] bf16: dU in [0, f), dZ in [f, 2f) (tensor-core operand of dX)
-    float* du;          // [cap][f] fp32 dU (weight gradients)
-    float* dz;          // [cap][f] fp32 dZ (weight gradients)
+    const int* plan;    // plan[3]: dense weight gradients of the overflow rows
+    uint16_t* duz_hi;   // [cap_r][2f]
+    uint16_t* duz_lo;   // [cap_r][2f]
+    uint16_t* h_hi;     // [cap_r][f]
+    uint16_t* h_lo;     // [cap_r][f]
+    float* du;          // [cap][f]
+    float* dz;          // [cap][f]
     float lambda;
     int f;
   };
   static constexpr int SMEM_BYTES = 0;
   static constexpr bool kSplitK = true;
+  __device__ static void hi_lo(const float (&v)[8], uint4& hi, uint4& lo) {
+    float h[8], l[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      h[e] = __bfloat162float(__float2bfloat16_rn(v[e]));
+      l[e] = v[e] - h[e];  // exact in fp32
+    }
+    hi = make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]), pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
+    lo = make_uint4(pack_bf16x2(l[0], l[1]), pack_bf16x2(l[2], l[3]), pack_bf16x2(l[4], l[5]), pack_bf16x2(l[6], l[7]));
+  }
   __device__ static void apply8(const Args& a, int row, int n, const float (&dh)[8]) {
     const size_t off = static_cast<size_t>(row) * a.f + n;
     float g8[8];
@@ -290,18 +310,30 @@ struct EpiBwdDH {
       du[e] = dh[e] * g8[e];
       dz[e] = g8[e] > 0.f ? fmaf(dh[e], u8[e], a.lambda) : 0.f;
     }
-
-    uint16_t* drow = a.duz + static_cast<size_t>(row) * 2 * a.f;
-    *reinterpret_cast<uint4*>(drow + n) = make_uint4(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]),
-                                                     pack_bf16x2(du[4], du[5]), pack_bf16x2(du[6], du[7]));
-    *reinterpret_cast<uint4*>(drow + a.f + n) = make_uint4(pack_bf16x2(dz[0], dz[1]), pack_bf16x2(dz[2], dz[3]),
-                                                           pack_bf16x2(dz[4], dz[5]), pack_bf16x2(dz[6], dz[7]));
-    float4* du32 = reinterpret_cast<float4*>(a.du + off);
-    float4* dz32 = reinterpret_cast<float4*>(a.dz + off);
-    du32[0] = make_float4(du[0], du[1], du[2], du[3]);
-    du32[1] = make_float4(du[4], du[5], du[6], du[7]);
-    dz32[0] = make_float4(dz[0], dz[1], dz[2], dz[3]);
-    dz32[1] = make_float4(dz[4], dz[5], dz[6], dz[7]);
+    const size_t orow = static_cast<size_t>(row) * 2 * a.f;
+    uint4 uh, ul, zh, zl;
+    hi_lo(du, uh, ul);
+    hi_lo(dz, zh, zl);
+    *reinterpret_cast<uint4*>(a.duz_hi + orow + n) = uh;
+    *reinterpret_cast<uint4*>(a.duz_hi + orow + a.f + n) = zh;
+    if (a.plan[3] != 0) {
+      *reinterpret_cast<uint4*>(a.duz_lo + orow + n) = ul;
+      *reinterpret_cast<uint4*>(a.duz_lo + orow + a.f + n) = zl;
+      float h[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) h[e] = g8[e] * u8[e];  // h = g u in fp32, as on the sparse path
+      uint4 hh, hl;
+      hi_lo(h, hh, hl);
+      *reinterpret_cast<uint4*>(a.h_hi + off) = hh;
+      *reinterpret_cast<uint4*>(a.h_lo + off) = hl;
+    } else {
+      float4* du32 = reinterpret_cast<float4*>(a.du + off);
+      float4* dz32 = reinterpret_cast<float4*>(a.dz + off);
+      du32[0] = make_float4(du[0], du[1], du[2], du[3]);
+      du32[1] = make_float4(du[4], du[5], du[6], du[7]);
+      dz32[0] = make_float4(dz[0], dz[1], dz[2], dz[3]);
+      dz32[1] = make_float4(dz[4], dz[5], dz[6], dz[7]);
+    }
   }
   __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
     run_apply8<EpiBwdDH>(a, m0, n0, M_eff, N, r, taddr);
@@ -421,24 +453,26 @@ cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uin
 
 cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const uint16_t* W_u,
                            const uint16_t* W_g, const uint16_t* g_ovf, const float* u_ovf, float lambda,
-                           const int* ovf_rows, const int* n_ovf, int cap, int M, int d, int f, uint16_t* duz_ovf,
-                           float* du_ovf, float* dz_ovf, float* dX, const SplitKBuffers& sk, uint32_t* status,
-                           cudaStream_t s) {
+                           const int* ovf_rows, const int* n_ovf, const int* plan, int cap, int M, int d, int f,
+                           const DenseWgradOperands& op, float* du_ovf, float* dz_ovf, float* dX,
+                           const SplitKBuffers& sk, uint32_t* status, cudaStream_t s) {
   if (cap <= 0) return cudaSuccess;
+  const int cap_r = dense_rows_padded(cap);
   CUtensorMap ta, tb, tbp, tdu, tdz, twu, twg;
   // dH = dY_ovf W_d: B = W_dt [f][d] (K-major)
   if (!make_tmap_bf16(&ta, dy_ovf, d, cap, static_cast<uint64_t>(d) * 2, kBK, kBM) ||
       !make_tmap_bf16(&tb, W_dt, d, f, static_cast<uint64_t>(d) * 2, kBK, 256) ||
       !make_tmap_bf16(&tbp, W_dt, d, f, static_cast<uint64_t>(d) * 2, kBK, 128) ||
-      // dX = dU W_u + dZ W_g: A segments are the two halves of duz, B = W_u / W_g as [K=f][N=d] (MN-major)
-      !make_tmap_bf16(&tdu, duz_ovf, f, cap, static_cast<uint64_t>(f) * 4, kBK, kBM) ||
-      !make_tmap_bf16(&tdz, duz_ovf + f, f, cap, static_cast<uint64_t>(f) * 4, kBK, kBM) ||
+      // dX = dU W_u + dZ W_g: A segments are the two halves of duz_hi, B = W_u / W_g as [K=f][N=d] (MN-major)
+      !make_tmap_bf16(&tdu, op.duz_hi, f, cap, static_cast<uint64_t>(f) * 4, kBK, kBM) ||
+      !make_tmap_bf16(&tdz, op.duz_hi + f, f, cap, static_cast<uint64_t>(f) * 4, kBK, kBM) ||
       !make_tmap_bf16(&twu, W_u, d, f, static_cast<uint64_t>(d) * 2, 64, kBK) ||
       !make_tmap_bf16(&twg, W_g, d, f, static_cast<uint64_t>(d) * 2, 64, kBK))
     return cudaErrorInvalidValue;
   GemmShape s1{cap, n_ovf, f, d, 0, status};
   use_split(s1, sk, cap);
-  EpiBwdDH::Args e1{g_ovf, u_ovf, duz_ovf, du_ovf, dz_ovf, lambda, f};
+  EpiBwdDH::Args e1{g_ovf, u_ovf, plan, op.duz_hi, op.duz_hi + static_cast<size_t>(cap_r) * 2 * f, op.h_hi,
+                    op.h_hi + static_cast<size_t>(cap_r) * f, du_ovf, dz_ovf, lambda, f};
   cudaError_t e = launch_rows_gemm<EpiBwdDH, false>("ovf_dh_gemm", ta, tb, ta, tb, tbp, tbp, s1, e1, cap, s);
   if (e != cudaSuccess) return e;
   GemmShape s2{cap, n_ovf, d, f, f, status};
@@ -450,32 +484,36 @@ cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const u
 cudaError_t launch_dense_wgrad(const DenseWgradOperands& op, const int* k_rows, int cap, int d, int f, float* dW_g,
                                float* dW_u, float* dW_d, uint32_t* status, cudaStream_t s) {
   if (cap <= 0) return cudaSuccess;
-  const uint64_t rows = dense_wgrad_rows(cap);
-  CUtensorMap ta, tb, ta2, tb2;
-  // the contraction runs over the operand rows (hi rows, then lo rows): every operand is [K = rows][M or N]
-  if (!make_tmap_bf16(&ta, op.duz2, 2 * static_cast<uint64_t>(f), rows, static_cast<uint64_t>(f) * 4, 64, kBK) ||
-      !make_tmap_bf16(&tb, op.x2, d, rows, static_cast<uint64_t>(d) * 2, 64, kBK) ||
-      !make_tmap_bf16(&ta2, op.dy2, d, rows, static_cast<uint64_t>(d) * 2, 64, kBK) ||
-      !make_tmap_bf16(&tb2, op.h2, f, rows, static_cast<uint64_t>(f) * 2, 64, kBK))
+  const uint64_t cap_r = dense_rows_padded(cap);
+  CUtensorMap ta0, ta1, tb, ta2, tb20, tb21;
+  // the contraction runs over the dense rows twice, once with the hi operand and once
+  // with the lo one (two K segments of *k_rows rows each); every operand is [K = rows][M or N]
+  if (!make_tmap_bf16(&ta0, op.duz_hi, 2 * static_cast<uint64_t>(f), cap_r, static_cast<uint64_t>(f) * 4, 64, kBK) ||
+      !make_tmap_bf16(&ta1, op.duz_hi + cap_r * 2 * f, 2 * static_cast<uint64_t>(f), cap_r,
+                      static_cast<uint64_t>(f) * 4, 64, kBK) ||
+      !make_tmap_bf16(&tb, op.x_rows, d, cap_r, static_cast<uint64_t>(d) * 2, 64, kBK) ||
+      !make_tmap_bf16(&ta2, op.dy_rows, d, cap_r, static_cast<uint64_t>(d) * 2, 64, kBK) ||
+      !make_tmap_bf16(&tb20, op.h_hi, f, cap_r, static_cast<uint64_t>(f) * 2, 64, kBK) ||
+      !make_tmap_bf16(&tb21, op.h_hi + cap_r * f, f, cap_r, static_cast<uint64_t>(f) * 2, 64, kBK))
     return cudaErrorInvalidValue;
   // [dW_u ; dW_g] (2 d_ff x d_model) = [dU | dZ]^T X_ovf
-  GemmShape s1{2 * f, nullptr, d, static_cast<int>(rows), 0, status};
+  GemmShape s1{2 * f, nullptr, d, static_cast<int>(cap_r), static_cast<int>(cap_r), status};
   s1.K_dev = k_rows;
   EpiStoreF32::Args e1{dW_u, dW_g, f, d};
 #if TWELL_PAIR_GEMM
-  cudaError_t e = launch_umma_pair<EpiStoreF32, true, kPairStages, true>("dense_wgrad_ug", ta, tb, ta, tb, s1, e1, s);
+  cudaError_t e = launch_umma_pair<EpiStoreF32, true, kPairStages, true>("dense_wgrad_ug", ta0, tb, ta1, tb, s1, e1, s);
 #else
-  cudaError_t e = launch_umma_gemm<EpiStoreF32, 256, true, kStages, true>("dense_wgrad_ug", ta, tb, ta, tb, s1, e1, s);
+  cudaError_t e = launch_umma_gemm<EpiStoreF32, 256, true, kStages, true>("dense_wgrad_ug", ta0, tb, ta1, tb, s1, e1, s);
 #endif
   if (e != cudaSuccess) return e;
   // dW_d (d_model x d_ff) = dY_ovf^T H_ovf
-  GemmShape s2{d, nullptr, f, static_cast<int>(rows), 0, status};
+  GemmShape s2{d, nullptr, f, static_cast<int>(cap_r), static_cast<int>(cap_r), status};
   s2.K_dev = k_rows;
   EpiStoreF32::Args e2{dW_d, dW_d, d, f};
 #if TWELL_PAIR_GEMM
-  return launch_umma_pair<EpiStoreF32, true, kPairStages, true>("dense_wgrad_d", ta2, tb2, ta2, tb2, s2, e2, s);
+  return launch_umma_pair<EpiStoreF32, true, kPairStages, true>("dense_wgrad_d", ta2, tb20, ta2, tb21, s2, e2, s);
 #else
-  return launch_umma_gemm<EpiStoreF32, 256, true, kStages, true>("dense_wgrad_d", ta2, tb2, ta2, tb2, s2, e2, s);
+  return launch_umma_gemm<EpiStoreF32, 256, true, kStages, true>("dense_wgrad_d", ta2, tb20, ta2, tb21, s2, e2, s);
 #endif
 }
 

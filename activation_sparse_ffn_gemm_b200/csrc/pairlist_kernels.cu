@@ -422,99 +422,80 @@ __global__ void __launch_bounds__(kWgWarps * 32, kWgMinBlocks) wgrad_kernel(cons
   }
 }
 
-// Operands of the dense weight gradients of the overflow rows (layout in
-// DenseWgradOperands), db_ovf[j] = sum over s < n of dZ[s][j] in ascending s,
-// and k_rows = np + n. When the plan keeps the overflow rows on the sparse
-// path, only k_rows = 0 and db_ovf = 0 are written. One block per operand row
-// pair (s, np + s), s < np.
-__device__ __forceinline__ void split_hi_lo(const float (&v)[8], uint4& hi, uint4& lo) {
-  float h[8], l[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    h[e] = __bfloat162float(__float2bfloat16_rn(v[e]));
-    l[e] = v[e] - h[e];  // exact in fp32
-  }
-  hi = make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]), pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
-  lo = make_uint4(pack_bf16x2(l[0], l[1]), pack_bf16x2(l[2], l[3]), pack_bf16x2(l[4], l[5]), pack_bf16x2(l[6], l[7]));
-}
-
-__global__ void ovf_operands_kernel(const int* __restrict__ n_ovf, const int* __restrict__ ovf_rows,
-                                    const int* __restrict__ plan, int cap, int M, int d, int f, uint32_t* status,
-                                    const uint16_t* __restrict__ X,
-                                    const uint16_t* __restrict__ dy_ovf, const float* __restrict__ du_ovf,
-                                    const float* __restrict__ dz_ovf, const uint16_t* __restrict__ g_ovf,
-                                    const float* __restrict__ u_ovf, DenseWgradOperands op, float* __restrict__ db_ovf,
-                                    int* __restrict__ k_rows) {
-  const bool dense = plan[3] != 0;
-  int n = dense ? n_ovf[0] : 0;
+// Rows of X and dY of the stored overflow rows (one block per row, grid-stride),
+// and, when the dense weight gradients run as GEMMs, zeros in the rows
+// [n, roundup(n, 64)) of every operand block (the GEMMs contract over whole
+// 64-row blocks; these rows must add nothing).
+__global__ void ovf_prep_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ dY,
+                                const int* __restrict__ ovf_rows, const int* __restrict__ n_ovf,
+                                const int* __restrict__ plan, int cap, int M, int d, int f, DenseWgradOperands op,
+                                uint32_t* status) {
+  int n = n_ovf[0];
   if (!in_bounds(n <= cap, status)) n = cap;
-  const int np = (n + 63) / 64 * 64;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *k_rows = n > 0 ? np + n : 0;
-  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < f; j += gridDim.x * blockDim.x) {
-    float acc = 0.f;
-    for (int sl = 0; sl < n; ++sl) acc += dz_ovf[static_cast<long>(sl) * f + j];
-    db_ovf[j] = acc;
-  }
+  const bool dense = plan[3] != 0;
+  const int np = dense ? (n + 63) / 64 * 64 : n;
+  const long cap_r = dense_rows_padded(cap);
   const uint4 z = make_uint4(0, 0, 0, 0);
   for (int sl = blockIdx.x; sl < np; sl += gridDim.x) {
-    const int src_row = sl < n ? ovf_rows[sl] : 0;
-    const bool live = sl < n && in_bounds(src_row >= 0 && src_row < M, status);
-    const long r_hi = sl, r_lo = static_cast<long>(np) + sl;
-    {
-      const uint4* xi = live ? reinterpret_cast<const uint4*>(X + static_cast<long>(src_row) * d) : nullptr;
-      const uint4* yi = live ? reinterpret_cast<const uint4*>(dy_ovf + static_cast<long>(sl) * d) : nullptr;
-      uint4* xh = reinterpret_cast<uint4*>(op.x2 + r_hi * d);
-      uint4* xl = reinterpret_cast<uint4*>(op.x2 + r_lo * d);
-      uint4* yh = reinterpret_cast<uint4*>(op.dy2 + r_hi * d);
-      uint4* yl = reinterpret_cast<uint4*>(op.dy2 + r_lo * d);
+    uint4* xo = reinterpret_cast<uint4*>(op.x_rows + static_cast<long>(sl) * d);
+    uint4* yo = reinterpret_cast<uint4*>(op.dy_rows + static_cast<long>(sl) * d);
+    const int r = sl < n ? ovf_rows[sl] : -1;
+    if (sl < n && in_bounds(r >= 0 && r < M, status)) {
+      const uint4* xi = reinterpret_cast<const uint4*>(X + static_cast<long>(r) * d);
+      const uint4* yi = reinterpret_cast<const uint4*>(dY + static_cast<long>(r) * d);
       for (int q = threadIdx.x; q < d / 8; q += blockDim.x) {
-        const uint4 xv = live ? xi[q] : z, yv = live ? yi[q] : z;
-        xh[q] = xv;
-        xl[q] = xv;
-        yh[q] = yv;
-        yl[q] = yv;
+        xo[q] = xi[q];
+        yo[q] = yi[q];
       }
+      continue;
     }
-    for (int q = threadIdx.x; q < f / 8; q += blockDim.x) {
-      uint4 uh = z, ul = z, zh = z, zl = z, hh = z, hl = z;
-      if (live) {
-        const long o = static_cast<long>(sl) * f + 8 * q;
-        float du[8], dz[8], h[8];
-        const float4 a0 = reinterpret_cast<const float4*>(du_ovf + o)[0], a1 = reinterpret_cast<const float4*>(du_ovf + o)[1];
-        const float4 b0 = reinterpret_cast<const float4*>(dz_ovf + o)[0], b1 = reinterpret_cast<const float4*>(dz_ovf + o)[1];
-        const float4 c0 = reinterpret_cast<const float4*>(u_ovf + o)[0], c1 = reinterpret_cast<const float4*>(u_ovf + o)[1];
-        float g8[8];
-        unpack8(*reinterpret_cast<const uint4*>(g_ovf + o), g8);
-        const float u8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        du[0] = a0.x; du[1] = a0.y; du[2] = a0.z; du[3] = a0.w; du[4] = a1.x; du[5] = a1.y; du[6] = a1.z; du[7] = a1.w;
-        dz[0] = b0.x; dz[1] = b0.y; dz[2] = b0.z; dz[3] = b0.w; dz[4] = b1.x; dz[5] = b1.y; dz[6] = b1.z; dz[7] = b1.w;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) h[e] = g8[e] * u8[e];  // h = g u in fp32, as on the sparse path
-        split_hi_lo(du, uh, ul);
-        split_hi_lo(dz, zh, zl);
-        split_hi_lo(h, hh, hl);
-      }
-      reinterpret_cast<uint4*>(op.duz2 + r_hi * 2 * f)[q] = uh;
-      reinterpret_cast<uint4*>(op.duz2 + r_lo * 2 * f)[q] = ul;
-      reinterpret_cast<uint4*>(op.duz2 + r_hi * 2 * f + f)[q] = zh;
-      reinterpret_cast<uint4*>(op.duz2 + r_lo * 2 * f + f)[q] = zl;
-      reinterpret_cast<uint4*>(op.h2 + r_hi * f)[q] = hh;
-      reinterpret_cast<uint4*>(op.h2 + r_lo * f)[q] = hl;
+    // a padding row of the dense weight gradients' blocks
+    for (int q = threadIdx.x; q < d / 8; q += blockDim.x) xo[q] = yo[q] = z;
+    for (int blk = 0; blk < 2; ++blk) {
+      uint4* du = reinterpret_cast<uint4*>(op.duz_hi + (blk * cap_r + sl) * 2 * f);
+      uint4* hh = reinterpret_cast<uint4*>(op.h_hi + (blk * cap_r + sl) * f);
+      for (int q = threadIdx.x; q < f / 4; q += blockDim.x) du[q] = z;
+      for (int q = threadIdx.x; q < f / 8; q += blockDim.x) hh[q] = z;
     }
+  }
+}
+
+// db_ovf[j] = sum over s < n of dZ[s][j] (hi + lo, ascending s) and
+// k_rows = n when the dense weight gradients run as GEMMs; else both 0.
+__global__ void ovf_db_kernel(const int* __restrict__ n_ovf, const int* __restrict__ plan, int cap, int f,
+                              DenseWgradOperands op, float* __restrict__ db_ovf, int* __restrict__ k_rows) {
+  const bool dense = plan[3] != 0;
+  int n = dense ? n_ovf[0] : 0;
+  n = n < cap ? n : cap;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *k_rows = n;
+  const long cap_r = dense_rows_padded(cap);
+  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < f; j += gridDim.x * blockDim.x) {
+    float acc = 0.f;
+    for (int sl = 0; sl < n; ++sl) {
+      const uint16_t hi = op.duz_hi[static_cast<long>(sl) * 2 * f + f + j];
+      const uint16_t lo = op.duz_hi[(cap_r + sl) * 2 * f + f + j];
+      acc += __uint_as_float(static_cast<uint32_t>(hi) << 16) + __uint_as_float(static_cast<uint32_t>(lo) << 16);
+    }
+    db_ovf[j] = acc;
   }
 }
 
 }  // namespace
 
-cudaError_t launch_ovf_operands(const int* n_ovf, const int* ovf_rows, const int* plan, int cap, int M, int d, int f,
-                                const uint16_t* X, const uint16_t* dy_ovf, const float* du_ovf, const float* dz_ovf,
-                                const uint16_t* g_ovf, const float* u_ovf, const DenseWgradOperands& op,
-                                float* db_ovf, int* k_rows, uint32_t* status, cudaStream_t s) {
+cudaError_t launch_ovf_prep(const uint16_t* X, const uint16_t* dY, const int* ovf_rows, const int* n_ovf,
+                            const int* plan, int cap, int M, int d, int f, const DenseWgradOperands& op,
+                            uint32_t* status, cudaStream_t s) {
   if (cap <= 0) return cudaSuccess;
-  const int g = device_sm_count() * 2;
-  TWELL_LAUNCH("ovf_operands", s,
-               ovf_operands_kernel<<<g, 256, 0, s>>>(n_ovf, ovf_rows, plan, cap, M, d, f, status, X, dy_ovf, du_ovf, dz_ovf,
-                                                     g_ovf, u_ovf, op, db_ovf, k_rows));
+  const int g = dense_rows_padded(cap) < device_sm_count() * 4 ? dense_rows_padded(cap) : device_sm_count() * 4;
+  TWELL_LAUNCH("ovf_prep", s,
+               ovf_prep_kernel<<<g, 256, 0, s>>>(X, dY, ovf_rows, n_ovf, plan, cap, M, d, f, op, status));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ovf_db(const int* n_ovf, const int* plan, int cap, int f, const DenseWgradOperands& op,
+                          float* db_ovf, int* k_rows, cudaStream_t s) {
+  if (cap <= 0) return cudaSuccess;
+  TWELL_LAUNCH("ovf_db", s, ovf_db_kernel<<<(f + 255) / 256, 256, 0, s>>>(n_ovf, plan, cap, f, op, db_ovf, k_rows));
   return cudaGetLastError();
 }
 

@@ -254,20 +254,6 @@ __global__ void ovf_gather_kernel(const int* __restrict__ n_ovf, const int* __re
   }
 }
 
-__global__ void gather_rows_kernel(const uint16_t* __restrict__ in, const int* __restrict__ rows,
-                                   const int* __restrict__ n_ovf, int cap, int M, int d, uint16_t* __restrict__ out,
-                                   uint32_t* status) {
-  int n = n_ovf[0];
-  if (!in_bounds(n <= cap, status)) n = cap;
-  for (int sl = blockIdx.x; sl < n; sl += gridDim.x) {
-    const int r = rows[sl];
-    if (!in_bounds(r >= 0 && r < M, status)) continue;
-    const uint4* src = reinterpret_cast<const uint4*>(in + static_cast<long>(r) * d);
-    uint4* dst = reinterpret_cast<uint4*>(out + static_cast<long>(sl) * d);
-    for (int q = threadIdx.x; q < d / 8; q += blockDim.x) dst[q] = src[q];
-  }
-}
-
 // out[c][r] = in[r][c] for a [rows][cols] bf16 matrix (rows, cols multiples of
 // 8). A CTA moves a 64-row x 128-column tile: every thread first issues its four
 // 16-byte loads (256 contiguous bytes per input row), then parks them in shared
@@ -335,14 +321,6 @@ cudaError_t launch_route(const uint16_t* count, const uint16_t* val, const uint8
                  ovf_gather_kernel<<<g, 256, 0, s>>>(n_ovf, ovf_rows, count, val, col, spill, M, f, K, cap, g_ovf, X,
                                                      d, x_ovf, status));
   }
-  return cudaGetLastError();
-}
-
-cudaError_t launch_gather_rows(const uint16_t* in, const int* rows, const int* n_ovf, int cap, int M, int d,
-                               uint16_t* out, uint32_t* status, cudaStream_t s) {
-  if (cap <= 0) return cudaSuccess;
-  int g = cap < device_sm_count() * 4 ? cap : device_sm_count() * 4;
-  TWELL_LAUNCH("gather_rows", s, gather_rows_kernel<<<g, 256, 0, s>>>(in, rows, n_ovf, cap, M, d, out, status));
   return cudaGetLastError();
 }
 

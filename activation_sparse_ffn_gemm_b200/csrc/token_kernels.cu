@@ -39,6 +39,12 @@
 #include "token_common.cuh"
 #include "trace.cuh"
 
+// Cache hints on the token's own rows (streaming loads and stores, so the
+// gathered weight rows keep L2); 0 builds the plain loads and stores.
+#ifndef TWELL_STREAM_HINTS
+#define TWELL_STREAM_HINTS 1
+#endif
+
 namespace twell {
 
 namespace {
@@ -93,6 +99,22 @@ __device__ __forceinline__ void load_row(const uint16_t* __restrict__ base, int 
   for (int q = 0; q < C; ++q) {
     const int idx = first + W * 32 * q;
     v[q] = (EXACT || idx < nch) ? __ldg(p + idx) : make_uint4(0, 0, 0, 0);
+  }
+}
+
+// The token's own row (x or dY): read once per piece, so it is loaded with the
+// streaming hint (evict first) and leaves L2 to the gathered weight rows.
+template <int C, int W, bool EXACT>
+__device__ __forceinline__ void load_token_row(const uint16_t* __restrict__ base, int first, int nch, uint4 (&v)[C]) {
+  const uint4* p = reinterpret_cast<const uint4*>(base);
+#pragma unroll
+  for (int q = 0; q < C; ++q) {
+    const int idx = first + W * 32 * q;
+#if TWELL_STREAM_HINTS
+    v[q] = (EXACT || idx < nch) ? __ldcs(p + idx) : make_uint4(0, 0, 0, 0);
+#else
+    v[q] = (EXACT || idx < nch) ? __ldg(p + idx) : make_uint4(0, 0, 0, 0);
+#endif
   }
 }
 
@@ -258,7 +280,7 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
   auto up = [&](long row, int ne) {
     {
       uint4 xp[C];
-      load_row<C, W, EXACT>(X + row * d, first, nch, xp);
+      load_token_row<C, W, EXACT>(X + row * d, first, nch, xp);
       gather_dots<C, W, B, EXACT>(g, ne, xp, Wu, d, first, nch, lane, g.c2, part[grp][wi]);
     }
     group_sync<W>(grp);
@@ -279,9 +301,15 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
 #pragma unroll
     for (int q = 0; q < C; ++q) {
       const int idx = first + W * 32 * q;
-      if (EXACT || idx < nch)
-        yr[idx] = make_uint4(pack_bf16x2(y[q][0].x, y[q][0].y), pack_bf16x2(y[q][1].x, y[q][1].y),
-                             pack_bf16x2(y[q][2].x, y[q][2].y), pack_bf16x2(y[q][3].x, y[q][3].y));
+      if (EXACT || idx < nch) {
+        const uint4 v = make_uint4(pack_bf16x2(y[q][0].x, y[q][0].y), pack_bf16x2(y[q][1].x, y[q][1].y),
+                                   pack_bf16x2(y[q][2].x, y[q][2].y), pack_bf16x2(y[q][3].x, y[q][3].y));
+#if TWELL_STREAM_HINTS
+        __stcs(yr + idx, v);
+#else
+        yr[idx] = v;
+#endif
+      }
     }
   };
 
@@ -341,7 +369,7 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
   auto dh_phase = [&](long row, int ne) {
     {
       uint4 dyp[C];
-      load_row<C, W, EXACT>(dY + row * d, first, nch, dyp);
+      load_token_row<C, W, EXACT>(dY + row * d, first, nch, dyp);
       gather_dots<C, W, B, EXACT>(g, ne, dyp, Wdt, d, first, nch, lane, dhv[grp], part[grp][wi]);
     }
     group_sync<W>(grp);

@@ -90,9 +90,9 @@ struct WsLayout {
   size_t yacc = 0;  // fp32 accumulator rows of rows split into several pieces
   size_t sk_partial = 0, sk_arrivals = 0;  // split-K scratch of the dense-backup GEMMs
   size_t spill = 0, x_ovf = 0, h_ovf = 0, w_dt = 0;
-  size_t x2 = 0, dy2 = 0, duz2 = 0, h2 = 0, db_ovf = 0, k_rows = 0;  // operands of the dense weight gradients
-  size_t dy_ovf = 0, duz = 0, du_ovf = 0, dz_ovf = 0, hdz_ell = 0, block_cnt = 0, unit_tot = 0, unit_ptr = 0, scan_arrive = 0,
-         csc_row = 0, csc_val = 0;
+  size_t x_rows = 0, dy_rows = 0, duz_hi = 0, h_hi = 0, db_ovf = 0, k_rows = 0;  // dense backward operands
+  size_t du_ovf = 0, dz_ovf = 0, hdz_ell = 0, block_cnt = 0, unit_tot = 0, unit_ptr = 0, scan_arrive = 0, csc_row = 0,
+         csc_val = 0;
   size_t total = 0;
 };
 
@@ -120,15 +120,13 @@ WsLayout ws_layout(twell_op op, int64_t M, int64_t d, int64_t f, int64_t K, int6
   }
   if (op == TWELL_OP_BWD) {
     L.w_dt = take(static_cast<size_t>(f * d * 2));
-    L.dy_ovf = take(static_cast<size_t>(cap1 * d * 2));
-    L.duz = take(static_cast<size_t>(cap1 * 2 * f * 2));
+    const int64_t cap_r = dense_rows_padded(static_cast<int>(cap1));
+    L.x_rows = take(static_cast<size_t>(cap_r * d * 2));
+    L.dy_rows = take(static_cast<size_t>(cap_r * d * 2));
+    L.duz_hi = take(static_cast<size_t>(2 * cap_r * 2 * f * 2));
+    L.h_hi = take(static_cast<size_t>(2 * cap_r * f * 2));
     L.du_ovf = take(static_cast<size_t>(cap1 * f * 4));
     L.dz_ovf = take(static_cast<size_t>(cap1 * f * 4));
-    const int64_t r2 = dense_wgrad_rows(cap1);
-    L.x2 = take(static_cast<size_t>(r2 * d * 2));
-    L.dy2 = take(static_cast<size_t>(r2 * d * 2));
-    L.duz2 = take(static_cast<size_t>(r2 * 2 * f * 2));
-    L.h2 = take(static_cast<size_t>(r2 * f * 2));
     L.db_ovf = take(static_cast<size_t>(f * 4));
     L.k_rows = take(64);
     L.hdz_ell = take(static_cast<size_t>(M * T * K * 16));
@@ -395,26 +393,23 @@ twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_
     if (launch_transpose_bf16(W_d, d, f, t, s) != cudaSuccess) return TWELL_ECUDA;
     wdt = t;
   }
-  uint16_t* dy_ovf = at<uint16_t>(ws, L.dy_ovf);
-  uint16_t* duz = at<uint16_t>(ws, L.duz);
   float4* hdz_ell = at<float4>(ws, L.hdz_ell);
-  if (launch_gather_rows(dY, h->ovf_rows, h->n_ovf, cap, M, d, dy_ovf, h->status, s) != cudaSuccess) return TWELL_ECUDA;
+  const DenseWgradOperands dw{at<uint16_t>(ws, L.x_rows), at<uint16_t>(ws, L.dy_rows), at<uint16_t>(ws, L.duz_hi),
+                              at<uint16_t>(ws, L.h_hi)};
+  if (launch_ovf_prep(X, dY, h->ovf_rows, h->n_ovf, h->row_plan, cap, M, d, f, dw, h->status, s) != cudaSuccess)
+    return TWELL_ECUDA;
   if (launch_ell_ffn_bwd(dY, W_u, W_g, wdt, h->count, h->val, h->col, h->row_plan, h->n_ovf, h->u_ell, lambda,
                          hdz_ell, dX, M, d, f, K, at<int>(ws, L.ctr), h->status, s) != cudaSuccess)
     return TWELL_ECUDA;
   float* du_ovf = at<float>(ws, L.du_ovf);
   float* dz_ovf = at<float>(ws, L.dz_ovf);
   const SplitKBuffers sk{at<float>(ws, L.sk_partial), at<unsigned long long>(ws, L.sk_arrivals)};
-  const DenseWgradOperands dw{at<uint16_t>(ws, L.x2), at<uint16_t>(ws, L.dy2), at<uint16_t>(ws, L.duz2),
-                              at<uint16_t>(ws, L.h2)};
   float* db_ovf = at<float>(ws, L.db_ovf);
   int* k_rows = at<int>(ws, L.k_rows);
-  if (launch_ovf_bwd(dy_ovf, wdt, W_u, W_g, h->g_ovf, h->u_ovf, lambda, h->ovf_rows, h->n_ovf, cap, M, d, f, duz,
-                     du_ovf, dz_ovf, dX, sk, h->status, s) != cudaSuccess)
+  if (launch_ovf_bwd(dw.dy_rows, wdt, W_u, W_g, h->g_ovf, h->u_ovf, lambda, h->ovf_rows, h->n_ovf, h->row_plan, cap, M,
+                     d, f, dw, du_ovf, dz_ovf, dX, sk, h->status, s) != cudaSuccess)
     return TWELL_ECUDA;
-  if (launch_ovf_operands(h->n_ovf, h->ovf_rows, h->row_plan, cap, M, d, f, X, dy_ovf, du_ovf, dz_ovf, h->g_ovf,
-                          h->u_ovf, dw, db_ovf, k_rows, h->status, s) != cudaSuccess)
-    return TWELL_ECUDA;
+  if (launch_ovf_db(h->n_ovf, h->row_plan, cap, f, dw, db_ovf, k_rows, s) != cudaSuccess) return TWELL_ECUDA;
   const long long nnz_cap = static_cast<long long>(M - cap) * (f / kTn) * K + static_cast<long long>(cap) * f;
   CscBuffers b{M, cap, nnz_cap, h->status, h->row_plan + kPlanHdr + M, at<int>(ws, L.block_cnt),
                at<int>(ws, L.unit_tot), at<unsigned long long>(ws, L.scan_arrive), at<int>(ws, L.unit_ptr),

@@ -147,10 +147,6 @@ cudaError_t launch_route(const uint16_t* count, const uint16_t* val, const uint8
 // launch shape they use); sizes the pieces of the row plan.
 int tok_groups(int M, int d);
 
-// out[s][:] = in[rows[s]][:] for s < n_ovf[0] (bf16 rows of width d, M rows in `in`).
-cudaError_t launch_gather_rows(const uint16_t* in, const int* rows, const int* n_ovf, int cap, int M, int d,
-                               uint16_t* out, uint32_t* status, cudaStream_t s);
-
 cudaError_t launch_transpose_bf16(const uint16_t* in, int rows, int cols, uint16_t* out, cudaStream_t s);
 
 // Fused sparse up + down over the pieces of the row plan (ELL rows only).
@@ -202,32 +198,52 @@ cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const ui
                                float4* hdz_ell, float* dX, int M, int d, int f, int K, int* ctr, uint32_t* status,
                                cudaStream_t s);
 
-// Dense backup backward for overflow rows: dU, dZ (fp32, and bf16 [dU | dZ] as
-// the next GEMM's operand) from dH = dY_ovf W_d, then dX[ovf_rows] = dU W_u + dZ W_g.
+// Operands of the dense backup backward and of the dense weight gradients of the
+// overflow rows, with cap_r = dense_rows_padded(cap) rows per block; for the n
+// stored overflow rows the first n rows of each block are live and the rows
+// [n, roundup(n, 64)) are zero when the weight gradients run as GEMMs:
+//   x_rows, dy_rows   [cap_r][d]        X and dY of the overflow rows (dy_rows is
+//                                        also the A operand of the dH GEMM)
+//   duz_hi            [2 cap_r][2f]      bf16 [dU | dZ] ("hi", the dX GEMM's operand),
+//                                        then the "lo" block bf16([dU | dZ] - hi)
+//   h_hi              [2 cap_r][f]       H = g u hi, then lo
+// hi + lo carries a value to about 2^-16 of it: bf16 alone loses too much where
+// one heavy token dominates a weight-gradient element.
+struct DenseWgradOperands {
+  uint16_t* x_rows;
+  uint16_t* dy_rows;
+  uint16_t* duz_hi;
+  uint16_t* h_hi;
+};
+__host__ __device__ inline int dense_rows_padded(int cap) { return (cap + 63) / 64 * 64; }
+
+// Rows of X and dY of the stored overflow rows into the operand blocks, and the
+// zero rows [n, roundup(n, 64)) of every block when plan[3] selects the dense
+// weight gradients.
+cudaError_t launch_ovf_prep(const uint16_t* X, const uint16_t* dY, const int* ovf_rows, const int* n_ovf,
+                            const int* plan, int cap, int M, int d, int f, const DenseWgradOperands& op,
+                            uint32_t* status, cudaStream_t s);
+
+// Dense backup backward for overflow rows, from dH = dY_ovf W_d: dU and dZ into
+// the operand blocks (and fp32 du / dz when the pair list takes the overflow
+// rows), then dX[ovf_rows] = dU W_u + dZ W_g.
 cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const uint16_t* W_u,
                            const uint16_t* W_g, const uint16_t* g_ovf, const float* u_ovf, float lambda,
-                           const int* ovf_rows, const int* n_ovf, int cap, int M, int d, int f, uint16_t* duz_ovf,
-                           float* du_ovf, float* dz_ovf, float* dX, const SplitKBuffers& sk, uint32_t* status,
-                           cudaStream_t s);
+                           const int* ovf_rows, const int* n_ovf, const int* plan, int cap, int M, int d, int f,
+                           const DenseWgradOperands& op, float* du_ovf, float* dz_ovf, float* dX,
+                           const SplitKBuffers& sk, uint32_t* status, cudaStream_t s);
 
-// Operands of the dense weight gradients of the overflow rows, each with
-// dense_wgrad_rows(cap) rows of bf16: for the n stored overflow rows and
-// np = roundup(n, 64), rows [0, n) hold the "hi" part and rows [np, np + n)
-// the "lo" part, so that hi + lo carries a value to about 2^-16 (bf16 alone
-// loses too much where one heavy token dominates a gradient element); every
-// other row up to 2 np is zero. X and dY are exact in bf16 and appear twice.
-struct DenseWgradOperands {
-  uint16_t* x2;    // [rows][d]   X[ovf_rows[s]] (hi and lo halves equal)
-  uint16_t* dy2;   // [rows][d]   dY[ovf_rows[s]]
-  uint16_t* duz2;  // [rows][2f]  [dU | dZ] hi / lo
-  uint16_t* h2;    // [rows][f]   H = g u hi / lo
-};
-inline int64_t dense_wgrad_rows(int64_t cap) { return 2 * ((cap + 63) / 64 * 64); }
+// After the dense backward: column sums of dZ over the overflow rows (db_ovf,
+// hi + lo in ascending row order) and the contraction length k_rows = n of the
+// dense weight-gradient GEMMs; both 0 when the plan keeps the overflow rows on
+// the sparse path (the pair list then carries them).
+cudaError_t launch_ovf_db(const int* n_ovf, const int* plan, int cap, int f, const DenseWgradOperands& op,
+                          float* db_ovf, int* k_rows, cudaStream_t s);
 
 // Weight gradients of the dense backup rows on the tensor cores, written
 // before the sparse kernel adds the ELL rows' sums: [dW_u ; dW_g] = [dU | dZ]^T X_ovf,
-// dW_d = dY_ovf^T H_ovf, contracting over the first *k_rows operand rows
-// (0: nothing is written).
+// dW_d = dY_ovf^T H_ovf, each over the hi and the lo operand (two K segments of
+// *k_rows rows; 0: nothing is written).
 cudaError_t launch_dense_wgrad(const DenseWgradOperands& op, const int* k_rows, int cap, int d, int f, float* dW_g,
                                float* dW_u, float* dW_d, uint32_t* status, cudaStream_t s);
 
@@ -251,16 +267,6 @@ cudaError_t launch_build_csc(const uint16_t* count, const uint8_t* col, const ui
                              const uint16_t* g_ovf, const float* u_ovf, const float4* hdz_ell, const float* du_ovf,
                              const float* dz_ovf, const int* plan, int M, int f, int K, const CscBuffers& b,
                              cudaStream_t s);
-
-// After the dense backward: the operands of the dense weight gradients (from X,
-// the gathered dY rows, fp32 dU / dZ and g, u of the overflow rows), column
-// sums of dZ over the overflow rows (db_ovf) and the contraction length
-// k_rows = roundup(n, 64) + n (0 when the plan keeps the overflow rows on the
-// sparse path, and then db_ovf = 0).
-cudaError_t launch_ovf_operands(const int* n_ovf, const int* ovf_rows, const int* plan, int cap, int M, int d, int f,
-                                const uint16_t* X, const uint16_t* dy_ovf, const float* du_ovf, const float* dz_ovf,
-                                const uint16_t* g_ovf, const float* u_ovf, const DenseWgradOperands& op,
-                                float* db_ovf, int* k_rows, uint32_t* status, cudaStream_t s);
 
 // dW_u = dU^T X, dW_g = dZ^T X, dW_d = dY^T H, db_g = column sums of dZ (plus
 // db_extra when non-null) over the pairs of the pair list; the weight

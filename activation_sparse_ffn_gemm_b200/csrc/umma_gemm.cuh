@@ -48,8 +48,9 @@ struct GemmShape {
   int K0;            // K extent of segment 0 (multiple of kBK)
   int K1;            // K extent of segment 1 (0: single segment)
   uint32_t* status;
-  const int* K_dev = nullptr;  // single segment only: K processed = min(*K_dev, K0), rounded up to kBK
-                               // (operand rows between *K_dev and the rounding must read as zero)
+  const int* K_dev = nullptr;  // K processed per segment = min(*K_dev, K0), rounded up to kBK, for both
+                               // segments when K1 > 0 (then K1 must equal K0); operand rows between *K_dev
+                               // and the rounding must read as zero
   float* partial = nullptr;  // split-K partials [split_max][split_rows][N] fp32 (nullptr: no split-K)
   int split_rows = 0;        // split-K only when the processed rows are at most this many
   int split_max = 1;
@@ -170,7 +171,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   __syncthreads();
   const int nk0 = *k0_eff_s / kBK;
-  const int nk = nk0 + shp.K1 / kBK;
+  const int nk = nk0 + (shp.K_dev && shp.K1 > 0 ? nk0 : shp.K1 / kBK);
   if (nk == 0) return;  // nothing to contract (a device-side K of zero)
   const int split = gemm_split(*m_eff_s, shp.N, BN, nk, shp, gridDim.x);
   if (shp.max_rows > 0 && *m_eff_s > shp.max_rows) return;  // the pair engine owns this row count

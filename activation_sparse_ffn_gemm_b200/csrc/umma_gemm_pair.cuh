@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int M_eff = *m_eff_s;
   const int nk0 = *k0_eff_s / kBK;
-  const int nk = nk0 + shp.K1 / kBK;
+  const int nk = nk0 + (shp.K_dev && shp.K1 > 0 ? nk0 : shp.K1 / kBK);
   const int num_m = (M_eff + kPairBM - 1) / kPairBM;
   const int num_n = (shp.N + kPairBN - 1) / kPairBN;
   const int num_tiles = nk > 0 && M_eff > shp.min_rows ? num_m * num_n : 0;

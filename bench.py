@@ -70,6 +70,9 @@ def parse_args():
     p.add_argument("--workload", default=MAIN_WORKLOAD, choices=["large", "train", "heavy"],
                    help="workload of the timed training step (synthetic.WORKLOADS)")
     p.add_argument("--no-extra", action="store_true", help="skip the two smaller workloads of the line")
+    p.add_argument("--step-only", action="store_true",
+                   help="time the training step alone (no trace, inference, 8-bit, end-to-end, dense or CPU legs, "
+                        "no smaller workloads): the command profiler captures run")
     p.add_argument("--sweep", action="store_true",
                    help="token-count x sparsity sweep at d_model=4096, d_ff=14336 (one JSON line per point)")
     p.add_argument("--sweep-m", default="512,2048,8192,32768,65536")
@@ -619,6 +622,9 @@ def run_twell(args, world, rank, local):
                            "max_count": float(cnt.max().item()), "mean_count": float(cnt.mean().item()),
                            "max_over_mean_count": float(cnt.max().item()) / max(float(cnt.mean().item()), 1e-30)}
         res["shape"] = (M, d, f, T, K)
+        if full and args.step_only:
+            res["clocks"] = clk.summary()
+            return res
         if full:
             res["clocks"] = clk.summary()
             # per-kernel breakdown: the same steps again with event tracing
@@ -750,6 +756,16 @@ def run_twell(args, world, rank, local):
 
     main = measure(args.workload, "train", full=True)
     others = {}
+    if args.step_only:
+        if dist is not None:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": main["M"] * world / (main["ms_step"] / 1e3),
+                              "unit": "tokens/s", "ms_per_step": main["ms_step"], "fwd_ms": main["ms_fwd"],
+                              "steps": args.steps, "warmup": max(3, args.warmup), "config": {
+                                  "workload": main["workload"], "note": "training step alone (profiling run)"},
+                              "sparsity": main["sparsity"], "gpu_launches": main["gpu_launches"]}), flush=True)
+        return
     if not args.no_extra:
         for key, wname, mode in OTHER_WORKLOADS:
             if wname != args.workload:
