@@ -44,10 +44,18 @@
 #ifndef TWELL_STREAM_HINTS
 #define TWELL_STREAM_HINTS 1
 #endif
+// 0: the fused sparse kernels; 1: the two-pass forward and backward (dots, then
+// the axpy over the other weight rows); 2: as 1 with the backward's dX pass
+// split into a W_u pass and a W_g pass.
+#ifndef TWELL_SPLIT_PHASES
+#define TWELL_SPLIT_PHASES 0
+#endif
 
 namespace twell {
 
 namespace {
+
+constexpr int kSplitPhases = TWELL_SPLIT_PHASES;
 
 // acc_lo += lo(a) * lo(w), acc_hi += hi(a) * hi(w) for two bf16x2 words: the
 // mixed-precision FMA takes the bf16 halves as they are (exact in fp32) with
@@ -254,6 +262,25 @@ __device__ __forceinline__ void store_acc(float* __restrict__ acc, int first, in
   }
 }
 
+// The bf16 row of Y from the fp32 accumulators (streaming store).
+template <int C, int W, bool EXACT>
+__device__ __forceinline__ void store_y(uint16_t* __restrict__ y_row, int first, int nch, const float2 (&y)[C][4]) {
+  uint4* yr = reinterpret_cast<uint4*>(y_row);
+#pragma unroll
+  for (int q = 0; q < C; ++q) {
+    const int idx = first + W * 32 * q;
+    if (EXACT || idx < nch) {
+      const uint4 v = make_uint4(pack_bf16x2(y[q][0].x, y[q][0].y), pack_bf16x2(y[q][1].x, y[q][1].y),
+                                 pack_bf16x2(y[q][2].x, y[q][2].y), pack_bf16x2(y[q][3].x, y[q][3].y));
+#if TWELL_STREAM_HINTS
+      __stcs(yr + idx, v);
+#else
+      yr[idx] = v;
+#endif
+    }
+  }
+}
+
 // yacc: [M][d] fp32 accumulator rows for rows split into several pieces.
 // TILES: tile-level routing; spill holds the dense slices of tiles with more
 // than K actives (u is not saved: an inference-only state).
@@ -426,6 +453,212 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
   }
 }
 
+// ------------------------------------------------------- two-pass variants
+// The same work as ell_fwd_kernel and ell_bwd_kernel, split so that each pass
+// gathers rows of fewer weight matrices: the resident working set of gathered
+// rows (one d_model-wide row per unit and matrix) then stays closer to L2's
+// capacity when the weights are large. The forward's first pass writes u per
+// kept slot (to u_ell, or to a workspace buffer for inference) and the second
+// reads it back; the backward's first pass writes (h, dU, dZ) per slot as the
+// fused kernel does, and the dX pass (or the two passes, W_u then W_g, adding
+// into dX) reads them. Each piece is still one pass's unit of work, and the
+// pieces of a split row still add their partials in order through the row's
+// turnstile, so results do not depend on scheduling.
+
+// List of entries [e0, e0 + ne) with the unit and both backward coefficients
+// (dU in c, dZ in c2) read from the per-slot record of the first pass.
+__device__ __forceinline__ void build_list_hdz(GroupSmem& g, long row, int T, int K, int e0, int ne, int gtid, int GT,
+                                               const uint8_t* __restrict__ col, const float4* __restrict__ hdz,
+                                               uint32_t* status) {
+  for (int e = gtid; e < ne; e += GT) {
+    int t, sl;
+    entry_of(g.off, T, e0 + e, t, sl);
+    const long base = (row * T + t) * K + sl;
+    const int c = col[base];
+    const bool ok = in_bounds(c < kTn, status);
+    g.j[e] = t * kTn + (ok ? c : 0);
+    const float4 v = hdz[base];
+    g.c[e] = ok ? v.y : 0.f;
+    g.c2[e] = ok ? v.z : 0.f;
+    g.slot[e] = t * K + sl;
+  }
+}
+
+template <int C, int W, bool EXACT>
+__global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>::WARPS * 32)) ell_up_kernel(
+    const uint16_t* __restrict__ X, const uint16_t* __restrict__ Wu, const uint16_t* __restrict__ count,
+    const uint16_t* __restrict__ val, const uint8_t* __restrict__ col, int* __restrict__ plan,
+    float* __restrict__ ubuf, int M, int d, int T, int K, int* __restrict__ ctr, uint32_t* status) {
+  using Cfg = TokCfg<C, W>;
+  constexpr int B = Cfg::B;
+  __shared__ GroupSmem gs[Cfg::G];
+  __shared__ float part[Cfg::G][W > 1 ? W : 1][kListCap];
+  __shared__ int s_next[Cfg::G];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = warp / W, wi = warp % W, gtid = wi * 32 + lane;
+  GroupSmem& g = gs[grp];
+  const int nch = d >> 3;
+  while (next_piece<W, false>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g, status)) {
+    const long row = g.row;
+    const int S = plan[1];
+    const int e0 = g.q * S;
+    const int ne = max(0, min(S, g.tot - e0));
+    build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, nullptr, status);
+    group_sync<W>(grp);
+    {
+      uint4 xp[C];
+      load_token_row<C, W, EXACT>(X + row * d, gtid, nch, xp);
+      gather_dots<C, W, B, EXACT>(g, ne, xp, Wu, d, gtid, nch, lane, g.c2, part[grp][wi]);
+    }
+    group_sync<W>(grp);
+    for (int e = gtid; e < ne; e += Cfg::GT) {
+      float u = g.c2[e];
+      if (W > 1) {
+        u = 0.f;
+#pragma unroll
+        for (int w = 0; w < W; ++w) u += part[grp][w][e];
+      }
+      ubuf[row * T * K + g.slot[e]] = u;
+    }
+    group_sync<W>(grp);  // the group's shared memory is rewritten for the next piece
+  }
+}
+
+template <int C, int W, bool EXACT>
+__global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>::WARPS * 32)) ell_down_kernel(
+    const uint16_t* __restrict__ Wdt, const uint16_t* __restrict__ count, const uint16_t* __restrict__ val,
+    const uint8_t* __restrict__ col, int* __restrict__ plan, const float* __restrict__ ubuf,
+    uint16_t* __restrict__ Y, int M, int d, int T, int K, int* __restrict__ ctr, float* __restrict__ yacc,
+    uint32_t* status) {
+  using Cfg = TokCfg<C, W>;
+  constexpr int B = Cfg::B;
+  __shared__ GroupSmem gs[Cfg::G];
+  __shared__ int s_next[Cfg::G];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = warp / W, wi = warp % W, gtid = wi * 32 + lane;
+  GroupSmem& g = gs[grp];
+  const int nch = d >> 3;
+  const int first = gtid;
+  int* turn = plan + kPlanHdr;
+  while (next_piece<W, false>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g, status)) {
+    const long row = g.row;
+    const int S = plan[1];
+    const int e0 = g.q * S;
+    const int ne = max(0, min(S, g.tot - e0));
+    build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, ubuf, status);
+    group_sync<W>(grp);
+    for (int e = gtid; e < ne; e += Cfg::GT) g.c[e] *= g.c2[e];  // h = g u
+    group_sync<W>(grp);
+    float2 y[C][4];
+    zero_acc<C>(y);
+    gather_axpy<C, W, B, EXACT>(g, ne, g.c, Wdt, d, first, nch, y);
+    const int rw = g.row, q = g.q, P = g.P;
+    if (P == 1) {
+      store_y<C, W, EXACT>(Y + static_cast<long>(rw) * d, first, nch, y);
+    } else {
+      float* acc = yacc + static_cast<long>(rw) * d;
+      turn_wait<W>(turn, rw, q, grp, gtid, status);
+      if (q > 0) add_acc<C, W, EXACT>(acc, first, nch, y);
+      if (q + 1 == P) store_y<C, W, EXACT>(Y + static_cast<long>(rw) * d, first, nch, y);
+      else store_acc<C, W, EXACT>(acc, first, nch, y);
+      turn_pass<W>(turn, rw, q, P, grp, gtid);
+    }
+    group_sync<W>(grp);
+  }
+}
+
+template <int C, int W, bool EXACT>
+__global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>::WARPS * 32)) ell_dh_kernel(
+    const uint16_t* __restrict__ dY, const uint16_t* __restrict__ Wdt, const uint16_t* __restrict__ count,
+    const uint16_t* __restrict__ val, const uint8_t* __restrict__ col, int* __restrict__ plan,
+    const int* __restrict__ n_ovf, const float* __restrict__ u_ell, float lambda, float4* __restrict__ hdz_ell,
+    int M, int d, int T, int K, int* __restrict__ ctr, uint32_t* status) {
+  using Cfg = TokCfg<C, W>;
+  constexpr int B = Cfg::B;
+  __shared__ GroupSmem gs[Cfg::G];
+  __shared__ float part[Cfg::G][W > 1 ? W : 1][kListCap];
+  __shared__ float dhv[Cfg::G][kListCap];
+  __shared__ int s_next[Cfg::G];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = warp / W, wi = warp % W, gtid = wi * 32 + lane;
+  GroupSmem& g = gs[grp];
+  const int nch = d >> 3;
+  if (plan[3] < 0) {  // a tile-routed (inference) state cannot serve the backward
+    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, TWELL_STATUS_BAD_STATE);
+    return;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0 && n_ovf[1] > n_ovf[0]) set_status(status, TWELL_STATUS_OVERFLOW_CAP);
+  while (next_piece<W, false>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g, status)) {
+    const long row = g.row;
+    const int S = plan[1];
+    const int e0 = g.q * S;
+    const int ne = max(0, min(S, g.tot - e0));
+    build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, u_ell, status);
+    group_sync<W>(grp);
+    {
+      uint4 dyp[C];
+      load_token_row<C, W, EXACT>(dY + row * d, gtid, nch, dyp);
+      gather_dots<C, W, B, EXACT>(g, ne, dyp, Wdt, d, gtid, nch, lane, dhv[grp], part[grp][wi]);
+    }
+    group_sync<W>(grp);
+    for (int e = gtid; e < ne; e += Cfg::GT) {
+      float s2 = dhv[grp][e];
+      if (W > 1) {
+        s2 = 0.f;
+#pragma unroll
+        for (int w = 0; w < W; ++w) s2 += part[grp][w][e];
+      }
+      const float gv = g.c[e], uv = g.c2[e];
+      hdz_ell[row * T * K + g.slot[e]] = make_float4(gv * uv, s2 * gv, fmaf(s2, uv, lambda), 0.f);
+    }
+    group_sync<W>(grp);
+  }
+}
+
+// MODE 0: dX = sum dU W_u[j] + dZ W_g[j]; 1: dX = sum dU W_u[j]; 2: dX += sum dZ W_g[j].
+template <int C, int W, bool EXACT, int MODE>
+__global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>::WARPS * 32)) ell_dx_kernel(
+    const uint16_t* __restrict__ Wu, const uint16_t* __restrict__ Wg, const uint16_t* __restrict__ count,
+    const uint8_t* __restrict__ col, int* __restrict__ plan, const float4* __restrict__ hdz_ell,
+    float* __restrict__ dX, int M, int d, int T, int K, int* __restrict__ ctr, uint32_t* status) {
+  using Cfg = TokCfg<C, W>;
+  constexpr int B = Cfg::B;
+  constexpr int B2 = MODE == 0 ? (B > 1 ? B / 2 : 1) : B;
+  __shared__ GroupSmem gs[Cfg::G];
+  __shared__ int s_next[Cfg::G];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = warp / W, wi = warp % W, gtid = wi * 32 + lane;
+  GroupSmem& g = gs[grp];
+  const int nch = d >> 3;
+  const int first = gtid;
+  int* turn = plan + kPlanHdr;
+  if (plan[3] < 0) return;
+  while (next_piece<W, false>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g, status)) {
+    const long row = g.row;
+    const int S = plan[1];
+    const int e0 = g.q * S;
+    const int ne = max(0, min(S, g.tot - e0));
+    build_list_hdz(g, row, T, K, e0, ne, gtid, Cfg::GT, col, hdz_ell, status);
+    group_sync<W>(grp);
+    float2 dx[C][4];
+    zero_acc<C>(dx);
+    if (MODE != 2) gather_axpy<C, W, B2, EXACT>(g, ne, g.c, Wu, d, first, nch, dx);
+    if (MODE != 1) gather_axpy<C, W, B2, EXACT>(g, ne, g.c2, Wg, d, first, nch, dx);
+    const int rw = g.row, q = g.q, P = g.P;
+    float* acc = dX + static_cast<long>(rw) * d;
+    if (P == 1) {
+      if (MODE == 2) add_acc<C, W, EXACT>(acc, first, nch, dx);
+      store_acc<C, W, EXACT>(acc, first, nch, dx);
+    } else {
+      turn_wait<W>(turn, rw, q, grp, gtid, status);
+      if (q > 0 || MODE == 2) add_acc<C, W, EXACT>(acc, first, nch, dx);
+      store_acc<C, W, EXACT>(acc, first, nch, dx);
+      turn_pass<W>(turn, rw, q, P, grp, gtid);
+    }
+    group_sync<W>(grp);
+  }
+}
+
 template <int C, int W, bool EXACT, typename... A>
 void launch_fwd_cw(int M, bool tiles, cudaStream_t s, A... a) {
   constexpr int threads = TokCfg<C, W>::WARPS * 32;
@@ -444,6 +677,59 @@ void launch_bwd_cw(int M, cudaStream_t s, A... a) {
                ell_bwd_kernel<C, W, EXACT><<<tok_grid(M, TokCfg<C, W>::G), threads, 0, s>>>(a...));
 }
 
+// Two-pass forward: u per slot, then Y. ctr is re-zeroed before each pass.
+template <int C, int W, bool EXACT>
+cudaError_t launch_fwd2_cw(int M, cudaStream_t s, const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
+                           const uint16_t* count, const uint16_t* val, const uint8_t* col, int* plan, float* ubuf,
+                           uint16_t* Y, int d, int T, int K, int* ctr, float* yacc, uint32_t* status) {
+  constexpr int threads = TokCfg<C, W>::WARPS * 32;
+  const int grid = tok_grid(M, TokCfg<C, W>::G);
+  cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
+  if (e != cudaSuccess) return e;
+  TWELL_LAUNCH("ell_up", s,
+               (ell_up_kernel<C, W, EXACT><<<grid, threads, 0, s>>>(X, W_u, count, val, col, plan, ubuf, M, d, T, K,
+                                                                    ctr, status)));
+  e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
+  if (e != cudaSuccess) return e;
+  TWELL_LAUNCH("ell_down", s,
+               (ell_down_kernel<C, W, EXACT><<<grid, threads, 0, s>>>(W_dt, count, val, col, plan, ubuf, Y, M, d, T,
+                                                                      K, ctr, yacc, status)));
+  return cudaGetLastError();
+}
+
+// Two- or three-pass backward: (h, dU, dZ) per slot, then dX (both weights in
+// one pass when split == 1; W_u, then W_g adding into dX, when split == 2).
+template <int C, int W, bool EXACT>
+cudaError_t launch_bwd2_cw(int M, int split, cudaStream_t s, const uint16_t* dY, const uint16_t* W_u,
+                           const uint16_t* W_g, const uint16_t* W_dt, const uint16_t* count, const uint16_t* val,
+                           const uint8_t* col, int* plan, const int* n_ovf, const float* u_ell, float lambda,
+                           float4* hdz_ell, float* dX, int d, int T, int K, int* ctr, uint32_t* status) {
+  constexpr int threads = TokCfg<C, W>::WARPS * 32;
+  const int grid = tok_grid(M, TokCfg<C, W>::G);
+  cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
+  if (e != cudaSuccess) return e;
+  TWELL_LAUNCH("ell_dh", s,
+               (ell_dh_kernel<C, W, EXACT><<<grid, threads, 0, s>>>(dY, W_dt, count, val, col, plan, n_ovf, u_ell,
+                                                                    lambda, hdz_ell, M, d, T, K, ctr, status)));
+  e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
+  if (e != cudaSuccess) return e;
+  if (split == 1) {
+    TWELL_LAUNCH("ell_dx", s,
+                 (ell_dx_kernel<C, W, EXACT, 0><<<grid, threads, 0, s>>>(W_u, W_g, count, col, plan, hdz_ell, dX, M, d,
+                                                                         T, K, ctr, status)));
+    return cudaGetLastError();
+  }
+  TWELL_LAUNCH("ell_dx", s,
+               (ell_dx_kernel<C, W, EXACT, 1><<<grid, threads, 0, s>>>(W_u, W_g, count, col, plan, hdz_ell, dX, M, d,
+                                                                       T, K, ctr, status)));
+  e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
+  if (e != cudaSuccess) return e;
+  TWELL_LAUNCH("ell_dx", s,
+               (ell_dx_kernel<C, W, EXACT, 2><<<grid, threads, 0, s>>>(W_u, W_g, count, col, plan, hdz_ell, dX, M, d,
+                                                                       T, K, ctr, status)));
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 int tok_groups(int M, int d) {
@@ -453,18 +739,36 @@ int tok_groups(int M, int d) {
   return tok_grid(M, G) * G;
 }
 
+int sparse_split_phases() { return kSplitPhases; }
+
 cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
                                const uint16_t* count, const uint16_t* val, const uint8_t* col,
-                               const uint16_t* spill, int* plan, float* u_ell, uint16_t* Y, int M, int d, int f,
-                               int K, int* ctr, float* yacc, uint32_t* status, cudaStream_t s) {
+                               const uint16_t* spill, int* plan, float* u_ell, float* ubuf, uint16_t* Y, int M, int d,
+                               int f, int K, int* ctr, float* yacc, uint32_t* status, cudaStream_t s) {
   const bool tiles = spill != nullptr;
   if (M <= 0) return cudaSuccess;
-  cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
-  if (e != cudaSuccess) return e;
   int C, W;
   tok_shape(d, C, W);
   const int T = f / kTn;
   const bool exact = d / 8 == W * 32 * C;
+  if (kSplitPhases > 0 && !tiles) {
+    float* ub = u_ell ? u_ell : ubuf;
+#define TWELL_FWD2(CC, WW)                                                                                      \
+  return exact ? launch_fwd2_cw<CC, WW, true>(M, s, X, W_u, W_dt, count, val, col, plan, ub, Y, d, T, K, ctr,    \
+                                              yacc, status)                                                     \
+               : launch_fwd2_cw<CC, WW, false>(M, s, X, W_u, W_dt, count, val, col, plan, ub, Y, d, T, K, ctr,   \
+                                               yacc, status)
+    if (W == 1 && C == 1) TWELL_FWD2(1, 1);
+    else if (W == 1 && C == 2) TWELL_FWD2(2, 1);
+    else if (W == 1 && C == 4) TWELL_FWD2(4, 1);
+    else if (W == 1) TWELL_FWD2(8, 1);
+    else if (W == 2) TWELL_FWD2(8, 2);
+    else if (W == 4) TWELL_FWD2(8, 4);
+    else TWELL_FWD2(8, 8);
+#undef TWELL_FWD2
+  }
+  cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
+  if (e != cudaSuccess) return e;
 #define TWELL_FWD(CC, WW)                                                                                   \
   (exact ? launch_fwd_cw<CC, WW, true>(M, tiles, s, X, W_u, W_dt, count, val, col, spill, plan, u_ell, Y, M, d, T, \
                                        K, ctr, yacc, status)                                                      \
@@ -487,12 +791,27 @@ cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const ui
                                float4* hdz_ell, float* dX, int M, int d, int f, int K, int* ctr, uint32_t* status,
                                cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
-  cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
-  if (e != cudaSuccess) return e;
   int C, W;
   tok_shape(d, C, W);
   const int T = f / kTn;
   const bool exact = d / 8 == W * 32 * C;
+  if (kSplitPhases > 0) {
+#define TWELL_BWD2(CC, WW)                                                                                       \
+  return exact ? launch_bwd2_cw<CC, WW, true>(M, kSplitPhases, s, dY, W_u, W_g, W_dt, count, val, col, plan,   \
+                                              n_ovf, u_ell, lambda, hdz_ell, dX, d, T, K, ctr, status)         \
+               : launch_bwd2_cw<CC, WW, false>(M, kSplitPhases, s, dY, W_u, W_g, W_dt, count, val, col, plan,  \
+                                               n_ovf, u_ell, lambda, hdz_ell, dX, d, T, K, ctr, status)
+    if (W == 1 && C == 1) TWELL_BWD2(1, 1);
+    else if (W == 1 && C == 2) TWELL_BWD2(2, 1);
+    else if (W == 1 && C == 4) TWELL_BWD2(4, 1);
+    else if (W == 1) TWELL_BWD2(8, 1);
+    else if (W == 2) TWELL_BWD2(8, 2);
+    else if (W == 4) TWELL_BWD2(8, 4);
+    else TWELL_BWD2(8, 8);
+#undef TWELL_BWD2
+  }
+  cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
+  if (e != cudaSuccess) return e;
 #define TWELL_BWD(CC, WW)                                                                                        \
   (exact ? launch_bwd_cw<CC, WW, true>(M, s, dY, W_u, W_g, W_dt, count, val, col, plan, n_ovf, u_ell, lambda,  \
                                        hdz_ell, dX, M, d, T, K, ctr, status)                                    \

@@ -89,7 +89,7 @@ struct WsLayout {
   size_t ctr = 0;   // row counter of the token kernels
   size_t yacc = 0;  // fp32 accumulator rows of rows split into several pieces
   size_t sk_partial = 0, sk_arrivals = 0;  // split-K scratch of the dense-backup GEMMs
-  size_t spill = 0, x_ovf = 0, h_ovf = 0, w_dt = 0;
+  size_t spill = 0, x_ovf = 0, h_ovf = 0, w_dt = 0, ubuf = 0;
   size_t x_rows = 0, dy_rows = 0, duz_hi = 0, h_hi = 0, db_ovf = 0, k_rows = 0;  // dense backward operands
   size_t du_ovf = 0, dz_ovf = 0, hdz_ell = 0, block_cnt = 0, unit_tot = 0, unit_ptr = 0, scan_arrive = 0, csc_row = 0,
          csc_val = 0;
@@ -117,6 +117,7 @@ WsLayout ws_layout(twell_op op, int64_t M, int64_t d, int64_t f, int64_t K, int6
     L.x_ovf = take(static_cast<size_t>(cap1 * d * 2));
     L.h_ovf = take(static_cast<size_t>(cap1 * f * 2));
     L.w_dt = take(static_cast<size_t>(f * d * 2));
+    if (sparse_split_phases() > 0) L.ubuf = take(static_cast<size_t>(M * T * K * 4));
   }
   if (op == TWELL_OP_BWD) {
     L.w_dt = take(static_cast<size_t>(f * d * 2));
@@ -309,7 +310,8 @@ twell_status ffn_fwd_impl(const uint16_t* X, const uint16_t* W_g, const uint16_t
       q8 ? launch_ell_ffn_fwd_q8(X, q8->W_u8, q8->s_u, q8->W_dt8, q8->s_d, h->count, h->val, h->col, h->row_plan,
                                  h->u_ell, Y, M, d, f, K, at<int>(ws, L.ctr), at<float>(ws, L.yacc), h->status, s)
          : launch_ell_ffn_fwd(X, W_u, wdt, h->count, h->val, h->col, tiles ? at<uint16_t>(ws, L.spill) : nullptr,
-                              h->row_plan, tiles ? nullptr : h->u_ell, Y, M, d, f, K, at<int>(ws, L.ctr),
+                              h->row_plan, tiles ? nullptr : h->u_ell,
+                              L.ubuf ? at<float>(ws, L.ubuf) : nullptr, Y, M, d, f, K, at<int>(ws, L.ctr),
                               at<float>(ws, L.yacc), h->status, s);
   if (ce != cudaSuccess) return TWELL_ECUDA;
   if (tiles) return TWELL_OK;

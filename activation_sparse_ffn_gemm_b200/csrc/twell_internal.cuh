@@ -154,10 +154,16 @@ cudaError_t launch_transpose_bf16(const uint16_t* in, int rows, int cols, uint16
 // yacc: [M][d] fp32 accumulator rows for rows split into several pieces.
 // spill: nullptr for row-level routing; for tile-level routing the dense
 // slices of tiles with more than K actives (and u_ell must be nullptr).
+// ubuf: [M][T][K] fp32 scratch for u when the two-pass schedule is built and
+// u_ell is nullptr (unused otherwise).
 cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
                                const uint16_t* count, const uint16_t* val, const uint8_t* col,
-                               const uint16_t* spill, int* plan, float* u_ell, uint16_t* Y, int M, int d, int f,
-                               int K, int* ctr, float* yacc, uint32_t* status, cudaStream_t s);
+                               const uint16_t* spill, int* plan, float* u_ell, float* ubuf, uint16_t* Y, int M, int d,
+                               int f, int K, int* ctr, float* yacc, uint32_t* status, cudaStream_t s);
+
+// Passes of the sparse kernels this library was built with: 0 fused, 1 or 2
+// two-pass (the forward then needs the ubuf scratch).
+int sparse_split_phases();
 
 // E4M3 codes of the rows of a bf16 matrix [rows][len] (len a multiple of 16),
 // one power-of-two scale per row (scale[r] = 2^e_r, e_r the smallest exponent

@@ -855,7 +855,10 @@ def bench_line(args, world, main, others):
 def kernel_table(breakdown, r, peaks, peak_src, steps, ms_step, wname):
     """Per-kernel time per step from the event trace, with the algorithmic work
     and roofline fraction of every kernel whose work is defined; and the
-    roofline object of the dominant kernel (the one with the most time)."""
+    roofline object of the dominant kernel (the one with the most time). Work
+    and time are per step: a dense-backup GEMM is launched on both GEMM engines
+    (the one that does not own the device-side row count returns at once), so
+    its per-step work is set against both launches' time."""
     M, d, f, T, K = r["shape"]
     table = {}
     for k, v in sorted(breakdown.items(), key=lambda kv: -kv[1]["ms"]):
@@ -863,8 +866,8 @@ def kernel_table(breakdown, r, peaks, peak_src, steps, ms_step, wname):
         bound, work = kernel_work(k, M, d, f, T, K, r["kept"], r["pairs"], r["n_ovf"], r["dense_wgrad"])
         if bound:
             peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) if bound == "tensor" else peaks["hbm_gbs"]
-            achieved = work / (v["ms_per_launch"] / 1e3) / (1e12 if bound == "tensor" else 1e9)
-            row.update({"bound": bound, "work_per_launch": work, "achieved": achieved,
+            achieved = work / (v["ms_per_step"] / 1e3) / (1e12 if bound == "tensor" else 1e9)
+            row.update({"bound": bound, "work_per_step": work, "achieved": achieved,
                         "unit": "TFLOP/s" if bound == "tensor" else "GB/s", "frac": achieved / peak})
         table[k] = row
     roofline = None
@@ -879,7 +882,7 @@ def kernel_table(breakdown, r, peaks, peak_src, steps, ms_step, wname):
                     "unit": row.get("unit"), "frac": row.get("frac"), "traffic": committed_traffic(top, wname),
                     "peak_source": f"{peak_src} ({'sustained bf16' if bound == 'tensor' else 'HBM copy'}, "
                                    "MEASURED_PEAKS.json)",
-                    "work_per_launch": row.get("work_per_launch"),
+                    "work_per_step": row.get("work_per_step"),
                     "share_of_step": breakdown[top]["ms_per_step"] / ms_step if ms_step else None}
     return table, roofline
 

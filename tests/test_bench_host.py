@@ -131,10 +131,13 @@ def test_kernel_table_and_dominant_kernel():
     peaks = {"hbm_gbs": 1000.0, "bf16_tflops": 2.0, "bf16_tflops_sustained": 1.0}
     r = {"shape": (128, 64, 256, 2, 8), "kept": 100, "pairs": 120, "n_ovf": 2, "dense_wgrad": 0}
     bd = {"gate_pack_gemm": {"launches": 2, "ms": 4.0, "ms_per_launch": 2.0, "ms_per_step": 2.0},
+          "ovf_up_gemm": {"launches": 4, "ms": 1.0, "ms_per_launch": 0.25, "ms_per_step": 0.5},
           "ell_updown": {"launches": 2, "ms": 1.0, "ms_per_launch": 0.5, "ms_per_step": 0.5},
           "row_flags": {"launches": 2, "ms": 0.1, "ms_per_launch": 0.05, "ms_per_step": 0.05}}
     table, roof = bench.kernel_table(bd, r, peaks, "measured", 2, 4.0, "large")
-    assert list(table) == ["gate_pack_gemm", "ell_updown", "row_flags"]
+    assert list(table) == ["gate_pack_gemm", "ovf_up_gemm", "ell_updown", "row_flags"]
+    # two launches per step (both GEMM engines): the step's work against the step's time
+    assert table["ovf_up_gemm"]["achieved"] == pytest.approx(2.0 * 2 * 64 * 256 / 0.5e-3 / 1e12)
     flops = 2.0 * 128 * 64 * 256
     assert table["gate_pack_gemm"]["achieved"] == pytest.approx(flops / 2e-3 / 1e12)
     assert table["gate_pack_gemm"]["frac"] == pytest.approx(flops / 2e-3 / 1e12 / 1.0)
