@@ -460,24 +460,66 @@ __global__ void ovf_prep_kernel(const uint16_t* __restrict__ X, const uint16_t* 
   }
 }
 
-// db_ovf[j] = sum over s < n of dZ[s][j] (hi + lo, ascending s) and
-// k_rows = n when the dense weight gradients run as GEMMs; else both 0.
-__global__ void ovf_db_kernel(const int* __restrict__ n_ovf, const int* __restrict__ plan, int cap, int f,
-                              DenseWgradOperands op, float* __restrict__ db_ovf, int* __restrict__ k_rows) {
+// db_ovf[j] = sum over s < n of dZ[s][j] (hi + lo) and k_rows = n when the
+// dense weight gradients run as GEMMs; else both 0. Two passes, each with a
+// fixed order: the rows are cut into kDbChunks ranges of ceil(cap/kDbChunks)
+// rows, each (range, 8-column group) summed by one thread in ascending row
+// order into part[range][j]; then the ranges are added in ascending order.
+constexpr int kDbChunks = 64;
+
+__device__ __forceinline__ void add_bf16x8(float (&acc)[8], uint4 hi, uint4 lo) {
+  const uint32_t h[4] = {hi.x, hi.y, hi.z, hi.w}, l[4] = {lo.x, lo.y, lo.z, lo.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    acc[2 * k] += __uint_as_float(h[k] << 16) + __uint_as_float(l[k] << 16);
+    acc[2 * k + 1] += __uint_as_float(h[k] & 0xffff0000u) + __uint_as_float(l[k] & 0xffff0000u);
+  }
+}
+
+__global__ void ovf_db_part_kernel(const int* __restrict__ n_ovf, const int* __restrict__ plan, int cap, int f,
+                                   DenseWgradOperands op, float* __restrict__ part) {
+  const bool dense = plan[3] != 0;
+  int n = dense ? n_ovf[0] : 0;
+  n = n < cap ? n : cap;
+  const int per = (cap + kDbChunks - 1) / kDbChunks;
+  const int s0 = blockIdx.y * per;
+  const int s1 = n < s0 + per ? n : s0 + per;
+  const long cap_r = dense_rows_padded(cap);
+  const int q = blockIdx.x * blockDim.x + threadIdx.x;  // 8-column group
+  if (q >= f / 8) return;
+  const uint4* hi = reinterpret_cast<const uint4*>(op.duz_hi + f) + q;
+  const uint4* lo = reinterpret_cast<const uint4*>(op.duz_hi + cap_r * 2 * f + f) + q;
+  const long rs = 2L * f / 8;  // a row of the [dU | dZ] block, in 16-byte words
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  int s = s0;
+  for (; s + 4 <= s1; s += 4) {
+    uint4 h[4], l[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      h[k] = hi[(s + k) * rs];
+      l[k] = lo[(s + k) * rs];
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) add_bf16x8(acc, h[k], l[k]);
+  }
+  for (; s < s1; ++s) add_bf16x8(acc, hi[s * rs], lo[s * rs]);
+  float4* out = reinterpret_cast<float4*>(part + static_cast<long>(blockIdx.y) * f) + 2 * q;
+  out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+}
+
+__global__ void ovf_db_sum_kernel(const int* __restrict__ n_ovf, const int* __restrict__ plan, int cap, int f,
+                                  const float* __restrict__ part, float* __restrict__ db_ovf, int* __restrict__ k_rows) {
   const bool dense = plan[3] != 0;
   int n = dense ? n_ovf[0] : 0;
   n = n < cap ? n : cap;
   if (blockIdx.x == 0 && threadIdx.x == 0) *k_rows = n;
-  const long cap_r = dense_rows_padded(cap);
-  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < f; j += gridDim.x * blockDim.x) {
-    float acc = 0.f;
-    for (int sl = 0; sl < n; ++sl) {
-      const uint16_t hi = op.duz_hi[static_cast<long>(sl) * 2 * f + f + j];
-      const uint16_t lo = op.duz_hi[(cap_r + sl) * 2 * f + f + j];
-      acc += __uint_as_float(static_cast<uint32_t>(hi) << 16) + __uint_as_float(static_cast<uint32_t>(lo) << 16);
-    }
-    db_ovf[j] = acc;
-  }
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= f) return;
+  float acc = 0.f;
+#pragma unroll 8
+  for (int c = 0; c < kDbChunks; ++c) acc += part[static_cast<long>(c) * f + j];
+  db_ovf[j] = acc;
 }
 
 }  // namespace
@@ -492,10 +534,16 @@ cudaError_t launch_ovf_prep(const uint16_t* X, const uint16_t* dY, const int* ov
   return cudaGetLastError();
 }
 
+size_t ovf_db_part_floats(int f) { return static_cast<size_t>(kDbChunks) * f; }
+
 cudaError_t launch_ovf_db(const int* n_ovf, const int* plan, int cap, int f, const DenseWgradOperands& op,
-                          float* db_ovf, int* k_rows, cudaStream_t s) {
+                          float* part, float* db_ovf, int* k_rows, cudaStream_t s) {
   if (cap <= 0) return cudaSuccess;
-  TWELL_LAUNCH("ovf_db", s, ovf_db_kernel<<<(f + 255) / 256, 256, 0, s>>>(n_ovf, plan, cap, f, op, db_ovf, k_rows));
+  TWELL_LAUNCH("ovf_db", s,
+               (ovf_db_part_kernel<<<dim3((f / 8 + 127) / 128, kDbChunks), 128, 0, s>>>(n_ovf, plan, cap, f, op,
+                                                                                       part)));
+  TWELL_LAUNCH("ovf_db", s,
+               ovf_db_sum_kernel<<<(f + 255) / 256, 256, 0, s>>>(n_ovf, plan, cap, f, part, db_ovf, k_rows));
   return cudaGetLastError();
 }
 

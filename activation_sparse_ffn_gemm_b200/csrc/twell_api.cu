@@ -90,7 +90,7 @@ struct WsLayout {
   size_t yacc = 0;  // fp32 accumulator rows of rows split into several pieces
   size_t sk_partial = 0, sk_arrivals = 0;  // split-K scratch of the dense-backup GEMMs
   size_t spill = 0, x_ovf = 0, h_ovf = 0, w_dt = 0, ubuf = 0;
-  size_t x_rows = 0, dy_rows = 0, duz_hi = 0, h_hi = 0, db_ovf = 0, k_rows = 0;  // dense backward operands
+  size_t x_rows = 0, dy_rows = 0, duz_hi = 0, h_hi = 0, db_ovf = 0, db_part = 0, k_rows = 0;  // dense backward operands
   size_t du_ovf = 0, dz_ovf = 0, hdz_ell = 0, block_cnt = 0, unit_tot = 0, unit_ptr = 0, scan_arrive = 0, csc_row = 0,
          csc_val = 0;
   size_t total = 0;
@@ -129,6 +129,7 @@ WsLayout ws_layout(twell_op op, int64_t M, int64_t d, int64_t f, int64_t K, int6
     L.du_ovf = take(static_cast<size_t>(cap1 * f * 4));
     L.dz_ovf = take(static_cast<size_t>(cap1 * f * 4));
     L.db_ovf = take(static_cast<size_t>(f * 4));
+    L.db_part = take(ovf_db_part_floats(static_cast<int>(f)) * 4);
     L.k_rows = take(64);
     L.hdz_ell = take(static_cast<size_t>(M * T * K * 16));
     const int64_t nrb = (M + kCscRows - 1) / kCscRows;
@@ -411,7 +412,7 @@ twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_
   if (launch_ovf_bwd(dw.dy_rows, wdt, W_u, W_g, h->g_ovf, h->u_ovf, lambda, h->ovf_rows, h->n_ovf, h->row_plan, cap, M,
                      d, f, dw, du_ovf, dz_ovf, dX, sk, h->status, s) != cudaSuccess)
     return TWELL_ECUDA;
-  if (launch_ovf_db(h->n_ovf, h->row_plan, cap, f, dw, db_ovf, k_rows, s) != cudaSuccess) return TWELL_ECUDA;
+  if (launch_ovf_db(h->n_ovf, h->row_plan, cap, f, dw, at<float>(ws, L.db_part), db_ovf, k_rows, s) != cudaSuccess) return TWELL_ECUDA;
   const long long nnz_cap = static_cast<long long>(M - cap) * (f / kTn) * K + static_cast<long long>(cap) * f;
   CscBuffers b{M, cap, nnz_cap, h->status, h->row_plan + kPlanHdr + M, at<int>(ws, L.block_cnt),
                at<int>(ws, L.unit_tot), at<unsigned long long>(ws, L.scan_arrive), at<int>(ws, L.unit_ptr),

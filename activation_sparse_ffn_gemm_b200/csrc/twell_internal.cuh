@@ -240,11 +240,14 @@ cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const u
                            const SplitKBuffers& sk, uint32_t* status, cudaStream_t s);
 
 // After the dense backward: column sums of dZ over the overflow rows (db_ovf,
-// hi + lo in ascending row order) and the contraction length k_rows = n of the
-// dense weight-gradient GEMMs; both 0 when the plan keeps the overflow rows on
-// the sparse path (the pair list then carries them).
+// hi + lo, in a fixed order: ascending rows within each of a fixed number of
+// row ranges, then the ranges in order) and the contraction length k_rows = n
+// of the dense weight-gradient GEMMs; both 0 when the plan keeps the overflow
+// rows on the sparse path (the pair list then carries them). part: scratch of
+// ovf_db_part_floats(f) floats.
+size_t ovf_db_part_floats(int f);
 cudaError_t launch_ovf_db(const int* n_ovf, const int* plan, int cap, int f, const DenseWgradOperands& op,
-                          float* db_ovf, int* k_rows, cudaStream_t s);
+                          float* part, float* db_ovf, int* k_rows, cudaStream_t s);
 
 // Weight gradients of the dense backup rows on the tensor cores, written
 // before the sparse kernel adds the ELL rows' sums: [dW_u ; dW_g] = [dU | dZ]^T X_ovf,
