@@ -110,6 +110,8 @@ def lib():
             L.twell_count_stats.argtypes = [ctypes.POINTER(TwellHybrid), _vp, _vp, _vp, _vp]
             L.twell_test_withhold_epilogue_arrival.restype = None
             L.twell_test_withhold_epilogue_arrival.argtypes = [ctypes.c_int]
+            L.twell_set_sparse_schedule.restype = ctypes.c_int
+            L.twell_set_sparse_schedule.argtypes = [ctypes.c_int, _i64]
             L.twell_status_read.restype = ctypes.c_int
             L.twell_status_read.argtypes = [ctypes.POINTER(TwellHybrid), ctypes.POINTER(ctypes.c_uint32),
                                             ctypes.c_int, _vp]
@@ -167,6 +169,17 @@ def test_withhold_epilogue_arrival(launches: int) -> None:
     that never reaches the split-K barrier, so its bounded wait runs out and the
     kernel sets TWELL_STATUS_TIMEOUT."""
     lib().twell_test_withhold_epilogue_arrival(int(launches))
+
+
+SCHED_AUTO, SCHED_FUSED, SCHED_PASSES = 0, 1, 2
+
+
+def set_sparse_schedule(mode: int = SCHED_AUTO, l2_budget_bytes: int = 0) -> None:
+    """Schedule of the sparse kernels (twell_set_sparse_schedule): SCHED_FUSED,
+    SCHED_PASSES (one pass per gathered weight matrix, chunked to
+    l2_budget_bytes; 0 = the library's default) or SCHED_AUTO. Process-wide;
+    the results are the same under every schedule."""
+    _check(lib().twell_set_sparse_schedule(int(mode), int(l2_budget_bytes)), "twell_set_sparse_schedule")
 
 
 def trace_enable(on: bool = True) -> None:

@@ -161,8 +161,11 @@ struct EpiTwell {
 };
 
 // The dense-backup epilogues are element-wise: apply8 handles eight columns
-// [n, n + 8) of accumulator row `row` (a valid row). run() feeds it from
-// tensor memory; the split-K reduction feeds it the summed partials.
+// [n, n + 8) of accumulator row `row` (a valid row), with the epilogue's own
+// inputs for those columns read beforehand by load8 (so that run() can have
+// the reads of a whole 32-column chunk in flight while the chunk's
+// accumulators come out of tensor memory). The split-K reduction feeds the
+// summed partials through the four-argument apply8, which reads and applies.
 template <class Epi>
 __device__ __forceinline__ void run_apply8(const typename Epi::Args& a, int m0, int n0, int M_eff, int N, int r,
                                            uint32_t taddr) {
@@ -175,6 +178,11 @@ __device__ __forceinline__ void run_apply8(const typename Epi::Args& a, int m0, 
     uint32_t v[32];
     __syncwarp();
     tmem_ld_32x32b_x32(taddr + ch * 32, v);
+    typename Epi::In in[4];
+    if (valid) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) Epi::load8(a, row, n + q * 8, in[q]);
+    }
     tmem_wait_ld();
     if (!valid) continue;
 #pragma unroll
@@ -182,10 +190,19 @@ __device__ __forceinline__ void run_apply8(const typename Epi::Args& a, int m0, 
       float acc[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[e] = __uint_as_float(v[q * 8 + e]);
-      Epi::apply8(a, row, n + q * 8, acc);
+      Epi::apply8(a, row, n + q * 8, acc, in[q]);
     }
   }
 }
+
+// The four-argument apply8 of an element-wise epilogue: its inputs, then the
+// epilogue.
+#define TWELL_APPLY8_DIRECT()                                                     \
+  __device__ static void apply8(const Args& a, int row, int n, const float (&v)[8]) { \
+    In in;                                                                           \
+    load8(a, row, n, in);                                                            \
+    apply8(a, row, n, v, in);                                                        \
+  }
 
 // ---------------------------------------- dense backup forward, first GEMM
 // u = X_ovf W_u^T (accumulator); H = bf16(g * u); u kept in fp32 when asked.
@@ -198,10 +215,16 @@ struct EpiGateMul {
   };
   static constexpr int SMEM_BYTES = 0;
   static constexpr bool kSplitK = true;
-  __device__ static void apply8(const Args& a, int row, int n, const float (&u)[8]) {
+  struct In {
+    uint4 g;
+  };
+  __device__ static void load8(const Args& a, int row, int n, In& in) {
+    in.g = __ldcs(reinterpret_cast<const uint4*>(a.g + static_cast<size_t>(row) * a.f + n));
+  }
+  __device__ static void apply8(const Args& a, int row, int n, const float (&u)[8], const In& in) {
     const size_t off = static_cast<size_t>(row) * a.f + n;
     float g8[8];
-    unpack8(*reinterpret_cast<const uint4*>(a.g + off), g8);
+    unpack8(in.g, g8);
     float h[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) h[e] = g8[e] * u[e];
@@ -213,6 +236,7 @@ struct EpiGateMul {
       up[1] = make_float4(u[4], u[5], u[6], u[7]);
     }
   }
+  TWELL_APPLY8_DIRECT()
   __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
     run_apply8<EpiGateMul>(a, m0, n0, M_eff, N, r, taddr);
   }
@@ -229,12 +253,17 @@ struct EpiScatterBf16 {
   };
   static constexpr int SMEM_BYTES = 0;
   static constexpr bool kSplitK = true;
-  __device__ static void apply8(const Args& a, int row, int n, const float (&v)[8]) {
-    const int dst = a.rows[row];
+  struct In {
+    int dst;
+  };
+  __device__ static void load8(const Args& a, int row, int, In& in) { in.dst = a.rows[row]; }
+  __device__ static void apply8(const Args& a, int, int n, const float (&v)[8], const In& in) {
+    const int dst = in.dst;
     if (!in_bounds(dst >= 0 && dst < a.rows_out, a.status)) return;
     *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(dst) * a.ld + n) =
         make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
   }
+  TWELL_APPLY8_DIRECT()
   __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
     run_apply8<EpiScatterBf16>(a, m0, n0, M_eff, N, r, taddr);
   }
@@ -250,13 +279,18 @@ struct EpiScatterF32 {
   };
   static constexpr int SMEM_BYTES = 0;
   static constexpr bool kSplitK = true;
-  __device__ static void apply8(const Args& a, int row, int n, const float (&v)[8]) {
-    const int dst = a.rows[row];
+  struct In {
+    int dst;
+  };
+  __device__ static void load8(const Args& a, int row, int, In& in) { in.dst = a.rows[row]; }
+  __device__ static void apply8(const Args& a, int, int n, const float (&v)[8], const In& in) {
+    const int dst = in.dst;
     if (!in_bounds(dst >= 0 && dst < a.rows_out, a.status)) return;
     float4* p = reinterpret_cast<float4*>(a.out + static_cast<size_t>(dst) * a.ld + n);
     p[0] = make_float4(v[0], v[1], v[2], v[3]);
     p[1] = make_float4(v[4], v[5], v[6], v[7]);
   }
+  TWELL_APPLY8_DIRECT()
   __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
     run_apply8<EpiScatterF32>(a, m0, n0, M_eff, N, r, taddr);
   }
@@ -297,13 +331,21 @@ struct EpiBwdDH {
     hi = make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]), pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
     lo = make_uint4(pack_bf16x2(l[0], l[1]), pack_bf16x2(l[2], l[3]), pack_bf16x2(l[4], l[5]), pack_bf16x2(l[6], l[7]));
   }
-  __device__ static void apply8(const Args& a, int row, int n, const float (&dh)[8]) {
+  struct In {
+    uint4 g;
+    float4 u0, u1;
+  };
+  __device__ static void load8(const Args& a, int row, int n, In& in) {
+    const size_t off = static_cast<size_t>(row) * a.f + n;
+    in.g = __ldcs(reinterpret_cast<const uint4*>(a.g + off));
+    in.u0 = __ldcs(reinterpret_cast<const float4*>(a.u + off));
+    in.u1 = __ldcs(reinterpret_cast<const float4*>(a.u + off) + 1);
+  }
+  __device__ static void apply8(const Args& a, int row, int n, const float (&dh)[8], const In& in) {
     const size_t off = static_cast<size_t>(row) * a.f + n;
     float g8[8];
-    unpack8(*reinterpret_cast<const uint4*>(a.g + off), g8);
-    const float4 u0 = reinterpret_cast<const float4*>(a.u + off)[0];
-    const float4 u1 = reinterpret_cast<const float4*>(a.u + off)[1];
-    const float u8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    unpack8(in.g, g8);
+    const float u8[8] = {in.u0.x, in.u0.y, in.u0.z, in.u0.w, in.u1.x, in.u1.y, in.u1.z, in.u1.w};
     float du[8], dz[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -335,6 +377,7 @@ struct EpiBwdDH {
       dz32[1] = make_float4(dz[4], dz[5], dz[6], dz[7]);
     }
   }
+  TWELL_APPLY8_DIRECT()
   __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
     run_apply8<EpiBwdDH>(a, m0, n0, M_eff, N, r, taddr);
   }
@@ -353,13 +396,16 @@ struct EpiStoreF32 {
   };
   static constexpr int SMEM_BYTES = 0;
   static constexpr bool kSplitK = false;
-  __device__ static void apply8(const Args& a, int row, int n, const float (&v)[8]) {
+  struct In {};
+  __device__ static void load8(const Args&, int, int, In&) {}
+  __device__ static void apply8(const Args& a, int row, int n, const float (&v)[8], const In&) {
     float* base = row < a.m_split ? a.out0 + static_cast<size_t>(row) * a.ld
                                   : a.out1 + static_cast<size_t>(row - a.m_split) * a.ld;
     float4* p = reinterpret_cast<float4*>(base + n);
     p[0] = make_float4(v[0], v[1], v[2], v[3]);
     p[1] = make_float4(v[4], v[5], v[6], v[7]);
   }
+  TWELL_APPLY8_DIRECT()
   __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
     run_apply8<EpiStoreF32>(a, m0, n0, M_eff, N, r, taddr);
   }

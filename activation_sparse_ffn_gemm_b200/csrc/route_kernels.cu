@@ -15,45 +15,20 @@ namespace twell {
 
 namespace {
 
-constexpr int kScanThreads = 1024;
-
-// row_ovf[i] = any_t(count[i][t] > K), or (dense_min > 0) the row has at
-// least dense_min active units; the row's kept entries
-// kept[i] = sum_t min(count[i][t], K), or -(1 + sum_t count[i][t]) for an
-// overflow row; one warp per row.
-// With tile-level routing no row overflows: row_ovf = 0, kept = every active unit.
-__global__ void row_flags_kernel(const uint16_t* __restrict__ count, int M, int T, int K, int dense_min, bool tiles,
-                                 uint8_t* __restrict__ row_ovf, int* __restrict__ kept) {
-  const int lane = threadIdx.x & 31;
-  const long warp0 = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const long nwarps = (static_cast<long>(gridDim.x) * blockDim.x) >> 5;
-  for (long row = warp0; row < M; row += nwarps) {
-    bool any = false;
-    int n = 0, all = 0;
-    for (int t = lane; t < T; t += 32) {
-      const int c = count[row * T + t];
-      any |= c > K;
-      n += c < K ? c : K;
-      all += c;
-    }
-    any = __any_sync(0xFFFFFFFFu, any);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      n += __shfl_xor_sync(0xFFFFFFFFu, n, o);
-      all += __shfl_xor_sync(0xFFFFFFFFu, all, o);
-    }
-    any |= dense_min > 0 && all >= dense_min;
-    if (tiles) any = false, n = all;
-    if (lane == 0) {
-      row_ovf[row] = any ? 1 : 0;
-      kept[row] = any ? -(1 + all) : n;
-    }
-  }
-}
-
-// Single block, after row_flags: the ascending list of overflow rows and the
-// row plan of the token kernels (layout in twell_internal.cuh), from the kept
-// counts parked in the turnstile words (negative for overflow rows).
+// The routing runs in three multi-block passes over fixed blocks of rows
+// (block b owns rows [b R, (b + 1) R), R = kRouteThreads * route_items(M)),
+// with per-block integer totals in the plan's scratch, so every block can
+// compute the same global values and its own offsets without a cross-block
+// wait; integer sums give the same result in any order.
+//   1. row_flags: each row's overflow flag and kept entries, and the block's
+//      totals (kept entries of ELL rows, active units and number of overflow
+//      rows);
+//   2. route_count: the piece size S from the totals, and the block's numbers
+//      of overflow rows and of pieces;
+//   3. route_write: the block's offsets from the counts of the blocks before
+//      it, then the ascending overflow list, each row's dense slot, the pieces
+//      and the plan header.
+// The plan (layout in twell_internal.cuh):
 //   * ovf_rows[0..min(n, cap)), n_ovf = {min(n, cap), n}, the capacity bit when
 //     n > cap, and row_slot[i] = the dense slot of row i (-1 when none);
 //   * pieces: S = clamp(ceil(total / groups), kPieceMin, kTokListCap);
@@ -63,23 +38,172 @@ __global__ void row_flags_kernel(const uint16_t* __restrict__ count, int M, int 
 //     model calibrated on B200 (tensor-core GEMMs over 2 n rows plus one more
 //     pass over the fp32 gradients, against two d_model-wide L2 row gathers
 //     per pair): P * 1000 > d_ff * (kDenseWgradPerRow * n + kDenseWgradFixed);
-//   * every turnstile word is left at zero.
-// Rows go in tiles of kScanThreads * kPlanItems; thread t owns kPlanItems
-// consecutive rows of a tile (read before it writes them).
-constexpr int kPlanItems = 8;
+//   * every turnstile word is left at zero (the kept counts are parked there
+//     between the passes, negative for overflow rows).
 
-__device__ __forceinline__ void load_kept(const int* kept, long r0, int M, int (&v)[kPlanItems]) {
-  if (r0 + kPlanItems <= M) {
-    const int4 a = *reinterpret_cast<const int4*>(kept + r0), b = *reinterpret_cast<const int4*>(kept + r0 + 4);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-  } else {
+struct RouteScratch {
+  long long* tot;  // [blocks][4]: kept entries of ELL rows, active units of overflow rows, overflow rows, 0
+  int* cnt;        // [blocks][2]: overflow rows, pieces
+};
+
+__device__ __forceinline__ RouteScratch route_scratch(int* plan, int M, int T, int K) {
+  const long off = plan_route_off(M, T, K);
+  return RouteScratch{reinterpret_cast<long long*>(plan + off), plan + off + 8L * kRouteBlocksMax};
+}
+
+template <typename V>
+__device__ __forceinline__ V warp_sum_v(V v) {
 #pragma unroll
-    for (int e = 0; e < kPlanItems; ++e) v[e] = r0 + e < M ? kept[r0 + e] : 0;
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+// Sum over the block of three integers (thread 0 gets the result).
+__device__ __forceinline__ void block_sum3(long long& a, long long& b, long long& c) {
+  __shared__ long long red[3][kRouteThreads / 32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  a = warp_sum_v(a);
+  b = warp_sum_v(b);
+  c = warp_sum_v(c);
+  if (lane == 0) {
+    red[0][w] = a;
+    red[1][w] = b;
+    red[2][w] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    a = b = c = 0;
+    for (int q = 0; q < kRouteThreads / 32; ++q) {
+      a += red[0][q];
+      b += red[1][q];
+      c += red[2][q];
+    }
+  }
+  __syncthreads();
+}
+
+// row_ovf[i] = any_t(count[i][t] > K), or (dense_min > 0) the row has at
+// least dense_min active units; the row's kept entries
+// kept[i] = sum_t min(count[i][t], K), or -(1 + sum_t count[i][t]) for an
+// overflow row; one warp per row. With tile-level routing no row overflows:
+// row_ovf = 0, kept = every active unit. Then the block's totals.
+__global__ void __launch_bounds__(kRouteThreads) row_flags_kernel(const uint16_t* __restrict__ count, int M, int T,
+                                                                  int K, int dense_min, bool tiles,
+                                                                  uint8_t* __restrict__ row_ovf, int* __restrict__ plan) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int* kept = plan + kPlanHdr;
+  const long R = static_cast<long>(kRouteThreads) * route_items(M);
+  const long r_begin = blockIdx.x * R;
+  const long r_end = r_begin + R < M ? r_begin + R : M;
+  long long k_tot = 0, a_ovf = 0, n_ovf = 0;
+  for (long row = r_begin + w; row < r_end; row += kRouteThreads / 32) {
+    bool any = false;
+    int n = 0, all = 0;
+    for (int t = lane; t < T; t += 32) {
+      const int c = count[row * T + t];
+      any |= c > K;
+      n += c < K ? c : K;
+      all += c;
+    }
+    any = __any_sync(0xFFFFFFFFu, any);
+    n = warp_sum_v(n);
+    all = warp_sum_v(all);
+    any |= dense_min > 0 && all >= dense_min;
+    if (tiles) any = false, n = all;
+    if (lane == 0) {
+      row_ovf[row] = any ? 1 : 0;
+      kept[row] = any ? -(1 + all) : n;
+      if (any) {
+        a_ovf += all;
+        ++n_ovf;
+      } else {
+        k_tot += n;
+      }
+    }
+  }
+  block_sum3(k_tot, a_ovf, n_ovf);
+  if (threadIdx.x == 0) {
+    long long* t = route_scratch(plan, M, T, K).tot + 4L * blockIdx.x;
+    t[0] = k_tot;
+    t[1] = a_ovf;
+    t[2] = n_ovf;
+    t[3] = 0;
   }
 }
 
-// Block-wide exclusive scan of two counts; returns the block totals.
-__device__ __forceinline__ int2 block_scan2(int a, int b, int& ea, int& eb, int2* warp_tot) {
+// The totals of all blocks (every thread gets them) and the piece size S.
+__device__ __forceinline__ int route_totals(const RouteScratch& rs, int nb, int groups, long long& total,
+                                            long long& total_ovf, long long& rows_ovf) {
+  __shared__ long long tot_s[3];
+  long long a = 0, b = 0, c = 0;
+  for (int q = threadIdx.x; q < nb; q += kRouteThreads) {
+    a += rs.tot[4L * q];
+    b += rs.tot[4L * q + 1];
+    c += rs.tot[4L * q + 2];
+  }
+  block_sum3(a, b, c);
+  if (threadIdx.x == 0) {
+    tot_s[0] = a;
+    tot_s[1] = b;
+    tot_s[2] = c;
+  }
+  __syncthreads();
+  total = tot_s[0];
+  total_ovf = tot_s[1];
+  rows_ovf = tot_s[2];
+  const long long g = groups > 0 ? groups : 1;
+  long long sz = (total + g - 1) / g;
+  sz = sz < kPieceMin ? kPieceMin : (sz > kTokListCap ? kTokListCap : sz);
+  return static_cast<int>(sz);
+}
+
+// This thread's rows [r0, r0 + items) of the block: kept counts, pieces per
+// row and the thread's numbers of overflow rows and pieces.
+template <int IT>
+__device__ __forceinline__ void thread_rows(const int* kept, long r0, long r_end, int S, int (&v)[IT], int (&P)[IT],
+                                            int& mo, int& mp) {
+  mo = mp = 0;
+#pragma unroll
+  for (int e = 0; e < IT; ++e) {
+    const bool in = r0 + e < r_end;
+    v[e] = in ? kept[r0 + e] : 0;
+    P[e] = (!in || v[e] < 0) ? 0 : (v[e] > 0 ? (v[e] + S - 1) / S : 1);
+    mo += in && v[e] < 0;
+    mp += P[e];
+  }
+}
+
+constexpr int kRouteItemsMax = 8;  // rows per thread handled in registers; more are looped
+
+__global__ void __launch_bounds__(kRouteThreads) route_count_kernel(int* __restrict__ plan, int M, int T, int K,
+                                                                    int groups) {
+  const RouteScratch rs = route_scratch(plan, M, T, K);
+  const int nb = gridDim.x;
+  long long total, total_ovf, rows_ovf;
+  const int S = route_totals(rs, nb, groups, total, total_ovf, rows_ovf);
+  const int* kept = plan + kPlanHdr;
+  const int items = route_items(M);
+  const long R = static_cast<long>(kRouteThreads) * items;
+  const long r_end = blockIdx.x * R + R < M ? blockIdx.x * R + R : M;
+  long long mo_t = 0, mp_t = 0, unused = 0;
+  for (int i0 = 0; i0 < items; i0 += kRouteItemsMax) {
+    const int n_here = items - i0 < kRouteItemsMax ? items - i0 : kRouteItemsMax;
+    const long r0 = blockIdx.x * R + static_cast<long>(kRouteThreads) * i0 + static_cast<long>(threadIdx.x) * n_here;
+    int v[kRouteItemsMax], P[kRouteItemsMax], mo, mp;
+    thread_rows<kRouteItemsMax>(kept, r0, r0 + n_here < r_end ? r0 + n_here : r_end, S, v, P, mo, mp);
+    mo_t += mo;
+    mp_t += mp;
+  }
+  block_sum3(mo_t, mp_t, unused);
+  if (threadIdx.x == 0) {
+    rs.cnt[2L * blockIdx.x] = static_cast<int>(mo_t);
+    rs.cnt[2L * blockIdx.x + 1] = static_cast<int>(mp_t);
+  }
+}
+
+// Exclusive block scan of two counts over kRouteThreads threads.
+__device__ __forceinline__ void block_scan2(int a, int b, int& ea, int& eb) {
+  __shared__ int2 warp_tot[kRouteThreads / 32];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   int ia = a, ib = b;
 #pragma unroll
@@ -92,94 +216,77 @@ __device__ __forceinline__ int2 block_scan2(int a, int b, int& ea, int& eb, int2
   }
   if (lane == 31) warp_tot[w] = make_int2(ia, ib);
   __syncthreads();
-  if (w == 0) {
-    const int2 t = warp_tot[lane];
-    int xa = t.x, xb = t.y;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int ta = __shfl_up_sync(0xFFFFFFFFu, xa, o), tb = __shfl_up_sync(0xFFFFFFFFu, xb, o);
-      if (lane >= o) {
-        xa += ta;
-        xb += tb;
-      }
-    }
-    warp_tot[lane] = make_int2(xa, xb);  // inclusive over warps
+  int2 before = make_int2(0, 0);
+  for (int q = 0; q < w; ++q) {
+    before.x += warp_tot[q].x;
+    before.y += warp_tot[q].y;
   }
-  __syncthreads();
-  const int2 before = w > 0 ? warp_tot[w - 1] : make_int2(0, 0);
   ea = before.x + ia - a;
   eb = before.y + ib - b;
-  const int2 tot = warp_tot[kScanThreads / 32 - 1];
   __syncthreads();
-  return tot;
 }
 
-__global__ void __launch_bounds__(kScanThreads) route_plan_kernel(int* __restrict__ plan, int M, int f, int groups,
-                                                                  int cap, bool tiles, int* __restrict__ ovf_rows,
-                                                                  int* __restrict__ n_ovf, uint32_t* status) {
-  __shared__ long long red[3][kScanThreads / 32];
-  __shared__ int2 warp_tot[kScanThreads / 32];
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+__global__ void __launch_bounds__(kRouteThreads) route_write_kernel(int* __restrict__ plan, int M, int T, int K,
+                                                                    int f, int groups, int cap, bool tiles,
+                                                                    int* __restrict__ ovf_rows, int* __restrict__ n_ovf,
+                                                                    uint32_t* status) {
+  const RouteScratch rs = route_scratch(plan, M, T, K);
+  const int nb = gridDim.x;
+  long long total, total_ovf, rows_ovf;
+  const int S = route_totals(rs, nb, groups, total, total_ovf, rows_ovf);
+  // offsets of this block: the counts of the blocks before it; block 0 also
+  // needs the counts of all blocks for the header
+  long long co = 0, cp = 0, ao = 0, ap = 0;
+  for (int q = threadIdx.x; q < nb; q += kRouteThreads) {
+    const long long o = rs.cnt[2L * q], pcs = rs.cnt[2L * q + 1];
+    if (q < static_cast<int>(blockIdx.x)) {
+      co += o;
+      cp += pcs;
+    }
+    ao += o;
+    ap += pcs;
+  }
+  long long unused = 0;
+  block_sum3(co, cp, unused);
+  unused = 0;
+  block_sum3(ao, ap, unused);
+  __shared__ int carry_s[4];
+  if (threadIdx.x == 0) {
+    carry_s[0] = static_cast<int>(co);
+    carry_s[1] = static_cast<int>(cp);
+    carry_s[2] = static_cast<int>(ao);
+    carry_s[3] = static_cast<int>(ap);
+  }
+  __syncthreads();
+  int carry_o = carry_s[0], carry_p = carry_s[1];
   int* kept = plan + kPlanHdr;
   int* row_slot = plan + kPlanHdr + M;
   int* pieces = plan + kPlanHdr + 2L * M;
-  constexpr long kTile = static_cast<long>(kScanThreads) * kPlanItems;
-
-  long long tot = 0, tot_ovf = 0, rows_ovf = 0;
-  for (long base = 0; base < M; base += kTile) {
-    int v[kPlanItems];
-    load_kept(kept, base + static_cast<long>(tid) * kPlanItems, M, v);
-#pragma unroll
-    for (int e = 0; e < kPlanItems; ++e) {
-      if (v[e] > 0) tot += v[e];
-      if (v[e] < 0) {
-        tot_ovf += -1LL - v[e];
-        ++rows_ovf;
-      }
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    tot += __shfl_xor_sync(0xFFFFFFFFu, tot, o);
-    tot_ovf += __shfl_xor_sync(0xFFFFFFFFu, tot_ovf, o);
-    rows_ovf += __shfl_xor_sync(0xFFFFFFFFu, rows_ovf, o);
-  }
-  if (lane == 0) {
-    red[0][w] = tot;
-    red[1][w] = tot_ovf;
-    red[2][w] = rows_ovf;
-  }
-  __syncthreads();
-  long long total = 0, total_ovf = 0, n_rows_ovf = 0;
-  for (int q = 0; q < kScanThreads / 32; ++q) {
-    total += red[0][q];
-    total_ovf += red[1][q];
-    n_rows_ovf += red[2][q];
-  }
-  const long long g = groups > 0 ? groups : 1;
-  long long sz = (total + g - 1) / g;
-  sz = sz < kPieceMin ? kPieceMin : (sz > kTokListCap ? kTokListCap : sz);
-  const int S = static_cast<int>(sz);
-
-  int carry_o = 0, carry_p = 0;
-  for (long base = 0; base < M; base += kTile) {
-    const long r0 = base + static_cast<long>(tid) * kPlanItems;
-    int v[kPlanItems], P[kPlanItems];
-    load_kept(kept, r0, M, v);
-    int mo = 0, mp = 0;
-#pragma unroll
-    for (int e = 0; e < kPlanItems; ++e) {
-      P[e] = (r0 + e >= M || v[e] < 0) ? 0 : (v[e] > 0 ? (v[e] + S - 1) / S : 1);
-      mo += r0 + e < M && v[e] < 0;
-      mp += P[e];
-    }
+  const int items = route_items(M);
+  const long R = static_cast<long>(kRouteThreads) * items;
+  const long r_end = blockIdx.x * R + R < M ? blockIdx.x * R + R : M;
+  // the block's rows in rounds of at most kRouteItemsMax consecutive rows per
+  // thread (round k: kRouteThreads * n_here rows, thread-major), so rounds in
+  // order and threads in order within a round keep ascending row order
+  for (int i0 = 0; i0 < items; i0 += kRouteItemsMax) {
+    const int n_here = items - i0 < kRouteItemsMax ? items - i0 : kRouteItemsMax;
+    const long r0 = blockIdx.x * R + static_cast<long>(kRouteThreads) * i0 + static_cast<long>(threadIdx.x) * n_here;
+    const long r1 = r0 + n_here < r_end ? r0 + n_here : r_end;
+    int v[kRouteItemsMax], P[kRouteItemsMax], mo, mp;
+    thread_rows<kRouteItemsMax>(kept, r0, r1, S, v, P, mo, mp);
     int eo, ep;
-    const int2 t = block_scan2(mo, mp, eo, ep, warp_tot);
+    block_scan2(mo, mp, eo, ep);
+    __shared__ int round_tot[2];
+    if (threadIdx.x == kRouteThreads - 1) {
+      round_tot[0] = eo + mo;
+      round_tot[1] = ep + mp;
+    }
+    __syncthreads();
     int pos = carry_o + eo, pc = carry_p + ep;
 #pragma unroll
-    for (int e = 0; e < kPlanItems; ++e) {
+    for (int e = 0; e < kRouteItemsMax; ++e) {
       const long r = r0 + e;
-      if (r >= M) continue;
+      if (r >= r1) continue;
       int slot = -1;
       if (v[e] < 0) {
         if (pos < cap) {
@@ -196,19 +303,21 @@ __global__ void __launch_bounds__(kScanThreads) route_plan_kernel(int* __restric
       row_slot[r] = slot;
       kept[r] = 0;
     }
-    carry_o += t.x;
-    carry_p += t.y;
+    carry_o += round_tot[0];
+    carry_p += round_tot[1];
+    __syncthreads();
   }
-  if (tid == 0) {
-    n_ovf[0] = carry_o < cap ? carry_o : cap;
-    n_ovf[1] = carry_o;
-    if (carry_o > cap) set_status(status, TWELL_STATUS_OVERFLOW_CAP);
-    plan[0] = carry_p;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    const int all_o = carry_s[2], all_p = carry_s[3];
+    n_ovf[0] = all_o < cap ? all_o : cap;
+    n_ovf[1] = all_o;
+    if (all_o > cap) set_status(status, TWELL_STATUS_OVERFLOW_CAP);
+    plan[0] = all_p;
     plan[1] = S;
     plan[2] = static_cast<int>(total < 0x7FFFFFFFLL ? total : 0x7FFFFFFFLL);
     plan[3] = tiles ? -1
-                    : (n_rows_ovf > 0 && total_ovf * 1000 > static_cast<long long>(f) * (kDenseWgradPerRow * n_rows_ovf +
-                                                                                         kDenseWgradFixed)
+                    : (rows_ovf > 0 && total_ovf * 1000 > static_cast<long long>(f) * (kDenseWgradPerRow * rows_ovf +
+                                                                                        kDenseWgradFixed)
                            ? 1 : 0);
   }
 }
@@ -307,14 +416,13 @@ cudaError_t launch_route(const uint16_t* count, const uint16_t* val, const uint8
                          bool tiles, uint32_t* status, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   const int T = f / kTn;
-  const int warps_needed = M;
-  int blocks = (warps_needed + 7) / 8;
-  const int max_blocks = device_sm_count() * 16;
-  if (blocks > max_blocks) blocks = max_blocks;
-  TWELL_LAUNCH("row_flags", s, row_flags_kernel<<<blocks, 256, 0, s>>>(count, M, T, K, dense_min, tiles, row_ovf,
-                                                                       plan + kPlanHdr));
+  const int nb = route_blocks(M);
+  TWELL_LAUNCH("row_flags", s,
+               row_flags_kernel<<<nb, kRouteThreads, 0, s>>>(count, M, T, K, dense_min, tiles, row_ovf, plan));
+  TWELL_LAUNCH("route_plan", s, route_count_kernel<<<nb, kRouteThreads, 0, s>>>(plan, M, T, K, groups));
   TWELL_LAUNCH("route_plan", s,
-               route_plan_kernel<<<1, kScanThreads, 0, s>>>(plan, M, f, groups, cap, tiles, ovf_rows, n_ovf, status));
+               route_write_kernel<<<nb, kRouteThreads, 0, s>>>(plan, M, T, K, f, groups, cap, tiles, ovf_rows, n_ovf,
+                                                               status));
   if (cap > 0 && !tiles) {
     int g = cap < device_sm_count() * 4 ? cap : device_sm_count() * 4;
     TWELL_LAUNCH("ovf_gather", s,

@@ -31,6 +31,7 @@ struct GroupSmem {
   int slot[kListCap];  // t * K + s (-1 for an entry read from a spilled slice)
   uint16_t tcnt[kMaxTiles];  // per-tile true counts (tile-level routing)
   int row, q, P;       // the piece being processed (re-read instead of kept live)
+  int ch;              // its chunk, for the kernels that walk the pieces once per chunk
 };
 
 template <int W>
@@ -155,16 +156,21 @@ __device__ __forceinline__ void turn_pass(int* turn, int row, int q, int P, int 
 
 // Reads piece p of the plan into the group's shared memory (row, q, P) with
 // the row's kept-entry offsets; returns false when the plan is exhausted.
+// With nchunks > 1 the pieces are handed out nchunks times, chunk by chunk
+// (item i is piece i % np of chunk i / np, in g.ch), so that every piece of
+// chunk c is claimed before any of chunk c + 1.
 template <int W, bool TILES>
 __device__ __forceinline__ bool next_piece(int* ctr, const int* plan, int M, const uint16_t* __restrict__ count, int T,
                                            int K, int grp, int wi, int lane, int* s_next, GroupSmem& g,
-                                           uint32_t* status) {
+                                           uint32_t* status, int nchunks = 1) {
   const int np = plan[0], S = plan[1];
   const int* pieces = plan + kPlanHdr + 2L * M;
-  int p, row, q;
+  int p, row, q, ch;
   for (;;) {  // a piece whose row is out of range is skipped (bounds-checked build)
-    p = static_cast<int>(next_row<W>(ctr, grp, wi, lane, s_next));
-    if (p >= np) return false;
+    const long i = next_row<W>(ctr, grp, wi, lane, s_next);
+    if (np <= 0 || i >= static_cast<long>(np) * nchunks) return false;
+    ch = static_cast<int>(i / np);
+    p = static_cast<int>(i - static_cast<long>(ch) * np);
     row = pieces[2 * p];
     q = pieces[2 * p + 1];
     if (in_bounds(row >= 0 && row < M && q >= 0, status)) break;
@@ -175,6 +181,7 @@ __device__ __forceinline__ bool next_piece(int* ctr, const int* plan, int M, con
     g.row = row;
     g.q = q;
     g.P = n > 0 ? (n + S - 1) / S : 1;
+    g.ch = ch;
   }
   group_sync<W>(grp);
   return true;

@@ -39,23 +39,19 @@
 #include "token_common.cuh"
 #include "trace.cuh"
 
+#include <algorithm>
+#include <atomic>
+#include <type_traits>
+
 // Cache hints on the token's own rows (streaming loads and stores, so the
 // gathered weight rows keep L2); 0 builds the plain loads and stores.
 #ifndef TWELL_STREAM_HINTS
 #define TWELL_STREAM_HINTS 1
 #endif
-// 0: the fused sparse kernels; 1: the two-pass forward and backward (dots, then
-// the axpy over the other weight rows); 2: as 1 with the backward's dX pass
-// split into a W_u pass and a W_g pass.
-#ifndef TWELL_SPLIT_PHASES
-#define TWELL_SPLIT_PHASES 0
-#endif
 
 namespace twell {
 
 namespace {
-
-constexpr int kSplitPhases = TWELL_SPLIT_PHASES;
 
 // acc_lo += lo(a) * lo(w), acc_hi += hi(a) * hi(w) for two bf16x2 words: the
 // mixed-precision FMA takes the bf16 halves as they are (exact in fp32) with
@@ -453,20 +449,36 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
   }
 }
 
-// ------------------------------------------------------- two-pass variants
-// The same work as ell_fwd_kernel and ell_bwd_kernel, split so that each pass
-// gathers rows of fewer weight matrices: the resident working set of gathered
-// rows (one d_model-wide row per unit and matrix) then stays closer to L2's
-// capacity when the weights are large. The forward's first pass writes u per
-// kept slot (to u_ell, or to a workspace buffer for inference) and the second
-// reads it back; the backward's first pass writes (h, dU, dZ) per slot as the
-// fused kernel does, and the dX pass (or the two passes, W_u then W_g, adding
-// into dX) reads them. Each piece is still one pass's unit of work, and the
-// pieces of a split row still add their partials in order through the row's
-// turnstile, so results do not depend on scheduling.
+// ------------------------------------------------------ multi-pass schedule
+// The work of ell_fwd_kernel and ell_bwd_kernel in passes that each gather
+// rows of one weight matrix (two for dX), walking the plan's pieces once per
+// chunk of that matrix when it is larger than the L2 budget: the up and dH
+// passes once per range of hidden tiles (each dot still over the whole
+// d_model row; an item's entries are its piece's entries in those tiles), the
+// down and dX passes once per range of d_model columns (an item gathers its
+// units' rows restricted to those columns). All of chunk c's items are
+// claimed before any of chunk c + 1's, so the gathered rows in use at a time
+// are one chunk's, which L2 holds, while the token's own rows (x, dY, the
+// per-slot records) are re-read once per chunk. Per output element the
+// arithmetic and its order are those of the one-pass kernels (the same sums
+// over the same entries, the pieces of a split row added in piece order
+// through that chunk's turnstile), so the results do not depend on the
+// schedule.
+
+// Entries [e0, e0 + ne) of the group's piece that lie in hidden-tile chunk
+// g.ch of tpc tiles.
+__device__ __forceinline__ void chunk_entries(const GroupSmem& g, int S, int T, int tpc, int& e0, int& ne) {
+  const int t0 = g.ch * tpc, t1 = t0 + tpc;
+  const int lo = t0 < T ? g.off[t0] : g.tot;
+  const int hi = t1 < T ? g.off[t1] : g.tot;
+  const int p0 = g.q * S;
+  const int p1 = min(p0 + S, g.tot);
+  e0 = max(p0, lo);
+  ne = max(0, min(p1, hi) - e0);
+}
 
 // List of entries [e0, e0 + ne) with the unit and both backward coefficients
-// (dU in c, dZ in c2) read from the per-slot record of the first pass.
+// (dU in c, dZ in c2) read from the per-slot record of the dH pass.
 __device__ __forceinline__ void build_list_hdz(GroupSmem& g, long row, int T, int K, int e0, int ne, int gtid, int GT,
                                                const uint8_t* __restrict__ col, const float4* __restrict__ hdz,
                                                uint32_t* status) {
@@ -484,11 +496,13 @@ __device__ __forceinline__ void build_list_hdz(GroupSmem& g, long row, int T, in
   }
 }
 
+// Up pass: u = x . W_u[j] per kept slot, into ubuf ([M][T][K]).
 template <int C, int W, bool EXACT>
 __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>::WARPS * 32)) ell_up_kernel(
     const uint16_t* __restrict__ X, const uint16_t* __restrict__ Wu, const uint16_t* __restrict__ count,
     const uint16_t* __restrict__ val, const uint8_t* __restrict__ col, int* __restrict__ plan,
-    float* __restrict__ ubuf, int M, int d, int T, int K, int* __restrict__ ctr, uint32_t* status) {
+    float* __restrict__ ubuf, int M, int d, int T, int K, int nhc, int tpc, int* __restrict__ ctr,
+    uint32_t* status) {
   using Cfg = TokCfg<C, W>;
   constexpr int B = Cfg::B;
   __shared__ GroupSmem gs[Cfg::G];
@@ -498,38 +512,42 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
   const int grp = warp / W, wi = warp % W, gtid = wi * 32 + lane;
   GroupSmem& g = gs[grp];
   const int nch = d >> 3;
-  while (next_piece<W, false>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g, status)) {
+  while (next_piece<W, false>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g, status, nhc)) {
     const long row = g.row;
-    const int S = plan[1];
-    const int e0 = g.q * S;
-    const int ne = max(0, min(S, g.tot - e0));
-    build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, nullptr, status);
-    group_sync<W>(grp);
-    {
-      uint4 xp[C];
-      load_token_row<C, W, EXACT>(X + row * d, gtid, nch, xp);
-      gather_dots<C, W, B, EXACT>(g, ne, xp, Wu, d, gtid, nch, lane, g.c2, part[grp][wi]);
-    }
-    group_sync<W>(grp);
-    for (int e = gtid; e < ne; e += Cfg::GT) {
-      float u = g.c2[e];
-      if (W > 1) {
-        u = 0.f;
-#pragma unroll
-        for (int w = 0; w < W; ++w) u += part[grp][w][e];
+    int e0, ne;
+    chunk_entries(g, plan[1], T, tpc, e0, ne);
+    if (ne > 0) {
+      build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, nullptr, status);
+      group_sync<W>(grp);
+      {
+        uint4 xp[C];
+        load_token_row<C, W, EXACT>(X + row * d, gtid, nch, xp);
+        gather_dots<C, W, B, EXACT>(g, ne, xp, Wu, d, gtid, nch, lane, g.c2, part[grp][wi]);
       }
-      ubuf[row * T * K + g.slot[e]] = u;
+      group_sync<W>(grp);
+      for (int e = gtid; e < ne; e += Cfg::GT) {
+        float u = g.c2[e];
+        if (W > 1) {
+          u = 0.f;
+#pragma unroll
+          for (int w = 0; w < W; ++w) u += part[grp][w][e];
+        }
+        ubuf[row * T * K + g.slot[e]] = u;
+      }
     }
-    group_sync<W>(grp);  // the group's shared memory is rewritten for the next piece
+    group_sync<W>(grp);  // the group's shared memory is rewritten for the next item
   }
 }
 
+// Down pass over columns [ch * dw, (ch + 1) * dw) of Y: Y += (g u) W_dt[j]
+// restricted to them. turn_x: [d / dw][M] turnstile words (zero before the
+// launch), or nullptr for the plan's own words when there is one chunk.
 template <int C, int W, bool EXACT>
 __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>::WARPS * 32)) ell_down_kernel(
     const uint16_t* __restrict__ Wdt, const uint16_t* __restrict__ count, const uint16_t* __restrict__ val,
     const uint8_t* __restrict__ col, int* __restrict__ plan, const float* __restrict__ ubuf,
-    uint16_t* __restrict__ Y, int M, int d, int T, int K, int* __restrict__ ctr, float* __restrict__ yacc,
-    uint32_t* status) {
+    uint16_t* __restrict__ Y, int M, int d, int T, int K, int dw, int* __restrict__ ctr, float* __restrict__ yacc,
+    int* __restrict__ turn_x, uint32_t* status) {
   using Cfg = TokCfg<C, W>;
   constexpr int B = Cfg::B;
   __shared__ GroupSmem gs[Cfg::G];
@@ -537,10 +555,8 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = warp / W, wi = warp % W, gtid = wi * 32 + lane;
   GroupSmem& g = gs[grp];
-  const int nch = d >> 3;
-  const int first = gtid;
-  int* turn = plan + kPlanHdr;
-  while (next_piece<W, false>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g, status)) {
+  const int nch = dw >> 3;
+  while (next_piece<W, false>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g, status, d / dw)) {
     const long row = g.row;
     const int S = plan[1];
     const int e0 = g.q * S;
@@ -549,30 +565,34 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
     group_sync<W>(grp);
     for (int e = gtid; e < ne; e += Cfg::GT) g.c[e] *= g.c2[e];  // h = g u
     group_sync<W>(grp);
+    const int c0 = g.ch * dw;
     float2 y[C][4];
     zero_acc<C>(y);
-    gather_axpy<C, W, B, EXACT>(g, ne, g.c, Wdt, d, first, nch, y);
+    gather_axpy<C, W, B, EXACT>(g, ne, g.c, Wdt + c0, d, gtid, nch, y);
     const int rw = g.row, q = g.q, P = g.P;
+    uint16_t* yrow = Y + static_cast<long>(rw) * d + c0;
     if (P == 1) {
-      store_y<C, W, EXACT>(Y + static_cast<long>(rw) * d, first, nch, y);
+      store_y<C, W, EXACT>(yrow, gtid, nch, y);
     } else {
-      float* acc = yacc + static_cast<long>(rw) * d;
+      int* turn = turn_x ? turn_x + static_cast<long>(g.ch) * M : plan + kPlanHdr;
+      float* acc = yacc + static_cast<long>(rw) * d + c0;
       turn_wait<W>(turn, rw, q, grp, gtid, status);
-      if (q > 0) add_acc<C, W, EXACT>(acc, first, nch, y);
-      if (q + 1 == P) store_y<C, W, EXACT>(Y + static_cast<long>(rw) * d, first, nch, y);
-      else store_acc<C, W, EXACT>(acc, first, nch, y);
+      if (q > 0) add_acc<C, W, EXACT>(acc, gtid, nch, y);
+      if (q + 1 == P) store_y<C, W, EXACT>(yrow, gtid, nch, y);
+      else store_acc<C, W, EXACT>(acc, gtid, nch, y);
       turn_pass<W>(turn, rw, q, P, grp, gtid);
     }
     group_sync<W>(grp);
   }
 }
 
+// dH pass: dH = dY . W_dt[j] per kept slot; writes (h, dU, dZ) per slot.
 template <int C, int W, bool EXACT>
 __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>::WARPS * 32)) ell_dh_kernel(
     const uint16_t* __restrict__ dY, const uint16_t* __restrict__ Wdt, const uint16_t* __restrict__ count,
     const uint16_t* __restrict__ val, const uint8_t* __restrict__ col, int* __restrict__ plan,
     const int* __restrict__ n_ovf, const float* __restrict__ u_ell, float lambda, float4* __restrict__ hdz_ell,
-    int M, int d, int T, int K, int* __restrict__ ctr, uint32_t* status) {
+    int M, int d, int T, int K, int nhc, int tpc, int* __restrict__ ctr, uint32_t* status) {
   using Cfg = TokCfg<C, W>;
   constexpr int B = Cfg::B;
   __shared__ GroupSmem gs[Cfg::G];
@@ -588,71 +608,73 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
     return;
   }
   if (blockIdx.x == 0 && threadIdx.x == 0 && n_ovf[1] > n_ovf[0]) set_status(status, TWELL_STATUS_OVERFLOW_CAP);
-  while (next_piece<W, false>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g, status)) {
+  while (next_piece<W, false>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g, status, nhc)) {
     const long row = g.row;
-    const int S = plan[1];
-    const int e0 = g.q * S;
-    const int ne = max(0, min(S, g.tot - e0));
-    build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, u_ell, status);
-    group_sync<W>(grp);
-    {
-      uint4 dyp[C];
-      load_token_row<C, W, EXACT>(dY + row * d, gtid, nch, dyp);
-      gather_dots<C, W, B, EXACT>(g, ne, dyp, Wdt, d, gtid, nch, lane, dhv[grp], part[grp][wi]);
-    }
-    group_sync<W>(grp);
-    for (int e = gtid; e < ne; e += Cfg::GT) {
-      float s2 = dhv[grp][e];
-      if (W > 1) {
-        s2 = 0.f;
-#pragma unroll
-        for (int w = 0; w < W; ++w) s2 += part[grp][w][e];
+    int e0, ne;
+    chunk_entries(g, plan[1], T, tpc, e0, ne);
+    if (ne > 0) {
+      build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, u_ell, status);
+      group_sync<W>(grp);
+      {
+        uint4 dyp[C];
+        load_token_row<C, W, EXACT>(dY + row * d, gtid, nch, dyp);
+        gather_dots<C, W, B, EXACT>(g, ne, dyp, Wdt, d, gtid, nch, lane, dhv[grp], part[grp][wi]);
       }
-      const float gv = g.c[e], uv = g.c2[e];
-      hdz_ell[row * T * K + g.slot[e]] = make_float4(gv * uv, s2 * gv, fmaf(s2, uv, lambda), 0.f);
+      group_sync<W>(grp);
+      for (int e = gtid; e < ne; e += Cfg::GT) {
+        float s2 = dhv[grp][e];
+        if (W > 1) {
+          s2 = 0.f;
+#pragma unroll
+          for (int w = 0; w < W; ++w) s2 += part[grp][w][e];
+        }
+        const float gv = g.c[e], uv = g.c2[e];
+        hdz_ell[row * T * K + g.slot[e]] = make_float4(gv * uv, s2 * gv, fmaf(s2, uv, lambda), 0.f);
+      }
     }
     group_sync<W>(grp);
   }
 }
 
-// MODE 0: dX = sum dU W_u[j] + dZ W_g[j]; 1: dX = sum dU W_u[j]; 2: dX += sum dZ W_g[j].
-template <int C, int W, bool EXACT, int MODE>
+// dX pass over columns [ch * dw, (ch + 1) * dw): dX = sum dU W_u[j] + dZ W_g[j]
+// restricted to them (fp32). turn_x as in ell_down_kernel.
+template <int C, int W, bool EXACT>
 __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>::WARPS * 32)) ell_dx_kernel(
     const uint16_t* __restrict__ Wu, const uint16_t* __restrict__ Wg, const uint16_t* __restrict__ count,
     const uint8_t* __restrict__ col, int* __restrict__ plan, const float4* __restrict__ hdz_ell,
-    float* __restrict__ dX, int M, int d, int T, int K, int* __restrict__ ctr, uint32_t* status) {
+    float* __restrict__ dX, int M, int d, int T, int K, int dw, int* __restrict__ ctr, int* __restrict__ turn_x,
+    uint32_t* status) {
   using Cfg = TokCfg<C, W>;
   constexpr int B = Cfg::B;
-  constexpr int B2 = MODE == 0 ? (B > 1 ? B / 2 : 1) : B;
+  constexpr int B2 = B > 1 ? B / 2 : 1;  // two rows (W_u, W_g) per unit
   __shared__ GroupSmem gs[Cfg::G];
   __shared__ int s_next[Cfg::G];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = warp / W, wi = warp % W, gtid = wi * 32 + lane;
   GroupSmem& g = gs[grp];
-  const int nch = d >> 3;
-  const int first = gtid;
-  int* turn = plan + kPlanHdr;
+  const int nch = dw >> 3;
   if (plan[3] < 0) return;
-  while (next_piece<W, false>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g, status)) {
+  while (next_piece<W, false>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g, status, d / dw)) {
     const long row = g.row;
     const int S = plan[1];
     const int e0 = g.q * S;
     const int ne = max(0, min(S, g.tot - e0));
     build_list_hdz(g, row, T, K, e0, ne, gtid, Cfg::GT, col, hdz_ell, status);
     group_sync<W>(grp);
+    const int c0 = g.ch * dw;
     float2 dx[C][4];
     zero_acc<C>(dx);
-    if (MODE != 2) gather_axpy<C, W, B2, EXACT>(g, ne, g.c, Wu, d, first, nch, dx);
-    if (MODE != 1) gather_axpy<C, W, B2, EXACT>(g, ne, g.c2, Wg, d, first, nch, dx);
+    gather_axpy<C, W, B2, EXACT>(g, ne, g.c, Wu + c0, d, gtid, nch, dx);
+    gather_axpy<C, W, B2, EXACT>(g, ne, g.c2, Wg + c0, d, gtid, nch, dx);
     const int rw = g.row, q = g.q, P = g.P;
-    float* acc = dX + static_cast<long>(rw) * d;
+    float* acc = dX + static_cast<long>(rw) * d + c0;
     if (P == 1) {
-      if (MODE == 2) add_acc<C, W, EXACT>(acc, first, nch, dx);
-      store_acc<C, W, EXACT>(acc, first, nch, dx);
+      store_acc<C, W, EXACT>(acc, gtid, nch, dx);
     } else {
+      int* turn = turn_x ? turn_x + static_cast<long>(g.ch) * M : plan + kPlanHdr;
       turn_wait<W>(turn, rw, q, grp, gtid, status);
-      if (q > 0 || MODE == 2) add_acc<C, W, EXACT>(acc, first, nch, dx);
-      store_acc<C, W, EXACT>(acc, first, nch, dx);
+      if (q > 0) add_acc<C, W, EXACT>(acc, gtid, nch, dx);
+      store_acc<C, W, EXACT>(acc, gtid, nch, dx);
       turn_pass<W>(turn, rw, q, P, grp, gtid);
     }
     group_sync<W>(grp);
@@ -677,57 +699,126 @@ void launch_bwd_cw(int M, cudaStream_t s, A... a) {
                ell_bwd_kernel<C, W, EXACT><<<tok_grid(M, TokCfg<C, W>::G), threads, 0, s>>>(a...));
 }
 
-// Two-pass forward: u per slot, then Y. ctr is re-zeroed before each pass.
-template <int C, int W, bool EXACT>
-cudaError_t launch_fwd2_cw(int M, cudaStream_t s, const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
-                           const uint16_t* count, const uint16_t* val, const uint8_t* col, int* plan, float* ubuf,
-                           uint16_t* Y, int d, int T, int K, int* ctr, float* yacc, uint32_t* status) {
-  constexpr int threads = TokCfg<C, W>::WARPS * 32;
-  const int grid = tok_grid(M, TokCfg<C, W>::G);
-  cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
-  if (e != cudaSuccess) return e;
-  TWELL_LAUNCH("ell_up", s,
-               (ell_up_kernel<C, W, EXACT><<<grid, threads, 0, s>>>(X, W_u, count, val, col, plan, ubuf, M, d, T, K,
-                                                                    ctr, status)));
-  e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
-  if (e != cudaSuccess) return e;
-  TWELL_LAUNCH("ell_down", s,
-               (ell_down_kernel<C, W, EXACT><<<grid, threads, 0, s>>>(W_dt, count, val, col, plan, ubuf, Y, M, d, T,
-                                                                      K, ctr, yacc, status)));
-  return cudaGetLastError();
+// Calls fn(C, W, EXACT) (as integral constants) for the token-group shape of a
+// row of w bf16.
+template <class F>
+cudaError_t with_tok_shape(int w, F&& fn) {
+  using std::integral_constant;
+  int C, W;
+  tok_shape(w, C, W);
+  const bool ex = w / 8 == W * 32 * C;
+#define TWELL_SHAPE(CC, WW)                                                                              \
+  return ex ? fn(integral_constant<int, CC>{}, integral_constant<int, WW>{}, integral_constant<bool, true>{}) \
+            : fn(integral_constant<int, CC>{}, integral_constant<int, WW>{}, integral_constant<bool, false>{})
+  if (W == 1 && C == 1) TWELL_SHAPE(1, 1);
+  if (W == 1 && C == 2) TWELL_SHAPE(2, 1);
+  if (W == 1 && C == 4) TWELL_SHAPE(4, 1);
+  if (W == 1) TWELL_SHAPE(8, 1);
+  if (W == 2) TWELL_SHAPE(8, 2);
+  if (W == 4) TWELL_SHAPE(8, 4);
+  TWELL_SHAPE(8, 8);
+#undef TWELL_SHAPE
 }
 
-// Two- or three-pass backward: (h, dU, dZ) per slot, then dX (both weights in
-// one pass when split == 1; W_u, then W_g adding into dX, when split == 2).
-template <int C, int W, bool EXACT>
-cudaError_t launch_bwd2_cw(int M, int split, cudaStream_t s, const uint16_t* dY, const uint16_t* W_u,
-                           const uint16_t* W_g, const uint16_t* W_dt, const uint16_t* count, const uint16_t* val,
-                           const uint8_t* col, int* plan, const int* n_ovf, const float* u_ell, float lambda,
-                           float4* hdz_ell, float* dX, int d, int T, int K, int* ctr, uint32_t* status) {
-  constexpr int threads = TokCfg<C, W>::WARPS * 32;
-  const int grid = tok_grid(M, TokCfg<C, W>::G);
+// Process-wide schedule of the sparse kernels (twell_set_sparse_schedule).
+std::atomic<int> g_sched_mode{TWELL_SCHED_AUTO};
+std::atomic<long long> g_l2_budget{kDefaultL2Budget};
+
+struct Chunks {
+  int nhc, tpc;  // hidden-tile chunks of the up and dH passes, tiles per chunk
+  int dw_y;      // column chunk width of the down pass
+  int dw_x;      // column chunk width of the dX pass
+};
+
+// Smallest chunk count whose share of `bytes` fits the budget: a hidden-tile
+// count (any) or a column count (a power of two dividing d / 8 and leaving at
+// least 256 columns).
+Chunks chunks_for(int d, int f, int T) {
+  const long long budget = g_l2_budget.load();
+  const long long wbytes = 2LL * d * f;
+  Chunks c{};
+  c.nhc = static_cast<int>(std::min<long long>(T, std::max<long long>(1, (wbytes + budget - 1) / budget)));
+  c.tpc = (T + c.nhc - 1) / c.nhc;
+  auto cols = [&](long long bytes) {
+    int n = 1;
+    while (bytes / n > budget && n < kMaxColChunks && (d / 8) % (2 * n) == 0 && d / (2 * n) >= 256) n *= 2;
+    return d / n;
+  };
+  c.dw_y = cols(wbytes);
+  c.dw_x = cols(2 * wbytes);
+  return c;
+}
+
+// The fused kernel gathers rows of all the direction's weights at once; the
+// passes pay for re-reading the token rows to keep fewer of them in L2. Auto:
+// passes when the three weight matrices do not fit in the device's L2.
+bool multi_pass(int d, int f) {
+  const int mode = g_sched_mode.load();
+  if (mode != TWELL_SCHED_AUTO) return mode == TWELL_SCHED_PASSES;
+  return 3LL * 2 * d * f > device_l2_bytes();
+}
+
+cudaError_t launch_fwd_passes(int M, cudaStream_t s, const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
+                              const uint16_t* count, const uint16_t* val, const uint8_t* col, int* plan, float* ubuf,
+                              uint16_t* Y, int d, int f, int K, int* ctr, float* yacc, int* turn_x,
+                              uint32_t* status) {
+  const int T = f / kTn;
+  const Chunks ch = chunks_for(d, f, T);
   cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
-  TWELL_LAUNCH("ell_dh", s,
-               (ell_dh_kernel<C, W, EXACT><<<grid, threads, 0, s>>>(dY, W_dt, count, val, col, plan, n_ovf, u_ell,
-                                                                    lambda, hdz_ell, M, d, T, K, ctr, status)));
-  e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
-  if (e != cudaSuccess) return e;
-  if (split == 1) {
-    TWELL_LAUNCH("ell_dx", s,
-                 (ell_dx_kernel<C, W, EXACT, 0><<<grid, threads, 0, s>>>(W_u, W_g, count, col, plan, hdz_ell, dX, M, d,
-                                                                         T, K, ctr, status)));
+  e = with_tok_shape(d, [&](auto cc, auto ww, auto ex) {
+    constexpr int C = decltype(cc)::value, W = decltype(ww)::value;
+    constexpr bool EX = decltype(ex)::value;
+    TWELL_LAUNCH("ell_up", s,
+                 (ell_up_kernel<C, W, EX><<<tok_grid(M, TokCfg<C, W>::G), TokCfg<C, W>::WARPS * 32, 0, s>>>(
+                     X, W_u, count, val, col, plan, ubuf, M, d, T, K, ch.nhc, ch.tpc, ctr, status)));
     return cudaGetLastError();
-  }
-  TWELL_LAUNCH("ell_dx", s,
-               (ell_dx_kernel<C, W, EXACT, 1><<<grid, threads, 0, s>>>(W_u, W_g, count, col, plan, hdz_ell, dX, M, d,
-                                                                       T, K, ctr, status)));
-  e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
+  });
   if (e != cudaSuccess) return e;
-  TWELL_LAUNCH("ell_dx", s,
-               (ell_dx_kernel<C, W, EXACT, 2><<<grid, threads, 0, s>>>(W_u, W_g, count, col, plan, hdz_ell, dX, M, d,
-                                                                       T, K, ctr, status)));
-  return cudaGetLastError();
+  const int ndc = d / ch.dw_y;
+  int* turn = ndc > 1 ? turn_x : nullptr;
+  if (turn && (e = cudaMemsetAsync(turn, 0, sizeof(int) * static_cast<size_t>(ndc) * M, s)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(ctr, 0, sizeof(int), s)) != cudaSuccess) return e;
+  return with_tok_shape(ch.dw_y, [&](auto cc, auto ww, auto ex) {
+    constexpr int C = decltype(cc)::value, W = decltype(ww)::value;
+    constexpr bool EX = decltype(ex)::value;
+    TWELL_LAUNCH("ell_down", s,
+                 (ell_down_kernel<C, W, EX><<<tok_grid(M, TokCfg<C, W>::G), TokCfg<C, W>::WARPS * 32, 0, s>>>(
+                     W_dt, count, val, col, plan, ubuf, Y, M, d, T, K, ch.dw_y, ctr, yacc, turn, status)));
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t launch_bwd_passes(int M, cudaStream_t s, const uint16_t* dY, const uint16_t* W_u, const uint16_t* W_g,
+                              const uint16_t* W_dt, const uint16_t* count, const uint16_t* val, const uint8_t* col,
+                              int* plan, const int* n_ovf, const float* u_ell, float lambda, float4* hdz_ell,
+                              float* dX, int d, int f, int K, int* ctr, int* turn_x, uint32_t* status) {
+  const int T = f / kTn;
+  const Chunks ch = chunks_for(d, f, T);
+  cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
+  if (e != cudaSuccess) return e;
+  e = with_tok_shape(d, [&](auto cc, auto ww, auto ex) {
+    constexpr int C = decltype(cc)::value, W = decltype(ww)::value;
+    constexpr bool EX = decltype(ex)::value;
+    TWELL_LAUNCH("ell_dh", s,
+                 (ell_dh_kernel<C, W, EX><<<tok_grid(M, TokCfg<C, W>::G), TokCfg<C, W>::WARPS * 32, 0, s>>>(
+                     dY, W_dt, count, val, col, plan, n_ovf, u_ell, lambda, hdz_ell, M, d, T, K, ch.nhc, ch.tpc, ctr,
+                     status)));
+    return cudaGetLastError();
+  });
+  if (e != cudaSuccess) return e;
+  const int ndc = d / ch.dw_x;
+  int* turn = ndc > 1 ? turn_x : nullptr;
+  if (turn && (e = cudaMemsetAsync(turn, 0, sizeof(int) * static_cast<size_t>(ndc) * M, s)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(ctr, 0, sizeof(int), s)) != cudaSuccess) return e;
+  return with_tok_shape(ch.dw_x, [&](auto cc, auto ww, auto ex) {
+    constexpr int C = decltype(cc)::value, W = decltype(ww)::value;
+    constexpr bool EX = decltype(ex)::value;
+    TWELL_LAUNCH("ell_dx", s,
+                 (ell_dx_kernel<C, W, EX><<<tok_grid(M, TokCfg<C, W>::G), TokCfg<C, W>::WARPS * 32, 0, s>>>(
+                     W_u, W_g, count, col, plan, hdz_ell, dX, M, d, T, K, ch.dw_x, ctr, turn, status)));
+    return cudaGetLastError();
+  });
 }
 
 }  // namespace
@@ -739,93 +830,53 @@ int tok_groups(int M, int d) {
   return tok_grid(M, G) * G;
 }
 
-int sparse_split_phases() { return kSplitPhases; }
+int set_sparse_schedule(int mode, long long l2_budget_bytes) {
+  if (mode < TWELL_SCHED_AUTO || mode > TWELL_SCHED_PASSES || l2_budget_bytes < 0) return TWELL_EINVAL;
+  g_sched_mode.store(mode);
+  g_l2_budget.store(l2_budget_bytes > 0 ? l2_budget_bytes : kDefaultL2Budget);
+  return TWELL_OK;
+}
 
 cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
                                const uint16_t* count, const uint16_t* val, const uint8_t* col,
                                const uint16_t* spill, int* plan, float* u_ell, float* ubuf, uint16_t* Y, int M, int d,
-                               int f, int K, int* ctr, float* yacc, uint32_t* status, cudaStream_t s) {
+                               int f, int K, int* ctr, float* yacc, int* turn_x, uint32_t* status, cudaStream_t s) {
   const bool tiles = spill != nullptr;
   if (M <= 0) return cudaSuccess;
-  int C, W;
-  tok_shape(d, C, W);
-  const int T = f / kTn;
-  const bool exact = d / 8 == W * 32 * C;
-  if (kSplitPhases > 0 && !tiles) {
-    float* ub = u_ell ? u_ell : ubuf;
-#define TWELL_FWD2(CC, WW)                                                                                      \
-  return exact ? launch_fwd2_cw<CC, WW, true>(M, s, X, W_u, W_dt, count, val, col, plan, ub, Y, d, T, K, ctr,    \
-                                              yacc, status)                                                     \
-               : launch_fwd2_cw<CC, WW, false>(M, s, X, W_u, W_dt, count, val, col, plan, ub, Y, d, T, K, ctr,   \
-                                               yacc, status)
-    if (W == 1 && C == 1) TWELL_FWD2(1, 1);
-    else if (W == 1 && C == 2) TWELL_FWD2(2, 1);
-    else if (W == 1 && C == 4) TWELL_FWD2(4, 1);
-    else if (W == 1) TWELL_FWD2(8, 1);
-    else if (W == 2) TWELL_FWD2(8, 2);
-    else if (W == 4) TWELL_FWD2(8, 4);
-    else TWELL_FWD2(8, 8);
-#undef TWELL_FWD2
-  }
+  if (!tiles && multi_pass(d, f))
+    return launch_fwd_passes(M, s, X, W_u, W_dt, count, val, col, plan, u_ell ? u_ell : ubuf, Y, d, f, K, ctr, yacc,
+                             turn_x, status);
   cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
-#define TWELL_FWD(CC, WW)                                                                                   \
-  (exact ? launch_fwd_cw<CC, WW, true>(M, tiles, s, X, W_u, W_dt, count, val, col, spill, plan, u_ell, Y, M, d, T, \
-                                       K, ctr, yacc, status)                                                      \
-         : launch_fwd_cw<CC, WW, false>(M, tiles, s, X, W_u, W_dt, count, val, col, spill, plan, u_ell, Y, M, d,   \
-                                        T, K, ctr, yacc, status))
-  if (W == 1 && C == 1) TWELL_FWD(1, 1);
-  else if (W == 1 && C == 2) TWELL_FWD(2, 1);
-  else if (W == 1 && C == 4) TWELL_FWD(4, 1);
-  else if (W == 1) TWELL_FWD(8, 1);
-  else if (W == 2) TWELL_FWD(8, 2);
-  else if (W == 4) TWELL_FWD(8, 4);
-  else TWELL_FWD(8, 8);
-#undef TWELL_FWD
-  return cudaGetLastError();
+  const int T = f / kTn;
+  return with_tok_shape(d, [&](auto cc, auto ww, auto ex) {
+    constexpr int C = decltype(cc)::value, W = decltype(ww)::value;
+    constexpr bool EX = decltype(ex)::value;
+    launch_fwd_cw<C, W, EX>(M, tiles, s, X, W_u, W_dt, count, val, col, spill, plan, u_ell, Y, M, d, T, K, ctr, yacc,
+                            status);
+    return cudaGetLastError();
+  });
 }
 
 cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const uint16_t* W_g,
                                const uint16_t* W_dt, const uint16_t* count, const uint16_t* val,
                                const uint8_t* col, int* plan, const int* n_ovf, const float* u_ell, float lambda,
-                               float4* hdz_ell, float* dX, int M, int d, int f, int K, int* ctr, uint32_t* status,
-                               cudaStream_t s) {
+                               float4* hdz_ell, float* dX, int M, int d, int f, int K, int* ctr, int* turn_x,
+                               uint32_t* status, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
-  int C, W;
-  tok_shape(d, C, W);
-  const int T = f / kTn;
-  const bool exact = d / 8 == W * 32 * C;
-  if (kSplitPhases > 0) {
-#define TWELL_BWD2(CC, WW)                                                                                       \
-  return exact ? launch_bwd2_cw<CC, WW, true>(M, kSplitPhases, s, dY, W_u, W_g, W_dt, count, val, col, plan,   \
-                                              n_ovf, u_ell, lambda, hdz_ell, dX, d, T, K, ctr, status)         \
-               : launch_bwd2_cw<CC, WW, false>(M, kSplitPhases, s, dY, W_u, W_g, W_dt, count, val, col, plan,  \
-                                               n_ovf, u_ell, lambda, hdz_ell, dX, d, T, K, ctr, status)
-    if (W == 1 && C == 1) TWELL_BWD2(1, 1);
-    else if (W == 1 && C == 2) TWELL_BWD2(2, 1);
-    else if (W == 1 && C == 4) TWELL_BWD2(4, 1);
-    else if (W == 1) TWELL_BWD2(8, 1);
-    else if (W == 2) TWELL_BWD2(8, 2);
-    else if (W == 4) TWELL_BWD2(8, 4);
-    else TWELL_BWD2(8, 8);
-#undef TWELL_BWD2
-  }
+  if (multi_pass(d, f))
+    return launch_bwd_passes(M, s, dY, W_u, W_g, W_dt, count, val, col, plan, n_ovf, u_ell, lambda, hdz_ell, dX, d, f,
+                             K, ctr, turn_x, status);
   cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
-#define TWELL_BWD(CC, WW)                                                                                        \
-  (exact ? launch_bwd_cw<CC, WW, true>(M, s, dY, W_u, W_g, W_dt, count, val, col, plan, n_ovf, u_ell, lambda,  \
-                                       hdz_ell, dX, M, d, T, K, ctr, status)                                    \
-         : launch_bwd_cw<CC, WW, false>(M, s, dY, W_u, W_g, W_dt, count, val, col, plan, n_ovf, u_ell, lambda, \
-                                        hdz_ell, dX, M, d, T, K, ctr, status))
-  if (W == 1 && C == 1) TWELL_BWD(1, 1);
-  else if (W == 1 && C == 2) TWELL_BWD(2, 1);
-  else if (W == 1 && C == 4) TWELL_BWD(4, 1);
-  else if (W == 1) TWELL_BWD(8, 1);
-  else if (W == 2) TWELL_BWD(8, 2);
-  else if (W == 4) TWELL_BWD(8, 4);
-  else TWELL_BWD(8, 8);
-#undef TWELL_BWD
-  return cudaGetLastError();
+  const int T = f / kTn;
+  return with_tok_shape(d, [&](auto cc, auto ww, auto ex) {
+    constexpr int C = decltype(cc)::value, W = decltype(ww)::value;
+    constexpr bool EX = decltype(ex)::value;
+    launch_bwd_cw<C, W, EX>(M, s, dY, W_u, W_g, W_dt, count, val, col, plan, n_ovf, u_ell, lambda, hdz_ell, dX, M, d,
+                            T, K, ctr, status);
+    return cudaGetLastError();
+  });
 }
 
 }  // namespace twell

@@ -24,6 +24,18 @@ int device_sm_count() {
   return v;
 }
 
+long long device_l2_bytes() {
+  static std::atomic<long long> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 126LL << 20;
+  long long v = cache[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  int b = 0;
+  v = cudaDeviceGetAttribute(&b, cudaDevAttrL2CacheSize, dev) == cudaSuccess && b > 0 ? b : 126LL << 20;
+  cache[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+
 unsigned long long next_launch_epoch() {
   static std::atomic<unsigned long long> next{1};
   constexpr unsigned long long kMask = (1ull << 56) - 1;
@@ -89,7 +101,7 @@ struct WsLayout {
   size_t ctr = 0;   // row counter of the token kernels
   size_t yacc = 0;  // fp32 accumulator rows of rows split into several pieces
   size_t sk_partial = 0, sk_arrivals = 0;  // split-K scratch of the dense-backup GEMMs
-  size_t spill = 0, x_ovf = 0, h_ovf = 0, w_dt = 0, ubuf = 0;
+  size_t spill = 0, x_ovf = 0, h_ovf = 0, w_dt = 0, ubuf = 0, turn_x = 0;
   size_t x_rows = 0, dy_rows = 0, duz_hi = 0, h_hi = 0, db_ovf = 0, db_part = 0, k_rows = 0;  // dense backward operands
   size_t du_ovf = 0, dz_ovf = 0, hdz_ell = 0, block_cnt = 0, unit_tot = 0, unit_ptr = 0, scan_arrive = 0, csc_row = 0,
          csc_val = 0;
@@ -107,6 +119,7 @@ WsLayout ws_layout(twell_op op, int64_t M, int64_t d, int64_t f, int64_t K, int6
   const int64_t T = f / kTn;
   const int64_t cap1 = cap > 0 ? cap : 1;
   if (op == TWELL_OP_FWD || op == TWELL_OP_BWD) L.ctr = take(64);
+  if (op == TWELL_OP_FWD || op == TWELL_OP_BWD) L.turn_x = take(static_cast<size_t>(kMaxColChunks) * M * 4);
   if (op == TWELL_OP_FWD) L.yacc = take(static_cast<size_t>(M * d * 4));
   if (op == TWELL_OP_FWD || op == TWELL_OP_BWD) {
     L.sk_partial = take(splitk_partial_floats(static_cast<int>(cap1), static_cast<int>(d), static_cast<int>(f)) * 4);
@@ -117,7 +130,7 @@ WsLayout ws_layout(twell_op op, int64_t M, int64_t d, int64_t f, int64_t K, int6
     L.x_ovf = take(static_cast<size_t>(cap1 * d * 2));
     L.h_ovf = take(static_cast<size_t>(cap1 * f * 2));
     L.w_dt = take(static_cast<size_t>(f * d * 2));
-    if (sparse_split_phases() > 0) L.ubuf = take(static_cast<size_t>(M * T * K * 4));
+    L.ubuf = take(static_cast<size_t>(M * T * K * 4));
   }
   if (op == TWELL_OP_BWD) {
     L.w_dt = take(static_cast<size_t>(f * d * 2));
@@ -312,8 +325,8 @@ twell_status ffn_fwd_impl(const uint16_t* X, const uint16_t* W_g, const uint16_t
                                  h->u_ell, Y, M, d, f, K, at<int>(ws, L.ctr), at<float>(ws, L.yacc), h->status, s)
          : launch_ell_ffn_fwd(X, W_u, wdt, h->count, h->val, h->col, tiles ? at<uint16_t>(ws, L.spill) : nullptr,
                               h->row_plan, tiles ? nullptr : h->u_ell,
-                              L.ubuf ? at<float>(ws, L.ubuf) : nullptr, Y, M, d, f, K, at<int>(ws, L.ctr),
-                              at<float>(ws, L.yacc), h->status, s);
+                              at<float>(ws, L.ubuf), Y, M, d, f, K, at<int>(ws, L.ctr), at<float>(ws, L.yacc),
+                              at<int>(ws, L.turn_x), h->status, s);
   if (ce != cudaSuccess) return TWELL_ECUDA;
   if (tiles) return TWELL_OK;
   const SplitKBuffers sk{at<float>(ws, L.sk_partial), at<unsigned long long>(ws, L.sk_arrivals)};
@@ -402,7 +415,8 @@ twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_
   if (launch_ovf_prep(X, dY, h->ovf_rows, h->n_ovf, h->row_plan, cap, M, d, f, dw, h->status, s) != cudaSuccess)
     return TWELL_ECUDA;
   if (launch_ell_ffn_bwd(dY, W_u, W_g, wdt, h->count, h->val, h->col, h->row_plan, h->n_ovf, h->u_ell, lambda,
-                         hdz_ell, dX, M, d, f, K, at<int>(ws, L.ctr), h->status, s) != cudaSuccess)
+                         hdz_ell, dX, M, d, f, K, at<int>(ws, L.ctr), at<int>(ws, L.turn_x), h->status,
+                         s) != cudaSuccess)
     return TWELL_ECUDA;
   float* du_ovf = at<float>(ws, L.du_ovf);
   float* dz_ovf = at<float>(ws, L.dz_ovf);
@@ -438,6 +452,10 @@ twell_status twell_count_stats(const twell_hybrid* h, int64_t* rows_by_max, int6
   if (h->dense_min < 0) return TWELL_EINVAL;
   return cuda_status(launch_count_stats(h->count, h->M, h->d_ff / kTn, h->dense_min, rows_by_max, act_by_max,
                                         tiles_by_count, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+twell_status twell_set_sparse_schedule(int mode, int64_t l2_budget_bytes) {
+  return static_cast<twell_status>(twell::set_sparse_schedule(mode, l2_budget_bytes));
 }
 
 void twell_test_withhold_epilogue_arrival(int launches) {

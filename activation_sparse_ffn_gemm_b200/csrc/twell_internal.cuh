@@ -42,9 +42,25 @@ constexpr long long kDenseWgradPerRow = TWELL_DENSE_WGRAD_PER_ROW;
 constexpr long long kDenseWgradFixed = TWELL_DENSE_WGRAD_FIXED;
 constexpr int kPieceMin = 32;
 constexpr long kPlanGroupsCap = 65536;  // bound on resident token groups of any device
-inline long plan_ints(long M, long T, long K) {
+// After the pieces, 16-byte aligned: the routing kernels' per-block scratch,
+// kRouteBlocksMax x (four int64 totals, two int32 counts). The routing runs in
+// blocks of kRouteThreads threads, each thread over route_items(M) consecutive
+// rows, so that at most kRouteBlocksMax blocks cover any M.
+constexpr int kRouteThreads = 256;
+constexpr int kRouteBlocksMax = 512;
+__host__ __device__ inline long plan_route_off(long M, long T, long K) {
   const long spill = (M * T * K + kTokListCap - 1) / kTokListCap;
-  return kPlanHdr + 2 * M + 2 * (M + (spill > kPlanGroupsCap ? spill : kPlanGroupsCap));
+  const long core = kPlanHdr + 2 * M + 2 * (M + (spill > kPlanGroupsCap ? spill : kPlanGroupsCap));
+  return (core + 3) & ~3L;
+}
+__host__ __device__ inline long plan_ints(long M, long T, long K) { return plan_route_off(M, T, K) + 10L * kRouteBlocksMax; }
+__host__ __device__ inline int route_items(long M) {
+  const long per = static_cast<long>(kRouteThreads) * kRouteBlocksMax;
+  return static_cast<int>((M + per - 1) / per > 1 ? (M + per - 1) / per : 1);
+}
+__host__ __device__ inline int route_blocks(long M) {
+  const long rb = static_cast<long>(kRouteThreads) * route_items(M);
+  return static_cast<int>((M + rb - 1) / rb);
 }
 
 // ------------------------------------------------------------ device helpers
@@ -102,6 +118,8 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
 
 // ------------------------------------------------------------ host helpers
 
+// L2 size of the current device in bytes (cached per device).
+long long device_l2_bytes();
 int device_sm_count();
 
 // Process-wide tag of one launch that counts block arrivals (1 .. 2^56 - 1,
@@ -154,16 +172,21 @@ cudaError_t launch_transpose_bf16(const uint16_t* in, int rows, int cols, uint16
 // yacc: [M][d] fp32 accumulator rows for rows split into several pieces.
 // spill: nullptr for row-level routing; for tile-level routing the dense
 // slices of tiles with more than K actives (and u_ell must be nullptr).
-// ubuf: [M][T][K] fp32 scratch for u when the two-pass schedule is built and
-// u_ell is nullptr (unused otherwise).
+// Under the multi-pass schedule (twell_set_sparse_schedule): ubuf, [M][T][K]
+// fp32 scratch for u when u_ell is nullptr; turn_x, [kMaxColChunks][M] ints of
+// turnstile scratch (both unused by the fused kernel).
 cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
                                const uint16_t* count, const uint16_t* val, const uint8_t* col,
                                const uint16_t* spill, int* plan, float* u_ell, float* ubuf, uint16_t* Y, int M, int d,
-                               int f, int K, int* ctr, float* yacc, uint32_t* status, cudaStream_t s);
+                               int f, int K, int* ctr, float* yacc, int* turn_x, uint32_t* status, cudaStream_t s);
 
-// Passes of the sparse kernels this library was built with: 0 fused, 1 or 2
-// two-pass (the forward then needs the ubuf scratch).
-int sparse_split_phases();
+// Column chunks of the multi-pass schedule at most, and the default L2 budget
+// that sizes the chunks (the gathered weight bytes one chunk may hold).
+constexpr int kMaxColChunks = 16;
+constexpr long long kDefaultL2Budget = 64LL << 20;
+
+// twell_set_sparse_schedule's implementation (mode and budget checked here).
+int set_sparse_schedule(int mode, long long l2_budget_bytes);
 
 // E4M3 codes of the rows of a bf16 matrix [rows][len] (len a multiple of 16),
 // one power-of-two scale per row (scale[r] = 2^e_r, e_r the smallest exponent
@@ -196,13 +219,14 @@ cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uin
                            cudaStream_t s);
 
 // Sparse backward over the pieces of the row plan: dH at kept actives, dU,
-// dZ, with (h = g u, dU, dZ, 0) stored per slot, and the rows of dX.
+// dZ, with (h = g u, dU, dZ, 0) stored per slot, and the rows of dX (turn_x as
+// in launch_ell_ffn_fwd).
 // Sets TWELL_STATUS_OVERFLOW_CAP when the forward flagged more overflow rows than it stored.
 cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const uint16_t* W_g,
                                const uint16_t* W_dt, const uint16_t* count, const uint16_t* val,
                                const uint8_t* col, int* plan, const int* n_ovf, const float* u_ell, float lambda,
-                               float4* hdz_ell, float* dX, int M, int d, int f, int K, int* ctr, uint32_t* status,
-                               cudaStream_t s);
+                               float4* hdz_ell, float* dX, int M, int d, int f, int K, int* ctr, int* turn_x,
+                               uint32_t* status, cudaStream_t s);
 
 // Operands of the dense backup backward and of the dense weight gradients of the
 // overflow rows, with cap_r = dense_rows_padded(cap) rows per block; for the n

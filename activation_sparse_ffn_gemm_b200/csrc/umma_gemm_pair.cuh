@@ -140,6 +140,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       k0 = (kv + kBK - 1) / kBK * kBK;
     }
     *k0_eff_s = k0;
+  }
+  __syncthreads();
+  const int M_eff = *m_eff_s;
+  const int nk0 = *k0_eff_s / kBK;
+  const int nk = nk0 + (shp.K_dev && shp.K1 > 0 ? nk0 : shp.K1 / kBK);
+  const int num_m = (M_eff + kPairBM - 1) / kPairBM;
+  const int num_n = (shp.N + kPairBN - 1) / kPairBN;
+  const int num_tiles = nk > 0 && M_eff > shp.min_rows ? num_m * num_n : 0;
+  // nothing to do (no rows, a zero K, or a row count the one-CTA engine owns):
+  // every CTA of every cluster reads the same counts and leaves here, before
+  // any barrier, tensor memory or cluster-wide step
+  if (num_tiles == 0) return;
+
+  if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -169,12 +183,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   cluster_sync_all();  // both CTAs' barriers are initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int M_eff = *m_eff_s;
-  const int nk0 = *k0_eff_s / kBK;
-  const int nk = nk0 + (shp.K_dev && shp.K1 > 0 ? nk0 : shp.K1 / kBK);
-  const int num_m = (M_eff + kPairBM - 1) / kPairBM;
-  const int num_n = (shp.N + kPairBN - 1) / kPairBN;
-  const int num_tiles = nk > 0 && M_eff > shp.min_rows ? num_m * num_n : 0;
 
   auto fail = [&]() {
     *abort_flag = 1;

@@ -295,9 +295,9 @@ def kernel_work(name, M, d, f, T, K, kept, pairs, n_ovf=0, dense_wgrad=0):
 # and the headers it compiles in); a committed DRAM capture applies only while
 # these files are unchanged.
 KERNEL_SOURCES = {
-    "gate_pack_gemm": ("gemm_kernels.cu", "umma_gemm.cuh", "sm100.cuh", "twell_internal.cuh"),
-    "ell_updown": ("token_kernels.cu", "sm100.cuh", "twell_internal.cuh"),
-    "ell_bwd": ("token_kernels.cu", "sm100.cuh", "twell_internal.cuh"),
+    "gate_pack_gemm": ("gemm_kernels.cu", "umma_gemm.cuh", "umma_gemm_pair.cuh", "sm100.cuh", "twell_internal.cuh"),
+    "ell_updown": ("token_kernels.cu", "token_common.cuh", "sm100.cuh", "twell_internal.cuh"),
+    "ell_bwd": ("token_kernels.cu", "token_common.cuh", "sm100.cuh", "twell_internal.cuh"),
     "weight_grads": ("pairlist_kernels.cu", "twell_internal.cuh"),
     "csc_fill": ("pairlist_kernels.cu", "twell_internal.cuh"),
     "transpose_wd": ("route_kernels.cu", "twell_internal.cuh"),

@@ -329,6 +329,34 @@ TWELL_API twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, con
 TWELL_API twell_status twell_count_stats(const twell_hybrid* h, int64_t* rows_by_max, int64_t* act_by_max,
                                          int64_t* tiles_by_count, twell_stream_t stream);
 
+/*
+ * Schedule of the sparse kernels of twell_ffn_fwd (row routing) and
+ * twell_ffn_bwd: a performance setting with no counterpart on the pages. The
+ * results are the same under every schedule, bit for bit.
+ *   TWELL_SCHED_FUSED   one kernel per direction: each token piece computes
+ *                       its dot products and its axpy in turn (x . W_u[j],
+ *                       then Y += h W_d[:, j]; dY . W_d[:, j], then
+ *                       dX += dU W_u[j] + dZ W_g[j]).
+ *   TWELL_SCHED_PASSES  one pass per gathered weight matrix (u per slot, then
+ *                       Y; dH, dU, dZ per slot, then dX), each pass walking
+ *                       the row plan's pieces once per chunk of its matrix of
+ *                       at most l2_budget_bytes (the up and dH passes by
+ *                       ranges of hidden tiles, the down and dX passes by
+ *                       ranges of d_model columns), so that the weight rows
+ *                       gathered at a time stay in L2 when the matrices do
+ *                       not; the token rows are re-read once per chunk.
+ *   TWELL_SCHED_AUTO    the default: TWELL_SCHED_PASSES when W_g, W_u and W_d
+ *                       together (3 d_model d_ff bf16) are larger than the
+ *                       device's L2, else TWELL_SCHED_FUSED.
+ * l2_budget_bytes: the chunk bound, 0 for the default (64 MiB).
+ * Process-wide; applies to the calls made after it returns. Tile routing
+ * (twell_ffn_fwd_tiles) and the 8-bit forward always run fused. Errors:
+ * TWELL_EINVAL for an unknown mode or a negative budget.
+ */
+typedef enum twell_sched { TWELL_SCHED_AUTO = 0, TWELL_SCHED_FUSED = 1, TWELL_SCHED_PASSES = 2 } twell_sched;
+
+TWELL_API twell_status twell_set_sparse_schedule(int mode, int64_t l2_budget_bytes);
+
 /* Copies the device status word to *out after synchronizing `stream`; clears
  * it when `clear` is non-zero. Returns TWELL_ECUDA if the copy fails. */
 TWELL_API twell_status twell_status_read(const twell_hybrid* h, uint32_t* out, int clear, twell_stream_t stream);

@@ -68,11 +68,15 @@ def test_hybrid_struct_matches_header(tw, tmp_path):
 
 def test_plan_ints(tw):
     L = tw.lib()
-    # 4 + 2 M + 2 * (M + max(65536, ceil(M * T * K / 256)))
-    assert L.twell_plan_ints(4096, 8192, 128, 8) == 4 + 2 * 4096 + 2 * (4096 + 65536)
+    # 4 + 2 M + 2 * (M + max(65536, ceil(M * T * K / 256))), rounded up to 4 ints,
+    # then the routing scratch: 512 blocks x (4 int64 + 2 int32)
+    def expect(core):
+        return (core + 3) // 4 * 4 + 512 * 10
+    assert L.twell_plan_ints(4096, 8192, 128, 8) == expect(4 + 2 * 4096 + 2 * (4096 + 65536))
     big = 65536 * 112 * 64 // 256
-    assert L.twell_plan_ints(65536, 14336, 128, 64) == 4 + 2 * 65536 + 2 * (65536 + big)
-    assert L.twell_plan_ints(0, 8192, 128, 8) == 4 + 2 * 65536
+    assert L.twell_plan_ints(65536, 14336, 128, 64) == expect(4 + 2 * 65536 + 2 * (65536 + big))
+    assert L.twell_plan_ints(0, 8192, 128, 8) == expect(4 + 2 * 65536)
+    assert L.twell_plan_ints(1, 8192, 128, 8) == expect(4 + 2 + 2 * (1 + 65536))
     assert L.twell_plan_ints(16, 8192, 64, 8) == 0
 
 
@@ -130,6 +134,13 @@ def test_host_side_errors(tw):
     assert L.twell_count_stats(ctypes.byref(hn), p, p, p, None) == 1
     assert L.twell_count_stats(ctypes.byref(bad), p, p, p, None) == 2
     assert L.twell_count_stats(None, p, p, p, None) == 1
+    # the sparse-kernel schedule: unknown modes and negative budgets are refused;
+    # the default is put back
+    assert L.twell_set_sparse_schedule(3, 0) == 1
+    assert L.twell_set_sparse_schedule(-1, 0) == 1
+    assert L.twell_set_sparse_schedule(tw.SCHED_PASSES, -5) == 1
+    assert L.twell_set_sparse_schedule(tw.SCHED_FUSED, 1 << 20) == 0
+    assert L.twell_set_sparse_schedule(tw.SCHED_AUTO, 0) == 0
 
 
 def test_missing_library_fails_loudly(tw, monkeypatch):

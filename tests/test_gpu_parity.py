@@ -212,6 +212,39 @@ def test_deterministic(tw):
         assert torch.equal(a, b)
 
 
+SCHEDULE_CASES = ("ragged", "k64", "long_rows_w2", "wide_d_w4", "heavy_small", "multi_tile", "min_d_model")
+
+
+@pytest.mark.parametrize("name", SCHEDULE_CASES)
+def test_schedules_agree_bit_for_bit(tw, name):
+    """The fused sparse kernels and the multi-pass schedule (one pass per
+    gathered weight matrix), the latter also with a 64 KiB L2 budget that cuts
+    the up and dH passes into many hidden-tile chunks and the down and dX passes
+    into column chunks: Y, the saved u and every gradient are identical, for a
+    training forward and for an inference forward (u in the workspace)."""
+    M, d, f, K, act, rs, seed = CASES[name]
+    w = Workload(name, M, d, f, 128, K, act, row_scale=rs, training=True, seed=seed)
+    D = _dev(make_inputs(w))
+    outs = {}
+    try:
+        for label, mode, budget in (("fused", tw.SCHED_FUSED, 0), ("passes", tw.SCHED_PASSES, 0),
+                                    ("chunked", tw.SCHED_PASSES, 64 << 10)):
+            tw.set_sparse_schedule(mode, budget)
+            Y, st = tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], K=K)
+            g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=1e-3)
+            Yi, sti = tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], K=K, save_for_backward=False)
+            torch.cuda.synchronize()
+            assert st.read_status() == 0 and sti.read_status() == 0, label
+            cnt = (st.count.to(torch.int32) & 0xFFFF).clamp(max=K)
+            kept = (torch.arange(K, device=cnt.device) < cnt[..., None]) & (st.row_ovf[:M] == 0)[:, None, None]
+            outs[label] = [Y, st.u_ell[kept], Yi] + [g[k] for k in sorted(g)]
+    finally:
+        tw.set_sparse_schedule(tw.SCHED_AUTO, 0)
+    for label in ("passes", "chunked"):
+        for a, b in zip(outs["fused"], outs[label]):
+            assert torch.equal(a, b), label
+
+
 def test_prepared_wdt_matches(tw):
     w = Workload("wdt", 256, 512, 1024, 128, 8, 0.03, training=True, seed=12)
     D = _dev(make_inputs(w))
