@@ -85,49 +85,62 @@ __device__ __forceinline__ void block_sum3(long long& a, long long& b, long long
 // row_ovf[i] = any_t(count[i][t] > K), or (dense_min > 0) the row has at
 // least dense_min active units; the row's kept entries
 // kept[i] = sum_t min(count[i][t], K), or -(1 + sum_t count[i][t]) for an
-// overflow row; one warp per row. With tile-level routing no row overflows:
-// row_ovf = 0, kept = every active unit. Then the block's totals.
+// overflow row; one warp per row, eight consecutive rows per block and
+// iteration. With tile-level routing no row overflows: row_ovf = 0, kept =
+// every active unit. The eight rows' totals are added (integer atomics, so
+// in any order) to those of the routing block that owns them, zeroed before
+// the launch.
 __global__ void __launch_bounds__(kRouteThreads) row_flags_kernel(const uint16_t* __restrict__ count, int M, int T,
                                                                   int K, int dense_min, bool tiles,
                                                                   uint8_t* __restrict__ row_ovf, int* __restrict__ plan) {
+  __shared__ long long part[3][kRouteThreads / 32];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  constexpr int kRows = kRouteThreads / 32;
   int* kept = plan + kPlanHdr;
+  long long* tot = route_scratch(plan, M, T, K).tot;
   const long R = static_cast<long>(kRouteThreads) * route_items(M);
-  const long r_begin = blockIdx.x * R;
-  const long r_end = r_begin + R < M ? r_begin + R : M;
-  long long k_tot = 0, a_ovf = 0, n_ovf = 0;
-  for (long row = r_begin + w; row < r_end; row += kRouteThreads / 32) {
-    bool any = false;
-    int n = 0, all = 0;
-    for (int t = lane; t < T; t += 32) {
-      const int c = count[row * T + t];
-      any |= c > K;
-      n += c < K ? c : K;
-      all += c;
-    }
-    any = __any_sync(0xFFFFFFFFu, any);
-    n = warp_sum_v(n);
-    all = warp_sum_v(all);
-    any |= dense_min > 0 && all >= dense_min;
-    if (tiles) any = false, n = all;
-    if (lane == 0) {
-      row_ovf[row] = any ? 1 : 0;
-      kept[row] = any ? -(1 + all) : n;
+  for (long base = static_cast<long>(blockIdx.x) * kRows; base < M; base += static_cast<long>(gridDim.x) * kRows) {
+    const long row = base + w;
+    long long k_tot = 0, a_ovf = 0, n_ovf = 0;
+    if (row < M) {
+      bool any = false;
+      int n = 0, all = 0;
+      for (int t = lane; t < T; t += 32) {
+        const int c = count[row * T + t];
+        any |= c > K;
+        n += c < K ? c : K;
+        all += c;
+      }
+      any = __any_sync(0xFFFFFFFFu, any);
+      n = warp_sum_v(n);
+      all = warp_sum_v(all);
+      any |= dense_min > 0 && all >= dense_min;
+      if (tiles) any = false, n = all;
+      if (lane == 0) {
+        row_ovf[row] = any ? 1 : 0;
+        kept[row] = any ? -(1 + all) : n;
+      }
       if (any) {
-        a_ovf += all;
-        ++n_ovf;
+        a_ovf = all;
+        n_ovf = 1;
       } else {
-        k_tot += n;
+        k_tot = n;
       }
     }
-  }
-  block_sum3(k_tot, a_ovf, n_ovf);
-  if (threadIdx.x == 0) {
-    long long* t = route_scratch(plan, M, T, K).tot + 4L * blockIdx.x;
-    t[0] = k_tot;
-    t[1] = a_ovf;
-    t[2] = n_ovf;
-    t[3] = 0;
+    if (lane == 0) {
+      part[0][w] = k_tot;
+      part[1][w] = a_ovf;
+      part[2][w] = n_ovf;
+    }
+    __syncthreads();
+    if (threadIdx.x < 3) {  // the eight rows share one routing block (R is a multiple of eight)
+      long long v = 0;
+      for (int q = 0; q < kRows; ++q) v += part[threadIdx.x][q];
+      if (v != 0)
+        atomicAdd(reinterpret_cast<unsigned long long*>(tot + 4 * (base / R) + threadIdx.x),
+                  static_cast<unsigned long long>(v));
+    }
+    __syncthreads();
   }
 }
 
@@ -417,8 +430,12 @@ cudaError_t launch_route(const uint16_t* count, const uint16_t* val, const uint8
   if (M <= 0) return cudaSuccess;
   const int T = f / kTn;
   const int nb = route_blocks(M);
+  cudaError_t e = cudaMemsetAsync(plan + plan_route_off(M, T, K), 0, sizeof(long long) * 4 * nb, s);
+  if (e != cudaSuccess) return e;
+  int fb = static_cast<int>((M + kRouteThreads / 32 - 1) / (kRouteThreads / 32));
+  if (fb > device_sm_count() * 8) fb = device_sm_count() * 8;
   TWELL_LAUNCH("row_flags", s,
-               row_flags_kernel<<<nb, kRouteThreads, 0, s>>>(count, M, T, K, dense_min, tiles, row_ovf, plan));
+               row_flags_kernel<<<fb, kRouteThreads, 0, s>>>(count, M, T, K, dense_min, tiles, row_ovf, plan));
   TWELL_LAUNCH("route_plan", s, route_count_kernel<<<nb, kRouteThreads, 0, s>>>(plan, M, T, K, groups));
   TWELL_LAUNCH("route_plan", s,
                route_write_kernel<<<nb, kRouteThreads, 0, s>>>(plan, M, T, K, f, groups, cap, tiles, ovf_rows, n_ovf,

@@ -450,6 +450,28 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
 }
 
 // ------------------------------------------------------ multi-pass schedule
+#ifndef TWELL_PASS_THREADS_PER_SM
+#define TWELL_PASS_THREADS_PER_SM 512
+#endif
+// Threads per SM the pass kernels are built and launched for (registers per
+// thread are capped accordingly): 512 (at most 128 registers) for the dot
+// passes and the down pass, whose wider rows need the registers, and 1024 for
+// the dX pass over column chunks of at most 1024 (measured: 15% faster there,
+// slower for the others, which then spill).
+constexpr int kPassThreadsPerSM = TWELL_PASS_THREADS_PER_SM;
+template <int C>
+constexpr int dx_threads_per_sm() {
+  return C <= 4 ? 2 * TWELL_PASS_THREADS_PER_SM : TWELL_PASS_THREADS_PER_SM;  // C = 8 would spill at 64 registers
+}
+
+// Grid of a pass kernel: enough CTAs for the rows, at most the resident ones.
+inline int pass_grid(int M, int G, int warps, int threads_per_sm = kPassThreadsPerSM) {
+  const long need = (static_cast<long>(M) + G - 1) / G;
+  const int per_sm = threads_per_sm / (warps * 32) > 0 ? threads_per_sm / (warps * 32) : 1;
+  const long cap = static_cast<long>(device_sm_count()) * per_sm;
+  return static_cast<int>(need < cap ? need : cap);
+}
+
 // The work of ell_fwd_kernel and ell_bwd_kernel in passes that each gather
 // rows of one weight matrix (two for dX), walking the plan's pieces once per
 // chunk of that matrix when it is larger than the L2 budget: the up and dH
@@ -498,7 +520,7 @@ __device__ __forceinline__ void build_list_hdz(GroupSmem& g, long row, int T, in
 
 // Up pass: u = x . W_u[j] per kept slot, into ubuf ([M][T][K]).
 template <int C, int W, bool EXACT>
-__global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>::WARPS * 32)) ell_up_kernel(
+__global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, kPassThreadsPerSM / (TokCfg<C, W>::WARPS * 32)) ell_up_kernel(
     const uint16_t* __restrict__ X, const uint16_t* __restrict__ Wu, const uint16_t* __restrict__ count,
     const uint16_t* __restrict__ val, const uint8_t* __restrict__ col, int* __restrict__ plan,
     float* __restrict__ ubuf, int M, int d, int T, int K, int nhc, int tpc, int* __restrict__ ctr,
@@ -543,7 +565,7 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
 // restricted to them. turn_x: [d / dw][M] turnstile words (zero before the
 // launch), or nullptr for the plan's own words when there is one chunk.
 template <int C, int W, bool EXACT>
-__global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>::WARPS * 32)) ell_down_kernel(
+__global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, kPassThreadsPerSM / (TokCfg<C, W>::WARPS * 32)) ell_down_kernel(
     const uint16_t* __restrict__ Wdt, const uint16_t* __restrict__ count, const uint16_t* __restrict__ val,
     const uint8_t* __restrict__ col, int* __restrict__ plan, const float* __restrict__ ubuf,
     uint16_t* __restrict__ Y, int M, int d, int T, int K, int dw, int* __restrict__ ctr, float* __restrict__ yacc,
@@ -588,7 +610,7 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
 
 // dH pass: dH = dY . W_dt[j] per kept slot; writes (h, dU, dZ) per slot.
 template <int C, int W, bool EXACT>
-__global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>::WARPS * 32)) ell_dh_kernel(
+__global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, kPassThreadsPerSM / (TokCfg<C, W>::WARPS * 32)) ell_dh_kernel(
     const uint16_t* __restrict__ dY, const uint16_t* __restrict__ Wdt, const uint16_t* __restrict__ count,
     const uint16_t* __restrict__ val, const uint8_t* __restrict__ col, int* __restrict__ plan,
     const int* __restrict__ n_ovf, const float* __restrict__ u_ell, float lambda, float4* __restrict__ hdz_ell,
@@ -639,7 +661,8 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
 // dX pass over columns [ch * dw, (ch + 1) * dw): dX = sum dU W_u[j] + dZ W_g[j]
 // restricted to them (fp32). turn_x as in ell_down_kernel.
 template <int C, int W, bool EXACT>
-__global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>::WARPS * 32)) ell_dx_kernel(
+__global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, dx_threads_per_sm<C>() / (TokCfg<C, W>::WARPS * 32))
+    ell_dx_kernel(
     const uint16_t* __restrict__ Wu, const uint16_t* __restrict__ Wg, const uint16_t* __restrict__ count,
     const uint8_t* __restrict__ col, int* __restrict__ plan, const float4* __restrict__ hdz_ell,
     float* __restrict__ dX, int M, int d, int T, int K, int dw, int* __restrict__ ctr, int* __restrict__ turn_x,
@@ -750,12 +773,18 @@ Chunks chunks_for(int d, int f, int T) {
 }
 
 // The fused kernel gathers rows of all the direction's weights at once; the
-// passes pay for re-reading the token rows to keep fewer of them in L2. Auto:
-// passes when the three weight matrices do not fit in the device's L2.
-bool multi_pass(int d, int f) {
+// passes pay for re-reading the token rows to keep fewer of them in L2, which
+// helps only when the weights are larger than L2 and the batch gathers each
+// weight row many times. Auto: passes when the three weight matrices do not
+// fit in the device's L2 and the batch has at least kPassesMinRows rows
+// (measured at d_model=4096, d_ff=14336, 99% sparsity: fused is faster at
+// M=512 and 2048, the passes from M=4096 on).
+constexpr int kPassesMinRows = 4096;
+
+bool multi_pass(int M, int d, int f) {
   const int mode = g_sched_mode.load();
   if (mode != TWELL_SCHED_AUTO) return mode == TWELL_SCHED_PASSES;
-  return 3LL * 2 * d * f > device_l2_bytes();
+  return 3LL * 2 * d * f > device_l2_bytes() && M >= kPassesMinRows;
 }
 
 cudaError_t launch_fwd_passes(int M, cudaStream_t s, const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
@@ -770,7 +799,7 @@ cudaError_t launch_fwd_passes(int M, cudaStream_t s, const uint16_t* X, const ui
     constexpr int C = decltype(cc)::value, W = decltype(ww)::value;
     constexpr bool EX = decltype(ex)::value;
     TWELL_LAUNCH("ell_up", s,
-                 (ell_up_kernel<C, W, EX><<<tok_grid(M, TokCfg<C, W>::G), TokCfg<C, W>::WARPS * 32, 0, s>>>(
+                 (ell_up_kernel<C, W, EX><<<pass_grid(M, TokCfg<C, W>::G, TokCfg<C, W>::WARPS), TokCfg<C, W>::WARPS * 32, 0, s>>>(
                      X, W_u, count, val, col, plan, ubuf, M, d, T, K, ch.nhc, ch.tpc, ctr, status)));
     return cudaGetLastError();
   });
@@ -783,7 +812,7 @@ cudaError_t launch_fwd_passes(int M, cudaStream_t s, const uint16_t* X, const ui
     constexpr int C = decltype(cc)::value, W = decltype(ww)::value;
     constexpr bool EX = decltype(ex)::value;
     TWELL_LAUNCH("ell_down", s,
-                 (ell_down_kernel<C, W, EX><<<tok_grid(M, TokCfg<C, W>::G), TokCfg<C, W>::WARPS * 32, 0, s>>>(
+                 (ell_down_kernel<C, W, EX><<<pass_grid(M, TokCfg<C, W>::G, TokCfg<C, W>::WARPS), TokCfg<C, W>::WARPS * 32, 0, s>>>(
                      W_dt, count, val, col, plan, ubuf, Y, M, d, T, K, ch.dw_y, ctr, yacc, turn, status)));
     return cudaGetLastError();
   });
@@ -801,7 +830,7 @@ cudaError_t launch_bwd_passes(int M, cudaStream_t s, const uint16_t* dY, const u
     constexpr int C = decltype(cc)::value, W = decltype(ww)::value;
     constexpr bool EX = decltype(ex)::value;
     TWELL_LAUNCH("ell_dh", s,
-                 (ell_dh_kernel<C, W, EX><<<tok_grid(M, TokCfg<C, W>::G), TokCfg<C, W>::WARPS * 32, 0, s>>>(
+                 (ell_dh_kernel<C, W, EX><<<pass_grid(M, TokCfg<C, W>::G, TokCfg<C, W>::WARPS), TokCfg<C, W>::WARPS * 32, 0, s>>>(
                      dY, W_dt, count, val, col, plan, n_ovf, u_ell, lambda, hdz_ell, M, d, T, K, ch.nhc, ch.tpc, ctr,
                      status)));
     return cudaGetLastError();
@@ -815,7 +844,8 @@ cudaError_t launch_bwd_passes(int M, cudaStream_t s, const uint16_t* dY, const u
     constexpr int C = decltype(cc)::value, W = decltype(ww)::value;
     constexpr bool EX = decltype(ex)::value;
     TWELL_LAUNCH("ell_dx", s,
-                 (ell_dx_kernel<C, W, EX><<<tok_grid(M, TokCfg<C, W>::G), TokCfg<C, W>::WARPS * 32, 0, s>>>(
+                 (ell_dx_kernel<C, W, EX><<<pass_grid(M, TokCfg<C, W>::G, TokCfg<C, W>::WARPS, dx_threads_per_sm<C>()),
+                                            TokCfg<C, W>::WARPS * 32, 0, s>>>(
                      W_u, W_g, count, col, plan, hdz_ell, dX, M, d, T, K, ch.dw_x, ctr, turn, status)));
     return cudaGetLastError();
   });
@@ -843,7 +873,7 @@ cudaError_t launch_ell_ffn_fwd(const uint16_t* X, const uint16_t* W_u, const uin
                                int f, int K, int* ctr, float* yacc, int* turn_x, uint32_t* status, cudaStream_t s) {
   const bool tiles = spill != nullptr;
   if (M <= 0) return cudaSuccess;
-  if (!tiles && multi_pass(d, f))
+  if (!tiles && multi_pass(M, d, f))
     return launch_fwd_passes(M, s, X, W_u, W_dt, count, val, col, plan, u_ell ? u_ell : ubuf, Y, d, f, K, ctr, yacc,
                              turn_x, status);
   cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
@@ -864,7 +894,7 @@ cudaError_t launch_ell_ffn_bwd(const uint16_t* dY, const uint16_t* W_u, const ui
                                float4* hdz_ell, float* dX, int M, int d, int f, int K, int* ctr, int* turn_x,
                                uint32_t* status, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
-  if (multi_pass(d, f))
+  if (multi_pass(M, d, f))
     return launch_bwd_passes(M, s, dY, W_u, W_g, W_dt, count, val, col, plan, n_ovf, u_ell, lambda, hdz_ell, dX, d, f,
                              K, ctr, turn_x, status);
   cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);

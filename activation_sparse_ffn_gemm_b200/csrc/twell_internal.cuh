@@ -40,7 +40,10 @@ constexpr int kPlanHdr = 4;
 #endif
 constexpr long long kDenseWgradPerRow = TWELL_DENSE_WGRAD_PER_ROW;
 constexpr long long kDenseWgradFixed = TWELL_DENSE_WGRAD_FIXED;
-constexpr int kPieceMin = 32;
+#ifndef TWELL_PIECE_MIN
+#define TWELL_PIECE_MIN 32
+#endif
+constexpr int kPieceMin = TWELL_PIECE_MIN;
 constexpr long kPlanGroupsCap = 65536;  // bound on resident token groups of any device
 // After the pieces, 16-byte aligned: the routing kernels' per-block scratch,
 // kRouteBlocksMax x (four int64 totals, two int32 counts). The routing runs in

@@ -39,7 +39,10 @@ namespace twell {
 constexpr int kBM = 128;
 constexpr int kBK = 64;  // 64 bf16 = 128 bytes: one swizzle row
 constexpr int kGemmThreads = 192;
-constexpr int kGroupM = 16;
+#ifndef TWELL_GROUP_M
+#define TWELL_GROUP_M 16
+#endif
+constexpr int kGroupM = TWELL_GROUP_M;  // M tiles per raster group (their A panels stay in L2)
 
 struct GemmShape {
   int M;             // static bound on rows of A / C

@@ -67,7 +67,7 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--no-trace", action="store_true")
-    p.add_argument("--workload", default=MAIN_WORKLOAD, choices=["large", "train", "heavy"],
+    p.add_argument("--workload", default=MAIN_WORKLOAD, choices=["large", "sweep8k", "train", "heavy"],
                    help="workload of the timed training step (synthetic.WORKLOADS)")
     p.add_argument("--no-extra", action="store_true", help="skip the two smaller workloads of the line")
     p.add_argument("--step-only", action="store_true",
@@ -82,7 +82,19 @@ def parse_args():
     p.add_argument("--sweep-k", default="",
                    help="with --sweep: time every K of this list at each point (e.g. 8,16,32,64) next to the "
                         "K chosen from the count statistics")
+    p.add_argument("--sched", default="auto", choices=["auto", "fused", "passes"],
+                   help="schedule of the sparse kernels (twell_set_sparse_schedule)")
+    p.add_argument("--l2-budget-mib", type=int, default=0,
+                   help="L2 budget of one chunk of the multi-pass schedule, MiB (0: the library default)")
     return p.parse_args()
+
+
+def apply_schedule(args):
+    """Sets the sparse-kernel schedule the command line asks for (process-wide)."""
+    import activation_sparse_ffn_gemm_b200 as tw
+
+    mode = {"auto": tw.SCHED_AUTO, "fused": tw.SCHED_FUSED, "passes": tw.SCHED_PASSES}[args.sched]
+    tw.set_sparse_schedule(mode, args.l2_budget_mib << 20)
 
 
 def reduce_max(x: float, dist=None, device=None) -> float:
@@ -763,7 +775,8 @@ def run_twell(args, world, rank, local):
             print(json.dumps({"metric": METRIC, "value": main["M"] * world / (main["ms_step"] / 1e3),
                               "unit": "tokens/s", "ms_per_step": main["ms_step"], "fwd_ms": main["ms_fwd"],
                               "steps": args.steps, "warmup": max(3, args.warmup), "config": {
-                                  "workload": main["workload"], "note": "training step alone (profiling run)"},
+                                  "workload": main["workload"], "note": "training step alone (profiling run)",
+                                  "sparse_schedule": args.sched, "l2_budget_mib": args.l2_budget_mib or None},
                               "sparsity": main["sparsity"], "gpu_launches": main["gpu_launches"]}), flush=True)
         return
     if not args.no_extra:
@@ -821,6 +834,8 @@ def bench_line(args, world, main, others):
                    "l2": "flushed before every timed step (256 MiB device write, outside the events); "
                          "the step's inputs are also larger than L2",
                    "accumulation": "fp32", "ovf_cap": main["ovf_cap"],
+                   "sparse_schedule": (args.sched + (f", L2 budget {args.l2_budget_mib} MiB" if args.l2_budget_mib
+                                                     else "")),
                    "parallelism": (f"dp{world}: every rank its own {M} tokens, weight gradients summed over "
                                    "ranks (NCCL all-reduce) inside each step" if world > 1 else "dp1")},
         "fwd": {"tokens_per_s": tokens / (ms_fwd / 1e3), "ms": ms_fwd,
@@ -1225,6 +1240,8 @@ def run_block(args, local):
 def main():
     args = parse_args()
     world, rank, local = dist_env()
+    if args.impl != "reference" and (args.sched != "auto" or args.l2_budget_mib):
+        apply_schedule(args)
     if args.block:
         run_block(args, local)
     elif args.sweep and args.sweep_k:

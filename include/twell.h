@@ -347,7 +347,7 @@ TWELL_API twell_status twell_count_stats(const twell_hybrid* h, int64_t* rows_by
  *                       not; the token rows are re-read once per chunk.
  *   TWELL_SCHED_AUTO    the default: TWELL_SCHED_PASSES when W_g, W_u and W_d
  *                       together (3 d_model d_ff bf16) are larger than the
- *                       device's L2, else TWELL_SCHED_FUSED.
+ *                       device's L2 and M >= 4096, else TWELL_SCHED_FUSED.
  * l2_budget_bytes: the chunk bound, 0 for the default (64 MiB).
  * Process-wide; applies to the calls made after it returns. Tile routing
  * (twell_ffn_fwd_tiles) and the 8-bit forward always run fused. Errors:

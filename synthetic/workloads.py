@@ -61,6 +61,8 @@ WORKLOADS = {
     # the largest single-GPU point of the d_model=4096, d_ff=14336 sweep at 99% sparsity,
     # run as a training step (the throughput workload of bench.py)
     "large": Workload("large", 65536, 4096, 14336, 128, 8, 0.01, row_scale="lognormal", training=True),
+    # the M=8192 point of the same sweep at 99% sparsity, as a training step
+    "sweep8k": Workload("sweep8k", 8192, 4096, 14336, 128, 8, 0.01, row_scale="lognormal", training=True),
 }
 
 
