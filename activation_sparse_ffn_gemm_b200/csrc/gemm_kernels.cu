@@ -162,15 +162,22 @@ struct EpiTwell {
 
 // The dense-backup epilogues are element-wise: apply8 handles eight columns
 // [n, n + 8) of accumulator row `row` (a valid row), with the epilogue's own
-// inputs for those columns read beforehand by load8 (so that run() can have
-// the reads of a whole 32-column chunk in flight while the chunk's
-// accumulators come out of tensor memory). The split-K reduction feeds the
+// inputs for those columns read beforehand by load8 (so that run() can keep
+// the reads of the next 32-column chunk in flight while a chunk's
+// accumulators come out of tensor memory and are applied). The split-K reduction feeds the
 // summed partials through the four-argument apply8, which reads and applies.
 template <class Epi>
 __device__ __forceinline__ void run_apply8(const typename Epi::Args& a, int m0, int n0, int M_eff, int N, int r,
                                            uint32_t taddr) {
   const int row = m0 + r;
   const bool valid = row < M_eff;
+  // inputs one chunk ahead: chunk ch + 1's reads are in flight while chunk
+  // ch is applied and stored
+  typename Epi::In cur[4], nxt[4];
+  if (valid && n0 < N) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) Epi::load8(a, row, n0 + q * 8, cur[q]);
+  }
 #pragma unroll 1
   for (int ch = 0; ch < 8; ++ch) {
     const int n = n0 + ch * 32;
@@ -178,19 +185,24 @@ __device__ __forceinline__ void run_apply8(const typename Epi::Args& a, int m0, 
     uint32_t v[32];
     __syncwarp();
     tmem_ld_32x32b_x32(taddr + ch * 32, v);
-    typename Epi::In in[4];
-    if (valid) {
+    const bool more = valid && ch + 1 < 8 && n + 32 < N;
+    if (more) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) Epi::load8(a, row, n + q * 8, in[q]);
+      for (int q = 0; q < 4; ++q) Epi::load8(a, row, n + 32 + q * 8, nxt[q]);
     }
     tmem_wait_ld();
-    if (!valid) continue;
+    if (valid) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      float acc[8];
+      for (int q = 0; q < 4; ++q) {
+        float acc[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] = __uint_as_float(v[q * 8 + e]);
-      Epi::apply8(a, row, n + q * 8, acc, in[q]);
+        for (int e = 0; e < 8; ++e) acc[e] = __uint_as_float(v[q * 8 + e]);
+        Epi::apply8(a, row, n + q * 8, acc, cur[q]);
+      }
+    }
+    if (more) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
     }
   }
 }
