@@ -162,21 +162,35 @@ struct EpiTwell {
 
 // The dense-backup epilogues are element-wise: apply8 handles eight columns
 // [n, n + 8) of accumulator row `row` (a valid row), with the epilogue's own
-// inputs for those columns read beforehand by load8 (so that run() can keep
-// the reads of the next 32-column chunk in flight while a chunk's
-// accumulators come out of tensor memory and are applied). The split-K reduction feeds the
-// summed partials through the four-argument apply8, which reads and applies.
+// inputs for those columns read beforehand by load8. run() takes each warp's
+// 32 rows x 32 columns out of tensor memory (one row per lane), turns the
+// block around in shared memory so that four consecutive lanes hold the 32
+// columns of one row (8 each) and a warp instruction touches 8 rows x 64
+// contiguous bytes instead of 32 rows x 16 bytes, and keeps the reads of the
+// next chunk's inputs in flight while a chunk is applied and stored. The
+// split-K reduction feeds the summed partials through the four-argument
+// apply8, which reads and applies.
+constexpr int kApplyPitch = 33;                               // floats per staged row (conflict-free)
+constexpr int kApplySmemBytes = 4 * 32 * kApplyPitch * 4;     // one 32 x 32 block per epilogue warp
+
 template <class Epi>
 __device__ __forceinline__ void run_apply8(const typename Epi::Args& a, int m0, int n0, int M_eff, int N, int r,
-                                           uint32_t taddr) {
-  const int row = m0 + r;
-  const bool valid = row < M_eff;
-  // inputs one chunk ahead: chunk ch + 1's reads are in flight while chunk
-  // ch is applied and stored
-  typename Epi::In cur[4], nxt[4];
-  if (valid && n0 < N) {
+                                           uint32_t taddr, uint8_t* smem) {
+  const int w = r >> 5, lane = r & 31;
+  float* buf = reinterpret_cast<float*>(smem) + w * 32 * kApplyPitch;
+  const int cq = (lane & 3) * 8;  // this lane's 8 columns of a 32-column chunk
+  int rows[4];
+  bool ok[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) Epi::load8(a, row, n0 + q * 8, cur[q]);
+  for (int k = 0; k < 4; ++k) {
+    rows[k] = m0 + w * 32 + (lane >> 2) + 8 * k;
+    ok[k] = rows[k] < M_eff;
+  }
+  typename Epi::In cur[4], nxt[4];
+  if (n0 < N) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (ok[k]) Epi::load8(a, rows[k], n0 + cq, cur[k]);
   }
 #pragma unroll 1
   for (int ch = 0; ch < 8; ++ch) {
@@ -185,24 +199,29 @@ __device__ __forceinline__ void run_apply8(const typename Epi::Args& a, int m0, 
     uint32_t v[32];
     __syncwarp();
     tmem_ld_32x32b_x32(taddr + ch * 32, v);
-    const bool more = valid && ch + 1 < 8 && n + 32 < N;
+    const bool more = ch + 1 < 8 && n + 32 < N;
     if (more) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) Epi::load8(a, row, n + 32 + q * 8, nxt[q]);
+      for (int k = 0; k < 4; ++k)
+        if (ok[k]) Epi::load8(a, rows[k], n + 32 + cq, nxt[k]);
     }
     tmem_wait_ld();
-    if (valid) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float acc[8];
+    for (int c = 0; c < 32; ++c) buf[lane * kApplyPitch + c] = __uint_as_float(v[c]);
+    __syncwarp();
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = __uint_as_float(v[q * 8 + e]);
-        Epi::apply8(a, row, n + q * 8, acc, cur[q]);
-      }
+    for (int k = 0; k < 4; ++k) {
+      if (!ok[k]) continue;
+      const float* src = buf + ((lane >> 2) + 8 * k) * kApplyPitch + cq;
+      float acc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = src[e];
+      Epi::apply8(a, rows[k], n + cq, acc, cur[k]);
     }
+    __syncwarp();  // the block is rewritten by the next chunk
     if (more) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
+      for (int k = 0; k < 4; ++k) cur[k] = nxt[k];
     }
   }
 }
@@ -225,7 +244,7 @@ struct EpiGateMul {
     float* u_save;      // nullable [cap][f]
     int f;
   };
-  static constexpr int SMEM_BYTES = 0;
+  static constexpr int SMEM_BYTES = kApplySmemBytes;
   static constexpr bool kSplitK = true;
   struct In {
     uint4 g;
@@ -249,8 +268,9 @@ struct EpiGateMul {
     }
   }
   TWELL_APPLY8_DIRECT()
-  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
-    run_apply8<EpiGateMul>(a, m0, n0, M_eff, N, r, taddr);
+  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr,
+                             uint8_t* smem) {
+    run_apply8<EpiGateMul>(a, m0, n0, M_eff, N, r, taddr, smem);
   }
 };
 
@@ -263,7 +283,7 @@ struct EpiScatterBf16 {
     int rows_out;
     uint32_t* status;
   };
-  static constexpr int SMEM_BYTES = 0;
+  static constexpr int SMEM_BYTES = kApplySmemBytes;
   static constexpr bool kSplitK = true;
   struct In {
     int dst;
@@ -276,8 +296,9 @@ struct EpiScatterBf16 {
         make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
   }
   TWELL_APPLY8_DIRECT()
-  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
-    run_apply8<EpiScatterBf16>(a, m0, n0, M_eff, N, r, taddr);
+  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr,
+                             uint8_t* smem) {
+    run_apply8<EpiScatterBf16>(a, m0, n0, M_eff, N, r, taddr, smem);
   }
 };
 
@@ -289,7 +310,7 @@ struct EpiScatterF32 {
     int rows_out;
     uint32_t* status;
   };
-  static constexpr int SMEM_BYTES = 0;
+  static constexpr int SMEM_BYTES = kApplySmemBytes;
   static constexpr bool kSplitK = true;
   struct In {
     int dst;
@@ -303,8 +324,9 @@ struct EpiScatterF32 {
     p[1] = make_float4(v[4], v[5], v[6], v[7]);
   }
   TWELL_APPLY8_DIRECT()
-  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
-    run_apply8<EpiScatterF32>(a, m0, n0, M_eff, N, r, taddr);
+  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr,
+                             uint8_t* smem) {
+    run_apply8<EpiScatterF32>(a, m0, n0, M_eff, N, r, taddr, smem);
   }
 };
 
@@ -331,7 +353,7 @@ struct EpiBwdDH {
     float lambda;
     int f;
   };
-  static constexpr int SMEM_BYTES = 0;
+  static constexpr int SMEM_BYTES = kApplySmemBytes;
   static constexpr bool kSplitK = true;
   __device__ static void hi_lo(const float (&v)[8], uint4& hi, uint4& lo) {
     float h[8], l[8];
@@ -390,8 +412,9 @@ struct EpiBwdDH {
     }
   }
   TWELL_APPLY8_DIRECT()
-  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
-    run_apply8<EpiBwdDH>(a, m0, n0, M_eff, N, r, taddr);
+  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr,
+                             uint8_t* smem) {
+    run_apply8<EpiBwdDH>(a, m0, n0, M_eff, N, r, taddr, smem);
   }
 };
 
@@ -406,7 +429,7 @@ struct EpiStoreF32 {
     int m_split;
     int ld;
   };
-  static constexpr int SMEM_BYTES = 0;
+  static constexpr int SMEM_BYTES = kApplySmemBytes;
   static constexpr bool kSplitK = false;
   struct In {};
   __device__ static void load8(const Args&, int, int, In&) {}
@@ -418,8 +441,9 @@ struct EpiStoreF32 {
     p[1] = make_float4(v[4], v[5], v[6], v[7]);
   }
   TWELL_APPLY8_DIRECT()
-  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr, uint8_t*) {
-    run_apply8<EpiStoreF32>(a, m0, n0, M_eff, N, r, taddr);
+  __device__ static void run(const Args& a, int m0, int n0, int M_eff, int N, int r, uint32_t taddr,
+                             uint8_t* smem) {
+    run_apply8<EpiStoreF32>(a, m0, n0, M_eff, N, r, taddr, smem);
   }
 };
 

@@ -288,6 +288,18 @@ def kernel_work(name, M, d, f, T, K, kept, pairs, n_ovf=0, dense_wgrad=0):
     if name == "ell_updown_q8":
         # as ell_updown, with the two gathered weights read as 1-byte codes (plus a scale per unit)
         return "hbm", (2 * m_ell * d + m_ell * T * (2 + 3 * K) + 4 * kept + 2 * m_ell * d + 2 * f * d + 2 * 4 * f)
+    if name == "ell_up":
+        # the up pass: X, TwELL, u written, W_u once
+        return "hbm", 2 * m_ell * d + m_ell * T * (2 + 3 * K) + 4 * kept + 2 * f * d
+    if name == "ell_down":
+        # the down pass: TwELL, u read, Y written, W_dt once
+        return "hbm", m_ell * T * (2 + 3 * K) + 4 * kept + 2 * m_ell * d + 2 * f * d
+    if name == "ell_dh":
+        # the dH pass: dY, TwELL, u read, (h, dU, dZ) per slot written, W_dt once
+        return "hbm", 2 * m_ell * d + m_ell * T * (2 + 3 * K) + 4 * kept + 16 * kept + 2 * f * d
+    if name == "ell_dx":
+        # the dX pass: counts and columns, (h, dU, dZ) per slot read, dX (fp32) written, W_u and W_g once
+        return "hbm", m_ell * T * (2 + K) + 16 * kept + 4 * m_ell * d + 2 * 2 * f * d
     if name == "ell_bwd":
         # dY, TwELL, u read; (h, dU, dZ) per slot written; dX (fp32) written; W_u, W_g, W_dt once
         return "hbm", (2 * m_ell * d + m_ell * T * (2 + 3 * K) + 4 * kept + 16 * kept + 4 * m_ell * d
@@ -310,6 +322,10 @@ KERNEL_SOURCES = {
     "gate_pack_gemm": ("gemm_kernels.cu", "umma_gemm.cuh", "umma_gemm_pair.cuh", "sm100.cuh", "twell_internal.cuh"),
     "ell_updown": ("token_kernels.cu", "token_common.cuh", "sm100.cuh", "twell_internal.cuh"),
     "ell_bwd": ("token_kernels.cu", "token_common.cuh", "sm100.cuh", "twell_internal.cuh"),
+    "ell_up": ("token_kernels.cu", "token_common.cuh", "sm100.cuh", "twell_internal.cuh"),
+    "ell_down": ("token_kernels.cu", "token_common.cuh", "sm100.cuh", "twell_internal.cuh"),
+    "ell_dh": ("token_kernels.cu", "token_common.cuh", "sm100.cuh", "twell_internal.cuh"),
+    "ell_dx": ("token_kernels.cu", "token_common.cuh", "sm100.cuh", "twell_internal.cuh"),
     "weight_grads": ("pairlist_kernels.cu", "twell_internal.cuh"),
     "csc_fill": ("pairlist_kernels.cu", "twell_internal.cuh"),
     "transpose_wd": ("route_kernels.cu", "twell_internal.cuh"),

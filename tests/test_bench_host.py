@@ -84,6 +84,17 @@ def test_kernel_work_by_hand():
     assert sparse == 4 * 32 + 20 * 12 + 12 * 256 * 8 + 4 * 256
     assert dense == 4 * 32 + 20 * 10 + 24 * 256 * 8 + 4 * 256
     assert bench.kernel_work("transpose_wd", M, d, f, T, K, kept, pairs) == ("hbm", 4 * 256 * 8)
+    # the passes of the multi-pass schedule: the fused kernels' bytes split by pass (the
+    # per-slot records written by one pass and read by the next counted on both sides)
+    up = bench.kernel_work("ell_up", M, d, f, T, K, kept, pairs)[1]
+    down = bench.kernel_work("ell_down", M, d, f, T, K, kept, pairs)[1]
+    assert up == 2 * 32 + 4 * 2 * 26 + 40 + 2 * 256 * 8
+    assert down == 4 * 2 * 26 + 40 + 2 * 32 + 2 * 256 * 8
+    assert up + down == bench.kernel_work("ell_updown", M, d, f, T, K, kept, pairs)[1] + 4 * 2 * 26 + 40
+    dh = bench.kernel_work("ell_dh", M, d, f, T, K, kept, pairs)[1]
+    dx = bench.kernel_work("ell_dx", M, d, f, T, K, kept, pairs)[1]
+    assert dh == 2 * 32 + 4 * 2 * 26 + 40 + 160 + 2 * 256 * 8
+    assert dx == 4 * 2 * 10 + 160 + 4 * 32 + 4 * 256 * 8
     assert bench.kernel_work("row_flags", M, d, f, T, K, kept, pairs) == (None, None)
 
 
