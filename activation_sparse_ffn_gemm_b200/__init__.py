@@ -112,6 +112,8 @@ def lib():
             L.twell_test_withhold_epilogue_arrival.argtypes = [ctypes.c_int]
             L.twell_set_sparse_schedule.restype = ctypes.c_int
             L.twell_set_sparse_schedule.argtypes = [ctypes.c_int, _i64]
+            L.twell_set_overlap.restype = None
+            L.twell_set_overlap.argtypes = [ctypes.c_int]
             L.twell_status_read.restype = ctypes.c_int
             L.twell_status_read.argtypes = [ctypes.POINTER(TwellHybrid), ctypes.POINTER(ctypes.c_uint32),
                                             ctypes.c_int, _vp]
@@ -180,6 +182,12 @@ def set_sparse_schedule(mode: int = SCHED_AUTO, l2_budget_bytes: int = 0) -> Non
     l2_budget_bytes; 0 = the library's default) or SCHED_AUTO. Process-wide;
     the results are the same under every schedule."""
     _check(lib().twell_set_sparse_schedule(int(mode), int(l2_budget_bytes)), "twell_set_sparse_schedule")
+
+
+def set_overlap(on: bool = True) -> None:
+    """twell_set_overlap: run the dense-backup GEMMs on the library's side stream
+    beside the sparse kernels (default) or everything on the caller's stream."""
+    lib().twell_set_overlap(1 if on else 0)
 
 
 def trace_enable(on: bool = True) -> None:

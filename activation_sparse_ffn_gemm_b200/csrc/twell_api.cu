@@ -36,6 +36,83 @@ long long device_l2_bytes() {
   return v;
 }
 
+// ---------------------------------------------- the dense-backup side stream
+// twell_set_overlap: the dense-backup GEMMs of a call run on a second stream
+// of the library (created per device at first use, at the highest priority,
+// so that the block scheduler places the persistent GEMM's CTAs before those
+// of the sparse kernels on the caller's stream); the sparse kernels then fill
+// the SMs' leftover shared memory and registers beside the GEMM. The caller's
+// stream forks to it after the routing and joins it before the first kernel
+// that reads what it wrote. The mutex keeps one call's fork/join from
+// interleaving with another host thread's.
+std::atomic<int> g_overlap{1};
+
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  std::mutex mu;
+};
+
+SideStream* side_stream() {
+  static SideStream side[64];
+  static std::mutex create_mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  SideStream& ss = side[dev];
+  std::lock_guard<std::mutex> lk(create_mu);
+  if (!ss.s) {
+    int lo = 0, hi = 0;
+    if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) return nullptr;
+    cudaStream_t st = nullptr;
+    cudaEvent_t a = nullptr, b = nullptr;
+    if (cudaStreamCreateWithPriority(&st, cudaStreamNonBlocking, hi) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&a, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&b, cudaEventDisableTiming) != cudaSuccess) {
+      cudaStreamDestroy(st);
+      if (a) cudaEventDestroy(a);
+      return nullptr;
+    }
+    ss.fork = a;
+    ss.join = b;
+    ss.s = st;
+  }
+  return &ss;
+}
+
+// Fork of one call: the stream the dense chain runs on (the caller's when the
+// overlap is off or the side stream cannot be had), and the join.
+class DenseFork {
+ public:
+  explicit DenseFork(cudaStream_t main) : main_(main), dense_(main) {
+    if (!g_overlap.load()) return;
+    ss_ = side_stream();
+    if (!ss_) return;
+    lk_ = std::unique_lock<std::mutex>(ss_->mu);
+    if (cudaEventRecord(ss_->fork, main_) != cudaSuccess || cudaStreamWaitEvent(ss_->s, ss_->fork, 0) != cudaSuccess) {
+      lk_.unlock();
+      ss_ = nullptr;
+      return;
+    }
+    dense_ = ss_->s;
+  }
+  cudaStream_t dense() const { return dense_; }
+  // Makes the caller's stream wait for the dense chain (idempotent).
+  cudaError_t join() {
+    if (!ss_ || joined_) return cudaSuccess;
+    joined_ = true;
+    cudaError_t e = cudaEventRecord(ss_->join, dense_);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(main_, ss_->join, 0);
+    return e;
+  }
+  ~DenseFork() { join(); }
+
+ private:
+  cudaStream_t main_, dense_;
+  SideStream* ss_ = nullptr;
+  std::unique_lock<std::mutex> lk_;
+  bool joined_ = false;
+};
+
 unsigned long long next_launch_epoch() {
   static std::atomic<unsigned long long> next{1};
   constexpr unsigned long long kMask = (1ull << 56) - 1;
@@ -320,18 +397,27 @@ twell_status ffn_fwd_impl(const uint16_t* X, const uint16_t* W_g, const uint16_t
   uint16_t* x_ovf = at<uint16_t>(ws, L.x_ovf);
   st = run_pack(X, W_g, b_g, d, h, z_debug, ws, L, X, x_ovf, tiles, s);
   if (st != TWELL_OK) return st;
+  if (tiles) {
+    return cuda_status(launch_ell_ffn_fwd(X, W_u, wdt, h->count, h->val, h->col, at<uint16_t>(ws, L.spill),
+                                          h->row_plan, nullptr, at<float>(ws, L.ubuf), Y, M, d, f, K,
+                                          at<int>(ws, L.ctr), at<float>(ws, L.yacc), at<int>(ws, L.turn_x),
+                                          h->status, s));
+  }
+  // the dense backup (its own rows of Y) first, on the side stream when the
+  // overlap is on; the sparse kernels (the other rows) on the caller's stream
+  DenseFork fk(s);
+  const SplitKBuffers sk{at<float>(ws, L.sk_partial), at<unsigned long long>(ws, L.sk_arrivals)};
+  if (launch_ovf_fwd(x_ovf, W_u, W_d, h->g_ovf, h->ovf_rows, h->n_ovf, cap, M, d, f, at<uint16_t>(ws, L.h_ovf),
+                     h->u_ovf, Y, sk, h->status, fk.dense()) != cudaSuccess)
+    return TWELL_ECUDA;
   const cudaError_t ce =
       q8 ? launch_ell_ffn_fwd_q8(X, q8->W_u8, q8->s_u, q8->W_dt8, q8->s_d, h->count, h->val, h->col, h->row_plan,
                                  h->u_ell, Y, M, d, f, K, at<int>(ws, L.ctr), at<float>(ws, L.yacc), h->status, s)
-         : launch_ell_ffn_fwd(X, W_u, wdt, h->count, h->val, h->col, tiles ? at<uint16_t>(ws, L.spill) : nullptr,
-                              h->row_plan, tiles ? nullptr : h->u_ell,
+         : launch_ell_ffn_fwd(X, W_u, wdt, h->count, h->val, h->col, nullptr, h->row_plan, h->u_ell,
                               at<float>(ws, L.ubuf), Y, M, d, f, K, at<int>(ws, L.ctr), at<float>(ws, L.yacc),
                               at<int>(ws, L.turn_x), h->status, s);
   if (ce != cudaSuccess) return TWELL_ECUDA;
-  if (tiles) return TWELL_OK;
-  const SplitKBuffers sk{at<float>(ws, L.sk_partial), at<unsigned long long>(ws, L.sk_arrivals)};
-  return cuda_status(launch_ovf_fwd(x_ovf, W_u, W_d, h->g_ovf, h->ovf_rows, h->n_ovf, cap, M, d, f,
-                                    at<uint16_t>(ws, L.h_ovf), h->u_ovf, Y, sk, h->status, s));
+  return cuda_status(fk.join());
 }
 
 }  // namespace
@@ -412,21 +498,33 @@ twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_
   float4* hdz_ell = at<float4>(ws, L.hdz_ell);
   const DenseWgradOperands dw{at<uint16_t>(ws, L.x_rows), at<uint16_t>(ws, L.dy_rows), at<uint16_t>(ws, L.duz_hi),
                               at<uint16_t>(ws, L.h_hi)};
-  if (launch_ovf_prep(X, dY, h->ovf_rows, h->n_ovf, h->row_plan, cap, M, d, f, dw, h->status, s) != cudaSuccess)
-    return TWELL_ECUDA;
-  if (launch_ell_ffn_bwd(dY, W_u, W_g, wdt, h->count, h->val, h->col, h->row_plan, h->n_ovf, h->u_ell, lambda,
-                         hdz_ell, dX, M, d, f, K, at<int>(ws, L.ctr), at<int>(ws, L.turn_x), h->status,
-                         s) != cudaSuccess)
-    return TWELL_ECUDA;
   float* du_ovf = at<float>(ws, L.du_ovf);
   float* dz_ovf = at<float>(ws, L.dz_ovf);
   const SplitKBuffers sk{at<float>(ws, L.sk_partial), at<unsigned long long>(ws, L.sk_arrivals)};
   float* db_ovf = at<float>(ws, L.db_ovf);
   int* k_rows = at<int>(ws, L.k_rows);
-  if (launch_ovf_bwd(dw.dy_rows, wdt, W_u, W_g, h->g_ovf, h->u_ovf, lambda, h->ovf_rows, h->n_ovf, h->row_plan, cap, M,
-                     d, f, dw, du_ovf, dz_ovf, dX, sk, h->status, s) != cudaSuccess)
-    return TWELL_ECUDA;
-  if (launch_ovf_db(h->n_ovf, h->row_plan, cap, f, dw, at<float>(ws, L.db_part), db_ovf, k_rows, s) != cudaSuccess) return TWELL_ECUDA;
+  {
+    // the dense rows' chain (their dX rows, db part and weight-gradient GEMMs)
+    // first, on the side stream when the overlap is on; the sparse passes and
+    // the pair list's counts on the caller's stream; joined before the pair
+    // list is filled (it reads the dense rows' dU and dZ) and the weight
+    // gradients (they add to what the GEMMs wrote)
+    DenseFork fk(s);
+    const cudaStream_t ds = fk.dense();
+    if (launch_ovf_prep(X, dY, h->ovf_rows, h->n_ovf, h->row_plan, cap, M, d, f, dw, h->status, ds) != cudaSuccess)
+      return TWELL_ECUDA;
+    if (launch_ovf_bwd(dw.dy_rows, wdt, W_u, W_g, h->g_ovf, h->u_ovf, lambda, h->ovf_rows, h->n_ovf, h->row_plan, cap,
+                       M, d, f, dw, du_ovf, dz_ovf, dX, sk, h->status, ds) != cudaSuccess)
+      return TWELL_ECUDA;
+    if (launch_ovf_db(h->n_ovf, h->row_plan, cap, f, dw, at<float>(ws, L.db_part), db_ovf, k_rows, ds) != cudaSuccess)
+      return TWELL_ECUDA;
+    if (launch_dense_wgrad(dw, k_rows, cap, d, f, dW_g, dW_u, dW_d, h->status, ds) != cudaSuccess) return TWELL_ECUDA;
+    if (launch_ell_ffn_bwd(dY, W_u, W_g, wdt, h->count, h->val, h->col, h->row_plan, h->n_ovf, h->u_ell, lambda,
+                           hdz_ell, dX, M, d, f, K, at<int>(ws, L.ctr), at<int>(ws, L.turn_x), h->status,
+                           s) != cudaSuccess)
+      return TWELL_ECUDA;
+    if (fk.join() != cudaSuccess) return TWELL_ECUDA;
+  }
   const long long nnz_cap = static_cast<long long>(M - cap) * (f / kTn) * K + static_cast<long long>(cap) * f;
   CscBuffers b{M, cap, nnz_cap, h->status, h->row_plan + kPlanHdr + M, at<int>(ws, L.block_cnt),
                at<int>(ws, L.unit_tot), at<unsigned long long>(ws, L.scan_arrive), at<int>(ws, L.unit_ptr),
@@ -434,7 +532,6 @@ twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_
   if (launch_build_csc(h->count, h->col, h->row_ovf, h->g_ovf, h->u_ovf, hdz_ell, du_ovf, dz_ovf, h->row_plan, M, f,
                        K, b, s) != cudaSuccess)
     return TWELL_ECUDA;
-  if (launch_dense_wgrad(dw, k_rows, cap, d, f, dW_g, dW_u, dW_d, h->status, s) != cudaSuccess) return TWELL_ECUDA;
   return cuda_status(launch_weight_grads(X, dY, b, d, f, cap > 0 ? db_ovf : nullptr, cap > 0 ? k_rows : nullptr,
                                          dW_g, dW_u, dW_d, db_g, s));
 }
@@ -453,6 +550,8 @@ twell_status twell_count_stats(const twell_hybrid* h, int64_t* rows_by_max, int6
   return cuda_status(launch_count_stats(h->count, h->M, h->d_ff / kTn, h->dense_min, rows_by_max, act_by_max,
                                         tiles_by_count, reinterpret_cast<cudaStream_t>(stream)));
 }
+
+void twell_set_overlap(int on) { g_overlap.store(on ? 1 : 0); }
 
 twell_status twell_set_sparse_schedule(int mode, int64_t l2_budget_bytes) {
   return static_cast<twell_status>(twell::set_sparse_schedule(mode, l2_budget_bytes));

@@ -30,6 +30,8 @@
 // outstanding copies and MMAs, frees its tensor memory and returns.
 #pragma once
 
+#include <atomic>
+
 #include "sm100.cuh"
 #include "trace.cuh"
 #include "twell_internal.cuh"
@@ -460,6 +462,21 @@ constexpr int gemm_smem_bytes() {
   return 1024 + GemmLayout<BN, STAGES>::EPI_OFF + Epi::SMEM_BYTES;
 }
 
+// Raises a kernel's dynamic shared-memory limit once per device (the
+// attribute call is host work that every launch would otherwise repeat).
+template <auto Kern>
+cudaError_t set_smem_once(int smem) {
+  static std::atomic<unsigned long long> done{0};  // one bit per device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = dev >= 0 && dev < 64 ? 1ull << dev : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
 // Launches the GEMM on min(#SMs, tiles) persistent CTAs. The static row bound
 // shp.M sizes the grid; rows beyond *M_dev are skipped by the device.
 template <class Epi, int BN, bool B_MN, int STAGES, bool A_MN = false>
@@ -469,7 +486,7 @@ cudaError_t launch_umma_gemm(const char* name, const CUtensorMap& a0, const CUte
   constexpr int smem = gemm_smem_bytes<Epi, BN, STAGES>();
   static_assert(smem <= 232448, "shared memory budget");
   auto kern = umma_gemm_kernel<Epi, BN, B_MN, STAGES, A_MN>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = set_smem_once<umma_gemm_kernel<Epi, BN, B_MN, STAGES, A_MN>>(smem);
   if (e != cudaSuccess) return e;
   const long tiles = static_cast<long>((shp.M + kBM - 1) / kBM) * ((shp.N + BN - 1) / BN);
   if (tiles <= 0) return cudaSuccess;

@@ -345,7 +345,7 @@ cudaError_t launch_umma_pair(const char* name, const CUtensorMap& a0, const CUte
   static_assert(smem <= 232448, "shared memory budget");
   if (shp.partial != nullptr) return cudaErrorInvalidValue;
   auto kern = umma_pair_kernel<Epi, B_MN, STAGES, A_MN>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = set_smem_once<umma_pair_kernel<Epi, B_MN, STAGES, A_MN>>(smem);
   if (e != cudaSuccess) return e;
   const long tiles = static_cast<long>((shp.M + kPairBM - 1) / kPairBM) * ((shp.N + kPairBN - 1) / kPairBN);
   if (tiles <= 0) return cudaSuccess;

@@ -86,6 +86,8 @@ def parse_args():
                    help="schedule of the sparse kernels (twell_set_sparse_schedule)")
     p.add_argument("--l2-budget-mib", type=int, default=0,
                    help="L2 budget of one chunk of the multi-pass schedule, MiB (0: the library default)")
+    p.add_argument("--overlap", default="on", choices=["on", "off"],
+                   help="dense-backup GEMMs on the library's side stream beside the sparse kernels (twell_set_overlap)")
     return p.parse_args()
 
 
@@ -95,6 +97,7 @@ def apply_schedule(args):
 
     mode = {"auto": tw.SCHED_AUTO, "fused": tw.SCHED_FUSED, "passes": tw.SCHED_PASSES}[args.sched]
     tw.set_sparse_schedule(mode, args.l2_budget_mib << 20)
+    tw.set_overlap(args.overlap == "on")
 
 
 def reduce_max(x: float, dist=None, device=None) -> float:
@@ -792,7 +795,8 @@ def run_twell(args, world, rank, local):
                               "unit": "tokens/s", "ms_per_step": main["ms_step"], "fwd_ms": main["ms_fwd"],
                               "steps": args.steps, "warmup": max(3, args.warmup), "config": {
                                   "workload": main["workload"], "note": "training step alone (profiling run)",
-                                  "sparse_schedule": args.sched, "l2_budget_mib": args.l2_budget_mib or None},
+                                  "sparse_schedule": args.sched, "l2_budget_mib": args.l2_budget_mib or None,
+                                  "overlap": args.overlap},
                               "sparsity": main["sparsity"], "gpu_launches": main["gpu_launches"]}), flush=True)
         return
     if not args.no_extra:
@@ -852,6 +856,7 @@ def bench_line(args, world, main, others):
                    "accumulation": "fp32", "ovf_cap": main["ovf_cap"],
                    "sparse_schedule": (args.sched + (f", L2 budget {args.l2_budget_mib} MiB" if args.l2_budget_mib
                                                      else "")),
+                   "dense_overlap": args.overlap,
                    "parallelism": (f"dp{world}: every rank its own {M} tokens, weight gradients summed over "
                                    "ranks (NCCL all-reduce) inside each step" if world > 1 else "dp1")},
         "fwd": {"tokens_per_s": tokens / (ms_fwd / 1e3), "ms": ms_fwd,
@@ -1256,7 +1261,7 @@ def run_block(args, local):
 def main():
     args = parse_args()
     world, rank, local = dist_env()
-    if args.impl != "reference" and (args.sched != "auto" or args.l2_budget_mib):
+    if args.impl != "reference" and (args.sched != "auto" or args.l2_budget_mib or args.overlap != "on"):
         apply_schedule(args)
     if args.block:
         run_block(args, local)

@@ -212,7 +212,8 @@ def test_deterministic(tw):
         assert torch.equal(a, b)
 
 
-SCHEDULE_CASES = ("ragged", "k64", "long_rows_w2", "wide_d_w4", "heavy_small", "multi_tile", "min_d_model")
+SCHEDULE_CASES = ("ragged", "k64", "long_rows_w2", "wide_d_w4", "widest_d_w8", "heavy_small", "multi_tile",
+                  "min_d_model", "max_d_ff", "dense_wgrad")
 
 
 @pytest.mark.parametrize("name", SCHEDULE_CASES)
@@ -243,6 +244,65 @@ def test_schedules_agree_bit_for_bit(tw, name):
     for label in ("passes", "chunked"):
         for a, b in zip(outs["fused"], outs[label]):
             assert torch.equal(a, b), label
+
+
+def test_overlap_agrees_and_captures(tw):
+    """The dense-backup chain on the library's side stream (twell_set_overlap)
+    gives the same Y and gradients as everything on the caller's stream, bit
+    for bit, on a batch whose dense backup runs split-K (170 overflow rows) and
+    on one whose dense rows' weight gradients run as GEMMs; and a forward +
+    backward with the side stream captured into a CUDA graph and replayed
+    reproduces them too (the fork and join are capturable)."""
+    for name in ("heavy_small", "dense_wgrad"):
+        M, d, f, K, act, rs, seed = CASES[name]
+        w = Workload(name, M, d, f, 128, K, act, row_scale=rs, training=True, seed=seed)
+        D = _dev(make_inputs(w))
+        outs = {}
+        try:
+            for on in (False, True):
+                tw.set_overlap(on)
+                Y, st = tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], K=K)
+                g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=1e-3)
+                torch.cuda.synchronize()
+                assert st.read_status() == 0
+                outs[on] = [Y] + [g[k] for k in sorted(g)]
+            for a, b in zip(outs[False], outs[True]):
+                assert torch.equal(a, b), name
+            # graph capture with the overlap on: preallocated state, workspaces and outputs
+            tw.set_overlap(True)
+            dev = D["X"].device
+            st = tw.HybridState(M, f, 128, K, M, dev, with_u=True)
+            wsf = tw.workspace(tw.OP_FWD, M, d, f, 128, K, M, dev)
+            wsb = tw.workspace(tw.OP_BWD, M, d, f, 128, K, M, dev)
+            Wdt = tw.transpose_wd(D["W_d"])
+            Y = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
+            out = dict(dX=torch.empty((M, d), device=dev), dW_g=torch.empty((f, d), device=dev),
+                       dW_u=torch.empty((f, d), device=dev), dW_d=torch.empty((d, f), device=dev),
+                       db_g=torch.empty((f,), device=dev))
+
+            def run():
+                tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], K=K, W_dt=Wdt, state=st, ws=wsf, Y=Y)
+                tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=1e-3, W_dt=Wdt, ws=wsb, out=out)
+
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                run()
+            torch.cuda.current_stream().wait_stream(side)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                run()
+            for k in out:
+                out[k].zero_()
+            Y.zero_()
+            graph.replay()
+            torch.cuda.synchronize()
+            assert st.read_status() == 0
+            for a, b in zip([Y] + [out[k] for k in sorted(out)], outs[True]):
+                assert torch.equal(a, b), name + " (graph replay)"
+            del graph
+        finally:
+            tw.set_overlap(True)
 
 
 def test_prepared_wdt_matches(tw):
