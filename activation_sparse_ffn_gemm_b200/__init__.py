@@ -186,7 +186,8 @@ def set_sparse_schedule(mode: int = SCHED_AUTO, l2_budget_bytes: int = 0) -> Non
 
 def set_overlap(on: bool = True) -> None:
     """twell_set_overlap: run the dense-backup GEMMs on the library's side stream
-    beside the sparse kernels (default) or everything on the caller's stream."""
+    beside the sparse kernels, or (off, the default) everything on the caller's
+    stream."""
     lib().twell_set_overlap(1 if on else 0)
 
 

@@ -29,6 +29,8 @@
 // split rows are those of the bf16 kernel (token_kernels.cu).
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 #include "token_common.cuh"
 #include "trace.cuh"
 
@@ -242,6 +244,23 @@ __device__ __forceinline__ void acc_io_q8(float* __restrict__ acc, int first, in
   }
 }
 
+// The bf16 row segment of Y (16 values per chunk) from the fp32 accumulators.
+template <int C8, int W, bool EXACT>
+__device__ __forceinline__ void store_y_q8(uint16_t* __restrict__ y_row, int first, int nch8,
+                                           const float2 (&y)[C8][8]) {
+  uint4* yr = reinterpret_cast<uint4*>(y_row);
+#pragma unroll
+  for (int q = 0; q < C8; ++q) {
+    const int idx = first + W * 32 * q;
+    if (!(EXACT || idx < nch8)) continue;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      yr[2 * idx + h] = make_uint4(pack_bf16x2(y[q][4 * h].x, y[q][4 * h].y), pack_bf16x2(y[q][4 * h + 1].x, y[q][4 * h + 1].y),
+                                   pack_bf16x2(y[q][4 * h + 2].x, y[q][4 * h + 2].y),
+                                   pack_bf16x2(y[q][4 * h + 3].x, y[q][4 * h + 3].y));
+  }
+}
+
 template <int C8, int W>
 struct Q8Cfg {
   static constexpr int WARPS = W > kTokWarps ? W : kTokWarps;
@@ -333,6 +352,119 @@ __global__ void __launch_bounds__(Q8Cfg<C8, W>::WARPS * 32, 512 / (Q8Cfg<C8, W>:
   }
 }
 
+// The multi-pass schedule with 8-bit rows (the bf16 passes of token_kernels.cu
+// with the q8 gathers): u per kept slot by hidden-tile chunks (the dot scaled
+// by the unit's W_u scale), then Y by column chunks (h times the unit's W_d
+// scale). The same sums in the same order as ell_fwd_q8_kernel.
+template <int C8, int W, bool EXACT>
+__global__ void __launch_bounds__(Q8Cfg<C8, W>::WARPS * 32, 512 / (Q8Cfg<C8, W>::WARPS * 32)) ell_up_q8_kernel(
+    const uint16_t* __restrict__ X, const uint8_t* __restrict__ Wu8, const float* __restrict__ su,
+    const uint16_t* __restrict__ count, const uint16_t* __restrict__ val, const uint8_t* __restrict__ col,
+    int* __restrict__ plan, float* __restrict__ ubuf, int M, int d, int T, int K, int nhc, int tpc,
+    int* __restrict__ ctr, uint32_t* status) {
+  using Cfg = Q8Cfg<C8, W>;
+  constexpr int B = Cfg::B;
+  __shared__ GroupSmem gs[Cfg::G];
+  __shared__ float part[Cfg::G][W > 1 ? W : 1][kListCap];
+  __shared__ int s_next[Cfg::G];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = warp / W, wi = warp % W, gtid = wi * 32 + lane;
+  GroupSmem& g = gs[grp];
+  const int nch8 = d >> 4;
+  while (next_piece<W, false>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g, status, nhc)) {
+    const long row = g.row;
+    int e0, ne;
+    chunk_entries(g, plan[1], T, tpc, e0, ne);
+    if (ne > 0) {
+      build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, nullptr, status);
+      group_sync<W>(grp);
+      {
+        uint4 xh[C8][2];
+        load_row_f16<C8, W, EXACT>(X + row * d, gtid, nch8, xh);
+        gather_dots_q8<C8, W, B, EXACT>(g, ne, xh, Wu8, d, gtid, nch8, lane, g.c2, part[grp][wi]);
+      }
+      group_sync<W>(grp);
+      for (int e = gtid; e < ne; e += Cfg::GT) {
+        float u = g.c2[e];
+        if (W > 1) {
+          u = 0.f;
+#pragma unroll
+          for (int w = 0; w < W; ++w) u += part[grp][w][e];
+        }
+        ubuf[row * T * K + g.slot[e]] = u * __ldg(su + g.j[e]);
+      }
+    }
+    group_sync<W>(grp);
+  }
+}
+
+template <int C8, int W, bool EXACT>
+__global__ void __launch_bounds__(Q8Cfg<C8, W>::WARPS * 32, 512 / (Q8Cfg<C8, W>::WARPS * 32)) ell_down_q8_kernel(
+    const uint8_t* __restrict__ Wdt8, const float* __restrict__ sd, const uint16_t* __restrict__ count,
+    const uint16_t* __restrict__ val, const uint8_t* __restrict__ col, int* __restrict__ plan,
+    const float* __restrict__ ubuf, uint16_t* __restrict__ Y, int M, int d, int T, int K, int dw,
+    int* __restrict__ ctr, float* __restrict__ yacc, int* __restrict__ turn_x, uint32_t* status) {
+  using Cfg = Q8Cfg<C8, W>;
+  constexpr int B = Cfg::B;
+  __shared__ GroupSmem gs[Cfg::G];
+  __shared__ int s_next[Cfg::G];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = warp / W, wi = warp % W, gtid = wi * 32 + lane;
+  GroupSmem& g = gs[grp];
+  const int nch8 = dw >> 4;
+  while (next_piece<W, false>(ctr, plan, M, count, T, K, grp, wi, lane, s_next, g, status, d / dw)) {
+    const long row = g.row;
+    const int S = plan[1];
+    const int e0 = g.q * S;
+    const int ne = max(0, min(S, g.tot - e0));
+    build_list(g, row, T, K, e0, ne, gtid, Cfg::GT, val, col, ubuf, status);
+    group_sync<W>(grp);
+    for (int e = gtid; e < ne; e += Cfg::GT) g.c[e] *= g.c2[e];  // h = g u
+    group_sync<W>(grp);
+    const int c0 = g.ch * dw;
+    float2 y[C8][8];
+#pragma unroll
+    for (int q = 0; q < C8; ++q)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) y[q][k] = make_float2(0.f, 0.f);
+    gather_axpy_q8<C8, W, B, EXACT>(g, ne, g.c, sd, Wdt8 + c0, d, gtid, nch8, y);
+    const int rw = g.row, q = g.q, P = g.P;
+    uint16_t* yrow = Y + static_cast<long>(rw) * d + c0;
+    if (P == 1) {
+      store_y_q8<C8, W, EXACT>(yrow, gtid, nch8, y);
+    } else {
+      int* turn = turn_x ? turn_x + static_cast<long>(g.ch) * M : plan + kPlanHdr;
+      float* acc = yacc + static_cast<long>(rw) * d + c0;
+      turn_wait<W>(turn, rw, q, grp, gtid, status);
+      acc_io_q8<C8, W, EXACT>(acc, gtid, nch8, y, q > 0, q + 1 < P);
+      if (q + 1 == P) store_y_q8<C8, W, EXACT>(yrow, gtid, nch8, y);
+      turn_pass<W>(turn, rw, q, P, grp, gtid);
+    }
+    group_sync<W>(grp);
+  }
+}
+
+// Calls fn(C8, W, EXACT) for the 8-bit kernels' shape of a row of w values:
+// the bf16 kernels' warps per token (tok_shape), 16 codes per lane chunk.
+template <class F>
+cudaError_t with_q8_shape(int w, F&& fn) {
+  using std::integral_constant;
+  int C, W;
+  tok_shape(w, C, W);
+  const int nch8 = w / 16;
+#define TWELL_Q8S(CC8, WW)                                                                                       \
+  return nch8 == WW * 32 * CC8                                                                                    \
+             ? fn(integral_constant<int, CC8>{}, integral_constant<int, WW>{}, integral_constant<bool, true>{})  \
+             : fn(integral_constant<int, CC8>{}, integral_constant<int, WW>{}, integral_constant<bool, false>{})
+  if (W == 1 && C <= 2) TWELL_Q8S(1, 1);
+  if (W == 1 && C == 4) TWELL_Q8S(2, 1);
+  if (W == 1) TWELL_Q8S(4, 1);
+  if (W == 2) TWELL_Q8S(4, 2);
+  if (W == 4) TWELL_Q8S(4, 4);
+  TWELL_Q8S(4, 8);
+#undef TWELL_Q8S
+}
+
 template <int C8, int W, bool EXACT, typename... A>
 void launch_q8_cw(int M, cudaStream_t s, A... a) {
   constexpr int threads = Q8Cfg<C8, W>::WARPS * 32;
@@ -354,11 +486,38 @@ cudaError_t launch_quantize_rows(const uint16_t* W, int rows, int len, uint8_t* 
 
 cudaError_t launch_ell_ffn_fwd_q8(const uint16_t* X, const uint8_t* W_u8, const float* s_u, const uint8_t* W_dt8,
                                   const float* s_d, const uint16_t* count, const uint16_t* val, const uint8_t* col,
-                                  int* plan, float* u_ell, uint16_t* Y, int M, int d, int f, int K, int* ctr,
-                                  float* yacc, uint32_t* status, cudaStream_t s) {
+                                  int* plan, float* u_ell, float* ubuf, uint16_t* Y, int M, int d, int f, int K,
+                                  int* ctr, float* yacc, int* turn_x, uint32_t* status, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
+  if (sparse_multi_pass(M, d, f)) {
+    const int T = f / kTn;
+    const PassChunks ch = pass_chunks(d, T, static_cast<long long>(d) * f);  // one byte per code
+    float* ub = u_ell ? u_ell : ubuf;
+    e = with_q8_shape(d, [&](auto cc, auto ww, auto ex) {
+      constexpr int C8 = decltype(cc)::value, W = decltype(ww)::value;
+      constexpr bool EX = decltype(ex)::value;
+      TWELL_LAUNCH("ell_up_q8", s,
+                   (ell_up_q8_kernel<C8, W, EX><<<tok_grid(M, Q8Cfg<C8, W>::G), Q8Cfg<C8, W>::WARPS * 32, 0, s>>>(
+                       X, W_u8, s_u, count, val, col, plan, ub, M, d, T, K, ch.nhc, ch.tpc, ctr, status)));
+      return cudaGetLastError();
+    });
+    if (e != cudaSuccess) return e;
+    const int ndc = d / ch.dw_y;
+    int* turn = ndc > 1 ? turn_x : nullptr;
+    if (turn && (e = cudaMemsetAsync(turn, 0, sizeof(int) * static_cast<size_t>(ndc) * M, s)) != cudaSuccess)
+      return e;
+    if ((e = cudaMemsetAsync(ctr, 0, sizeof(int), s)) != cudaSuccess) return e;
+    return with_q8_shape(ch.dw_y, [&](auto cc, auto ww, auto ex) {
+      constexpr int C8 = decltype(cc)::value, W = decltype(ww)::value;
+      constexpr bool EX = decltype(ex)::value;
+      TWELL_LAUNCH("ell_down_q8", s,
+                   (ell_down_q8_kernel<C8, W, EX><<<tok_grid(M, Q8Cfg<C8, W>::G), Q8Cfg<C8, W>::WARPS * 32, 0, s>>>(
+                       W_dt8, s_d, count, val, col, plan, ub, Y, M, d, T, K, ch.dw_y, ctr, yacc, turn, status)));
+      return cudaGetLastError();
+    });
+  }
   int C, W;
   tok_shape(d, C, W);  // the bf16 kernel's token groups, so the row plan's piece size fits this launch too
   const int T = f / kTn;

@@ -187,6 +187,18 @@ __device__ __forceinline__ bool next_piece(int* ctr, const int* plan, int M, con
   return true;
 }
 
+// Entries [e0, e0 + ne) of the group's piece that lie in hidden-tile chunk
+// g.ch of tpc tiles (the multi-pass schedule's dot passes).
+__device__ __forceinline__ void chunk_entries(const GroupSmem& g, int S, int T, int tpc, int& e0, int& ne) {
+  const int t0 = g.ch * tpc, t1 = t0 + tpc;
+  const int lo = t0 < T ? g.off[t0] : g.tot;
+  const int hi = t1 < T ? g.off[t1] : g.tot;
+  const int p0 = g.q * S;
+  const int p1 = min(p0 + S, g.tot);
+  e0 = max(p0, lo);
+  ne = max(0, min(p1, hi) - e0);
+}
+
 // Chunks per lane C and warps per token W for a row of d bf16 (d/8 chunks).
 inline void tok_shape(int d, int& C, int& W) {
   const int nch = d / 8;

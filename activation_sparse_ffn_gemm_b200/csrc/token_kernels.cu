@@ -487,18 +487,6 @@ inline int pass_grid(int M, int G, int warps, int threads_per_sm = kPassThreadsP
 // through that chunk's turnstile), so the results do not depend on the
 // schedule.
 
-// Entries [e0, e0 + ne) of the group's piece that lie in hidden-tile chunk
-// g.ch of tpc tiles.
-__device__ __forceinline__ void chunk_entries(const GroupSmem& g, int S, int T, int tpc, int& e0, int& ne) {
-  const int t0 = g.ch * tpc, t1 = t0 + tpc;
-  const int lo = t0 < T ? g.off[t0] : g.tot;
-  const int hi = t1 < T ? g.off[t1] : g.tot;
-  const int p0 = g.q * S;
-  const int p1 = min(p0 + S, g.tot);
-  e0 = max(p0, lo);
-  ne = max(0, min(p1, hi) - e0);
-}
-
 // List of entries [e0, e0 + ne) with the unit and both backward coefficients
 // (dU in c, dZ in c2) read from the per-slot record of the dH pass.
 __device__ __forceinline__ void build_list_hdz(GroupSmem& g, long row, int T, int K, int e0, int ne, int gtid, int GT,
@@ -747,19 +735,14 @@ cudaError_t with_tok_shape(int w, F&& fn) {
 std::atomic<int> g_sched_mode{TWELL_SCHED_AUTO};
 std::atomic<long long> g_l2_budget{kDefaultL2Budget};
 
-struct Chunks {
-  int nhc, tpc;  // hidden-tile chunks of the up and dH passes, tiles per chunk
-  int dw_y;      // column chunk width of the down pass
-  int dw_x;      // column chunk width of the dX pass
-};
+}  // namespace
 
 // Smallest chunk count whose share of `bytes` fits the budget: a hidden-tile
 // count (any) or a column count (a power of two dividing d / 8 and leaving at
-// least 256 columns).
-Chunks chunks_for(int d, int f, int T) {
+// least 256 columns). wbytes: the bytes of one gathered weight matrix.
+PassChunks pass_chunks(int d, int T, long long wbytes) {
   const long long budget = g_l2_budget.load();
-  const long long wbytes = 2LL * d * f;
-  Chunks c{};
+  PassChunks c{};
   c.nhc = static_cast<int>(std::min<long long>(T, std::max<long long>(1, (wbytes + budget - 1) / budget)));
   c.tpc = (T + c.nhc - 1) / c.nhc;
   auto cols = [&](long long bytes) {
@@ -772,6 +755,10 @@ Chunks chunks_for(int d, int f, int T) {
   return c;
 }
 
+namespace {
+
+PassChunks chunks_for(int d, int f, int T) { return pass_chunks(d, T, 2LL * d * f); }
+
 // The fused kernel gathers rows of all the direction's weights at once; the
 // passes pay for re-reading the token rows to keep fewer of them in L2, which
 // helps only when the weights are larger than L2 and the batch gathers each
@@ -781,18 +768,24 @@ Chunks chunks_for(int d, int f, int T) {
 // M=512 and 2048, the passes from M=4096 on).
 constexpr int kPassesMinRows = 4096;
 
-bool multi_pass(int M, int d, int f) {
+}  // namespace
+
+bool sparse_multi_pass(int M, int d, int f) {
   const int mode = g_sched_mode.load();
   if (mode != TWELL_SCHED_AUTO) return mode == TWELL_SCHED_PASSES;
   return 3LL * 2 * d * f > device_l2_bytes() && M >= kPassesMinRows;
 }
+
+namespace {
+
+bool multi_pass(int M, int d, int f) { return sparse_multi_pass(M, d, f); }
 
 cudaError_t launch_fwd_passes(int M, cudaStream_t s, const uint16_t* X, const uint16_t* W_u, const uint16_t* W_dt,
                               const uint16_t* count, const uint16_t* val, const uint8_t* col, int* plan, float* ubuf,
                               uint16_t* Y, int d, int f, int K, int* ctr, float* yacc, int* turn_x,
                               uint32_t* status) {
   const int T = f / kTn;
-  const Chunks ch = chunks_for(d, f, T);
+  const PassChunks ch = chunks_for(d, f, T);
   cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
   e = with_tok_shape(d, [&](auto cc, auto ww, auto ex) {
@@ -823,7 +816,7 @@ cudaError_t launch_bwd_passes(int M, cudaStream_t s, const uint16_t* dY, const u
                               int* plan, const int* n_ovf, const float* u_ell, float lambda, float4* hdz_ell,
                               float* dX, int d, int f, int K, int* ctr, int* turn_x, uint32_t* status) {
   const int T = f / kTn;
-  const Chunks ch = chunks_for(d, f, T);
+  const PassChunks ch = chunks_for(d, f, T);
   cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
   e = with_tok_shape(d, [&](auto cc, auto ww, auto ex) {

@@ -191,19 +191,30 @@ constexpr long long kDefaultL2Budget = 64LL << 20;
 // twell_set_sparse_schedule's implementation (mode and budget checked here).
 int set_sparse_schedule(int mode, long long l2_budget_bytes);
 
+// The multi-pass schedule's decision and chunking (shared by the bf16 and the
+// 8-bit kernels): whether a call with these sizes runs the passes, and the
+// chunks of passes gathering a weight matrix of `wbytes` bytes.
+struct PassChunks {
+  int nhc, tpc;  // hidden-tile chunks of the dot passes, tiles per chunk
+  int dw_y;      // column chunk width of a pass over one matrix
+  int dw_x;      // column chunk width of a pass over two matrices
+};
+bool sparse_multi_pass(int M, int d, int f);
+PassChunks pass_chunks(int d, int T, long long wbytes);
+
 // E4M3 codes of the rows of a bf16 matrix [rows][len] (len a multiple of 16),
 // one power-of-two scale per row (scale[r] = 2^e_r, e_r the smallest exponent
 // with max |W[r]| <= 448 * 2^e_r), and optionally the dequantised bf16 rows.
 cudaError_t launch_quantize_rows(const uint16_t* W, int rows, int len, uint8_t* q, float* scale, uint16_t* deq,
                                  cudaStream_t s);
 
-// The fused sparse up + down of launch_ell_ffn_fwd (row-level routing) with the
-// gathered rows read as E4M3 codes: W_u8 / s_u for the rows of W_u, W_dt8 / s_d
-// for the rows of W_d^T.
+// The sparse up + down of launch_ell_ffn_fwd (row-level routing; fused or
+// multi-pass as for the bf16 weights) with the gathered rows read as E4M3
+// codes: W_u8 / s_u for the rows of W_u, W_dt8 / s_d for the rows of W_d^T.
 cudaError_t launch_ell_ffn_fwd_q8(const uint16_t* X, const uint8_t* W_u8, const float* s_u, const uint8_t* W_dt8,
                                   const float* s_d, const uint16_t* count, const uint16_t* val, const uint8_t* col,
-                                  int* plan, float* u_ell, uint16_t* Y, int M, int d, int f, int K, int* ctr,
-                                  float* yacc, uint32_t* status, cudaStream_t s);
+                                  int* plan, float* u_ell, float* ubuf, uint16_t* Y, int M, int d, int f, int K,
+                                  int* ctr, float* yacc, int* turn_x, uint32_t* status, cudaStream_t s);
 
 // Split-K scratch of the dense-backup GEMMs (one GEMM at a time): fp32
 // partials and per-output-tile arrival words (any initial contents).

@@ -86,7 +86,7 @@ def parse_args():
                    help="schedule of the sparse kernels (twell_set_sparse_schedule)")
     p.add_argument("--l2-budget-mib", type=int, default=0,
                    help="L2 budget of one chunk of the multi-pass schedule, MiB (0: the library default)")
-    p.add_argument("--overlap", default="on", choices=["on", "off"],
+    p.add_argument("--overlap", default="off", choices=["on", "off"],
                    help="dense-backup GEMMs on the library's side stream beside the sparse kernels (twell_set_overlap)")
     return p.parse_args()
 
@@ -1261,7 +1261,7 @@ def run_block(args, local):
 def main():
     args = parse_args()
     world, rank, local = dist_env()
-    if args.impl != "reference" and (args.sched != "auto" or args.l2_budget_mib or args.overlap != "on"):
+    if args.impl != "reference" and (args.sched != "auto" or args.l2_budget_mib or args.overlap != "off"):
         apply_schedule(args)
     if args.block:
         run_block(args, local)

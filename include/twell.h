@@ -359,16 +359,16 @@ TWELL_API twell_status twell_set_sparse_schedule(int mode, int64_t l2_budget_byt
 
 /*
  * Overlap of the dense backup with the sparse kernels (a performance setting
- * with no counterpart on the pages; results do not change). When on (the
- * default), twell_ffn_fwd, twell_ffn_fwd_e4m3 and twell_ffn_bwd run the
+ * with no counterpart on the pages; results do not change). When on,
+ * twell_ffn_fwd, twell_ffn_fwd_e4m3 and twell_ffn_bwd run the
  * dense-backup chain (the overflow rows' GEMMs and their gathers) on a second
  * stream owned by the library, created per device at first use at the
  * highest stream priority, forked from the caller's stream after the routing
  * and joined back into it before the call's remaining kernels; the sparse
  * kernels stay on the caller's stream and use what the GEMM leaves of each
  * SM. The call stays asynchronous and stream-ordered for the caller, and is
- * capturable into a CUDA graph. 0 runs every kernel on the caller's stream.
- * Process-wide; applies to the calls made after it returns.
+ * capturable into a CUDA graph. 0 (the default) runs every kernel on the
+ * caller's stream. Process-wide; applies to the calls made after it returns.
  */
 TWELL_API void twell_set_overlap(int on);
 

@@ -302,7 +302,7 @@ def test_overlap_agrees_and_captures(tw):
                 assert torch.equal(a, b), name + " (graph replay)"
             del graph
         finally:
-            tw.set_overlap(True)
+            tw.set_overlap(False)
 
 
 def test_prepared_wdt_matches(tw):

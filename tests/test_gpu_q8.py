@@ -102,3 +102,31 @@ def test_fwd_e4m3_sweep_scale(tw, orc):
     seeded sample of rows plus every overflow row."""
     gap = _check_q8_forward(tw, orc, sweep_workload(8192, 0.01), sample=256)
     assert gap["rel_l2"] < 0.1  # E4M3 keeps 4 significant bits: a few percent, not a different function
+
+
+@pytest.mark.parametrize("name", ["ragged", "heavy_small", "wide_d_w4", "min_d_model"])
+def test_fwd_e4m3_schedules_agree(tw, name):
+    """The 8-bit forward under the fused and the multi-pass schedule (the latter
+    also with a 64 KiB L2 budget, so the passes run in many hidden-tile and
+    column chunks): Y bit-identical, for an inference forward (u in the
+    workspace) and with u saved."""
+    M, d, f, K, act, rs, seed = CASES[name]
+    w = Workload(name, M, d, f, 128, K, act, row_scale=rs, training=True, seed=seed)
+    inp = make_inputs(w)
+    D = {k: to_dev(v) for k, v in inp.items() if k != "meta"}
+    q8 = tw.quantize_weights(D["W_u"], D["W_d"])
+    outs = {}
+    try:
+        for label, mode, budget in (("fused", tw.SCHED_FUSED, 0), ("passes", tw.SCHED_PASSES, 0),
+                                    ("chunked", tw.SCHED_PASSES, 64 << 10)):
+            tw.set_sparse_schedule(mode, budget)
+            Y, st = tw.ffn_fwd_e4m3(D["X"], D["W_g"], D["b_g"], q8, K=K)
+            Ys, sts = tw.ffn_fwd_e4m3(D["X"], D["W_g"], D["b_g"], q8, K=K, save_for_backward=True)
+            torch.cuda.synchronize()
+            assert st.read_status() == 0 and sts.read_status() == 0, label
+            outs[label] = (Y, Ys)
+    finally:
+        tw.set_sparse_schedule(tw.SCHED_AUTO, 0)
+    for label in ("passes", "chunked"):
+        for a, b in zip(outs["fused"], outs[label]):
+            assert torch.equal(a, b), label
