@@ -12,6 +12,7 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
   ffn_fwd           pinned: brute-force loops, torch float64, closed forms
   ffn_fwd_hybrid    pinned: equals ffn_fwd (round_g=1) on the same active set
   ffn_bwd           pinned: torch float64 autograd, closed form of the L1 term
+  ffn_bwd_units     pinned: equals ffn_bwd (C) on the listed units, given the same g
   gmat input        pinned: with gmat = the oracle's own packed g, equals round_g
   e4m3_value        pinned: torch's float8_e4m3fn reading of all 256 codes
   e4m3_round        pinned: brute-force nearest code with the tie rule; torch's cast
@@ -289,4 +290,41 @@ def ffn_bwd(X, W_g, b_g, W_u, W_d, dY, lam: float = 0.0, mask=None, round_g: boo
                               out["dX"], out["dW_g"], out["dW_u"], out["dW_d"], _ptr(out["db_g"]))
     if rc:
         raise MemoryError("oracle_ffn_bwd")
+    return out
+
+
+def ffn_bwd_units(X, W_u, W_d, dY, lam: float, units, gcols) -> dict:
+    """The weight gradients of the listed hidden units only, for L = sum(Y * dY)
+    + lam * sum(g) ("Sakana AI и NVIDIA представили TwELL", paragraph 2: the
+    backward over the hybrid format; the formulas of ffn_bwd restricted to unit j):
+        dW_u[j] = sum_i dU_ij x_i,  dW_g[j] = sum_i dZ_ij x_i,
+        dW_d[:, j] = sum_i h_ij dY_i,  db_g[j] = sum_i dZ_ij,
+    over the rows i where unit j is active, with g_ij given as the stored bf16
+    value (gcols [M, len(units)] bit patterns; active iff nonzero, as ffn_bwd's
+    gmat), u_ij = x_i . W_u[j], dH_ij = dY_i . W_d[:, j], dU = dH g,
+    dZ = dH u + lam, h = g u. float64; numpy's matrix products as the sums.
+    Returns dW_g, dW_u [n, d], dW_d [d, n] and db_g [n] for the n listed units."""
+    X, W_u, W_d, dY = (_c(a, np.uint16) for a in (X, W_u, W_d, dY))
+    units = np.asarray(units, np.int64)
+    gcols = np.asarray(gcols, np.uint16)
+    M, d = X.shape
+    n = units.size
+    if gcols.shape != (M, n):
+        raise ValueError("gcols must be [M, len(units)]")
+    out = dict(dW_g=np.zeros((n, d)), dW_u=np.zeros((n, d)), dW_d=np.zeros((d, n)), db_g=np.zeros(n))
+    for k, j in enumerate(units):
+        rows = np.nonzero(gcols[:, k])[0]
+        if rows.size == 0:
+            continue
+        g = bf16_to_f64(gcols[rows, k])
+        x = bf16_to_f64(X[rows])
+        dy = bf16_to_f64(dY[rows])
+        u = x @ bf16_to_f64(W_u[j])
+        dh = dy @ bf16_to_f64(W_d[:, j])
+        du = dh * g
+        dz = dh * u + lam
+        out["dW_u"][k] = du @ x
+        out["dW_g"][k] = dz @ x
+        out["dW_d"][:, k] = (g * u) @ dy
+        out["db_g"][k] = dz.sum()
     return out

@@ -372,6 +372,40 @@ def test_gmat_input_equals_stored_g_definition(orc):
     assert np.array_equal(orc.ffn_fwd(X, Wg, bg, Wu, Wd, rows=rows, gmat=G[rows]), y1[rows])
 
 
+def test_bwd_units_equals_full_backward(orc):
+    """ffn_bwd_units (the weight gradients of listed units, numpy) against the C
+    oracle's full backward given the same stored g: the same numbers to rounding
+    order, for units active in many rows, in one row and in none, and lambda != 0;
+    and a unit's gradients move by the definition when its g doubles in one row."""
+    X, Wg, bg, Wu, Wd, dY = _problem(31, 40, 64, 256, -0.5)
+    Z = orc.gate(X, Wg, bg)
+    G = orc.unpack(orc.pack(Z, 128, 8), 256, 128, 8)
+    G[:, 7] = 0           # a unit active nowhere
+    G[1:, 9] = 0          # a unit active in row 0 only (if at all)
+    full = orc.ffn_bwd(X, Wg, bg, Wu, Wd, dY, 0.03, gmat=G)
+    units = np.array([0, 5, 7, 9, 130, 255])
+    part = orc.ffn_bwd_units(X, Wu, Wd, dY, 0.03, units, G[:, units])
+    for k in ("dW_g", "dW_u"):
+        ref = full[k][units]
+        assert np.abs(part[k] - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max()), k
+    ref = full["dW_d"][:, units]
+    assert np.abs(part["dW_d"] - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
+    assert np.abs(part["db_g"] - full["db_g"][units]).max() <= 1e-12 * max(1.0, np.abs(full["db_g"]).max())
+    assert not part["dW_u"][2].any() and part["db_g"][2] == 0.0
+    # doubling g_ij doubles row i's term of dW_u[j] (dU = dH g) and of dW_d[:, j] (h = g u)
+    i = int(np.nonzero(G[:, 5])[0][0])
+    G2 = G.copy()
+    G2[i, 5] = bf16_bits_from_f64(2 * _f64(G[i:i + 1, 5:6]))[0, 0]
+    a = orc.ffn_bwd_units(X, Wu, Wd, dY, 0.03, [5], G[:, [5]])
+    b = orc.ffn_bwd_units(X, Wu, Wd, dY, 0.03, [5], G2[:, [5]])
+    x, wu, wd, dy = _f64(X), _f64(Wu), _f64(Wd), _f64(dY)
+    gij = _f64(G[i:i + 1, 5:6])[0, 0]
+    dh = dy[i] @ wd[:, 5]
+    assert np.abs((b["dW_u"][0] - a["dW_u"][0]) - dh * gij * x[i]).max() < 1e-10
+    assert np.abs((b["dW_d"][:, 0] - a["dW_d"][:, 0]) - gij * (x[i] @ wu[5]) * dy[i]).max() < 1e-10
+    assert np.abs(b["dW_g"] - a["dW_g"]).max() == 0.0  # dZ does not depend on g's value
+
+
 def test_count_stats_hand_counted(orc):
     """Bins counted by hand for a 3-row, 2-tile batch with T_n = 4."""
     count = np.array([[1, 3], [0, 0], [4, 2]], dtype=np.uint16)
