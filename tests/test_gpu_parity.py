@@ -16,7 +16,8 @@ import pytest
 
 from synthetic import WORKLOADS, Workload, make_inputs, sweep_workload
 from twell_testlib import (assert_active_set, assert_gate_close, assert_matches_oracle, assert_pack_equal,
-                           assert_plan_valid, bits_of, f32_of_bits, gate_error_bound, gpu_gmat, state_to_numpy, to_dev)
+                           assert_plan_valid, bits_of, f32_of_bits, gate_error_bound, gpu_gmat, gpu_gmat_cols,
+                           gpu_gmat_rows, state_to_numpy, to_dev)
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -572,6 +573,67 @@ def test_sweep_scale_training(tw, orc, activity):
     torch.cuda.synchronize()
     assert st.read_status() == 0
     _check_bwd(orc, inp, g, G, 1e-3, w.name, per_row=True)
+
+
+def test_headline_full_size(tw, orc):
+    """The benchmark's headline workload at full size, in its launch configuration:
+    d_model=4096, d_ff=14336, M=65536 tokens, 99% sparsity, lognormal rows, K=8,
+    dense-backup capacity M/4, the default (multi-pass) schedule, a training step
+    with lambda = 1e-3. On a seeded sample of 192 rows plus 64 overflow rows: the
+    pack bit-exact against the oracle's pack of the GPU's z, z element by element,
+    Y and dX against the oracle given the GPU's stored g. The weight gradients of
+    16 units (12 seeded, 4 active in overflow rows) against the oracle's
+    per-unit gradients over all 65536 rows."""
+    w = WORKLOADS["large"]
+    inp = make_inputs(w)
+    M, d, f, K, T_n = w.M, w.d_model, w.d_ff, w.K, w.T_n
+    D = _dev(inp)
+    Y, st, z = tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], T_n=T_n, K=K, ovf_cap=M // 4,
+                          save_for_backward=True, z_debug=True)
+    g = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=1e-3)
+    torch.cuda.synchronize()
+    assert st.read_status() == 0
+    p = state_to_numpy(st)
+    n = p["n_ovf"]
+    assert n > 1000 and p["n_ovf_total"] == n
+    plan = assert_plan_valid(st)
+    assert plan["dense_wgrad"] and plan["split_rows"] > 0
+    rows = _sample_rows(M, 192, 11, extra=p["ovf_rows"][:n][:: max(1, n // 64)][:64])
+    zr = z[torch.from_numpy(rows.astype(np.int64)).to(z.device)].cpu().numpy()
+    del z
+    # pack of the sampled rows (row-local) against the oracle's pack of the GPU's z
+    ref = orc.pack(zr.astype(np.float64), T_n, K)
+    for k in ("count", "val", "col", "row_ovf"):
+        assert np.array_equal(p[k][rows], ref[k]), k
+    is_ovf = p["row_ovf"][rows] != 0
+    slots = np.searchsorted(p["ovf_rows"][:n], rows[is_ovf])
+    assert np.array_equal(p["g_ovf"][slots], ref["g_ovf"][:ref["n_ovf"]])
+    # gate output on the sampled rows
+    z64 = orc.gate(inp["X"], inp["W_g"], inp["b_g"], rows=rows)
+    assert_gate_close(zr, z64, gate_error_bound(inp["X"], inp["W_g"], inp["b_g"], rows=rows))
+    assert_active_set(zr, z64, float(np.sqrt(np.mean(z64 ** 2))))
+    # Y and dX on the sampled rows (both row-local), given the GPU's stored g
+    Gr = gpu_gmat_rows(p, rows, f, T_n, K)
+    assert np.array_equal(Gr, orc.unpack(ref, f, T_n, K))
+    args = (inp["X"], inp["W_g"], inp["b_g"], inp["W_u"], inp["W_d"])
+    yg = f32_of_bits(bits_of(Y))[rows]
+    assert_matches_oracle(yg, orc.ffn_fwd(*args, rows=rows, gmat=Gr), orc.ffn_fwd(*args, rows=rows), "headline Y",
+                          bf16_out=True, per_row=True)
+    Xs, dYs = inp["X"][rows], inp["dY"][rows]
+    sub = (Xs, inp["W_g"], inp["b_g"], inp["W_u"], inp["W_d"], dYs, 1e-3)
+    assert_matches_oracle(g["dX"].cpu().numpy()[rows], orc.ffn_bwd(*sub, gmat=Gr)["dX"],
+                          orc.ffn_bwd(*sub, mask=(Gr != 0).astype(np.uint8))["dX"], "headline dX", per_row=True)
+    # the weight gradients of sampled units over every row
+    rng = np.random.default_rng(12)
+    busy = np.nonzero(p["g_ovf"][:n].any(axis=0))[0]
+    units = np.unique(np.concatenate([rng.choice(f, 12, replace=False), rng.choice(busy, 4, replace=False)]))
+    ru = orc.ffn_bwd_units(inp["X"], inp["W_u"], inp["W_d"], inp["dY"], 1e-3, units,
+                           gpu_gmat_cols(p, units, M, T_n, K))
+    ut = torch.from_numpy(units).to(g["dW_u"].device)
+    for k, a in (("dW_g", g["dW_g"][ut]), ("dW_u", g["dW_u"][ut]), ("dW_d", g["dW_d"][:, ut].t())):
+        o = ru[k] if k != "dW_d" else ru[k].T
+        assert_matches_oracle(a.cpu().numpy(), o, o, f"headline {k} (sampled units)", per_row=True)
+    assert_matches_oracle(g["db_g"][ut].cpu().numpy(), ru["db_g"], ru["db_g"], "headline db_g (sampled units)")
 
 
 def test_split_epilogue_barrier_gives_up(tw):

@@ -136,6 +136,38 @@ def gpu_gmat(p: dict, M: int, f: int, T_n: int, K: int) -> np.ndarray:
     return G
 
 
+def gpu_gmat_rows(p: dict, rows, f: int, T_n: int, K: int) -> np.ndarray:
+    """gpu_gmat restricted to the listed rows ([len(rows), f] bf16 bits)."""
+    rows = np.asarray(rows, np.int64)
+    G = np.zeros((rows.size, f), np.uint16)
+    cnt = np.minimum(p["count"][rows].astype(np.int64), K)
+    rr, tt, ss = np.nonzero(np.arange(K)[None, None, :] < cnt[:, :, None])
+    ell = p["row_ovf"][rows[rr]] == 0
+    rr, tt, ss = rr[ell], tt[ell], ss[ell]
+    G[rr, tt * T_n + p["col"][rows[rr], tt, ss].astype(np.int64)] = p["val"][rows[rr], tt, ss]
+    n = p["n_ovf"]
+    is_ovf = p["row_ovf"][rows] != 0
+    slots = np.searchsorted(p["ovf_rows"][:n], rows[is_ovf])
+    G[np.nonzero(is_ovf)[0]] = p["g_ovf"][slots]
+    return G
+
+
+def gpu_gmat_cols(p: dict, units, M: int, T_n: int, K: int) -> np.ndarray:
+    """gpu_gmat restricted to the listed units ([M, len(units)] bf16 bits)."""
+    units = np.asarray(units, np.int64)
+    G = np.zeros((M, units.size), np.uint16)
+    ell = p["row_ovf"][:M] == 0
+    for k, j in enumerate(units):
+        t, c = divmod(int(j), T_n)
+        cnt = np.minimum(p["count"][:, t].astype(np.int64), K)
+        hit = (np.arange(K)[None, :] < cnt[:, None]) & (p["col"][:, t, :] == c) & ell[:, None]
+        ii, ss = np.nonzero(hit)
+        G[ii, k] = p["val"][ii, t, ss]
+    n = p["n_ovf"]
+    G[p["ovf_rows"][:n]] = p["g_ovf"][:n][:, units]
+    return G
+
+
 def output_rounding(o: np.ndarray) -> np.ndarray:
     """|bf16(o) - o| per element: how far rounding the exact value to the bf16
     output format moves it (round to nearest even, by the oracle's rounding)."""
