@@ -26,6 +26,7 @@ namespace {
 
 constexpr int kStages = 4;
 constexpr int kPairStages = 6;  // 32 KB per stage on a CTA pair (A 128 x 64 and half of B)
+constexpr int kStages128 = 6;   // 128 x 128 tiles of the one-CTA engine: 32 KB per stage
 
 __device__ __forceinline__ void load_bias32(const uint16_t* b, float (&out)[32]) {
   const uint4* p = reinterpret_cast<const uint4*>(b);
@@ -63,6 +64,7 @@ struct EpiTwell {
   // per-thread slot staging: K bf16 values + K column bytes (K <= 64)
   static constexpr int SMEM_BYTES = 128 * kMaxK * 3;
   static constexpr bool kSplitK = false;
+  static constexpr bool kReduceAhead = false;  // split-K reduction with one item of lookahead
 
   __device__ static void run(const Args& a, int m0, int n0, int M_eff, int /*N*/, int r, uint32_t taddr,
                              uint8_t* smem) {
@@ -246,6 +248,7 @@ struct EpiGateMul {
   };
   static constexpr int SMEM_BYTES = kApplySmemBytes;
   static constexpr bool kSplitK = true;
+  static constexpr bool kReduceAhead = false;  // split-K reduction with one item of lookahead
   struct In {
     uint4 g;
   };
@@ -285,6 +288,7 @@ struct EpiScatterBf16 {
   };
   static constexpr int SMEM_BYTES = kApplySmemBytes;
   static constexpr bool kSplitK = true;
+  static constexpr bool kReduceAhead = true;  // split-K reduction with one item of lookahead
   struct In {
     int dst;
   };
@@ -312,6 +316,7 @@ struct EpiScatterF32 {
   };
   static constexpr int SMEM_BYTES = kApplySmemBytes;
   static constexpr bool kSplitK = true;
+  static constexpr bool kReduceAhead = true;  // split-K reduction with one item of lookahead
   struct In {
     int dst;
   };
@@ -355,6 +360,7 @@ struct EpiBwdDH {
   };
   static constexpr int SMEM_BYTES = kApplySmemBytes;
   static constexpr bool kSplitK = true;
+  static constexpr bool kReduceAhead = false;  // split-K reduction with one item of lookahead
   __device__ static void hi_lo(const float (&v)[8], uint4& hi, uint4& lo) {
     float h[8], l[8];
 #pragma unroll
@@ -431,6 +437,7 @@ struct EpiStoreF32 {
   };
   static constexpr int SMEM_BYTES = kApplySmemBytes;
   static constexpr bool kSplitK = false;
+  static constexpr bool kReduceAhead = false;  // split-K reduction with one item of lookahead
   struct In {};
   __device__ static void load8(const Args&, int, int, In&) {}
   __device__ static void apply8(const Args& a, int row, int n, const float (&v)[8], const In&) {
@@ -484,7 +491,10 @@ void use_split(GemmShape& shp, const SplitKBuffers& sk, int cap) {
 // the one that does not own the count returns at once (no host synchronisation
 // learns the count). b_pair is B's tensor map with 128-row boxes for the pair
 // engine (the same map as b when B is MN-major).
-template <class Epi, bool B_MN, bool A_MN = false>
+// BN1 = 128: the one-CTA engine runs 128 x 128 tiles (B's map must then have
+// 128-row boxes), for a GEMM whose N gives too few 256-wide tiles to occupy
+// the GPU when only a few rows overflow: twice the CTAs streaming the weight.
+template <class Epi, bool B_MN, bool A_MN = false, int BN1 = 256>
 cudaError_t launch_rows_gemm(const char* name, const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
                              const CUtensorMap& b1, const CUtensorMap& b0_pair, const CUtensorMap& b1_pair,
                              GemmShape shp, const typename Epi::Args& ea, int cap, cudaStream_t s) {
@@ -495,7 +505,11 @@ cudaError_t launch_rows_gemm(const char* name, const CUtensorMap& a0, const CUte
 #endif
   GemmShape one = shp;
   if (pair) one.max_rows = kSplitRows;
-  cudaError_t e = launch_umma_gemm<Epi, 256, B_MN, kStages, A_MN>(name, a0, b0, a1, b1, one, ea, s);
+  cudaError_t e;
+  if constexpr (BN1 == 128)
+    e = launch_umma_gemm<Epi, 128, B_MN, kStages128, A_MN>(name, a0, b0, a1, b1, one, ea, s);
+  else
+    e = launch_umma_gemm<Epi, 256, B_MN, kStages, A_MN>(name, a0, b0, a1, b1, one, ea, s);
   if (e != cudaSuccess || !pair) return e;
   GemmShape two = shp;
   two.partial = nullptr;
@@ -525,7 +539,10 @@ cudaError_t launch_ovf_fwd(const uint16_t* x_ovf, const uint16_t* W_u, const uin
   GemmShape s1{cap, n_ovf, f, d, 0, status};
   use_split(s1, sk, cap);
   EpiGateMul::Args e1{g_ovf, h_ovf, u_ovf, f};
-  cudaError_t e = launch_rows_gemm<EpiGateMul, false>("ovf_up_gemm", ta, tb, ta, tb, tbp, tbp, s1, e1, cap, s);
+  cudaError_t e = f / 256 < device_sm_count() / 2
+                      ? launch_rows_gemm<EpiGateMul, false, false, 128>("ovf_up_gemm", ta, tbp, ta, tbp, tbp, tbp, s1,
+                                                                        e1, cap, s)
+                      : launch_rows_gemm<EpiGateMul, false>("ovf_up_gemm", ta, tb, ta, tb, tbp, tbp, s1, e1, cap, s);
   if (e != cudaSuccess) return e;
   GemmShape s2{cap, n_ovf, d, f, 0, status};
   use_split(s2, sk, cap);
@@ -555,7 +572,10 @@ cudaError_t launch_ovf_bwd(const uint16_t* dy_ovf, const uint16_t* W_dt, const u
   use_split(s1, sk, cap);
   EpiBwdDH::Args e1{g_ovf, u_ovf, plan, op.duz_hi, op.duz_hi + static_cast<size_t>(cap_r) * 2 * f, op.h_hi,
                     op.h_hi + static_cast<size_t>(cap_r) * f, du_ovf, dz_ovf, lambda, f};
-  cudaError_t e = launch_rows_gemm<EpiBwdDH, false>("ovf_dh_gemm", ta, tb, ta, tb, tbp, tbp, s1, e1, cap, s);
+  cudaError_t e = f / 256 < device_sm_count() / 2
+                      ? launch_rows_gemm<EpiBwdDH, false, false, 128>("ovf_dh_gemm", ta, tbp, ta, tbp, tbp, tbp, s1, e1,
+                                                                      cap, s)
+                      : launch_rows_gemm<EpiBwdDH, false>("ovf_dh_gemm", ta, tb, ta, tb, tbp, tbp, s1, e1, cap, s);
   if (e != cudaSuccess) return e;
   GemmShape s2{cap, n_ovf, d, f, f, status};
   use_split(s2, sk, cap);

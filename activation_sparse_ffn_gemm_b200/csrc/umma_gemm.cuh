@@ -359,7 +359,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
       if (split == 1) {
-        Epi::run(ea, mb * kBM, nb * BN, M_eff, shp.N, r, taddr, epi_smem);
+        // the tile's columns end at n0 + BN (or N): an epilogue that walks
+        // 32-column chunks stops there
+        Epi::run(ea, mb * kBM, nb * BN, M_eff, min(shp.N, (nb + 1) * BN), r, taddr, epi_smem);
       } else {
         // fp32 partial of K range ks for this accumulator row
         const int row = mb * kBM + r;
@@ -413,12 +415,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             __threadfence();
             const int rows_here = min(kBM, M_eff - mb * kBM);
             const int items = rows_here * (BN / 8);
-#pragma unroll 1
-            for (int it = r; it < items; it += kBM) {
+            // item it: (row, 8-column chunk) of the tile; its partials from
+            // every range, loaded together
+            auto load_item = [&](int it, float4 (&pa)[kSplitMax], float4 (&pb)[kSplitMax]) {
               const int row2 = mb * kBM + it / (BN / 8);
               const int n = nb * BN + (it % (BN / 8)) * 8;
-              if (n >= shp.N) continue;
-              float4 pa[kSplitMax], pb[kSplitMax];
+              if (n >= shp.N) return;
 #pragma unroll
               for (int k2 = 0; k2 < kSplitMax; ++k2) {
                 if (k2 < split) {
@@ -428,6 +430,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                   pb[k2] = __ldcg(p + 1);
                 }
               }
+            };
+            auto apply_item = [&](int it, const float4 (&pa)[kSplitMax], const float4 (&pb)[kSplitMax]) {
+              const int row2 = mb * kBM + it / (BN / 8);
+              const int n = nb * BN + (it % (BN / 8)) * 8;
+              if (n >= shp.N) return;
               float accv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
               for (int k2 = 0; k2 < kSplitMax; ++k2) {
@@ -437,6 +444,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
               }
               Epi::apply8(ea, row2, n, accv);
+            };
+            if constexpr (Epi::kReduceAhead) {
+              // the next item's partials are in flight while this one is applied
+              float4 pa[kSplitMax], pb[kSplitMax], qa[kSplitMax], qb[kSplitMax];
+              int it = r;
+              if (it < items) load_item(it, pa, pb);
+#pragma unroll 1
+              for (; it < items; it += kBM) {
+                const bool more = it + kBM < items;
+                if (more) load_item(it + kBM, qa, qb);
+                apply_item(it, pa, pb);
+                if (more) {
+#pragma unroll
+                  for (int k2 = 0; k2 < kSplitMax; ++k2) {
+                    pa[k2] = qa[k2];
+                    pb[k2] = qb[k2];
+                  }
+                }
+              }
+            } else {
+#pragma unroll 1
+              for (int it = r; it < items; it += kBM) {
+                float4 pa[kSplitMax], pb[kSplitMax];
+                load_item(it, pa, pb);
+                apply_item(it, pa, pb);
+              }
             }
           }
         }
