@@ -248,11 +248,15 @@ __global__ void __launch_bounds__(256) csc_fill_kernel(
 // to back; entries come from shared-memory broadcasts and accumulation uses the
 // two-lane FMA. Each unit's sums are taken in list order, whichever warp runs
 // it, so the result is the same on every run. dW_d[:, j] is transposed through
-// shared memory so that each output row gets 8 consecutive units (32 bytes).
+// shared memory so that each output row gets the CTA's consecutive units (32
+// bytes for 8).
 constexpr int kWgBatch = 4;   // pairs whose row loads are issued together (2, 6, 8 measured slower)
 constexpr int kWgChunks = 2;  // 16-byte chunks per lane and row: per-pair work amortised over 2 chunks
 constexpr int kWgCols = 256 * kWgChunks;
-constexpr int kWgUnits = 8;   // units per CTA
+#ifndef TWELL_WG_UNITS
+#define TWELL_WG_UNITS 8
+#endif
+constexpr int kWgUnits = TWELL_WG_UNITS;  // units per CTA (a multiple of 4)
 constexpr int kWgWarps = 4;   // warps per CTA
 constexpr int kWgMinBlocks = kWgChunks == 1 ? 6 : 4;
 
@@ -269,7 +273,10 @@ __global__ void __launch_bounds__(kWgWarps * 32, kWgMinBlocks) wgrad_kernel(cons
                                                                             float* __restrict__ dWu,
                                                                             float* __restrict__ dWd,
                                                                             float* __restrict__ dbg) {
-  __shared__ float s_dwd[kWgCols][kWgUnits + 1];
+  // dW_d sums of the CTA's units, unit-major with a 4-word pad: each lane
+  // stores its 8 consecutive columns as two 16-byte words, and the write-out
+  // reads one word per (row, unit), both without bank conflicts beyond 2-way
+  __shared__ __align__(16) float s_dwd[kWgUnits][kWgCols + 4];
   __shared__ int s_row[kWgWarps][32];
   __shared__ float4 s_val[kWgWarps][32];
   __shared__ int s_order[kWgUnits];
@@ -397,11 +404,9 @@ __global__ void __launch_bounds__(kWgWarps * 32, kWgMinBlocks) wgrad_kernel(cons
         pg[0] = g0;
         pg[1] = g1;
       }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        s_dwd[256 * q + lane * 8 + 2 * e][lu] = ad[q][e].x;
-        s_dwd[256 * q + lane * 8 + 2 * e + 1][lu] = ad[q][e].y;
-      }
+      float4* sd = reinterpret_cast<float4*>(&s_dwd[lu][256 * q + lane * 8]);
+      sd[0] = make_float4(ad[q][0].x, ad[q][0].y, ad[q][1].x, ad[q][1].y);
+      sd[1] = make_float4(ad[q][2].x, ad[q][2].y, ad[q][3].x, ad[q][3].y);
     }
     if (blockIdx.y == 0 && lane == 0 && dbg != nullptr) dbg[j] = db_extra ? db + db_extra[j] : db;
   }
@@ -410,15 +415,15 @@ __global__ void __launch_bounds__(kWgWarps * 32, kWgMinBlocks) wgrad_kernel(cons
     const int cc = c0 + r;
     if (cc >= d) continue;
     float4* pd = reinterpret_cast<float4*>(dWd + static_cast<long>(cc) * f + j0);
-    float4 d0 = make_float4(s_dwd[r][0], s_dwd[r][1], s_dwd[r][2], s_dwd[r][3]);
-    float4 d1 = make_float4(s_dwd[r][4], s_dwd[r][5], s_dwd[r][6], s_dwd[r][7]);
-    if (acc_old) {
-      const float4 o0 = pd[0], o1 = pd[1];
-      d0 = make_float4(o0.x + d0.x, o0.y + d0.y, o0.z + d0.z, o0.w + d0.w);
-      d1 = make_float4(o1.x + d1.x, o1.y + d1.y, o1.z + d1.z, o1.w + d1.w);
+#pragma unroll
+    for (int k = 0; k < kWgUnits / 4; ++k) {
+      float4 v = make_float4(s_dwd[4 * k][r], s_dwd[4 * k + 1][r], s_dwd[4 * k + 2][r], s_dwd[4 * k + 3][r]);
+      if (acc_old) {
+        const float4 o = pd[k];
+        v = make_float4(o.x + v.x, o.y + v.y, o.z + v.z, o.w + v.w);
+      }
+      pd[k] = v;
     }
-    pd[0] = d0;
-    pd[1] = d1;
   }
 }
 
