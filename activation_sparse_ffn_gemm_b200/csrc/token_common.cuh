@@ -60,7 +60,7 @@ __device__ __forceinline__ void row_offsets(const uint16_t* __restrict__ count, 
     const int t = t0 + lane;
     int c = 0;
     if (t < T) {
-      c = count[row * T + t];
+      c = __ldcs(count + row * T + t);  // read once per piece and chunk: streamed past L2's weight rows
       if (TILES) g.tcnt[t] = static_cast<uint16_t>(c);
       else c = c < K ? c : K;
     }
@@ -112,11 +112,11 @@ __device__ __forceinline__ void build_list(GroupSmem& g, long row, int T, int K,
     int t, sl;
     entry_of(g.off, T, e0 + e, t, sl);
     const long base = (row * T + t) * K + sl;
-    const int c = col[base];
+    const int c = __ldcs(col + base);
     const bool ok = in_bounds(c < kTn, status);
     g.j[e] = t * kTn + (ok ? c : 0);
-    g.c[e] = ok ? __uint_as_float(static_cast<uint32_t>(val[base]) << 16) : 0.f;
-    if (u_ell) g.c2[e] = u_ell[base];
+    g.c[e] = ok ? __uint_as_float(static_cast<uint32_t>(__ldcs(val + base)) << 16) : 0.f;
+    if (u_ell) g.c2[e] = __ldcs(u_ell + base);
     g.slot[e] = t * K + sl;
   }
 }
@@ -186,6 +186,8 @@ __device__ __forceinline__ bool next_piece(int* ctr, const int* plan, int M, con
   group_sync<W>(grp);
   return true;
 }
+
+__device__ __forceinline__ float4 ldcs_f4(const float4* p) { return __ldcs(p); }
 
 // Entries [e0, e0 + ne) of the group's piece that lie in hidden-tile chunk
 // g.ch of tpc tiles (the multi-pass schedule's dot passes).

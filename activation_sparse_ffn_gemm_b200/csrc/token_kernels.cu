@@ -245,15 +245,27 @@ __device__ __forceinline__ void add_acc(const float* __restrict__ acc, int first
   }
 }
 
-template <int C, int W, bool EXACT>
+// FINAL: the row's final values (dX), stored with the streaming hint so that
+// they do not displace the gathered weight rows from L2; otherwise a partial
+// sum that the row's next piece reads back.
+template <int C, int W, bool EXACT, bool FINAL = false>
 __device__ __forceinline__ void store_acc(float* __restrict__ acc, int first, int nch, const float2 (&y)[C][4]) {
   float4* p = reinterpret_cast<float4*>(acc);
 #pragma unroll
   for (int q = 0; q < C; ++q) {
     const int idx = first + W * 32 * q;
     if (EXACT || idx < nch) {
-      p[2 * idx] = make_float4(y[q][0].x, y[q][0].y, y[q][1].x, y[q][1].y);
-      p[2 * idx + 1] = make_float4(y[q][2].x, y[q][2].y, y[q][3].x, y[q][3].y);
+      const float4 a = make_float4(y[q][0].x, y[q][0].y, y[q][1].x, y[q][1].y);
+      const float4 b = make_float4(y[q][2].x, y[q][2].y, y[q][3].x, y[q][3].y);
+#if TWELL_STREAM_HINTS
+      if (FINAL) {
+        __stcs(p + 2 * idx, a);
+        __stcs(p + 2 * idx + 1, b);
+        continue;
+      }
+#endif
+      p[2 * idx] = a;
+      p[2 * idx + 1] = b;
     }
   }
 }
@@ -437,11 +449,12 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, 512 / (TokCfg<C, W>:
       const int rw = g.row, q = g.q, P = g.P;
       float* acc = dX + static_cast<long>(rw) * d;
       if (P == 1) {
-        store_acc<C, W, EXACT>(acc, first, nch, dx);
+        store_acc<C, W, EXACT, true>(acc, first, nch, dx);
       } else {
         turn_wait<W>(turn, rw, q, grp, gtid, status);
         if (q > 0) add_acc<C, W, EXACT>(acc, first, nch, dx);
-        store_acc<C, W, EXACT>(acc, first, nch, dx);
+        if (q + 1 == P) store_acc<C, W, EXACT, true>(acc, first, nch, dx);
+        else store_acc<C, W, EXACT>(acc, first, nch, dx);
         turn_pass<W>(turn, rw, q, P, grp, gtid);
       }
     }
@@ -496,10 +509,10 @@ __device__ __forceinline__ void build_list_hdz(GroupSmem& g, long row, int T, in
     int t, sl;
     entry_of(g.off, T, e0 + e, t, sl);
     const long base = (row * T + t) * K + sl;
-    const int c = col[base];
+    const int c = __ldcs(col + base);
     const bool ok = in_bounds(c < kTn, status);
     g.j[e] = t * kTn + (ok ? c : 0);
-    const float4 v = hdz[base];
+    const float4 v = ldcs_f4(hdz + base);
     g.c[e] = ok ? v.y : 0.f;
     g.c2[e] = ok ? v.z : 0.f;
     g.slot[e] = t * K + sl;
@@ -680,12 +693,13 @@ __global__ void __launch_bounds__(TokCfg<C, W>::WARPS * 32, dx_threads_per_sm<C>
     const int rw = g.row, q = g.q, P = g.P;
     float* acc = dX + static_cast<long>(rw) * d + c0;
     if (P == 1) {
-      store_acc<C, W, EXACT>(acc, gtid, nch, dx);
+      store_acc<C, W, EXACT, true>(acc, gtid, nch, dx);
     } else {
       int* turn = turn_x ? turn_x + static_cast<long>(g.ch) * M : plan + kPlanHdr;
       turn_wait<W>(turn, rw, q, grp, gtid, status);
       if (q > 0) add_acc<C, W, EXACT>(acc, gtid, nch, dx);
-      store_acc<C, W, EXACT>(acc, gtid, nch, dx);
+      if (q + 1 == P) store_acc<C, W, EXACT, true>(acc, gtid, nch, dx);
+      else store_acc<C, W, EXACT>(acc, gtid, nch, dx);
       turn_pass<W>(turn, rw, q, P, grp, gtid);
     }
     group_sync<W>(grp);

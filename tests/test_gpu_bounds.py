@@ -101,6 +101,42 @@ def test_bounds_checked_run_on_guarded_buffers(tw, name):
         assert torch.equal(out[k], g0[k]), k
 
 
+@pytest.mark.parametrize("name", ["k64_split_rows", "heavy_small", "ovf_rows_8"])
+def test_bounds_checked_passes_on_guarded_buffers(tw, name):
+    """The same, under the multi-pass schedule with a 64 KiB L2 budget (the dot
+    passes in many hidden-tile chunks, the axpy passes in column chunks with
+    their own turnstile words in the workspace), and the 8-bit forward: guards
+    intact, no bounds bit, the regular library's results."""
+    M, d, f, K, act, rs, seed = CASES[name]
+    w = Workload(name, M, d, f, 128, K, act, row_scale=rs, training=True, seed=seed)
+    D = {k: to_dev(v) for k, v in make_inputs(w).items() if k != "meta"}
+    try:
+        tw.set_sparse_schedule(tw.SCHED_PASSES, 64 << 10)
+        Y0, st0 = tw.ffn_fwd(D["X"], D["W_g"], D["b_g"], D["W_u"], D["W_d"], K=K)
+        g0 = tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st0, D["dY"], lam=1e-3)
+        q8 = tw.quantize_weights(D["W_u"], D["W_d"])
+        Yq0, _ = tw.ffn_fwd_e4m3(D["X"], D["W_g"], D["b_g"], q8, K=K)
+        G = Guarded()
+        with tw.bounds_checked():
+            tw.set_sparse_schedule(tw.SCHED_PASSES, 64 << 10)  # the checked library keeps its own setting
+            st, wsb, Wdt, Y, out = _run(tw, D, w, G, K)
+            tw.ffn_bwd(D["X"], D["W_g"], D["W_u"], D["W_d"], st, D["dY"], lam=1e-3, W_dt=Wdt, ws=wsb, out=out)
+            stq = tw.HybridState(M, f, 128, K, None, "cuda", alloc=G.empty)
+            wsq = tw.workspace(tw.OP_FWD, M, d, f, 128, K, M, alloc=G.empty)
+            Yq = G.empty((M, d), torch.bfloat16)
+            tw.ffn_fwd_e4m3(D["X"], D["W_g"], D["b_g"], q8, K=K, state=stq, ws=wsq, Y=Yq)
+            torch.cuda.synchronize()
+            assert st.read_status() == 0 and stq.read_status() == 0
+        assert G.intact(), "a kernel wrote outside its arrays"
+        assert torch.equal(Y, Y0) and torch.equal(Yq, Yq0)
+        for k in out:
+            assert torch.equal(out[k], g0[k]), k
+    finally:
+        tw.set_sparse_schedule(tw.SCHED_AUTO, 0)
+        with tw.bounds_checked():
+            tw.set_sparse_schedule(tw.SCHED_AUTO, 0)
+
+
 def test_bounds_checked_build_flags_a_corrupt_column(tw):
     """An in-tile column of 130 (>= T_n = 128) in an ELL slot of row r < 32,
     tile 0: the backward's kernels that read it (the sparse backward and the
