@@ -112,7 +112,7 @@ def lib():
             L.twell_test_withhold_epilogue_arrival.argtypes = [ctypes.c_int]
             L.twell_set_sparse_schedule.restype = ctypes.c_int
             L.twell_set_sparse_schedule.argtypes = [ctypes.c_int, _i64]
-            L.twell_set_overlap.restype = None
+            L.twell_set_overlap.restype = ctypes.c_int
             L.twell_set_overlap.argtypes = [ctypes.c_int]
             L.twell_status_read.restype = ctypes.c_int
             L.twell_status_read.argtypes = [ctypes.POINTER(TwellHybrid), ctypes.POINTER(ctypes.c_uint32),
@@ -184,11 +184,15 @@ def set_sparse_schedule(mode: int = SCHED_AUTO, l2_budget_bytes: int = 0) -> Non
     _check(lib().twell_set_sparse_schedule(int(mode), int(l2_budget_bytes)), "twell_set_sparse_schedule")
 
 
-def set_overlap(on: bool = True) -> None:
+OVERLAP_OFF, OVERLAP_ON, OVERLAP_AUTO = 0, 1, 2
+
+
+def set_overlap(mode: int = OVERLAP_ON) -> None:
     """twell_set_overlap: run the dense-backup GEMMs on the library's side stream
-    beside the sparse kernels, or (off, the default) everything on the caller's
-    stream."""
-    lib().twell_set_overlap(1 if on else 0)
+    beside the sparse kernels (OVERLAP_ON, or True), everything on the caller's
+    stream (OVERLAP_OFF, or False), or OVERLAP_AUTO (the default: on below 4096
+    rows). Process-wide; the results are the same either way."""
+    _check(lib().twell_set_overlap(int(mode)), "twell_set_overlap")
 
 
 def trace_enable(on: bool = True) -> None:

@@ -37,17 +37,25 @@ long long device_l2_bytes() {
 }
 
 // ---------------------------------------------- the dense-backup side stream
-// twell_set_overlap (off by default: measured 1.4% slower on the d_model=4096,
-// d_ff=14336, M=65536 training step, 1-2% faster at M=8192): the dense-backup
-// GEMMs of a call run on a second stream
+// twell_set_overlap: the dense-backup GEMMs of a call run on a second stream
 // of the library (created per device at first use, at the highest priority,
 // so that the block scheduler places the persistent GEMM's CTAs before those
 // of the sparse kernels on the caller's stream); the sparse kernels then fill
 // the SMs' leftover shared memory and registers beside the GEMM. The caller's
 // stream forks to it after the routing and joins it before the first kernel
 // that reads what it wrote. The mutex keeps one call's fork/join from
-// interleaving with another host thread's.
-std::atomic<int> g_overlap{0};
+// interleaving with another host thread's. Auto (the default) overlaps below
+// kOverlapMaxRows rows, where the sparse kernels alone leave most of each SM
+// idle: measured at d_model=4096, d_ff=14336, 99% sparsity, the forward is 9%
+// and the training step 10% faster at M=512, 6% and 4% at M=2048; from
+// M=8192 on it is within -2% .. +2.5% (1.4% slower at M=65536).
+constexpr int kOverlapMaxRows = 4096;
+std::atomic<int> g_overlap{TWELL_OVERLAP_AUTO};
+
+bool overlap_for(int M) {
+  const int m = g_overlap.load();
+  return m == TWELL_OVERLAP_ON || (m == TWELL_OVERLAP_AUTO && M < kOverlapMaxRows);
+}
 
 struct SideStream {
   cudaStream_t s = nullptr;
@@ -85,8 +93,8 @@ SideStream* side_stream() {
 // overlap is off or the side stream cannot be had), and the join.
 class DenseFork {
  public:
-  explicit DenseFork(cudaStream_t main) : main_(main), dense_(main) {
-    if (!g_overlap.load()) return;
+  DenseFork(cudaStream_t main, bool on) : main_(main), dense_(main) {
+    if (!on) return;
     ss_ = side_stream();
     if (!ss_) return;
     lk_ = std::unique_lock<std::mutex>(ss_->mu);
@@ -407,7 +415,7 @@ twell_status ffn_fwd_impl(const uint16_t* X, const uint16_t* W_g, const uint16_t
   }
   // the dense backup (its own rows of Y) first, on the side stream when the
   // overlap is on; the sparse kernels (the other rows) on the caller's stream
-  DenseFork fk(s);
+  DenseFork fk(s, overlap_for(M));
   const SplitKBuffers sk{at<float>(ws, L.sk_partial), at<unsigned long long>(ws, L.sk_arrivals)};
   if (launch_ovf_fwd(x_ovf, W_u, W_d, h->g_ovf, h->ovf_rows, h->n_ovf, cap, M, d, f, at<uint16_t>(ws, L.h_ovf),
                      h->u_ovf, Y, sk, h->status, fk.dense()) != cudaSuccess)
@@ -512,7 +520,7 @@ twell_status twell_ffn_bwd(const uint16_t* X, const uint16_t* W_g, const uint16_
     // the pair list's counts on the caller's stream; joined before the pair
     // list is filled (it reads the dense rows' dU and dZ) and the weight
     // gradients (they add to what the GEMMs wrote)
-    DenseFork fk(s);
+    DenseFork fk(s, overlap_for(M));
     const cudaStream_t ds = fk.dense();
     if (launch_ovf_prep(X, dY, h->ovf_rows, h->n_ovf, h->row_plan, cap, M, d, f, dw, h->status, ds) != cudaSuccess)
       return TWELL_ECUDA;
@@ -554,7 +562,11 @@ twell_status twell_count_stats(const twell_hybrid* h, int64_t* rows_by_max, int6
                                         tiles_by_count, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-void twell_set_overlap(int on) { g_overlap.store(on ? 1 : 0); }
+twell_status twell_set_overlap(int mode) {
+  if (mode < TWELL_OVERLAP_OFF || mode > TWELL_OVERLAP_AUTO) return TWELL_EINVAL;
+  g_overlap.store(mode);
+  return TWELL_OK;
+}
 
 twell_status twell_set_sparse_schedule(int mode, int64_t l2_budget_bytes) {
   return static_cast<twell_status>(twell::set_sparse_schedule(mode, l2_budget_bytes));

@@ -86,8 +86,9 @@ def parse_args():
                    help="schedule of the sparse kernels (twell_set_sparse_schedule)")
     p.add_argument("--l2-budget-mib", type=int, default=0,
                    help="L2 budget of one chunk of the multi-pass schedule, MiB (0: the library default)")
-    p.add_argument("--overlap", default="off", choices=["on", "off"],
-                   help="dense-backup GEMMs on the library's side stream beside the sparse kernels (twell_set_overlap)")
+    p.add_argument("--overlap", default="auto", choices=["auto", "on", "off"],
+                   help="dense-backup GEMMs on the library's side stream beside the sparse kernels "
+                        "(twell_set_overlap; auto: below 4096 rows)")
     return p.parse_args()
 
 
@@ -97,7 +98,7 @@ def apply_schedule(args):
 
     mode = {"auto": tw.SCHED_AUTO, "fused": tw.SCHED_FUSED, "passes": tw.SCHED_PASSES}[args.sched]
     tw.set_sparse_schedule(mode, args.l2_budget_mib << 20)
-    tw.set_overlap(args.overlap == "on")
+    tw.set_overlap({"auto": tw.OVERLAP_AUTO, "on": tw.OVERLAP_ON, "off": tw.OVERLAP_OFF}[args.overlap])
 
 
 def reduce_max(x: float, dist=None, device=None) -> float:
@@ -1261,7 +1262,7 @@ def run_block(args, local):
 def main():
     args = parse_args()
     world, rank, local = dist_env()
-    if args.impl != "reference" and (args.sched != "auto" or args.l2_budget_mib or args.overlap != "off"):
+    if args.impl != "reference" and (args.sched != "auto" or args.l2_budget_mib or args.overlap != "auto"):
         apply_schedule(args)
     if args.block:
         run_block(args, local)

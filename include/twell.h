@@ -367,10 +367,15 @@ TWELL_API twell_status twell_set_sparse_schedule(int mode, int64_t l2_budget_byt
  * and joined back into it before the call's remaining kernels; the sparse
  * kernels stay on the caller's stream and use what the GEMM leaves of each
  * SM. The call stays asynchronous and stream-ordered for the caller, and is
- * capturable into a CUDA graph. 0 (the default) runs every kernel on the
- * caller's stream. Process-wide; applies to the calls made after it returns.
+ * capturable into a CUDA graph. OFF runs every kernel on the caller's stream;
+ * AUTO (the default) overlaps calls of fewer than 4096 rows, where the sparse
+ * kernels alone leave most of each SM idle. Process-wide; applies to the calls
+ * made after it returns. Returns TWELL_EINVAL for any other mode (the setting
+ * is then unchanged).
  */
-TWELL_API void twell_set_overlap(int on);
+typedef enum twell_overlap { TWELL_OVERLAP_OFF = 0, TWELL_OVERLAP_ON = 1, TWELL_OVERLAP_AUTO = 2 } twell_overlap;
+
+TWELL_API twell_status twell_set_overlap(int mode);
 
 /* Copies the device status word to *out after synchronizing `stream`; clears
  * it when `clear` is non-zero. Returns TWELL_ECUDA if the copy fails. */

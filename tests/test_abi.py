@@ -141,6 +141,8 @@ def test_host_side_errors(tw):
     assert L.twell_set_sparse_schedule(tw.SCHED_PASSES, -5) == 1
     assert L.twell_set_sparse_schedule(tw.SCHED_FUSED, 1 << 20) == 0
     assert L.twell_set_sparse_schedule(tw.SCHED_AUTO, 0) == 0
+    assert L.twell_set_overlap(3) == 1 and L.twell_set_overlap(-1) == 1
+    assert L.twell_set_overlap(tw.OVERLAP_OFF) == 0 and L.twell_set_overlap(tw.OVERLAP_AUTO) == 0
 
 
 def test_missing_library_fails_loudly(tw, monkeypatch):

@@ -303,7 +303,7 @@ def test_overlap_agrees_and_captures(tw):
                 assert torch.equal(a, b), name + " (graph replay)"
             del graph
         finally:
-            tw.set_overlap(False)
+            tw.set_overlap(tw.OVERLAP_AUTO)
 
 
 def test_prepared_wdt_matches(tw):
