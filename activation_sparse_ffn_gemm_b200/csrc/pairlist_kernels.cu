@@ -411,19 +411,23 @@ __global__ void __launch_bounds__(kWgWarps * 32, kWgMinBlocks) wgrad_kernel(cons
     if (blockIdx.y == 0 && lane == 0 && dbg != nullptr) dbg[j] = db_extra ? db + db_extra[j] : db;
   }
   __syncthreads();
-  for (int r = threadIdx.x; r < kWgCols; r += kWgWarps * 32) {
+  // dW_d write-out: row cc gets the CTA's kWgUnits consecutive units (kWgQ
+  // 16-byte words); consecutive lanes take consecutive words of a row, so a
+  // warp's store covers whole 32-byte sectors of 32 / kWgQ rows (one lane per
+  // row wrote half-sectors of 32 rows, twice the transactions: 80 us of the
+  // kernel's 270 at M=512)
+  constexpr int kWgQ = kWgUnits / 4;
+  for (int i = threadIdx.x; i < kWgQ * kWgCols; i += kWgWarps * 32) {
+    const int r = i / kWgQ, k = i % kWgQ;
     const int cc = c0 + r;
     if (cc >= d) continue;
-    float4* pd = reinterpret_cast<float4*>(dWd + static_cast<long>(cc) * f + j0);
-#pragma unroll
-    for (int k = 0; k < kWgUnits / 4; ++k) {
-      float4 v = make_float4(s_dwd[4 * k][r], s_dwd[4 * k + 1][r], s_dwd[4 * k + 2][r], s_dwd[4 * k + 3][r]);
-      if (acc_old) {
-        const float4 o = pd[k];
-        v = make_float4(o.x + v.x, o.y + v.y, o.z + v.z, o.w + v.w);
-      }
-      pd[k] = v;
+    float4* pd = reinterpret_cast<float4*>(dWd + static_cast<long>(cc) * f + j0) + k;
+    float4 v = make_float4(s_dwd[4 * k][r], s_dwd[4 * k + 1][r], s_dwd[4 * k + 2][r], s_dwd[4 * k + 3][r]);
+    if (acc_old) {
+      const float4 o = *pd;
+      v = make_float4(o.x + v.x, o.y + v.y, o.z + v.z, o.w + v.w);
     }
+    *pd = v;
   }
 }
 

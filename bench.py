@@ -67,7 +67,7 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--no-trace", action="store_true")
-    p.add_argument("--workload", default=MAIN_WORKLOAD, choices=["large", "sweep8k", "train", "heavy"],
+    p.add_argument("--workload", default=MAIN_WORKLOAD, choices=["large", "sweep8k", "sweep2k", "sweep512", "train", "heavy"],
                    help="workload of the timed training step (synthetic.WORKLOADS)")
     p.add_argument("--no-extra", action="store_true", help="skip the two smaller workloads of the line")
     p.add_argument("--step-only", action="store_true",

@@ -63,6 +63,9 @@ WORKLOADS = {
     "large": Workload("large", 65536, 4096, 14336, 128, 8, 0.01, row_scale="lognormal", training=True),
     # the M=8192 point of the same sweep at 99% sparsity, as a training step
     "sweep8k": Workload("sweep8k", 8192, 4096, 14336, 128, 8, 0.01, row_scale="lognormal", training=True),
+    # the sweep's small batches at 99% sparsity, as training steps
+    "sweep2k": Workload("sweep2k", 2048, 4096, 14336, 128, 8, 0.01, row_scale="lognormal", training=True),
+    "sweep512": Workload("sweep512", 512, 4096, 14336, 128, 8, 0.01, row_scale="lognormal", training=True),
 }
 
 
