@@ -33,36 +33,42 @@ __device__ __forceinline__ float warp_sum(float v) {
 // of its group with the same unit is then a popcount of that mask below its
 // lane, and group and chunk offsets come from prefix sums of the popcounts.
 
-// In-tile columns active for row r in tile t: the ELL slots of a non-overflow
-// row, or the nonzeros of its dense backup row (none when the dense backup's
-// weight gradients run as dense GEMMs); calls fn(c, ell_slot_or_-1).
+// In-tile columns active for the ELL row r in tile t (its first min(count, K)
+// slots); calls fn(c, ell_slot).
 template <typename Fn>
-__device__ __forceinline__ void for_row_entries(long r, int t, int T, int K, int f, const uint16_t* __restrict__ count,
-                                                const uint8_t* __restrict__ col, const uint8_t* __restrict__ row_ovf,
-                                                const int* __restrict__ row_slot, const uint16_t* __restrict__ g_ovf,
-                                                bool dense_ovf, int cap, uint32_t* status, Fn&& fn) {
-  if (!row_ovf[r]) {
-    const int c0 = count[r * T + t];
-    const int n = c0 < K ? c0 : K;
-    const long base = (r * T + t) * K;
-    for (int s = 0; s < n; ++s) {
-      const int c = col[base + s];
-      if (in_bounds(c < kTn, status)) fn(c, base + s);
-    }
-  } else {
-    if (dense_ovf) return;
-    const int sl = row_slot[r];
-    if (sl < 0 || !in_bounds(sl < cap, status)) return;
-    const uint4* gp = reinterpret_cast<const uint4*>(g_ovf + static_cast<long>(sl) * f + t * kTn);
-    for (int q = 0; q < kTn / 8; ++q) {
-      const uint4 v = gp[q];
-      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+__device__ __forceinline__ void for_ell_entries(long r, int t, int T, int K, const uint16_t* __restrict__ count,
+                                                const uint8_t* __restrict__ col, uint32_t* status, Fn&& fn) {
+  const int c0 = count[r * T + t];
+  const int n = c0 < K ? c0 : K;
+  const long base = (r * T + t) * K;
+  for (int s = 0; s < n; ++s) {
+    const int c = col[base + s];
+    if (in_bounds(c < kTn, status)) fn(c, base + s);
+  }
+}
+
+// The overflow rows of a warp's group of 32 rows (lane L holds row r0 + L),
+// taken one at a time by the whole warp: for each row whose pairs stay in the
+// list (none when the dense backup's weight gradients run as dense GEMMs), lane
+// i reads in-tile columns 4i .. 4i + 3 of its dense backup row and calls
+// fn(L, sl, c) for each nonzero. (One lane per row walked the 128 columns and
+// their entries one after another, a chain of dependent loads per heavy row.)
+template <typename Fn>
+__device__ __forceinline__ void for_ovf_rows(long r0, int M, int t, int f, const uint8_t* __restrict__ row_ovf,
+                                             const int* __restrict__ row_slot, const uint16_t* __restrict__ g_ovf,
+                                             bool dense_ovf, int cap, int lane, uint32_t* status, Fn&& fn) {
+  const long r = r0 + lane;
+  uint32_t rows = __ballot_sync(0xFFFFFFFFu, !dense_ovf && r < M && row_ovf[r]);
+  while (rows) {
+    const int L = __ffs(rows) - 1;
+    rows &= rows - 1;
+    const int sl = row_slot[r0 + L];
+    if (sl < 0 || !in_bounds(sl < cap, status)) continue;
+    const uint2 v = *reinterpret_cast<const uint2*>(g_ovf + static_cast<long>(sl) * f + t * kTn + 4 * lane);
+    const uint32_t w2[2] = {v.x, v.y};
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const uint32_t bits = (w4[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
-        if (bits) fn(q * 8 + e, -1L);
-      }
-    }
+    for (int e = 0; e < 4; ++e)
+      if ((w2[e >> 1] >> (16 * (e & 1))) & 0xFFFFu) fn(L, sl, 4 * lane + e);
   }
 }
 
@@ -87,9 +93,10 @@ __global__ void __launch_bounds__(256) csc_count_kernel(const uint16_t* __restri
 #pragma unroll
     for (int q = 0; q < kTn / 32; ++q) mask[w][lane + 32 * q] = 0u;
     __syncwarp();
-    if (r < M)
-      for_row_entries(r, t, T, K, f, count, col, row_ovf, row_slot, g_ovf, dense_ovf, cap, status,
-                      [&](int c, long) { atomicOr(&mask[w][c], 1u << lane); });
+    if (r < M && !row_ovf[r])
+      for_ell_entries(r, t, T, K, count, col, status, [&](int c, long) { atomicOr(&mask[w][c], 1u << lane); });
+    for_ovf_rows(r - lane, M, t, f, row_ovf, row_slot, g_ovf, dense_ovf, cap, lane, status,
+                 [&](int L, int, int c) { atomicOr(&mask[w][c], 1u << L); });
     __syncwarp();
 #pragma unroll
     for (int q = 0; q < kTn / 32; ++q) {
@@ -203,9 +210,10 @@ __global__ void __launch_bounds__(256) csc_fill_kernel(
 #pragma unroll
     for (int q = 0; q < kTn / 32; ++q) mask[g][lane + 32 * q] = 0u;
     __syncwarp();
-    if (r < M)
-      for_row_entries(r, t, T, K, f, count, col, row_ovf, row_slot, g_ovf, dense_ovf, cap, status,
-                      [&](int c, long) { atomicOr(&mask[g][c], 1u << lane); });
+    if (r < M && !row_ovf[r])
+      for_ell_entries(r, t, T, K, count, col, status, [&](int c, long) { atomicOr(&mask[g][c], 1u << lane); });
+    for_ovf_rows(r - lane, M, t, f, row_ovf, row_slot, g_ovf, dense_ovf, cap, lane, status,
+                 [&](int L, int, int c) { atomicOr(&mask[g][c], 1u << L); });
   }
   __syncthreads();
   if (threadIdx.x < kTn) {
@@ -220,21 +228,20 @@ __global__ void __launch_bounds__(256) csc_fill_kernel(
   const uint32_t below = (1u << lane) - 1u;
   for (int g = w; g < kCscGroups; g += 8) {
     const long r = static_cast<long>(chunk) * kCscRows + g * 32 + lane;
-    if (r >= M) continue;
-    const int sl = row_ovf[r] ? row_slot[r] : -1;
-    for_row_entries(r, t, T, K, f, count, col, row_ovf, row_slot, g_ovf, dense_ovf, cap, status, [&](int c, long slot) {
-      const int p = gbase[g][c] + __popc(mask[g][c] & below);
+    if (r < M && !row_ovf[r])
+      for_ell_entries(r, t, T, K, count, col, status, [&](int c, long slot) {
+        const int p = gbase[g][c] + __popc(mask[g][c] & below);
+        if (!in_bounds(p >= 0 && p < nnz_cap, status)) return;
+        csc_row[p] = static_cast<int>(r);
+        csc_val[p] = hdz_ell[slot];
+      });
+    for_ovf_rows(r - lane, M, t, f, row_ovf, row_slot, g_ovf, dense_ovf, cap, lane, status, [&](int L, int sl, int c) {
+      const int p = gbase[g][c] + __popc(mask[g][c] & ((1u << L) - 1u));
       if (!in_bounds(p >= 0 && p < nnz_cap, status)) return;
-      float4 v;
-      if (slot >= 0) {
-        v = hdz_ell[slot];
-      } else {
-        const long o = static_cast<long>(sl) * f + t * kTn + c;
-        const float gv = __uint_as_float(static_cast<uint32_t>(g_ovf[o]) << 16);
-        v = make_float4(gv * u_ovf[o], du_ovf[o], dz_ovf[o], 0.f);
-      }
-      csc_row[p] = static_cast<int>(r);
-      csc_val[p] = v;
+      const long o = static_cast<long>(sl) * f + t * kTn + c;
+      const float gv = __uint_as_float(static_cast<uint32_t>(g_ovf[o]) << 16);
+      csc_row[p] = static_cast<int>(r - lane + L);
+      csc_val[p] = make_float4(gv * u_ovf[o], du_ovf[o], dz_ovf[o], 0.f);
     });
   }
 }
