@@ -498,6 +498,7 @@ __global__ void ovf_db_part_kernel(const int* __restrict__ n_ovf, const int* __r
   int n = dense ? n_ovf[0] : 0;
   n = n < cap ? n : cap;
   const int per = (cap + kDbChunks - 1) / kDbChunks;
+  if (n == 0) return;  // the sum writes zeros without reading the partials
   const int s0 = blockIdx.y * per;
   const int s1 = n < s0 + per ? n : s0 + per;
   const long cap_r = dense_rows_padded(cap);
@@ -533,8 +534,10 @@ __global__ void ovf_db_sum_kernel(const int* __restrict__ n_ovf, const int* __re
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= f) return;
   float acc = 0.f;
+  if (n > 0) {
 #pragma unroll 8
-  for (int c = 0; c < kDbChunks; ++c) acc += part[static_cast<long>(c) * f + j];
+    for (int c = 0; c < kDbChunks; ++c) acc += part[static_cast<long>(c) * f + j];
+  }
   db_ovf[j] = acc;
 }
 
