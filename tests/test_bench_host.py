@@ -130,6 +130,10 @@ def test_workloads_of_the_line():
     assert (w.M, w.d_model, w.d_ff, w.T_n, w.K, w.activity, w.row_scale) == (
         65536, 4096, 14336, 128, 8, 0.01, "lognormal")
     assert "M=65536" in bench.workload_desc(w, seed) and "99% sparsity" in bench.workload_desc(w, seed)
+    for name, M in (("sweep8k", 8192), ("sweep2k", 2048), ("sweep512", 512)):
+        w, _ = bench.workload(name)
+        assert (w.M, w.d_model, w.d_ff, w.K, w.activity, w.row_scale, w.training) == (
+            M, 4096, 14336, 8, 0.01, "lognormal", True)
     w, seed = bench.workload("uniform")
     assert (w.M, w.d_model, w.d_ff, w.T_n, w.K, w.activity) == (4096, 2048, 8192, 128, 8, 0.01)
     with open(bench.os.path.join(bench.ROOT, "tests", "golden", "uniform_seed.json")) as fh:
