@@ -12,6 +12,8 @@
 //                 go to a dense backup) run as dense GEMMs:
 //                 forward  H = bf16(g * (X_ovf W_u^T)),  Y[rows] = bf16(H W_d^T)
 //                 backward [dU | dZ] from dH = dY_ovf W_d,  dX[rows] = dU W_u + dZ W_g
+#include <type_traits>
+
 #include "umma_gemm.cuh"
 #include "umma_gemm_pair.cuh"
 
@@ -175,6 +177,13 @@ struct EpiTwell {
 constexpr int kApplyPitch = 33;                               // floats per staged row (conflict-free)
 constexpr int kApplySmemBytes = 4 * 32 * kApplyPitch * 4;     // one 32 x 32 block per epilogue warp
 
+// Whether an epilogue asks for an L2 prefetch of its inputs two chunks ahead
+// (Epi::prefetch8), on top of the one chunk held in registers.
+template <class E, class = void>
+struct HasPrefetch8 : std::false_type {};
+template <class E>
+struct HasPrefetch8<E, std::void_t<decltype(&E::prefetch8)>> : std::true_type {};
+
 template <class Epi>
 __device__ __forceinline__ void run_apply8(const typename Epi::Args& a, int m0, int n0, int M_eff, int N, int r,
                                            uint32_t taddr, uint8_t* smem) {
@@ -206,6 +215,13 @@ __device__ __forceinline__ void run_apply8(const typename Epi::Args& a, int m0, 
 #pragma unroll
       for (int k = 0; k < 4; ++k)
         if (ok[k]) Epi::load8(a, rows[k], n + 32 + cq, nxt[k]);
+    }
+    if constexpr (HasPrefetch8<Epi>::value) {
+      if (ch + 2 < 8 && n + 64 < N) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (ok[k]) Epi::prefetch8(a, rows[k], n + 64 + cq);
+      }
     }
     tmem_wait_ld();
 #pragma unroll
@@ -380,6 +396,11 @@ struct EpiBwdDH {
     in.g = __ldcs(reinterpret_cast<const uint4*>(a.g + off));
     in.u0 = __ldcs(reinterpret_cast<const float4*>(a.u + off));
     in.u1 = __ldcs(reinterpret_cast<const float4*>(a.u + off) + 1);
+  }
+  __device__ static void prefetch8(const Args& a, int row, int n) {
+    const size_t off = static_cast<size_t>(row) * a.f + n;
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.g + off));
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.u + off));
   }
   __device__ static void apply8(const Args& a, int row, int n, const float (&dh)[8], const In& in) {
     const size_t off = static_cast<size_t>(row) * a.f + n;
