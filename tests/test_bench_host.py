@@ -179,3 +179,22 @@ def test_reference_arm_prints_the_contract_line():
     assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"]
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_schedule_flags_reach_the_library(monkeypatch):
+    """--sched, --l2-budget-mib and --overlap set the process-wide schedule and overlap
+    through the binding (no GPU: the binding's setters are replaced)."""
+    import activation_sparse_ffn_gemm_b200 as tw
+
+    calls = []
+    monkeypatch.setattr(tw, "set_sparse_schedule", lambda mode, budget: calls.append(("sched", mode, budget)))
+    monkeypatch.setattr(tw, "set_overlap", lambda mode: calls.append(("overlap", mode)))
+    for argv, want in ((["--sched", "passes", "--l2-budget-mib", "32", "--overlap", "on"],
+                        [("sched", tw.SCHED_PASSES, 32 << 20), ("overlap", tw.OVERLAP_ON)]),
+                       (["--sched", "fused", "--overlap", "off"],
+                        [("sched", tw.SCHED_FUSED, 0), ("overlap", tw.OVERLAP_OFF)]),
+                       ([], [("sched", tw.SCHED_AUTO, 0), ("overlap", tw.OVERLAP_AUTO)])):
+        calls.clear()
+        monkeypatch.setattr(sys, "argv", ["bench.py"] + argv)
+        bench.apply_schedule(bench.parse_args())
+        assert calls == want, argv
